@@ -1,0 +1,175 @@
+"""Pins for the fp64 RWKV-4 WKV oracle, each checked against something other
+than the oracle's own formula: closed forms, invariants that the
+time-parallel WKV_t formula implies, brute force, finite differences and the
+decay-simulator defaults printed on the flashpapers explainer page
+("4. Interactive Simulator").  A mistake such as a dropped bonus term, an
+off-by-one lag, a sign flip of w or swapped k/v fails at least one of them."""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+import wkv_inputs as wi
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+
+
+def _problem(B, T, C, seed, outliers=False, gy=False):
+    p = wi.wkv4_problem(B, T, C, seed, outliers=outliers, with_gy=gy)
+    return {k: v.double().numpy() for k, v in p.items()}
+
+
+def test_first_output_is_first_value():
+    # Empty sum over past tokens: WKV_1 = e^{u+k_1} v_1 / e^{u+k_1} = v_1.
+    p = _problem(3, 5, 16, 1, outliers=True)
+    y = oracle.wkv4_forward(p["w"], p["u"], p["k"], p["v"])
+    np.testing.assert_allclose(y[:, 0], p["v"][:, 0], rtol=1e-15, atol=0)
+
+
+def test_convex_combination_bounds():
+    # All weights e^{...} > 0, so WKV_t lies between min and max of v_1..v_t.
+    p = _problem(2, 200, 32, 2, outliers=True)
+    y = oracle.wkv4_forward(p["w"], p["u"], p["k"], p["v"])
+    lo = np.minimum.accumulate(p["v"], axis=1)
+    hi = np.maximum.accumulate(p["v"], axis=1)
+    assert np.all(y >= lo - 1e-12) and np.all(y <= hi + 1e-12)
+
+
+def test_constant_values():
+    p = _problem(2, 100, 8, 3, outliers=True)
+    v = np.full_like(p["v"], -1.75)
+    y = oracle.wkv4_forward(p["w"], p["u"], p["k"], v)
+    np.testing.assert_allclose(y, -1.75, rtol=2e-15, atol=0)
+
+
+def test_shift_invariance_in_k():
+    # A constant added to every key scales numerator and denominator alike.
+    p = _problem(2, 120, 8, 4)
+    shift = np.linspace(-7.0, 9.0, 8)
+    y0 = oracle.wkv4_forward(p["w"], p["u"], p["k"], p["v"])
+    y1 = oracle.wkv4_forward(p["w"], p["u"], p["k"] + shift, p["v"])
+    np.testing.assert_allclose(y1, y0, rtol=1e-12, atol=1e-12)
+
+
+def test_fast_decay_limit_is_two_token_softmax():
+    # w = 50: every token older than lag 0 is damped by <= e^{-50}, leaving
+    # (e^{k_{t-1}} v_{t-1} + e^{u+k_t} v_t) / (e^{k_{t-1}} + e^{u+k_t}).
+    p = _problem(1, 64, 16, 5)
+    w = np.full(16, 50.0)
+    k, v, u = p["k"][0], p["v"][0], p["u"]
+    y = oracle.wkv4_forward(w, u, p["k"], p["v"])[0]
+    prev_w = np.exp(k[:-1])
+    cur_w = np.exp(u + k[1:])
+    expect = (prev_w * v[:-1] + cur_w * v[1:]) / (prev_w + cur_w)
+    np.testing.assert_allclose(y[1:], expect, rtol=1e-12, atol=1e-14)
+
+
+def test_no_decay_no_bonus_is_running_softmax():
+    # w = 0, u = 0: WKV_t = sum_{i<=t} e^{k_i} v_i / sum_{i<=t} e^{k_i}, a
+    # running softmax-weighted mean of v (numpy cumulative sums).
+    p = _problem(2, 300, 8, 6)
+    w = np.zeros(8)
+    u = np.zeros(8)
+    y = oracle.wkv4_forward(w, u, p["k"], p["v"])
+    e = np.exp(p["k"])
+    expect = np.cumsum(e * p["v"], axis=1) / np.cumsum(e, axis=1)
+    np.testing.assert_allclose(y, expect, rtol=1e-12, atol=1e-12)
+
+
+def test_decay_simulator_defaults():
+    g = json.load(open(os.path.join(HERE, "golden", "p4_decay_simulator.json")))
+    w0, u0 = g["w"], g["u"]
+    lags = g["lag_of_position"]
+    T = len(lags)
+    raw = [math.exp(-n * w0) if n is not None else math.exp(u0) for n in lags]
+    weights = np.array(raw) / sum(raw)
+    # one channel per position: v is one-hot at that position, all keys zero
+    v = np.eye(T)[None]  # [1, T(time), C=T]
+    k = np.zeros_like(v)
+    y = oracle.wkv4_forward(np.full(T, w0), np.full(T, u0), k, v)
+    np.testing.assert_allclose(y[0, T - 1], weights, rtol=1e-14, atol=1e-16)
+    assert np.all(np.diff(weights) > 0)  # newer tokens weigh more, bonus highest
+
+
+@pytest.mark.parametrize("outliers", [False, True])
+def test_recurrent_equals_time_parallel(outliers):
+    p = _problem(2, 96, 24, 7, outliers=outliers)
+    y_rec = oracle.wkv4_forward(p["w"], p["u"], p["k"], p["v"])
+    y_par = oracle.wkv4_forward_bruteforce(p["w"], p["u"], p["k"], p["v"])
+    np.testing.assert_allclose(y_rec, y_par, rtol=1e-12, atol=1e-12)
+
+
+def test_split_sequence_resume():
+    p = _problem(2, 150, 12, 8, outliers=True)
+    y_full, s_full = oracle.wkv4_forward(p["w"], p["u"], p["k"], p["v"], return_state=True)
+    y1, s1 = oracle.wkv4_forward(p["w"], p["u"], p["k"][:, :61], p["v"][:, :61], return_state=True)
+    y2, s2 = oracle.wkv4_forward(p["w"], p["u"], p["k"][:, 61:], p["v"][:, 61:], state_in=s1,
+                                 return_state=True)
+    np.testing.assert_array_equal(np.concatenate([y1, y2], axis=1), y_full)
+    np.testing.assert_array_equal(s2, s_full)
+
+
+def test_step_matches_sequence():
+    p = _problem(3, 40, 10, 9, outliers=True)
+    y_full, s_full = oracle.wkv4_forward(p["w"], p["u"], p["k"], p["v"], return_state=True)
+    _, s = oracle.wkv4_forward(p["w"], p["u"], p["k"][:, :25], p["v"][:, :25], return_state=True)
+    for t in range(25, 40):
+        y, s = oracle.wkv4_step(p["w"], p["u"], p["k"][:, t], p["v"][:, t], s)
+        np.testing.assert_array_equal(y, y_full[:, t])
+    np.testing.assert_array_equal(s, s_full)
+
+
+def _loss(p, **over):
+    q = dict(p)
+    q.update(over)
+    y = oracle.wkv4_forward(q["w"], q["u"], q["k"], q["v"], state_in=q.get("s0"))
+    return float(np.sum(q["gy"] * y))
+
+
+@pytest.mark.parametrize("with_state", [False, True])
+def test_backward_finite_differences(with_state):
+    B, T, C = 1, 16, 4
+    p = _problem(B, T, C, 10, gy=True)
+    p["k"][0, 3, 1] = 6.0   # a large key, to exercise more than the typical range
+    p["w"] = np.array([0.01, 0.3, 1.7, 5.0])
+    s0 = None
+    if with_state:
+        s0 = np.stack([np.array([[0.4, -1.2, 2.0, 0.1]]), np.array([[1.5, 0.7, 3.0, 0.2]])])
+        p["s0"] = s0
+    gk, gv, gw, gu = oracle.wkv4_backward(p["w"], p["u"], p["k"], p["v"], p["gy"], state_in=s0)
+    h = 1e-6
+
+    def fd(name, idx):
+        plus, minus = p[name].copy(), p[name].copy()
+        plus[idx] += h
+        minus[idx] -= h
+        return (_loss(p, **{name: plus}) - _loss(p, **{name: minus})) / (2 * h)
+
+    for idx in np.ndindex(B, T, C):
+        assert fd("k", idx) == pytest.approx(gk[idx], rel=1e-6, abs=1e-8)
+        assert fd("v", idx) == pytest.approx(gv[idx], rel=1e-6, abs=1e-8)
+    for c in range(C):
+        assert fd("w", (c,)) == pytest.approx(gw[c], rel=1e-6, abs=1e-8)
+        assert fd("u", (c,)) == pytest.approx(gu[c], rel=1e-6, abs=1e-8)
+
+
+def test_backward_invariants():
+    # From shift invariance in k: sum_t dL/dk_t = 0 per channel (zero state).
+    # From WKV(v + c) = WKV(v) + c: sum_t dL/dv_t = sum_t gy_t per channel.
+    p = _problem(2, 300, 16, 11, outliers=True, gy=True)
+    gk, gv, gw, gu = oracle.wkv4_backward(p["w"], p["u"], p["k"], p["v"], p["gy"])
+    scale = np.abs(gk).sum(axis=1)
+    assert np.all(np.abs(gk.sum(axis=1)) <= 1e-11 * scale + 1e-13)
+    np.testing.assert_allclose(gv.sum(axis=1), p["gy"].sum(axis=1), rtol=1e-11, atol=1e-11)
+
+
+@pytest.mark.parametrize("outliers", [False, True])
+def test_backward_recurrent_equals_time_parallel(outliers):
+    p = _problem(2, 64, 12, 12, outliers=outliers, gy=True)
+    a = oracle.wkv4_backward(p["w"], p["u"], p["k"], p["v"], p["gy"])
+    b = oracle.wkv4_backward_bruteforce(p["w"], p["u"], p["k"], p["v"], p["gy"])
+    for x, y in zip(a, b):
+        np.testing.assert_allclose(x, y, rtol=1e-10, atol=1e-10)
