@@ -1,0 +1,350 @@
+"""Benchmark: RWKV-4 WKV forward + backward on the 1.5B-width training shape.
+
+One step = one forward (y and state checkpoints) + one backward (gk, gv, gw,
+gu) over B=8, T=4096, C=2048 fp32, keys with 1 % +-U(20,40) outliers,
+gy ~ N(0,1), all synthetic and seeded.  Prints one JSON line (rank 0).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 (launched by torch.distributed.run, one process per GPU) every rank
+runs its own independent problem (the operator shards over batch rows with no
+exchange); ``value`` is the whole job's elements/s over the max of the ranks'
+device times.  ``--impl reference`` times the fp64 CPU oracle on the host on a
+bounded sample of the same workload (rank 0 only).
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+B, T, C = 8, 4096, 2048
+SEED = 20261204  # seed base + workload index 2
+ELEM = B * T * C
+FWD_BYTES = 3 * 4 * ELEM                     # k, v read; y written
+BWD_BYTES = 5 * 4 * ELEM + 2 * 4 * C         # k, v, gy read; gk, gv written; gw, gu
+METRIC = "WKV fwd+bwd elements/s and HBM GB/s (% of peak) at B8·T4096·C2048"
+WORKLOAD = "RWKV-4 WKV forward+backward, fp32, B=8 T=4096 C=2048, 1% +-U(20,40) key outliers"
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+class ClockSampler:
+    """Samples nvidia-smi SM clocks and throttle reasons while running."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        sm.sort()
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def _dist():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def run_reference(args):
+    """The fp64 CPU oracle, as it stands, on a bounded sample of the workload."""
+    world, rank, _ = _dist()
+    if rank != 0:
+        return
+    import numpy as np
+    import torch
+
+    import oracle
+    import wkv_inputs as wi
+
+    n_ch = args.ref_channels
+    chans = torch.arange(0, C, C // n_ch)[:n_ch]
+    w, u = wi.wkv4_params(SEED, C)
+    b_sel = torch.arange(B).repeat_interleave(n_ch)
+    c_sel = chans.repeat(B)
+    k = wi.btc_field("k", SEED, B, T, C, b_sel=b_sel, c_sel=c_sel, outliers=True).T.reshape(B, n_ch, T)
+    v = wi.btc_field("v", SEED, B, T, C, b_sel=b_sel, c_sel=c_sel).T.reshape(B, n_ch, T)
+    gy = wi.btc_field("gy", SEED, B, T, C, b_sel=b_sel, c_sel=c_sel).T.reshape(B, n_ch, T)
+    k, v, gy = (np.ascontiguousarray(x.permute(0, 2, 1).double().numpy()) for x in (k, v, gy))
+    ws, us = w[chans].double().numpy(), u[chans].double().numpy()
+    elems = B * T * n_ch
+
+    def step():
+        oracle.wkv4_forward(ws, us, k, v)
+        oracle.wkv4_backward(ws, us, k, v, gy)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = (time.perf_counter() - t0) / args.steps
+    val = elems / dt
+    sample = f"all {B} batch rows x {T} steps x {n_ch} of {C} channels (every {C // n_ch}th), fp64"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": val, "unit": "elements/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "B": B, "T": T, "C": C, "sample_channels": n_ch},
+        "cpu_baseline": {"value": val, "unit": "elements/s", "cores": oracle.num_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": val, "unit": "elements/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def cpu_baseline(seconds_target=10.0):
+    """Times the oracle (fp64, OpenMP) on a bounded sample: all batch rows and
+    steps of a few channels, sized to a few seconds of CPU work."""
+    import numpy as np
+    import torch
+
+    import oracle
+    import wkv_inputs as wi
+
+    n_ch = 32
+    chans = torch.arange(0, C, C // n_ch)[:n_ch]
+    w, u = wi.wkv4_params(SEED, C)
+    b_sel = torch.arange(B).repeat_interleave(n_ch)
+    c_sel = chans.repeat(B)
+
+    def field(kind, out=False):
+        x = wi.btc_field(kind, SEED, B, T, C, b_sel=b_sel, c_sel=c_sel, outliers=out)  # [T, B*n]
+        return np.ascontiguousarray(x.T.reshape(B, n_ch, T).permute(0, 2, 1).double().numpy())
+
+    k, v, gy = field("k", True), field("v"), field("gy")
+    ws, us = w[chans].double().numpy(), u[chans].double().numpy()
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        oracle.wkv4_forward(ws, us, k, v)
+        oracle.wkv4_backward(ws, us, k, v, gy)
+        reps += 1
+        if time.perf_counter() - t0 >= seconds_target or reps >= 1000:
+            break
+    dt = (time.perf_counter() - t0) / reps
+    return {"value": B * T * n_ch / dt, "unit": "elements/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{reps} x forward+backward over all {B} batch rows x {T} steps x {n_ch} of {C} channels, fp64"}
+
+
+def run_ours(args):
+    import torch
+
+    import rwkv_wkv_recurrence_b200 as rw
+    import wkv_inputs as wi
+
+    world, rank, local = _dist()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    h = rw.lib()
+    stream = torch.cuda.current_stream()
+    # each rank its own independent problem (weak scaling)
+    p = wi.wkv4_problem(B, T, C, SEED + 1000 * rank, outliers=True, with_gy=True, device=dev)
+    w, u, k, v, gy = p["w"], p["u"], p["k"], p["v"], p["gy"]
+    y = torch.empty_like(k)
+    gk, gv = torch.empty_like(k), torch.empty_like(k)
+    gw = torch.empty(C, device=dev)
+    gu = torch.empty(C, device=dev)
+    nck = int(h.rwkv_wkv4_num_checkpoints(T, rw.CHUNK_LEN))
+    ck = torch.empty((nck, 3, B, C), device=dev)
+    fws = int(h.rwkv_wkv4_forward_workspace_bytes(B, T, C, rw.ALGO_AUTO))
+    bws = int(h.rwkv_wkv4_backward_workspace_bytes(B, T, C, rw.CHUNK_LEN, 1))
+    fw = torch.empty(max(fws, 1), dtype=torch.uint8, device=dev)
+    bw = torch.empty(bws, dtype=torch.uint8, device=dev)
+    sp = rw._stream(stream)
+    P = rw._ptr
+
+    def fwd():
+        s = h.rwkv_wkv4_forward(B, T, C, rw.F32, P(w), P(u), P(k), P(v), P(y), None, None, P(ck), rw.CHUNK_LEN,
+                                rw.ALGO_AUTO, P(fw), fws, sp)
+        if s:
+            raise rw.RwkvError("rwkv_wkv4_forward", s)
+
+    def bwd():
+        s = h.rwkv_wkv4_backward(B, T, C, rw.F32, P(w), P(u), P(k), P(v), P(gy), None, P(ck), rw.CHUNK_LEN,
+                                 P(gk), P(gv), P(gw), P(gu), P(bw), bws, sp)
+        if s:
+            raise rw.RwkvError("rwkv_wkv4_backward", s)
+
+    launches_per_step = 3  # forward scan; backward scan + gw/gu batch reduction
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        fwd()
+        bwd()
+    barrier()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        barrier()
+        start.record(stream)
+        for i in range(args.steps):
+            evs[i][0].record(stream)
+            fwd()
+            evs[i][1].record(stream)
+            bwd()
+            evs[i][2].record(stream)
+        end.record(stream)
+        barrier()
+    rw.rwkv_check_device_error()
+    total_ms = start.elapsed_time(end)
+    fwd_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
+    bwd_ms = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
+    t_max = torch.tensor([total_ms], device=dev)
+    if dist is not None:
+        dist.all_reduce(t_max, op=dist.ReduceOp.MAX)
+    ms_step = t_max.item() / args.steps
+    value = world * ELEM / (ms_step * 1e-3)
+
+    # end to end through the public API with host buffers (pinned), copies timed
+    hk, hv, hgy = (x.cpu().pin_memory() for x in (k, v, gy))
+    hw, hu = w.cpu().pin_memory(), u.cpu().pin_memory()
+    hgk, hgv = torch.empty_like(hk).pin_memory(), torch.empty_like(hv).pin_memory()
+    hgw, hgu = torch.empty(C).pin_memory(), torch.empty(C).pin_memory()
+
+    def e2e_step():
+        for dst, src in ((k, hk), (v, hv), (gy, hgy), (w, hw), (u, hu)):
+            dst.copy_(src, non_blocking=True)
+        fwd()
+        bwd()
+        for dst, src in ((hgk, gk), (hgv, gv), (hgw, gw), (hgu, gu)):
+            dst.copy_(src, non_blocking=True)
+
+    e2e_steps = max(1, min(args.steps, 5))
+    e2e_step()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    barrier()
+    e_ms = torch.tensor([e0.elapsed_time(e1) / e2e_steps], device=dev)
+    if dist is not None:
+        dist.all_reduce(e_ms, op=dist.ReduceOp.MAX)
+    e2e_val = world * ELEM / (e_ms.item() * 1e-3)
+
+    if rank == 0:
+        peak, peak_kind = _peaks()
+        bwd_gbs = BWD_BYTES / (bwd_ms * 1e-3) / 1e9
+        step_gbs = (FWD_BYTES + BWD_BYTES) / (ms_step * 1e-3) / 1e9
+        line = {
+            "metric": METRIC, "value": value, "unit": "elements/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "B": B, "T": T, "C": C, "per_gpu_problem": "independent",
+                       "l2": "no flush: every input (k, v, gy: 268 MB each) is larger than the 126 MB L2",
+                       "parallelism": f"{world} independent problems, no collective"},
+            "hbm_gbs_step": step_gbs, "hbm_frac_step": step_gbs / peak,
+            "kernels_ms": {"wkv4_forward": fwd_ms, "wkv4_backward": bwd_ms},
+            "roofline": {"bound": "hbm", "kernel": "wkv4_bwd_kernel (+ its gw/gu batch reduction)",
+                         "achieved": bwd_gbs, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                         "frac": bwd_gbs / peak, "traffic": args.traffic},
+            "e2e": {"value": e2e_val, "unit": "elements/s",
+                    "h2d_bytes_per_step": 3 * 4 * ELEM + 2 * 4 * C, "d2h_bytes_per_step": 2 * 4 * ELEM + 2 * 4 * C},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clk.summary(),
+        }
+        if not args.no_cpu_baseline and world == 1:
+            line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--ref-channels", type=int, default=256)
+    ap.add_argument("--traffic", type=float, default=None,
+                    help="ncu dram bytes per backward launch, if captured for this kernel version")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,174 @@
+/*
+ * rwkv_wkv.h — C ABI of the B200 (sm_100a) WKV operator library.
+ *
+ * The operator is RWKV's WKV:
+ *
+ *   RWKV-4 ("RWKV - Transformer 시대에 RNN을 재발명하다", Method / (2) Time-mixing
+ *   (WKV); same formula in "RWKV: Reinventing RNNs for the Transformer Era",
+ *   3. How It Works / The WKV Operator), per channel c:
+ *
+ *     wkv_t = ( Σ_{i<t} e^{-(t-1-i) w + k_i} v_i + e^{u + k_t} v_t )
+ *           / ( Σ_{i<t} e^{-(t-1-i) w + k_i}     + e^{u + k_t} )
+ *
+ *   and its recurrent form with state (a_t, b_t):
+ *     wkv_t = (a_{t-1} + e^{u+k_t} v_t) / (b_{t-1} + e^{u+k_t}),
+ *     a_t = e^{-w} a_{t-1} + e^{k_t} v_t,   b_t = e^{-w} b_{t-1} + e^{k_t}.
+ *
+ *   Eagle / RWKV-5 ("RWKV-5 Eagle과 RWKV-6 Finch", section Eagle), per head:
+ *     y_t = r_t · (s + diag(u) k_tᵀ v_t),   s ← diag(w) s + k_tᵀ v_t,
+ *     w = exp(-exp(ω)),  s[i][j] with i = key index (row), j = value index.
+ *
+ * Conventions for every call
+ *   - All tensor arguments are DEVICE pointers owned by the caller, on the
+ *     current CUDA device; the library never allocates, frees or keeps them.
+ *     Work is enqueued on `stream` (NULL = the legacy default stream) and the
+ *     call returns without synchronising.  Inputs must stay valid and outputs
+ *     untouched until the stream has run the work.
+ *   - Layouts are dense row-major: WKV-4 k, v, y, gy, gk, gv are [B, T, C]
+ *     (C fastest); w, u, gw, gu are [C] fp32.  WKV-5 r, k, v, y are
+ *     [B, T, H, N] bf16; omega, u are [H, N] fp32; s is [B, H, N, N] fp32.
+ *   - `w` (WKV-4) is the positive decay RATE of the formula above (the raw
+ *     parameter mapped through -exp(.) by the model), not a factor.
+ *   - WKV-4 state: [3, B, C] fp32 planes (a, b, p) meaning A = a·2^p,
+ *     B = b·2^p (p an exponent of two).  A zero state is a = b = 0 (any p).
+ *     Any finite (A, B) with A, B within fp32 range may be passed as (A, B, 0).
+ *     The representation is not unique: compare states through a/b and
+ *     log2(b) + p.
+ *   - Returns RWKV_OK or an error status; nothing throws or aborts.
+ *     Negative sizes or a NULL required pointer give RWKV_ERR_INVALID_ARG
+ *     before anything is enqueued.  A launch failure gives RWKV_ERR_CUDA.
+ *     Zero-sized problems are a successful no-op (T = 0 copies the state).
+ *   - Values are data: no range validation; NaN and Inf propagate.
+ *   - Alignment: k, v, gy (and r for WKV-5) must be 16-byte aligned with
+ *     C·sizeof(element) a multiple of 16 (TMA row pitch), else
+ *     RWKV_ERR_UNSUPPORTED.
+ */
+#ifndef RWKV_WKV_H
+#define RWKV_WKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define RWKV_API __attribute__((visibility("default")))
+#else
+#define RWKV_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st *rwkv_stream_t;
+
+typedef enum {
+    RWKV_OK = 0,
+    RWKV_ERR_INVALID_ARG = 1,    /* bad size, NULL required pointer, bad enum */
+    RWKV_ERR_UNSUPPORTED = 2,    /* valid request this build does not handle */
+    RWKV_ERR_WORKSPACE = 3,      /* workspace NULL or smaller than the query */
+    RWKV_ERR_CUDA = 4,           /* a CUDA runtime call or launch failed */
+    RWKV_ERR_DEVICE_TIMEOUT = 5  /* a kernel's bounded wait gave up */
+} rwkv_status;
+
+/* Element type of WKV-4 k, v, y, gy, gk, gv (arithmetic is fp32 either way). */
+typedef enum { RWKV_F32 = 0, RWKV_BF16 = 1 } rwkv_dtype;
+
+/* WKV-4 forward schedule.  SEQUENTIAL: one thread scans one channel over all
+ * of T.  CHUNKED: time is cut into segments scanned in parallel from a zero
+ * state, joined by an associative carry pass, then rescanned for outputs
+ * (for problems with too few channels to fill the GPU).  AUTO picks. */
+typedef enum { RWKV_ALGO_AUTO = 0, RWKV_ALGO_SEQUENTIAL = 1, RWKV_ALGO_CHUNKED = 2 } rwkv_algo;
+
+/* Human-readable name of a status code (static string). */
+RWKV_API const char *rwkv_status_string(rwkv_status s);
+
+/* Library ABI version, (major << 16) | minor. */
+RWKV_API int rwkv_version(void);
+
+/* Number of WKV-4 checkpoints for T steps at interval chunk_len:
+ * ceil(T / chunk_len); -1 if chunk_len is not a positive multiple of 16. */
+RWKV_API int64_t rwkv_wkv4_num_checkpoints(int64_t T, int64_t chunk_len);
+
+/* Workspace bytes rwkv_wkv4_forward needs for this shape and algo (0 if none). */
+RWKV_API size_t rwkv_wkv4_forward_workspace_bytes(int64_t B, int64_t T, int64_t C, int algo);
+
+/*
+ * WKV-4 forward (time-parallel training form; the recurrent form gives the
+ * same values).
+ *   k, v      [B,T,C] dtype, read.           y [B,T,C] dtype, written.
+ *   w, u      [C] fp32, read.
+ *   state_in  [3,B,C] or NULL (zero state).  state_out [3,B,C] or NULL:
+ *             the state after the last token; may equal state_in.
+ *   ckpt      [num_checkpoints(T, chunk_len), 3, B, C] or NULL: ckpt[j] is
+ *             the state before token j·chunk_len (ckpt[0] = state_in); it is
+ *             what rwkv_wkv4_backward reads.  chunk_len must be 16 today.
+ *   algo      rwkv_algo.   workspace: device scratch of
+ *             rwkv_wkv4_forward_workspace_bytes() bytes (may be NULL if 0).
+ */
+RWKV_API rwkv_status rwkv_wkv4_forward(int64_t B, int64_t T, int64_t C, rwkv_dtype dtype,
+                              const float *w, const float *u, const void *k, const void *v, void *y,
+                              const float *state_in, float *state_out, float *ckpt, int64_t chunk_len,
+                              int algo, void *workspace, size_t workspace_bytes, rwkv_stream_t stream);
+
+/* Workspace bytes rwkv_wkv4_backward needs; have_ckpt = 0 adds room to
+ * recompute the checkpoints. */
+RWKV_API size_t rwkv_wkv4_backward_workspace_bytes(int64_t B, int64_t T, int64_t C, int64_t chunk_len, int have_ckpt);
+
+/*
+ * WKV-4 backward: gradients of L = Σ gy·y with respect to k, v, w, u.
+ * The pages print no backward; this is the derivative of the formula above.
+ *   k, v, gy  [B,T,C] dtype, read.          gk, gv [B,T,C] dtype, written.
+ *   gw, gu    [C] fp32, OVERWRITTEN with the sum over batch and time.
+ *   state_in  the forward's initial state, or NULL (zero); used only when
+ *             ckpt is NULL.
+ *   ckpt      the checkpoints written by rwkv_wkv4_forward with the same
+ *             inputs and chunk_len (16), or NULL to recompute them into the
+ *             workspace.
+ *   Deterministic: the same inputs give bit-identical outputs.
+ */
+RWKV_API rwkv_status rwkv_wkv4_backward(int64_t B, int64_t T, int64_t C, rwkv_dtype dtype,
+                               const float *w, const float *u, const void *k, const void *v,
+                               const void *gy, const float *state_in, const float *ckpt,
+                               int64_t chunk_len, void *gk, void *gv, float *gw, float *gu,
+                               void *workspace, size_t workspace_bytes, rwkv_stream_t stream);
+
+/*
+ * WKV-4 recurrent decode: one token for each of B independent streams.
+ *   k, v, y   [B,C] dtype.   w, u [C] fp32.
+ *   state_in  [3,B,C] or NULL (zero).  state_out [3,B,C]; may equal
+ *             state_in (in-place update).
+ */
+RWKV_API rwkv_status rwkv_wkv4_step(int64_t B, int64_t C, rwkv_dtype dtype, const float *w, const float *u,
+                           const void *k, const void *v, void *y, const float *state_in,
+                           float *state_out, rwkv_stream_t stream);
+
+/* Workspace bytes rwkv_wkv5_forward needs (0 if none). */
+RWKV_API size_t rwkv_wkv5_forward_workspace_bytes(int64_t B, int64_t T, int64_t H, int64_t N);
+
+/*
+ * Eagle / RWKV-5 multi-head matrix-state WKV forward.
+ *   r, k, v   [B,T,H,N] bf16, read.      y [B,T,H,N] bf16, written.
+ *   omega, u  [H,N] fp32 (w = exp(-exp(omega)) is formed inside).
+ *   s_in      [B,H,N,N] fp32 or NULL (zero).  s_out [B,H,N,N] fp32 or NULL;
+ *             may equal s_in.
+ *   N must be 64 (RWKV_ERR_UNSUPPORTED otherwise).
+ */
+RWKV_API rwkv_status rwkv_wkv5_forward(int64_t B, int64_t T, int64_t H, int64_t N,
+                              const void *r, const void *k, const void *v,
+                              const float *omega, const float *u, void *y,
+                              const float *s_in, float *s_out,
+                              void *workspace, size_t workspace_bytes, rwkv_stream_t stream);
+
+/*
+ * Synchronises `stream`, then reports and clears the device error word that
+ * kernels set when a bounded wait gives up (RWKV_ERR_DEVICE_TIMEOUT), or
+ * RWKV_ERR_CUDA if the stream itself failed.
+ */
+RWKV_API rwkv_status rwkv_check_device_error(rwkv_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RWKV_WKV_H */

@@ -1,0 +1,330 @@
+// C-ABI layer: argument validation, workspace planning, TMA descriptors and
+// kernel dispatch for the calls declared in include/rwkv_wkv.h.
+#include <climits>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/rwkv_wkv.h"
+#include "launch.h"
+
+namespace rwkv {
+
+// The library's device error word (one per device that loads the library).
+__device__ unsigned int g_device_error = 0;
+
+cudaError_t launch_wkv5_fwd(int B, int T, int H, const void* r, const void* k, const void* v, const float* omega,
+                            const float* u, void* y, const float* s_in, float* s_out, cudaStream_t st);
+
+namespace {
+
+constexpr int kDesignSMs = 148;  // B200 SM count the schedules are planned for
+constexpr int kCkLen = 16;       // checkpoint interval the backward reads
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// Tensor map over a dense [B, T, C] tensor, box = [1, box_t, 32] (C innermost).
+bool make_btc_map(CUtensorMap* m, const void* base, bool bf16, int B, int T, int C, int box_t) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return false;
+  const size_t esz = bf16 ? 2 : 4;
+  cuuint64_t dims[3] = {(cuuint64_t)C, (cuuint64_t)T, (cuuint64_t)B};
+  cuuint64_t strides[2] = {(cuuint64_t)C * esz, (cuuint64_t)C * T * esz};
+  cuuint32_t box[3] = {32u, (cuuint32_t)box_t, 1u};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  std::memset(m, 0, sizeof(*m));
+  CUresult r = enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3,
+                   const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+unsigned int* device_error_word() {
+  unsigned int* p = nullptr;
+  if (cudaGetSymbolAddress(reinterpret_cast<void**>(&p), g_device_error) != cudaSuccess) return nullptr;
+  return p;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool fits_int(int64_t x) { return x >= 0 && x <= INT_MAX; }
+
+struct FwdPlan {
+  int algo;      // RWKV_ALGO_SEQUENTIAL or RWKV_ALGO_CHUNKED
+  int seg_len;
+  int nseg;
+  size_t ws_bytes;
+};
+
+FwdPlan plan_forward(int64_t B, int64_t T, int64_t C, int algo) {
+  FwdPlan pl{RWKV_ALGO_SEQUENTIAL, 0, 1, 0};
+  const int tt = fwd_tile_steps();
+  const int64_t lane_tiles = B * ((C + 31) / 32);
+  int a = algo;
+  if (a == RWKV_ALGO_AUTO) a = (lane_tiles >= 3 * kDesignSMs || T <= 128) ? RWKV_ALGO_SEQUENTIAL : RWKV_ALGO_CHUNKED;
+  if (a == RWKV_ALGO_CHUNKED && T > 0 && lane_tiles > 0) {
+    const int64_t want = (8 * kDesignSMs + lane_tiles - 1) / lane_tiles;
+    int64_t seg = (T + want - 1) / want;
+    seg = ((seg + tt - 1) / tt) * tt;
+    if (seg < 64) seg = 64;
+    const int64_t nseg = (T + seg - 1) / seg;
+    if (nseg > 1) {
+      pl.algo = RWKV_ALGO_CHUNKED;
+      pl.seg_len = (int)seg;
+      pl.nseg = (int)nseg;
+      pl.ws_bytes = (size_t)nseg * 3 * B * C * sizeof(float);
+      return pl;
+    }
+  }
+  pl.seg_len = (int)(((T + tt - 1) / tt) * tt);
+  if (pl.seg_len == 0) pl.seg_len = tt;
+  return pl;
+}
+
+// Runs the forward pass (outputs optional) on already-validated arguments.
+rwkv_status run_forward(int B, int T, int C, bool bf16, const float* w, const float* u, const void* k,
+                        const void* v, void* y, const float* state_in, float* state_out, float* ckpt, int ckpt_len,
+                        const FwdPlan& pl, void* ws, cudaStream_t st) {
+  unsigned int* err = device_error_word();
+  if (err == nullptr) return RWKV_ERR_CUDA;
+  const int tt = fwd_tile_steps();
+  CUtensorMap mk, mv;
+  if (!make_btc_map(&mk, k, bf16, B, T, C, tt) || !make_btc_map(&mv, v, bf16, B, T, C, tt)) return RWKV_ERR_CUDA;
+  Fwd4Params p{};
+  p.B = B;
+  p.T = T;
+  p.C = C;
+  p.ctiles = (C + 31) / 32;
+  p.w = w;
+  p.u = u;
+  p.err = err;
+  p.ckpt_len = ckpt_len;
+  const long long seg_stride = 3LL * B * C;
+  if (pl.algo == RWKV_ALGO_SEQUENTIAL) {
+    p.seg_len = pl.seg_len;
+    p.nseg = 1;
+    p.stages = fwd_stages(bf16, pl.seg_len);
+    p.y = y;
+    p.start = state_in;
+    p.end = state_out;
+    p.ckpt = ckpt;
+    if (launch_wkv4_fwd(bf16, mk, mv, p, st) != cudaSuccess) return RWKV_ERR_CUDA;
+    return RWKV_OK;
+  }
+  float* wsf = static_cast<float*>(ws);
+  // 1) segment summaries from a zero state
+  p.seg_len = pl.seg_len;
+  p.nseg = pl.nseg;
+  p.stages = fwd_stages(bf16, pl.seg_len);
+  p.y = nullptr;
+  p.start = nullptr;
+  p.end = wsf;
+  p.end_seg_stride = seg_stride;
+  p.ckpt = nullptr;
+  if (launch_wkv4_fwd(bf16, mk, mv, p, st) != cudaSuccess) return RWKV_ERR_CUDA;
+  // 2) carries (in place) and the final state
+  if (launch_wkv4_carry(B, C, T, pl.nseg, pl.seg_len, w, state_in, wsf, state_out, st) != cudaSuccess)
+    return RWKV_ERR_CUDA;
+  // 3) outputs and checkpoints from each segment's carry
+  p.y = y;
+  p.start = wsf;
+  p.start_seg_stride = seg_stride;
+  p.end = nullptr;
+  p.ckpt = ckpt;
+  if (launch_wkv4_fwd(bf16, mk, mv, p, st) != cudaSuccess) return RWKV_ERR_CUDA;
+  return RWKV_OK;
+}
+
+}  // namespace
+}  // namespace rwkv
+
+using namespace rwkv;
+
+extern "C" {
+
+const char* rwkv_status_string(rwkv_status s) {
+  switch (s) {
+    case RWKV_OK: return "ok";
+    case RWKV_ERR_INVALID_ARG: return "invalid argument";
+    case RWKV_ERR_UNSUPPORTED: return "unsupported shape, alignment or option";
+    case RWKV_ERR_WORKSPACE: return "workspace missing or too small";
+    case RWKV_ERR_CUDA: return "CUDA runtime or launch error";
+    case RWKV_ERR_DEVICE_TIMEOUT: return "a kernel's bounded wait timed out";
+  }
+  return "unknown status";
+}
+
+int rwkv_version(void) { return (1 << 16) | 0; }
+
+int64_t rwkv_wkv4_num_checkpoints(int64_t T, int64_t chunk_len) {
+  if (chunk_len <= 0 || chunk_len % 16 != 0 || T < 0) return -1;
+  return (T + chunk_len - 1) / chunk_len;
+}
+
+size_t rwkv_wkv4_forward_workspace_bytes(int64_t B, int64_t T, int64_t C, int algo) {
+  if (B <= 0 || T <= 0 || C <= 0) return 0;
+  return plan_forward(B, T, C, algo).ws_bytes;
+}
+
+rwkv_status rwkv_wkv4_forward(int64_t B, int64_t T, int64_t C, rwkv_dtype dtype, const float* w, const float* u,
+                              const void* k, const void* v, void* y, const float* state_in, float* state_out,
+                              float* ckpt, int64_t chunk_len, int algo, void* workspace, size_t workspace_bytes,
+                              rwkv_stream_t stream) {
+  if (!fits_int(B) || !fits_int(T) || !fits_int(C)) return RWKV_ERR_INVALID_ARG;
+  if (dtype != RWKV_F32 && dtype != RWKV_BF16) return RWKV_ERR_INVALID_ARG;
+  if (algo < RWKV_ALGO_AUTO || algo > RWKV_ALGO_CHUNKED) return RWKV_ERR_INVALID_ARG;
+  if (ckpt != nullptr && (chunk_len <= 0 || chunk_len % 16 != 0)) return RWKV_ERR_INVALID_ARG;
+  if (ckpt != nullptr && chunk_len != kCkLen) return RWKV_ERR_UNSUPPORTED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (B == 0 || C == 0) return RWKV_OK;
+  if (w == nullptr || u == nullptr) return RWKV_ERR_INVALID_ARG;
+  if (T == 0) {
+    if (state_out != nullptr && launch_copy_state((int)B, (int)C, state_in, state_out, st) != cudaSuccess)
+      return RWKV_ERR_CUDA;
+    return RWKV_OK;
+  }
+  if (k == nullptr || v == nullptr) return RWKV_ERR_INVALID_ARG;
+  if (y == nullptr && state_out == nullptr && ckpt == nullptr) return RWKV_ERR_INVALID_ARG;
+  const bool bf16 = dtype == RWKV_BF16;
+  if (!aligned16(k) || !aligned16(v) || (C * (bf16 ? 2 : 4)) % 16 != 0) return RWKV_ERR_UNSUPPORTED;
+  const FwdPlan pl = plan_forward(B, T, C, algo);
+  if (pl.ws_bytes > 0 && (workspace == nullptr || workspace_bytes < pl.ws_bytes)) return RWKV_ERR_WORKSPACE;
+  return run_forward((int)B, (int)T, (int)C, bf16, w, u, k, v, y, state_in, state_out, ckpt, (int)chunk_len, pl,
+                     workspace, st);
+}
+
+size_t rwkv_wkv4_backward_workspace_bytes(int64_t B, int64_t T, int64_t C, int64_t chunk_len, int have_ckpt) {
+  if (B <= 0 || T <= 0 || C <= 0) return 0;
+  if (chunk_len <= 0) chunk_len = kCkLen;
+  size_t bytes = (size_t)2 * B * C * sizeof(double);  // per-lane gw, gu partial sums
+  if (!have_ckpt) bytes += (size_t)((T + chunk_len - 1) / chunk_len) * 3 * B * C * sizeof(float);
+  return bytes;
+}
+
+rwkv_status rwkv_wkv4_backward(int64_t B, int64_t T, int64_t C, rwkv_dtype dtype, const float* w, const float* u,
+                               const void* k, const void* v, const void* gy, const float* state_in,
+                               const float* ckpt, int64_t chunk_len, void* gk, void* gv, float* gw, float* gu,
+                               void* workspace, size_t workspace_bytes, rwkv_stream_t stream) {
+  if (!fits_int(B) || !fits_int(T) || !fits_int(C)) return RWKV_ERR_INVALID_ARG;
+  if (dtype != RWKV_F32 && dtype != RWKV_BF16) return RWKV_ERR_INVALID_ARG;
+  if (chunk_len <= 0 || chunk_len % 16 != 0) return RWKV_ERR_INVALID_ARG;
+  if (chunk_len != kCkLen) return RWKV_ERR_UNSUPPORTED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (C == 0) return RWKV_OK;
+  if (gw == nullptr || gu == nullptr || w == nullptr || u == nullptr) return RWKV_ERR_INVALID_ARG;
+  if (B == 0 || T == 0) {  // empty sums: gradients of w and u are zero
+    if (cudaMemsetAsync(gw, 0, C * sizeof(float), st) != cudaSuccess) return RWKV_ERR_CUDA;
+    if (cudaMemsetAsync(gu, 0, C * sizeof(float), st) != cudaSuccess) return RWKV_ERR_CUDA;
+    return RWKV_OK;
+  }
+  if (k == nullptr || v == nullptr || gy == nullptr || gk == nullptr || gv == nullptr) return RWKV_ERR_INVALID_ARG;
+  const bool bf16 = dtype == RWKV_BF16;
+  if (!aligned16(k) || !aligned16(v) || !aligned16(gy) || (C * (bf16 ? 2 : 4)) % 16 != 0)
+    return RWKV_ERR_UNSUPPORTED;
+  const size_t need = rwkv_wkv4_backward_workspace_bytes(B, T, C, chunk_len, ckpt != nullptr);
+  if (workspace == nullptr || workspace_bytes < need) return RWKV_ERR_WORKSPACE;
+  const int iB = (int)B, iT = (int)T, iC = (int)C;
+  double* part = static_cast<double*>(workspace);
+  const float* ck = ckpt;
+  if (ck == nullptr) {
+    float* ckw = reinterpret_cast<float*>(part + (size_t)2 * B * C);
+    const FwdPlan pl = plan_forward(B, T, C, RWKV_ALGO_SEQUENTIAL);
+    rwkv_status s = run_forward(iB, iT, iC, bf16, w, u, k, v, nullptr, state_in, nullptr, ckw, kCkLen, pl,
+                                nullptr, st);
+    if (s != RWKV_OK) return s;
+    ck = ckw;
+  }
+  unsigned int* err = device_error_word();
+  if (err == nullptr) return RWKV_ERR_CUDA;
+  const int box_t = bwd_tile_steps();
+  CUtensorMap mk, mv, mg;
+  if (!make_btc_map(&mk, k, bf16, iB, iT, iC, box_t) || !make_btc_map(&mv, v, bf16, iB, iT, iC, box_t) ||
+      !make_btc_map(&mg, gy, bf16, iB, iT, iC, box_t))
+    return RWKV_ERR_CUDA;
+  Bwd4Params p{};
+  p.B = iB;
+  p.T = iT;
+  p.C = iC;
+  p.ctiles = (iC + 31) / 32;
+  p.stages = bwd_stages(bf16, iT);
+  p.w = w;
+  p.u = u;
+  p.ckpt = ck;
+  p.gk = gk;
+  p.gv = gv;
+  p.part = part;
+  p.err = err;
+  if (launch_wkv4_bwd(bf16, mk, mv, mg, p, st) != cudaSuccess) return RWKV_ERR_CUDA;
+  if (launch_wkv4_reduce_wu(iB, iC, part, gw, gu, st) != cudaSuccess) return RWKV_ERR_CUDA;
+  return RWKV_OK;
+}
+
+rwkv_status rwkv_wkv4_step(int64_t B, int64_t C, rwkv_dtype dtype, const float* w, const float* u, const void* k,
+                           const void* v, void* y, const float* state_in, float* state_out, rwkv_stream_t stream) {
+  if (!fits_int(B) || !fits_int(C)) return RWKV_ERR_INVALID_ARG;
+  if (dtype != RWKV_F32 && dtype != RWKV_BF16) return RWKV_ERR_INVALID_ARG;
+  if (B == 0 || C == 0) return RWKV_OK;
+  if (w == nullptr || u == nullptr || k == nullptr || v == nullptr || y == nullptr || state_out == nullptr)
+    return RWKV_ERR_INVALID_ARG;
+  const bool bf16 = dtype == RWKV_BF16;
+  const bool vec4 = !bf16 && C % 4 == 0 && aligned16(k) && aligned16(v) && aligned16(y) &&
+                    (state_in == nullptr || aligned16(state_in)) && aligned16(state_out);
+  if (launch_wkv4_step(bf16, (int)B, (int)C, w, u, k, v, y, state_in, state_out, vec4,
+                       reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return RWKV_ERR_CUDA;
+  return RWKV_OK;
+}
+
+size_t rwkv_wkv5_forward_workspace_bytes(int64_t B, int64_t T, int64_t H, int64_t N) {
+  (void)B;
+  (void)T;
+  (void)H;
+  (void)N;
+  return 0;
+}
+
+rwkv_status rwkv_wkv5_forward(int64_t B, int64_t T, int64_t H, int64_t N, const void* r, const void* k,
+                              const void* v, const float* omega, const float* u, void* y, const float* s_in,
+                              float* s_out, void* workspace, size_t workspace_bytes, rwkv_stream_t stream) {
+  (void)workspace;
+  (void)workspace_bytes;
+  if (!fits_int(B) || !fits_int(T) || !fits_int(H) || !fits_int(N)) return RWKV_ERR_INVALID_ARG;
+  if (N != 64) return RWKV_ERR_UNSUPPORTED;
+  if (B == 0 || H == 0) return RWKV_OK;
+  if (omega == nullptr || u == nullptr) return RWKV_ERR_INVALID_ARG;
+  if (T > 0 && (r == nullptr || k == nullptr || v == nullptr || y == nullptr)) return RWKV_ERR_INVALID_ARG;
+  if (T > 0 && (!aligned16(r) || !aligned16(k) || !aligned16(v) || !aligned16(y))) return RWKV_ERR_UNSUPPORTED;
+  if ((int64_t)B * H * T * N > (int64_t)INT_MAX * 8) return RWKV_ERR_UNSUPPORTED;
+  if (launch_wkv5_fwd((int)B, (int)T, (int)H, r, k, v, omega, u, y, s_in, s_out,
+                      reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return RWKV_ERR_CUDA;
+  return RWKV_OK;
+}
+
+rwkv_status rwkv_check_device_error(rwkv_stream_t stream) {
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return RWKV_ERR_CUDA;
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_device_error, sizeof(v)) != cudaSuccess) return RWKV_ERR_CUDA;
+  if (v != 0) {
+    const unsigned int zero = 0;
+    if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero)) != cudaSuccess) return RWKV_ERR_CUDA;
+    return RWKV_ERR_DEVICE_TIMEOUT;
+  }
+  return RWKV_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,61 @@
+// Internal launch interface between the C-ABI layer (api.cu) and the kernel
+// translation units.  Not part of the public header.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace rwkv {
+
+// Parameters of the WKV-4 forward kernel.  A CTA owns 32 channels of one
+// batch row over one time segment [seg*seg_len, min(T, (seg+1)*seg_len)).
+struct Fwd4Params {
+  int B, T, C;
+  int ctiles;   // ceil(C / 32)
+  int seg_len;  // time steps per segment (multiple of the 64-step tile)
+  int nseg;
+  int stages;   // TMA pipeline depth
+  const float* w;
+  const float* u;
+  void* y;                        // [B,T,C] or null (state-only pass)
+  const float* start;             // start state per segment, or null = zero
+  long long start_seg_stride;     // floats between consecutive segments' start states
+  float* end;                     // end state per segment, or null
+  long long end_seg_stride;
+  float* ckpt;                    // [nck,3,B,C] states before tokens 0, L, 2L, ... or null
+  int ckpt_len;                   // L (multiple of 16) when ckpt != null
+  unsigned int* err;              // device error word
+};
+
+struct Bwd4Params {
+  int B, T, C;
+  int ctiles;
+  int stages;
+  const float* w;
+  const float* u;
+  const float* ckpt;  // [ceil(T/16),3,B,C], interval 16
+  void* gk;
+  void* gv;
+  double* part;       // [2,B,C] per-lane gw, gu partial sums
+  unsigned int* err;  // device error word
+};
+
+int fwd_tile_steps();
+int fwd_stages(bool bf16, int seg_len);
+int bwd_tile_steps();
+int bwd_stages(bool bf16, int T);
+cudaError_t launch_wkv4_fwd(bool bf16, const CUtensorMap& mk, const CUtensorMap& mv, const Fwd4Params& p,
+                            cudaStream_t st);
+cudaError_t launch_wkv4_carry(int B, int C, int T, int nseg, int seg_len, const float* w, const float* state_in,
+                              float* ws, float* state_out, cudaStream_t st);
+cudaError_t launch_wkv4_bwd(bool bf16, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mgy,
+                            const Bwd4Params& p, cudaStream_t st);
+cudaError_t launch_wkv4_reduce_wu(int B, int C, const double* part, float* gw, float* gu, cudaStream_t st);
+cudaError_t launch_wkv4_step(bool bf16, int B, int C, const float* w, const float* u, const void* k, const void* v,
+                             void* y, const float* state_in, float* state_out, bool vec4, cudaStream_t st);
+cudaError_t launch_copy_state(int B, int C, const float* state_in, float* state_out, cudaStream_t st);
+
+// Sets the dynamic shared-memory limit of `func` once per device.
+cudaError_t ensure_smem_attr(const void* func, int bytes, unsigned* device_mask);
+
+}  // namespace rwkv

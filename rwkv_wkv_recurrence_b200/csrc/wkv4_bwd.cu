@@ -1,0 +1,357 @@
+// RWKV-4 WKV backward kernels (sm_100a).
+//
+// The pages print no backward; this is the chain rule through the recurrent
+// form of "RWKV - Transformer 시대에 RNN을 재발명하다", Method / (2) Time-mixing
+// (WKV), for L = Σ gy_t WKV_t.  With D_t = B_{t-1} + e^{u+k_t},
+// g_t = gy_t / D_t, h_t = gy_t WKV_t / D_t and the reverse sums
+//   α_t = Σ_{s>t} e^{-(s-t-1)w} g_s,   β_t = -Σ_{s>t} e^{-(s-t-1)w} h_s
+// (the gradients of L with respect to the state A_t, B_t):
+//   gv_t = e^{k_t} (e^u g_t + α_t)
+//   gk_t = e^{k_t} (e^u (g_t v_t - h_t) + α_t v_t + β_t)
+//   gu   = Σ e^{u+k_t} (g_t v_t - h_t)
+//   gw   = -e^{-w} Σ (α_t A_{t-1} + β_t B_{t-1})          (summed over b and t)
+// α and β obey α_{t-1} = g_t + e^{-w} α_t (likewise β with -h_t), a linear
+// reverse recurrence: the same associativity as the forward lets the four
+// 16-step chunks of a tile run their reverse walks in parallel once each has
+// its carry, and the carries come from folding each chunk's local sums.
+//
+// Scaling.  Inside a chunk everything is measured against one power of two
+// 2^q: e_t = e^{k_t} 2^{-q}, d_t = D_t 2^{-q}, G_t = gy_t / d_t, and the
+// carries are kept as α~ = α 2^q; then e^{k_t} α_t = e_t α~_t and
+// α_t A_{t-1} = α~_t a_{t-1}, so the scale cancels from every gradient.
+// Precision.  The gradient terms cancel each other (α_t v_t + β_t is small
+// when the state's mean is close to v_t), so fp32 sums over thousands of steps
+// would not hold 1e-4 relative accuracy.  Steps inside a chunk run in fp32 with
+// the decay e^{-w} = lh + ll split into fp32 hi and lo parts; the carries
+// folded from chunk to chunk and the per-lane gw, gu sums are fp64, so fp32
+// rounding accumulates over 16 steps at most.
+//
+// Kernel shape.  A CTA owns 32 channels of one batch row over all of T,
+// processed in 64-step tiles from the last to the first; warp w takes the
+// tile's w-th 16-step chunk: it recomputes that chunk's forward from the
+// forward pass's checkpoint, keeps e_t, G_t, y_t and b_{t-1} in registers,
+// sums its local reverse carries, folds the carries of the chunks after it,
+// then walks the chunk backwards writing gk and gv.  k, v, gy arrive by TMA
+// (no multicast); each element is read once and each gradient written once.
+// Per-lane gw, gu partials are reduced over the batch by a second kernel.
+#include "launch.h"
+#include "wkv_common.cuh"
+
+namespace rwkv {
+namespace {
+
+constexpr int kW = 4;
+constexpr int kL = 16;
+constexpr int kTile = kW * kL;
+
+struct RSumm {  // a chunk's own reverse sums from a zero carry, at scale 2^q
+  float la;  // α~ carried out of the chunk (into the step before its first)
+  float lg;  // γ at the chunk's first step
+  float ys;  // y at the chunk's first step
+  float ye;  // y at the chunk's last step
+  float q;
+  float pad;  // 24 bytes: two stages of boxes plus these still fit four CTAs per SM
+};
+
+// Phase A: forward recompute of one chunk from its checkpoint state (a, b) at
+// scale 2^q, keeping e_t, G_t = gy_t / d_t, y_t and b_{t-1}.
+template <typename T, bool FULL>
+__device__ __forceinline__ void chunk_recompute(const T* ks, const T* vs, const T* gs, int cnt, float qf, float U,
+                                                float lh, float ll, float a, float b, float (&E)[kL],
+                                                float (&G)[kL], float (&Y)[kL], float (&BP)[kL]) {
+#pragma unroll
+  for (int j = 0; j < kL; ++j) {
+    if (FULL || j < cnt) {
+      const float e = tok_weight(IO<T>::to_f(ks[j * 32]), qf);
+      const float eu = e * U;
+      const float vj = IO<T>::to_f(vs[j * 32]);
+      const float d = b + eu;
+      const float rd = __fdividef(1.f, d);
+      const bool ok = d > 0.f;  // d == 0: no history and e^{u+k} underflowed, WKV = v locally
+      Y[j] = ok ? fmaf(eu, vj, a) * rd : vj;
+      G[j] = ok ? IO<T>::to_f(gs[j * 32]) * rd : 0.f;
+      E[j] = e;
+      BP[j] = b;
+      a = decay_add(a, e * vj, lh, ll);
+      b = decay_add(b, e, lh, ll);
+    }
+  }
+}
+
+// Phase B: the chunk's own reverse sums from a zero carry at its end.
+template <bool FULL>
+__device__ __forceinline__ void chunk_local_sums(int cnt, const float (&G)[kL], const float (&Y)[kL], float lh,
+                                                 float ll, float& la, float& lg, float& ye) {
+  la = 0.f;
+  lg = 0.f;
+  ye = FULL ? Y[kL - 1] : 0.f;
+#pragma unroll
+  for (int j = kL - 1; j >= 0; --j) {
+    if (FULL || j < cnt) {
+      if (!FULL && j == cnt - 1) ye = Y[j];
+      la = decay_add(la, G[j], lh, ll);
+      if (j > 0) lg = decay_add(lg, (Y[j - 1] - Y[j]) * la, lh, ll);
+    }
+  }
+}
+
+// Phase D: the reverse walk of one chunk from its carry (al, ga) at the last
+// step, writing gk, gv upwards from row pointer gkp, gvp (rows C apart).
+template <typename T, bool FULL>
+__device__ __forceinline__ void chunk_walk(const T* vs, int cnt, const float (&E)[kL], const float (&G)[kL],
+                                           const float (&Y)[kL], const float (&BP)[kL], float U, float lh,
+                                           float ll, float al, float ga, T* gkp, T* gvp, size_t C, bool valid,
+                                           float& gws, float& gus) {
+#pragma unroll
+  for (int j = kL - 1; j >= 0; --j) {
+    if (FULL || j < cnt) {
+      const float vj = IO<T>::to_f(vs[j * 32]);
+      const float ug = U * G[j];
+      const float dv = vj - Y[j];
+      const float eu = E[j] * U;
+      const float gvt = E[j] * (ug + al);
+      const float gkt = fmaf(dv, gvt, E[j] * ga);
+      // α~ a_{t-1} + β~ b_{t-1} = b_{t-1} γ_t - α~ e^u e_t (v_t - y_t)
+      gws = fmaf(BP[j], ga, fmaf(-al * eu, dv, gws));
+      gus = fmaf(ug * E[j], dv, gus);
+      al = decay_add(al, G[j], lh, ll);
+      if (j > 0) ga = decay_add(ga, (Y[j - 1] - Y[j]) * al, lh, ll);
+      if (valid) {
+        gkp[(size_t)j * C] = IO<T>::from_f(gkt);
+        gvp[(size_t)j * C] = IO<T>::from_f(gvt);
+      }
+    }
+  }
+}
+
+struct RCarry {  // reverse carry at a chunk boundary, per lane (see phase C)
+  double a, g;
+  float y;
+  int p;
+};
+
+template <typename T>
+__global__ void __launch_bounds__(kW * 32, 4) wkv4_bwd_kernel(const __grid_constant__ CUtensorMap mk,
+                                                              const __grid_constant__ CUtensorMap mv,
+                                                              const __grid_constant__ CUtensorMap mg,
+                                                              const Bwd4Params p) {
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  constexpr uint32_t kBoxElems = kTile * 32;
+  constexpr uint32_t kBoxBytes = kBoxElems * sizeof(T);
+  T* tiles = reinterpret_cast<T*>(smem_raw);  // [stages][k|v|gy][kTile][32]
+  RSumm* rs = reinterpret_cast<RSumm*>(smem_raw + (size_t)p.stages * 3 * kBoxBytes);  // [2][kW][32]
+  RCarry* cslot = reinterpret_cast<RCarry*>(rs + 2 * kW * 32);                        // [2][32]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(cslot + 2 * 32);
+  int* abort_flag = reinterpret_cast<int*>(bars + p.stages);
+
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int ct = blockIdx.x % p.ctiles;
+  const int bb = blockIdx.x / p.ctiles;
+  const int c = ct * 32 + lane;
+  const bool valid = c < p.C;
+  const int ntile = (p.T + kTile - 1) / kTile;
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    prefetch_tensormap(&mk);
+    prefetch_tensormap(&mv);
+    prefetch_tensormap(&mg);
+    for (int s = 0; s < p.stages; ++s) mbar_init(&bars[s], 1);
+    fence_mbar_init();
+    const int pre = min(p.stages, ntile);
+    for (int s = 0; s < pre; ++s) {
+      const int tc = (ntile - 1 - s) * kTile;
+      mbar_arrive_expect_tx(&bars[s], 3 * kBoxBytes);
+      tma_load_3d(tiles + (size_t)(3 * s) * kBoxElems, &mk, &bars[s], ct * 32, tc, bb);
+      tma_load_3d(tiles + (size_t)(3 * s + 1) * kBoxElems, &mv, &bars[s], ct * 32, tc, bb);
+      tma_load_3d(tiles + (size_t)(3 * s + 2) * kBoxElems, &mg, &bars[s], ct * 32, tc, bb);
+    }
+  }
+  if (warp == 0) cslot[32 + lane] = RCarry{0.0, 0.0, 0.f, 0};  // nothing flows back from after the end
+  __syncthreads();
+
+  const float w = valid ? p.w[c] : 0.f;
+  const float u = valid ? p.u[c] : 0.f;
+  const double lam = exp(-(double)w);
+  const double lam15 = lam_pow(lam, kL - 1);
+  const float lh = (float)lam, ll = (float)(lam - (double)lh);
+  const float U = expf(u);
+  const size_t plane = (size_t)p.B * p.C;
+  const size_t lane_off = (size_t)bb * p.C + c;
+  const size_t C = (size_t)p.C;
+
+  double gw_acc = 0.0, gu_acc = 0.0;
+
+  for (int i = 0; i < ntile; ++i) {
+    const int tile = ntile - 1 - i;
+    const int s = i % p.stages;
+    const uint32_t ph = (uint32_t)(i / p.stages) & 1u;
+    const int tb = tile * kTile;
+    const int ts = tb + warp * kL;
+    const int cnt = max(0, min(kL, p.T - ts));
+    // checkpoint of this chunk (independent of the pipeline)
+    State st{0.0, 0.0, 0};
+    if (cnt > 0 && valid) {
+      const float* ck = p.ckpt + (size_t)(ts / kL) * 3 * plane + lane_off;
+      st = load_state(ck[0], ck[plane], ck[2 * plane]);
+    }
+    if (!mbar_wait_bounded(&bars[s], ph, p.err)) *abort_flag = 1;
+    const T* ks = tiles + (size_t)(3 * s) * kBoxElems + warp * kL * 32 + lane;
+    const T* vs = ks + kBoxElems;
+    const T* gs = vs + kBoxElems;
+
+    // A. forward recompute of the chunk at one scale 2^q
+    float E[kL], G[kL], Y[kL], BP[kL];
+    float kmax = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < kL; ++j)
+      if (j < cnt) kmax = fmaxf(kmax, IO<T>::to_f(ks[j * 32]) * kL2eHi);
+    const int q = cnt > 0 ? segment_scale(kmax, st) : 0;
+    st = rescale(st, q);
+    if (cnt == kL)
+      chunk_recompute<T, true>(ks, vs, gs, cnt, (float)q, U, lh, ll, (float)st.a, (float)st.b, E, G, Y, BP);
+    else if (cnt > 0)
+      chunk_recompute<T, false>(ks, vs, gs, cnt, (float)q, U, lh, ll, (float)st.a, (float)st.b, E, G, Y, BP);
+
+    // B. the chunk's own reverse sums
+    float la = 0.f, lg = 0.f, ye = 0.f;
+    if (cnt == kL)
+      chunk_local_sums<true>(cnt, G, Y, lh, ll, la, lg, ye);
+    else if (cnt > 0)
+      chunk_local_sums<false>(cnt, G, Y, lh, ll, la, lg, ye);
+    RSumm* sb = rs + (i & 1) * kW * 32;
+    sb[warp * 32 + lane] = RSumm{la, lg, cnt > 0 ? Y[0] : 0.f, ye, (float)q, 0.f};
+    __syncthreads();
+    if (*abort_flag) break;
+    if (threadIdx.x == 0 && i >= 1 && i - 1 + p.stages < ntile) {
+      const int sp = (i - 1) % p.stages;
+      const int tc = (ntile - 1 - (i - 1 + p.stages)) * kTile;
+      fence_proxy_async();
+      mbar_arrive_expect_tx(&bars[sp], 3 * kBoxBytes);
+      tma_load_3d(tiles + (size_t)(3 * sp) * kBoxElems, &mk, &bars[sp], ct * 32, tc, bb);
+      tma_load_3d(tiles + (size_t)(3 * sp + 1) * kBoxElems, &mv, &bars[sp], ct * 32, tc, bb);
+      tma_load_3d(tiles + (size_t)(3 * sp + 2) * kBoxElems, &mg, &bars[sp], ct * 32, tc, bb);
+    }
+
+    // C. fold the carries of the later chunks.  A carry is (α~ out of a chunk,
+    //    γ at that chunk's first step, y there) at scale 2^kp.  Entering a
+    //    chunk with last step e:   α~_e = α~,  γ_e = e^{-w} γ + (y_e - y) α~_e;
+    //    leaving it (n steps, first step s):
+    //      α~ = e^{-wn} α~_e + La,  γ_s = e^{-w(n-1)} (γ_e + (y_s - y_e) α~_e) + Lg.
+    //    Warp 0 folds all four chunks, giving the carry into the next tile.
+    const RCarry cin = cslot[((i + 1) & 1) * 32 + lane];
+    double ka = cin.a, kg = cin.g;
+    float ky = cin.y;
+    int kp = cin.p;
+    double ae = 0.0, ge = 0.0;  // this chunk's (α~_e, γ_e)
+    for (int j = kW - 1; j >= warp; --j) {
+      const int cj = max(0, min(kL, p.T - (tb + j * kL)));
+      if (cj == 0) continue;
+      const RSumm x = sb[j * 32 + lane];
+      // carries scale inversely to the state: α~ = α 2^q, so moving from 2^kp to 2^q multiplies by 2^(q - kp)
+      const double f = pow2d((int)x.q - kp);
+      const double a_e = ka * f;
+      const double g_e = fma(lam, kg * f, (double)(x.ye - ky) * a_e);
+      if (j == warp) {
+        ae = a_e;
+        ge = g_e;
+        if (warp != 0) break;
+      }
+      const double lamN1 = cj == kL ? lam15 : lam_pow(lam, cj - 1);
+      ka = fma(lamN1 * lam, a_e, (double)x.la);
+      kg = fma(lamN1, fma(a_e, (double)(x.ys - x.ye), g_e), (double)x.lg);
+      ky = x.ys;
+      kp = (int)x.q;
+    }
+    if (warp == 0) cslot[(i & 1) * 32 + lane] = RCarry{ka, kg, ky, kp};
+
+    // D. reverse walk with the true carry.  Besides α~ it carries
+    //   γ_t = y_t α~_t + β~_t = Σ_{s>t} e^{-(s-t-1)w} G_s (y_t - y_s),
+    // built from small increments (y_{t-1} - y_t) α~_{t-1}, so that
+    //   gk_t = (v_t - y_t) gv_t + e_t γ_t
+    // never subtracts two large nearly equal fp32 numbers.
+    if (cnt > 0) {
+      float gws = 0.f, gus = 0.f;
+      T* gkp = reinterpret_cast<T*>(p.gk) + ((size_t)bb * p.T + ts) * C + c;
+      T* gvp = reinterpret_cast<T*>(p.gv) + ((size_t)bb * p.T + ts) * C + c;
+      if (cnt == kL)
+        chunk_walk<T, true>(vs, cnt, E, G, Y, BP, U, lh, ll, (float)ae, (float)ge, gkp, gvp, C, valid, gws, gus);
+      else
+        chunk_walk<T, false>(vs, cnt, E, G, Y, BP, U, lh, ll, (float)ae, (float)ge, gkp, gvp, C, valid, gws, gus);
+      gw_acc += (double)gws;
+      gu_acc += (double)gus;
+    }
+  }
+
+  // reduce the four warps' gw, gu partials of each lane
+  __syncthreads();
+  double2* red = reinterpret_cast<double2*>(rs);
+  red[warp * 32 + lane] = make_double2(gw_acc, gu_acc);
+  __syncthreads();
+  if (warp == 0 && valid) {
+    double sw = 0.0, su = 0.0;
+#pragma unroll
+    for (int j = 0; j < kW; ++j) {
+      sw += red[j * 32 + lane].x;
+      su += red[j * 32 + lane].y;
+    }
+    p.part[lane_off] = -lam * sw;
+    p.part[plane + lane_off] = su;
+  }
+}
+
+// gw[c] = Σ_b part[0][b][c], gu[c] = Σ_b part[1][b][c], fp64, in batch order.
+__global__ void wkv4_reduce_wu_kernel(int B, int C, const double* __restrict__ part, float* __restrict__ gw,
+                                      float* __restrict__ gu) {
+  const int c = blockIdx.x * blockDim.x + threadIdx.x;
+  if (c >= C) return;
+  const size_t plane = (size_t)B * C;
+  double sw = 0.0, su = 0.0;
+  for (int b = 0; b < B; ++b) {
+    sw += part[(size_t)b * C + c];
+    su += part[plane + (size_t)b * C + c];
+  }
+  gw[c] = (float)sw;
+  gu[c] = (float)su;
+}
+
+template <typename T>
+size_t bwd_smem_bytes(int stages) {
+  return (size_t)stages * 3 * kTile * 32 * sizeof(T) + 2 * kW * 32 * sizeof(RSumm) + 2 * 32 * sizeof(RCarry) +
+         (size_t)stages * 8 + 16;
+}
+
+template <typename T>
+cudaError_t launch_bwd_t(const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mg, const Bwd4Params& p,
+                         cudaStream_t st) {
+  const size_t smem = bwd_smem_bytes<T>(p.stages);
+  static unsigned device_mask = 0;
+  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(wkv4_bwd_kernel<T>), (int)smem, &device_mask);
+  if (e != cudaSuccess) return e;
+  const long long nblk = (long long)p.ctiles * p.B;
+  wkv4_bwd_kernel<T><<<(unsigned)nblk, kW * 32, smem, st>>>(mk, mv, mg, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+int bwd_tile_steps() { return kTile; }
+
+int bwd_stages(bool bf16, int T) {
+  const int want = bf16 ? 4 : 2;  // 48 KB of boxes keeps four CTAs per SM
+  const int ntile = (T + kTile - 1) / kTile;
+  return max(2, min(want, ntile));
+}
+
+cudaError_t launch_wkv4_bwd(bool bf16, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mg,
+                            const Bwd4Params& p, cudaStream_t st) {
+  return bf16 ? launch_bwd_t<__nv_bfloat16>(mk, mv, mg, p, st) : launch_bwd_t<float>(mk, mv, mg, p, st);
+}
+
+cudaError_t launch_wkv4_reduce_wu(int B, int C, const double* part, float* gw, float* gu, cudaStream_t st) {
+  wkv4_reduce_wu_kernel<<<(C + 127) / 128, 128, 0, st>>>(B, C, part, gw, gu);
+  return cudaGetLastError();
+}
+
+}  // namespace rwkv

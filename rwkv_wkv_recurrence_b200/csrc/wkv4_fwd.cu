@@ -1,0 +1,306 @@
+// RWKV-4 WKV forward kernels (sm_100a).
+//
+// Operator: "RWKV - Transformer 시대에 RNN을 재발명하다", Method / (2) Time-mixing
+// (WKV), time-parallel formula and its recurrent form; identical formula in
+// "RWKV: Reinventing RNNs for the Transformer Era" (flashpapers), 3. How It
+// Works / The WKV Operator.  The time-parallel form is a decayed prefix sum of
+// numerator and denominator, and "exp decay + sum" is associative: that is
+// what lets each warp below scan its own 16 steps independently and have the
+// pieces joined by a fold.
+//
+// Kernel shape.  A CTA owns 32 consecutive channels of one batch row (one
+// thread per channel lane in each warp) over a range of time, processed in
+// tiles of 64 steps.  The 4 warps split a tile into four 16-step segments:
+//   1. each warp scans its segment from a zero state (segment summary),
+//   2. each warp folds the CTA's running state with the summaries before its
+//      segment (and all four, for the next tile),
+//   3. each warp rescans its segment from that state and writes y (and, at
+//      segment starts, the checkpoints the backward reads).
+// k and v arrive in [64 x 32] boxes through a multi-stage TMA pipeline
+// without multicast, so every input element is read from HBM once.
+//
+// Precision.  Steps inside a segment run in fp32 with the decay applied as
+// e^{-w} = lh + ll (hi and lo fp32 parts), one power-of-two scale per segment;
+// the running state carried from segment to segment is fp64.  So fp32 rounding
+// accumulates over 16 steps at most, never over the whole sequence, which the
+// backward's cancelling gradient terms would not tolerate.
+#include "launch.h"
+#include "wkv_common.cuh"
+
+namespace rwkv {
+namespace {
+
+constexpr int kW = 4;           // warps per CTA = segments per tile
+constexpr int kL = 16;          // steps per segment (= checkpoint interval)
+constexpr int kTile = kW * kL;  // steps per tile
+
+struct Summ {  // a segment scanned from a zero state, at scale 2^p
+  float a, b, p, pad;
+};
+
+// Phase 1 of one segment: scan from a zero state at scale 2^p1, where p1 is
+// at least every k log2 e of the segment (so all weights are <= 1).  Keeps
+// the token weights for phase 3.
+template <typename T, bool FULL>
+__device__ __forceinline__ void seg_summary(const T* ks, const T* vs, int cnt, float lh, float ll, float& kmax,
+                                            int& p1, float& la, float& lb, float (&E)[kL]) {
+  float kk[kL];
+  kmax = -INFINITY;
+#pragma unroll
+  for (int j = 0; j < kL; ++j) {
+    if (FULL || j < cnt) {
+      kk[j] = IO<T>::to_f(ks[j * 32]);
+      kmax = fmaxf(kmax, kk[j] * kL2eHi);
+    }
+  }
+  p1 = clamp_scale((int)fminf(fmaxf(ceilf(kmax), -(float)kScaleMax), (float)kScaleMax));
+  const float p1f = (float)p1;
+  la = 0.f;
+  lb = 0.f;
+#pragma unroll
+  for (int j = 0; j < kL; ++j) {
+    if (FULL || j < cnt) {
+      const float e = tok_weight(kk[j], p1f);
+      E[j] = e;
+      la = decay_add(la, e * IO<T>::to_f(vs[j * 32]), lh, ll);
+      lb = decay_add(lb, e, lh, ll);
+    }
+  }
+}
+
+// Phase 3 of one segment: rescan from the true state (a, b) at the segment's
+// scale, weights E * f, writing y to yp, yp + C, ...
+template <typename T, bool FULL>
+__device__ __forceinline__ void seg_output(const T* vs, int cnt, const float (&E)[kL], float f, float U, float a,
+                                           float b, float lh, float ll, T* yp, size_t C, bool valid) {
+#pragma unroll
+  for (int j = 0; j < kL; ++j) {
+    if (FULL || j < cnt) {
+      const float e = E[j] * f;
+      const float eu = e * U;
+      const float vj = IO<T>::to_f(vs[j * 32]);
+      const float d = b + eu;
+      const float n = fmaf(eu, vj, a);
+      const float y = d > 0.f ? __fdividef(n, d) : vj;  // d == 0: no history and e^{u+k} underflowed
+      if (valid) *yp = IO<T>::from_f(y);
+      yp += C;
+      a = decay_add(a, e * vj, lh, ll);
+      b = decay_add(b, e, lh, ll);
+    }
+  }
+}
+
+struct CarrySlot {  // CTA running state at a tile boundary, per lane
+  double a, b;
+  int p, pad;
+};
+
+template <typename T>
+__global__ void __launch_bounds__(kW * 32, 4) wkv4_fwd_kernel(const __grid_constant__ CUtensorMap mk,
+                                                              const __grid_constant__ CUtensorMap mv,
+                                                              const Fwd4Params p) {
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  constexpr uint32_t kBoxElems = kTile * 32;
+  constexpr uint32_t kBoxBytes = kBoxElems * sizeof(T);
+  T* tiles = reinterpret_cast<T*>(smem_raw);  // [stages][k|v][kTile][32]
+  Summ* summ = reinterpret_cast<Summ*>(smem_raw + (size_t)p.stages * 2 * kBoxBytes);  // [2][kW][32]
+  CarrySlot* cslot = reinterpret_cast<CarrySlot*>(summ + 2 * kW * 32);                // [2][32]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(cslot + 2 * 32);                         // [stages]
+  int* abort_flag = reinterpret_cast<int*>(bars + p.stages);
+
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  int blk = blockIdx.x;
+  const int ct = blk % p.ctiles;
+  blk /= p.ctiles;
+  const int bb = blk % p.B;
+  const int seg = blk / p.B;
+  const int c = ct * 32 + lane;
+  const bool valid = c < p.C;
+  const int t0 = seg * p.seg_len;
+  const int t1 = min(p.T, t0 + p.seg_len);
+  const int ntile = (t1 - t0 + kTile - 1) / kTile;
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    prefetch_tensormap(&mk);
+    prefetch_tensormap(&mv);
+    for (int s = 0; s < p.stages; ++s) mbar_init(&bars[s], 1);
+    fence_mbar_init();
+    const int pre = min(p.stages, ntile);
+    for (int s = 0; s < pre; ++s) {
+      mbar_arrive_expect_tx(&bars[s], 2 * kBoxBytes);
+      tma_load_3d(tiles + (size_t)(2 * s) * kBoxElems, &mk, &bars[s], ct * 32, t0 + s * kTile, bb);
+      tma_load_3d(tiles + (size_t)(2 * s + 1) * kBoxElems, &mv, &bars[s], ct * 32, t0 + s * kTile, bb);
+    }
+  }
+
+  const float w = valid ? p.w[c] : 0.f;
+  const float u = valid ? p.u[c] : 0.f;
+  const double lam = exp(-(double)w);
+  const double lam16 = lam_pow(lam, kL);
+  const float lh = (float)lam, ll = (float)(lam - (double)lh);
+  const float U = expf(u);
+  const size_t plane = (size_t)p.B * p.C;
+  const size_t lane_off = (size_t)bb * p.C + c;
+  const size_t C = (size_t)p.C;
+
+  if (warp == kW - 1) {  // running state entering the first tile
+    State s0{0.0, 0.0, 0};
+    if (p.start != nullptr && valid) {
+      const float* sp = p.start + (size_t)seg * p.start_seg_stride;
+      s0 = load_state(sp[lane_off], sp[plane + lane_off], sp[2 * plane + lane_off]);
+    }
+    cslot[32 + lane] = CarrySlot{s0.a, s0.b, s0.p, 0};  // slot of "tile -1"
+  }
+  __syncthreads();
+
+  T* ybase = p.y ? reinterpret_cast<T*>(p.y) + (size_t)bb * p.T * C + c : nullptr;
+  const bool rescan = (p.y != nullptr) || (p.ckpt != nullptr);
+  State total{0.0, 0.0, 0};
+
+  for (int i = 0; i < ntile; ++i) {
+    const int s = i % p.stages;
+    const uint32_t ph = (uint32_t)(i / p.stages) & 1u;
+    if (!mbar_wait_bounded(&bars[s], ph, p.err)) *abort_flag = 1;
+    const int tb = t0 + i * kTile;
+    const int ts = tb + warp * kL;
+    const int cnt = max(0, min(kL, t1 - ts));
+    const T* ks = tiles + (size_t)(2 * s) * kBoxElems + warp * kL * 32 + lane;
+    const T* vs = ks + kBoxElems;
+
+    // 1. this warp's segment from a zero state
+    float E[kL], kmax = -INFINITY, la = 0.f, lb = 0.f;
+    int p1 = 0;
+    if (cnt == kL)
+      seg_summary<T, true>(ks, vs, cnt, lh, ll, kmax, p1, la, lb, E);
+    else if (cnt > 0)
+      seg_summary<T, false>(ks, vs, cnt, lh, ll, kmax, p1, la, lb, E);
+    Summ* sb = summ + (i & 1) * kW * 32;
+    sb[warp * 32 + lane] = Summ{la, lb, (float)p1, 0.f};
+    __syncthreads();
+    if (*abort_flag) break;
+    // every warp is done with tile i-1: refill its stage
+    if (threadIdx.x == 0 && i >= 1 && i - 1 + p.stages < ntile) {
+      const int sp = (i - 1) % p.stages;
+      const int tn = t0 + (i - 1 + p.stages) * kTile;
+      fence_proxy_async();
+      mbar_arrive_expect_tx(&bars[sp], 2 * kBoxBytes);
+      tma_load_3d(tiles + (size_t)(2 * sp) * kBoxElems, &mk, &bars[sp], ct * 32, tn, bb);
+      tma_load_3d(tiles + (size_t)(2 * sp + 1) * kBoxElems, &mv, &bars[sp], ct * 32, tn, bb);
+    }
+
+    // 2. fold: the state at this warp's segment start is the running state
+    //    folded with the summaries of the segments before it; the last warp
+    //    also folds its own, giving the running state for the next tile.
+    const CarrySlot cs = cslot[((i + 1) & 1) * 32 + lane];
+    State mine{cs.a, cs.b, cs.p};
+    for (int j = 0; j < warp; ++j) {
+      const int cj = max(0, min(kL, t1 - (tb + j * kL)));
+      if (cj > 0) {
+        const Summ x = sb[j * 32 + lane];
+        mine = fold(mine, cj == kL ? lam16 : lam_pow(lam, cj), State{(double)x.a, (double)x.b, (int)x.p});
+      }
+    }
+    if (warp == kW - 1) {
+      total = mine;
+      if (cnt > 0) total = fold(mine, cnt == kL ? lam16 : lam_pow(lam, cnt), State{(double)la, (double)lb, p1});
+      cslot[(i & 1) * 32 + lane] = CarrySlot{total.a, total.b, total.p, 0};
+    }
+
+    // 3. rescan from the true state: outputs and checkpoints
+    if (cnt > 0 && rescan) {
+      if (p.ckpt != nullptr && valid && (ts % p.ckpt_len) == 0) {
+        float* ck = p.ckpt + (size_t)(ts / p.ckpt_len) * 3 * plane + lane_off;
+        store_state(mine, &ck[0], &ck[plane], &ck[2 * plane]);
+      }
+      if (ybase != nullptr) {
+        const int q = segment_scale(kmax, mine);
+        const State sc = rescale(mine, q);
+        const float f = pow2f_neg(p1 - q);
+        T* yp = ybase + (size_t)ts * C;
+        if (cnt == kL)
+          seg_output<T, true>(vs, cnt, E, f, U, (float)sc.a, (float)sc.b, lh, ll, yp, C, valid);
+        else
+          seg_output<T, false>(vs, cnt, E, f, U, (float)sc.a, (float)sc.b, lh, ll, yp, C, valid);
+      }
+    }
+  }
+
+  if (p.end != nullptr && valid && warp == kW - 1) {
+    float* e = p.end + (size_t)seg * p.end_seg_stride;
+    store_state(total, &e[lane_off], &e[plane + lane_off], &e[2 * plane + lane_off]);
+  }
+}
+
+// Carry pass of the multi-CTA (chunked) forward: turns per-segment summaries
+// (each the state reached from a zero state over that segment alone) into the
+// state at the start of every segment, in place, by the associative fold
+//   S_{<=j} = e^{-w len_j} S_{<=j-1}  (+)  summary_j,
+// and writes the final state.  One thread per lane (b, c), fp64 arithmetic.
+__global__ void wkv4_carry_kernel(int B, int C, int T, int nseg, int seg_len, const float* __restrict__ w,
+                                  const float* __restrict__ state_in, float* __restrict__ ws,
+                                  float* __restrict__ state_out) {
+  const size_t plane = (size_t)B * C;
+  const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= plane) return;
+  const int c = (int)(i % C);
+  State st{0.0, 0.0, 0};
+  if (state_in != nullptr) st = load_state(state_in[i], state_in[plane + i], state_in[2 * plane + i]);
+  const double lam = exp(-(double)w[c]);
+  const double lam16 = lam_pow(lam, 16);
+  for (int j = 0; j < nseg; ++j) {
+    float* sj = ws + (size_t)j * 3 * plane + i;
+    const State x = load_state(sj[0], sj[plane], sj[2 * plane]);
+    store_state(st, &sj[0], &sj[plane], &sj[2 * plane]);
+    // e^{-w len} as the product of len factors e^{-w}, len = 16 q + r
+    const int len = min(seg_len, T - j * seg_len);
+    double lamL = lam_pow(lam, len & 15);
+    for (int q = 0; q < (len >> 4); ++q) lamL *= lam16;
+    st = fold(st, lamL, x);
+  }
+  if (state_out != nullptr) store_state(st, &state_out[i], &state_out[plane + i], &state_out[2 * plane + i]);
+}
+
+template <typename T>
+size_t fwd_smem_bytes(int stages) {
+  return (size_t)stages * 2 * kTile * 32 * sizeof(T) + 2 * kW * 32 * sizeof(Summ) + 2 * 32 * sizeof(CarrySlot) +
+         (size_t)stages * 8 + 16;
+}
+
+template <typename T>
+cudaError_t launch_fwd_t(const CUtensorMap& mk, const CUtensorMap& mv, const Fwd4Params& p, cudaStream_t st) {
+  const size_t smem = fwd_smem_bytes<T>(p.stages);
+  static unsigned device_mask = 0;
+  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(wkv4_fwd_kernel<T>), (int)smem, &device_mask);
+  if (e != cudaSuccess) return e;
+  const long long nblk = (long long)p.ctiles * p.B * p.nseg;
+  wkv4_fwd_kernel<T><<<(unsigned)nblk, kW * 32, smem, st>>>(mk, mv, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+int fwd_tile_steps() { return kTile; }
+
+int fwd_stages(bool bf16, int seg_len) {
+  // three stages of fp32 boxes (48 KB) keep four CTAs per SM; bf16 boxes are half as big
+  const int want = bf16 ? 6 : 3;
+  const int ntile = (seg_len + kTile - 1) / kTile;
+  return max(2, min(want, ntile));
+}
+
+cudaError_t launch_wkv4_fwd(bool bf16, const CUtensorMap& mk, const CUtensorMap& mv, const Fwd4Params& p,
+                            cudaStream_t st) {
+  return bf16 ? launch_fwd_t<__nv_bfloat16>(mk, mv, p, st) : launch_fwd_t<float>(mk, mv, p, st);
+}
+
+cudaError_t launch_wkv4_carry(int B, int C, int T, int nseg, int seg_len, const float* w, const float* state_in,
+                              float* ws, float* state_out, cudaStream_t st) {
+  const size_t n = (size_t)B * C;
+  const unsigned grid = (unsigned)((n + 255) / 256);
+  wkv4_carry_kernel<<<grid, 256, 0, st>>>(B, C, T, nseg, seg_len, w, state_in, ws, state_out);
+  return cudaGetLastError();
+}
+
+}  // namespace rwkv

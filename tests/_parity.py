@@ -1,0 +1,93 @@
+"""Comparison rules shared by the GPU parity tests.
+
+Tolerances (stated once, used everywhere):
+* fp32 WKV-4 outputs:      |got - ref| <= 1e-5 * max(1, |ref|)
+* fp32 WKV-4 gradients gk, gv:   |got - ref| <= 1e-4 * max(1, |ref|) elementwise
+* fp32 WKV-4 gradients gw, gu (each entry a sum over B*T terms that cancel):
+                           max |got - ref| <= 1e-4 * max(1, max |ref|)  (norm-wise)
+* bf16 I/O (fp32 inside):  |got - ref| <= 8e-3 * max(|ref|, rms(ref))
+  (rms over the compared tensor; a bf16 output alone is rounded by <= 2^-9 relative)
+* WKV-4 states compare through a/b (1e-5 * max(1, |A/B|)) and log2 b + p
+  (2e-5 absolute), because (a, b, p) is defined only up to a power of two.
+"""
+import numpy as np
+import torch
+
+TOL_Y = 1e-5
+TOL_GRAD = 1e-4
+TOL_BF16 = 8e-3
+
+
+def _np(x):
+    if isinstance(x, torch.Tensor):
+        x = x.detach().cpu()
+        if x.dtype == torch.bfloat16:
+            x = x.float()
+        return x.double().numpy()
+    return np.asarray(x, dtype=np.float64)
+
+
+def assert_close_abs1(got, ref, tol, what=""):
+    """|got - ref| <= tol * max(1, |ref|) elementwise."""
+    g, r = _np(got), _np(ref)
+    assert g.shape == r.shape, (what, g.shape, r.shape)
+    assert np.all(np.isfinite(g)), f"{what}: non-finite GPU values"
+    bound = tol * np.maximum(1.0, np.abs(r))
+    err = np.abs(g - r)
+    worst = np.unravel_index(np.argmax(err / bound), err.shape)
+    assert np.all(err <= bound), (f"{what}: max |err|/bound = {np.max(err / bound):.3g} at {worst}: "
+                                  f"got {g[worst]!r} ref {r[worst]!r}")
+    return float(np.max(err / bound))
+
+
+def assert_close_normwise(got, ref, tol, what=""):
+    """max |got - ref| <= tol * max(1, max |ref|): relative error of a vector of
+    reductions, measured against its largest entry."""
+    g, r = _np(got), _np(ref)
+    assert g.shape == r.shape, (what, g.shape, r.shape)
+    assert np.all(np.isfinite(g)), f"{what}: non-finite GPU values"
+    bound = tol * max(1.0, float(np.max(np.abs(r))))
+    err = float(np.max(np.abs(g - r)))
+    assert err <= bound, f"{what}: max |err| = {err:.3g} > {bound:.3g} (norm-wise)"
+    return err / bound
+
+
+def assert_grads_close(got, ref, what=""):
+    """(gk, gv, gw, gu) against the oracle: elementwise for gk, gv, norm-wise for gw, gu."""
+    for g, r, name in zip(got, ref, ("gk", "gv", "gw", "gu")):
+        if name in ("gk", "gv"):
+            assert_close_abs1(g, r, TOL_GRAD, f"{what}{name}")
+        else:
+            assert_close_normwise(g, r, TOL_GRAD, f"{what}{name}")
+
+
+def assert_close_rms(got, ref, tol, what=""):
+    """|got - ref| <= tol * max(|ref|, rms(ref)) elementwise."""
+    g, r = _np(got), _np(ref)
+    assert g.shape == r.shape, (what, g.shape, r.shape)
+    assert np.all(np.isfinite(g)), f"{what}: non-finite GPU values"
+    rms = float(np.sqrt(np.mean(r * r)))
+    bound = tol * np.maximum(np.abs(r), rms)
+    err = np.abs(g - r)
+    worst = np.unravel_index(np.argmax(err / bound), err.shape)
+    assert np.all(err <= bound), (f"{what}: max |err|/bound = {np.max(err / bound):.3g} at {worst}: "
+                                  f"got {g[worst]!r} ref {r[worst]!r}")
+    return float(np.max(err / bound))
+
+
+def assert_state_close(gpu_state, ref_ab, what="state"):
+    """gpu_state [3,...] = (a, b, p); ref_ab [2,...] = (A, B) in fp64."""
+    s = _np(gpu_state)
+    r = _np(ref_ab)
+    a, b, p = s[0], s[1], s[2]
+    assert_close_abs1(a / b, r[0] / r[1], TOL_Y, what + " a/b")
+    lg = np.log2(b) + p
+    lr = np.log2(r[1])
+    assert np.all(np.abs(lg - lr) <= 2e-5), f"{what}: log2 b + p off by {np.max(np.abs(lg - lr)):.3g}"
+
+
+def sample_lanes(B, C, n, seed=0):
+    """n distinct (b, c) lanes, reproducibly."""
+    rng = np.random.default_rng(seed)
+    flat = rng.choice(B * C, size=min(n, B * C), replace=False)
+    return torch.from_numpy(flat // C), torch.from_numpy(flat % C)

@@ -1,0 +1,115 @@
+"""Host-side checks of the C-ABI library, no GPU needed: it loads, it exports
+every function that include/rwkv_wkv.h declares, and argument validation
+answers before any CUDA work is enqueued."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import rwkv_wkv_recurrence_b200 as rw
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = []
+    inc = os.path.join(ROOT, "include")
+    for f in sorted(os.listdir(inc)):
+        if f.endswith(".h"):
+            src = open(os.path.join(inc, f)).read()
+            names += re.findall(r"^RWKV_API\s+[\w\s\*]+?\**\s*(\w+)\s*\(", src, flags=re.M)
+    return names
+
+
+def test_library_exports_every_declared_symbol():
+    names = _declared()
+    assert "rwkv_wkv4_forward" in names and "rwkv_wkv5_forward" in names
+    h = ctypes.CDLL(rw.LIB_PATH)
+    missing = [n for n in names if not hasattr(h, n)]
+    assert not missing, missing
+
+
+def test_status_strings_and_version():
+    h = rw.lib()
+    assert h.rwkv_status_string(0) == b"ok"
+    for s in range(1, 6):
+        assert h.rwkv_status_string(s) not in (b"ok", b"unknown status")
+    assert h.rwkv_status_string(99) == b"unknown status"
+    assert h.rwkv_version() >> 16 == 1
+
+
+def test_checkpoint_and_workspace_queries():
+    h = rw.lib()
+    assert h.rwkv_wkv4_num_checkpoints(4096, 16) == 256
+    assert h.rwkv_wkv4_num_checkpoints(4097, 16) == 257
+    assert h.rwkv_wkv4_num_checkpoints(0, 16) == 0
+    assert h.rwkv_wkv4_num_checkpoints(100, 12) == -1
+    assert h.rwkv_wkv4_num_checkpoints(100, 0) == -1
+    B, T, C = 8, 4096, 2048
+    assert h.rwkv_wkv4_backward_workspace_bytes(B, T, C, 16, 1) == 2 * B * C * 8
+    assert h.rwkv_wkv4_backward_workspace_bytes(B, T, C, 16, 0) == 2 * B * C * 8 + 256 * 3 * B * C * 4
+    # many channels: the sequential schedule needs no workspace
+    assert h.rwkv_wkv4_forward_workspace_bytes(B, T, C, rw.ALGO_AUTO) == 0
+    assert h.rwkv_wkv4_forward_workspace_bytes(B, T, C, rw.ALGO_SEQUENTIAL) == 0
+    # few channels: the chunked schedule keeps one state per segment
+    ws = h.rwkv_wkv4_forward_workspace_bytes(8, 1024, 768, rw.ALGO_AUTO)
+    assert ws > 0 and ws % (3 * 8 * 768 * 4) == 0
+    assert h.rwkv_wkv4_forward_workspace_bytes(0, 10, 10, 0) == 0
+
+
+def test_validation_before_any_cuda_work():
+    h = rw.lib()
+    P = ctypes.c_void_p
+    fake = P(0x1000)  # never dereferenced: every call below fails validation first
+    # negative sizes
+    assert h.rwkv_wkv4_forward(-1, 4, 4, 0, fake, fake, fake, fake, fake, None, None, None, 16, 0, None, 0,
+                               None) == 1
+    # bad dtype / algo
+    assert h.rwkv_wkv4_forward(1, 4, 4, 7, fake, fake, fake, fake, fake, None, None, None, 16, 0, None, 0,
+                               None) == 1
+    assert h.rwkv_wkv4_forward(1, 4, 4, 0, fake, fake, fake, fake, fake, None, None, None, 16, 9, None, 0,
+                               None) == 1
+    # checkpoint interval not a multiple of 16 / not supported
+    assert h.rwkv_wkv4_forward(1, 4, 4, 0, fake, fake, fake, fake, fake, None, None, fake, 12, 0, None, 0,
+                               None) == 1
+    assert h.rwkv_wkv4_forward(1, 4, 4, 0, fake, fake, fake, fake, fake, None, None, fake, 32, 0, None, 0,
+                               None) == 2
+    # empty problems are a no-op
+    assert h.rwkv_wkv4_forward(0, 4, 4, 0, fake, fake, fake, fake, fake, None, None, None, 16, 0, None, 0,
+                               None) == 0
+    # null required pointers
+    assert h.rwkv_wkv4_forward(1, 4, 4, 0, None, fake, fake, fake, fake, None, None, None, 16, 0, None, 0,
+                               None) == 1
+    assert h.rwkv_wkv4_forward(1, 4, 4, 0, fake, fake, None, fake, fake, None, None, None, 16, 0, None, 0,
+                               None) == 1
+    # misaligned k, or a row pitch that is not a multiple of 16 bytes
+    assert h.rwkv_wkv4_forward(1, 4, 4, 0, fake, fake, P(0x1004), fake, fake, None, None, None, 16, 0, None,
+                               0, None) == 2
+    assert h.rwkv_wkv4_forward(1, 4, 6, 0, fake, fake, fake, fake, fake, None, None, None, 16, 0, None, 0,
+                               None) == 2
+    # chunked schedule without its workspace
+    assert h.rwkv_wkv4_forward(8, 1024, 768, 0, fake, fake, fake, fake, fake, None, None, None, 16, 0, None, 0,
+                               None) == 3
+    # backward: bad interval, missing workspace, null gradient
+    assert h.rwkv_wkv4_backward(1, 4, 4, 0, fake, fake, fake, fake, fake, None, fake, 8, fake, fake, fake,
+                                fake, fake, 1 << 20, None) == 1
+    assert h.rwkv_wkv4_backward(1, 4, 4, 0, fake, fake, fake, fake, fake, None, fake, 16, fake, fake, fake,
+                                fake, None, 0, None) == 3
+    assert h.rwkv_wkv4_backward(1, 4, 4, 0, fake, fake, fake, fake, fake, None, fake, 16, None, fake, fake,
+                                fake, fake, 1 << 20, None) == 1
+    # step: null output state
+    assert h.rwkv_wkv4_step(2, 4, 0, fake, fake, fake, fake, fake, None, None, None) == 1
+    assert h.rwkv_wkv4_step(-2, 4, 0, fake, fake, fake, fake, fake, None, fake, None) == 1
+    # WKV-5: only N = 64
+    assert h.rwkv_wkv5_forward(1, 4, 2, 32, fake, fake, fake, fake, fake, fake, None, None, None, 0,
+                               None) == 2
+    assert h.rwkv_wkv5_forward(1, 4, 2, 64, fake, fake, fake, None, fake, fake, None, None, None, 0,
+                               None) == 1
+
+
+def test_binding_fails_loudly_without_library(monkeypatch):
+    monkeypatch.setattr(rw, "_lib", None)
+    monkeypatch.setattr(rw, "LIB_PATH", "/nonexistent/librwkv_wkv.so")
+    with pytest.raises(RuntimeError, match="missing"):
+        rw.lib()

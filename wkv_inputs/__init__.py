@@ -116,15 +116,17 @@ def normal(seed: int, tid: int, idx: torch.Tensor) -> torch.Tensor:
     return rad * torch.cos((2.0 * math.pi) * u2)
 
 
-def _index_btc(B: int, T: int, C: int, t0: int, t1: int, b_sel, c_sel, device):
+def _index_btc(B: int, T: int, C: int, t0: int, t1: int, b_sel, c_sel, device, b0=0, b1=None):
     """Flat indices (b*T + t)*C + c of the [B, T, C] tensor for t in [t0, t1).
 
-    Without a selection the result is [B, t1-t0, C]; with ``b_sel``/``c_sel``
-    (equal-length 1-D index tensors naming lanes) it is [t1-t0, n_lanes].
+    Without a selection the result is [b1-b0, t1-t0, C] for batch rows
+    [b0, b1); with ``b_sel``/``c_sel`` (equal-length 1-D index tensors naming
+    lanes) it is [t1-t0, n_lanes].
     """
     t = torch.arange(t0, t1, device=device, dtype=torch.int64)
     if b_sel is None:
-        b = torch.arange(B, device=device, dtype=torch.int64).view(B, 1, 1)
+        b1 = B if b1 is None else b1
+        b = torch.arange(b0, b1, device=device, dtype=torch.int64).view(-1, 1, 1)
         c = torch.arange(C, device=device, dtype=torch.int64).view(1, 1, C)
         return (b * T + t.view(1, -1, 1)) * C + c
     b_sel = torch.as_tensor(b_sel, dtype=torch.int64, device=device).view(1, -1)
@@ -134,8 +136,10 @@ def _index_btc(B: int, T: int, C: int, t0: int, t1: int, b_sel, c_sel, device):
 
 def btc_field(kind: str, seed: int, B: int, T: int, C: int, t0: int = 0, t1=None,
               b_sel=None, c_sel=None, outliers: bool = False,
-              dtype=torch.float32, device="cpu", block: int = 1 << 23) -> torch.Tensor:
-    """A [B, T, C] input (k, v or gy) restricted to time steps [t0, t1).
+              dtype=torch.float32, device="cpu", block: int = 1 << 23,
+              b0: int = 0, b1=None) -> torch.Tensor:
+    """A [B, T, C] input (k, v or gy) restricted to time steps [t0, t1) and
+    batch rows [b0, b1) (or to the lanes ``b_sel``, ``c_sel``).
 
     ``outliers`` replaces each key, independently with probability 0.01, by
     ``s * U(20, 40)`` with a fair random sign ``s`` (the heavy-tailed keys that
@@ -143,7 +147,7 @@ def btc_field(kind: str, seed: int, B: int, T: int, C: int, t0: int = 0, t1=None
     """
     t1 = T if t1 is None else t1
     tid = TID[kind]
-    idx = _index_btc(B, T, C, t0, t1, b_sel, c_sel, device)
+    idx = _index_btc(B, T, C, t0, t1, b_sel, c_sel, device, b0, b1)
     flat = idx.reshape(-1)
     out = torch.empty(flat.numel(), dtype=dtype, device=device)
     for s in range(0, flat.numel(), block):
