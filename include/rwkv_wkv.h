@@ -160,6 +160,34 @@ RWKV_API rwkv_status rwkv_wkv5_forward(int64_t B, int64_t T, int64_t H, int64_t 
                               const float *s_in, float *s_out,
                               void *workspace, size_t workspace_bytes, rwkv_stream_t stream);
 
+/* Largest B * C that rwkv_wkv4_backward_noalloc accepts. */
+#define RWKV_NOALLOC_MAX_LANES 262144
+
+/*
+ * WKV-4 backward that allocates nothing and needs no workspace.
+ * The pages have no counterpart: this is a library convenience for callers
+ * that cannot allocate device memory where they run the backward (device
+ * memory owned in full by another allocator, latency-critical loops that
+ * must not pay cudaMalloc's implicit synchronisation, systems that allocate
+ * only at start-up).  Same arguments and results as rwkv_wkv4_backward with
+ * ckpt required (the forward's checkpoints) and no workspace; the per-lane
+ * scratch lives in a fixed array inside the library (RWKV_NOALLOC_MAX_LANES
+ * lanes, 4 MiB, held on every GPU that loads the library until exit).
+ *   - B * C > RWKV_NOALLOC_MAX_LANES returns RWKV_ERR_WORKSPACE (too big for
+ *     the fixed scratch); ckpt == NULL returns RWKV_ERR_INVALID_ARG.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - All calls share the array: calls whose GPU work overlaps (other
+ *     streams, other threads) race and must be ordered by the caller.
+ *   - Calls no cudaMalloc, cudaFree or allocating library routine.
+ */
+RWKV_API rwkv_status rwkv_wkv4_backward_noalloc(int64_t B, int64_t T, int64_t C, rwkv_dtype dtype,
+                                                const float *w, const float *u, const void *k,
+                                                const void *v, const void *gy, const float *ckpt,
+                                                int64_t chunk_len, void *gk, void *gv, float *gw,
+                                                float *gu, rwkv_stream_t stream);
+
 /*
  * Synchronises `stream`, then reports and clears the device error word that
  * kernels set when a bounded wait gives up (RWKV_ERR_DEVICE_TIMEOUT), or

@@ -20,7 +20,8 @@ import os
 
 __all__ = [
     "LIB_PATH", "lib", "RwkvError", "RWKV_OK", "F32", "BF16", "ALGO_AUTO", "ALGO_SEQUENTIAL",
-    "ALGO_CHUNKED", "CHUNK_LEN", "rwkv_wkv4_forward", "rwkv_wkv4_backward", "rwkv_wkv4_step",
+    "ALGO_CHUNKED", "CHUNK_LEN", "NOALLOC_MAX_LANES", "rwkv_wkv4_forward", "rwkv_wkv4_backward",
+    "rwkv_wkv4_backward_noalloc", "rwkv_wkv4_step",
     "rwkv_wkv5_forward", "rwkv_check_device_error", "state_to_ab",
 ]
 
@@ -30,6 +31,7 @@ RWKV_OK = 0
 F32, BF16 = 0, 1
 ALGO_AUTO, ALGO_SEQUENTIAL, ALGO_CHUNKED = 0, 1, 2
 CHUNK_LEN = 16  # checkpoint interval of the WKV-4 forward/backward pair
+NOALLOC_MAX_LANES = 262144  # RWKV_NOALLOC_MAX_LANES: largest B*C of rwkv_wkv4_backward_noalloc
 
 _lib = None
 
@@ -62,6 +64,7 @@ def lib():
         "rwkv_wkv4_step": ([I64, I64, I, P, P, P, P, P, P, P, P], I),
         "rwkv_wkv5_forward_workspace_bytes": ([I64, I64, I64, I64], S),
         "rwkv_wkv5_forward": ([I64, I64, I64, I64, P, P, P, P, P, P, P, P, P, S, P], I),
+        "rwkv_wkv4_backward_noalloc": ([I64, I64, I64, I, P, P, P, P, P, P, I64, P, P, P, P, P], I),
         "rwkv_check_device_error": ([P], I),
     }
     for name, (args, res) in sig.items():
@@ -175,6 +178,29 @@ def rwkv_wkv4_backward(w, u, k, v, gy, ckpt=None, state_in=None, *, stream=None,
            h.rwkv_wkv4_backward(B, T, C, _dtype_code(k), _ptr(w), _ptr(u), _ptr(k), _ptr(v), _ptr(gy),
                                 _ptr(state_in), _ptr(ckpt), CHUNK_LEN, _ptr(gk), _ptr(gv), _ptr(gw),
                                 _ptr(gu), _ptr(ws), wsb, _stream(stream)))
+    return gk, gv, gw, gu
+
+
+def rwkv_wkv4_backward_noalloc(w, u, k, v, gy, ckpt, *, stream=None, out=None):
+    """WKV-4 backward through the entry point that allocates no device memory
+    and takes no workspace (its scratch is a fixed array inside the library,
+    shared by all calls; see include/rwkv_wkv.h).  ``ckpt`` is required.
+    Output tensors are still the caller's: pass ``out=(gk, gv, gw, gu)`` to
+    keep this call free of allocations from Python too."""
+    import torch
+
+    _need_cuda(w, u, k, v, gy, ckpt)
+    B, T, C = k.shape
+    if out is None:
+        gk, gv = torch.empty_like(k), torch.empty_like(v)
+        gw = torch.empty(C, dtype=torch.float32, device=k.device)
+        gu = torch.empty(C, dtype=torch.float32, device=k.device)
+    else:
+        gk, gv, gw, gu = out
+    _check("rwkv_wkv4_backward_noalloc",
+           lib().rwkv_wkv4_backward_noalloc(B, T, C, _dtype_code(k), _ptr(w), _ptr(u), _ptr(k), _ptr(v), _ptr(gy),
+                                            _ptr(ckpt), CHUNK_LEN, _ptr(gk), _ptr(gv), _ptr(gw), _ptr(gu),
+                                            _stream(stream)))
     return gk, gv, gw, gu
 
 

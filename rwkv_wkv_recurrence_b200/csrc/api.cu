@@ -15,11 +15,6 @@ __device__ unsigned int g_device_error = 0;
 cudaError_t launch_wkv5_fwd(int B, int T, int H, const void* r, const void* k, const void* v, const float* omega,
                             const float* u, void* y, const float* s_in, float* s_out, cudaStream_t st);
 
-namespace {
-
-constexpr int kDesignSMs = 148;  // B200 SM count the schedules are planned for
-constexpr int kCkLen = 16;       // checkpoint interval the backward reads
-
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                    CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
@@ -58,6 +53,11 @@ unsigned int* device_error_word() {
   if (cudaGetSymbolAddress(reinterpret_cast<void**>(&p), g_device_error) != cudaSuccess) return nullptr;
   return p;
 }
+
+namespace {
+
+constexpr int kDesignSMs = 148;  // B200 SM count the schedules are planned for
+constexpr int kCkLen = 16;       // checkpoint interval the backward reads
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 

@@ -55,6 +55,11 @@ cudaError_t launch_wkv4_step(bool bf16, int B, int C, const float* w, const floa
                              void* y, const float* state_in, float* state_out, bool vec4, cudaStream_t st);
 cudaError_t launch_copy_state(int B, int C, const float* state_in, float* state_out, cudaStream_t st);
 
+// Tensor map over a dense [B, T, C] tensor with boxes of [1, box_t, 32].
+bool make_btc_map(CUtensorMap* m, const void* base, bool bf16, int B, int T, int C, int box_t);
+// Device address of the library's error word on the current device (null on failure).
+unsigned int* device_error_word();
+
 // Sets the dynamic shared-memory limit of `func` once per device.
 cudaError_t ensure_smem_attr(const void* func, int bytes, unsigned* device_mask);
 
