@@ -45,59 +45,83 @@ def _peaks():
 
 
 class ClockSampler:
-    """Samples nvidia-smi SM clocks and throttle reasons while running."""
+    """Polls nvidia-smi (one query at a time, so nothing is lost to output
+    buffering) for SM clocks and throttle reasons while the benchmark runs."""
 
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
 
-    def __init__(self, index: int):
+    def __init__(self, index: int, period: float = 0.05):
         self.index = index
-        self.proc = None
-        self.lines = []
+        self.period = period
+        self.samples = []  # (time, sm_mhz, max_mhz, [reasons])
+        self._stop = threading.Event()
+        self.window = None
+
+    def _poll(self):
+        while not self._stop.is_set():
+            try:
+                out = subprocess.run(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                                      "--format=csv,noheader,nounits"], capture_output=True, text=True,
+                                     timeout=5).stdout.strip()
+                parts = [x.strip() for x in out.split(",")]
+                if len(parts) >= 8:
+                    reasons = [n for n, v in zip(self.NAMES, parts[4:8]) if v.lower().startswith("active")]
+                    self.samples.append((time.perf_counter(), float(parts[0]), float(parts[1]), reasons))
+            except Exception:
+                return
+            self._stop.wait(self.period)
 
     def __enter__(self):
-        try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.thread = threading.Thread(target=self._read, daemon=True)
-            self.thread.start()
-        except Exception:
-            self.proc = None
+        self.thread = threading.Thread(target=self._poll, daemon=True)
+        self.thread.start()
         return self
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
+    def mark(self, t0, t1):
+        self.window = (t0, t1)
 
     def __exit__(self, *a):
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except Exception:
-                self.proc.kill()
+        self._stop.set()
+        self.thread.join(timeout=10)
 
     def summary(self):
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [x.strip() for x in ln.split(",")]
-            if len(parts) < 8:
-                continue
-            try:
-                sm.append(float(parts[0]))
-                mx = float(parts[1])
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[4:8]):
-                if v.lower().startswith("active"):
-                    reasons.add(n)
-        if not sm:
+        if not self.samples:
             return None
-        sm.sort()
-        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+        chosen, where = self.samples, "benchmark run (warm-up and timed steps)"
+        if self.window is not None:
+            t0, t1 = self.window
+            inside = [x for x in self.samples if t0 <= x[0] <= t1]
+            if inside:
+                chosen, where = inside, "timed region"
+        sm = sorted(x[1] for x in chosen)
+        reasons = sorted({r for x in chosen for r in x[3]})
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": chosen[-1][2], "reasons": reasons,
+                "samples": len(chosen), "window": where}
+
+
+def _kernel_source_hash():
+    import hashlib
+
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "rwkv_wkv_recurrence_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.startswith("wkv4_bwd") or f in ("wkv_common.cuh", "launch.h"):
+            with open(os.path.join(csrc, f), "rb") as fh:
+                h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def _recorded_traffic():
+    """DRAM bytes per backward launch from the committed ncu capture, if it was
+    taken on the kernel source as it is now (else None)."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            d = json.load(f)["wkv4_bwd_kernel"]
+        return d["dram_bytes_per_launch"] if d.get("source_hash") == _kernel_source_hash() else None
+    except Exception:
+        return None
 
 
 def _dist():
@@ -250,6 +274,7 @@ def run_ours(args):
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clk:
         barrier()
+        wall0 = time.perf_counter()
         start.record(stream)
         for i in range(args.steps):
             evs[i][0].record(stream)
@@ -259,6 +284,7 @@ def run_ours(args):
             evs[i][2].record(stream)
         end.record(stream)
         barrier()
+        clk.mark(wall0, time.perf_counter())
     rw.rwkv_check_device_error()
     total_ms = start.elapsed_time(end)
     fwd_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
@@ -312,7 +338,8 @@ def run_ours(args):
             "kernels_ms": {"wkv4_forward": fwd_ms, "wkv4_backward": bwd_ms},
             "roofline": {"bound": "hbm", "kernel": "wkv4_bwd_kernel (+ its gw/gu batch reduction)",
                          "achieved": bwd_gbs, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
-                         "frac": bwd_gbs / peak, "traffic": args.traffic},
+                         "frac": bwd_gbs / peak,
+                         "traffic": args.traffic if args.traffic is not None else _recorded_traffic()},
             "e2e": {"value": e2e_val, "unit": "elements/s",
                     "h2d_bytes_per_step": 3 * 4 * ELEM + 2 * 4 * C, "d2h_bytes_per_step": 2 * 4 * ELEM + 2 * 4 * C},
             "gpu_launches": launches_per_step * args.steps,
@@ -326,12 +353,129 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
+def _timed(fn, steps, warmup, stream, local):
+    """W untimed calls, then K calls bracketed by synchronisation, CUDA events
+    on the launching stream; returns (ms per call, clock summary)."""
+    import torch
+
+    for _ in range(warmup):
+        fn(0)
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        torch.cuda.synchronize()
+        wall0 = time.perf_counter()
+        start.record(stream)
+        for i in range(steps):
+            fn(i)
+        end.record(stream)
+        torch.cuda.synchronize()
+        clk.mark(wall0, time.perf_counter())
+    return start.elapsed_time(end) / steps, clk.summary()
+
+
+def run_decode(args):
+    """Recurrent decode: 4096 independent streams x 4096 channels, one token per
+    step for every stream (state in and out in place), inputs of 256 distinct
+    tokens pre-generated on the device and cycled."""
+    import torch
+
+    import rwkv_wkv_recurrence_b200 as rw
+    import wkv_inputs as wi
+
+    _, _, local = _dist()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    Bd, Cd, Tp, Td = 4096, 4096, 128, 256
+    seed = SEED + 1
+    w, u = wi.wkv4_params(seed, Cd, device=dev)
+    kp = wi.btc_field("k", seed, Bd, Tp + Td, Cd, t0=0, t1=Tp, device=dev)
+    vp = wi.btc_field("v", seed, Bd, Tp + Td, Cd, t0=0, t1=Tp, device=dev)
+    _, st = rw.rwkv_wkv4_forward(w, u, kp, vp, return_state=True)
+    del kp, vp
+    ks = [wi.btc_field("k", seed, Bd, Tp + Td, Cd, t0=t, t1=t + 1, device=dev)[:, 0].contiguous()
+          for t in range(Tp, Tp + Td)]
+    vs = [wi.btc_field("v", seed, Bd, Tp + Td, Cd, t0=t, t1=t + 1, device=dev)[:, 0].contiguous()
+          for t in range(Tp, Tp + Td)]
+    y = torch.empty(Bd, Cd, device=dev)
+    h = rw.lib()
+    stream = torch.cuda.current_stream()
+    sp, P = rw._stream(stream), rw._ptr
+
+    def step(i):
+        j = i % Td
+        s = h.rwkv_wkv4_step(Bd, Cd, rw.F32, P(w), P(u), P(ks[j]), P(vs[j]), P(y), P(st), P(st), sp)
+        if s:
+            raise rw.RwkvError("rwkv_wkv4_step", s)
+
+    ms, clk = _timed(step, args.steps, args.warmup, stream, local)
+    rw.rwkv_check_device_error()
+    lanes = Bd * Cd
+    bytes_step = 36 * lanes  # state 12 B in + 12 B out, k, v, y 4 B each
+    gbs = bytes_step / (ms * 1e-3) / 1e9
+    peak, kind = _peaks()
+    print(json.dumps({
+        "metric": "WKV-4 decode lane-steps/s and HBM GB/s (4096 streams x C4096)", "value": lanes / (ms * 1e-3),
+        "unit": "lane-steps/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": "RWKV-4 WKV decode, fp32, 4096 streams x C=4096, state in place, 256 tokens cycled",
+                   "l2": "no flush: 604 MB moved per step, above the 126 MB L2"},
+        "roofline": {"bound": "hbm", "kernel": "wkv4_step_kernel", "achieved": gbs, "peak": peak,
+                     "peak_kind": kind, "unit": "GB/s", "frac": gbs / peak, "traffic": None},
+        "gpu_launches": args.steps, "clocks": clk}), flush=True)
+
+
+def run_eagle(args):
+    """Eagle / RWKV-5 forward, B4 T4096 H40 N64 bf16, zero initial state."""
+    import torch
+
+    import rwkv_wkv_recurrence_b200 as rw
+    import wkv_inputs as wi
+
+    _, _, local = _dist()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    Be, Te, He, Ne = 4, 4096, 40, 64
+    q = wi.wkv5_problem(Be, Te, He, Ne, seed=SEED + 2, device=dev)
+    y = torch.empty_like(q["r"])
+    s_out = torch.empty(Be, He, Ne, Ne, device=dev)
+    h = rw.lib()
+    stream = torch.cuda.current_stream()
+    sp, P = rw._stream(stream), rw._ptr
+    wsb = int(h.rwkv_wkv5_forward_workspace_bytes(Be, Te, He, Ne))
+    ws = torch.empty(max(wsb, 1), dtype=torch.uint8, device=dev)
+
+    def call(i):
+        s = h.rwkv_wkv5_forward(Be, Te, He, Ne, P(q["r"]), P(q["k"]), P(q["v"]), P(q["omega"]), P(q["u"]), P(y),
+                                None, P(s_out), P(ws), wsb, sp)
+        if s:
+            raise rw.RwkvError("rwkv_wkv5_forward", s)
+
+    ms, clk = _timed(call, args.steps, args.warmup, stream, local)
+    rw.rwkv_check_device_error()
+    elems = Be * Te * He * Ne
+    nbytes = 4 * 2 * elems + Be * He * Ne * Ne * 4 + 2 * He * Ne * 4  # r, k, v, y bf16; s_out; omega, u
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    peak, kind = _peaks()
+    print(json.dumps({
+        "metric": "Eagle WKV forward elements/s and HBM GB/s (B4 T4096 H40 N64)", "value": elems / (ms * 1e-3),
+        "unit": "elements/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "dtype": "bf16 I/O, fp32 state", "data": "synthetic",
+        "config": {"workload": "Eagle / RWKV-5 WKV forward, B=4 T=4096 H=40 N=64, bf16 r,k,v,y, fp32 state",
+                   "l2": "no flush: 338 MB moved per call, above the 126 MB L2"},
+        "roofline": {"bound": "hbm", "kernel": "wkv5 forward", "achieved": gbs, "peak": peak, "peak_kind": kind,
+                     "unit": "GB/s", "frac": gbs / peak, "traffic": None},
+        "gpu_launches": args.steps, "clocks": clk}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=["train", "decode", "eagle"], default="train",
+                    help="train: the headline forward+backward step; decode, eagle: the other hot-path rows")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--ref-channels", type=int, default=256)
@@ -342,6 +486,10 @@ def main():
         args.warmup = 3
     if args.impl == "reference":
         run_reference(args)
+    elif args.workload == "decode":
+        run_decode(args)
+    elif args.workload == "eagle":
+        run_eagle(args)
     else:
         run_ours(args)
 
