@@ -12,9 +12,6 @@ namespace rwkv {
 // The library's device error word (one per device that loads the library).
 __device__ unsigned int g_device_error = 0;
 
-cudaError_t launch_wkv5_fwd(int B, int T, int H, const void* r, const void* k, const void* v, const float* omega,
-                            const float* u, void* y, const float* s_in, float* s_out, cudaStream_t st);
-
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                    CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
@@ -45,6 +42,20 @@ bool make_btc_map(CUtensorMap* m, const void* base, bool bf16, int B, int T, int
   CUresult r = enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3,
                    const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                    CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool make_bf16_box64_map(CUtensorMap* m, const void* base, int B, int T, int W) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)W, (cuuint64_t)T, (cuuint64_t)B};
+  cuuint64_t strides[2] = {(cuuint64_t)W * 2, (cuuint64_t)W * T * 2};
+  cuuint32_t box[3] = {64u, 64u, 1u};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  std::memset(m, 0, sizeof(*m));
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
@@ -306,12 +317,40 @@ rwkv_status rwkv_wkv5_forward(int64_t B, int64_t T, int64_t H, int64_t N, const 
   if (N != 64) return RWKV_ERR_UNSUPPORTED;
   if (B == 0 || H == 0) return RWKV_OK;
   if (omega == nullptr || u == nullptr) return RWKV_ERR_INVALID_ARG;
-  if (T > 0 && (r == nullptr || k == nullptr || v == nullptr || y == nullptr)) return RWKV_ERR_INVALID_ARG;
-  if (T > 0 && (!aligned16(r) || !aligned16(k) || !aligned16(v) || !aligned16(y))) return RWKV_ERR_UNSUPPORTED;
-  if ((int64_t)B * H * T * N > (int64_t)INT_MAX * 8) return RWKV_ERR_UNSUPPORTED;
-  if (launch_wkv5_fwd((int)B, (int)T, (int)H, r, k, v, omega, u, y, s_in, s_out,
-                      reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (T == 0) {  // no tokens: the state passes through
+    if (s_out != nullptr && s_out != s_in) {
+      const size_t n = (size_t)B * H * 64 * 64 * sizeof(float);
+      cudaError_t e = s_in ? cudaMemcpyAsync(s_out, s_in, n, cudaMemcpyDeviceToDevice, st)
+                           : cudaMemsetAsync(s_out, 0, n, st);
+      if (e != cudaSuccess) return RWKV_ERR_CUDA;
+    }
+    return RWKV_OK;
+  }
+  if (r == nullptr || k == nullptr || v == nullptr || y == nullptr) return RWKV_ERR_INVALID_ARG;
+  if (!aligned16(r) || !aligned16(k) || !aligned16(v) || !aligned16(y)) return RWKV_ERR_UNSUPPORTED;
+  if ((int64_t)H * 64 > INT_MAX || (int64_t)B * H > INT_MAX) return RWKV_ERR_UNSUPPORTED;
+  unsigned int* err = device_error_word();
+  if (err == nullptr) return RWKV_ERR_CUDA;
+  const int iB = (int)B, iT = (int)T, iH = (int)H;
+  CUtensorMap mr, mk, mv;
+  if (!make_bf16_box64_map(&mr, r, iB, iT, iH * 64) || !make_bf16_box64_map(&mk, k, iB, iT, iH * 64) ||
+      !make_bf16_box64_map(&mv, v, iB, iT, iH * 64))
     return RWKV_ERR_CUDA;
+  Wkv5Params p{};
+  p.B = iB;
+  p.T = iT;
+  p.H = iH;
+  p.r = static_cast<const __nv_bfloat16*>(r);
+  p.k = static_cast<const __nv_bfloat16*>(k);
+  p.v = static_cast<const __nv_bfloat16*>(v);
+  p.omega = omega;
+  p.u = u;
+  p.y = static_cast<__nv_bfloat16*>(y);
+  p.s_in = s_in;
+  p.s_out = s_out;
+  p.err = err;
+  if (launch_wkv5_fwd(mr, mk, mv, p, st) != cudaSuccess) return RWKV_ERR_CUDA;
   return RWKV_OK;
 }
 

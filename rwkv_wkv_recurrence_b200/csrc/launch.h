@@ -3,6 +3,7 @@
 #pragma once
 
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 namespace rwkv {
@@ -40,6 +41,19 @@ struct Bwd4Params {
   unsigned int* err;  // device error word
 };
 
+struct Wkv5Params {
+  int B, T, H;
+  const __nv_bfloat16* r;
+  const __nv_bfloat16* k;
+  const __nv_bfloat16* v;
+  const float* omega;   // [H,64]
+  const float* u;       // [H,64]
+  __nv_bfloat16* y;
+  const float* s_in;    // [B,H,64,64] or null
+  float* s_out;         // [B,H,64,64] or null
+  unsigned int* err;
+};
+
 int fwd_tile_steps();
 int fwd_stages(bool bf16, int seg_len);
 int bwd_tile_steps();
@@ -57,6 +71,10 @@ cudaError_t launch_copy_state(int B, int C, const float* state_in, float* state_
 
 // Tensor map over a dense [B, T, C] tensor with boxes of [1, box_t, 32].
 bool make_btc_map(CUtensorMap* m, const void* base, bool bf16, int B, int T, int C, int box_t);
+// Tensor map over a bf16 [B, T, W] tensor with [1, 64, 64] boxes and the 128-byte swizzle.
+bool make_bf16_box64_map(CUtensorMap* m, const void* base, int B, int T, int W);
+cudaError_t launch_wkv5_fwd(const CUtensorMap& mr, const CUtensorMap& mk, const CUtensorMap& mv, const Wkv5Params& p,
+                            cudaStream_t st);
 // Device address of the library's error word on the current device (null on failure).
 unsigned int* device_error_word();
 

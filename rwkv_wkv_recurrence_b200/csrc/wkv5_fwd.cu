@@ -1,95 +1,432 @@
-// Eagle / RWKV-5 multi-head matrix-state WKV forward (sm_100a), recurrent
-// form on CUDA cores.
+// Eagle / RWKV-5 multi-head matrix-state WKV forward (sm_100a): chunked form
+// on the tcgen05 tensor cores.
 //
 // "RWKV-5 Eagle과 RWKV-6 Finch", section Eagle: per head,
 //   s' = diag(w) s + kᵀ v,   wkv' = s + diag(u) kᵀ v,   w = exp(-exp(ω)),
-// and the receptance reads the state like a query: y_t = r_t (s + diag(u) k_tᵀ v_t),
+// and the receptance reads the state like a query:
+//   y_t = r_t (s_t + diag(u) k_tᵀ v_t),   s_{t+1} = diag(w) s_t + k_tᵀ v_t,
 // with s[i][j] indexed (key i, value j) as in the RWKV-7 page's update
 // kv[d,e] = k_d v_e, out_e = Σ_d r_d state[d,e].
 //
-// Shape: one CTA of N = 64 threads per (batch, head); thread j owns value
-// column j of the fp32 state (64 registers).  Tokens are staged 32 at a time
-// in shared memory (converted to fp32 once), so r and k are read as
-// broadcasts.  Columns never interact, so the only per-token dependency is the
-// thread's own column.
+// Chunked form (chunk of L = 64 tokens starting at state S, λ_d = -exp(ω_d),
+// w_d = e^{λ_d}; τ, ι are positions inside the chunk):
+//   y[τ]   = Σ_d r[τ,d] e^{λ_d τ} S[d,:]                          (inter-chunk)
+//          + Σ_{ι<τ} A[τ,ι] v[ι,:] + (Σ_d r[τ,d] u_d k[τ,d]) v[τ,:]   (intra-chunk)
+//   A[τ,ι] = Σ_d r[τ,d] e^{λ_d (τ-1-ι)} k[ι,d]
+//          = Σ_d (r[τ,d] e^{λ_d (τ-32)}) (k[ι,d] e^{λ_d (31-ι)})       (a plain product)
+//   S'     = e^{64 λ} ⊙ S + Σ_ι (k[ι,:] e^{λ (63-ι)})ᵀ v[ι,:]
+// The four products (A, the inter-chunk read of S, A·v, and the state
+// increment) are 64x64x64 tf32 matrix products on tcgen05 with fp32
+// accumulators in tensor memory; the fp32 master state lives in registers and
+// its decay is applied on CUDA cores, so the state is never rounded below
+// fp32.  Splitting e^{λ(τ-1-ι)} around the chunk middle keeps both factors
+// within e^{±32|λ|}; a head with |λ| > 2.5 in any channel (w < 0.082) would
+// leave the fp32 range there and is computed by the recurrence instead.
+//
+// CTA: one (batch, head), 128 threads.  Thread 0 issues the TMA loads of the
+// raw r, k, v tiles (one [64 tokens x 64] bf16 box each, 128-byte swizzle, no
+// multicast) and the tcgen05.mma instructions; all threads build the operand
+// tiles and read the accumulators back.
 #include "launch.h"
 #include "wkv_common.cuh"
 
 namespace rwkv {
 namespace {
 
-constexpr int kN = 64;
-constexpr int kTok = 32;
+constexpr int kN = 64;                 // head size
+constexpr int kL = 64;                 // tokens per chunk
+constexpr int kThreads = 128;
+constexpr int kStages = 2;             // raw-tile pipeline depth
+constexpr uint32_t kRawBytes = kL * kN * 2;    // one bf16 [64 x 64] box
+constexpr float kMaxRate = 2.5f;       // largest -λ the chunked factorization accepts
+constexpr uint32_t kTmemCols = 256;
 
-__global__ void __launch_bounds__(kN) wkv5_fwd_recurrent_kernel(int B, int T, int H,
-                                                                const __nv_bfloat16* __restrict__ r,
-                                                                const __nv_bfloat16* __restrict__ k,
-                                                                const __nv_bfloat16* __restrict__ v,
-                                                                const float* __restrict__ omega,
-                                                                const float* __restrict__ u,
-                                                                __nv_bfloat16* __restrict__ y,
-                                                                const float* s_in, float* s_out) {
-  __shared__ float rs[kTok][kN];
-  __shared__ float ks[kTok][kN];
-  __shared__ float vs[kTok][kN];
-  __shared__ float bonus[kTok];
-  __shared__ float wd[kN];
-  __shared__ float ud[kN];
+// --------------------------------------------------------------- tcgen05 PTX
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst)),
+               "r"(ncols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
 
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// D[tmem] (+)= A[smem] * B[smem]ᵀ, both K-major, kind::tf32.
+__device__ __forceinline__ void umma_tf32(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0), "r"(0), "r"(0), "r"(0)
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+// 32 lanes x 32 bits x 64 columns: thread i of the warp gets TMEM lane (32*warp + i), columns col..col+63.
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
+  uint32_t r[64];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x64.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,"
+      "%28,%29,%30,%31,%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,"
+      "%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%64];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]),
+        "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]),
+        "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]),
+        "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]),
+        "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+      : "r"(taddr)
+      : "memory");
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Shared-memory matrix descriptor, K-major without swizzle: core matrices of
+// 8 rows x 16 bytes, K-adjacent core matrices lbo bytes apart, 8-row groups
+// sbo bytes apart.
+__device__ __forceinline__ uint64_t smem_desc(const void* p, uint32_t lbo, uint32_t sbo) {
+  const uint64_t addr = smem_u32(p);
+  return ((addr >> 4) & 0x3FFFull) | ((uint64_t)((lbo >> 4) & 0x3FFF) << 16) |
+         ((uint64_t)((sbo >> 4) & 0x3FFF) << 32) | (1ull << 46);
+}
+
+// Instruction descriptor: kind::tf32, fp32 accumulator, A and B K-major, M = 64, N = 64.
+constexpr uint32_t kIdesc = (1u << 4) | (2u << 7) | (2u << 10) | ((64u >> 3) << 17) | ((64u >> 4) << 24);
+
+// Float offset of element (row, k) of a [64 x 64] tf32 operand in the
+// K-major core-matrix layout: core matrix (row/8, k/4) is 32 floats, rows of
+// a core matrix 4 floats apart; 16 core matrices per 8-row group.
+__device__ __forceinline__ int op_off(int row, int k) {
+  return (((row >> 3) * 16 + (k >> 2)) << 5) + ((row & 7) << 2) + (k & 3);
+}
+constexpr uint32_t kLbo = 128;       // next 4 k (16 bytes of tf32) in the same rows
+constexpr uint32_t kSbo = 16 * 128;  // next 8 rows
+
+// Element (row, col) of a raw bf16 [64 x 64] box written by TMA with the
+// 128-byte swizzle (16-byte chunk c of row r stored at chunk c ^ (r & 7)).
+__device__ __forceinline__ float raw_at(const __nv_bfloat16* tile, int row, int col) {
+  const int chunk = (col >> 3) ^ (row & 7);
+  return __bfloat162float(tile[row * 64 + chunk * 8 + (col & 7)]);
+}
+
+// The recurrence for one head (used when a channel decays too fast for the
+// chunked factorization): thread j < 64 owns value column j of the state.
+__device__ void head_recurrent(int b, int h, int T, int H, const __nv_bfloat16* __restrict__ r,
+                               const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
+                               const float* wdec, const float* ud, __nv_bfloat16* __restrict__ y,
+                               const float* s_in, float* s_out, float* sm_r, float* sm_k) {
   const int j = threadIdx.x;
-  const int bh = blockIdx.x;
-  const int b = bh / H, h = bh % H;
-  wd[j] = expf(-expf(omega[h * kN + j]));
-  ud[j] = u[h * kN + j];
-
+  const size_t sbase = ((size_t)b * H + h) * kN * kN;
   float s[kN];
-  const size_t sbase = (size_t)bh * kN * kN;
+  if (j < kN) {
 #pragma unroll
-  for (int i = 0; i < kN; ++i) s[i] = s_in ? s_in[sbase + (size_t)i * kN + j] : 0.f;
-
-  for (int t0 = 0; t0 < T; t0 += kTok) {
-    const int cnt = min(kTok, T - t0);
+    for (int i = 0; i < kN; ++i) s[i] = s_in ? s_in[sbase + (size_t)i * kN + j] : 0.f;
+  }
+  for (int t = 0; t < T; ++t) {
+    const size_t off = (((size_t)b * T + t) * H + h) * kN;
     __syncthreads();
-    for (int tt = 0; tt < cnt; ++tt) {
-      const size_t off = (((size_t)b * T + t0 + tt) * H + h) * kN + j;
-      rs[tt][j] = __bfloat162float(r[off]);
-      ks[tt][j] = __bfloat162float(k[off]);
-      vs[tt][j] = __bfloat162float(v[off]);
+    if (j < kN) {
+      sm_r[j] = __bfloat162float(r[off + j]);
+      sm_k[j] = __bfloat162float(k[off + j]);
     }
     __syncthreads();
-    if (j < cnt) {
-      float acc = 0.f;
-      for (int i = 0; i < kN; ++i) acc = fmaf(rs[j][i] * ud[i], ks[j][i], acc);
-      bonus[j] = acc;
-    }
-    __syncthreads();
-    for (int tt = 0; tt < cnt; ++tt) {
-      const float vj = vs[tt][j];
-      float acc = bonus[tt] * vj;
+    if (j < kN) {
+      const float vj = __bfloat162float(v[off + j]);
+      float bonus = 0.f, acc = 0.f;
 #pragma unroll
-      for (int i = 0; i < kN; ++i) acc = fmaf(rs[tt][i], s[i], acc);
+      for (int i = 0; i < kN; ++i) {
+        bonus = fmaf(sm_r[i] * ud[i], sm_k[i], bonus);
+        acc = fmaf(sm_r[i], s[i], acc);
+      }
+      acc = fmaf(bonus, vj, acc);
 #pragma unroll
-      for (int i = 0; i < kN; ++i) s[i] = fmaf(wd[i], s[i], ks[tt][i] * vj);
-      y[(((size_t)b * T + t0 + tt) * H + h) * kN + j] = __float2bfloat16_rn(acc);
+      for (int i = 0; i < kN; ++i) s[i] = fmaf(wdec[i], s[i], sm_k[i] * vj);
+      y[off + j] = __float2bfloat16_rn(acc);
     }
   }
-  if (s_out != nullptr) {
-    __syncthreads();  // s_out may alias s_in: every thread has read its column above
+  if (s_out != nullptr && j < kN) {
 #pragma unroll
     for (int i = 0; i < kN; ++i) s_out[sbase + (size_t)i * kN + j] = s[i];
   }
 }
 
+struct Wkv5Smem {
+  alignas(1024) __nv_bfloat16 raw[kStages][3][kL * kN];  // r, k, v boxes (128-byte swizzle)
+  alignas(128) float opR[64 * 64];    // r e^{λ(τ-32)}      [τ][d]  (A of the score product)
+  alignas(128) float opK[64 * 64];    // k e^{λ(31-ι)}      [ι][d]  (B of the score product)
+  alignas(128) float opRh[64 * 64];   // r e^{λ τ}          [τ][d]  (A of the state read)
+  alignas(128) float opS[64 * 64];    // state, transposed  [j][d]  (B of the state read)
+  alignas(128) float opKh[64 * 64];   // k e^{λ(63-ι)}, transposed [d][ι]  (A of the state increment)
+  alignas(128) float opVt[64 * 64];   // v transposed       [j][ι]  (B of the increment and of A v)
+  alignas(128) float opA[64 * 64];    // masked scores      [τ][ι]  (A of A v)
+  alignas(16) float dec[96 * 64];     // e^{λ_d (m - 32)}, m in [0, 96)
+  float diag[kL];                     // Σ_d r u k per token (bonus)
+  float ud[kN];
+  float wdec[kN];
+  float decL[kN];                     // e^{64 λ_d}
+  alignas(8) uint64_t bar_tma[kStages];
+  alignas(8) uint64_t bar_mma;
+  uint32_t tmem_base;
+  int slow;
+  int abort_flag;
+};
+
+__global__ void __launch_bounds__(kThreads, 1) wkv5_fwd_tc_kernel(const __grid_constant__ CUtensorMap mr,
+                                                                  const __grid_constant__ CUtensorMap mk,
+                                                                  const __grid_constant__ CUtensorMap mv,
+                                                                  Wkv5Params p) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  // TMA destinations with the 128-byte swizzle need 1024-byte alignment: align by hand
+  const uint32_t base_s = smem_u32(smem_raw);
+  Wkv5Smem& sm = *reinterpret_cast<Wkv5Smem*>(smem_raw + ((1024u - (base_s & 1023u)) & 1023u));
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int b = blockIdx.x / p.H, h = blockIdx.x % p.H;
+  const int nchunk = (p.T + kL - 1) / kL;
+
+  // per-channel constants and the decay table
+  if (tid < kN) {
+    const float om = p.omega[h * kN + tid];
+    const float rate = expf(om);  // -λ
+    sm.ud[tid] = p.u[h * kN + tid];
+    sm.wdec[tid] = expf(-rate);
+    sm.decL[tid] = expf(-64.f * rate);
+  }
+  if (tid == 0) {
+    sm.slow = 0;
+    sm.abort_flag = 0;
+  }
+  __syncthreads();
+  if (tid < kN && !(expf(p.omega[h * kN + tid]) <= kMaxRate)) atomicOr(&sm.slow, 1);
+  for (int i = tid; i < 96 * 64; i += kThreads) {
+    const int m = i >> 6, d = i & 63;
+    sm.dec[i] = expf(-expf(p.omega[h * kN + d]) * (float)(m - 32));
+  }
+  __syncthreads();
+  if (sm.slow) {
+    head_recurrent(b, h, p.T, p.H, p.r, p.k, p.v, sm.wdec, sm.ud, p.y, p.s_in, p.s_out, sm.opR, sm.opK);
+    return;
+  }
+
+  if (warp == 0) tmem_alloc(&sm.tmem_base, kTmemCols);
+  if (tid == 0) {
+    prefetch_tensormap(&mr);
+    prefetch_tensormap(&mk);
+    prefetch_tensormap(&mv);
+    for (int s = 0; s < kStages; ++s) mbar_init(&sm.bar_tma[s], 1);
+    mbar_init(&sm.bar_mma, 1);
+    fence_mbar_init();
+    for (int s = 0; s < kStages && s < nchunk; ++s) {
+      mbar_arrive_expect_tx(&sm.bar_tma[s], 3 * kRawBytes);
+      tma_load_3d(sm.raw[s][0], &mr, &sm.bar_tma[s], h * kN, s * kL, b);
+      tma_load_3d(sm.raw[s][1], &mk, &sm.bar_tma[s], h * kN, s * kL, b);
+      tma_load_3d(sm.raw[s][2], &mv, &sm.bar_tma[s], h * kN, s * kL, b);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = sm.tmem_base;
+  const uint32_t tA = tbase, tY = tbase + 64, tD = tbase + 128;
+  const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
+
+  // fp32 master state: rows d = 16*warp + lane held by lanes 0..15 (the M = 64
+  // accumulator layout puts row m in TMEM lane (m % 16) + 32 (m / 16)).
+  const bool holds_row = lane < 16;
+  const int srow = 16 * warp + lane;
+  const size_t sbase = ((size_t)b * p.H + h) * kN * kN;
+  float S[64];
+#pragma unroll
+  for (int j = 0; j < 64; ++j) S[j] = (holds_row && p.s_in) ? p.s_in[sbase + (size_t)srow * kN + j] : 0.f;
+  if (holds_row) {
+#pragma unroll
+    for (int j = 0; j < 64; ++j) sm.opS[op_off(j, srow)] = S[j];
+  }
+  const float my_decL = holds_row ? sm.decL[srow] : 0.f;
+
+  uint32_t mma_phase = 0;
+  for (int c = 0; c < nchunk; ++c) {
+    const int st = c % kStages;
+    const int t0 = c * kL;
+    const int cnt = min(kL, p.T - t0);
+    if (!mbar_wait_bounded(&sm.bar_tma[st], (uint32_t)(c / kStages) & 1u, p.err)) sm.abort_flag = 1;
+    const __nv_bfloat16* Rr = sm.raw[st][0];
+    const __nv_bfloat16* Kr = sm.raw[st][1];
+    const __nv_bfloat16* Vr = sm.raw[st][2];
+
+    // T1: operands.  Each warp-quarter writes one core matrix (8 rows x 4 k).
+    // (the state increment of a partial last chunk uses e^{λ(cnt-1-ι)}: m = 31 + cnt - ι)
+    for (int q = tid; q < 256; q += kThreads) {
+      const int row = ((q >> 5) << 3) + (q & 7);  // 8-row group (q / 32), row inside it (q % 8)
+      const int kg = (q >> 3) & 3;
+      for (int kq = kg; kq < 16; kq += 4) {
+        const int k0 = kq * 4;
+        float4 vr, vk, vrh, vkh, vvt;
+        float* pr = &vr.x;
+        float* pk = &vk.x;
+        float* prh = &vrh.x;
+        float* pkh = &vkh.x;
+        float* pvt = &vvt.x;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int col = k0 + e;
+          const float rv = raw_at(Rr, row, col), kv = raw_at(Kr, row, col);
+          pr[e] = rv * sm.dec[row * 64 + col];             // e^{λ(τ-32)}, m = τ
+          prh[e] = rv * sm.dec[(row + 32) * 64 + col];     // e^{λ τ}
+          pk[e] = kv * sm.dec[(63 - row) * 64 + col];      // e^{λ(31-ι)}, m = 63 - ι
+          // transposed operands: element (row = d or j, k = ι = col)
+          pkh[e] = raw_at(Kr, col, row) * sm.dec[max(0, 31 + cnt - col) * 64 + row];  // k[ι][d] e^{λ_d (cnt-1-ι)}
+          pvt[e] = raw_at(Vr, col, row);                                   // v[ι][j]
+        }
+        const int o = op_off(row, k0);
+        *reinterpret_cast<float4*>(&sm.opR[o]) = vr;
+        *reinterpret_cast<float4*>(&sm.opRh[o]) = vrh;
+        *reinterpret_cast<float4*>(&sm.opK[o]) = vk;
+        *reinterpret_cast<float4*>(&sm.opKh[o]) = vkh;
+        *reinterpret_cast<float4*>(&sm.opVt[o]) = vvt;
+      }
+    }
+    // bonus Σ_d r u k for each token (exact, fp32)
+    {
+      const int tok = tid >> 1, half = tid & 1;
+      float acc = 0.f;
+      for (int d = half * 32; d < half * 32 + 32; ++d)
+        acc = fmaf(raw_at(Rr, tok, d) * sm.ud[d], raw_at(Kr, tok, d), acc);
+      acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+      if (half == 0) sm.diag[tok] = acc;
+    }
+    // rows past the end of the sequence hold zero keys and values (TMA zero fill)
+    fence_proxy_async();
+    tc_fence_before();
+    __syncthreads();
+    if (sm.abort_flag) break;
+    if (tid == 0) {
+      tc_fence_after();
+      // M1: scores A = r~ k~ᵀ; y = r^ S; ΔS = k^ᵀ v  (8 k-steps of 8 each)
+#pragma unroll
+      for (int s = 0; s < 8; ++s)
+        umma_tf32(tA, smem_desc(&sm.opR[s * 64], kLbo, kSbo), smem_desc(&sm.opK[s * 64], kLbo, kSbo), kIdesc, s);
+#pragma unroll
+      for (int s = 0; s < 8; ++s)
+        umma_tf32(tY, smem_desc(&sm.opRh[s * 64], kLbo, kSbo), smem_desc(&sm.opS[s * 64], kLbo, kSbo), kIdesc, s);
+#pragma unroll
+      for (int s = 0; s < 8; ++s)
+        umma_tf32(tD, smem_desc(&sm.opKh[s * 64], kLbo, kSbo), smem_desc(&sm.opVt[s * 64], kLbo, kSbo), kIdesc, s);
+      umma_commit(&sm.bar_mma);
+      // this chunk's raw tiles are consumed: refill the stage
+      if (c + kStages < nchunk) {
+        fence_proxy_async();
+        mbar_arrive_expect_tx(&sm.bar_tma[st], 3 * kRawBytes);
+        tma_load_3d(sm.raw[st][0], &mr, &sm.bar_tma[st], h * kN, (c + kStages) * kL, b);
+        tma_load_3d(sm.raw[st][1], &mk, &sm.bar_tma[st], h * kN, (c + kStages) * kL, b);
+        tma_load_3d(sm.raw[st][2], &mv, &sm.bar_tma[st], h * kN, (c + kStages) * kL, b);
+      }
+    }
+    if (!mbar_wait_bounded(&sm.bar_mma, mma_phase, p.err)) sm.abort_flag = 1;
+    mma_phase ^= 1u;
+    tc_fence_after();
+
+    // T2: masked scores -> opA; state update S' = e^{64λ} S + ΔS -> opS
+    {
+      float a[64];
+      tmem_ld64(tA + lane_base, a);
+      if (holds_row) {
+        const int tau = srow;
+#pragma unroll
+        for (int kq = 0; kq < 16; ++kq) {
+          float4 o;
+          float* po = &o.x;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int io = kq * 4 + e;
+            po[e] = io < tau ? a[io] : (io == tau ? sm.diag[tau] : 0.f);
+          }
+          *reinterpret_cast<float4*>(&sm.opA[op_off(tau, kq * 4)]) = o;
+        }
+      }
+      float ds[64];
+      tmem_ld64(tD + lane_base, ds);
+      if (holds_row) {
+        const float dl = cnt == kL ? my_decL : expf(-expf(p.omega[h * kN + srow]) * (float)cnt);
+#pragma unroll
+        for (int j = 0; j < 64; ++j) {
+          S[j] = fmaf(dl, S[j], ds[j]);
+          sm.opS[op_off(j, srow)] = S[j];
+        }
+      }
+    }
+    fence_proxy_async();
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0) {
+      tc_fence_after();
+      // M2: y += A v
+#pragma unroll
+      for (int s = 0; s < 8; ++s)
+        umma_tf32(tY, smem_desc(&sm.opA[s * 64], kLbo, kSbo), smem_desc(&sm.opVt[s * 64], kLbo, kSbo), kIdesc, 1);
+      umma_commit(&sm.bar_mma);
+    }
+    if (!mbar_wait_bounded(&sm.bar_mma, mma_phase, p.err)) sm.abort_flag = 1;
+    mma_phase ^= 1u;
+    tc_fence_after();
+
+    // T3: y rows -> bf16 -> global
+    {
+      float yv[64];
+      tmem_ld64(tY + lane_base, yv);
+      if (holds_row && srow < cnt) {
+        __nv_bfloat16* yp = p.y + (((size_t)b * p.T + t0 + srow) * p.H + h) * kN;
+#pragma unroll
+        for (int j = 0; j < 64; j += 8) {
+          uint4 pk;
+          __nv_bfloat162* q2 = reinterpret_cast<__nv_bfloat162*>(&pk);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) q2[e] = __floats2bfloat162_rn(yv[j + 2 * e], yv[j + 2 * e + 1]);
+          *reinterpret_cast<uint4*>(yp + j) = pk;
+        }
+      }
+    }
+    tc_fence_before();
+    __syncthreads();
+  }
+
+  if (p.s_out != nullptr && holds_row) {
+#pragma unroll
+    for (int j = 0; j < 64; ++j) p.s_out[sbase + (size_t)srow * kN + j] = S[j];
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tbase, kTmemCols);
+  }
+}
+
 }  // namespace
 
-cudaError_t launch_wkv5_fwd(int B, int T, int H, const void* r, const void* k, const void* v, const float* omega,
-                            const float* u, void* y, const float* s_in, float* s_out, cudaStream_t st) {
-  const unsigned grid = (unsigned)(B * H);
-  wkv5_fwd_recurrent_kernel<<<grid, kN, 0, st>>>(B, T, H, static_cast<const __nv_bfloat16*>(r),
-                                                  static_cast<const __nv_bfloat16*>(k),
-                                                  static_cast<const __nv_bfloat16*>(v), omega, u,
-                                                  static_cast<__nv_bfloat16*>(y), s_in, s_out);
+cudaError_t launch_wkv5_fwd(const CUtensorMap& mr, const CUtensorMap& mk, const CUtensorMap& mv, const Wkv5Params& p,
+                            cudaStream_t st) {
+  const size_t smem = sizeof(Wkv5Smem) + 1024;  // + alignment slack
+  static unsigned device_mask = 0;
+  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(wkv5_fwd_tc_kernel), (int)smem, &device_mask);
+  if (e != cudaSuccess) return e;
+  wkv5_fwd_tc_kernel<<<(unsigned)(p.B * p.H), kThreads, smem, st>>>(mr, mk, mv, p);
   return cudaGetLastError();
 }
+
+size_t wkv5_smem_bytes() { return sizeof(Wkv5Smem) + 1024; }
 
 }  // namespace rwkv

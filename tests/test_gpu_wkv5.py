@@ -19,10 +19,21 @@ def _cuda(p, dev):
     return {k: v.to(dev) for k, v in p.items()}
 
 
-@pytest.mark.parametrize("shape", [(1, 100, 2), (2, 33, 3), (1, 1, 1), (1, 64, 1)])
+@pytest.mark.parametrize("shape", [(1, 64, 1), (1, 100, 2), (2, 33, 3), (1, 1, 1), (2, 200, 3)])
 def test_forward_small(cuda_device, shape):
     B, T, H = shape
     p = wi.wkv5_problem(B, T, H, 64, seed=30)
+    y, s = rw.rwkv_wkv5_forward(**_cuda(p, cuda_device), return_state=True)
+    ref, ref_s = oracle.wkv5_forward(p["r"], p["k"], p["v"], p["omega"], p["u"], return_state=True)
+    assert_close_rms(y, ref, TOL_BF16, "y")
+    assert_close_rms(s, ref_s, TOL_BF16, "s_out")
+
+
+@pytest.mark.parametrize("omega_range", [(-1.0, 2.0), (-8.0, -4.0), (0.5, 0.9)])
+def test_forward_decay_ranges(cuda_device, omega_range):
+    # fast decays (exp(omega) > 2.5, w < 0.082) take the recurrent path inside
+    # the kernel; slow and moderate decays the chunked tensor-core path
+    p = wi.wkv5_problem(2, 150, 3, 64, seed=32, omega_range=omega_range)
     y, s = rw.rwkv_wkv5_forward(**_cuda(p, cuda_device), return_state=True)
     ref, ref_s = oracle.wkv5_forward(p["r"], p["k"], p["v"], p["omega"], p["u"], return_state=True)
     assert_close_rms(y, ref, TOL_BF16, "y")
