@@ -101,25 +101,30 @@ class ClockSampler:
                 "samples": len(chosen), "window": where}
 
 
-def _kernel_source_hash():
+# kernel name in profiles/traffic.json -> prefix of the source files it is built from
+_TRAFFIC_SOURCES = {"wkv4_bwd_kernel": "wkv4_bwd", "wkv5_fwd_tc_kernel": "wkv5_fwd"}
+
+
+def _kernel_source_hash(kernel="wkv4_bwd_kernel"):
     import hashlib
 
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "rwkv_wkv_recurrence_b200", "csrc")
+    prefix = _TRAFFIC_SOURCES[kernel]
     for f in sorted(os.listdir(csrc)):
-        if f.startswith("wkv4_bwd") or f in ("wkv_common.cuh", "launch.h"):
+        if f.startswith(prefix) or f in ("wkv_common.cuh", "launch.h"):
             with open(os.path.join(csrc, f), "rb") as fh:
                 h.update(fh.read())
     return h.hexdigest()[:16]
 
 
-def _recorded_traffic():
-    """DRAM bytes per backward launch from the committed ncu capture, if it was
+def _recorded_traffic(kernel="wkv4_bwd_kernel"):
+    """DRAM bytes per launch of `kernel` from the committed ncu capture, if it was
     taken on the kernel source as it is now (else None)."""
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
-            d = json.load(f)["wkv4_bwd_kernel"]
-        return d["dram_bytes_per_launch"] if d.get("source_hash") == _kernel_source_hash() else None
+            d = json.load(f)[kernel]
+        return d["dram_bytes_per_launch"] if d.get("source_hash") == _kernel_source_hash(kernel) else None
     except Exception:
         return None
 
@@ -464,7 +469,7 @@ def run_eagle(args):
         "config": {"workload": "Eagle / RWKV-5 WKV forward, B=4 T=4096 H=40 N=64, bf16 r,k,v,y, fp32 state",
                    "l2": "no flush: 338 MB moved per call, above the 126 MB L2"},
         "roofline": {"bound": "hbm", "kernel": "wkv5 forward", "achieved": gbs, "peak": peak, "peak_kind": kind,
-                     "unit": "GB/s", "frac": gbs / peak, "traffic": None},
+                     "unit": "GB/s", "frac": gbs / peak, "traffic": _recorded_traffic("wkv5_fwd_tc_kernel")},
         "gpu_launches": args.steps, "clocks": clk}), flush=True)
 
 

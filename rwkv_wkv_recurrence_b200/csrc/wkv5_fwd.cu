@@ -15,18 +15,36 @@
 //   A[τ,ι] = Σ_d r[τ,d] e^{λ_d (τ-1-ι)} k[ι,d]
 //          = Σ_d (r[τ,d] e^{λ_d (τ-32)}) (k[ι,d] e^{λ_d (31-ι)})       (a plain product)
 //   S'     = e^{64 λ} ⊙ S + Σ_ι (k[ι,:] e^{λ (63-ι)})ᵀ v[ι,:]
-// The four products (A, the inter-chunk read of S, A·v, and the state
-// increment) are 64x64x64 tf32 matrix products on tcgen05 with fp32
-// accumulators in tensor memory; the fp32 master state lives in registers and
-// its decay is applied on CUDA cores, so the state is never rounded below
-// fp32.  Splitting e^{λ(τ-1-ι)} around the chunk middle keeps both factors
-// within e^{±32|λ|}; a head with |λ| > 2.5 in any channel (w < 0.082) would
-// leave the fp32 range there and is computed by the recurrence instead.
+// Per chunk the tensor cores (tcgen05, kind::tf32, fp32 accumulators in tensor
+// memory) run three chains of eight K = 8 steps:
+//   [A | Y] = r̃ [k̃ ; e^{32λ} Sᵀ]ᵀ          M = 64, N = 128: scores [τ][ι] and the
+//                                           inter-chunk read [τ][j] share operand r̃
+//   Y      += A_masked vᵀᵀ                 M = 64, N = 64 (intra-chunk term)
+//   ΔS      = k̃ᵀ vᵀᵀ                       M = 64, N = 64, k̃ᵀ read from tensor memory
+// with r̃ = r e^{λ(τ-32)}, k̃ = k e^{λ(31-ι)}, so that r̃·k̃ = r e^{λ(τ-1-ι)} k and
+// e^{32λ} (r̃ S) = r e^{λτ} S; the state increment is scaled by e^{λ(cnt-32)} per
+// key channel when it is folded into the fp32 master state, which lives in
+// registers (S' = e^{cnt λ} S + e^{(cnt-32) λ} ΔS), so the state is never
+// rounded below fp32.  Splitting e^{λ(τ-1-ι)} around the chunk middle keeps
+// every factor within e^{±32|λ|}; a head with -λ > 2.5 in any channel
+// (w < 0.082) would leave the fp32 range there and is computed by the
+// recurrence instead.
 //
-// CTA: one (batch, head), 128 threads.  Thread 0 issues the TMA loads of the
-// raw r, k, v tiles (one [64 tokens x 64] bf16 box each, 128-byte swizzle, no
-// multicast) and the tcgen05.mma instructions; all threads build the operand
-// tiles and read the accumulators back.
+// The tensor core takes tf32 operands K-major only, so the operand tiles are
+// fp32 [rows][64] in the K-major core-matrix layout without swizzle (8 rows x
+// 16 bytes per core matrix); k̃ᵀ and vᵀ are transposed on the way in with
+// ldmatrix.trans.  Each tcgen05.mma of these sizes costs its issuing thread
+// about 70 cycles whatever M and N are, so the kernel uses the widest shapes
+// the data allows (N = 128 for the first chain) and the issuing thread hands
+// the first chain out in pairs between the other work of its warp.
+//
+// CTA: one (batch, head), 8 warps, about 106 KB of shared memory and 256 TMEM
+// columns, two CTAs per SM.  Thread 0 issues the TMA loads of the raw r, k, v
+// tiles (one [64 tokens x 64] bf16 box each, 128-byte swizzle, no multicast)
+// and the MMAs; all warps build operands, mask the scores, fold the state and
+// write the output rows.
+#include <cstddef>
+
 #include "launch.h"
 #include "wkv_common.cuh"
 
@@ -35,11 +53,10 @@ namespace {
 
 constexpr int kN = 64;                 // head size
 constexpr int kL = 64;                 // tokens per chunk
-constexpr int kThreads = 128;
-constexpr int kStages = 2;             // raw-tile pipeline depth
+constexpr int kThreads = 256;
 constexpr uint32_t kRawBytes = kL * kN * 2;    // one bf16 [64 x 64] box
 constexpr float kMaxRate = 2.5f;       // largest -λ the chunked factorization accepts
-constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kTmemCols = 256;  // [scores | output rows], state increment, k̃ᵀ (64 columns each)
 
 // --------------------------------------------------------------- tcgen05 PTX
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst, uint32_t ncols) {
@@ -72,27 +89,80 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
                : "memory");
 }
 
-// 32 lanes x 32 bits x 64 columns: thread i of the warp gets TMEM lane (32*warp + i), columns col..col+63.
-__device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
-  uint32_t r[64];
+// 16 lanes x 256 bits, 4 repetitions (32 columns).  Register 4 i + 2 r + e of
+// thread t goes to lane (base + t/4 + 8 r), column (base + 8 i + 2 (t%4) + e).
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
   asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x64.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,"
-      "%28,%29,%30,%31,%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,"
-      "%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%64];"
+      "tcgen05.st.sync.aligned.16x256b.x4.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+          taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// 16 lanes x 128 bits, 8 repetitions (32 columns).  Register 2 q + r of
+// thread t holds lane (base + t/4 + 8 r), column (base + 4 q + t%4).
+__device__ __forceinline__ void tmem_ld16x128(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x128b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
       : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]),
-        "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]),
-        "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]),
-        "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]),
-        "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
       : "r"(taddr)
       : "memory");
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
-  for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(r[i]);
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// 32 lanes x 32 bits x 32 columns: thread t gets lane (base + t), 32 consecutive columns.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,"
+      "%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+
+// D[tmem] (+)= A[tmem] * B[smem]ᵀ, kind::tf32 (A rows in the accumulator layout).
+__device__ __forceinline__ void umma_tf32_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, {%5, %6, %7, %8}, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0), "r"(0), "r"(0), "r"(0)
+      : "memory");
+}
+
+// Four 8x8 bf16 matrices from shared memory, transposed (row addresses from lanes
+// 8m..8m+7): register m of thread t holds rows 2 (t%4), +1 of column t/4 of matrix m.
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&q)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(q[0]), "=r"(q[1]), "=r"(q[2]), "=r"(q[3])
+               : "r"(addr)
+               : "memory");
+}
+
+// Two packed bf16 (low half first) to fp32.
+__device__ __forceinline__ float2 bf2_to_f2(uint32_t x) {
+  return make_float2(__uint_as_float(x << 16), __uint_as_float(x & 0xFFFF0000u));
 }
 
 // Shared-memory matrix descriptor, K-major without swizzle: core matrices of
@@ -116,16 +186,9 @@ __device__ __forceinline__ int op_off(int row, int k) {
 constexpr uint32_t kLbo = 128;       // next 4 k (16 bytes of tf32) in the same rows
 constexpr uint32_t kSbo = 16 * 128;  // next 8 rows
 
-// Element (row, col) of a raw bf16 [64 x 64] box written by TMA with the
-// 128-byte swizzle (16-byte chunk c of row r stored at chunk c ^ (r & 7)).
-__device__ __forceinline__ float raw_at(const __nv_bfloat16* tile, int row, int col) {
-  const int chunk = (col >> 3) ^ (row & 7);
-  return __bfloat162float(tile[row * 64 + chunk * 8 + (col & 7)]);
-}
-
 // The recurrence for one head (used when a channel decays too fast for the
 // chunked factorization): thread j < 64 owns value column j of the state.
-__device__ void head_recurrent(int b, int h, int T, int H, const __nv_bfloat16* __restrict__ r,
+__device__ __noinline__ void head_recurrent(int b, int h, int T, int H, const __nv_bfloat16* __restrict__ r,
                                const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
                                const float* wdec, const float* ud, __nv_bfloat16* __restrict__ y,
                                const float* s_in, float* s_out, float* sm_r, float* sm_k) {
@@ -165,27 +228,29 @@ __device__ void head_recurrent(int b, int h, int T, int H, const __nv_bfloat16* 
 }
 
 struct Wkv5Smem {
-  alignas(1024) __nv_bfloat16 raw[kStages][3][kL * kN];  // r, k, v boxes (128-byte swizzle)
-  alignas(128) float opR[64 * 64];    // r e^{λ(τ-32)}      [τ][d]  (A of the score product)
-  alignas(128) float opK[64 * 64];    // k e^{λ(31-ι)}      [ι][d]  (B of the score product)
-  alignas(128) float opRh[64 * 64];   // r e^{λ τ}          [τ][d]  (A of the state read)
-  alignas(128) float opS[64 * 64];    // state, transposed  [j][d]  (B of the state read)
-  alignas(128) float opKh[64 * 64];   // k e^{λ(63-ι)}, transposed [d][ι]  (A of the state increment)
-  alignas(128) float opVt[64 * 64];   // v transposed       [j][ι]  (B of the increment and of A v)
-  alignas(128) float opA[64 * 64];    // masked scores      [τ][ι]  (A of A v)
-  alignas(16) float dec[96 * 64];     // e^{λ_d (m - 32)}, m in [0, 96)
-  float diag[kL];                     // Σ_d r u k per token (bonus)
-  float ud[kN];
-  float wdec[kN];
-  float decL[kN];                     // e^{64 λ_d}
-  alignas(8) uint64_t bar_tma[kStages];
-  alignas(8) uint64_t bar_mma;
+  alignas(1024) __nv_bfloat16 raw[3][kL * kN];  // r, k, v boxes [token][channel] (128-byte swizzle)
+  alignas(128) float opR[64 * 64];   // r̃ = r e^{λ(τ-32)}   [τ][d]: A of the scores and of the state read
+  alignas(128) float opK[64 * 64];   // k̃ = k e^{λ(31-ι)}   [ι][d]: B rows 0..63 of the first product
+  alignas(128) float opS[64 * 64];   // e^{32λ} ⊙ Sᵀ         [j][d]: B rows 64..127 of the first product
+  alignas(128) float opVt[64 * 64];  // vᵀ                   [j][ι]: B of A v and of the state increment
+  alignas(128) float opA[64 * 64];   // masked scores       [τ][ι]: A of A v
+  float diag_part[8][kL];            // per-warp parts of Σ_d r u k (the bonus term)
+  float diag[kL];                    // Σ_d r u k per token
+  alignas(8) uint64_t bar_tma;
+  alignas(8) uint64_t bar_sc;        // scores and state read done
+  alignas(8) uint64_t bar_av;        // A v done
+  alignas(8) uint64_t bar_ds;        // state increment done
   uint32_t tmem_base;
   int slow;
   int abort_flag;
 };
+static_assert(offsetof(Wkv5Smem, opS) == offsetof(Wkv5Smem, opK) + 64 * 64 * sizeof(float),
+              "the first product reads k̃ and e^{32λ} Sᵀ as one 128-row operand");
 
-__global__ void __launch_bounds__(kThreads, 1) wkv5_fwd_tc_kernel(const __grid_constant__ CUtensorMap mr,
+// kind::tf32, fp32 accumulator, K-major A and B, M = 64, N = 128.
+constexpr uint32_t kIdesc128 = (kIdesc & ~(0x3Fu << 17)) | ((128u >> 3) << 17);
+
+__global__ void __launch_bounds__(kThreads, 2) wkv5_fwd_tc_kernel(const __grid_constant__ CUtensorMap mr,
                                                                   const __grid_constant__ CUtensorMap mk,
                                                                   const __grid_constant__ CUtensorMap mv,
                                                                   Wkv5Params p) {
@@ -194,30 +259,26 @@ __global__ void __launch_bounds__(kThreads, 1) wkv5_fwd_tc_kernel(const __grid_c
   const uint32_t base_s = smem_u32(smem_raw);
   Wkv5Smem& sm = *reinterpret_cast<Wkv5Smem*>(smem_raw + ((1024u - (base_s & 1023u)) & 1023u));
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int t4 = lane >> 2, tq = lane & 3;
+  const int q4 = warp & 3, hc = warp >> 2;  // TMEM lane quarter and column half of this warp
   const int b = blockIdx.x / p.H, h = blockIdx.x % p.H;
   const int nchunk = (p.T + kL - 1) / kL;
+  const float* om = p.omega + h * kN;
 
-  // per-channel constants and the decay table
-  if (tid < kN) {
-    const float om = p.omega[h * kN + tid];
-    const float rate = expf(om);  // -λ
-    sm.ud[tid] = p.u[h * kN + tid];
-    sm.wdec[tid] = expf(-rate);
-    sm.decL[tid] = expf(-64.f * rate);
-  }
   if (tid == 0) {
     sm.slow = 0;
     sm.abort_flag = 0;
   }
   __syncthreads();
-  if (tid < kN && !(expf(p.omega[h * kN + tid]) <= kMaxRate)) atomicOr(&sm.slow, 1);
-  for (int i = tid; i < 96 * 64; i += kThreads) {
-    const int m = i >> 6, d = i & 63;
-    sm.dec[i] = expf(-expf(p.omega[h * kN + d]) * (float)(m - 32));
-  }
+  if (tid < kN && !(expf(om[tid]) <= kMaxRate)) atomicOr(&sm.slow, 1);
   __syncthreads();
   if (sm.slow) {
-    head_recurrent(b, h, p.T, p.H, p.r, p.k, p.v, sm.wdec, sm.ud, p.y, p.s_in, p.s_out, sm.opR, sm.opK);
+    if (tid < kN) {  // opR/opK double as scratch for the recurrence
+      sm.opS[tid] = expf(-expf(om[tid]));
+      sm.opS[64 + tid] = p.u[h * kN + tid];
+    }
+    __syncthreads();
+    head_recurrent(b, h, p.T, p.H, p.r, p.k, p.v, &sm.opS[0], &sm.opS[64], p.y, p.s_in, p.s_out, sm.opR, sm.opK);
     return;
   }
 
@@ -226,171 +287,233 @@ __global__ void __launch_bounds__(kThreads, 1) wkv5_fwd_tc_kernel(const __grid_c
     prefetch_tensormap(&mr);
     prefetch_tensormap(&mk);
     prefetch_tensormap(&mv);
-    for (int s = 0; s < kStages; ++s) mbar_init(&sm.bar_tma[s], 1);
-    mbar_init(&sm.bar_mma, 1);
+    mbar_init(&sm.bar_tma, 1);
+    mbar_init(&sm.bar_sc, 1);
+    mbar_init(&sm.bar_av, 1);
+    mbar_init(&sm.bar_ds, 1);
     fence_mbar_init();
-    for (int s = 0; s < kStages && s < nchunk; ++s) {
-      mbar_arrive_expect_tx(&sm.bar_tma[s], 3 * kRawBytes);
-      tma_load_3d(sm.raw[s][0], &mr, &sm.bar_tma[s], h * kN, s * kL, b);
-      tma_load_3d(sm.raw[s][1], &mk, &sm.bar_tma[s], h * kN, s * kL, b);
-      tma_load_3d(sm.raw[s][2], &mv, &sm.bar_tma[s], h * kN, s * kL, b);
-    }
+    mbar_arrive_expect_tx(&sm.bar_tma, 3 * kRawBytes);
+    tma_load_3d(sm.raw[0], &mr, &sm.bar_tma, h * kN, 0, b);
+    tma_load_3d(sm.raw[1], &mk, &sm.bar_tma, h * kN, 0, b);
+    tma_load_3d(sm.raw[2], &mv, &sm.bar_tma, h * kN, 0, b);
   }
+
+  // ---- r̃, k̃: warp w owns channels 8w..8w+7; lane holds token row 8 ib + rr, channels dR, dR + 1.
+  // A half-warp then writes one whole core matrix (eight 16-byte rows): no bank conflicts.
+  const int rr = lane & 7, rp = lane >> 3;
+  const int dR = 8 * warp + 2 * rp;
+  float fr0[2], frs[2], fk0[2], fks[2], uA[2];
+#pragma unroll
+  for (int e = 0; e < 2; ++e) {
+    const float rate = expf(om[dR + e]);  // -λ
+    fr0[e] = expf(-rate * (float)(rr - 32));
+    frs[e] = expf(-8.f * rate);
+    fk0[e] = expf(-rate * (float)(31 - rr));
+    fks[e] = expf(8.f * rate);
+    uA[e] = p.u[h * kN + dR + e];
+  }
+  const uint32_t offRK = (uint32_t)rr * 128u + (uint32_t)((warp ^ rr) << 4) + (uint32_t)rp * 4u;
+  const int lrow = lane & 7, lmat = lane >> 3;
+  // ---- vᵀ (shared memory): ldmatrix.trans of block column w; lanes whose bit 1 and bit 4 differ
+  // trade their pair with lane ^ 18 so that each half-warp again covers one core matrix.
+  const int sw = ((lane >> 1) ^ (lane >> 4)) & 1;
+  const int srow = t4 ^ (sw << 2), stq = tq ^ (sw << 1);
+  const uint32_t offT = (uint32_t)(lmat * 8 + lrow) * 128u + (uint32_t)((warp ^ lrow) << 4);
+  // ---- k̃ᵀ (tensor memory, A of the state increment), .16x256b fragment of warp w:
+  // rows d = 16 q4 + t4 + 8 r, columns ι = 32 hc + 8 i + 2 tq + e  ->  register 4 i + 2 r + e
+  float fc0[2][2], fcs[2];
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    const float rate = expf(om[16 * q4 + 8 * r + t4]);
+#pragma unroll
+    for (int e = 0; e < 2; ++e) fc0[r][e] = expf(-rate * (float)(31 - 32 * hc - 2 * tq - e));
+    fcs[r] = expf(8.f * rate);
+  }
+  const uint32_t offKt = (uint32_t)((4 * hc + (lmat >> 1)) * 8 + lrow) * 128u +
+                         (uint32_t)(((2 * q4 + (lmat & 1)) ^ lrow) << 4);
+
+  // ---- state S[d][j] (fp32 master copy) in the .16x128b fragment of warp w:
+  // d = 16 q4 + t4 + 8 r, j = 32 hc + 4 q + tq  ->  S[2 q + r]
+  const int drow = 16 * q4 + t4;
+  const int jcol = 32 * hc + tq;
+  const uint32_t tquar = (uint32_t)(32 * q4) << 16;
+  float e32[2];
+#pragma unroll
+  for (int r = 0; r < 2; ++r) e32[r] = expf(-32.f * expf(om[drow + 8 * r]));
+  const size_t sbase = ((size_t)b * p.H + h) * kN * kN;
+  float S[16];
+#pragma unroll
+  for (int q = 0; q < 8; ++q)
+#pragma unroll
+    for (int r = 0; r < 2; ++r)
+      S[2 * q + r] = p.s_in ? p.s_in[sbase + (size_t)(drow + 8 * r) * kN + jcol + 4 * q] : 0.f;
+#pragma unroll
+  for (int q = 0; q < 8; ++q)
+#pragma unroll
+    for (int r = 0; r < 2; ++r) sm.opS[op_off(jcol + 4 * q, drow + 8 * r)] = e32[r] * S[2 * q + r];
+
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = sm.tmem_base;
-  const uint32_t tA = tbase, tY = tbase + 64, tD = tbase + 128;
-  const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
+  const uint32_t tSc = tbase, tY = tbase + 64, tDS = tbase + 128, tKt = tbase + 192;
+  const uint32_t rawR = smem_u32(sm.raw[0]), rawK = smem_u32(sm.raw[1]), rawV = smem_u32(sm.raw[2]);
+  const bool issuer = tid == 0;
 
-  // fp32 master state: rows d = 16*warp + lane held by lanes 0..15 (the M = 64
-  // accumulator layout puts row m in TMEM lane (m % 16) + 32 (m / 16)).
-  const bool holds_row = lane < 16;
-  const int srow = 16 * warp + lane;
-  const size_t sbase = ((size_t)b * p.H + h) * kN * kN;
-  float S[64];
-#pragma unroll
-  for (int j = 0; j < 64; ++j) S[j] = (holds_row && p.s_in) ? p.s_in[sbase + (size_t)srow * kN + j] : 0.f;
-  if (holds_row) {
-#pragma unroll
-    for (int j = 0; j < 64; ++j) sm.opS[op_off(j, srow)] = S[j];
-  }
-  const float my_decL = holds_row ? sm.decL[srow] : 0.f;
-
-  uint32_t mma_phase = 0;
   for (int c = 0; c < nchunk; ++c) {
-    const int st = c % kStages;
     const int t0 = c * kL;
     const int cnt = min(kL, p.T - t0);
-    if (!mbar_wait_bounded(&sm.bar_tma[st], (uint32_t)(c / kStages) & 1u, p.err)) sm.abort_flag = 1;
-    const __nv_bfloat16* Rr = sm.raw[st][0];
-    const __nv_bfloat16* Kr = sm.raw[st][1];
-    const __nv_bfloat16* Vr = sm.raw[st][2];
+    const uint32_t ph = (uint32_t)c & 1u;
+    if (!mbar_wait_bounded(&sm.bar_tma, ph, p.err)) sm.abort_flag = 1;
 
-    // T1: operands.  Each warp-quarter writes one core matrix (8 rows x 4 k).
-    // (the state increment of a partial last chunk uses e^{λ(cnt-1-ι)}: m = 31 + cnt - ι)
-    for (int q = tid; q < 256; q += kThreads) {
-      const int row = ((q >> 5) << 3) + (q & 7);  // 8-row group (q / 32), row inside it (q % 8)
-      const int kg = (q >> 3) & 3;
-      for (int kq = kg; kq < 16; kq += 4) {
-        const int k0 = kq * 4;
-        float4 vr, vk, vrh, vkh, vvt;
-        float* pr = &vr.x;
-        float* pk = &vk.x;
-        float* prh = &vrh.x;
-        float* pkh = &vkh.x;
-        float* pvt = &vvt.x;
+    // T1a: r̃, k̃ and the bonus parts (rows past the sequence end hold zeros from the TMA fill)
+    {
+      float fr[2] = {fr0[0], fr0[1]}, fk[2] = {fk0[0], fk0[1]};
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int col = k0 + e;
-          const float rv = raw_at(Rr, row, col), kv = raw_at(Kr, row, col);
-          pr[e] = rv * sm.dec[row * 64 + col];             // e^{λ(τ-32)}, m = τ
-          prh[e] = rv * sm.dec[(row + 32) * 64 + col];     // e^{λ τ}
-          pk[e] = kv * sm.dec[(63 - row) * 64 + col];      // e^{λ(31-ι)}, m = 63 - ι
-          // transposed operands: element (row = d or j, k = ι = col)
-          pkh[e] = raw_at(Kr, col, row) * sm.dec[max(0, 31 + cnt - col) * 64 + row];  // k[ι][d] e^{λ_d (cnt-1-ι)}
-          pvt[e] = raw_at(Vr, col, row);                                   // v[ι][j]
+      for (int ib = 0; ib < 8; ++ib) {
+        const float2 rv = bf2_to_f2(lds_u32(rawR + offRK + ib * 1024u));
+        const float2 kv = bf2_to_f2(lds_u32(rawK + offRK + ib * 1024u));
+        const int row = 8 * ib + rr;
+        *reinterpret_cast<float2*>(&sm.opR[op_off(row, dR)]) = make_float2(rv.x * fr[0], rv.y * fr[1]);
+        *reinterpret_cast<float2*>(&sm.opK[op_off(row, dR)]) = make_float2(kv.x * fk[0], kv.y * fk[1]);
+        float part = fmaf(rv.x * uA[0], kv.x, rv.y * uA[1] * kv.y);
+        part += __shfl_xor_sync(0xffffffffu, part, 8);
+        part += __shfl_xor_sync(0xffffffffu, part, 16);
+        if (rp == 0) sm.diag_part[warp][row] = part;
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          fr[e] *= frs[e];
+          fk[e] *= fks[e];
         }
-        const int o = op_off(row, k0);
-        *reinterpret_cast<float4*>(&sm.opR[o]) = vr;
-        *reinterpret_cast<float4*>(&sm.opRh[o]) = vrh;
-        *reinterpret_cast<float4*>(&sm.opK[o]) = vk;
-        *reinterpret_cast<float4*>(&sm.opKh[o]) = vkh;
-        *reinterpret_cast<float4*>(&sm.opVt[o]) = vvt;
       }
     }
-    // bonus Σ_d r u k for each token (exact, fp32)
-    {
-      const int tok = tid >> 1, half = tid & 1;
-      float acc = 0.f;
-      for (int d = half * 32; d < half * 32 + 32; ++d)
-        acc = fmaf(raw_at(Rr, tok, d) * sm.ud[d], raw_at(Kr, tok, d), acc);
-      acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-      if (half == 0) sm.diag[tok] = acc;
-    }
-    // rows past the end of the sequence hold zero keys and values (TMA zero fill)
     fence_proxy_async();
     tc_fence_before();
     __syncthreads();
     if (sm.abort_flag) break;
-    if (tid == 0) {
-      tc_fence_after();
-      // M1: scores A = r~ k~ᵀ; y = r^ S; ΔS = k^ᵀ v  (8 k-steps of 8 each)
+    // [scores | Y] = r̃ [k̃ ; e^{32λ} Sᵀ]ᵀ: causal scores [τ][ι] and the state read [τ][j].  The
+    // issuing thread hands the eight K steps out in pairs between its warp's T1b steps, so that
+    // the warp never waits on a full MMA queue.
+    auto issue_first = [&](int s0) {
+      if (issuer) {
+        if (s0 == 0) tc_fence_after();
 #pragma unroll
-      for (int s = 0; s < 8; ++s)
-        umma_tf32(tA, smem_desc(&sm.opR[s * 64], kLbo, kSbo), smem_desc(&sm.opK[s * 64], kLbo, kSbo), kIdesc, s);
-#pragma unroll
-      for (int s = 0; s < 8; ++s)
-        umma_tf32(tY, smem_desc(&sm.opRh[s * 64], kLbo, kSbo), smem_desc(&sm.opS[s * 64], kLbo, kSbo), kIdesc, s);
-#pragma unroll
-      for (int s = 0; s < 8; ++s)
-        umma_tf32(tD, smem_desc(&sm.opKh[s * 64], kLbo, kSbo), smem_desc(&sm.opVt[s * 64], kLbo, kSbo), kIdesc, s);
-      umma_commit(&sm.bar_mma);
-      // this chunk's raw tiles are consumed: refill the stage
-      if (c + kStages < nchunk) {
-        fence_proxy_async();
-        mbar_arrive_expect_tx(&sm.bar_tma[st], 3 * kRawBytes);
-        tma_load_3d(sm.raw[st][0], &mr, &sm.bar_tma[st], h * kN, (c + kStages) * kL, b);
-        tma_load_3d(sm.raw[st][1], &mk, &sm.bar_tma[st], h * kN, (c + kStages) * kL, b);
-        tma_load_3d(sm.raw[st][2], &mv, &sm.bar_tma[st], h * kN, (c + kStages) * kL, b);
+        for (int s = s0; s < s0 + 2; ++s)
+          umma_tf32(tSc, smem_desc(&sm.opR[s * 64], kLbo, kSbo), smem_desc(&sm.opK[s * 64], kLbo, kSbo),
+                    kIdesc128, s);
+        if (s0 == 6) umma_commit(&sm.bar_sc);
       }
-    }
-    if (!mbar_wait_bounded(&sm.bar_mma, mma_phase, p.err)) sm.abort_flag = 1;
-    mma_phase ^= 1u;
-    tc_fence_after();
+    };
+    issue_first(0);
 
-    // T2: masked scores -> opA; state update S' = e^{64λ} S + ΔS -> opS
+    // T1b: k̃ᵀ into tensor memory, vᵀ into shared memory, the bonus sums
     {
-      float a[64];
-      tmem_ld64(tA + lane_base, a);
-      if (holds_row) {
-        const int tau = srow;
+      if (tid < kL) {
+        float sum = 0.f;
 #pragma unroll
-        for (int kq = 0; kq < 16; ++kq) {
-          float4 o;
-          float* po = &o.x;
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int io = kq * 4 + e;
-            po[e] = io < tau ? a[io] : (io == tau ? sm.diag[tau] : 0.f);
-          }
-          *reinterpret_cast<float4*>(&sm.opA[op_off(tau, kq * 4)]) = o;
-        }
+        for (int w = 0; w < 8; ++w) sum += sm.diag_part[w][tid];
+        sm.diag[tid] = sum;
       }
-      float ds[64];
-      tmem_ld64(tD + lane_base, ds);
-      if (holds_row) {
-        const float dl = cnt == kL ? my_decL : expf(-expf(p.omega[h * kN + srow]) * (float)cnt);
+      uint32_t kt[16];
 #pragma unroll
-        for (int j = 0; j < 64; ++j) {
-          S[j] = fmaf(dl, S[j], ds[j]);
-          sm.opS[op_off(j, srow)] = S[j];
+      for (int pp = 0; pp < 2; ++pp) {
+        uint32_t qk[4];
+        ldsm_x4_t(rawK + offKt + pp * 2048u, qk);
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          const int i = 2 * pp + (m >> 1), r = m & 1;
+          const float2 f = bf2_to_f2(qk[m]);
+          const float g = i == 0 ? 1.f : (i == 1 ? fcs[r] : (i == 2 ? fcs[r] * fcs[r] : fcs[r] * fcs[r] * fcs[r]));
+          kt[4 * i + 2 * r] = __float_as_uint(f.x * fc0[r][0] * g);
+          kt[4 * i + 2 * r + 1] = __float_as_uint(f.y * fc0[r][1] * g);
         }
+        issue_first(2 + 2 * pp);
+      }
+      tmem_st16(tKt + tquar + (uint32_t)(32 * hc), kt);
+#pragma unroll
+      for (int pp = 0; pp < 2; ++pp) {
+        uint32_t qv[4];
+        ldsm_x4_t(rawV + offT + pp * 4096u, qv);
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          const int ib = 4 * pp + m;
+          const uint32_t xv = __shfl_xor_sync(0xffffffffu, qv[m], 18);
+          *reinterpret_cast<float2*>(&sm.opVt[op_off(8 * warp + srow, 8 * ib + 2 * stq)]) =
+              bf2_to_f2(sw ? xv : qv[m]);
+        }
+        if (pp == 0) issue_first(6);
       }
     }
     fence_proxy_async();
     tc_fence_before();
     __syncthreads();
-    if (tid == 0) {
+    if (issuer) {
       tc_fence_after();
-      // M2: y += A v
+      // the raw boxes are consumed: load the next chunk while this one computes
+      if (c + 1 < nchunk) {
+        fence_proxy_async();
+        mbar_arrive_expect_tx(&sm.bar_tma, 3 * kRawBytes);
+        tma_load_3d(sm.raw[0], &mr, &sm.bar_tma, h * kN, (c + 1) * kL, b);
+        tma_load_3d(sm.raw[1], &mk, &sm.bar_tma, h * kN, (c + 1) * kL, b);
+        tma_load_3d(sm.raw[2], &mv, &sm.bar_tma, h * kN, (c + 1) * kL, b);
+      }
+    }
+
+    // T2a: causal mask of the scores (ι < τ kept, ι = τ the bonus Σ_d r u k, ι > τ zero) -> opA.
+    // .16x128b fragment: rows τ = 16 q4 + t4 + 8 r, columns ι = 32 hc + 4 q + tq  ->  register 2 q + r
+    if (!mbar_wait_bounded(&sm.bar_sc, ph, p.err)) sm.abort_flag = 1;
+    tc_fence_after();
+    {
+      const int tau0 = 16 * q4 + t4;
+      if (hc > (q4 >> 1)) {  // strictly above the diagonal
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+#pragma unroll
+          for (int r = 0; r < 2; ++r) sm.opA[op_off(tau0 + 8 * r, 32 * hc + 4 * q + tq)] = 0.f;
+      } else {
+        float a[16];
+        tmem_ld16x128(tSc + tquar + (uint32_t)(32 * hc), a);
+        float dg[2] = {0.f, 0.f};
+        if ((q4 >> 1) == hc) {  // the fragment holds the diagonal
+          dg[0] = sm.diag[tau0];
+          dg[1] = sm.diag[tau0 + 8];
+        }
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+#pragma unroll
+          for (int r = 0; r < 2; ++r) {
+            const int io = 32 * hc + 4 * q + tq, tau = tau0 + 8 * r;
+            sm.opA[op_off(tau, io)] = io < tau ? a[2 * q + r] : (io == tau ? dg[r] : 0.f);
+          }
+      }
+    }
+    fence_proxy_async();
+    tc_fence_before();
+    __syncthreads();
+    if (issuer) {
+      tc_fence_after();
+      // Y += (masked scores) v
 #pragma unroll
       for (int s = 0; s < 8; ++s)
         umma_tf32(tY, smem_desc(&sm.opA[s * 64], kLbo, kSbo), smem_desc(&sm.opVt[s * 64], kLbo, kSbo), kIdesc, 1);
-      umma_commit(&sm.bar_mma);
-    }
-    if (!mbar_wait_bounded(&sm.bar_mma, mma_phase, p.err)) sm.abort_flag = 1;
-    mma_phase ^= 1u;
-    tc_fence_after();
-
-    // T3: y rows -> bf16 -> global
-    {
-      float yv[64];
-      tmem_ld64(tY + lane_base, yv);
-      if (holds_row && srow < cnt) {
-        __nv_bfloat16* yp = p.y + (((size_t)b * p.T + t0 + srow) * p.H + h) * kN;
+      umma_commit(&sm.bar_av);
+      // ΔS = k̃ᵀ v [d][j], k̃ᵀ read from tensor memory
 #pragma unroll
-        for (int j = 0; j < 64; j += 8) {
+      for (int s = 0; s < 8; ++s) umma_tf32_ts(tDS, tKt + 8 * s, smem_desc(&sm.opVt[s * 64], kLbo, kSbo), kIdesc, s);
+      umma_commit(&sm.bar_ds);
+    }
+
+    // T3: Y rows -> bf16 -> global (TMEM lanes 0..15 of each quarter hold the rows)
+    if (!mbar_wait_bounded(&sm.bar_av, ph, p.err)) sm.abort_flag = 1;
+    tc_fence_after();
+    {
+      float yv[32];
+      tmem_ld32(tY + tquar + (uint32_t)(32 * hc), yv);
+      const int tau = 16 * q4 + lane;
+      if (lane < 16 && tau < cnt) {
+        __nv_bfloat16* yp = p.y + (((size_t)b * p.T + t0 + tau) * p.H + h) * kN + 32 * hc;
+#pragma unroll
+        for (int j = 0; j < 32; j += 8) {
           uint4 pk;
           __nv_bfloat162* q2 = reinterpret_cast<__nv_bfloat162*>(&pk);
 #pragma unroll
@@ -399,13 +522,40 @@ __global__ void __launch_bounds__(kThreads, 1) wkv5_fwd_tc_kernel(const __grid_c
         }
       }
     }
-    tc_fence_before();
-    __syncthreads();
+
+    // T2b: S <- e^{cnt λ} S + e^{(cnt-32) λ} ΔS; e^{32λ} Sᵀ into opS for the next chunk
+    if (!mbar_wait_bounded(&sm.bar_ds, ph, p.err)) sm.abort_flag = 1;
+    tc_fence_after();
+    {
+      float ds[16];
+      tmem_ld16x128(tDS + tquar + (uint32_t)(32 * hc), ds);
+      if (cnt == kL) {
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+#pragma unroll
+          for (int r = 0; r < 2; ++r) {
+            const int x = 2 * q + r;
+            const float g = e32[r];
+            S[x] = g * fmaf(g, S[x], ds[x]);
+            sm.opS[op_off(jcol + 4 * q, drow + 8 * r)] = g * S[x];
+          }
+      } else {  // last, partial chunk: no later chunk reads opS
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          const float rate = expf(om[drow + 8 * r]);
+          const float dl = expf(-rate * (float)cnt), gs = expf(-rate * (float)(cnt - 32));
+#pragma unroll
+          for (int q = 0; q < 8; ++q) S[2 * q + r] = fmaf(dl, S[2 * q + r], gs * ds[2 * q + r]);
+        }
+      }
+    }
   }
 
-  if (p.s_out != nullptr && holds_row) {
+  if (p.s_out != nullptr) {
 #pragma unroll
-    for (int j = 0; j < 64; ++j) p.s_out[sbase + (size_t)srow * kN + j] = S[j];
+    for (int q = 0; q < 8; ++q)
+#pragma unroll
+      for (int r = 0; r < 2; ++r) p.s_out[sbase + (size_t)(drow + 8 * r) * kN + jcol + 4 * q] = S[2 * q + r];
   }
   tc_fence_before();
   __syncthreads();
@@ -417,9 +567,11 @@ __global__ void __launch_bounds__(kThreads, 1) wkv5_fwd_tc_kernel(const __grid_c
 
 }  // namespace
 
+size_t wkv5_smem_bytes() { return sizeof(Wkv5Smem) + 1024; }  // + alignment slack
+
 cudaError_t launch_wkv5_fwd(const CUtensorMap& mr, const CUtensorMap& mk, const CUtensorMap& mv, const Wkv5Params& p,
                             cudaStream_t st) {
-  const size_t smem = sizeof(Wkv5Smem) + 1024;  // + alignment slack
+  const size_t smem = wkv5_smem_bytes();
   static unsigned device_mask = 0;
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(wkv5_fwd_tc_kernel), (int)smem, &device_mask);
   if (e != cudaSuccess) return e;
@@ -427,6 +579,5 @@ cudaError_t launch_wkv5_fwd(const CUtensorMap& mr, const CUtensorMap& mk, const 
   return cudaGetLastError();
 }
 
-size_t wkv5_smem_bytes() { return sizeof(Wkv5Smem) + 1024; }
 
 }  // namespace rwkv
