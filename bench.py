@@ -221,6 +221,7 @@ def run_ours(args):
 
     import rwkv_wkv_recurrence_b200 as rw
     import wkv_inputs as wi
+    from rwkv_wkv_recurrence_b200.dist_timing import max_over_ranks, rank_seed, weak_scaling_throughput
 
     world, rank, local = _dist()
     torch.cuda.set_device(local)
@@ -237,7 +238,7 @@ def run_ours(args):
     h = rw.lib()
     stream = torch.cuda.current_stream()
     # each rank its own independent problem (weak scaling)
-    p = wi.wkv4_problem(B, T, C, SEED + 1000 * rank, outliers=True, with_gy=True, device=dev)
+    p = wi.wkv4_problem(B, T, C, rank_seed(SEED, rank), outliers=True, with_gy=True, device=dev)
     w, u, k, v, gy = p["w"], p["u"], p["k"], p["v"], p["gy"]
     y = torch.empty_like(k)
     gk, gv = torch.empty_like(k), torch.empty_like(k)
@@ -294,11 +295,8 @@ def run_ours(args):
     total_ms = start.elapsed_time(end)
     fwd_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
     bwd_ms = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
-    t_max = torch.tensor([total_ms], device=dev)
-    if dist is not None:
-        dist.all_reduce(t_max, op=dist.ReduceOp.MAX)
-    ms_step = t_max.item() / args.steps
-    value = world * ELEM / (ms_step * 1e-3)
+    ms_step = max_over_ranks(total_ms, dev) / args.steps
+    value = weak_scaling_throughput(ELEM, world, ms_step)
 
     # end to end through the public API with host buffers (pinned), copies timed
     hk, hv, hgy = (x.cpu().pin_memory() for x in (k, v, gy))
@@ -323,10 +321,7 @@ def run_ours(args):
         e2e_step()
     e1.record(stream)
     barrier()
-    e_ms = torch.tensor([e0.elapsed_time(e1) / e2e_steps], device=dev)
-    if dist is not None:
-        dist.all_reduce(e_ms, op=dist.ReduceOp.MAX)
-    e2e_val = world * ELEM / (e_ms.item() * 1e-3)
+    e2e_val = weak_scaling_throughput(ELEM, world, max_over_ranks(e0.elapsed_time(e1) / e2e_steps, dev))
 
     if rank == 0:
         peak, peak_kind = _peaks()
