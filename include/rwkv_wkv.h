@@ -101,8 +101,10 @@ RWKV_API size_t rwkv_wkv4_forward_workspace_bytes(int64_t B, int64_t T, int64_t 
  *   state_in  [3,B,C] or NULL (zero state).  state_out [3,B,C] or NULL:
  *             the state after the last token; may equal state_in.
  *   ckpt      [num_checkpoints(T, chunk_len), 3, B, C] or NULL: ckpt[j] is
- *             the state before token j·chunk_len (ckpt[0] = state_in); it is
- *             what rwkv_wkv4_backward reads.  chunk_len must be 16 today.
+ *             the state before token j·chunk_len (ckpt[0] = state_in), in
+ *             the state format, with p chosen at least ceil(k·log2 e) for
+ *             every key of that chunk and b < 1; rwkv_wkv4_backward reads it
+ *             and relies on that choice.  chunk_len must be 16 today.
  *   algo      rwkv_algo.   workspace: device scratch of
  *             rwkv_wkv4_forward_workspace_bytes() bytes (may be NULL if 0).
  */

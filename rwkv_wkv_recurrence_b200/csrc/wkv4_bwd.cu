@@ -16,7 +16,9 @@
 // its carry, and the carries come from folding each chunk's local sums.
 //
 // Scaling.  Inside a chunk everything is measured against one power of two
-// 2^q: e_t = e^{k_t} 2^{-q}, d_t = D_t 2^{-q}, G_t = gy_t / d_t, and the
+// 2^q, the exponent the forward wrote the chunk's checkpoint at (q is at least
+// every k log2 e of the chunk, so no weight exceeds 1, and above the state's
+// b): e_t = e^{k_t} 2^{-q}, d_t = D_t 2^{-q}, G_t = gy_t / d_t, and the
 // carries are kept as α~ = α 2^q; then e^{k_t} α_t = e_t α~_t and
 // α_t A_{t-1} = α~_t a_{t-1}, so the scale cancels from every gradient.
 // Precision.  The gradient terms cancel each other (α_t v_t + β_t is small
@@ -201,14 +203,11 @@ __global__ void __launch_bounds__(kW * 32, 4) wkv4_bwd_kernel(const __grid_const
     const T* vs = ks + kBoxElems;
     const T* gs = vs + kBoxElems;
 
-    // A. forward recompute of the chunk at one scale 2^q
+    // A. forward recompute of the chunk at one scale 2^q: the forward wrote the
+    //    checkpoint at the chunk's scale (at least every k log2 e of the chunk,
+    //    and b < 1), so q is the checkpoint's exponent
     float E[kL], G[kL], Y[kL], BP[kL];
-    float kmax = -INFINITY;
-#pragma unroll
-    for (int j = 0; j < kL; ++j)
-      if (j < cnt) kmax = fmaxf(kmax, IO<T>::to_f(ks[j * 32]) * kL2eHi);
-    const int q = cnt > 0 ? segment_scale(kmax, st) : 0;
-    st = rescale(st, q);
+    const int q = st.p;
     if (cnt == kL)
       chunk_recompute<T, true>(ks, vs, gs, cnt, (float)q, U, lh, ll, (float)st.a, (float)st.b, E, G, Y, BP);
     else if (cnt > 0)

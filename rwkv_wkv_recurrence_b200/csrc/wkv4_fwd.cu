@@ -210,13 +210,17 @@ __global__ void __launch_bounds__(kW * 32, 4) wkv4_fwd_kernel(const __grid_const
 
     // 3. rescan from the true state: outputs and checkpoints
     if (cnt > 0 && rescan) {
+      // the segment's scale: at least every k log2 e of the segment and above the state's b
+      const int q = segment_scale(kmax, mine);
+      const State sc = rescale(mine, q);
       if (p.ckpt != nullptr && valid && (ts % p.ckpt_len) == 0) {
+        // checkpoints are written at that scale (b < 1), so the backward takes q from them
         float* ck = p.ckpt + (size_t)(ts / p.ckpt_len) * 3 * plane + lane_off;
-        store_state(mine, &ck[0], &ck[plane], &ck[2 * plane]);
+        ck[0] = (float)sc.a;
+        ck[plane] = (float)sc.b;
+        ck[2 * plane] = (float)q;
       }
       if (ybase != nullptr) {
-        const int q = segment_scale(kmax, mine);
-        const State sc = rescale(mine, q);
         const float f = pow2f_neg(p1 - q);
         T* yp = ybase + (size_t)ts * C;
         if (cnt == kL)
