@@ -113,8 +113,13 @@ rwkv_status run_forward(int B, int T, int C, bool bf16, const float* w, const fl
   unsigned int* err = device_error_word();
   if (err == nullptr) return RWKV_ERR_CUDA;
   const int tt = fwd_tile_steps();
-  CUtensorMap mk, mv;
+  CUtensorMap mk, mv, my;
   if (!make_btc_map(&mk, k, bf16, B, T, C, tt) || !make_btc_map(&mv, v, bf16, B, T, C, tt)) return RWKV_ERR_CUDA;
+  if (y != nullptr) {
+    if (!make_btc_map(&my, y, bf16, B, T, C, fwd_store_steps())) return RWKV_ERR_CUDA;
+  } else {
+    my = mk;  // not read without y
+  }
   Fwd4Params p{};
   p.B = B;
   p.T = T;
@@ -133,7 +138,7 @@ rwkv_status run_forward(int B, int T, int C, bool bf16, const float* w, const fl
     p.start = state_in;
     p.end = state_out;
     p.ckpt = ckpt;
-    if (launch_wkv4_fwd(bf16, mk, mv, p, st) != cudaSuccess) return RWKV_ERR_CUDA;
+    if (launch_wkv4_fwd(bf16, mk, mv, my, p, st) != cudaSuccess) return RWKV_ERR_CUDA;
     return RWKV_OK;
   }
   float* wsf = static_cast<float*>(ws);
@@ -146,7 +151,7 @@ rwkv_status run_forward(int B, int T, int C, bool bf16, const float* w, const fl
   p.end = wsf;
   p.end_seg_stride = seg_stride;
   p.ckpt = nullptr;
-  if (launch_wkv4_fwd(bf16, mk, mv, p, st) != cudaSuccess) return RWKV_ERR_CUDA;
+  if (launch_wkv4_fwd(bf16, mk, mv, my, p, st) != cudaSuccess) return RWKV_ERR_CUDA;
   // 2) carries (in place) and the final state
   if (launch_wkv4_carry(B, C, T, pl.nseg, pl.seg_len, w, state_in, wsf, state_out, st) != cudaSuccess)
     return RWKV_ERR_CUDA;
@@ -156,7 +161,7 @@ rwkv_status run_forward(int B, int T, int C, bool bf16, const float* w, const fl
   p.start_seg_stride = seg_stride;
   p.end = nullptr;
   p.ckpt = ckpt;
-  if (launch_wkv4_fwd(bf16, mk, mv, p, st) != cudaSuccess) return RWKV_ERR_CUDA;
+  if (launch_wkv4_fwd(bf16, mk, mv, my, p, st) != cudaSuccess) return RWKV_ERR_CUDA;
   return RWKV_OK;
 }
 
@@ -211,7 +216,8 @@ rwkv_status rwkv_wkv4_forward(int64_t B, int64_t T, int64_t C, rwkv_dtype dtype,
   if (k == nullptr || v == nullptr) return RWKV_ERR_INVALID_ARG;
   if (y == nullptr && state_out == nullptr && ckpt == nullptr) return RWKV_ERR_INVALID_ARG;
   const bool bf16 = dtype == RWKV_BF16;
-  if (!aligned16(k) || !aligned16(v) || (C * (bf16 ? 2 : 4)) % 16 != 0) return RWKV_ERR_UNSUPPORTED;
+  if (!aligned16(k) || !aligned16(v) || (y != nullptr && !aligned16(y)) || (C * (bf16 ? 2 : 4)) % 16 != 0)
+    return RWKV_ERR_UNSUPPORTED;
   const FwdPlan pl = plan_forward(B, T, C, algo);
   if (pl.ws_bytes > 0 && (workspace == nullptr || workspace_bytes < pl.ws_bytes)) return RWKV_ERR_WORKSPACE;
   return run_forward((int)B, (int)T, (int)C, bf16, w, u, k, v, y, state_in, state_out, ckpt, (int)chunk_len, pl,

@@ -55,11 +55,14 @@ struct Wkv5Params {
 };
 
 int fwd_tile_steps();
+int fwd_store_steps();
 int fwd_stages(bool bf16, int seg_len);
 int bwd_tile_steps();
 int bwd_stages(bool bf16, int T);
-cudaError_t launch_wkv4_fwd(bool bf16, const CUtensorMap& mk, const CUtensorMap& mv, const Fwd4Params& p,
-                            cudaStream_t st);
+// mk, mv: [fwd_tile_steps() x 32] boxes over k, v; my: [fwd_store_steps() x 32] boxes over y
+// (TMA stores; any valid map when p.y is null).
+cudaError_t launch_wkv4_fwd(bool bf16, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& my,
+                            const Fwd4Params& p, cudaStream_t st);
 cudaError_t launch_wkv4_carry(int B, int C, int T, int nseg, int seg_len, const float* w, const float* state_in,
                               float* ws, float* state_out, cudaStream_t st);
 cudaError_t launch_wkv4_bwd(bool bf16, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mgy,

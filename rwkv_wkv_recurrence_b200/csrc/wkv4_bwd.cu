@@ -68,8 +68,8 @@ __device__ __forceinline__ void chunk_recompute(const T* ks, const T* vs, const 
       const float eu = e * U;
       const float vj = IO<T>::to_f(vs[j * 32]);
       const float d = b + eu;
-      const float rd = __fdividef(1.f, d);
-      const bool ok = d > 0.f;  // d == 0: no history and e^{u+k} underflowed, WKV = v locally
+      const float rd = rcp_approx(d);
+      const bool ok = d >= kMinDen;  // else no history and e^{u+k} underflowed: WKV = v locally
       Y[j] = ok ? fmaf(eu, vj, a) * rd : vj;
       G[j] = ok ? IO<T>::to_f(gs[j * 32]) * rd : 0.f;
       E[j] = e;

@@ -69,10 +69,11 @@ __device__ __forceinline__ void seg_summary(const T* ks, const T* vs, int cnt, f
 }
 
 // Phase 3 of one segment: rescan from the true state (a, b) at the segment's
-// scale, weights E * f, writing y to yp, yp + C, ...
+// scale, weights E * f, writing y_j to ys[j * 32] (the segment's k rows in
+// shared memory, which phase 1 has consumed).
 template <typename T, bool FULL>
 __device__ __forceinline__ void seg_output(const T* vs, int cnt, const float (&E)[kL], float f, float U, float a,
-                                           float b, float lh, float ll, T* yp, size_t C, bool valid) {
+                                           float b, float lh, float ll, T* ys) {
 #pragma unroll
   for (int j = 0; j < kL; ++j) {
     if (FULL || j < cnt) {
@@ -81,9 +82,8 @@ __device__ __forceinline__ void seg_output(const T* vs, int cnt, const float (&E
       const float vj = IO<T>::to_f(vs[j * 32]);
       const float d = b + eu;
       const float n = fmaf(eu, vj, a);
-      const float y = d > 0.f ? __fdividef(n, d) : vj;  // d == 0: no history and e^{u+k} underflowed
-      if (valid) *yp = IO<T>::from_f(y);
-      yp += C;
+      const float y = d >= kMinDen ? n * rcp_approx(d) : vj;
+      ys[j * 32] = IO<T>::from_f(y);
       a = decay_add(a, e * vj, lh, ll);
       b = decay_add(b, e, lh, ll);
     }
@@ -98,6 +98,7 @@ struct CarrySlot {  // CTA running state at a tile boundary, per lane
 template <typename T>
 __global__ void __launch_bounds__(kW * 32, 4) wkv4_fwd_kernel(const __grid_constant__ CUtensorMap mk,
                                                               const __grid_constant__ CUtensorMap mv,
+                                                              const __grid_constant__ CUtensorMap my,
                                                               const Fwd4Params p) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   constexpr uint32_t kBoxElems = kTile * 32;
@@ -143,7 +144,6 @@ __global__ void __launch_bounds__(kW * 32, 4) wkv4_fwd_kernel(const __grid_const
   const float U = expf(u);
   const size_t plane = (size_t)p.B * p.C;
   const size_t lane_off = (size_t)bb * p.C + c;
-  const size_t C = (size_t)p.C;
 
   if (warp == kW - 1) {  // running state entering the first tile
     State s0{0.0, 0.0, 0};
@@ -155,7 +155,7 @@ __global__ void __launch_bounds__(kW * 32, 4) wkv4_fwd_kernel(const __grid_const
   }
   __syncthreads();
 
-  T* ybase = p.y ? reinterpret_cast<T*>(p.y) + (size_t)bb * p.T * C + c : nullptr;
+  const bool write_y = p.y != nullptr;
   const bool rescan = (p.y != nullptr) || (p.ckpt != nullptr);
   State total{0.0, 0.0, 0};
 
@@ -178,6 +178,8 @@ __global__ void __launch_bounds__(kW * 32, 4) wkv4_fwd_kernel(const __grid_const
       seg_summary<T, false>(ks, vs, cnt, lh, ll, kmax, p1, la, lb, E);
     Summ* sb = summ + (i & 1) * kW * 32;
     sb[warp * 32 + lane] = Summ{la, lb, (float)p1, 0.f};
+    // the previous tile's y box must be out of shared memory before its stage is refilled below
+    if (lane == 0) bulk_wait_read();
     __syncthreads();
     if (*abort_flag) break;
     // every warp is done with tile i-1: refill its stage
@@ -220,16 +222,24 @@ __global__ void __launch_bounds__(kW * 32, 4) wkv4_fwd_kernel(const __grid_const
         ck[plane] = (float)sc.b;
         ck[2 * plane] = (float)q;
       }
-      if (ybase != nullptr) {
+      if (write_y) {
         const float f = pow2f_neg(p1 - q);
-        T* yp = ybase + (size_t)ts * C;
+        T* const yw = const_cast<T*>(ks) - lane;  // this warp's [16][32] k rows
         if (cnt == kL)
-          seg_output<T, true>(vs, cnt, E, f, U, (float)sc.a, (float)sc.b, lh, ll, yp, C, valid);
+          seg_output<T, true>(vs, cnt, E, f, U, (float)sc.a, (float)sc.b, lh, ll, yw + lane);
         else
-          seg_output<T, false>(vs, cnt, E, f, U, (float)sc.a, (float)sc.b, lh, ll, yp, C, valid);
+          seg_output<T, false>(vs, cnt, E, f, U, (float)sc.a, (float)sc.b, lh, ll, yw + lane);
+        // y of the segment as one [16 x 32] box (rows past T and channels past C are clipped)
+        fence_proxy_async();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_3d(&my, yw, ct * 32, ts, bb);
+          bulk_commit();
+        }
       }
     }
   }
+  if (lane == 0) bulk_wait_all();
 
   if (p.end != nullptr && valid && warp == kW - 1) {
     float* e = p.end + (size_t)seg * p.end_seg_stride;
@@ -273,19 +283,22 @@ size_t fwd_smem_bytes(int stages) {
 }
 
 template <typename T>
-cudaError_t launch_fwd_t(const CUtensorMap& mk, const CUtensorMap& mv, const Fwd4Params& p, cudaStream_t st) {
+cudaError_t launch_fwd_t(const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& my, const Fwd4Params& p,
+                         cudaStream_t st) {
   const size_t smem = fwd_smem_bytes<T>(p.stages);
   static unsigned device_mask = 0;
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(wkv4_fwd_kernel<T>), (int)smem, &device_mask);
   if (e != cudaSuccess) return e;
   const long long nblk = (long long)p.ctiles * p.B * p.nseg;
-  wkv4_fwd_kernel<T><<<(unsigned)nblk, kW * 32, smem, st>>>(mk, mv, p);
+  wkv4_fwd_kernel<T><<<(unsigned)nblk, kW * 32, smem, st>>>(mk, mv, my, p);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 int fwd_tile_steps() { return kTile; }
+
+int fwd_store_steps() { return kL; }
 
 int fwd_stages(bool bf16, int seg_len) {
   // three stages of fp32 boxes (48 KB) keep four CTAs per SM; bf16 boxes are half as big
@@ -294,9 +307,9 @@ int fwd_stages(bool bf16, int seg_len) {
   return max(2, min(want, ntile));
 }
 
-cudaError_t launch_wkv4_fwd(bool bf16, const CUtensorMap& mk, const CUtensorMap& mv, const Fwd4Params& p,
-                            cudaStream_t st) {
-  return bf16 ? launch_fwd_t<__nv_bfloat16>(mk, mv, p, st) : launch_fwd_t<float>(mk, mv, p, st);
+cudaError_t launch_wkv4_fwd(bool bf16, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& my,
+                            const Fwd4Params& p, cudaStream_t st) {
+  return bf16 ? launch_fwd_t<__nv_bfloat16>(mk, mv, my, p, st) : launch_fwd_t<float>(mk, mv, my, p, st);
 }
 
 cudaError_t launch_wkv4_carry(int B, int C, int T, int nseg, int seg_len, const float* w, const float* state_in,

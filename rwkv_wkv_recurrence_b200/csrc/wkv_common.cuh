@@ -81,6 +81,20 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
       : "memory");
 }
 
+// 3-D tiled TMA store (shared -> global) of one box, tracked by the issuing
+// thread's bulk async-group; the box is clipped at the tensor's bounds.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* src, int c0, int c1, int c2) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// The thread's bulk stores have finished reading shared memory.
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// The thread's bulk stores are complete.
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -91,6 +105,19 @@ __device__ __forceinline__ float ex2(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+
+// 1/x on the special-function unit (PTX rcp.approx.ftz.f32, ~1 ulp); callers
+// only pass normal x (x >= FLT_MIN), the denominators of the WKV ratio.
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// A WKV denominator too small to divide by: it is below FLT_MIN only when a
+// token arrives with no history and its own weight e^{u+k} underflowed at the
+// segment's scale, where the ratio is v itself.
+constexpr float kMinDen = 1.17549435e-38f;
 
 // ---------------------------------------------------------------- I/O types
 template <typename T>
@@ -281,7 +308,7 @@ __device__ __forceinline__ float wkv4_step_careful(float& a, float& b, float& p,
   const float eu = e * L.U;
   const float d = b + eu;
   const float n = fmaf(eu, vt, a);
-  const float y = (d > 0.f) ? __fdividef(n, d) : vt;  // d == 0 only if no history and e^{u+k} underflowed
+  const float y = (d >= kMinDen) ? n * rcp_approx(d) : vt;
   a = fmaf(L.lam, a, fmaf(L.lam_lo, a, e * vt));
   b = fmaf(L.lam, b, fmaf(L.lam_lo, b, e));
   return y;
