@@ -39,7 +39,7 @@
  *     before anything is enqueued.  A launch failure gives RWKV_ERR_CUDA.
  *     Zero-sized problems are a successful no-op (T = 0 copies the state).
  *   - Values are data: no range validation; NaN and Inf propagate.
- *   - Alignment: the WKV-4 [B,T,C] tensors k, v, y, gy (and the WKV-5
+ *   - Alignment: the WKV-4 [B,T,C] tensors k, v, y, gy, gk, gv (and the WKV-5
  *     tensors r, k, v, y) must be 16-byte aligned with C·sizeof(element) a
  *     multiple of 16 (TMA row pitch), else RWKV_ERR_UNSUPPORTED.
  */

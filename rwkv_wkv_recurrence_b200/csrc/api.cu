@@ -250,7 +250,8 @@ rwkv_status rwkv_wkv4_backward(int64_t B, int64_t T, int64_t C, rwkv_dtype dtype
   }
   if (k == nullptr || v == nullptr || gy == nullptr || gk == nullptr || gv == nullptr) return RWKV_ERR_INVALID_ARG;
   const bool bf16 = dtype == RWKV_BF16;
-  if (!aligned16(k) || !aligned16(v) || !aligned16(gy) || (C * (bf16 ? 2 : 4)) % 16 != 0)
+  if (!aligned16(k) || !aligned16(v) || !aligned16(gy) || !aligned16(gk) || !aligned16(gv) ||
+      (C * (bf16 ? 2 : 4)) % 16 != 0)
     return RWKV_ERR_UNSUPPORTED;
   const size_t need = rwkv_wkv4_backward_workspace_bytes(B, T, C, chunk_len, ckpt != nullptr);
   if (workspace == nullptr || workspace_bytes < need) return RWKV_ERR_WORKSPACE;
@@ -268,9 +269,11 @@ rwkv_status rwkv_wkv4_backward(int64_t B, int64_t T, int64_t C, rwkv_dtype dtype
   unsigned int* err = device_error_word();
   if (err == nullptr) return RWKV_ERR_CUDA;
   const int box_t = bwd_tile_steps();
-  CUtensorMap mk, mv, mg;
+  CUtensorMap mk, mv, mg, mgk, mgv;
   if (!make_btc_map(&mk, k, bf16, iB, iT, iC, box_t) || !make_btc_map(&mv, v, bf16, iB, iT, iC, box_t) ||
-      !make_btc_map(&mg, gy, bf16, iB, iT, iC, box_t))
+      !make_btc_map(&mg, gy, bf16, iB, iT, iC, box_t) ||
+      !make_btc_map(&mgk, gk, bf16, iB, iT, iC, bwd_store_steps()) ||
+      !make_btc_map(&mgv, gv, bf16, iB, iT, iC, bwd_store_steps()))
     return RWKV_ERR_CUDA;
   Bwd4Params p{};
   p.B = iB;
@@ -285,7 +288,7 @@ rwkv_status rwkv_wkv4_backward(int64_t B, int64_t T, int64_t C, rwkv_dtype dtype
   p.gv = gv;
   p.part = part;
   p.err = err;
-  if (launch_wkv4_bwd(bf16, mk, mv, mg, p, st) != cudaSuccess) return RWKV_ERR_CUDA;
+  if (launch_wkv4_bwd(bf16, mk, mv, mg, mgk, mgv, p, st) != cudaSuccess) return RWKV_ERR_CUDA;
   if (launch_wkv4_reduce_wu(iB, iC, part, gw, gu, st) != cudaSuccess) return RWKV_ERR_CUDA;
   return RWKV_OK;
 }

@@ -33,9 +33,12 @@
 // tile's w-th 16-step chunk: it recomputes that chunk's forward from the
 // forward pass's checkpoint, keeps e_t, G_t, y_t and b_{t-1} in registers,
 // sums its local reverse carries, folds the carries of the chunks after it,
-// then walks the chunk backwards writing gk and gv.  k, v, gy arrive by TMA
-// (no multicast); each element is read once and each gradient written once.
-// Per-lane gw, gu partials are reduced over the batch by a second kernel.
+// then walks the chunk backwards.  k, v, gy arrive by TMA (no multicast); the
+// walk writes gk and gv over the chunk's consumed k and v rows in shared
+// memory and the warp sends its two [16 x 32] boxes out with TMA stores, so
+// each element is read once and each gradient written once, without
+// per-element address arithmetic.  Per-lane gw, gu partials are reduced over
+// the batch by a second kernel.
 #include "launch.h"
 #include "wkv_common.cuh"
 
@@ -98,12 +101,11 @@ __device__ __forceinline__ void chunk_local_sums(int cnt, const float (&G)[kL], 
 }
 
 // Phase D: the reverse walk of one chunk from its carry (al, ga) at the last
-// step, writing gk, gv upwards from row pointer gkp, gvp (rows C apart).
+// step, writing gk_j over k_j (ks[j * 32]) and gv_j over v_j (vs[j * 32]).
 template <typename T, bool FULL>
-__device__ __forceinline__ void chunk_walk(const T* vs, int cnt, const float (&E)[kL], const float (&G)[kL],
+__device__ __forceinline__ void chunk_walk(T* ks, T* vs, int cnt, const float (&E)[kL], const float (&G)[kL],
                                            const float (&Y)[kL], const float (&BP)[kL], float U, float lh,
-                                           float ll, float al, float ga, T* gkp, T* gvp, size_t C, bool valid,
-                                           float& gws, float& gus) {
+                                           float ll, float al, float ga, float& gws, float& gus) {
 #pragma unroll
   for (int j = kL - 1; j >= 0; --j) {
     if (FULL || j < cnt) {
@@ -118,10 +120,8 @@ __device__ __forceinline__ void chunk_walk(const T* vs, int cnt, const float (&E
       gus = fmaf(ug * E[j], dv, gus);
       al = decay_add(al, G[j], lh, ll);
       if (j > 0) ga = decay_add(ga, (Y[j - 1] - Y[j]) * al, lh, ll);
-      if (valid) {
-        gkp[(size_t)j * C] = IO<T>::from_f(gkt);
-        gvp[(size_t)j * C] = IO<T>::from_f(gvt);
-      }
+      ks[j * 32] = IO<T>::from_f(gkt);
+      vs[j * 32] = IO<T>::from_f(gvt);
     }
   }
 }
@@ -136,6 +136,8 @@ template <typename T>
 __global__ void __launch_bounds__(kW * 32, 4) wkv4_bwd_kernel(const __grid_constant__ CUtensorMap mk,
                                                               const __grid_constant__ CUtensorMap mv,
                                                               const __grid_constant__ CUtensorMap mg,
+                                                              const __grid_constant__ CUtensorMap mgk,
+                                                              const __grid_constant__ CUtensorMap mgv,
                                                               const Bwd4Params p) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   constexpr uint32_t kBoxElems = kTile * 32;
@@ -181,7 +183,6 @@ __global__ void __launch_bounds__(kW * 32, 4) wkv4_bwd_kernel(const __grid_const
   const float U = expf(u);
   const size_t plane = (size_t)p.B * p.C;
   const size_t lane_off = (size_t)bb * p.C + c;
-  const size_t C = (size_t)p.C;
 
   double gw_acc = 0.0, gu_acc = 0.0;
 
@@ -199,8 +200,10 @@ __global__ void __launch_bounds__(kW * 32, 4) wkv4_bwd_kernel(const __grid_const
       st = load_state(ck[0], ck[plane], ck[2 * plane]);
     }
     if (!mbar_wait_bounded(&bars[s], ph, p.err)) *abort_flag = 1;
-    const T* ks = tiles + (size_t)(3 * s) * kBoxElems + warp * kL * 32 + lane;
-    const T* vs = ks + kBoxElems;
+    T* const kw = tiles + (size_t)(3 * s) * kBoxElems + warp * kL * 32;  // this warp's [16][32] rows
+    T* const vw = kw + kBoxElems;
+    T* const ks = kw + lane;
+    T* const vs = vw + lane;
     const T* gs = vs + kBoxElems;
 
     // A. forward recompute of the chunk at one scale 2^q: the forward wrote the
@@ -221,6 +224,8 @@ __global__ void __launch_bounds__(kW * 32, 4) wkv4_bwd_kernel(const __grid_const
       chunk_local_sums<false>(cnt, G, Y, lh, ll, la, lg, ye);
     RSumm* sb = rs + (i & 1) * kW * 32;
     sb[warp * 32 + lane] = RSumm{la, lg, cnt > 0 ? Y[0] : 0.f, ye, (float)q, 0.f};
+    // the previous tile's gradient boxes must be out of shared memory before its stage is refilled below
+    if (lane == 0) bulk_wait_read();
     __syncthreads();
     if (*abort_flag) break;
     if (threadIdx.x == 0 && i >= 1 && i - 1 + p.stages < ntile) {
@@ -272,16 +277,23 @@ __global__ void __launch_bounds__(kW * 32, 4) wkv4_bwd_kernel(const __grid_const
     // never subtracts two large nearly equal fp32 numbers.
     if (cnt > 0) {
       float gws = 0.f, gus = 0.f;
-      T* gkp = reinterpret_cast<T*>(p.gk) + ((size_t)bb * p.T + ts) * C + c;
-      T* gvp = reinterpret_cast<T*>(p.gv) + ((size_t)bb * p.T + ts) * C + c;
       if (cnt == kL)
-        chunk_walk<T, true>(vs, cnt, E, G, Y, BP, U, lh, ll, (float)ae, (float)ge, gkp, gvp, C, valid, gws, gus);
+        chunk_walk<T, true>(ks, vs, cnt, E, G, Y, BP, U, lh, ll, (float)ae, (float)ge, gws, gus);
       else
-        chunk_walk<T, false>(vs, cnt, E, G, Y, BP, U, lh, ll, (float)ae, (float)ge, gkp, gvp, C, valid, gws, gus);
+        chunk_walk<T, false>(ks, vs, cnt, E, G, Y, BP, U, lh, ll, (float)ae, (float)ge, gws, gus);
       gw_acc += (double)gws;
       gu_acc += (double)gus;
+      // gk, gv of the chunk: one [16 x 32] box each (rows past T and channels past C are clipped)
+      fence_proxy_async();
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_3d(&mgk, kw, ct * 32, ts, bb);
+        tma_store_3d(&mgv, vw, ct * 32, ts, bb);
+        bulk_commit();
+      }
     }
   }
+  if (lane == 0) bulk_wait_all();
 
   // reduce the four warps' gw, gu partials of each lane
   __syncthreads();
@@ -322,20 +334,22 @@ size_t bwd_smem_bytes(int stages) {
 }
 
 template <typename T>
-cudaError_t launch_bwd_t(const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mg, const Bwd4Params& p,
-                         cudaStream_t st) {
+cudaError_t launch_bwd_t(const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mg, const CUtensorMap& mgk,
+                         const CUtensorMap& mgv, const Bwd4Params& p, cudaStream_t st) {
   const size_t smem = bwd_smem_bytes<T>(p.stages);
   static unsigned device_mask = 0;
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(wkv4_bwd_kernel<T>), (int)smem, &device_mask);
   if (e != cudaSuccess) return e;
   const long long nblk = (long long)p.ctiles * p.B;
-  wkv4_bwd_kernel<T><<<(unsigned)nblk, kW * 32, smem, st>>>(mk, mv, mg, p);
+  wkv4_bwd_kernel<T><<<(unsigned)nblk, kW * 32, smem, st>>>(mk, mv, mg, mgk, mgv, p);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 int bwd_tile_steps() { return kTile; }
+
+int bwd_store_steps() { return kL; }
 
 int bwd_stages(bool bf16, int T) {
   const int want = bf16 ? 4 : 2;  // 48 KB of boxes keeps four CTAs per SM
@@ -344,8 +358,9 @@ int bwd_stages(bool bf16, int T) {
 }
 
 cudaError_t launch_wkv4_bwd(bool bf16, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mg,
-                            const Bwd4Params& p, cudaStream_t st) {
-  return bf16 ? launch_bwd_t<__nv_bfloat16>(mk, mv, mg, p, st) : launch_bwd_t<float>(mk, mv, mg, p, st);
+                            const CUtensorMap& mgk, const CUtensorMap& mgv, const Bwd4Params& p, cudaStream_t st) {
+  return bf16 ? launch_bwd_t<__nv_bfloat16>(mk, mv, mg, mgk, mgv, p, st)
+              : launch_bwd_t<float>(mk, mv, mg, mgk, mgv, p, st);
 }
 
 cudaError_t launch_wkv4_reduce_wu(int B, int C, const double* part, float* gw, float* gu, cudaStream_t st) {

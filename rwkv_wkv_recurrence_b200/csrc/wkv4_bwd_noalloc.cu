@@ -82,7 +82,8 @@ extern "C" rwkv_status rwkv_wkv4_backward_noalloc(int64_t B, int64_t T, int64_t 
   if (k == nullptr || v == nullptr || gy == nullptr || ckpt == nullptr || gk == nullptr || gv == nullptr)
     return RWKV_ERR_INVALID_ARG;
   const bool bf16 = dtype == RWKV_BF16;
-  if (!aligned16(k) || !aligned16(v) || !aligned16(gy) || (C * (bf16 ? 2 : 4)) % 16 != 0)
+  if (!aligned16(k) || !aligned16(v) || !aligned16(gy) || !aligned16(gk) || !aligned16(gv) ||
+      (C * (bf16 ? 2 : 4)) % 16 != 0)
     return RWKV_ERR_UNSUPPORTED;
   double* scratch = nullptr;
   if (scratch_for_current_device(&scratch) != cudaSuccess) return RWKV_ERR_CUDA;
@@ -90,9 +91,11 @@ extern "C" rwkv_status rwkv_wkv4_backward_noalloc(int64_t B, int64_t T, int64_t 
   if (err == nullptr) return RWKV_ERR_CUDA;
   const int iB = (int)B, iT = (int)T, iC = (int)C;
   const int box_t = bwd_tile_steps();
-  CUtensorMap mk, mv, mg;
+  CUtensorMap mk, mv, mg, mgk, mgv;
   if (!make_btc_map(&mk, k, bf16, iB, iT, iC, box_t) || !make_btc_map(&mv, v, bf16, iB, iT, iC, box_t) ||
-      !make_btc_map(&mg, gy, bf16, iB, iT, iC, box_t))
+      !make_btc_map(&mg, gy, bf16, iB, iT, iC, box_t) ||
+      !make_btc_map(&mgk, gk, bf16, iB, iT, iC, bwd_store_steps()) ||
+      !make_btc_map(&mgv, gv, bf16, iB, iT, iC, bwd_store_steps()))
     return RWKV_ERR_CUDA;
   Bwd4Params p{};
   p.B = iB;
@@ -107,7 +110,7 @@ extern "C" rwkv_status rwkv_wkv4_backward_noalloc(int64_t B, int64_t T, int64_t 
   p.gv = gv;
   p.part = scratch;  // [2][B*C] within the fixed array
   p.err = err;
-  if (launch_wkv4_bwd(bf16, mk, mv, mg, p, st) != cudaSuccess) return RWKV_ERR_CUDA;
+  if (launch_wkv4_bwd(bf16, mk, mv, mg, mgk, mgv, p, st) != cudaSuccess) return RWKV_ERR_CUDA;
   if (launch_wkv4_reduce_wu(iB, iC, scratch, gw, gu, st) != cudaSuccess) return RWKV_ERR_CUDA;
   return RWKV_OK;
 }
