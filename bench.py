@@ -468,14 +468,60 @@ def run_eagle(args):
         "gpu_launches": args.steps, "clocks": clk}), flush=True)
 
 
+def run_eagle_decode(args):
+    """Eagle / RWKV-5 decode step: 512 streams x 40 heads x 64, fp32 state
+    [512,40,64,64] updated in place, 16 pre-generated bf16 tokens cycled."""
+    import torch
+
+    import rwkv_wkv_recurrence_b200 as rw
+    import wkv_inputs as wi
+
+    _, _, local = _dist()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    Bs, Hs, Ns, Tt = 512, 40, 64, 16
+    q = wi.wkv5_problem(Bs, Tt, Hs, Ns, seed=SEED + 5, device=dev)
+    toks = [{n: q[n][:, t].contiguous() for n in ("r", "k", "v")} for t in range(Tt)]
+    state = torch.zeros(Bs, Hs, Ns, Ns, device=dev)
+    y = torch.empty(Bs, Hs, Ns, dtype=torch.bfloat16, device=dev)
+    h = rw.lib()
+    stream = torch.cuda.current_stream()
+    sp, P = rw._stream(stream), rw._ptr
+
+    def step(i):
+        t = toks[i % Tt]
+        s = h.rwkv_wkv5_step(Bs, Hs, Ns, P(t["r"]), P(t["k"]), P(t["v"]), P(q["omega"]), P(q["u"]), P(y),
+                             P(state), P(state), sp)
+        if s:
+            raise rw.RwkvError("rwkv_wkv5_step", s)
+
+    ms, clk = _timed(step, args.steps, args.warmup, stream, local)
+    heads = Bs * Hs
+    bytes_step = heads * (2 * Ns * Ns * 4 + 4 * Ns * 2) + 2 * Hs * Ns * 4  # state in + out; r, k, v, y; omega, u
+    gbs = bytes_step / (ms * 1e-3) / 1e9
+    peak, kind = _peaks()
+    print(json.dumps({
+        "metric": "Eagle decode head-steps/s and HBM GB/s (512 streams x H40 x N64)",
+        "value": heads / (ms * 1e-3), "unit": "head-steps/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "dtype": "bf16 I/O, fp32 state",
+        "data": "synthetic",
+        "config": {"workload": "Eagle / RWKV-5 decode step, 512 streams x H=40 x N=64, fp32 state in place, "
+                               "16 tokens cycled",
+                   "l2": "no flush: 682 MB moved per step, above the 126 MB L2"},
+        "roofline": {"bound": "hbm", "kernel": "wkv5_step_kernel", "achieved": gbs, "peak": peak,
+                     "peak_kind": kind, "unit": "GB/s", "frac": gbs / peak, "traffic": None},
+        "gpu_launches": args.steps, "clocks": clk}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["train", "decode", "eagle"], default="train",
-                    help="train: the headline forward+backward step; decode, eagle: the other hot-path rows")
+    ap.add_argument("--workload", choices=["train", "decode", "eagle", "eagle_decode"], default="train",
+                    help="train: the headline forward+backward step; decode, eagle, eagle_decode: the other "
+                         "hot-path rows")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--ref-channels", type=int, default=256)
@@ -490,6 +536,8 @@ def main():
         run_decode(args)
     elif args.workload == "eagle":
         run_eagle(args)
+    elif args.workload == "eagle_decode":
+        run_eagle_decode(args)
     else:
         run_ours(args)
 

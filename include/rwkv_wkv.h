@@ -162,6 +162,22 @@ RWKV_API rwkv_status rwkv_wkv5_forward(int64_t B, int64_t T, int64_t H, int64_t 
                               const float *s_in, float *s_out,
                               void *workspace, size_t workspace_bytes, rwkv_stream_t stream);
 
+/*
+ * Eagle / RWKV-5 recurrent decode: one token for each of B independent
+ * streams ("RWKV-5 Eagle과 RWKV-6 Finch", section Eagle): per head,
+ *   y = r·(s + diag(u)·kᵀv),   then   s <- diag(w)·s + kᵀv,  w = exp(-exp(ω)),
+ * which is rwkv_wkv5_forward with T = 1.
+ *   r, k, v, y  [B,H,N] bf16 (the token of every stream and head).
+ *   omega, u    [H,N] fp32.
+ *   s_in        [B,H,N,N] fp32, or NULL (zero state).
+ *   s_out       [B,H,N,N] fp32, required; may equal s_in (in-place update).
+ *   N must be 64 (RWKV_ERR_UNSUPPORTED otherwise); s_in and s_out must be
+ *   16-byte aligned (RWKV_ERR_UNSUPPORTED otherwise).
+ */
+RWKV_API rwkv_status rwkv_wkv5_step(int64_t B, int64_t H, int64_t N, const void *r, const void *k,
+                           const void *v, const float *omega, const float *u, void *y,
+                           const float *s_in, float *s_out, rwkv_stream_t stream);
+
 /* Largest B * C that rwkv_wkv4_backward_noalloc accepts. */
 #define RWKV_NOALLOC_MAX_LANES 262144
 

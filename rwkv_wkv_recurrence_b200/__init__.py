@@ -22,7 +22,7 @@ __all__ = [
     "LIB_PATH", "lib", "RwkvError", "RWKV_OK", "F32", "BF16", "ALGO_AUTO", "ALGO_SEQUENTIAL",
     "ALGO_CHUNKED", "CHUNK_LEN", "NOALLOC_MAX_LANES", "rwkv_wkv4_forward", "rwkv_wkv4_backward",
     "rwkv_wkv4_backward_noalloc", "rwkv_wkv4_step",
-    "rwkv_wkv5_forward", "rwkv_check_device_error", "state_to_ab",
+    "rwkv_wkv5_forward", "rwkv_wkv5_step", "rwkv_check_device_error", "state_to_ab",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "librwkv_wkv.so")
@@ -65,6 +65,7 @@ def lib():
         "rwkv_wkv5_forward_workspace_bytes": ([I64, I64, I64, I64], S),
         "rwkv_wkv5_forward": ([I64, I64, I64, I64, P, P, P, P, P, P, P, P, P, S, P], I),
         "rwkv_wkv4_backward_noalloc": ([I64, I64, I64, I, P, P, P, P, P, P, I64, P, P, P, P, P], I),
+        "rwkv_wkv5_step": ([I64, I64, I64, P, P, P, P, P, P, P, P, P], I),
         "rwkv_check_device_error": ([P], I),
     }
     for name, (args, res) in sig.items():
@@ -240,6 +241,27 @@ def rwkv_wkv5_forward(r, k, v, omega, u, s_in=None, *, return_state=False, strea
            h.rwkv_wkv5_forward(B, T, H, N, _ptr(r), _ptr(k), _ptr(v), _ptr(omega), _ptr(u), _ptr(y),
                                _ptr(s_in), _ptr(so), _ptr(ws), wsb, _stream(stream)))
     return (y, so) if return_state else y
+
+
+def rwkv_wkv5_step(r, k, v, omega, u, state=None, *, state_out=None, stream=None, out=None):
+    """Eagle / RWKV-5 decode step: r, k, v [B,H,N] bf16 (one token per stream);
+    omega, u [H,N] fp32; state [B,H,N,N] fp32 or None (zero).  Returns
+    (y [B,H,N] bf16, new state).  state_out may be `state` (in-place)."""
+    import torch
+
+    _need_cuda(r, k, v, omega, u, state, state_out)
+    B, H, N = r.shape
+    for t in (r, k, v):
+        if t.dtype != torch.bfloat16 or t.shape != r.shape:
+            raise ValueError("r, k, v must be bf16 of the same shape")
+    _f32("omega", omega, H * N)
+    _f32("u", u, H * N)
+    y = torch.empty_like(r) if out is None else out
+    so = state_out if state_out is not None else torch.empty((B, H, N, N), dtype=torch.float32, device=r.device)
+    _check("rwkv_wkv5_step",
+           lib().rwkv_wkv5_step(B, H, N, _ptr(r), _ptr(k), _ptr(v), _ptr(omega), _ptr(u), _ptr(y), _ptr(state),
+                                _ptr(so), _stream(stream)))
+    return y, so
 
 
 def rwkv_check_device_error(stream=None):

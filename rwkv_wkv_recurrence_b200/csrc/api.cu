@@ -363,6 +363,32 @@ rwkv_status rwkv_wkv5_forward(int64_t B, int64_t T, int64_t H, int64_t N, const 
   return RWKV_OK;
 }
 
+rwkv_status rwkv_wkv5_step(int64_t B, int64_t H, int64_t N, const void* r, const void* k, const void* v,
+                           const float* omega, const float* u, void* y, const float* s_in, float* s_out,
+                           rwkv_stream_t stream) {
+  if (!fits_int(B) || !fits_int(H) || !fits_int(N)) return RWKV_ERR_INVALID_ARG;
+  if (N != 64) return RWKV_ERR_UNSUPPORTED;
+  if (B == 0 || H == 0) return RWKV_OK;
+  if (r == nullptr || k == nullptr || v == nullptr || omega == nullptr || u == nullptr || y == nullptr ||
+      s_out == nullptr)
+    return RWKV_ERR_INVALID_ARG;
+  if ((s_in != nullptr && !aligned16(s_in)) || !aligned16(s_out)) return RWKV_ERR_UNSUPPORTED;
+  if ((int64_t)B * H > INT_MAX) return RWKV_ERR_UNSUPPORTED;
+  Wkv5StepParams p{};
+  p.B = (int)B;
+  p.H = (int)H;
+  p.r = static_cast<const __nv_bfloat16*>(r);
+  p.k = static_cast<const __nv_bfloat16*>(k);
+  p.v = static_cast<const __nv_bfloat16*>(v);
+  p.omega = omega;
+  p.u = u;
+  p.y = static_cast<__nv_bfloat16*>(y);
+  p.s_in = s_in;
+  p.s_out = s_out;
+  if (launch_wkv5_step(p, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return RWKV_ERR_CUDA;
+  return RWKV_OK;
+}
+
 rwkv_status rwkv_check_device_error(rwkv_stream_t stream) {
   if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return RWKV_ERR_CUDA;
   unsigned int v = 0;

@@ -41,6 +41,18 @@ struct Bwd4Params {
   unsigned int* err;  // device error word
 };
 
+struct Wkv5StepParams {
+  int B, H;
+  const __nv_bfloat16* r;  // [B,H,64]
+  const __nv_bfloat16* k;
+  const __nv_bfloat16* v;
+  const float* omega;      // [H,64]
+  const float* u;          // [H,64]
+  __nv_bfloat16* y;        // [B,H,64]
+  const float* s_in;       // [B,H,64,64] or null (zero state)
+  float* s_out;            // [B,H,64,64]; may equal s_in
+};
+
 struct Wkv5Params {
   int B, T, H;
   const __nv_bfloat16* r;
@@ -79,6 +91,7 @@ cudaError_t launch_copy_state(int B, int C, const float* state_in, float* state_
 bool make_btc_map(CUtensorMap* m, const void* base, bool bf16, int B, int T, int C, int box_t);
 // Tensor map over a bf16 [B, T, W] tensor with [1, 64, 64] boxes and the 128-byte swizzle.
 bool make_bf16_box64_map(CUtensorMap* m, const void* base, int B, int T, int W);
+cudaError_t launch_wkv5_step(const Wkv5StepParams& p, cudaStream_t st);
 cudaError_t launch_wkv5_fwd(const CUtensorMap& mr, const CUtensorMap& mk, const CUtensorMap& mv, const Wkv5Params& p,
                             cudaStream_t st);
 // Device address of the library's error word on the current device (null on failure).

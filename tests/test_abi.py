@@ -106,6 +106,14 @@ def test_validation_before_any_cuda_work():
                                None) == 2
     assert h.rwkv_wkv5_forward(1, 4, 2, 64, fake, fake, fake, None, fake, fake, None, None, None, 0,
                                None) == 1
+    # WKV-5 decode step: only N = 64, output state required, 16-byte aligned states
+    assert h.rwkv_wkv5_step(2, 3, 32, fake, fake, fake, fake, fake, fake, None, fake, None) == 2
+    assert h.rwkv_wkv5_step(2, 3, 64, fake, fake, fake, fake, fake, fake, None, None, None) == 1
+    assert h.rwkv_wkv5_step(2, 3, 64, fake, None, fake, fake, fake, fake, None, fake, None) == 1
+    assert h.rwkv_wkv5_step(2, 3, 64, fake, fake, fake, fake, fake, fake, None, P(0x1004), None) == 2
+    assert h.rwkv_wkv5_step(2, 3, 64, fake, fake, fake, fake, fake, fake, P(0x1008), fake, None) == 2
+    assert h.rwkv_wkv5_step(-2, 3, 64, fake, fake, fake, fake, fake, fake, None, fake, None) == 1
+    assert h.rwkv_wkv5_step(0, 3, 64, fake, fake, fake, fake, fake, fake, None, fake, None) == 0
 
 
 def test_binding_fails_loudly_without_library(monkeypatch):

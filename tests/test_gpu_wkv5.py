@@ -1,5 +1,5 @@
-"""GPU parity of the Eagle / RWKV-5 matrix-state WKV forward against the fp64
-oracle, through the C-ABI.  bf16 inputs are widened exactly for the oracle.
+"""GPU parity of the Eagle / RWKV-5 matrix-state WKV forward and decode step
+against the fp64 oracle, through the C-ABI.  bf16 inputs are widened exactly for the oracle.
 Tolerance for the bf16 output y and for the fp32 final state alike:
 |got - ref| <= 8e-3 * max(|ref|, rms(ref))."""
 import numpy as np
@@ -66,3 +66,72 @@ def test_eagle_workload_full_size(cuda_device):
                                          p["u"][h:h + 1], return_state=True)
         assert_close_rms(y[b:b + 1, :, h:h + 1], ref, TOL_BF16, f"y head ({b},{h})")
         assert_close_rms(s[b:b + 1, h:h + 1], ref_s, TOL_BF16, f"s head ({b},{h})")
+
+
+# ------------------------------------------------------------------ decode step
+def _token(p, t):
+    return {n: p[n][:, t].contiguous() for n in ("r", "k", "v")}
+
+
+def _prefix_state(p, t0):
+    """The oracle's fp64 state after the first t0 tokens of problem p, as fp32."""
+    _, s = oracle.wkv5_forward(p["r"][:, :t0], p["k"][:, :t0], p["v"][:, :t0], p["omega"], p["u"],
+                               return_state=True)
+    return torch.from_numpy(s).float()
+
+
+def test_step_matches_oracle(cuda_device):
+    B, H, t0 = 3, 5, 20
+    p = wi.wkv5_problem(B, t0 + 1, H, 64, seed=33)
+    s0 = _prefix_state(p, t0)
+    tok = _token(p, t0)
+    y, s1 = rw.rwkv_wkv5_step(**_cuda(tok, cuda_device), omega=p["omega"].to(cuda_device),
+                              u=p["u"].to(cuda_device), state=s0.to(cuda_device))
+    ref, ref_s = oracle.wkv5_forward(tok["r"][:, None], tok["k"][:, None], tok["v"][:, None], p["omega"], p["u"],
+                                     s0.double().numpy(), return_state=True)
+    assert_close_rms(y, ref[:, 0], TOL_BF16, "y")
+    assert_close_rms(s1, ref_s, TOL_BF16, "s_out")
+
+
+@pytest.mark.parametrize("omega_range", [(-6.0, 0.0), (-1.0, 2.0)])
+def test_step_sequence_matches_forward_oracle(cuda_device, omega_range):
+    # T steps from a zero state, state updated in place, against the oracle's forward over the same tokens
+    B, T, H = 2, 40, 3
+    p = wi.wkv5_problem(B, T, H, 64, seed=34, omega_range=omega_range)
+    g = _cuda(p, cuda_device)
+    state = torch.zeros(B, H, 64, 64, device=cuda_device)
+    ys = []
+    for t in range(T):
+        y, _ = rw.rwkv_wkv5_step(**_token(g, t), omega=g["omega"], u=g["u"], state=None if t == 0 else state,
+                                 state_out=state)
+        ys.append(y)
+    ref, ref_s = oracle.wkv5_forward(p["r"], p["k"], p["v"], p["omega"], p["u"], return_state=True)
+    assert_close_rms(torch.stack(ys, 1), ref, TOL_BF16, "y")
+    assert_close_rms(state, ref_s, TOL_BF16, "state")
+
+
+def test_step_in_place_equals_out_of_place(cuda_device):
+    B, H = 4, 6
+    p = wi.wkv5_problem(B, 9, H, 64, seed=35)
+    g = _cuda(p, cuda_device)
+    s0 = _prefix_state(p, 8).to(cuda_device)
+    tok = _token(g, 8)
+    y1, s1 = rw.rwkv_wkv5_step(**tok, omega=g["omega"], u=g["u"], state=s0)
+    s_in_place = s0.clone()
+    y2, s2 = rw.rwkv_wkv5_step(**tok, omega=g["omega"], u=g["u"], state=s_in_place, state_out=s_in_place)
+    assert torch.equal(y1, y2) and torch.equal(s1, s2) and s2.data_ptr() == s_in_place.data_ptr()
+
+
+def test_step_workload_full_size(cuda_device):
+    # the decode bench's shape: 512 streams x 40 heads x 64, one step from a state
+    # reached after 16 tokens; every head checked
+    B, H, t0 = 512, 40, 16
+    p = wi.wkv5_problem(B, t0 + 1, H, 64, seed=SEED + 5)
+    s0 = _prefix_state(p, t0)
+    tok = _token(p, t0)
+    y, s1 = rw.rwkv_wkv5_step(**_cuda(tok, cuda_device), omega=p["omega"].to(cuda_device),
+                              u=p["u"].to(cuda_device), state=s0.to(cuda_device))
+    ref, ref_s = oracle.wkv5_forward(tok["r"][:, None], tok["k"][:, None], tok["v"][:, None], p["omega"], p["u"],
+                                     s0.double().numpy(), return_state=True)
+    assert_close_rms(y, ref[:, 0], TOL_BF16, "y")
+    assert_close_rms(s1, ref_s, TOL_BF16, "s_out")
