@@ -88,6 +88,9 @@ def test_validation_before_any_cuda_work():
                                0, None) == 2
     assert h.rwkv_wkv4_forward(1, 4, 6, 0, fake, fake, fake, fake, fake, None, None, None, 16, 0, None, 0,
                                None) == 2
+    # misaligned y (written by TMA stores)
+    assert h.rwkv_wkv4_forward(1, 4, 4, 0, fake, fake, fake, fake, P(0x1004), None, None, None, 16, 0, None,
+                               0, None) == 2
     # chunked schedule without its workspace
     assert h.rwkv_wkv4_forward(8, 1024, 768, 0, fake, fake, fake, fake, fake, None, None, None, 16, 0, None, 0,
                                None) == 3
@@ -98,6 +101,11 @@ def test_validation_before_any_cuda_work():
                                 fake, None, 0, None) == 3
     assert h.rwkv_wkv4_backward(1, 4, 4, 0, fake, fake, fake, fake, fake, None, fake, 16, None, fake, fake,
                                 fake, fake, 1 << 20, None) == 1
+    # backward: misaligned gk or gv (written by TMA stores)
+    assert h.rwkv_wkv4_backward(1, 4, 4, 0, fake, fake, fake, fake, fake, None, fake, 16, P(0x1004), fake,
+                                fake, fake, fake, 1 << 20, None) == 2
+    assert h.rwkv_wkv4_backward(1, 4, 4, 0, fake, fake, fake, fake, fake, None, fake, 16, fake, P(0x1008),
+                                fake, fake, fake, 1 << 20, None) == 2
     # step: null output state
     assert h.rwkv_wkv4_step(2, 4, 0, fake, fake, fake, fake, fake, None, None, None) == 1
     assert h.rwkv_wkv4_step(-2, 4, 0, fake, fake, fake, fake, fake, None, fake, None) == 1
