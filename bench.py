@@ -102,7 +102,8 @@ class ClockSampler:
 
 
 # kernel name in profiles/traffic.json -> prefix of the source files it is built from
-_TRAFFIC_SOURCES = {"wkv4_bwd_kernel": "wkv4_bwd", "wkv5_fwd_tc_kernel": "wkv5_fwd"}
+_TRAFFIC_SOURCES = {"wkv4_bwd_kernel": "wkv4_bwd", "wkv5_fwd_tc_kernel": "wkv5_fwd", "wkv4_step_kernel": "wkv4_step",
+                    "wkv5_step_kernel": "wkv5_step"}
 
 
 def _kernel_source_hash(kernel="wkv4_bwd_kernel"):
@@ -421,7 +422,8 @@ def run_decode(args):
         "config": {"workload": "RWKV-4 WKV decode, fp32, 4096 streams x C=4096, state in place, 256 tokens cycled",
                    "l2": "no flush: 604 MB moved per step, above the 126 MB L2"},
         "roofline": {"bound": "hbm", "kernel": "wkv4_step_kernel", "achieved": gbs, "peak": peak,
-                     "peak_kind": kind, "unit": "GB/s", "frac": gbs / peak, "traffic": None},
+                     "peak_kind": kind, "unit": "GB/s", "frac": gbs / peak,
+                     "traffic": _recorded_traffic("wkv4_step_kernel")},
         "gpu_launches": args.steps, "clocks": clk}), flush=True)
 
 
@@ -509,7 +511,8 @@ def run_eagle_decode(args):
                                "16 tokens cycled",
                    "l2": "no flush: 682 MB moved per step, above the 126 MB L2"},
         "roofline": {"bound": "hbm", "kernel": "wkv5_step_kernel", "achieved": gbs, "peak": peak,
-                     "peak_kind": kind, "unit": "GB/s", "frac": gbs / peak, "traffic": None},
+                     "peak_kind": kind, "unit": "GB/s", "frac": gbs / peak,
+                     "traffic": _recorded_traffic("wkv5_step_kernel")},
         "gpu_launches": args.steps, "clocks": clk}), flush=True)
 
 
