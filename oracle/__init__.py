@@ -49,6 +49,8 @@ def _load():
             "oracle_wkv4_step": [I, I, P, P, P, P, P, P],
             "oracle_wkv5_forward": [I, I, I, I, P, P, P, P, P, P, P, P],
             "oracle_wkv5_forward_bruteforce": [I, I, I, I, P, P, P, P, P, P],
+            "oracle_wkv6_forward": [I, I, I, I, P, P, P, P, P, P, P, P],
+            "oracle_wkv6_forward_bruteforce": [I, I, I, I, P, P, P, P, P, P],
         }
         for name, args in sigs.items():
             f = getattr(lib, name)
@@ -174,4 +176,29 @@ def wkv5_forward_bruteforce(r, k, v, omega, u):
     y = np.empty((B, T, H, N))
     _check(lib.oracle_wkv5_forward_bruteforce(B, T, H, N, _p(r), _p(k), _p(v), _p(omega), _p(u),
                                               _p(y)), "wkv5_forward_bruteforce")
+    return y
+
+
+def wkv6_forward(r, k, v, omega, u, s_in=None, return_state=False):
+    """Finch / RWKV-6 WKV forward (per-token decay).  r, k, v, omega [B,T,H,N];
+    u [H,N]; s_in [B,H,N,N] or None.  Returns y [B,T,H,N] (and s_out [B,H,N,N])."""
+    lib = _load()
+    r, k, v, omega, u, s0 = map(_f64, (r, k, v, omega, u, s_in))
+    B, T, H, N = r.shape
+    y = np.empty((B, T, H, N))
+    s1 = np.empty((B, H, N, N))
+    _check(lib.oracle_wkv6_forward(B, T, H, N, _p(r), _p(k), _p(v), _p(omega), _p(u), _p(s0),
+                                   _p(y), _p(s1)), "wkv6_forward")
+    return (y, s1) if return_state else y
+
+
+def wkv6_forward_bruteforce(r, k, v, omega, u):
+    """Finch / RWKV-6 WKV forward as an explicit sum over past tokens with the
+    decay products formed term by term, zero state."""
+    lib = _load()
+    r, k, v, omega, u = map(_f64, (r, k, v, omega, u))
+    B, T, H, N = r.shape
+    y = np.empty((B, T, H, N))
+    _check(lib.oracle_wkv6_forward_bruteforce(B, T, H, N, _p(r), _p(k), _p(v), _p(omega), _p(u),
+                                              _p(y)), "wkv6_forward_bruteforce")
     return y

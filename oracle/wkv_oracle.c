@@ -18,6 +18,9 @@
  *  [P3] "RWKV-5 Eagle과 RWKV-6 Finch", section "Eagle: 벡터 기억을 행렬 기억으로
  *       확장": s' = diag(w) s + k^T v, wkv' = s + diag(u) k^T v, w = exp(-exp(ω)),
  *       receptance reads the state like a query.
+ *  [P3] also, section "Finch: recurrence를 입력에 반응시키기": Finch keeps the
+ *       Eagle update and makes the decay data dependent (a per-token decay
+ *       vector, corrected from the input through a LoRA).
  *  [P5] "RWKV-7 \"Goose\" 아키텍처 분석", the per-token state-update pseudo-code:
  *       kv[d,e] = k_d v_e and out_e = Σ_d r_d state[d,e] (rows = key index,
  *       columns = value index).
@@ -36,11 +39,17 @@
  *  - Eagle reads the state before the current token's k^T v is added, and
  *    diag(w), diag(u) scale the key (row) index; w is a multiplicative factor in
  *    (0, 1), unlike RWKV-4's rate.
+ *  - Finch's data-dependent decay is read as omega_t [B, T, H, N], one omega
+ *    per token and channel with w_t = exp(-exp(omega_t)) as in Eagle, and the
+ *    decay of token t multiplies the state when token t's k^T v is added (the
+ *    Eagle update with w replaced by w_t), so token t reads a state in which
+ *    token i < t has been decayed by w_{i+1} ... w_{t-1}.
  *
  * Layouts: WKV-4 k, v, y, gy, gk, gv are [B, T, C] (C fastest); w, u, gw, gu
  * are [C]; the fp64 state is [2, B, C] = (numerator A, denominator B) without
  * any rescaling.  WKV-5 r, k, v, y are [B, T, H, N]; omega, u are [H, N]; the
  * state is [B, H, N, N] with s[b, h, i, j], i = key index, j = value index.
+ * Finch takes the same tensors with omega [B, T, H, N].
  *
  * Every function returns the number of non-finite outputs it produced (0 on
  * a healthy run), so a test can tell an overflow from a mismatch.
@@ -400,6 +409,93 @@ int64_t oracle_wkv5_forward_bruteforce(int64_t B, int64_t T, int64_t H, int64_t 
                         for (int64_t d = 0; d < N; ++d)
                             att += r[IDX4(b, t, h, d)] * exp(-(double)(t - 1 - i) * exp(omega[h * N + d])) *
                                    k[IDX4(b, i, h, d)];
+                        acc += att * v[IDX4(b, i, h, j)];
+                    }
+                    double bonus = 0.0;
+                    for (int64_t d = 0; d < N; ++d)
+                        bonus += r[IDX4(b, t, h, d)] * u[h * N + d] * k[IDX4(b, t, h, d)];
+                    acc += bonus * v[IDX4(b, t, h, j)];
+                    if (!isfinite(acc)) ++bad;
+                    y[IDX4(b, t, h, j)] = acc;
+                }
+            }
+        }
+    }
+    return bad;
+}
+
+/*
+ * Finch / RWKV-6 WKV forward [P3 Finch: the decay of the Eagle update becomes
+ * data dependent, one decay vector per token], per (batch b, head h):
+ *   y_t[j] = Σ_i r_t[i] (s[i][j] + u_i k_t[i] v_t[j]),
+ *   s[i][j] <- w_t[i] s[i][j] + k_t[i] v_t[j],   w_t[i] = exp(-exp(omega_t[i])),
+ * i.e. the Eagle recurrence above with omega [B,T,H,N] read at the current
+ * token; starts from s_in [B,H,N,N] (or zero), s_out receives the final state.
+ */
+int64_t oracle_wkv6_forward(int64_t B, int64_t T, int64_t H, int64_t N,
+                            const double *r, const double *k, const double *v,
+                            const double *omega, const double *u,
+                            const double *s_in, double *y, double *s_out)
+{
+    int64_t bad = 0;
+#pragma omp parallel reduction(+ : bad)
+    {
+        double *s = (double *)malloc((size_t)(N * N) * sizeof(double));
+#pragma omp for collapse(2) schedule(static)
+        for (int64_t b = 0; b < B; ++b) {
+            for (int64_t h = 0; h < H; ++h) {
+                for (int64_t ij = 0; ij < N * N; ++ij)
+                    s[ij] = s_in ? s_in[((b * H + h) * N) * N + ij] : 0.0;
+                for (int64_t t = 0; t < T; ++t) {
+                    for (int64_t j = 0; j < N; ++j) {
+                        double acc = 0.0;
+                        for (int64_t i = 0; i < N; ++i)
+                            acc += r[IDX4(b, t, h, i)] *
+                                   (s[i * N + j] + u[h * N + i] * k[IDX4(b, t, h, i)] * v[IDX4(b, t, h, j)]);
+                        if (!isfinite(acc)) ++bad;
+                        y[IDX4(b, t, h, j)] = acc;
+                    }
+                    for (int64_t i = 0; i < N; ++i) {
+                        const double wt = exp(-exp(omega[IDX4(b, t, h, i)]));
+                        for (int64_t j = 0; j < N; ++j)
+                            s[i * N + j] = wt * s[i * N + j] + k[IDX4(b, t, h, i)] * v[IDX4(b, t, h, j)];
+                    }
+                }
+                if (s_out)
+                    for (int64_t ij = 0; ij < N * N; ++ij) s_out[((b * H + h) * N) * N + ij] = s[ij];
+            }
+        }
+        free(s);
+    }
+    return bad;
+}
+
+/*
+ * Finch / RWKV-6 WKV forward unrolled into its sum over past tokens, zero
+ * initial state: token i's k_i^T v_i enters the state after token i and is
+ * then multiplied by the decay of every later token up to t-1, so
+ *   y_t[j] = Σ_{i<t} Σ_d r_t[d] (Π_{m=i+1}^{t-1} w_m[d]) k_i[d] v_i[j]
+ *          + Σ_d r_t[d] u_d k_t[d] v_t[j],      w_m[d] = exp(-exp(omega_m[d])).
+ * The product is formed term by term (O(T^3 N^2) per head: tiny inputs only).
+ */
+int64_t oracle_wkv6_forward_bruteforce(int64_t B, int64_t T, int64_t H, int64_t N,
+                                       const double *r, const double *k, const double *v,
+                                       const double *omega, const double *u, double *y)
+{
+    int64_t bad = 0;
+#pragma omp parallel for collapse(3) schedule(static) reduction(+ : bad)
+    for (int64_t b = 0; b < B; ++b) {
+        for (int64_t h = 0; h < H; ++h) {
+            for (int64_t t = 0; t < T; ++t) {
+                for (int64_t j = 0; j < N; ++j) {
+                    double acc = 0.0;
+                    for (int64_t i = 0; i < t; ++i) {
+                        double att = 0.0;
+                        for (int64_t d = 0; d < N; ++d) {
+                            double decay = 1.0;
+                            for (int64_t m = i + 1; m < t; ++m) decay *= exp(-exp(omega[IDX4(b, m, h, d)]));
+                            att += r[IDX4(b, t, h, d)] * decay * k[IDX4(b, i, h, d)];
+                        }
                         acc += att * v[IDX4(b, i, h, j)];
                     }
                     double bonus = 0.0;

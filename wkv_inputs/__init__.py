@@ -10,6 +10,10 @@ distributions that the WKV workloads use:
   ``gy ~ N(0, 1)``.
 * Eagle / RWKV-5 WKV: ``r, k, v ~ N(0, 1)/sqrt(N)`` rounded to bf16, per-channel
   ``omega ~ U(-6, 0)`` and ``u ~ U(-1, 1)`` of shape ``[H, N]``.
+* Finch / RWKV-6 WKV: as Eagle, with a per-token decay parameter
+  ``omega[b, t, h, n] = omega0[h, n] + 0.5 * z`` (fp32), a per-channel base
+  ``omega0 ~ U(-6, 0)`` plus an i.i.d. ``z ~ N(0, 1)`` per token: the
+  input-dependent correction of the decay around a learned per-channel value.
 
 Generator.  Every value is a pure function of ``(seed, tensor id, flat
 index)``: the SplitMix64 finaliser (Steele, Lea and Flood, "Fast splittable
@@ -38,6 +42,7 @@ __all__ = [
     "wkv4_params",
     "wkv4_problem",
     "wkv5_problem",
+    "wkv6_problem",
     "CONFIG_SEED_BASE",
 ]
 
@@ -59,6 +64,7 @@ TID = {
     "r": 6,
     "omega": 7,
     "k_outlier": 8,
+    "omega_t": 9,
 }
 
 
@@ -208,4 +214,22 @@ def wkv5_problem(B: int, T: int, H: int, N: int, seed: int, device="cpu",
     lo, hi = omega_range
     out["omega"] = (lo + (hi - lo) * uniform(seed, TID["omega"], hn)).to(torch.float32).view(H, N)
     out["u"] = (-1.0 + 2.0 * uniform(seed, TID["u"], hn)).to(torch.float32).view(H, N)
+    return out
+
+
+def wkv6_problem(B: int, T: int, H: int, N: int, seed: int, device="cpu",
+                 omega_range=(-6.0, 0.0), omega_jitter: float = 0.5) -> dict:
+    """Finch / RWKV-6 WKV inputs: the Eagle inputs of ``wkv5_problem`` with the
+    per-channel ``omega`` [H, N] widened to a per-token ``omega`` [B, T, H, N]
+    fp32: ``omega0[h, n] + omega_jitter * N(0, 1)``."""
+    out = wkv5_problem(B, T, H, N, seed, device=device, omega_range=omega_range)
+    base = out["omega"]
+    n = B * T * H * N
+    om = torch.empty(n, dtype=torch.float32, device=device)
+    blk = 1 << 23
+    for s in range(0, n, blk):
+        ix = torch.arange(s, min(n, s + blk), dtype=torch.int64, device=device)
+        om[s:s + blk] = (base.reshape(-1)[ix % (H * N)].double() +
+                         omega_jitter * normal(seed, TID["omega_t"], ix)).to(torch.float32)
+    out["omega"] = om.view(B, T, H, N)
     return out
