@@ -103,7 +103,8 @@ class ClockSampler:
 
 # kernel name in profiles/traffic.json -> prefix of the source files it is built from
 _TRAFFIC_SOURCES = {"wkv4_bwd_kernel": "wkv4_bwd", "wkv5_fwd_tc_kernel": "wkv5_fwd", "wkv4_step_kernel": "wkv4_step",
-                    "wkv5_step_kernel": "wkv5_step"}
+                    "wkv5_step_kernel": "wkv5_step", "wkv6_fwd_tc_kernel": "wkv6_fwd",
+                    "wkv5_step_kernel/finch": "wkv5_step"}
 
 
 def _kernel_source_hash(kernel="wkv4_bwd_kernel"):
@@ -113,7 +114,7 @@ def _kernel_source_hash(kernel="wkv4_bwd_kernel"):
     csrc = os.path.join(ROOT, "rwkv_wkv_recurrence_b200", "csrc")
     prefix = _TRAFFIC_SOURCES[kernel]
     for f in sorted(os.listdir(csrc)):
-        if f.startswith(prefix) or f in ("wkv_common.cuh", "launch.h"):
+        if f.startswith(prefix) or f.endswith(".cuh") or f == "launch.h":
             with open(os.path.join(csrc, f), "rb") as fh:
                 h.update(fh.read())
     return h.hexdigest()[:16]
@@ -427,8 +428,10 @@ def run_decode(args):
         "gpu_launches": args.steps, "clocks": clk}), flush=True)
 
 
-def run_eagle(args):
-    """Eagle / RWKV-5 forward, B4 T4096 H40 N64 bf16, zero initial state."""
+def run_eagle(args, finch=False):
+    """Eagle / RWKV-5 forward, B4 T4096 H40 N64 bf16, zero initial state; with
+    finch, the Finch / RWKV-6 forward on the same shape with a per-token fp32
+    omega [B,T,H,N]."""
     import torch
 
     import rwkv_wkv_recurrence_b200 as rw
@@ -438,41 +441,57 @@ def run_eagle(args):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     Be, Te, He, Ne = 4, 4096, 40, 64
-    q = wi.wkv5_problem(Be, Te, He, Ne, seed=SEED + 2, device=dev)
+    gen = wi.wkv6_problem if finch else wi.wkv5_problem
+    q = gen(Be, Te, He, Ne, seed=SEED + (4 if finch else 2), device=dev)
     y = torch.empty_like(q["r"])
     s_out = torch.empty(Be, He, Ne, Ne, device=dev)
     h = rw.lib()
     stream = torch.cuda.current_stream()
     sp, P = rw._stream(stream), rw._ptr
-    wsb = int(h.rwkv_wkv5_forward_workspace_bytes(Be, Te, He, Ne))
+    fwd = h.rwkv_wkv6_forward if finch else h.rwkv_wkv5_forward
+    name = "rwkv_wkv6_forward" if finch else "rwkv_wkv5_forward"
+    wsb = int((h.rwkv_wkv6_forward_workspace_bytes if finch else h.rwkv_wkv5_forward_workspace_bytes)(
+        Be, Te, He, Ne))
     ws = torch.empty(max(wsb, 1), dtype=torch.uint8, device=dev)
 
     def call(i):
-        s = h.rwkv_wkv5_forward(Be, Te, He, Ne, P(q["r"]), P(q["k"]), P(q["v"]), P(q["omega"]), P(q["u"]), P(y),
-                                None, P(s_out), P(ws), wsb, sp)
+        s = fwd(Be, Te, He, Ne, P(q["r"]), P(q["k"]), P(q["v"]), P(q["omega"]), P(q["u"]), P(y), None, P(s_out),
+                P(ws), wsb, sp)
         if s:
-            raise rw.RwkvError("rwkv_wkv5_forward", s)
+            raise rw.RwkvError(name, s)
 
     ms, clk = _timed(call, args.steps, args.warmup, stream, local)
     rw.rwkv_check_device_error()
     elems = Be * Te * He * Ne
-    nbytes = 4 * 2 * elems + Be * He * Ne * Ne * 4 + 2 * He * Ne * 4  # r, k, v, y bf16; s_out; omega, u
+    # r, k, v, y bf16; s_out; u (and omega: per token fp32 for Finch, [H,N] fp32 for Eagle)
+    nbytes = 4 * 2 * elems + Be * He * Ne * Ne * 4 + He * Ne * 4 + (4 * elems if finch else He * Ne * 4)
     gbs = nbytes / (ms * 1e-3) / 1e9
     peak, kind = _peaks()
+    if finch:
+        metric = "Finch WKV forward elements/s and HBM GB/s (B4 T4096 H40 N64, per-token decay)"
+        workload = ("Finch / RWKV-6 WKV forward, B=4 T=4096 H=40 N=64, bf16 r,k,v,y, fp32 per-token omega "
+                    "(U(-6,0) per channel + 0.5 N(0,1) per token), fp32 state")
+        l2 = "no flush: 506 MB moved per call, above the 126 MB L2"
+        kernel = "wkv6_fwd_tc_kernel"
+    else:
+        metric = "Eagle WKV forward elements/s and HBM GB/s (B4 T4096 H40 N64)"
+        workload = "Eagle / RWKV-5 WKV forward, B=4 T=4096 H=40 N=64, bf16 r,k,v,y, fp32 state"
+        l2 = "no flush: 338 MB moved per call, above the 126 MB L2"
+        kernel = "wkv5_fwd_tc_kernel"
     print(json.dumps({
-        "metric": "Eagle WKV forward elements/s and HBM GB/s (B4 T4096 H40 N64)", "value": elems / (ms * 1e-3),
+        "metric": metric, "value": elems / (ms * 1e-3),
         "unit": "elements/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "dtype": "bf16 I/O, fp32 state", "data": "synthetic",
-        "config": {"workload": "Eagle / RWKV-5 WKV forward, B=4 T=4096 H=40 N=64, bf16 r,k,v,y, fp32 state",
-                   "l2": "no flush: 338 MB moved per call, above the 126 MB L2"},
-        "roofline": {"bound": "hbm", "kernel": "wkv5 forward", "achieved": gbs, "peak": peak, "peak_kind": kind,
-                     "unit": "GB/s", "frac": gbs / peak, "traffic": _recorded_traffic("wkv5_fwd_tc_kernel")},
+        "config": {"workload": workload, "l2": l2},
+        "roofline": {"bound": "hbm", "kernel": kernel, "achieved": gbs, "peak": peak, "peak_kind": kind,
+                     "unit": "GB/s", "frac": gbs / peak, "traffic": _recorded_traffic(kernel)},
         "gpu_launches": args.steps, "clocks": clk}), flush=True)
 
 
-def run_eagle_decode(args):
+def run_eagle_decode(args, finch=False):
     """Eagle / RWKV-5 decode step: 512 streams x 40 heads x 64, fp32 state
-    [512,40,64,64] updated in place, 16 pre-generated bf16 tokens cycled."""
+    [512,40,64,64] updated in place, 16 pre-generated bf16 tokens cycled; with
+    finch, the Finch / RWKV-6 step with each token's own fp32 omega [512,40,64]."""
     import torch
 
     import rwkv_wkv_recurrence_b200 as rw
@@ -482,8 +501,10 @@ def run_eagle_decode(args):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     Bs, Hs, Ns, Tt = 512, 40, 64, 16
-    q = wi.wkv5_problem(Bs, Tt, Hs, Ns, seed=SEED + 5, device=dev)
-    toks = [{n: q[n][:, t].contiguous() for n in ("r", "k", "v")} for t in range(Tt)]
+    gen = wi.wkv6_problem if finch else wi.wkv5_problem
+    q = gen(Bs, Tt, Hs, Ns, seed=SEED + (7 if finch else 5), device=dev)
+    names = ("r", "k", "v", "omega") if finch else ("r", "k", "v")
+    toks = [{n: q[n][:, t].contiguous() for n in names} for t in range(Tt)]
     state = torch.zeros(Bs, Hs, Ns, Ns, device=dev)
     y = torch.empty(Bs, Hs, Ns, dtype=torch.bfloat16, device=dev)
     h = rw.lib()
@@ -492,27 +513,33 @@ def run_eagle_decode(args):
 
     def step(i):
         t = toks[i % Tt]
-        s = h.rwkv_wkv5_step(Bs, Hs, Ns, P(t["r"]), P(t["k"]), P(t["v"]), P(q["omega"]), P(q["u"]), P(y),
-                             P(state), P(state), sp)
+        if finch:
+            s = h.rwkv_wkv6_step(Bs, Hs, Ns, P(t["r"]), P(t["k"]), P(t["v"]), P(t["omega"]), P(q["u"]), P(y),
+                                 P(state), P(state), sp)
+        else:
+            s = h.rwkv_wkv5_step(Bs, Hs, Ns, P(t["r"]), P(t["k"]), P(t["v"]), P(q["omega"]), P(q["u"]), P(y),
+                                 P(state), P(state), sp)
         if s:
-            raise rw.RwkvError("rwkv_wkv5_step", s)
+            raise rw.RwkvError("rwkv_wkv6_step" if finch else "rwkv_wkv5_step", s)
 
     ms, clk = _timed(step, args.steps, args.warmup, stream, local)
     heads = Bs * Hs
-    bytes_step = heads * (2 * Ns * Ns * 4 + 4 * Ns * 2) + 2 * Hs * Ns * 4  # state in + out; r, k, v, y; omega, u
+    # state in + out; r, k, v, y bf16; u (and omega: per stream for Finch, per head for Eagle)
+    bytes_step = heads * (2 * Ns * Ns * 4 + 4 * Ns * 2) + Hs * Ns * 4 + (heads * Ns * 4 if finch else Hs * Ns * 4)
     gbs = bytes_step / (ms * 1e-3) / 1e9
     peak, kind = _peaks()
+    tag = "Finch" if finch else "Eagle"
     print(json.dumps({
-        "metric": "Eagle decode head-steps/s and HBM GB/s (512 streams x H40 x N64)",
+        "metric": f"{tag} decode head-steps/s and HBM GB/s (512 streams x H40 x N64)",
         "value": heads / (ms * 1e-3), "unit": "head-steps/s", "n_gpus": 1, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "dtype": "bf16 I/O, fp32 state",
         "data": "synthetic",
-        "config": {"workload": "Eagle / RWKV-5 decode step, 512 streams x H=40 x N=64, fp32 state in place, "
-                               "16 tokens cycled",
-                   "l2": "no flush: 682 MB moved per step, above the 126 MB L2"},
+        "config": {"workload": (f"{tag} / RWKV-{6 if finch else 5} decode step, 512 streams x H=40 x N=64, fp32 "
+                                f"state in place, 16 tokens cycled" + (", per-token fp32 omega" if finch else "")),
+                   "l2": f"no flush: {bytes_step / 1e6:.0f} MB moved per step, above the 126 MB L2"},
         "roofline": {"bound": "hbm", "kernel": "wkv5_step_kernel", "achieved": gbs, "peak": peak,
                      "peak_kind": kind, "unit": "GB/s", "frac": gbs / peak,
-                     "traffic": _recorded_traffic("wkv5_step_kernel")},
+                     "traffic": _recorded_traffic("wkv5_step_kernel/finch" if finch else "wkv5_step_kernel")},
         "gpu_launches": args.steps, "clocks": clk}), flush=True)
 
 
@@ -522,9 +549,10 @@ def main():
     ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["train", "decode", "eagle", "eagle_decode"], default="train",
-                    help="train: the headline forward+backward step; decode, eagle, eagle_decode: the other "
-                         "hot-path rows")
+    ap.add_argument("--workload", choices=["train", "decode", "eagle", "eagle_decode", "finch", "finch_decode"],
+                    default="train",
+                    help="train: the headline forward+backward step; decode, eagle, eagle_decode, finch, "
+                         "finch_decode: the other hot-path rows")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--ref-channels", type=int, default=256)
@@ -541,6 +569,10 @@ def main():
         run_eagle(args)
     elif args.workload == "eagle_decode":
         run_eagle_decode(args)
+    elif args.workload == "finch":
+        run_eagle(args, finch=True)
+    elif args.workload == "finch_decode":
+        run_eagle_decode(args, finch=True)
     else:
         run_ours(args)
 

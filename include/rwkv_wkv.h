@@ -18,6 +18,10 @@
  *     y_t = r_t · (s + diag(u) k_tᵀ v_t),   s ← diag(w) s + k_tᵀ v_t,
  *     w = exp(-exp(ω)),  s[i][j] with i = key index (row), j = value index.
  *
+ *   Finch / RWKV-6 (same page, section Finch): the Eagle update with a
+ *   data-dependent decay, w_t = exp(-exp(ω_t)) for every token t:
+ *     y_t = r_t · (s + diag(u) k_tᵀ v_t),   s ← diag(w_t) s + k_tᵀ v_t.
+ *
  * Conventions for every call
  *   - All tensor arguments are DEVICE pointers owned by the caller, on the
  *     current CUDA device; the library never allocates, frees or keeps them.
@@ -27,6 +31,7 @@
  *   - Layouts are dense row-major: WKV-4 k, v, y, gy, gk, gv are [B, T, C]
  *     (C fastest); w, u, gw, gu are [C] fp32.  WKV-5 r, k, v, y are
  *     [B, T, H, N] bf16; omega, u are [H, N] fp32; s is [B, H, N, N] fp32.
+ *     Finch takes the same with omega [B, T, H, N] fp32 (step: [B, H, N]).
  *   - `w` (WKV-4) is the positive decay RATE of the formula above (the raw
  *     parameter mapped through -exp(.) by the model), not a factor.
  *   - WKV-4 state: [3, B, C] fp32 planes (a, b, p) meaning A = a·2^p,
@@ -40,8 +45,9 @@
  *     Zero-sized problems are a successful no-op (T = 0 copies the state).
  *   - Values are data: no range validation; NaN and Inf propagate.
  *   - Alignment: the WKV-4 [B,T,C] tensors k, v, y, gy, gk, gv (and the WKV-5
- *     tensors r, k, v, y) must be 16-byte aligned with C·sizeof(element) a
- *     multiple of 16 (TMA row pitch), else RWKV_ERR_UNSUPPORTED.
+ *     tensors r, k, v, y, and Finch's omega) must be 16-byte aligned with
+ *     C·sizeof(element) a multiple of 16 (TMA row pitch), else
+ *     RWKV_ERR_UNSUPPORTED.
  */
 #ifndef RWKV_WKV_H
 #define RWKV_WKV_H
@@ -175,6 +181,44 @@ RWKV_API rwkv_status rwkv_wkv5_forward(int64_t B, int64_t T, int64_t H, int64_t 
  *   16-byte aligned (RWKV_ERR_UNSUPPORTED otherwise).
  */
 RWKV_API rwkv_status rwkv_wkv5_step(int64_t B, int64_t H, int64_t N, const void *r, const void *k,
+                           const void *v, const float *omega, const float *u, void *y,
+                           const float *s_in, float *s_out, rwkv_stream_t stream);
+
+/* Workspace bytes rwkv_wkv6_forward needs (0 if none). */
+RWKV_API size_t rwkv_wkv6_forward_workspace_bytes(int64_t B, int64_t T, int64_t H, int64_t N);
+
+/*
+ * Finch / RWKV-6 multi-head matrix-state WKV forward with a per-token decay
+ * ("RWKV-5 Eagle과 RWKV-6 Finch", section Finch: Eagle's recurrence with the
+ * decay made data dependent).  Per head, for t = 0 .. T-1:
+ *   y_t = r_t · (s + diag(u) k_tᵀ v_t),   then   s <- diag(w_t) s + k_tᵀ v_t,
+ *   w_t = exp(-exp(omega_t)),
+ * so token i < t reaches token t decayed by w_{i+1} ⋯ w_{t-1}.
+ *   r, k, v   [B,T,H,N] bf16, read.      y [B,T,H,N] bf16, written.
+ *   omega     [B,T,H,N] fp32 (one value per token and channel), read.
+ *   u         [H,N] fp32.
+ *   s_in      [B,H,N,N] fp32 or NULL (zero).  s_out [B,H,N,N] fp32 or NULL;
+ *             may equal s_in.
+ *   N must be 64 (RWKV_ERR_UNSUPPORTED otherwise); omega follows the
+ *   alignment rule of the [B,T,.] tensors.
+ */
+RWKV_API rwkv_status rwkv_wkv6_forward(int64_t B, int64_t T, int64_t H, int64_t N,
+                              const void *r, const void *k, const void *v,
+                              const float *omega, const float *u, void *y,
+                              const float *s_in, float *s_out,
+                              void *workspace, size_t workspace_bytes, rwkv_stream_t stream);
+
+/*
+ * Finch / RWKV-6 recurrent decode: one token for each of B independent
+ * streams, rwkv_wkv6_forward with T = 1.
+ *   r, k, v, y  [B,H,N] bf16.   omega [B,H,N] fp32 (this token's decay).
+ *   u           [H,N] fp32.
+ *   s_in        [B,H,N,N] fp32, or NULL (zero state).
+ *   s_out       [B,H,N,N] fp32, required; may equal s_in (in-place update).
+ *   N must be 64; s_in and s_out must be 16-byte aligned
+ *   (RWKV_ERR_UNSUPPORTED otherwise).
+ */
+RWKV_API rwkv_status rwkv_wkv6_step(int64_t B, int64_t H, int64_t N, const void *r, const void *k,
                            const void *v, const float *omega, const float *u, void *y,
                            const float *s_in, float *s_out, rwkv_stream_t stream);
 

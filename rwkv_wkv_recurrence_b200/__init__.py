@@ -22,7 +22,8 @@ __all__ = [
     "LIB_PATH", "lib", "RwkvError", "RWKV_OK", "F32", "BF16", "ALGO_AUTO", "ALGO_SEQUENTIAL",
     "ALGO_CHUNKED", "CHUNK_LEN", "NOALLOC_MAX_LANES", "rwkv_wkv4_forward", "rwkv_wkv4_backward",
     "rwkv_wkv4_backward_noalloc", "rwkv_wkv4_step",
-    "rwkv_wkv5_forward", "rwkv_wkv5_step", "rwkv_check_device_error", "state_to_ab",
+    "rwkv_wkv5_forward", "rwkv_wkv5_step", "rwkv_wkv6_forward", "rwkv_wkv6_step", "rwkv_check_device_error",
+    "state_to_ab",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "librwkv_wkv.so")
@@ -66,6 +67,9 @@ def lib():
         "rwkv_wkv5_forward": ([I64, I64, I64, I64, P, P, P, P, P, P, P, P, P, S, P], I),
         "rwkv_wkv4_backward_noalloc": ([I64, I64, I64, I, P, P, P, P, P, P, I64, P, P, P, P, P], I),
         "rwkv_wkv5_step": ([I64, I64, I64, P, P, P, P, P, P, P, P, P], I),
+        "rwkv_wkv6_forward_workspace_bytes": ([I64, I64, I64, I64], S),
+        "rwkv_wkv6_forward": ([I64, I64, I64, I64, P, P, P, P, P, P, P, P, P, S, P], I),
+        "rwkv_wkv6_step": ([I64, I64, I64, P, P, P, P, P, P, P, P, P], I),
         "rwkv_check_device_error": ([P], I),
     }
     for name, (args, res) in sig.items():
@@ -260,6 +264,52 @@ def rwkv_wkv5_step(r, k, v, omega, u, state=None, *, state_out=None, stream=None
     so = state_out if state_out is not None else torch.empty((B, H, N, N), dtype=torch.float32, device=r.device)
     _check("rwkv_wkv5_step",
            lib().rwkv_wkv5_step(B, H, N, _ptr(r), _ptr(k), _ptr(v), _ptr(omega), _ptr(u), _ptr(y), _ptr(state),
+                                _ptr(so), _stream(stream)))
+    return y, so
+
+
+# ------------------------------------------------------------------ WKV-6
+def rwkv_wkv6_forward(r, k, v, omega, u, s_in=None, *, return_state=False, stream=None, out=None):
+    """Finch / RWKV-6 forward (per-token decay): r, k, v [B,T,H,N] bf16;
+    omega [B,T,H,N] fp32; u [H,N] fp32; s_in [B,H,N,N] fp32 or None."""
+    import torch
+
+    _need_cuda(r, k, v, omega, u, s_in)
+    B, T, H, N = r.shape
+    for t in (r, k, v):
+        if t.dtype != torch.bfloat16 or t.shape != r.shape:
+            raise ValueError("r, k, v must be bf16 of the same shape")
+    if omega.dtype != torch.float32 or omega.shape != r.shape or not omega.is_contiguous():
+        raise ValueError("omega must be a contiguous float32 tensor shaped like r")
+    _f32("u", u, H * N)
+    h = lib()
+    y = torch.empty_like(r) if out is None else out
+    so = torch.empty((B, H, N, N), dtype=torch.float32, device=r.device) if return_state else None
+    wsb = int(h.rwkv_wkv6_forward_workspace_bytes(B, T, H, N))
+    ws = torch.empty(wsb, dtype=torch.uint8, device=r.device) if wsb else None
+    _check("rwkv_wkv6_forward",
+           h.rwkv_wkv6_forward(B, T, H, N, _ptr(r), _ptr(k), _ptr(v), _ptr(omega), _ptr(u), _ptr(y),
+                               _ptr(s_in), _ptr(so), _ptr(ws), wsb, _stream(stream)))
+    return (y, so) if return_state else y
+
+
+def rwkv_wkv6_step(r, k, v, omega, u, state=None, *, state_out=None, stream=None, out=None):
+    """Finch / RWKV-6 decode step: r, k, v [B,H,N] bf16 and omega [B,H,N] fp32
+    (one token per stream); u [H,N] fp32; state [B,H,N,N] fp32 or None (zero).
+    Returns (y [B,H,N] bf16, new state).  state_out may be `state` (in-place)."""
+    import torch
+
+    _need_cuda(r, k, v, omega, u, state, state_out)
+    B, H, N = r.shape
+    for t in (r, k, v):
+        if t.dtype != torch.bfloat16 or t.shape != r.shape:
+            raise ValueError("r, k, v must be bf16 of the same shape")
+    _f32("omega", omega, B * H * N)
+    _f32("u", u, H * N)
+    y = torch.empty_like(r) if out is None else out
+    so = state_out if state_out is not None else torch.empty((B, H, N, N), dtype=torch.float32, device=r.device)
+    _check("rwkv_wkv6_step",
+           lib().rwkv_wkv6_step(B, H, N, _ptr(r), _ptr(k), _ptr(v), _ptr(omega), _ptr(u), _ptr(y), _ptr(state),
                                 _ptr(so), _stream(stream)))
     return y, so
 

@@ -17,7 +17,7 @@ CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "librwkv_wkv.so")
 HEADER = os.path.join(ROOT, "include", "rwkv_wkv.h")
 
-SOURCES = ["api.cu", "wkv4_fwd.cu", "wkv4_bwd.cu", "wkv4_bwd_noalloc.cu", "wkv4_step.cu", "wkv5_fwd.cu",
+SOURCES = ["api.cu", "wkv4_fwd.cu", "wkv4_bwd.cu", "wkv4_bwd_noalloc.cu", "wkv4_step.cu", "wkv5_fwd.cu", "wkv6_fwd.cu",
            "wkv5_step.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

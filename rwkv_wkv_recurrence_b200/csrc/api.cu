@@ -59,6 +59,20 @@ bool make_bf16_box64_map(CUtensorMap* m, const void* base, int B, int T, int W) 
   return r == CUDA_SUCCESS;
 }
 
+bool make_f32_box32_map(CUtensorMap* m, const void* base, int B, int T, int W) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)W, (cuuint64_t)T, (cuuint64_t)B};
+  cuuint64_t strides[2] = {(cuuint64_t)W * 4, (cuuint64_t)W * T * 4};
+  cuuint32_t box[3] = {32u, 64u, 1u};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  std::memset(m, 0, sizeof(*m));
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 unsigned int* device_error_word() {
   unsigned int* p = nullptr;
   if (cudaGetSymbolAddress(reinterpret_cast<void**>(&p), g_device_error) != cudaSuccess) return nullptr;
@@ -184,7 +198,7 @@ const char* rwkv_status_string(rwkv_status s) {
   return "unknown status";
 }
 
-int rwkv_version(void) { return (1 << 16) | 0; }
+int rwkv_version(void) { return (1 << 16) | 1; }
 
 int64_t rwkv_wkv4_num_checkpoints(int64_t T, int64_t chunk_len) {
   if (chunk_len <= 0 || chunk_len % 16 != 0 || T < 0) return -1;
@@ -381,6 +395,89 @@ rwkv_status rwkv_wkv5_step(int64_t B, int64_t H, int64_t N, const void* r, const
   p.k = static_cast<const __nv_bfloat16*>(k);
   p.v = static_cast<const __nv_bfloat16*>(v);
   p.omega = omega;
+  p.omega_per_stream = 0;
+  p.u = u;
+  p.y = static_cast<__nv_bfloat16*>(y);
+  p.s_in = s_in;
+  p.s_out = s_out;
+  if (launch_wkv5_step(p, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return RWKV_ERR_CUDA;
+  return RWKV_OK;
+}
+
+size_t rwkv_wkv6_forward_workspace_bytes(int64_t B, int64_t T, int64_t H, int64_t N) {
+  (void)B;
+  (void)T;
+  (void)H;
+  (void)N;
+  return 0;
+}
+
+rwkv_status rwkv_wkv6_forward(int64_t B, int64_t T, int64_t H, int64_t N, const void* r, const void* k,
+                              const void* v, const float* omega, const float* u, void* y, const float* s_in,
+                              float* s_out, void* workspace, size_t workspace_bytes, rwkv_stream_t stream) {
+  (void)workspace;
+  (void)workspace_bytes;
+  if (!fits_int(B) || !fits_int(T) || !fits_int(H) || !fits_int(N)) return RWKV_ERR_INVALID_ARG;
+  if (N != 64) return RWKV_ERR_UNSUPPORTED;
+  if (B == 0 || H == 0) return RWKV_OK;
+  if (u == nullptr) return RWKV_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (T == 0) {  // no tokens: the state passes through
+    if (s_out != nullptr && s_out != s_in) {
+      const size_t n = (size_t)B * H * 64 * 64 * sizeof(float);
+      cudaError_t e = s_in ? cudaMemcpyAsync(s_out, s_in, n, cudaMemcpyDeviceToDevice, st)
+                           : cudaMemsetAsync(s_out, 0, n, st);
+      if (e != cudaSuccess) return RWKV_ERR_CUDA;
+    }
+    return RWKV_OK;
+  }
+  if (r == nullptr || k == nullptr || v == nullptr || omega == nullptr || y == nullptr) return RWKV_ERR_INVALID_ARG;
+  if (!aligned16(r) || !aligned16(k) || !aligned16(v) || !aligned16(y) || !aligned16(omega))
+    return RWKV_ERR_UNSUPPORTED;
+  if ((int64_t)H * 64 > INT_MAX || (int64_t)B * H > INT_MAX) return RWKV_ERR_UNSUPPORTED;
+  unsigned int* err = device_error_word();
+  if (err == nullptr) return RWKV_ERR_CUDA;
+  const int iB = (int)B, iT = (int)T, iH = (int)H;
+  CUtensorMap mr, mk, mv, mw;
+  if (!make_bf16_box64_map(&mr, r, iB, iT, iH * 64) || !make_bf16_box64_map(&mk, k, iB, iT, iH * 64) ||
+      !make_bf16_box64_map(&mv, v, iB, iT, iH * 64) || !make_f32_box32_map(&mw, omega, iB, iT, iH * 64))
+    return RWKV_ERR_CUDA;
+  Wkv6Params p{};
+  p.B = iB;
+  p.T = iT;
+  p.H = iH;
+  p.r = static_cast<const __nv_bfloat16*>(r);
+  p.k = static_cast<const __nv_bfloat16*>(k);
+  p.v = static_cast<const __nv_bfloat16*>(v);
+  p.omega = omega;
+  p.u = u;
+  p.y = static_cast<__nv_bfloat16*>(y);
+  p.s_in = s_in;
+  p.s_out = s_out;
+  p.err = err;
+  if (launch_wkv6_fwd(mr, mk, mv, mw, p, st) != cudaSuccess) return RWKV_ERR_CUDA;
+  return RWKV_OK;
+}
+
+rwkv_status rwkv_wkv6_step(int64_t B, int64_t H, int64_t N, const void* r, const void* k, const void* v,
+                           const float* omega, const float* u, void* y, const float* s_in, float* s_out,
+                           rwkv_stream_t stream) {
+  if (!fits_int(B) || !fits_int(H) || !fits_int(N)) return RWKV_ERR_INVALID_ARG;
+  if (N != 64) return RWKV_ERR_UNSUPPORTED;
+  if (B == 0 || H == 0) return RWKV_OK;
+  if (r == nullptr || k == nullptr || v == nullptr || omega == nullptr || u == nullptr || y == nullptr ||
+      s_out == nullptr)
+    return RWKV_ERR_INVALID_ARG;
+  if ((s_in != nullptr && !aligned16(s_in)) || !aligned16(s_out)) return RWKV_ERR_UNSUPPORTED;
+  if ((int64_t)B * H > INT_MAX) return RWKV_ERR_UNSUPPORTED;
+  Wkv5StepParams p{};
+  p.B = (int)B;
+  p.H = (int)H;
+  p.r = static_cast<const __nv_bfloat16*>(r);
+  p.k = static_cast<const __nv_bfloat16*>(k);
+  p.v = static_cast<const __nv_bfloat16*>(v);
+  p.omega = omega;
+  p.omega_per_stream = 1;
   p.u = u;
   p.y = static_cast<__nv_bfloat16*>(y);
   p.s_in = s_in;

@@ -46,7 +46,8 @@ struct Wkv5StepParams {
   const __nv_bfloat16* r;  // [B,H,64]
   const __nv_bfloat16* k;
   const __nv_bfloat16* v;
-  const float* omega;      // [H,64]
+  const float* omega;      // [H,64], or [B,H,64] when omega_per_stream
+  int omega_per_stream;    // 1: one decay per stream and head (Finch), 0: per head (Eagle)
   const float* u;          // [H,64]
   __nv_bfloat16* y;        // [B,H,64]
   const float* s_in;       // [B,H,64,64] or null (zero state)
@@ -59,6 +60,19 @@ struct Wkv5Params {
   const __nv_bfloat16* k;
   const __nv_bfloat16* v;
   const float* omega;   // [H,64]
+  const float* u;       // [H,64]
+  __nv_bfloat16* y;
+  const float* s_in;    // [B,H,64,64] or null
+  float* s_out;         // [B,H,64,64] or null
+  unsigned int* err;
+};
+
+struct Wkv6Params {
+  int B, T, H;
+  const __nv_bfloat16* r;
+  const __nv_bfloat16* k;
+  const __nv_bfloat16* v;
+  const float* omega;   // [B,T,H,64]: one decay per token and channel
   const float* u;       // [H,64]
   __nv_bfloat16* y;
   const float* s_in;    // [B,H,64,64] or null
@@ -94,6 +108,11 @@ bool make_bf16_box64_map(CUtensorMap* m, const void* base, int B, int T, int W);
 cudaError_t launch_wkv5_step(const Wkv5StepParams& p, cudaStream_t st);
 cudaError_t launch_wkv5_fwd(const CUtensorMap& mr, const CUtensorMap& mk, const CUtensorMap& mv, const Wkv5Params& p,
                             cudaStream_t st);
+// mw: [1, 64, 32] fp32 boxes (128-byte swizzle) over omega [B, T, H*64].
+cudaError_t launch_wkv6_fwd(const CUtensorMap& mr, const CUtensorMap& mk, const CUtensorMap& mv,
+                            const CUtensorMap& mw, const Wkv6Params& p, cudaStream_t st);
+// Tensor map over an fp32 [B, T, W] tensor with [1, 64, 32] boxes and the 128-byte swizzle.
+bool make_f32_box32_map(CUtensorMap* m, const void* base, int B, int T, int W);
 // Device address of the library's error word on the current device (null on failure).
 unsigned int* device_error_word();
 

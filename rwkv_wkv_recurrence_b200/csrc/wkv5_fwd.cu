@@ -46,10 +46,13 @@
 #include <cstddef>
 
 #include "launch.h"
+#include "tc_common.cuh"
 #include "wkv_common.cuh"
 
 namespace rwkv {
 namespace {
+
+using namespace tc;
 
 constexpr int kN = 64;                 // head size
 constexpr int kL = 64;                 // tokens per chunk
@@ -57,134 +60,6 @@ constexpr int kThreads = 256;
 constexpr uint32_t kRawBytes = kL * kN * 2;    // one bf16 [64 x 64] box
 constexpr float kMaxRate = 2.5f;       // largest -λ the chunked factorization accepts
 constexpr uint32_t kTmemCols = 256;  // [scores | output rows], state increment, k̃ᵀ (64 columns each)
-
-// --------------------------------------------------------------- tcgen05 PTX
-__device__ __forceinline__ void tmem_alloc(uint32_t* dst, uint32_t ncols) {
-  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst)),
-               "r"(ncols)
-               : "memory");
-  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-}
-
-__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
-  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
-}
-
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-
-// D[tmem] (+)= A[smem] * B[smem]ᵀ, both K-major, kind::tf32.
-__device__ __forceinline__ void umma_tf32(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                          uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0), "r"(0), "r"(0), "r"(0)
-      : "memory");
-}
-
-__device__ __forceinline__ void umma_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
-               : "memory");
-}
-
-// 16 lanes x 256 bits, 4 repetitions (32 columns).  Register 4 i + 2 r + e of
-// thread t goes to lane (base + t/4 + 8 r), column (base + 8 i + 2 (t%4) + e).
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.16x256b.x4.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
-          taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
-      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
-      : "memory");
-  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-}
-
-// 16 lanes x 128 bits, 8 repetitions (32 columns).  Register 2 q + r of
-// thread t holds lane (base + t/4 + 8 r), column (base + 4 q + t%4).
-__device__ __forceinline__ void tmem_ld16x128(uint32_t taddr, float (&v)[16]) {
-  uint32_t r[16];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.16x128b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr)
-      : "memory");
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
-}
-
-// 32 lanes x 32 bits x 32 columns: thread t gets lane (base + t), 32 consecutive columns.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
-  uint32_t r[32];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,"
-      "%28,%29,%30,%31}, [%32];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr)
-      : "memory");
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-}
-
-__device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
-  uint32_t v;
-  asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
-  return v;
-}
-
-// D[tmem] (+)= A[tmem] * B[smem]ᵀ, kind::tf32 (A rows in the accumulator layout).
-__device__ __forceinline__ void umma_tf32_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                             uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, {%5, %6, %7, %8}, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0), "r"(0), "r"(0), "r"(0)
-      : "memory");
-}
-
-// Four 8x8 bf16 matrices from shared memory, transposed (row addresses from lanes
-// 8m..8m+7): register m of thread t holds rows 2 (t%4), +1 of column t/4 of matrix m.
-__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&q)[4]) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(q[0]), "=r"(q[1]), "=r"(q[2]), "=r"(q[3])
-               : "r"(addr)
-               : "memory");
-}
-
-// Two packed bf16 (low half first) to fp32.
-__device__ __forceinline__ float2 bf2_to_f2(uint32_t x) {
-  return make_float2(__uint_as_float(x << 16), __uint_as_float(x & 0xFFFF0000u));
-}
-
-// Shared-memory matrix descriptor, K-major without swizzle: core matrices of
-// 8 rows x 16 bytes, K-adjacent core matrices lbo bytes apart, 8-row groups
-// sbo bytes apart.
-__device__ __forceinline__ uint64_t smem_desc(const void* p, uint32_t lbo, uint32_t sbo) {
-  const uint64_t addr = smem_u32(p);
-  return ((addr >> 4) & 0x3FFFull) | ((uint64_t)((lbo >> 4) & 0x3FFF) << 16) |
-         ((uint64_t)((sbo >> 4) & 0x3FFF) << 32) | (1ull << 46);
-}
-
-// Instruction descriptor: kind::tf32, fp32 accumulator, A and B K-major, M = 64, N = 64.
-constexpr uint32_t kIdesc = (1u << 4) | (2u << 7) | (2u << 10) | ((64u >> 3) << 17) | ((64u >> 4) << 24);
-
-// Float offset of element (row, k) of a [64 x 64] tf32 operand in the
-// K-major core-matrix layout: core matrix (row/8, k/4) is 32 floats, rows of
-// a core matrix 4 floats apart; 16 core matrices per 8-row group.
-__device__ __forceinline__ int op_off(int row, int k) {
-  return (((row >> 3) * 16 + (k >> 2)) << 5) + ((row & 7) << 2) + (k & 3);
-}
-constexpr uint32_t kLbo = 128;       // next 4 k (16 bytes of tf32) in the same rows
-constexpr uint32_t kSbo = 16 * 128;  // next 8 rows
 
 // The recurrence for one head (used when a channel decays too fast for the
 // chunked factorization): thread j < 64 owns value column j of the state.
@@ -246,9 +121,6 @@ struct Wkv5Smem {
 };
 static_assert(offsetof(Wkv5Smem, opS) == offsetof(Wkv5Smem, opK) + 64 * 64 * sizeof(float),
               "the first product reads k̃ and e^{32λ} Sᵀ as one 128-row operand");
-
-// kind::tf32, fp32 accumulator, K-major A and B, M = 64, N = 128.
-constexpr uint32_t kIdesc128 = (kIdesc & ~(0x3Fu << 17)) | ((128u >> 3) << 17);
 
 __global__ void __launch_bounds__(kThreads, 2) wkv5_fwd_tc_kernel(const __grid_constant__ CUtensorMap mr,
                                                                   const __grid_constant__ CUtensorMap mk,

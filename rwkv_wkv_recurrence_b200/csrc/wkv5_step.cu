@@ -5,7 +5,9 @@
 // indexed (key i, value j),
 //   y_j   = Σ_i r_i (s_ij + u_i k_i v_j) = Σ_i r_i s_ij + (Σ_i r_i u_i k_i) v_j,
 //   s'_ij = w_i s_ij + k_i v_j,   w_i = exp(-exp(ω_i)),
-// the one-token case of the forward.
+// the one-token case of the forward.  The same kernel is the Finch / RWKV-6
+// decode step (section Finch: the decay becomes data dependent), where ω is
+// one [H, N] vector per stream, the current token's.
 //
 // The step is a pass over the fp32 state (16 KB per head, read once and
 // written once); everything else is 64-element vectors.  One CTA of 256
@@ -37,7 +39,7 @@ __global__ void __launch_bounds__(kThreads) wkv5_step_kernel(Wkv5StepParams p) {
     sr[tid] = __bfloat162float(p.r[tok + tid]);
     sk[tid] = __bfloat162float(p.k[tok + tid]);
     sv[tid] = __bfloat162float(p.v[tok + tid]);
-    sw[tid] = expf(-expf(p.omega[h * kN + tid]));
+    sw[tid] = expf(-expf(p.omega[(p.omega_per_stream ? tok : (size_t)h * kN) + tid]));
   }
   __syncthreads();
   if (tid < 32) {  // Σ_i r_i u_i k_i

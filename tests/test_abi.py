@@ -24,7 +24,7 @@ def _declared():
 
 def test_library_exports_every_declared_symbol():
     names = _declared()
-    assert "rwkv_wkv4_forward" in names and "rwkv_wkv5_forward" in names
+    assert "rwkv_wkv4_forward" in names and "rwkv_wkv5_forward" in names and "rwkv_wkv6_forward" in names
     h = ctypes.CDLL(rw.LIB_PATH)
     missing = [n for n in names if not hasattr(h, n)]
     assert not missing, missing
@@ -122,6 +122,24 @@ def test_validation_before_any_cuda_work():
     assert h.rwkv_wkv5_step(2, 3, 64, fake, fake, fake, fake, fake, fake, P(0x1008), fake, None) == 2
     assert h.rwkv_wkv5_step(-2, 3, 64, fake, fake, fake, fake, fake, fake, None, fake, None) == 1
     assert h.rwkv_wkv5_step(0, 3, 64, fake, fake, fake, fake, fake, fake, None, fake, None) == 0
+    # WKV-6 forward: only N = 64; omega required and 16-byte aligned (TMA); T = 0 without s_out is a no-op
+    assert h.rwkv_wkv6_forward(1, 4, 2, 32, fake, fake, fake, fake, fake, fake, None, None, None, 0, None) == 2
+    assert h.rwkv_wkv6_forward(1, 4, 2, 64, fake, fake, fake, None, fake, fake, None, None, None, 0, None) == 1
+    assert h.rwkv_wkv6_forward(1, 4, 2, 64, fake, fake, fake, fake, None, fake, None, None, None, 0, None) == 1
+    assert h.rwkv_wkv6_forward(1, 4, 2, 64, fake, fake, fake, fake, fake, None, None, None, None, 0, None) == 1
+    assert h.rwkv_wkv6_forward(1, 4, 2, 64, fake, fake, fake, P(0x1004), fake, fake, None, None, None, 0,
+                               None) == 2
+    assert h.rwkv_wkv6_forward(1, 4, 2, 64, fake, fake, fake, fake, fake, P(0x1008), None, None, None, 0,
+                               None) == 2
+    assert h.rwkv_wkv6_forward(-1, 4, 2, 64, fake, fake, fake, fake, fake, fake, None, None, None, 0, None) == 1
+    assert h.rwkv_wkv6_forward(0, 4, 2, 64, fake, fake, fake, fake, fake, fake, None, None, None, 0, None) == 0
+    assert h.rwkv_wkv6_forward(1, 0, 2, 64, None, None, None, None, fake, None, None, None, None, 0, None) == 0
+    # WKV-6 decode step: as the WKV-5 step, with a per-stream omega
+    assert h.rwkv_wkv6_step(2, 3, 32, fake, fake, fake, fake, fake, fake, None, fake, None) == 2
+    assert h.rwkv_wkv6_step(2, 3, 64, fake, fake, fake, None, fake, fake, None, fake, None) == 1
+    assert h.rwkv_wkv6_step(2, 3, 64, fake, fake, fake, fake, fake, fake, None, None, None) == 1
+    assert h.rwkv_wkv6_step(2, 3, 64, fake, fake, fake, fake, fake, fake, None, P(0x1004), None) == 2
+    assert h.rwkv_wkv6_step(0, 3, 64, fake, fake, fake, fake, fake, fake, None, fake, None) == 0
 
 
 def test_binding_fails_loudly_without_library(monkeypatch):
