@@ -13,21 +13,27 @@
 //          + Σ_{ι<τ} A[τ,ι] v[ι,:] + (Σ_d r[τ,d] u_d k[τ,d]) v[τ,:]
 //   A[τ,ι] = Σ_d (r[τ,d] e^{Λ_{τ-1,d} - R_d}) (k[ι,d] e^{R_d - Λ_{ι,d}})
 //   S'     = e^{Λ_last} ⊙ S + e^{Λ_last - R} ⊙ Σ_ι (k[ι,:] e^{R - Λ_ι})ᵀ v[ι,:]
-// with the per-channel reference R = Λ_31 (the middle of the chunk) and
-// Λ_last the log-decay of the whole chunk.  With r̃ = r e^{Λ_{τ-1} - R} and
-// k̃ = k e^{R - Λ_ι} the chunk is the Eagle kernel's three tensor-core chains
+// with a per-channel reference R and Λ_last the log-decay of the whole chunk.
+// With r̃ = r e^{Λ_{τ-1} - R} and k̃ = k e^{R - Λ_ι} the chunk is the Eagle
+// kernel's three tensor-core chains
 //   [A | Y] = r̃ [k̃ ; e^{R} Sᵀ]ᵀ,   Y += A_masked v,   ΔS = k̃ᵀ v
-// (the Eagle kernel is the case Λ_τ = λ (τ + 1)).  Every factor stays in fp32
-// range while the log-decay of each half chunk, -R and R - Λ_last, is at most
-// 80 in every channel; a chunk that decays faster in some channel is computed
-// by the per-token recurrence instead, on the same state registers.
+// (the Eagle kernel is the case Λ_τ = λ (τ + 1), R = Λ_31).  Any R gives the
+// same products; every factor stays in fp32 range while -R and R - Λ_last
+// are at most 80 in every channel.  The first chunk takes R = Λ_31, the middle
+// of its own decay; every later chunk takes half the log-decay of the chunk
+// before it (the middle again while the decay rate holds), which is known when
+// the previous chunk folds its state, so that fold also writes e^{R} ⊙ Sᵀ for
+// the next chunk's state read as in the Eagle kernel.  A chunk whose decay
+// leaves that range in some channel (a fast decay, or one that jumps) is
+// computed by the per-token recurrence instead, on the same state registers.
 //
 // Decay prologue per chunk: each thread forms λ for 8 tokens x 2 channels
-// (ω arrives by TMA as two fp32 [64 tokens x 32 channels] boxes), the
-// cumulative sums come from 8-lane shuffle scans plus a running carry, and the
-// factors are exponentials of differences of those sums, so the rounding of
-// the cumulative decay never compounds from chunk to chunk beyond one fp32
-// product per chunk.
+// (ω arrives by TMA as two fp32 [64 tokens x 32 channels] boxes); the
+// cumulative sums come from 8-lane shuffle scans, all 16 of a thread's scans
+// advancing one shuffle step at a time so that their latencies overlap, plus a
+// running carry; the factors are exponentials of differences of those sums, so
+// the rounding of the cumulative decay never compounds from chunk to chunk
+// beyond one fp32 product per chunk.
 //
 // CTA: one (batch, head), 8 warps, about 109 KB of shared memory and 256 TMEM
 // columns, two CTAs per SM.  The fp32 master state lives in registers in the
@@ -60,7 +66,7 @@ struct Wkv6Smem {
   alignas(128) float opVt[64 * 64];  // vᵀ [j][ι]: B of A v and of ΔS; reduction scratch of the recurrent path
   float diag_part[8][kL];            // per-warp parts of Σ_d r u k
   float diag[kL];
-  float Rv[2][kN];                   // R = Λ_31 per channel, by chunk parity
+  float Rv[2][kN];                   // R per channel (the chunk's reference), by chunk parity
   float Lend[2][kN];                 // Λ_last per channel, by chunk parity
   alignas(8) uint64_t bar_tma;
   alignas(8) uint64_t bar_sc;
@@ -100,6 +106,10 @@ __device__ __forceinline__ uint32_t om_off(int tau, int d) {
   return (uint32_t)(d >> 5) * kOmBytes + (uint32_t)tau * 128u + ((uint32_t)(((d & 31) >> 2) ^ (tau & 7)) << 4) +
          (uint32_t)(d & 3) * 4u;
 }
+
+// Reference point of the next chunk's factorization: half of this chunk's log-decay
+// (the middle of the chunk if the decay rate stays put), no lower than -79.
+__device__ __forceinline__ float next_ref(float lend) { return fmaxf(0.5f * lend, -79.f); }
 
 struct Frag16 {
   float v[16];
@@ -234,6 +244,7 @@ __global__ void __launch_bounds__(kThreads, 2) wkv6_fwd_tc_kernel(const __grid_c
   const uint32_t opKs = smem_u32(sm.opK);
   const bool issuer = tid == 0;
   uint32_t nfast = 0;  // chunks done on the tensor cores (phase of the MMA barriers)
+  float Rnext[2] = {0.f, 0.f};  // reference of the next chunk: half the log-decay of this one
 
   for (int c = 0; c < nchunk; ++c) {
     const int t0 = c * kL;
@@ -245,34 +256,54 @@ __global__ void __launch_bounds__(kThreads, 2) wkv6_fwd_tc_kernel(const __grid_c
     // bonus parts.  Rows past the sequence end (zeros from the TMA fill) get λ = 0.
     int bad = 0;
     {
-      float lam[8][2], lin[8][2], carry[2] = {0.f, 0.f}, R[2] = {0.f, 0.f};
+      float lam[8][2], lin[8][2], carry[2] = {0.f, 0.f}, R[2] = {Rnext[0], Rnext[1]};
+      // stage-major: the 16 loads and exponentials, then each shuffle step for all 16 values at once
 #pragma unroll
       for (int ib = 0; ib < 8; ++ib) {
         const bool live = 8 * ib + rr < cnt;
         const float2 om = lds_f2(omS + offW + ib * 1024u);
-        float x[2] = {live ? -__expf(om.x) : 0.f, live ? -__expf(om.y) : 0.f};
+        lam[ib][0] = live ? -__expf(om.x) : 0.f;
+        lam[ib][1] = live ? -__expf(om.y) : 0.f;
+        lin[ib][0] = lam[ib][0];
+        lin[ib][1] = lam[ib][1];
+      }
 #pragma unroll
-        for (int e = 0; e < 2; ++e) lam[ib][e] = x[e];
+      for (int o = 1; o < 8; o <<= 1) {
+        float up[8][2];
 #pragma unroll
-        for (int o = 1; o < 8; o <<= 1) {
+        for (int ib = 0; ib < 8; ++ib)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) up[ib][e] = __shfl_up_sync(0xffffffffu, lin[ib][e], o, 8);
+#pragma unroll
+        for (int ib = 0; ib < 8; ++ib)
+#pragma unroll
+          for (int e = 0; e < 2; ++e)
+            if (rr >= o) lin[ib][e] += up[ib][e];
+      }
+      {
+        float tot[8][2];
+#pragma unroll
+        for (int ib = 0; ib < 8; ++ib)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) tot[ib][e] = __shfl_sync(0xffffffffu, lin[ib][e], 7, 8);
+#pragma unroll
+        for (int ib = 0; ib < 8; ++ib) {
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
-            const float y = __shfl_up_sync(0xffffffffu, x[e], o, 8);
-            if (rr >= o) x[e] += y;
+            lin[ib][e] += carry[e];
+            carry[e] += tot[ib][e];
           }
-        }
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          lin[ib][e] = carry[e] + x[e];
-          carry[e] += __shfl_sync(0xffffffffu, x[e], 7, 8);
-        }
-        if (ib == 3) {
-          R[0] = carry[0];
-          R[1] = carry[1];
+          if (ib == 3 && c == 0) {
+            R[0] = carry[0];
+            R[1] = carry[1];
+          }
         }
       }
 #pragma unroll
-      for (int e = 0; e < 2; ++e) bad |= !(-R[e] <= kMaxHalfDecay && R[e] - carry[e] <= kMaxHalfDecay);
+      for (int e = 0; e < 2; ++e) {
+        bad |= !(-R[e] <= kMaxHalfDecay && R[e] - carry[e] <= kMaxHalfDecay);
+        Rnext[e] = next_ref(carry[e]);
+      }
       if (rr == 0) {
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
@@ -280,6 +311,7 @@ __global__ void __launch_bounds__(kThreads, 2) wkv6_fwd_tc_kernel(const __grid_c
           sm.Lend[par][dR + e] = carry[e];
         }
       }
+      float part[8];
 #pragma unroll
       for (int ib = 0; ib < 8; ++ib) {
         const float2 rv = bf2_to_f2(lds_u32(rawR + offRK + ib * 1024u));
@@ -289,10 +321,15 @@ __global__ void __launch_bounds__(kThreads, 2) wkv6_fwd_tc_kernel(const __grid_c
         const float fk0 = __expf(R[0] - lin[ib][0]), fk1 = __expf(R[1] - lin[ib][1]);
         *reinterpret_cast<float2*>(&sm.opRA[op_off(row, dR)]) = make_float2(rv.x * fr0, rv.y * fr1);
         *reinterpret_cast<float2*>(&sm.opK[op_off(row, dR)]) = make_float2(kv.x * fk0, kv.y * fk1);
-        float part = fmaf(rv.x * uA[0], kv.x, rv.y * uA[1] * kv.y);
-        part += __shfl_xor_sync(0xffffffffu, part, 8);
-        part += __shfl_xor_sync(0xffffffffu, part, 16);
-        if (rp == 0) sm.diag_part[warp][row] = part;
+        part[ib] = fmaf(rv.x * uA[0], kv.x, rv.y * uA[1] * kv.y);
+      }
+#pragma unroll
+      for (int ib = 0; ib < 8; ++ib) part[ib] += __shfl_xor_sync(0xffffffffu, part[ib], 8);
+#pragma unroll
+      for (int ib = 0; ib < 8; ++ib) part[ib] += __shfl_xor_sync(0xffffffffu, part[ib], 16);
+      if (rp == 0) {
+#pragma unroll
+        for (int ib = 0; ib < 8; ++ib) sm.diag_part[warp][8 * ib + rr] = part[ib];
       }
     }
     fence_proxy_async();
@@ -302,6 +339,14 @@ __global__ void __launch_bounds__(kThreads, 2) wkv6_fwd_tc_kernel(const __grid_c
 
     if (slow) {  // some channel decays too fast for the factorization: per-token recurrence
       S = chunk_recurrent(S, sm, p, b, h, t0, cnt);
+      if (c + 1 < nchunk) {
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          const float eR = __expf(next_ref(sm.Lend[par][drow + 8 * r]));
+#pragma unroll
+          for (int q = 0; q < 8; ++q) sm.opS[op_off(jcol + 4 * q, drow + 8 * r)] = eR * S.v[2 * q + r];
+        }
+      }
       if (issuer && c + 1 < nchunk) {
         fence_proxy_async();
         mbar_arrive_expect_tx(&sm.bar_tma, 3 * kRawBytes + 2 * kOmBytes);
@@ -314,16 +359,17 @@ __global__ void __launch_bounds__(kThreads, 2) wkv6_fwd_tc_kernel(const __grid_c
       continue;
     }
 
-    // e^{R} ⊙ Sᵀ for this chunk's state read (R of this chunk, S as the previous chunk left it)
+    if (c == 0) {  // e^{R} ⊙ Sᵀ of the initial state (later chunks get it from the previous state fold)
 #pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      const float eR = __expf(sm.Rv[par][drow + 8 * r]);
+      for (int r = 0; r < 2; ++r) {
+        const float eR = __expf(sm.Rv[par][drow + 8 * r]);
 #pragma unroll
-      for (int q = 0; q < 8; ++q) sm.opS[op_off(jcol + 4 * q, drow + 8 * r)] = eR * S.v[2 * q + r];
+        for (int q = 0; q < 8; ++q) sm.opS[op_off(jcol + 4 * q, drow + 8 * r)] = eR * S.v[2 * q + r];
+      }
+      fence_proxy_async();
+      tc_fence_before();
+      __syncthreads();
     }
-    fence_proxy_async();
-    tc_fence_before();
-    __syncthreads();
 
     const uint32_t phm = nfast & 1u;
     auto issue_first = [&](int s0) {
@@ -459,9 +505,12 @@ __global__ void __launch_bounds__(kThreads, 2) wkv6_fwd_tc_kernel(const __grid_c
 #pragma unroll
       for (int r = 0; r < 2; ++r) {
         const float le = sm.Lend[par][drow + 8 * r], rv = sm.Rv[par][drow + 8 * r];
-        const float gD = __expf(le), gS = __expf(le - rv);
+        const float gD = __expf(le), gS = __expf(le - rv), eR = __expf(next_ref(le));
 #pragma unroll
-        for (int q = 0; q < 8; ++q) S.v[2 * q + r] = fmaf(gD, S.v[2 * q + r], gS * ds[2 * q + r]);
+        for (int q = 0; q < 8; ++q) {
+          S.v[2 * q + r] = fmaf(gD, S.v[2 * q + r], gS * ds[2 * q + r]);
+          sm.opS[op_off(jcol + 4 * q, drow + 8 * r)] = eR * S.v[2 * q + r];
+        }
       }
     }
     ++nfast;
