@@ -50,6 +50,8 @@ def _load():
             "oracle_wkv5_forward": [I, I, I, I, P, P, P, P, P, P, P, P],
             "oracle_wkv5_forward_bruteforce": [I, I, I, I, P, P, P, P, P, P],
             "oracle_wkv6_forward": [I, I, I, I, P, P, P, P, P, P, P, P],
+            "oracle_wkv4_gated_forward": [I, I, I, P, P, P, P, P, P, P, P],
+            "oracle_wkv4_gated_backward": [I, I, I, P, P, P, P, P, P, P, P, P, P, P, P],
             "oracle_wkv6_forward_bruteforce": [I, I, I, I, P, P, P, P, P, P],
         }
         for name, args in sigs.items():
@@ -202,3 +204,28 @@ def wkv6_forward_bruteforce(r, k, v, omega, u):
     _check(lib.oracle_wkv6_forward_bruteforce(B, T, H, N, _p(r), _p(k), _p(v), _p(omega), _p(u),
                                               _p(y)), "wkv6_forward_bruteforce")
     return y
+
+
+def wkv4_gated_forward(w, u, k, v, r, state_in=None, return_state=False):
+    """Receptance-gated WKV-4 forward o = sigmoid(r) * WKV.  k, v, r [B,T,C];
+    w, u [C]; state_in [2,B,C] or None.  Returns o (and the state [2,B,C])."""
+    lib = _load()
+    w, u, k, v, r, s0 = map(_f64, (w, u, k, v, r, state_in))
+    B, T, C = k.shape
+    o = np.empty((B, T, C))
+    s1 = np.empty((2, B, C))
+    _check(lib.oracle_wkv4_gated_forward(B, T, C, _p(w), _p(u), _p(k), _p(v), _p(r), _p(s0), _p(o), _p(s1)),
+           "wkv4_gated_forward")
+    return (o, s1) if return_state else o
+
+
+def wkv4_gated_backward(w, u, k, v, r, go, state_in=None):
+    """Gradients of sum(go * o) for the gated forward: (gk, gv, gr, gw, gu)."""
+    lib = _load()
+    w, u, k, v, r, go, s0 = map(_f64, (w, u, k, v, r, go, state_in))
+    B, T, C = k.shape
+    gk, gv, gr = np.empty((B, T, C)), np.empty((B, T, C)), np.empty((B, T, C))
+    gw, gu = np.empty(C), np.empty(C)
+    _check(lib.oracle_wkv4_gated_backward(B, T, C, _p(w), _p(u), _p(k), _p(v), _p(r), _p(go), _p(s0),
+                                          _p(gk), _p(gv), _p(gr), _p(gw), _p(gu)), "wkv4_gated_backward")
+    return gk, gv, gr, gw, gu

@@ -18,6 +18,8 @@
  *  [P3] "RWKV-5 Eagle과 RWKV-6 Finch", section "Eagle: 벡터 기억을 행렬 기억으로
  *       확장": s' = diag(w) s + k^T v, wkv' = s + diag(u) k^T v, w = exp(-exp(ω)),
  *       receptance reads the state like a query.
+ *  [P1] also (2) output line o_t = W_o (σ(r_t) ⊙ WKV_t) and (4) Receptance
+ *       Gating: σ(r_t) decides per channel how much of the aggregate passes.
  *  [P3] also, section "Finch: recurrence를 입력에 반응시키기": Finch keeps the
  *       Eagle update and makes the decay data dependent (a per-token decay
  *       vector, corrected from the input through a LoRA).
@@ -508,5 +510,48 @@ int64_t oracle_wkv6_forward_bruteforce(int64_t B, int64_t T, int64_t H, int64_t 
             }
         }
     }
+    return bad;
+}
+
+/*
+ * Receptance-gated WKV-4 forward [P1 (2) output line o_t = W_o (σ(r_t) ⊙ WKV_t)
+ * and (4) Receptance Gating; the projection W_o is not part of the operator]:
+ *   o_t = σ(r_t) WKV_t,   σ(x) = 1 / (1 + e^{-x}),
+ * with WKV_t from oracle_wkv4_forward (same state conventions).
+ */
+int64_t oracle_wkv4_gated_forward(int64_t B, int64_t T, int64_t C,
+                                  const double *w, const double *u,
+                                  const double *k, const double *v, const double *r,
+                                  const double *state_in, double *o, double *state_out)
+{
+    const int64_t bad = oracle_wkv4_forward(B, T, C, w, u, k, v, state_in, o, state_out);
+    for (int64_t i = 0; i < B * T * C; ++i) o[i] *= 1.0 / (1.0 + exp(-r[i]));
+    return bad;
+}
+
+/*
+ * Gradients of L = Σ go_t o_t for the gated forward above, by the chain rule:
+ * L depends on WKV through gy_t = σ(r_t) go_t, so gk, gv, gw, gu are
+ * oracle_wkv4_backward with that gy, and
+ *   gr_t = go_t WKV_t σ(r_t) (1 - σ(r_t)).
+ */
+int64_t oracle_wkv4_gated_backward(int64_t B, int64_t T, int64_t C,
+                                   const double *w, const double *u,
+                                   const double *k, const double *v, const double *r,
+                                   const double *go, const double *state_in,
+                                   double *gk, double *gv, double *gr, double *gw, double *gu)
+{
+    const int64_t n = B * T * C;
+    double *wkv = (double *)malloc((size_t)n * sizeof(double));
+    double *gy = (double *)malloc((size_t)n * sizeof(double));
+    int64_t bad = oracle_wkv4_forward(B, T, C, w, u, k, v, state_in, wkv, NULL);
+    for (int64_t i = 0; i < n; ++i) {
+        const double s = 1.0 / (1.0 + exp(-r[i]));
+        gy[i] = s * go[i];
+        gr[i] = go[i] * wkv[i] * s * (1.0 - s);
+    }
+    bad += oracle_wkv4_backward(B, T, C, w, u, k, v, gy, state_in, gk, gv, gw, gu);
+    free(wkv);
+    free(gy);
     return bad;
 }

@@ -7,7 +7,8 @@ distributions that the WKV workloads use:
 * RWKV-4 WKV: per-channel decay rate ``w`` log-uniform on [0.01, 5], bonus
   ``u ~ U(-1, 1)``, keys and values ``k, v ~ N(0, 1)`` i.i.d., optionally 1 % of
   the keys replaced by ``±U(20, 40)`` outliers, upstream gradient
-  ``gy ~ N(0, 1)``.
+  ``gy ~ N(0, 1)``; with the receptance gate, ``r ~ N(0, 1)`` and the upstream
+  gradient of the gated output ``go ~ N(0, 1)``.
 * Eagle / RWKV-5 WKV: ``r, k, v ~ N(0, 1)/sqrt(N)`` rounded to bf16, per-channel
   ``omega ~ U(-6, 0)`` and ``u ~ U(-1, 1)`` of shape ``[H, N]``.
 * Finch / RWKV-6 WKV: as Eagle, with a per-token decay parameter
@@ -179,8 +180,10 @@ def wkv4_params(seed: int, C: int, c_sel=None, device="cpu"):
 
 
 def wkv4_problem(B: int, T: int, C: int, seed: int, outliers: bool = False,
-                 with_gy: bool = False, dtype=torch.float32, device="cpu") -> dict:
-    """Full RWKV-4 WKV inputs: w, u [C] fp32; k, v (and gy) [B, T, C] of ``dtype``."""
+                 with_gy: bool = False, dtype=torch.float32, device="cpu", gated: bool = False) -> dict:
+    """Full RWKV-4 WKV inputs: w, u [C] fp32; k, v (and gy) [B, T, C] of ``dtype``;
+    with ``gated``, also the receptance r and (with ``with_gy``) the gradient
+    ``go`` of the gated output [B, T, C] (``go`` is drawn from gy's stream)."""
     w, u = wkv4_params(seed, C, device=device)
     p = {
         "w": w,
@@ -189,7 +192,9 @@ def wkv4_problem(B: int, T: int, C: int, seed: int, outliers: bool = False,
         "v": btc_field("v", seed, B, T, C, dtype=dtype, device=device),
     }
     if with_gy:
-        p["gy"] = btc_field("gy", seed, B, T, C, dtype=dtype, device=device)
+        p["go" if gated else "gy"] = btc_field("gy", seed, B, T, C, dtype=dtype, device=device)
+    if gated:
+        p["r"] = btc_field("r", seed, B, T, C, dtype=dtype, device=device)
     return p
 
 
