@@ -104,7 +104,7 @@ class ClockSampler:
 # kernel name in profiles/traffic.json -> prefix of the source files it is built from
 _TRAFFIC_SOURCES = {"wkv4_bwd_kernel": "wkv4_bwd", "wkv5_fwd_tc_kernel": "wkv5_fwd", "wkv4_step_kernel": "wkv4_step",
                     "wkv5_step_kernel": "wkv5_step", "wkv6_fwd_tc_kernel": "wkv6_fwd",
-                    "wkv5_step_kernel/finch": "wkv5_step"}
+                    "wkv5_step_kernel/finch": "wkv5_step", "wkv4_bwd_kernel/gated": "wkv4_bwd"}
 
 
 def _kernel_source_hash(kernel="wkv4_bwd_kernel"):
@@ -428,6 +428,72 @@ def run_decode(args):
         "gpu_launches": args.steps, "clocks": clk}), flush=True)
 
 
+def run_train_gated(args):
+    """Receptance-gated RWKV-4 training step: o = sigmoid(r) * WKV forward and its
+    backward (gk, gv, gr, gw, gu), fp32, B=8 T=4096 C=2048, as the headline step."""
+    import torch
+
+    import rwkv_wkv_recurrence_b200 as rw
+    import wkv_inputs as wi
+
+    _, _, local = _dist()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    p = wi.wkv4_problem(B, T, C, SEED, outliers=True, with_gy=True, gated=True, device=dev)
+    w, u, k, v, r, go = p["w"], p["u"], p["k"], p["v"], p["r"], p["go"]
+    o = torch.empty_like(k)
+    gk, gv, gr = torch.empty_like(k), torch.empty_like(k), torch.empty_like(k)
+    gw, gu = torch.empty(C, device=dev), torch.empty(C, device=dev)
+    h = rw.lib()
+    nck = int(h.rwkv_wkv4_num_checkpoints(T, rw.CHUNK_LEN))
+    ck = torch.empty((nck, 3, B, C), device=dev)
+    fws = int(h.rwkv_wkv4_forward_workspace_bytes(B, T, C, rw.ALGO_AUTO))
+    bws = int(h.rwkv_wkv4_backward_workspace_bytes(B, T, C, rw.CHUNK_LEN, 1))
+    fw = torch.empty(max(fws, 1), dtype=torch.uint8, device=dev)
+    bw = torch.empty(bws, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    sp, P = rw._stream(stream), rw._ptr
+
+    def fwd(i=0):
+        s = h.rwkv_wkv4_forward_gated(B, T, C, rw.F32, P(w), P(u), P(k), P(v), P(r), P(o), None, None, P(ck),
+                                      rw.CHUNK_LEN, rw.ALGO_AUTO, P(fw), fws, sp)
+        if s:
+            raise rw.RwkvError("rwkv_wkv4_forward_gated", s)
+
+    def bwd(i=0):
+        s = h.rwkv_wkv4_backward_gated(B, T, C, rw.F32, P(w), P(u), P(k), P(v), P(r), P(go), None, P(ck),
+                                       rw.CHUNK_LEN, P(gk), P(gv), P(gr), P(gw), P(gu), P(bw), bws, sp)
+        if s:
+            raise rw.RwkvError("rwkv_wkv4_backward_gated", s)
+
+    def step(i):
+        fwd()
+        bwd()
+
+    ms, clk = _timed(step, args.steps, args.warmup, stream, local)
+    fwd_ms, _ = _timed(fwd, args.steps, args.warmup, stream, local)
+    bwd_ms, _ = _timed(bwd, args.steps, args.warmup, stream, local)
+    rw.rwkv_check_device_error()
+    fwd_bytes = 4 * 4 * ELEM                      # k, v, r read; o written
+    bwd_bytes = 7 * 4 * ELEM + 2 * 4 * C          # k, v, r, go read; gk, gv, gr written; gw, gu
+    peak, kind = _peaks()
+    bwd_gbs = bwd_bytes / (bwd_ms * 1e-3) / 1e9
+    step_gbs = (fwd_bytes + bwd_bytes) / (ms * 1e-3) / 1e9
+    print(json.dumps({
+        "metric": "Gated WKV fwd+bwd elements/s and HBM GB/s (o = sigmoid(r) * WKV) at B8 T4096 C2048",
+        "value": ELEM / (ms * 1e-3), "unit": "elements/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": "RWKV-4 receptance-gated WKV forward+backward, fp32, B=8 T=4096 C=2048, 1% "
+                               "+-U(20,40) key outliers, r, go ~ N(0,1)",
+                   "l2": "no flush: every input (268 MB each) is larger than the 126 MB L2"},
+        "hbm_gbs_step": step_gbs, "hbm_frac_step": step_gbs / peak,
+        "kernels_ms": {"wkv4_forward_gated": fwd_ms, "wkv4_backward_gated": bwd_ms},
+        "roofline": {"bound": "hbm", "kernel": "wkv4_bwd_kernel<float, gated> (+ its gw/gu batch reduction)",
+                     "achieved": bwd_gbs, "peak": peak, "peak_kind": kind, "unit": "GB/s",
+                     "frac": bwd_gbs / peak, "traffic": _recorded_traffic("wkv4_bwd_kernel/gated")},
+        "gpu_launches": 3 * args.steps, "clocks": clk}), flush=True)
+
+
 def run_eagle(args, finch=False):
     """Eagle / RWKV-5 forward, B4 T4096 H40 N64 bf16, zero initial state; with
     finch, the Finch / RWKV-6 forward on the same shape with a per-token fp32
@@ -549,10 +615,11 @@ def main():
     ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["train", "decode", "eagle", "eagle_decode", "finch", "finch_decode"],
+    ap.add_argument("--workload", choices=["train", "train_gated", "decode", "eagle", "eagle_decode", "finch",
+                                           "finch_decode"],
                     default="train",
-                    help="train: the headline forward+backward step; decode, eagle, eagle_decode, finch, "
-                         "finch_decode: the other hot-path rows")
+                    help="train: the headline forward+backward step; train_gated, decode, eagle, eagle_decode, "
+                         "finch, finch_decode: the other hot-path rows")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--ref-channels", type=int, default=256)
@@ -565,6 +632,8 @@ def main():
         run_reference(args)
     elif args.workload == "decode":
         run_decode(args)
+    elif args.workload == "train_gated":
+        run_train_gated(args)
     elif args.workload == "eagle":
         run_eagle(args)
     elif args.workload == "eagle_decode":

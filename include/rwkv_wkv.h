@@ -44,7 +44,7 @@
  *     before anything is enqueued.  A launch failure gives RWKV_ERR_CUDA.
  *     Zero-sized problems are a successful no-op (T = 0 copies the state).
  *   - Values are data: no range validation; NaN and Inf propagate.
- *   - Alignment: the WKV-4 [B,T,C] tensors k, v, y, gy, gk, gv (and the WKV-5
+ *   - Alignment: the WKV-4 [B,T,C] tensors k, v, y, gy, gk, gv, r, o, go, gr (and the WKV-5
  *     tensors r, k, v, y, and Finch's omega) must be 16-byte aligned with
  *     C·sizeof(element) a multiple of 16 (TMA row pitch), else
  *     RWKV_ERR_UNSUPPORTED.
@@ -119,6 +119,24 @@ RWKV_API rwkv_status rwkv_wkv4_forward(int64_t B, int64_t T, int64_t C, rwkv_dty
                               const float *state_in, float *state_out, float *ckpt, int64_t chunk_len,
                               int algo, void *workspace, size_t workspace_bytes, rwkv_stream_t stream);
 
+/*
+ * Receptance-gated WKV-4 forward: the time-mixing output of the same page,
+ * o_t = W_o (σ(r_t) ⊙ WKV_t) ((2) and (4) Receptance Gating), without the
+ * projection W_o (a GEMM outside the operator):
+ *   o = σ(r) ⊙ WKV,   σ(x) = 1 / (1 + e^{-x}),
+ * in one pass: the same arguments as rwkv_wkv4_forward plus
+ *   r         [B,T,C] dtype, read (required);
+ *   o         [B,T,C] dtype, written (required; replaces y).
+ * state_out and ckpt are those of the ungated forward over the same k, v (the
+ * gate does not enter the recurrence), so rwkv_wkv4_backward_gated reads the
+ * same checkpoints.  Workspace: rwkv_wkv4_forward_workspace_bytes().
+ */
+RWKV_API rwkv_status rwkv_wkv4_forward_gated(int64_t B, int64_t T, int64_t C, rwkv_dtype dtype,
+                                    const float *w, const float *u, const void *k, const void *v,
+                                    const void *r, void *o, const float *state_in, float *state_out,
+                                    float *ckpt, int64_t chunk_len, int algo, void *workspace,
+                                    size_t workspace_bytes, rwkv_stream_t stream);
+
 /* Workspace bytes rwkv_wkv4_backward needs; have_ckpt = 0 adds room to
  * recompute the checkpoints. */
 RWKV_API size_t rwkv_wkv4_backward_workspace_bytes(int64_t B, int64_t T, int64_t C, int64_t chunk_len, int have_ckpt);
@@ -140,6 +158,22 @@ RWKV_API rwkv_status rwkv_wkv4_backward(int64_t B, int64_t T, int64_t C, rwkv_dt
                                const void *gy, const float *state_in, const float *ckpt,
                                int64_t chunk_len, void *gk, void *gv, float *gw, float *gu,
                                void *workspace, size_t workspace_bytes, rwkv_stream_t stream);
+
+/*
+ * Backward of the receptance-gated forward: gradients of L = Σ go·o with
+ * o = σ(r) ⊙ WKV.  The same arguments as rwkv_wkv4_backward with gy replaced
+ * by r and go, plus gr:
+ *   r, go     [B,T,C] dtype, read (required).
+ *   gr        [B,T,C] dtype, written: go · WKV · σ(r)(1 - σ(r)).
+ *   gk, gv, gw, gu as rwkv_wkv4_backward with gy = σ(r) ⊙ go.
+ * Workspace: rwkv_wkv4_backward_workspace_bytes().  Deterministic.
+ */
+RWKV_API rwkv_status rwkv_wkv4_backward_gated(int64_t B, int64_t T, int64_t C, rwkv_dtype dtype,
+                                     const float *w, const float *u, const void *k, const void *v,
+                                     const void *r, const void *go, const float *state_in,
+                                     const float *ckpt, int64_t chunk_len, void *gk, void *gv, void *gr,
+                                     float *gw, float *gu, void *workspace, size_t workspace_bytes,
+                                     rwkv_stream_t stream);
 
 /*
  * WKV-4 recurrent decode: one token for each of B independent streams.

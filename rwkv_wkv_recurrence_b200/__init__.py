@@ -21,7 +21,7 @@ import os
 __all__ = [
     "LIB_PATH", "lib", "RwkvError", "RWKV_OK", "F32", "BF16", "ALGO_AUTO", "ALGO_SEQUENTIAL",
     "ALGO_CHUNKED", "CHUNK_LEN", "NOALLOC_MAX_LANES", "rwkv_wkv4_forward", "rwkv_wkv4_backward",
-    "rwkv_wkv4_backward_noalloc", "rwkv_wkv4_step",
+    "rwkv_wkv4_backward_noalloc", "rwkv_wkv4_step", "rwkv_wkv4_forward_gated", "rwkv_wkv4_backward_gated",
     "rwkv_wkv5_forward", "rwkv_wkv5_step", "rwkv_wkv6_forward", "rwkv_wkv6_step", "rwkv_check_device_error",
     "state_to_ab",
 ]
@@ -63,6 +63,8 @@ def lib():
         "rwkv_wkv4_backward_workspace_bytes": ([I64, I64, I64, I64, I], S),
         "rwkv_wkv4_backward": ([I64, I64, I64, I, P, P, P, P, P, P, P, I64, P, P, P, P, P, S, P], I),
         "rwkv_wkv4_step": ([I64, I64, I, P, P, P, P, P, P, P, P], I),
+        "rwkv_wkv4_forward_gated": ([I64, I64, I64, I, P, P, P, P, P, P, P, P, P, I64, I, P, S, P], I),
+        "rwkv_wkv4_backward_gated": ([I64, I64, I64, I, P, P, P, P, P, P, P, P, I64, P, P, P, P, P, P, S, P], I),
         "rwkv_wkv5_forward_workspace_bytes": ([I64, I64, I64, I64], S),
         "rwkv_wkv5_forward": ([I64, I64, I64, I64, P, P, P, P, P, P, P, P, P, S, P], I),
         "rwkv_wkv4_backward_noalloc": ([I64, I64, I64, I, P, P, P, P, P, P, I64, P, P, P, P, P], I),
@@ -184,6 +186,67 @@ def rwkv_wkv4_backward(w, u, k, v, gy, ckpt=None, state_in=None, *, stream=None,
                                 _ptr(state_in), _ptr(ckpt), CHUNK_LEN, _ptr(gk), _ptr(gv), _ptr(gw),
                                 _ptr(gu), _ptr(ws), wsb, _stream(stream)))
     return gk, gv, gw, gu
+
+
+def rwkv_wkv4_forward_gated(w, u, k, v, r, state_in=None, *, return_state=False, checkpoints=False,
+                            algo=ALGO_AUTO, stream=None, out=None):
+    """Receptance-gated WKV-4 forward: o = sigmoid(r) * WKV in one pass.  k, v, r
+    [B,T,C] (fp32 or bf16); w, u [C] fp32.  Returns o (plus the state and the
+    checkpoints as ``rwkv_wkv4_forward``)."""
+    import torch
+
+    _need_cuda(w, u, k, v, r, state_in)
+    B, T, C = k.shape
+    for name, t in (("v", v), ("r", r)):
+        if t.shape != k.shape or t.dtype != k.dtype:
+            raise ValueError(f"{name} must match k in shape and dtype")
+    _f32("w", w, C)
+    _f32("u", u, C)
+    if state_in is not None:
+        _f32("state_in", state_in, 3 * B * C)
+    h = lib()
+    o = torch.empty_like(k) if out is None else out
+    st = torch.empty((3, B, C), dtype=torch.float32, device=k.device) if return_state else None
+    nck = int(h.rwkv_wkv4_num_checkpoints(T, CHUNK_LEN))
+    ck = torch.empty((nck, 3, B, C), dtype=torch.float32, device=k.device) if checkpoints else None
+    wsb = int(h.rwkv_wkv4_forward_workspace_bytes(B, T, C, algo))
+    ws = torch.empty(wsb, dtype=torch.uint8, device=k.device) if wsb else None
+    _check("rwkv_wkv4_forward_gated",
+           h.rwkv_wkv4_forward_gated(B, T, C, _dtype_code(k), _ptr(w), _ptr(u), _ptr(k), _ptr(v), _ptr(r), _ptr(o),
+                                     _ptr(state_in), _ptr(st), _ptr(ck), CHUNK_LEN, algo, _ptr(ws), wsb,
+                                     _stream(stream)))
+    res = (o,)
+    if return_state:
+        res += (st,)
+    if checkpoints:
+        res += (ck,)
+    return res[0] if len(res) == 1 else res
+
+
+def rwkv_wkv4_backward_gated(w, u, k, v, r, go, ckpt=None, state_in=None, *, stream=None, out=None):
+    """Backward of the gated forward: returns (gk, gv, gr, gw, gu) for
+    L = sum(go * o), o = sigmoid(r) * WKV."""
+    import torch
+
+    _need_cuda(w, u, k, v, r, go, ckpt, state_in)
+    B, T, C = k.shape
+    for name, t in (("v", v), ("r", r), ("go", go)):
+        if t.shape != k.shape or t.dtype != k.dtype:
+            raise ValueError(f"{name} must match k in shape and dtype")
+    h = lib()
+    if out is None:
+        gk, gv, gr = torch.empty_like(k), torch.empty_like(v), torch.empty_like(r)
+        gw = torch.empty(C, dtype=torch.float32, device=k.device)
+        gu = torch.empty(C, dtype=torch.float32, device=k.device)
+    else:
+        gk, gv, gr, gw, gu = out
+    wsb = int(h.rwkv_wkv4_backward_workspace_bytes(B, T, C, CHUNK_LEN, 1 if ckpt is not None else 0))
+    ws = torch.empty(max(wsb, 1), dtype=torch.uint8, device=k.device)
+    _check("rwkv_wkv4_backward_gated",
+           h.rwkv_wkv4_backward_gated(B, T, C, _dtype_code(k), _ptr(w), _ptr(u), _ptr(k), _ptr(v), _ptr(r),
+                                      _ptr(go), _ptr(state_in), _ptr(ckpt), CHUNK_LEN, _ptr(gk), _ptr(gv),
+                                      _ptr(gr), _ptr(gw), _ptr(gu), _ptr(ws), wsb, _stream(stream)))
+    return gk, gv, gr, gw, gu
 
 
 def rwkv_wkv4_backward_noalloc(w, u, k, v, gy, ckpt, *, stream=None, out=None):

@@ -120,15 +120,21 @@ FwdPlan plan_forward(int64_t B, int64_t T, int64_t C, int algo) {
   return pl;
 }
 
-// Runs the forward pass (outputs optional) on already-validated arguments.
+// Runs the forward pass (outputs optional) on already-validated arguments.  With r, the
+// output pass writes σ(r) ⊙ WKV (the receptance-gated kernel) instead of WKV.
 rwkv_status run_forward(int B, int T, int C, bool bf16, const float* w, const float* u, const void* k,
                         const void* v, void* y, const float* state_in, float* state_out, float* ckpt, int ckpt_len,
-                        const FwdPlan& pl, void* ws, cudaStream_t st) {
+                        const FwdPlan& pl, void* ws, cudaStream_t st, const void* r = nullptr) {
   unsigned int* err = device_error_word();
   if (err == nullptr) return RWKV_ERR_CUDA;
   const int tt = fwd_tile_steps();
-  CUtensorMap mk, mv, my;
+  const bool gate = r != nullptr && y != nullptr;
+  CUtensorMap mk, mv, my, mr;
   if (!make_btc_map(&mk, k, bf16, B, T, C, tt) || !make_btc_map(&mv, v, bf16, B, T, C, tt)) return RWKV_ERR_CUDA;
+  if (gate && !make_btc_map(&mr, r, bf16, B, T, C, tt)) return RWKV_ERR_CUDA;
+  auto launch_out = [&](const Fwd4Params& q) {  // the pass that writes the outputs
+    return gate ? launch_wkv4_fwd_gated(bf16, mk, mv, my, mr, q, st) : launch_wkv4_fwd(bf16, mk, mv, my, q, st);
+  };
   if (y != nullptr) {
     if (!make_btc_map(&my, y, bf16, B, T, C, fwd_store_steps())) return RWKV_ERR_CUDA;
   } else {
@@ -147,12 +153,12 @@ rwkv_status run_forward(int B, int T, int C, bool bf16, const float* w, const fl
   if (pl.algo == RWKV_ALGO_SEQUENTIAL) {
     p.seg_len = pl.seg_len;
     p.nseg = 1;
-    p.stages = fwd_stages(bf16, pl.seg_len);
+    p.stages = fwd_stages(bf16, pl.seg_len, gate);
     p.y = y;
     p.start = state_in;
     p.end = state_out;
     p.ckpt = ckpt;
-    if (launch_wkv4_fwd(bf16, mk, mv, my, p, st) != cudaSuccess) return RWKV_ERR_CUDA;
+    if (launch_out(p) != cudaSuccess) return RWKV_ERR_CUDA;
     return RWKV_OK;
   }
   float* wsf = static_cast<float*>(ws);
@@ -175,7 +181,8 @@ rwkv_status run_forward(int B, int T, int C, bool bf16, const float* w, const fl
   p.start_seg_stride = seg_stride;
   p.end = nullptr;
   p.ckpt = ckpt;
-  if (launch_wkv4_fwd(bf16, mk, mv, my, p, st) != cudaSuccess) return RWKV_ERR_CUDA;
+  p.stages = fwd_stages(bf16, pl.seg_len, gate);
+  if (launch_out(p) != cudaSuccess) return RWKV_ERR_CUDA;
   return RWKV_OK;
 }
 
@@ -198,7 +205,7 @@ const char* rwkv_status_string(rwkv_status s) {
   return "unknown status";
 }
 
-int rwkv_version(void) { return (1 << 16) | 1; }
+int rwkv_version(void) { return (1 << 16) | 2; }
 
 int64_t rwkv_wkv4_num_checkpoints(int64_t T, int64_t chunk_len) {
   if (chunk_len <= 0 || chunk_len % 16 != 0 || T < 0) return -1;
@@ -238,6 +245,33 @@ rwkv_status rwkv_wkv4_forward(int64_t B, int64_t T, int64_t C, rwkv_dtype dtype,
                      workspace, st);
 }
 
+rwkv_status rwkv_wkv4_forward_gated(int64_t B, int64_t T, int64_t C, rwkv_dtype dtype, const float* w,
+                                    const float* u, const void* k, const void* v, const void* r, void* o,
+                                    const float* state_in, float* state_out, float* ckpt, int64_t chunk_len, int algo,
+                                    void* workspace, size_t workspace_bytes, rwkv_stream_t stream) {
+  if (!fits_int(B) || !fits_int(T) || !fits_int(C)) return RWKV_ERR_INVALID_ARG;
+  if (dtype != RWKV_F32 && dtype != RWKV_BF16) return RWKV_ERR_INVALID_ARG;
+  if (algo < RWKV_ALGO_AUTO || algo > RWKV_ALGO_CHUNKED) return RWKV_ERR_INVALID_ARG;
+  if (ckpt != nullptr && (chunk_len <= 0 || chunk_len % 16 != 0)) return RWKV_ERR_INVALID_ARG;
+  if (ckpt != nullptr && chunk_len != kCkLen) return RWKV_ERR_UNSUPPORTED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (B == 0 || C == 0) return RWKV_OK;
+  if (w == nullptr || u == nullptr) return RWKV_ERR_INVALID_ARG;
+  if (T == 0) {
+    if (state_out != nullptr && launch_copy_state((int)B, (int)C, state_in, state_out, st) != cudaSuccess)
+      return RWKV_ERR_CUDA;
+    return RWKV_OK;
+  }
+  if (k == nullptr || v == nullptr || r == nullptr || o == nullptr) return RWKV_ERR_INVALID_ARG;
+  const bool bf16 = dtype == RWKV_BF16;
+  if (!aligned16(k) || !aligned16(v) || !aligned16(r) || !aligned16(o) || (C * (bf16 ? 2 : 4)) % 16 != 0)
+    return RWKV_ERR_UNSUPPORTED;
+  const FwdPlan pl = plan_forward(B, T, C, algo);
+  if (pl.ws_bytes > 0 && (workspace == nullptr || workspace_bytes < pl.ws_bytes)) return RWKV_ERR_WORKSPACE;
+  return run_forward((int)B, (int)T, (int)C, bf16, w, u, k, v, o, state_in, state_out, ckpt, (int)chunk_len, pl,
+                     workspace, st, r);
+}
+
 size_t rwkv_wkv4_backward_workspace_bytes(int64_t B, int64_t T, int64_t C, int64_t chunk_len, int have_ckpt) {
   if (B <= 0 || T <= 0 || C <= 0) return 0;
   if (chunk_len <= 0) chunk_len = kCkLen;
@@ -246,10 +280,17 @@ size_t rwkv_wkv4_backward_workspace_bytes(int64_t B, int64_t T, int64_t C, int64
   return bytes;
 }
 
-rwkv_status rwkv_wkv4_backward(int64_t B, int64_t T, int64_t C, rwkv_dtype dtype, const float* w, const float* u,
-                               const void* k, const void* v, const void* gy, const float* state_in,
-                               const float* ckpt, int64_t chunk_len, void* gk, void* gv, float* gw, float* gu,
-                               void* workspace, size_t workspace_bytes, rwkv_stream_t stream) {
+}  // extern "C"
+
+namespace rwkv {
+namespace {
+
+// The WKV-4 backward, plain (gy given) or receptance-gated (r and go given instead, gr written).
+rwkv_status backward_impl(int64_t B, int64_t T, int64_t C, rwkv_dtype dtype, const float* w, const float* u,
+                          const void* k, const void* v, const void* gy, const void* r, const void* go,
+                          const float* state_in, const float* ckpt, int64_t chunk_len, void* gk, void* gv, void* gr,
+                          float* gw, float* gu, void* workspace, size_t workspace_bytes, rwkv_stream_t stream) {
+  const bool gate = r != nullptr || go != nullptr || gr != nullptr;
   if (!fits_int(B) || !fits_int(T) || !fits_int(C)) return RWKV_ERR_INVALID_ARG;
   if (dtype != RWKV_F32 && dtype != RWKV_BF16) return RWKV_ERR_INVALID_ARG;
   if (chunk_len <= 0 || chunk_len % 16 != 0) return RWKV_ERR_INVALID_ARG;
@@ -262,9 +303,11 @@ rwkv_status rwkv_wkv4_backward(int64_t B, int64_t T, int64_t C, rwkv_dtype dtype
     if (cudaMemsetAsync(gu, 0, C * sizeof(float), st) != cudaSuccess) return RWKV_ERR_CUDA;
     return RWKV_OK;
   }
-  if (k == nullptr || v == nullptr || gy == nullptr || gk == nullptr || gv == nullptr) return RWKV_ERR_INVALID_ARG;
+  if (k == nullptr || v == nullptr || gk == nullptr || gv == nullptr) return RWKV_ERR_INVALID_ARG;
+  if (gate ? (r == nullptr || go == nullptr || gr == nullptr) : gy == nullptr) return RWKV_ERR_INVALID_ARG;
   const bool bf16 = dtype == RWKV_BF16;
-  if (!aligned16(k) || !aligned16(v) || !aligned16(gy) || !aligned16(gk) || !aligned16(gv) ||
+  const bool in_ok = gate ? aligned16(r) && aligned16(go) && aligned16(gr) : aligned16(gy);
+  if (!aligned16(k) || !aligned16(v) || !in_ok || !aligned16(gk) || !aligned16(gv) ||
       (C * (bf16 ? 2 : 4)) % 16 != 0)
     return RWKV_ERR_UNSUPPORTED;
   const size_t need = rwkv_wkv4_backward_workspace_bytes(B, T, C, chunk_len, ckpt != nullptr);
@@ -283,18 +326,21 @@ rwkv_status rwkv_wkv4_backward(int64_t B, int64_t T, int64_t C, rwkv_dtype dtype
   unsigned int* err = device_error_word();
   if (err == nullptr) return RWKV_ERR_CUDA;
   const int box_t = bwd_tile_steps();
-  CUtensorMap mk, mv, mg, mgk, mgv;
+  CUtensorMap mk, mv, mg, mgk, mgv, mo, mgr;
   if (!make_btc_map(&mk, k, bf16, iB, iT, iC, box_t) || !make_btc_map(&mv, v, bf16, iB, iT, iC, box_t) ||
-      !make_btc_map(&mg, gy, bf16, iB, iT, iC, box_t) ||
+      !make_btc_map(&mg, gate ? r : gy, bf16, iB, iT, iC, box_t) ||
       !make_btc_map(&mgk, gk, bf16, iB, iT, iC, bwd_store_steps()) ||
       !make_btc_map(&mgv, gv, bf16, iB, iT, iC, bwd_store_steps()))
+    return RWKV_ERR_CUDA;
+  if (gate && (!make_btc_map(&mo, go, bf16, iB, iT, iC, box_t) ||
+               !make_btc_map(&mgr, gr, bf16, iB, iT, iC, bwd_store_steps())))
     return RWKV_ERR_CUDA;
   Bwd4Params p{};
   p.B = iB;
   p.T = iT;
   p.C = iC;
   p.ctiles = (iC + 31) / 32;
-  p.stages = bwd_stages(bf16, iT);
+  p.stages = bwd_stages(bf16, iT, gate);
   p.w = w;
   p.u = u;
   p.ckpt = ck;
@@ -302,9 +348,34 @@ rwkv_status rwkv_wkv4_backward(int64_t B, int64_t T, int64_t C, rwkv_dtype dtype
   p.gv = gv;
   p.part = part;
   p.err = err;
-  if (launch_wkv4_bwd(bf16, mk, mv, mg, mgk, mgv, p, st) != cudaSuccess) return RWKV_ERR_CUDA;
+  const cudaError_t e = gate ? launch_wkv4_bwd_gated(bf16, mk, mv, mg, mo, mgk, mgv, mgr, p, st)
+                             : launch_wkv4_bwd(bf16, mk, mv, mg, mgk, mgv, p, st);
+  if (e != cudaSuccess) return RWKV_ERR_CUDA;
   if (launch_wkv4_reduce_wu(iB, iC, part, gw, gu, st) != cudaSuccess) return RWKV_ERR_CUDA;
   return RWKV_OK;
+}
+
+}  // namespace
+}  // namespace rwkv
+
+extern "C" {
+
+rwkv_status rwkv_wkv4_backward(int64_t B, int64_t T, int64_t C, rwkv_dtype dtype, const float* w, const float* u,
+                               const void* k, const void* v, const void* gy, const float* state_in,
+                               const float* ckpt, int64_t chunk_len, void* gk, void* gv, float* gw, float* gu,
+                               void* workspace, size_t workspace_bytes, rwkv_stream_t stream) {
+  return backward_impl(B, T, C, dtype, w, u, k, v, gy, nullptr, nullptr, state_in, ckpt, chunk_len, gk, gv,
+                       nullptr, gw, gu, workspace, workspace_bytes, stream);
+}
+
+rwkv_status rwkv_wkv4_backward_gated(int64_t B, int64_t T, int64_t C, rwkv_dtype dtype, const float* w,
+                                     const float* u, const void* k, const void* v, const void* r, const void* go,
+                                     const float* state_in, const float* ckpt, int64_t chunk_len, void* gk, void* gv,
+                                     void* gr, float* gw, float* gu, void* workspace, size_t workspace_bytes,
+                                     rwkv_stream_t stream) {
+  if (r == nullptr && go == nullptr && gr == nullptr) r = k;  // all three missing: rejected below as a gated call
+  return backward_impl(B, T, C, dtype, w, u, k, v, nullptr, r, go, state_in, ckpt, chunk_len, gk, gv, gr, gw, gu,
+                       workspace, workspace_bytes, stream);
 }
 
 rwkv_status rwkv_wkv4_step(int64_t B, int64_t C, rwkv_dtype dtype, const float* w, const float* u, const void* k,

@@ -82,20 +82,27 @@ struct Wkv6Params {
 
 int fwd_tile_steps();
 int fwd_store_steps();
-int fwd_stages(bool bf16, int seg_len);
+int fwd_stages(bool bf16, int seg_len, bool gate = false);
 int bwd_tile_steps();
 int bwd_store_steps();
-int bwd_stages(bool bf16, int T);
+int bwd_stages(bool bf16, int T, bool gate = false);
 // mk, mv: [fwd_tile_steps() x 32] boxes over k, v; my: [fwd_store_steps() x 32] boxes over y
 // (TMA stores; any valid map when p.y is null).
 cudaError_t launch_wkv4_fwd(bool bf16, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& my,
                             const Fwd4Params& p, cudaStream_t st);
+// The receptance-gated forward: also reads r ([fwd_tile_steps() x 32] boxes) and writes σ(r) ⊙ WKV.
+cudaError_t launch_wkv4_fwd_gated(bool bf16, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& my,
+                                  const CUtensorMap& mr, const Fwd4Params& p, cudaStream_t st);
 cudaError_t launch_wkv4_carry(int B, int C, int T, int nseg, int seg_len, const float* w, const float* state_in,
                               float* ws, float* state_out, cudaStream_t st);
 // mk, mv, mgy: [bwd_tile_steps() x 32] boxes over k, v, gy; mgk, mgv: [bwd_store_steps() x 32]
 // boxes over gk, gv (written by TMA stores).
 cudaError_t launch_wkv4_bwd(bool bf16, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mgy,
                             const CUtensorMap& mgk, const CUtensorMap& mgv, const Bwd4Params& p, cudaStream_t st);
+// The receptance-gated backward: mr, mo are [bwd_tile_steps() x 32] boxes over r and go; mgr stores gr.
+cudaError_t launch_wkv4_bwd_gated(bool bf16, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mr,
+                                  const CUtensorMap& mo, const CUtensorMap& mgk, const CUtensorMap& mgv,
+                                  const CUtensorMap& mgr, const Bwd4Params& p, cudaStream_t st);
 cudaError_t launch_wkv4_reduce_wu(int B, int C, const double* part, float* gw, float* gu, cudaStream_t st);
 cudaError_t launch_wkv4_step(bool bf16, int B, int C, const float* w, const float* u, const void* k, const void* v,
                              void* y, const float* state_in, float* state_out, bool vec4, cudaStream_t st);

@@ -39,6 +39,12 @@
 // each element is read once and each gradient written once, without
 // per-element address arithmetic.  Per-lane gw, gu partials are reduced over
 // the batch by a second kernel.
+//
+// Receptance gate (GATE): gradients of L = Σ go_t σ(r_t) WKV_t (the gated
+// output of the same page's time mixing).  r and go replace gy as the third
+// and fourth boxes of a stage; the recompute phase forms gy_t = σ(r_t) go_t and
+// gr_t = go_t WKV_t σ(r_t) (1 - σ(r_t)) from the WKV_t it recomputes anyway,
+// writes gr over the consumed r rows, and the chunk's gr leaves with gk and gv.
 #include "launch.h"
 #include "wkv_common.cuh"
 
@@ -59,10 +65,12 @@ struct RSumm {  // a chunk's own reverse sums from a zero carry, at scale 2^q
 };
 
 // Phase A: forward recompute of one chunk from its checkpoint state (a, b) at
-// scale 2^q, keeping e_t, G_t = gy_t / d_t, y_t and b_{t-1}.
-template <typename T, bool FULL>
-__device__ __forceinline__ void chunk_recompute(const T* ks, const T* vs, const T* gs, int cnt, float qf, float U,
-                                                float lh, float ll, float a, float b, float (&E)[kL],
+// scale 2^q, keeping e_t, G_t = gy_t / d_t, y_t and b_{t-1}.  With GATE, gs
+// holds the r rows and os the go rows: gy_t = σ(r_t) go_t, and gr_t is written
+// over r_t.
+template <typename T, bool FULL, bool GATE>
+__device__ __forceinline__ void chunk_recompute(const T* ks, const T* vs, T* gs, const T* os, int cnt, float qf,
+                                                float U, float lh, float ll, float a, float b, float (&E)[kL],
                                                 float (&G)[kL], float (&Y)[kL], float (&BP)[kL]) {
 #pragma unroll
   for (int j = 0; j < kL; ++j) {
@@ -74,7 +82,16 @@ __device__ __forceinline__ void chunk_recompute(const T* ks, const T* vs, const 
       const float rd = rcp_approx(d);
       const bool ok = d >= kMinDen;  // else no history and e^{u+k} underflowed: WKV = v locally
       Y[j] = ok ? fmaf(eu, vj, a) * rd : vj;
-      G[j] = ok ? IO<T>::to_f(gs[j * 32]) * rd : 0.f;
+      float gy;
+      if constexpr (GATE) {
+        const float sg = sigmoid(IO<T>::to_f(gs[j * 32]));
+        const float go = IO<T>::to_f(os[j * 32]);
+        gy = sg * go;
+        gs[j * 32] = IO<T>::from_f(go * Y[j] * (sg - sg * sg));
+      } else {
+        gy = IO<T>::to_f(gs[j * 32]);
+      }
+      G[j] = ok ? gy * rd : 0.f;
       E[j] = e;
       BP[j] = b;
       a = decay_add(a, e * vj, lh, ll);
@@ -132,18 +149,22 @@ struct RCarry {  // reverse carry at a chunk boundary, per lane (see phase C)
   int p;
 };
 
-template <typename T>
+// mg: gy boxes, or with GATE r boxes; mo: go boxes (GATE only); mgr: gr store boxes (GATE only).
+template <typename T, bool GATE>
 __global__ void __launch_bounds__(kW * 32, 4) wkv4_bwd_kernel(const __grid_constant__ CUtensorMap mk,
                                                               const __grid_constant__ CUtensorMap mv,
                                                               const __grid_constant__ CUtensorMap mg,
                                                               const __grid_constant__ CUtensorMap mgk,
                                                               const __grid_constant__ CUtensorMap mgv,
+                                                              const __grid_constant__ CUtensorMap mo,
+                                                              const __grid_constant__ CUtensorMap mgr,
                                                               const Bwd4Params p) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   constexpr uint32_t kBoxElems = kTile * 32;
   constexpr uint32_t kBoxBytes = kBoxElems * sizeof(T);
-  T* tiles = reinterpret_cast<T*>(smem_raw);  // [stages][k|v|gy][kTile][32]
-  RSumm* rs = reinterpret_cast<RSumm*>(smem_raw + (size_t)p.stages * 3 * kBoxBytes);  // [2][kW][32]
+  constexpr int kNB = GATE ? 4 : 3;  // boxes per stage: k, v, gy  or  k, v, r, go
+  T* tiles = reinterpret_cast<T*>(smem_raw);  // [stages][k|v|gy or k|v|r|go][kTile][32]
+  RSumm* rs = reinterpret_cast<RSumm*>(smem_raw + (size_t)p.stages * kNB * kBoxBytes);  // [2][kW][32]
   RCarry* cslot = reinterpret_cast<RCarry*>(rs + 2 * kW * 32);                        // [2][32]
   uint64_t* bars = reinterpret_cast<uint64_t*>(cslot + 2 * 32);
   int* abort_flag = reinterpret_cast<int*>(bars + p.stages);
@@ -161,15 +182,17 @@ __global__ void __launch_bounds__(kW * 32, 4) wkv4_bwd_kernel(const __grid_const
     prefetch_tensormap(&mk);
     prefetch_tensormap(&mv);
     prefetch_tensormap(&mg);
+    if constexpr (GATE) prefetch_tensormap(&mo);
     for (int s = 0; s < p.stages; ++s) mbar_init(&bars[s], 1);
     fence_mbar_init();
     const int pre = min(p.stages, ntile);
     for (int s = 0; s < pre; ++s) {
       const int tc = (ntile - 1 - s) * kTile;
-      mbar_arrive_expect_tx(&bars[s], 3 * kBoxBytes);
-      tma_load_3d(tiles + (size_t)(3 * s) * kBoxElems, &mk, &bars[s], ct * 32, tc, bb);
-      tma_load_3d(tiles + (size_t)(3 * s + 1) * kBoxElems, &mv, &bars[s], ct * 32, tc, bb);
-      tma_load_3d(tiles + (size_t)(3 * s + 2) * kBoxElems, &mg, &bars[s], ct * 32, tc, bb);
+      mbar_arrive_expect_tx(&bars[s], kNB * kBoxBytes);
+      tma_load_3d(tiles + (size_t)(kNB * s) * kBoxElems, &mk, &bars[s], ct * 32, tc, bb);
+      tma_load_3d(tiles + (size_t)(kNB * s + 1) * kBoxElems, &mv, &bars[s], ct * 32, tc, bb);
+      tma_load_3d(tiles + (size_t)(kNB * s + 2) * kBoxElems, &mg, &bars[s], ct * 32, tc, bb);
+      if constexpr (GATE) tma_load_3d(tiles + (size_t)(kNB * s + 3) * kBoxElems, &mo, &bars[s], ct * 32, tc, bb);
     }
   }
   if (warp == 0) cslot[32 + lane] = RCarry{0.0, 0.0, 0.f, 0};  // nothing flows back from after the end
@@ -200,11 +223,13 @@ __global__ void __launch_bounds__(kW * 32, 4) wkv4_bwd_kernel(const __grid_const
       st = load_state(ck[0], ck[plane], ck[2 * plane]);
     }
     if (!mbar_wait_bounded(&bars[s], ph, p.err)) *abort_flag = 1;
-    T* const kw = tiles + (size_t)(3 * s) * kBoxElems + warp * kL * 32;  // this warp's [16][32] rows
+    T* const kw = tiles + (size_t)(kNB * s) * kBoxElems + warp * kL * 32;  // this warp's [16][32] rows
     T* const vw = kw + kBoxElems;
+    T* const gw_rows = vw + kBoxElems;  // gy rows, or with GATE the r rows that receive gr
     T* const ks = kw + lane;
     T* const vs = vw + lane;
-    const T* gs = vs + kBoxElems;
+    T* const gs = gw_rows + lane;
+    const T* os = gs + kBoxElems;  // go rows (GATE only)
 
     // A. forward recompute of the chunk at one scale 2^q: the forward wrote the
     //    checkpoint at the chunk's scale (at least every k log2 e of the chunk,
@@ -212,9 +237,11 @@ __global__ void __launch_bounds__(kW * 32, 4) wkv4_bwd_kernel(const __grid_const
     float E[kL], G[kL], Y[kL], BP[kL];
     const int q = st.p;
     if (cnt == kL)
-      chunk_recompute<T, true>(ks, vs, gs, cnt, (float)q, U, lh, ll, (float)st.a, (float)st.b, E, G, Y, BP);
+      chunk_recompute<T, true, GATE>(ks, vs, gs, os, cnt, (float)q, U, lh, ll, (float)st.a, (float)st.b, E, G, Y,
+                                     BP);
     else if (cnt > 0)
-      chunk_recompute<T, false>(ks, vs, gs, cnt, (float)q, U, lh, ll, (float)st.a, (float)st.b, E, G, Y, BP);
+      chunk_recompute<T, false, GATE>(ks, vs, gs, os, cnt, (float)q, U, lh, ll, (float)st.a, (float)st.b, E, G,
+                                      Y, BP);
 
     // B. the chunk's own reverse sums
     float la = 0.f, lg = 0.f, ye = 0.f;
@@ -232,10 +259,11 @@ __global__ void __launch_bounds__(kW * 32, 4) wkv4_bwd_kernel(const __grid_const
       const int sp = (i - 1) % p.stages;
       const int tc = (ntile - 1 - (i - 1 + p.stages)) * kTile;
       fence_proxy_async();
-      mbar_arrive_expect_tx(&bars[sp], 3 * kBoxBytes);
-      tma_load_3d(tiles + (size_t)(3 * sp) * kBoxElems, &mk, &bars[sp], ct * 32, tc, bb);
-      tma_load_3d(tiles + (size_t)(3 * sp + 1) * kBoxElems, &mv, &bars[sp], ct * 32, tc, bb);
-      tma_load_3d(tiles + (size_t)(3 * sp + 2) * kBoxElems, &mg, &bars[sp], ct * 32, tc, bb);
+      mbar_arrive_expect_tx(&bars[sp], kNB * kBoxBytes);
+      tma_load_3d(tiles + (size_t)(kNB * sp) * kBoxElems, &mk, &bars[sp], ct * 32, tc, bb);
+      tma_load_3d(tiles + (size_t)(kNB * sp + 1) * kBoxElems, &mv, &bars[sp], ct * 32, tc, bb);
+      tma_load_3d(tiles + (size_t)(kNB * sp + 2) * kBoxElems, &mg, &bars[sp], ct * 32, tc, bb);
+      if constexpr (GATE) tma_load_3d(tiles + (size_t)(kNB * sp + 3) * kBoxElems, &mo, &bars[sp], ct * 32, tc, bb);
     }
 
     // C. fold the carries of the later chunks.  A carry is (α~ out of a chunk,
@@ -289,6 +317,7 @@ __global__ void __launch_bounds__(kW * 32, 4) wkv4_bwd_kernel(const __grid_const
       if (lane == 0) {
         tma_store_3d(&mgk, kw, ct * 32, ts, bb);
         tma_store_3d(&mgv, vw, ct * 32, ts, bb);
+        if constexpr (GATE) tma_store_3d(&mgr, gw_rows, ct * 32, ts, bb);
         bulk_commit();
       }
     }
@@ -327,21 +356,23 @@ __global__ void wkv4_reduce_wu_kernel(int B, int C, const double* __restrict__ p
   gu[c] = (float)su;
 }
 
-template <typename T>
+template <typename T, bool GATE>
 size_t bwd_smem_bytes(int stages) {
-  return (size_t)stages * 3 * kTile * 32 * sizeof(T) + 2 * kW * 32 * sizeof(RSumm) + 2 * 32 * sizeof(RCarry) +
-         (size_t)stages * 8 + 16;
+  return (size_t)stages * (GATE ? 4 : 3) * kTile * 32 * sizeof(T) + 2 * kW * 32 * sizeof(RSumm) +
+         2 * 32 * sizeof(RCarry) + (size_t)stages * 8 + 16;
 }
 
-template <typename T>
+template <typename T, bool GATE>
 cudaError_t launch_bwd_t(const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mg, const CUtensorMap& mgk,
-                         const CUtensorMap& mgv, const Bwd4Params& p, cudaStream_t st) {
-  const size_t smem = bwd_smem_bytes<T>(p.stages);
+                         const CUtensorMap& mgv, const CUtensorMap& mo, const CUtensorMap& mgr, const Bwd4Params& p,
+                         cudaStream_t st) {
+  const size_t smem = bwd_smem_bytes<T, GATE>(p.stages);
   static unsigned device_mask = 0;
-  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(wkv4_bwd_kernel<T>), (int)smem, &device_mask);
+  cudaError_t e =
+      ensure_smem_attr(reinterpret_cast<const void*>(wkv4_bwd_kernel<T, GATE>), (int)smem, &device_mask);
   if (e != cudaSuccess) return e;
   const long long nblk = (long long)p.ctiles * p.B;
-  wkv4_bwd_kernel<T><<<(unsigned)nblk, kW * 32, smem, st>>>(mk, mv, mg, mgk, mgv, p);
+  wkv4_bwd_kernel<T, GATE><<<(unsigned)nblk, kW * 32, smem, st>>>(mk, mv, mg, mgk, mgv, mo, mgr, p);
   return cudaGetLastError();
 }
 
@@ -351,16 +382,25 @@ int bwd_tile_steps() { return kTile; }
 
 int bwd_store_steps() { return kL; }
 
-int bwd_stages(bool bf16, int T) {
-  const int want = bf16 ? 4 : 2;  // 48 KB of boxes keeps four CTAs per SM
+int bwd_stages(bool bf16, int T, bool gate) {
+  // 48 KB of k, v, gy boxes keeps four CTAs per SM; the gate's four boxes per stage take 64 KB (fp32) in two
+  // stages, three CTAs per SM
+  const int want = gate ? (bf16 ? 3 : 2) : (bf16 ? 4 : 2);
   const int ntile = (T + kTile - 1) / kTile;
   return max(2, min(want, ntile));
 }
 
 cudaError_t launch_wkv4_bwd(bool bf16, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mg,
                             const CUtensorMap& mgk, const CUtensorMap& mgv, const Bwd4Params& p, cudaStream_t st) {
-  return bf16 ? launch_bwd_t<__nv_bfloat16>(mk, mv, mg, mgk, mgv, p, st)
-              : launch_bwd_t<float>(mk, mv, mg, mgk, mgv, p, st);
+  return bf16 ? launch_bwd_t<__nv_bfloat16, false>(mk, mv, mg, mgk, mgv, mk, mgk, p, st)
+              : launch_bwd_t<float, false>(mk, mv, mg, mgk, mgv, mk, mgk, p, st);
+}
+
+cudaError_t launch_wkv4_bwd_gated(bool bf16, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mr,
+                                  const CUtensorMap& mo, const CUtensorMap& mgk, const CUtensorMap& mgv,
+                                  const CUtensorMap& mgr, const Bwd4Params& p, cudaStream_t st) {
+  return bf16 ? launch_bwd_t<__nv_bfloat16, true>(mk, mv, mr, mgk, mgv, mo, mgr, p, st)
+              : launch_bwd_t<float, true>(mk, mv, mr, mgk, mgv, mo, mgr, p, st);
 }
 
 cudaError_t launch_wkv4_reduce_wu(int B, int C, const double* part, float* gw, float* gu, cudaStream_t st) {

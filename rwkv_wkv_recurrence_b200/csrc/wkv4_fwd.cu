@@ -19,6 +19,12 @@
 // k and v arrive in [64 x 32] boxes through a multi-stage TMA pipeline
 // without multicast, so every input element is read from HBM once.
 //
+// Receptance gate (GATE).  The time-mixing output of the same page is
+// o_t = W_o (σ(r_t) ⊙ WKV_t) ((2) and (4) Receptance Gating); W_o is a GEMM
+// outside the operator, σ(r) ⊙ WKV is fused here: r arrives as a third box
+// per stage and the rescan writes σ(r_t) WKV_t instead of WKV_t, so the gate
+// costs one more input stream instead of a separate pass over y and r.
+//
 // Precision.  Steps inside a segment run in fp32 with the decay applied as
 // e^{-w} = lh + ll (hi and lo fp32 parts), one power-of-two scale per segment;
 // the running state carried from segment to segment is fp64.  So fp32 rounding
@@ -71,9 +77,10 @@ __device__ __forceinline__ void seg_summary(const T* ks, const T* vs, int cnt, f
 // Phase 3 of one segment: rescan from the true state (a, b) at the segment's
 // scale, weights E * f, writing y_j to ys[j * 32] (the segment's k rows in
 // shared memory, which phase 1 has consumed).
-template <typename T, bool FULL>
-__device__ __forceinline__ void seg_output(const T* vs, int cnt, const float (&E)[kL], float f, float U, float a,
-                                           float b, float lh, float ll, T* ys) {
+// With GATE, rs holds the segment's r rows and y_j is multiplied by σ(r_j).
+template <typename T, bool FULL, bool GATE>
+__device__ __forceinline__ void seg_output(const T* vs, const T* rs, int cnt, const float (&E)[kL], float f,
+                                           float U, float a, float b, float lh, float ll, T* ys) {
 #pragma unroll
   for (int j = 0; j < kL; ++j) {
     if (FULL || j < cnt) {
@@ -82,7 +89,8 @@ __device__ __forceinline__ void seg_output(const T* vs, int cnt, const float (&E
       const float vj = IO<T>::to_f(vs[j * 32]);
       const float d = b + eu;
       const float n = fmaf(eu, vj, a);
-      const float y = d >= kMinDen ? n * rcp_approx(d) : vj;
+      float y = d >= kMinDen ? n * rcp_approx(d) : vj;
+      if constexpr (GATE) y *= sigmoid(IO<T>::to_f(rs[j * 32]));
       ys[j * 32] = IO<T>::from_f(y);
       a = decay_add(a, e * vj, lh, ll);
       b = decay_add(b, e, lh, ll);
@@ -95,16 +103,18 @@ struct CarrySlot {  // CTA running state at a tile boundary, per lane
   int p, pad;
 };
 
-template <typename T>
+template <typename T, bool GATE>
 __global__ void __launch_bounds__(kW * 32, 4) wkv4_fwd_kernel(const __grid_constant__ CUtensorMap mk,
                                                               const __grid_constant__ CUtensorMap mv,
                                                               const __grid_constant__ CUtensorMap my,
+                                                              const __grid_constant__ CUtensorMap mr,
                                                               const Fwd4Params p) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   constexpr uint32_t kBoxElems = kTile * 32;
   constexpr uint32_t kBoxBytes = kBoxElems * sizeof(T);
-  T* tiles = reinterpret_cast<T*>(smem_raw);  // [stages][k|v][kTile][32]
-  Summ* summ = reinterpret_cast<Summ*>(smem_raw + (size_t)p.stages * 2 * kBoxBytes);  // [2][kW][32]
+  constexpr int kNB = GATE ? 3 : 2;  // boxes per stage: k, v (, r)
+  T* tiles = reinterpret_cast<T*>(smem_raw);  // [stages][k|v(|r)][kTile][32]
+  Summ* summ = reinterpret_cast<Summ*>(smem_raw + (size_t)p.stages * kNB * kBoxBytes);  // [2][kW][32]
   CarrySlot* cslot = reinterpret_cast<CarrySlot*>(summ + 2 * kW * 32);                // [2][32]
   uint64_t* bars = reinterpret_cast<uint64_t*>(cslot + 2 * 32);                         // [stages]
   int* abort_flag = reinterpret_cast<int*>(bars + p.stages);
@@ -126,13 +136,16 @@ __global__ void __launch_bounds__(kW * 32, 4) wkv4_fwd_kernel(const __grid_const
     *abort_flag = 0;
     prefetch_tensormap(&mk);
     prefetch_tensormap(&mv);
+    if constexpr (GATE) prefetch_tensormap(&mr);
     for (int s = 0; s < p.stages; ++s) mbar_init(&bars[s], 1);
     fence_mbar_init();
     const int pre = min(p.stages, ntile);
     for (int s = 0; s < pre; ++s) {
-      mbar_arrive_expect_tx(&bars[s], 2 * kBoxBytes);
-      tma_load_3d(tiles + (size_t)(2 * s) * kBoxElems, &mk, &bars[s], ct * 32, t0 + s * kTile, bb);
-      tma_load_3d(tiles + (size_t)(2 * s + 1) * kBoxElems, &mv, &bars[s], ct * 32, t0 + s * kTile, bb);
+      mbar_arrive_expect_tx(&bars[s], kNB * kBoxBytes);
+      tma_load_3d(tiles + (size_t)(kNB * s) * kBoxElems, &mk, &bars[s], ct * 32, t0 + s * kTile, bb);
+      tma_load_3d(tiles + (size_t)(kNB * s + 1) * kBoxElems, &mv, &bars[s], ct * 32, t0 + s * kTile, bb);
+      if constexpr (GATE)
+        tma_load_3d(tiles + (size_t)(kNB * s + 2) * kBoxElems, &mr, &bars[s], ct * 32, t0 + s * kTile, bb);
     }
   }
 
@@ -166,8 +179,9 @@ __global__ void __launch_bounds__(kW * 32, 4) wkv4_fwd_kernel(const __grid_const
     const int tb = t0 + i * kTile;
     const int ts = tb + warp * kL;
     const int cnt = max(0, min(kL, t1 - ts));
-    const T* ks = tiles + (size_t)(2 * s) * kBoxElems + warp * kL * 32 + lane;
+    const T* ks = tiles + (size_t)(kNB * s) * kBoxElems + warp * kL * 32 + lane;
     const T* vs = ks + kBoxElems;
+    const T* rs = vs + kBoxElems;  // the r rows (GATE only)
 
     // 1. this warp's segment from a zero state
     float E[kL], kmax = -INFINITY, la = 0.f, lb = 0.f;
@@ -187,9 +201,10 @@ __global__ void __launch_bounds__(kW * 32, 4) wkv4_fwd_kernel(const __grid_const
       const int sp = (i - 1) % p.stages;
       const int tn = t0 + (i - 1 + p.stages) * kTile;
       fence_proxy_async();
-      mbar_arrive_expect_tx(&bars[sp], 2 * kBoxBytes);
-      tma_load_3d(tiles + (size_t)(2 * sp) * kBoxElems, &mk, &bars[sp], ct * 32, tn, bb);
-      tma_load_3d(tiles + (size_t)(2 * sp + 1) * kBoxElems, &mv, &bars[sp], ct * 32, tn, bb);
+      mbar_arrive_expect_tx(&bars[sp], kNB * kBoxBytes);
+      tma_load_3d(tiles + (size_t)(kNB * sp) * kBoxElems, &mk, &bars[sp], ct * 32, tn, bb);
+      tma_load_3d(tiles + (size_t)(kNB * sp + 1) * kBoxElems, &mv, &bars[sp], ct * 32, tn, bb);
+      if constexpr (GATE) tma_load_3d(tiles + (size_t)(kNB * sp + 2) * kBoxElems, &mr, &bars[sp], ct * 32, tn, bb);
     }
 
     // 2. fold: the state at this warp's segment start is the running state
@@ -226,9 +241,9 @@ __global__ void __launch_bounds__(kW * 32, 4) wkv4_fwd_kernel(const __grid_const
         const float f = pow2f_neg(p1 - q);
         T* const yw = const_cast<T*>(ks) - lane;  // this warp's [16][32] k rows
         if (cnt == kL)
-          seg_output<T, true>(vs, cnt, E, f, U, (float)sc.a, (float)sc.b, lh, ll, yw + lane);
+          seg_output<T, true, GATE>(vs, rs, cnt, E, f, U, (float)sc.a, (float)sc.b, lh, ll, yw + lane);
         else
-          seg_output<T, false>(vs, cnt, E, f, U, (float)sc.a, (float)sc.b, lh, ll, yw + lane);
+          seg_output<T, false, GATE>(vs, rs, cnt, E, f, U, (float)sc.a, (float)sc.b, lh, ll, yw + lane);
         // y of the segment as one [16 x 32] box (rows past T and channels past C are clipped)
         fence_proxy_async();
         __syncwarp();
@@ -276,21 +291,22 @@ __global__ void wkv4_carry_kernel(int B, int C, int T, int nseg, int seg_len, co
   if (state_out != nullptr) store_state(st, &state_out[i], &state_out[plane + i], &state_out[2 * plane + i]);
 }
 
-template <typename T>
+template <typename T, bool GATE>
 size_t fwd_smem_bytes(int stages) {
-  return (size_t)stages * 2 * kTile * 32 * sizeof(T) + 2 * kW * 32 * sizeof(Summ) + 2 * 32 * sizeof(CarrySlot) +
-         (size_t)stages * 8 + 16;
+  return (size_t)stages * (GATE ? 3 : 2) * kTile * 32 * sizeof(T) + 2 * kW * 32 * sizeof(Summ) +
+         2 * 32 * sizeof(CarrySlot) + (size_t)stages * 8 + 16;
 }
 
-template <typename T>
-cudaError_t launch_fwd_t(const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& my, const Fwd4Params& p,
-                         cudaStream_t st) {
-  const size_t smem = fwd_smem_bytes<T>(p.stages);
+template <typename T, bool GATE>
+cudaError_t launch_fwd_t(const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& my, const CUtensorMap& mr,
+                         const Fwd4Params& p, cudaStream_t st) {
+  const size_t smem = fwd_smem_bytes<T, GATE>(p.stages);
   static unsigned device_mask = 0;
-  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(wkv4_fwd_kernel<T>), (int)smem, &device_mask);
+  cudaError_t e =
+      ensure_smem_attr(reinterpret_cast<const void*>(wkv4_fwd_kernel<T, GATE>), (int)smem, &device_mask);
   if (e != cudaSuccess) return e;
   const long long nblk = (long long)p.ctiles * p.B * p.nseg;
-  wkv4_fwd_kernel<T><<<(unsigned)nblk, kW * 32, smem, st>>>(mk, mv, my, p);
+  wkv4_fwd_kernel<T, GATE><<<(unsigned)nblk, kW * 32, smem, st>>>(mk, mv, my, mr, p);
   return cudaGetLastError();
 }
 
@@ -300,16 +316,24 @@ int fwd_tile_steps() { return kTile; }
 
 int fwd_store_steps() { return kL; }
 
-int fwd_stages(bool bf16, int seg_len) {
-  // three stages of fp32 boxes (48 KB) keep four CTAs per SM; bf16 boxes are half as big
-  const int want = bf16 ? 6 : 3;
+int fwd_stages(bool bf16, int seg_len, bool gate) {
+  // three stages of fp32 k, v boxes (48 KB) keep four CTAs per SM; bf16 boxes are half as big; with the
+  // gate's r box, two stages (fp32) or four (bf16) stay within the same 48 KB
+  const int want = gate ? (bf16 ? 4 : 2) : (bf16 ? 6 : 3);
   const int ntile = (seg_len + kTile - 1) / kTile;
   return max(2, min(want, ntile));
 }
 
 cudaError_t launch_wkv4_fwd(bool bf16, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& my,
                             const Fwd4Params& p, cudaStream_t st) {
-  return bf16 ? launch_fwd_t<__nv_bfloat16>(mk, mv, my, p, st) : launch_fwd_t<float>(mk, mv, my, p, st);
+  return bf16 ? launch_fwd_t<__nv_bfloat16, false>(mk, mv, my, mk, p, st)
+              : launch_fwd_t<float, false>(mk, mv, my, mk, p, st);
+}
+
+cudaError_t launch_wkv4_fwd_gated(bool bf16, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& my,
+                                  const CUtensorMap& mr, const Fwd4Params& p, cudaStream_t st) {
+  return bf16 ? launch_fwd_t<__nv_bfloat16, true>(mk, mv, my, mr, p, st)
+              : launch_fwd_t<float, true>(mk, mv, my, mr, p, st);
 }
 
 cudaError_t launch_wkv4_carry(int B, int C, int T, int nseg, int seg_len, const float* w, const float* state_in,

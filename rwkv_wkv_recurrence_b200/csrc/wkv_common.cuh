@@ -114,6 +114,10 @@ __device__ __forceinline__ float rcp_approx(float x) {
   return y;
 }
 
+// Logistic sigmoid 1 / (1 + e^{-x}) (the receptance gate); saturates to 0 and 1
+// without NaN: e^{-x} = inf gives 0, e^{-x} = 0 gives 1.
+__device__ __forceinline__ float sigmoid(float x) { return rcp_approx(1.f + __expf(-x)); }
+
 // A WKV denominator too small to divide by: it is below FLT_MIN only when a
 // token arrives with no history and its own weight e^{u+k} underflowed at the
 // segment's scale, where the ratio is v itself.

@@ -122,6 +122,27 @@ def test_validation_before_any_cuda_work():
     assert h.rwkv_wkv5_step(2, 3, 64, fake, fake, fake, fake, fake, fake, P(0x1008), fake, None) == 2
     assert h.rwkv_wkv5_step(-2, 3, 64, fake, fake, fake, fake, fake, fake, None, fake, None) == 1
     assert h.rwkv_wkv5_step(0, 3, 64, fake, fake, fake, fake, fake, fake, None, fake, None) == 0
+    # gated WKV-4: r and o required and aligned; the backward needs r, go and gr together
+    assert h.rwkv_wkv4_forward_gated(1, 4, 4, 0, fake, fake, fake, fake, None, fake, None, None, None, 16, 0,
+                                     None, 0, None) == 1
+    assert h.rwkv_wkv4_forward_gated(1, 4, 4, 0, fake, fake, fake, fake, fake, None, None, None, None, 16, 0,
+                                     None, 0, None) == 1
+    assert h.rwkv_wkv4_forward_gated(1, 4, 4, 0, fake, fake, fake, fake, P(0x1004), fake, None, None, None, 16,
+                                     0, None, 0, None) == 2
+    assert h.rwkv_wkv4_forward_gated(-1, 4, 4, 0, fake, fake, fake, fake, fake, fake, None, None, None, 16, 0,
+                                     None, 0, None) == 1
+    assert h.rwkv_wkv4_forward_gated(0, 4, 4, 0, fake, fake, fake, fake, fake, fake, None, None, None, 16, 0,
+                                     None, 0, None) == 0
+    assert h.rwkv_wkv4_backward_gated(1, 4, 4, 0, fake, fake, fake, fake, None, fake, None, fake, 16, fake,
+                                      fake, fake, fake, fake, fake, 1 << 20, None) == 1
+    assert h.rwkv_wkv4_backward_gated(1, 4, 4, 0, fake, fake, fake, fake, fake, fake, None, fake, 16, fake,
+                                      fake, None, fake, fake, fake, 1 << 20, None) == 1
+    assert h.rwkv_wkv4_backward_gated(1, 4, 4, 0, fake, fake, fake, fake, None, None, None, fake, 16, fake,
+                                      fake, None, fake, fake, fake, 1 << 20, None) == 1
+    assert h.rwkv_wkv4_backward_gated(1, 4, 4, 0, fake, fake, fake, fake, fake, fake, None, fake, 16, fake,
+                                      fake, P(0x1004), fake, fake, fake, 1 << 20, None) == 2
+    assert h.rwkv_wkv4_backward_gated(1, 4, 4, 0, fake, fake, fake, fake, fake, fake, None, fake, 16, fake,
+                                      fake, fake, fake, fake, None, 0, None) == 3
     # WKV-6 forward: only N = 64; omega required and 16-byte aligned (TMA); T = 0 without s_out is a no-op
     assert h.rwkv_wkv6_forward(1, 4, 2, 32, fake, fake, fake, fake, fake, fake, None, None, None, 0, None) == 2
     assert h.rwkv_wkv6_forward(1, 4, 2, 64, fake, fake, fake, None, fake, fake, None, None, None, 0, None) == 1
