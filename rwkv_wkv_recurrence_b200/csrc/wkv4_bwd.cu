@@ -80,7 +80,7 @@ __device__ __forceinline__ void chunk_recompute(const T* ks, const T* vs, T* gs,
       const float vj = IO<T>::to_f(vs[j * 32]);
       const float d = b + eu;
       const float rd = rcp_approx(d);
-      const bool ok = d >= kMinDen;  // else no history and e^{u+k} underflowed: WKV = v locally
+      const bool ok = !(d < kMinDen);  // else no history and e^{u+k} underflowed: WKV = v locally (NaN: ok)
       Y[j] = ok ? fmaf(eu, vj, a) * rd : vj;
       float gy;
       if constexpr (GATE) {

@@ -89,7 +89,7 @@ __device__ __forceinline__ void seg_output(const T* vs, const T* rs, int cnt, co
       const float vj = IO<T>::to_f(vs[j * 32]);
       const float d = b + eu;
       const float n = fmaf(eu, vj, a);
-      float y = d >= kMinDen ? n * rcp_approx(d) : vj;
+      float y = !(d < kMinDen) ? n * rcp_approx(d) : vj;  // a NaN d propagates
       if constexpr (GATE) y *= sigmoid(IO<T>::to_f(rs[j * 32]));
       ys[j * 32] = IO<T>::from_f(y);
       a = decay_add(a, e * vj, lh, ll);

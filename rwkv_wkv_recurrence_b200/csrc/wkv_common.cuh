@@ -120,7 +120,8 @@ __device__ __forceinline__ float sigmoid(float x) { return rcp_approx(1.f + __ex
 
 // A WKV denominator too small to divide by: it is below FLT_MIN only when a
 // token arrives with no history and its own weight e^{u+k} underflowed at the
-// segment's scale, where the ratio is v itself.
+// segment's scale, where the ratio is v itself.  The kernels test !(d < kMinDen)
+// so that a NaN denominator (a NaN input upstream) still divides and propagates.
 constexpr float kMinDen = 1.17549435e-38f;
 
 // ---------------------------------------------------------------- I/O types
@@ -312,7 +313,7 @@ __device__ __forceinline__ float wkv4_step_careful(float& a, float& b, float& p,
   const float eu = e * L.U;
   const float d = b + eu;
   const float n = fmaf(eu, vt, a);
-  const float y = (d >= kMinDen) ? n * rcp_approx(d) : vt;
+  const float y = !(d < kMinDen) ? n * rcp_approx(d) : vt;  // a NaN d propagates
   a = fmaf(L.lam, a, fmaf(L.lam_lo, a, e * vt));
   b = fmaf(L.lam, b, fmaf(L.lam_lo, b, e));
   return y;
