@@ -44,23 +44,62 @@ def _peaks():
         return 6650.0, "fallback"
 
 
+def _gpu_id(local):
+    """The UUID of CUDA device ``local`` ("GPU-..."), which NVML and nvidia-smi
+    accept whatever CUDA_VISIBLE_DEVICES renumbers; the index if unknown."""
+    try:
+        import torch
+
+        u = torch.cuda.get_device_properties(local).uuid
+        return "GPU-" + str(u)
+    except Exception:
+        return local
+
+
 class ClockSampler:
-    """Polls nvidia-smi (one query at a time, so nothing is lost to output
-    buffering) for SM clocks and throttle reasons while the benchmark runs."""
+    """Samples SM clocks and throttle reasons while the benchmark runs (read only).
+
+    NVML (the driver's management library, through nvidia_ml_py) answers in
+    microseconds, so even a timed region of a few milliseconds holds many
+    samples; without it, nvidia-smi is polled one query at a time."""
 
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
     NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    # NVML clocks-event reason bits for the names above
+    NVML_BITS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20, "sw_power_cap": 0x4}
 
-    def __init__(self, index: int, period: float = 0.05):
-        self.index = index
+    def __init__(self, index, period: float = 0.05):
+        self.index = _gpu_id(index)  # the device's UUID where torch reports one, else its index
         self.period = period
         self.samples = []  # (time, sm_mhz, max_mhz, [reasons])
         self._stop = threading.Event()
         self.window = None
+        self.source = None
 
-    def _poll(self):
+    def _poll_nvml(self):
+        import pynvml
+
+        pynvml.nvmlInit()
+        try:
+            h = (pynvml.nvmlDeviceGetHandleByUUID(self.index) if isinstance(self.index, str)
+                 else pynvml.nvmlDeviceGetHandleByIndex(self.index))
+            sm_max = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            get_reasons = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+            self.source = "nvml"
+            while not self._stop.is_set():
+                sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+                bits = get_reasons(h)
+                reasons = [n for n, b in self.NVML_BITS.items() if bits & b]
+                self.samples.append((time.perf_counter(), float(sm), float(sm_max), reasons))
+                self._stop.wait(0.002)
+        finally:
+            pynvml.nvmlShutdown()
+
+    def _poll_smi(self):
+        self.source = "nvidia-smi"
         while not self._stop.is_set():
             try:
                 out = subprocess.run(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
@@ -74,9 +113,19 @@ class ClockSampler:
                 return
             self._stop.wait(self.period)
 
+    def _poll(self):
+        try:
+            self._poll_nvml()
+        except Exception:
+            if not self.samples:
+                self._poll_smi()
+
     def __enter__(self):
         self.thread = threading.Thread(target=self._poll, daemon=True)
         self.thread.start()
+        t_end = time.perf_counter() + 2.0  # the first sample before anything is timed
+        while not self.samples and self.thread.is_alive() and time.perf_counter() < t_end:
+            time.sleep(0.001)
         return self
 
     def mark(self, t0, t1):
@@ -98,7 +147,7 @@ class ClockSampler:
         sm = sorted(x[1] for x in chosen)
         reasons = sorted({r for x in chosen for r in x[3]})
         return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": chosen[-1][2], "reasons": reasons,
-                "samples": len(chosen), "window": where}
+                "samples": len(chosen), "window": where, "source": self.source}
 
 
 # kernel name in profiles/traffic.json -> prefix of the source files it is built from
