@@ -286,11 +286,10 @@ namespace rwkv {
 namespace {
 
 // The WKV-4 backward, plain (gy given) or receptance-gated (r and go given instead, gr written).
-rwkv_status backward_impl(int64_t B, int64_t T, int64_t C, rwkv_dtype dtype, const float* w, const float* u,
-                          const void* k, const void* v, const void* gy, const void* r, const void* go,
+rwkv_status backward_impl(bool gate, int64_t B, int64_t T, int64_t C, rwkv_dtype dtype, const float* w,
+                          const float* u, const void* k, const void* v, const void* gy, const void* r, const void* go,
                           const float* state_in, const float* ckpt, int64_t chunk_len, void* gk, void* gv, void* gr,
                           float* gw, float* gu, void* workspace, size_t workspace_bytes, rwkv_stream_t stream) {
-  const bool gate = r != nullptr || go != nullptr || gr != nullptr;
   if (!fits_int(B) || !fits_int(T) || !fits_int(C)) return RWKV_ERR_INVALID_ARG;
   if (dtype != RWKV_F32 && dtype != RWKV_BF16) return RWKV_ERR_INVALID_ARG;
   if (chunk_len <= 0 || chunk_len % 16 != 0) return RWKV_ERR_INVALID_ARG;
@@ -364,7 +363,7 @@ rwkv_status rwkv_wkv4_backward(int64_t B, int64_t T, int64_t C, rwkv_dtype dtype
                                const void* k, const void* v, const void* gy, const float* state_in,
                                const float* ckpt, int64_t chunk_len, void* gk, void* gv, float* gw, float* gu,
                                void* workspace, size_t workspace_bytes, rwkv_stream_t stream) {
-  return backward_impl(B, T, C, dtype, w, u, k, v, gy, nullptr, nullptr, state_in, ckpt, chunk_len, gk, gv,
+  return backward_impl(false, B, T, C, dtype, w, u, k, v, gy, nullptr, nullptr, state_in, ckpt, chunk_len, gk, gv,
                        nullptr, gw, gu, workspace, workspace_bytes, stream);
 }
 
@@ -373,9 +372,8 @@ rwkv_status rwkv_wkv4_backward_gated(int64_t B, int64_t T, int64_t C, rwkv_dtype
                                      const float* state_in, const float* ckpt, int64_t chunk_len, void* gk, void* gv,
                                      void* gr, float* gw, float* gu, void* workspace, size_t workspace_bytes,
                                      rwkv_stream_t stream) {
-  if (r == nullptr && go == nullptr && gr == nullptr) r = k;  // all three missing: rejected below as a gated call
-  return backward_impl(B, T, C, dtype, w, u, k, v, nullptr, r, go, state_in, ckpt, chunk_len, gk, gv, gr, gw, gu,
-                       workspace, workspace_bytes, stream);
+  return backward_impl(true, B, T, C, dtype, w, u, k, v, nullptr, r, go, state_in, ckpt, chunk_len, gk, gv, gr, gw,
+                       gu, workspace, workspace_bytes, stream);
 }
 
 rwkv_status rwkv_wkv4_step(int64_t B, int64_t C, rwkv_dtype dtype, const float* w, const float* u, const void* k,
