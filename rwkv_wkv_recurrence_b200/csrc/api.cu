@@ -325,14 +325,11 @@ rwkv_status backward_impl(bool gate, int64_t B, int64_t T, int64_t C, rwkv_dtype
   unsigned int* err = device_error_word();
   if (err == nullptr) return RWKV_ERR_CUDA;
   const int box_t = bwd_tile_steps();
-  CUtensorMap mk, mv, mg, mgk, mgv, mo, mgr;
+  CUtensorMap mk, mv, mg, mgk, mgv;
   if (!make_btc_map(&mk, k, bf16, iB, iT, iC, box_t) || !make_btc_map(&mv, v, bf16, iB, iT, iC, box_t) ||
-      !make_btc_map(&mg, gate ? r : gy, bf16, iB, iT, iC, box_t) ||
+      !make_btc_map(&mg, gate ? go : gy, bf16, iB, iT, iC, box_t) ||
       !make_btc_map(&mgk, gk, bf16, iB, iT, iC, bwd_store_steps()) ||
       !make_btc_map(&mgv, gv, bf16, iB, iT, iC, bwd_store_steps()))
-    return RWKV_ERR_CUDA;
-  if (gate && (!make_btc_map(&mo, go, bf16, iB, iT, iC, box_t) ||
-               !make_btc_map(&mgr, gr, bf16, iB, iT, iC, bwd_store_steps())))
     return RWKV_ERR_CUDA;
   Bwd4Params p{};
   p.B = iB;
@@ -347,7 +344,9 @@ rwkv_status backward_impl(bool gate, int64_t B, int64_t T, int64_t C, rwkv_dtype
   p.gv = gv;
   p.part = part;
   p.err = err;
-  const cudaError_t e = gate ? launch_wkv4_bwd_gated(bf16, mk, mv, mg, mo, mgk, mgv, mgr, p, st)
+  p.r = r;
+  p.gr = gr;
+  const cudaError_t e = gate ? launch_wkv4_bwd_gated(bf16, mk, mv, mg, mgk, mgv, p, st)
                              : launch_wkv4_bwd(bf16, mk, mv, mg, mgk, mgv, p, st);
   if (e != cudaSuccess) return RWKV_ERR_CUDA;
   if (launch_wkv4_reduce_wu(iB, iC, part, gw, gu, st) != cudaSuccess) return RWKV_ERR_CUDA;

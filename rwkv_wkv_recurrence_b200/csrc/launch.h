@@ -39,6 +39,8 @@ struct Bwd4Params {
   void* gv;
   double* part;       // [2,B,C] per-lane gw, gu partial sums
   unsigned int* err;  // device error word
+  const void* r;      // [B,T,C] receptance (gated backward only)
+  void* gr;           // [B,T,C] its gradient (gated backward only)
 };
 
 struct Wkv5StepParams {
@@ -99,10 +101,11 @@ cudaError_t launch_wkv4_carry(int B, int C, int T, int nseg, int seg_len, const 
 // boxes over gk, gv (written by TMA stores).
 cudaError_t launch_wkv4_bwd(bool bf16, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mgy,
                             const CUtensorMap& mgk, const CUtensorMap& mgv, const Bwd4Params& p, cudaStream_t st);
-// The receptance-gated backward: mr, mo are [bwd_tile_steps() x 32] boxes over r and go; mgr stores gr.
-cudaError_t launch_wkv4_bwd_gated(bool bf16, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mr,
-                                  const CUtensorMap& mo, const CUtensorMap& mgk, const CUtensorMap& mgv,
-                                  const CUtensorMap& mgr, const Bwd4Params& p, cudaStream_t st);
+// The receptance-gated backward: mo are [bwd_tile_steps() x 32] boxes over go; p.r is read and p.gr
+// written with plain coalesced accesses.
+cudaError_t launch_wkv4_bwd_gated(bool bf16, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mo,
+                                  const CUtensorMap& mgk, const CUtensorMap& mgv, const Bwd4Params& p,
+                                  cudaStream_t st);
 cudaError_t launch_wkv4_reduce_wu(int B, int C, const double* part, float* gw, float* gu, cudaStream_t st);
 cudaError_t launch_wkv4_step(bool bf16, int B, int C, const float* w, const float* u, const void* k, const void* v,
                              void* y, const float* state_in, float* state_out, bool vec4, cudaStream_t st);

@@ -44,10 +44,14 @@
 // the batch by a second kernel.
 //
 // Receptance gate (GATE): gradients of L = Σ go_t σ(r_t) WKV_t (the gated
-// output of the same page's time mixing).  r and go replace gy as the third
-// and fourth boxes of a stage; the recompute phase forms gy_t = σ(r_t) go_t and
+// output of the same page's time mixing).  go takes gy's place as the third
+// box of a stage, so the gated kernel keeps the plain one's shared memory and
+// all of a training shape's CTAs resident (a fourth box would leave three CTAs
+// per SM and a second wave).  r is read with plain loads (a warp reads one
+// 128-byte row per step; the rows of the next tile are prefetched into L2),
+// the recompute phase forms gy_t = σ(r_t) go_t and
 // gr_t = go_t WKV_t σ(r_t) (1 - σ(r_t)) from the WKV_t it recomputes anyway,
-// writes gr over the consumed r rows, and the chunk's gr leaves with gk and gv.
+// and gr leaves with plain coalesced stores.
 #include "launch.h"
 #include "wkv_common.cuh"
 
@@ -68,13 +72,19 @@ struct RSumm {  // a chunk's own reverse sums from a zero carry, at scale 2^q
 };
 
 // Phase A: forward recompute of one chunk from its checkpoint state (a, b) at
-// scale 2^q, keeping e_t, G_t = gy_t / d_t, y_t and b_{t-1}.  With GATE, gs
-// holds the r rows and os the go rows: gy_t = σ(r_t) go_t, and gr_t is written
-// over r_t.
+// scale 2^q, keeping e_t, G_t = gy_t / d_t, y_t and b_{t-1}.  gs holds the gy
+// rows, or with GATE the go rows: then gy_t = σ(r_t) go_t with r_t read from
+// rg[t * C], and gr_t is stored to grg[t * C].
 template <typename T, bool FULL, bool GATE>
-__device__ __forceinline__ void chunk_recompute(const T* ks, const T* vs, T* gs, const T* os, int cnt, float qf,
-                                                float U, float lh, float ll, float a, float b, float (&E)[kL],
-                                                float (&G)[kL], float (&Y)[kL], float (&BP)[kL]) {
+__device__ __forceinline__ void chunk_recompute(const T* ks, const T* vs, const T* gs, const T* rg, T* grg,
+                                                int C, int cnt, float qf, float U, float lh, float ll, float a,
+                                                float b, float (&E)[kL], float (&G)[kL], float (&Y)[kL],
+                                                float (&BP)[kL]) {
+  float rv[GATE ? kL : 1];
+  if constexpr (GATE) {
+#pragma unroll
+    for (int j = 0; j < kL; ++j) rv[j] = (rg != nullptr && (FULL || j < cnt)) ? IO<T>::load(rg + (size_t)j * C) : 0.f;
+  }
 #pragma unroll
   for (int j = 0; j < kL; ++j) {
     if (FULL || j < cnt) {
@@ -87,10 +97,10 @@ __device__ __forceinline__ void chunk_recompute(const T* ks, const T* vs, T* gs,
       Y[j] = ok ? fmaf(eu, vj, a) * rd : vj;
       float gy;
       if constexpr (GATE) {
-        const float sg = sigmoid(IO<T>::to_f(gs[j * 32]));
-        const float go = IO<T>::to_f(os[j * 32]);
+        const float sg = sigmoid(rv[j]);
+        const float go = IO<T>::to_f(gs[j * 32]);
         gy = sg * go;
-        gs[j * 32] = IO<T>::from_f(go * Y[j] * (sg - sg * sg));
+        if (grg != nullptr) grg[(size_t)j * C] = IO<T>::from_f(go * Y[j] * (sg - sg * sg));
       } else {
         gy = IO<T>::to_f(gs[j * 32]);
       }
@@ -152,21 +162,19 @@ struct RCarry {  // reverse carry at a chunk boundary, per lane (see phase C)
   int p;
 };
 
-// mg: gy boxes, or with GATE r boxes; mo: go boxes (GATE only); mgr: gr store boxes (GATE only).
+// mg: gy boxes, or with GATE go boxes.
 template <typename T, bool GATE>
 __global__ void __launch_bounds__(kW * 32, 4) wkv4_bwd_kernel(const __grid_constant__ CUtensorMap mk,
                                                               const __grid_constant__ CUtensorMap mv,
                                                               const __grid_constant__ CUtensorMap mg,
                                                               const __grid_constant__ CUtensorMap mgk,
                                                               const __grid_constant__ CUtensorMap mgv,
-                                                              const __grid_constant__ CUtensorMap mo,
-                                                              const __grid_constant__ CUtensorMap mgr,
                                                               const Bwd4Params p) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   constexpr uint32_t kBoxElems = kTile * 32;
   constexpr uint32_t kBoxBytes = kBoxElems * sizeof(T);
-  constexpr int kNB = GATE ? 4 : 3;  // boxes per stage: k, v, gy  or  k, v, r, go
-  T* tiles = reinterpret_cast<T*>(smem_raw);  // [stages][k|v|gy or k|v|r|go][kTile][32]
+  constexpr int kNB = 3;  // boxes per stage: k, v, and gy (or go)
+  T* tiles = reinterpret_cast<T*>(smem_raw);  // [stages][k|v|gy][kTile][32]
   RSumm* rs = reinterpret_cast<RSumm*>(smem_raw + (size_t)p.stages * kNB * kBoxBytes);  // [2][kW][32]
   RCarry* cslot = reinterpret_cast<RCarry*>(rs + 2 * kW * 32);                        // [2][32]
   uint64_t* bars = reinterpret_cast<uint64_t*>(cslot + 2 * 32);
@@ -185,7 +193,6 @@ __global__ void __launch_bounds__(kW * 32, 4) wkv4_bwd_kernel(const __grid_const
     prefetch_tensormap(&mk);
     prefetch_tensormap(&mv);
     prefetch_tensormap(&mg);
-    if constexpr (GATE) prefetch_tensormap(&mo);
     for (int s = 0; s < p.stages; ++s) mbar_init(&bars[s], 1);
     fence_mbar_init();
     const int pre = min(p.stages, ntile);
@@ -195,7 +202,6 @@ __global__ void __launch_bounds__(kW * 32, 4) wkv4_bwd_kernel(const __grid_const
       tma_load_3d(tiles + (size_t)(kNB * s) * kBoxElems, &mk, &bars[s], ct * 32, tc, bb);
       tma_load_3d(tiles + (size_t)(kNB * s + 1) * kBoxElems, &mv, &bars[s], ct * 32, tc, bb);
       tma_load_3d(tiles + (size_t)(kNB * s + 2) * kBoxElems, &mg, &bars[s], ct * 32, tc, bb);
-      if constexpr (GATE) tma_load_3d(tiles + (size_t)(kNB * s + 3) * kBoxElems, &mo, &bars[s], ct * 32, tc, bb);
     }
   }
   if (warp == 0) cslot[32 + lane] = RCarry{0.0, 0.0, 0.f, 0};  // nothing flows back from after the end
@@ -240,6 +246,12 @@ __global__ void __launch_bounds__(kW * 32, 4) wkv4_bwd_kernel(const __grid_const
         ckb = ck[plane];
         ckp = ck[2 * plane];
       }
+      if constexpr (GATE) {  // the next tile's r rows into L2: lane j < 16 one 32-channel row of this warp's chunk
+        if (tile >= 1 && lane < kL && tsn + lane < p.T) {
+          const T* rrow = static_cast<const T*>(p.r) + ((size_t)bb * p.T + tsn + lane) * p.C + (size_t)ct * 32;
+          asm volatile("prefetch.global.L2 [%0];" ::"l"(rrow) : "memory");
+        }
+      }
       if (tile >= 2 && valid) {  // and the one after it into L2
         const float* ck2 = p.ckpt + (size_t)((tsn - kTile) / kL) * 3 * plane + lane_off;
         asm volatile("prefetch.global.L2 [%0];" ::"l"(ck2) : "memory");
@@ -250,11 +262,13 @@ __global__ void __launch_bounds__(kW * 32, 4) wkv4_bwd_kernel(const __grid_const
     if (!mbar_wait_bounded(&bars[s], ph, p.err)) *abort_flag = 1;
     T* const kw = tiles + (size_t)(kNB * s) * kBoxElems + warp * kL * 32;  // this warp's [16][32] rows
     T* const vw = kw + kBoxElems;
-    T* const gw_rows = vw + kBoxElems;  // gy rows, or with GATE the r rows that receive gr
     T* const ks = kw + lane;
     T* const vs = vw + lane;
-    T* const gs = gw_rows + lane;
-    const T* os = gs + kBoxElems;  // go rows (GATE only)
+    const T* gs = vs + kBoxElems;  // gy rows (go with GATE)
+    // GATE: this lane's r and gr of the chunk, token stride C
+    const size_t tok0 = ((size_t)bb * p.T + (size_t)max(ts, 0)) * p.C + (size_t)c;
+    const T* rg = (GATE && valid) ? static_cast<const T*>(p.r) + tok0 : nullptr;  // lanes past C: no access
+    T* grg = (GATE && valid) ? static_cast<T*>(p.gr) + tok0 : nullptr;
 
     // A. forward recompute of the chunk at one scale 2^q: the forward wrote the
     //    checkpoint at the chunk's scale (at least every k log2 e of the chunk,
@@ -262,11 +276,11 @@ __global__ void __launch_bounds__(kW * 32, 4) wkv4_bwd_kernel(const __grid_const
     float E[kL], G[kL], Y[kL], BP[kL];
     const int q = st.p;
     if (cnt == kL)
-      chunk_recompute<T, true, GATE>(ks, vs, gs, os, cnt, (float)q, U, lh, ll, (float)st.a, (float)st.b, E, G, Y,
-                                     BP);
+      chunk_recompute<T, true, GATE>(ks, vs, gs, rg, grg, p.C, cnt, (float)q, U, lh, ll, (float)st.a, (float)st.b,
+                                     E, G, Y, BP);
     else if (cnt > 0)
-      chunk_recompute<T, false, GATE>(ks, vs, gs, os, cnt, (float)q, U, lh, ll, (float)st.a, (float)st.b, E, G,
-                                      Y, BP);
+      chunk_recompute<T, false, GATE>(ks, vs, gs, rg, grg, p.C, cnt, (float)q, U, lh, ll, (float)st.a,
+                                      (float)st.b, E, G, Y, BP);
 
     // B. the chunk's own reverse sums
     float la = 0.f, lg = 0.f, ye = 0.f;
@@ -288,7 +302,6 @@ __global__ void __launch_bounds__(kW * 32, 4) wkv4_bwd_kernel(const __grid_const
       tma_load_3d(tiles + (size_t)(kNB * sp) * kBoxElems, &mk, &bars[sp], ct * 32, tc, bb);
       tma_load_3d(tiles + (size_t)(kNB * sp + 1) * kBoxElems, &mv, &bars[sp], ct * 32, tc, bb);
       tma_load_3d(tiles + (size_t)(kNB * sp + 2) * kBoxElems, &mg, &bars[sp], ct * 32, tc, bb);
-      if constexpr (GATE) tma_load_3d(tiles + (size_t)(kNB * sp + 3) * kBoxElems, &mo, &bars[sp], ct * 32, tc, bb);
     }
 
     // C. fold the carries of the later chunks.  A carry is (α~ out of a chunk,
@@ -342,7 +355,7 @@ __global__ void __launch_bounds__(kW * 32, 4) wkv4_bwd_kernel(const __grid_const
       if (lane == 0) {
         tma_store_3d(&mgk, kw, ct * 32, ts, bb);
         tma_store_3d(&mgv, vw, ct * 32, ts, bb);
-        if constexpr (GATE) tma_store_3d(&mgr, gw_rows, ct * 32, ts, bb);
+
         bulk_commit();
       }
     }
@@ -381,23 +394,22 @@ __global__ void wkv4_reduce_wu_kernel(int B, int C, const double* __restrict__ p
   gu[c] = (float)su;
 }
 
-template <typename T, bool GATE>
+template <typename T>
 size_t bwd_smem_bytes(int stages) {
-  return (size_t)stages * (GATE ? 4 : 3) * kTile * 32 * sizeof(T) + 2 * kW * 32 * sizeof(RSumm) +
-         2 * 32 * sizeof(RCarry) + (size_t)stages * 8 + 16;
+  return (size_t)stages * 3 * kTile * 32 * sizeof(T) + 2 * kW * 32 * sizeof(RSumm) + 2 * 32 * sizeof(RCarry) +
+         (size_t)stages * 8 + 16;
 }
 
 template <typename T, bool GATE>
 cudaError_t launch_bwd_t(const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mg, const CUtensorMap& mgk,
-                         const CUtensorMap& mgv, const CUtensorMap& mo, const CUtensorMap& mgr, const Bwd4Params& p,
-                         cudaStream_t st) {
-  const size_t smem = bwd_smem_bytes<T, GATE>(p.stages);
+                         const CUtensorMap& mgv, const Bwd4Params& p, cudaStream_t st) {
+  const size_t smem = bwd_smem_bytes<T>(p.stages);
   static unsigned device_mask = 0;
   cudaError_t e =
       ensure_smem_attr(reinterpret_cast<const void*>(wkv4_bwd_kernel<T, GATE>), (int)smem, &device_mask);
   if (e != cudaSuccess) return e;
   const long long nblk = (long long)p.ctiles * p.B;
-  wkv4_bwd_kernel<T, GATE><<<(unsigned)nblk, kW * 32, smem, st>>>(mk, mv, mg, mgk, mgv, mo, mgr, p);
+  wkv4_bwd_kernel<T, GATE><<<(unsigned)nblk, kW * 32, smem, st>>>(mk, mv, mg, mgk, mgv, p);
   return cudaGetLastError();
 }
 
@@ -408,24 +420,23 @@ int bwd_tile_steps() { return kTile; }
 int bwd_store_steps() { return kL; }
 
 int bwd_stages(bool bf16, int T, bool gate) {
-  // 48 KB of k, v, gy boxes keeps four CTAs per SM; the gate's four boxes per stage take 64 KB (fp32) in two
-  // stages, three CTAs per SM
-  const int want = gate ? (bf16 ? 3 : 2) : (bf16 ? 4 : 2);
+  (void)gate;  // the gated kernel streams the same three boxes (k, v, go)
+  const int want = bf16 ? 4 : 2;  // 48 KB of boxes keeps four CTAs per SM
   const int ntile = (T + kTile - 1) / kTile;
   return max(2, min(want, ntile));
 }
 
 cudaError_t launch_wkv4_bwd(bool bf16, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mg,
                             const CUtensorMap& mgk, const CUtensorMap& mgv, const Bwd4Params& p, cudaStream_t st) {
-  return bf16 ? launch_bwd_t<__nv_bfloat16, false>(mk, mv, mg, mgk, mgv, mk, mgk, p, st)
-              : launch_bwd_t<float, false>(mk, mv, mg, mgk, mgv, mk, mgk, p, st);
+  return bf16 ? launch_bwd_t<__nv_bfloat16, false>(mk, mv, mg, mgk, mgv, p, st)
+              : launch_bwd_t<float, false>(mk, mv, mg, mgk, mgv, p, st);
 }
 
-cudaError_t launch_wkv4_bwd_gated(bool bf16, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mr,
-                                  const CUtensorMap& mo, const CUtensorMap& mgk, const CUtensorMap& mgv,
-                                  const CUtensorMap& mgr, const Bwd4Params& p, cudaStream_t st) {
-  return bf16 ? launch_bwd_t<__nv_bfloat16, true>(mk, mv, mr, mgk, mgv, mo, mgr, p, st)
-              : launch_bwd_t<float, true>(mk, mv, mr, mgk, mgv, mo, mgr, p, st);
+cudaError_t launch_wkv4_bwd_gated(bool bf16, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mo,
+                                  const CUtensorMap& mgk, const CUtensorMap& mgv, const Bwd4Params& p,
+                                  cudaStream_t st) {
+  return bf16 ? launch_bwd_t<__nv_bfloat16, true>(mk, mv, mo, mgk, mgv, p, st)
+              : launch_bwd_t<float, true>(mk, mv, mo, mgk, mgv, p, st);
 }
 
 cudaError_t launch_wkv4_reduce_wu(int B, int C, const double* part, float* gw, float* gu, cudaStream_t st) {
