@@ -461,6 +461,7 @@ def run_decode(args):
 
     ms, clk = _timed(step, args.steps, args.warmup, stream, local)
     rw.rwkv_check_device_error()
+    graph = _graph_decode_timing(rw, h, st, w, u, ks, vs, y, Bd, Cd, Td, dev)
     lanes = Bd * Cd
     bytes_step = 36 * lanes  # state 12 B in + 12 B out, k, v, y 4 B each
     gbs = bytes_step / (ms * 1e-3) / 1e9
@@ -474,7 +475,54 @@ def run_decode(args):
         "roofline": {"bound": "hbm", "kernel": "wkv4_step_kernel", "achieved": gbs, "peak": peak,
                      "peak_kind": kind, "unit": "GB/s", "frac": gbs / peak,
                      "traffic": _recorded_traffic("wkv4_step_kernel")},
-        "gpu_launches": args.steps, "clocks": clk}), flush=True)
+        "gpu_launches": args.steps, "clocks": clk, "cuda_graph": graph}), flush=True)
+
+
+def _graph_decode_timing(rw, h, st, w, u, ks, vs, y, Bd, Cd, Td, dev):
+    """The decode loop as a CUDA graph: the Td-token loop of the full shape captured
+    once and replayed, and the same for a small batch of 16 streams, where each
+    step is a few microseconds and launch overhead matters; eager timing beside it."""
+    import torch
+
+    P = rw._ptr
+
+    def loop(stream, nb, state, kk, vv, yy):
+        sp = rw._stream(stream)
+        for j in range(Td):
+            s = h.rwkv_wkv4_step(nb, Cd, rw.F32, P(w), P(u), P(kk[j]), P(vv[j]), P(yy), P(state), P(state), sp)
+            if s:
+                raise rw.RwkvError("rwkv_wkv4_step", s)
+
+    def time_it(fn, reps):
+        fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / reps / Td
+
+    out = {"steps_per_graph": Td}
+    for name, nb in (("full", Bd), ("16_streams", 16)):
+        state = st[:, :nb].contiguous() if nb != Bd else st
+        kk = ks if nb == Bd else [x[:nb].contiguous() for x in ks]
+        vv = vs if nb == Bd else [x[:nb].contiguous() for x in vs]
+        yy = y if nb == Bd else y[:nb].contiguous()
+        eager_ms = time_it(lambda: loop(torch.cuda.current_stream(), nb, state, kk, vv, yy), 3)
+        g = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            loop(side, nb, state, kk, vv, yy)  # warm the launch path on the capture stream
+        torch.cuda.current_stream().wait_stream(side)
+        with torch.cuda.graph(g):
+            loop(torch.cuda.current_stream(), nb, state, kk, vv, yy)
+        graph_ms = time_it(g.replay, 3)
+        out[name] = {"streams": nb, "eager_us_per_step": eager_ms * 1e3, "graph_us_per_step": graph_ms * 1e3}
+        del g
+    return out
 
 
 def run_train_gated(args):
