@@ -51,6 +51,8 @@ def _load():
             "oracle_wkv5_forward_bruteforce": [I, I, I, I, P, P, P, P, P, P],
             "oracle_wkv6_forward": [I, I, I, I, P, P, P, P, P, P, P, P],
             "oracle_wkv4_gated_forward": [I, I, I, P, P, P, P, P, P, P, P],
+            "oracle_wkv5_backward": [I, I, I, I, P, P, P, P, P, P, P, P, P, P, P, P, P, P],
+            "oracle_wkv6_backward": [I, I, I, I, P, P, P, P, P, P, P, P, P, P, P, P, P, P],
             "oracle_wkv4_gated_backward": [I, I, I, P, P, P, P, P, P, P, P, P, P, P, P],
             "oracle_wkv6_forward_bruteforce": [I, I, I, I, P, P, P, P, P, P],
         }
@@ -229,3 +231,29 @@ def wkv4_gated_backward(w, u, k, v, r, go, state_in=None):
     _check(lib.oracle_wkv4_gated_backward(B, T, C, _p(w), _p(u), _p(k), _p(v), _p(r), _p(go), _p(s0),
                                           _p(gk), _p(gv), _p(gr), _p(gw), _p(gu)), "wkv4_gated_backward")
     return gk, gv, gr, gw, gu
+
+
+def _wkv56_backward(fn, name, r, k, v, omega, u, gy, s_in=None, gs_out=None, per_token=False):
+    lib = _load()
+    r, k, v, omega, u, gy, s0, gso = map(_f64, (r, k, v, omega, u, gy, s_in, gs_out))
+    B, T, H, N = r.shape
+    gr, gk, gv = np.empty((B, T, H, N)), np.empty((B, T, H, N)), np.empty((B, T, H, N))
+    gom = np.empty((B, T, H, N) if per_token else (H, N))
+    gu = np.empty((H, N))
+    gsi = np.empty((B, H, N, N))
+    _check(getattr(lib, fn)(B, T, H, N, _p(r), _p(k), _p(v), _p(omega), _p(u), _p(s0), _p(gy), _p(gso),
+                            _p(gr), _p(gk), _p(gv), _p(gom), _p(gu), _p(gsi)), name)
+    return gr, gk, gv, gom, gu, gsi
+
+
+def wkv5_backward(r, k, v, omega, u, gy, s_in=None, gs_out=None):
+    """Gradients of sum(gy * y) + sum(gs_out * s_out) for the Eagle forward: returns
+    (gr, gk, gv, gomega [H,N], gu [H,N], gs_in [B,H,N,N])."""
+    return _wkv56_backward("oracle_wkv5_backward", "wkv5_backward", r, k, v, omega, u, gy, s_in, gs_out)
+
+
+def wkv6_backward(r, k, v, omega, u, gy, s_in=None, gs_out=None):
+    """Gradients of sum(gy * y) + sum(gs_out * s_out) for the Finch forward: returns
+    (gr, gk, gv, gomega [B,T,H,N], gu [H,N], gs_in [B,H,N,N])."""
+    return _wkv56_backward("oracle_wkv6_backward", "wkv6_backward", r, k, v, omega, u, gy, s_in, gs_out,
+                           per_token=True)

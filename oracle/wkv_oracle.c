@@ -41,6 +41,10 @@
  *  - Eagle reads the state before the current token's k^T v is added, and
  *    diag(w), diag(u) scale the key (row) index; w is a multiplicative factor in
  *    (0, 1), unlike RWKV-4's rate.
+ *  - The Eagle and Finch backward are not printed either: oracle_wkv5_backward and
+ *    oracle_wkv6_backward take the chain rule through the recurrence, with the
+ *    gradient of L = Σ gy·y + Σ gs_out·s_out; gomega and gu are summed over
+ *    batch (and over time for Eagle's per-channel omega).
  *  - Finch's data-dependent decay is read as omega_t [B, T, H, N], one omega
  *    per token and channel with w_t = exp(-exp(omega_t)) as in Eagle, and the
  *    decay of token t multiplies the state when token t's k^T v is added (the
@@ -554,4 +558,107 @@ int64_t oracle_wkv4_gated_backward(int64_t B, int64_t T, int64_t C,
     free(wkv);
     free(gy);
     return bad;
+}
+
+/*
+ * Backward of the Eagle / RWKV-5 forward above (and, with omega_per_token, of the
+ * Finch / RWKV-6 forward): gradients of
+ *   L = Σ_t Σ_j gy_t[j] y_t[j] + Σ_{i,j} gs_out[i][j] s_out[i][j]
+ * by the chain rule through the recurrence (the pages print no backward).  With
+ * S_t the state before token t and G the gradient of L with respect to S_{t+1},
+ * walking t = T-1 .. 0:
+ *   gr_t[i] = Σ_j gy_t[j] (S_t[i][j] + u_i k_t[i] v_t[j])
+ *   gk_t[i] = Σ_j G[i][j] v_t[j] + u_i r_t[i] Σ_j gy_t[j] v_t[j]
+ *   gv_t[j] = Σ_i G[i][j] k_t[i] + (Σ_i r_t[i] u_i k_t[i]) gy_t[j]
+ *   gu[i]  += r_t[i] k_t[i] Σ_j gy_t[j] v_t[j]
+ *   gw_t[i] = Σ_j G[i][j] S_t[i][j]                (S_{t+1} = diag(w_t) S_t + k_t^T v_t)
+ *   G      <- diag(w_t) G + r_t^T gy_t              (then G is the gradient for S_t)
+ * gomega = gw * dw/domega = gw * (-exp(omega)) * w, per token for Finch, summed over
+ * tokens and batch for Eagle; gu is summed over batch; gs_in = G after the walk.
+ * gy [B,T,H,N]; gs_out [B,H,N,N] or NULL; outputs gr, gk, gv [B,T,H,N], gomega [H,N]
+ * (Eagle) or [B,T,H,N] (Finch), gu [H,N], gs_in [B,H,N,N] (or NULL).  The states of
+ * every token are recomputed and kept per head (O(T N^2) memory: small inputs).
+ */
+static int64_t wkv56_backward(int64_t B, int64_t T, int64_t H, int64_t N, const double *r, const double *k,
+                              const double *v, const double *omega, int omega_per_token, const double *u,
+                              const double *s_in, const double *gy, const double *gs_out, double *gr, double *gk,
+                              double *gv, double *gomega, double *gu, double *gs_in)
+{
+    int64_t bad = 0;
+    const int64_t nomega = omega_per_token ? B * T * H * N : H * N;
+    for (int64_t i = 0; i < nomega; ++i) gomega[i] = 0.0;
+    for (int64_t i = 0; i < H * N; ++i) gu[i] = 0.0;
+    double *S = (double *)malloc((size_t)((T + 1) * N * N) * sizeof(double));
+    double *G = (double *)malloc((size_t)(N * N) * sizeof(double));
+    double *wt = (double *)malloc((size_t)N * sizeof(double));
+    for (int64_t b = 0; b < B; ++b) {
+        for (int64_t h = 0; h < H; ++h) {
+            /* forward: S[t] = state before token t, S[T] = s_out */
+            for (int64_t ij = 0; ij < N * N; ++ij) S[ij] = s_in ? s_in[((b * H + h) * N) * N + ij] : 0.0;
+            for (int64_t t = 0; t < T; ++t) {
+                for (int64_t i = 0; i < N; ++i)
+                    wt[i] = exp(-exp(omega_per_token ? omega[IDX4(b, t, h, i)] : omega[h * N + i]));
+                for (int64_t i = 0; i < N; ++i)
+                    for (int64_t j = 0; j < N; ++j)
+                        S[(t + 1) * N * N + i * N + j] =
+                            wt[i] * S[t * N * N + i * N + j] + k[IDX4(b, t, h, i)] * v[IDX4(b, t, h, j)];
+            }
+            for (int64_t ij = 0; ij < N * N; ++ij) G[ij] = gs_out ? gs_out[((b * H + h) * N) * N + ij] : 0.0;
+            for (int64_t t = T - 1; t >= 0; --t) {
+                const double *St = S + t * N * N;
+                double gyv = 0.0, ruk = 0.0;
+                for (int64_t j = 0; j < N; ++j) gyv += gy[IDX4(b, t, h, j)] * v[IDX4(b, t, h, j)];
+                for (int64_t i = 0; i < N; ++i) ruk += r[IDX4(b, t, h, i)] * u[h * N + i] * k[IDX4(b, t, h, i)];
+                for (int64_t i = 0; i < N; ++i) {
+                    const double ui = u[h * N + i], ri = r[IDX4(b, t, h, i)], ki = k[IDX4(b, t, h, i)];
+                    double a = 0.0, c = 0.0, gw = 0.0;
+                    for (int64_t j = 0; j < N; ++j) {
+                        a += gy[IDX4(b, t, h, j)] * (St[i * N + j] + ui * ki * v[IDX4(b, t, h, j)]);
+                        c += G[i * N + j] * v[IDX4(b, t, h, j)];
+                        gw += G[i * N + j] * St[i * N + j];
+                    }
+                    gr[IDX4(b, t, h, i)] = a;
+                    gk[IDX4(b, t, h, i)] = c + ui * ri * gyv;
+                    gu[h * N + i] += ri * ki * gyv;
+                    const double om = omega_per_token ? omega[IDX4(b, t, h, i)] : omega[h * N + i];
+                    const double dw = -exp(om) * exp(-exp(om));
+                    if (omega_per_token) gomega[IDX4(b, t, h, i)] = gw * dw;
+                    else gomega[h * N + i] += gw * dw;
+                    if (!isfinite(a) || !isfinite(c)) ++bad;
+                }
+                for (int64_t j = 0; j < N; ++j) {
+                    double a = 0.0;
+                    for (int64_t i = 0; i < N; ++i) a += G[i * N + j] * k[IDX4(b, t, h, i)];
+                    gv[IDX4(b, t, h, j)] = a + ruk * gy[IDX4(b, t, h, j)];
+                }
+                for (int64_t i = 0; i < N; ++i) {
+                    const double w_i = exp(-exp(omega_per_token ? omega[IDX4(b, t, h, i)] : omega[h * N + i]));
+                    for (int64_t j = 0; j < N; ++j)
+                        G[i * N + j] = w_i * G[i * N + j] + r[IDX4(b, t, h, i)] * gy[IDX4(b, t, h, j)];
+                }
+            }
+            if (gs_in)
+                for (int64_t ij = 0; ij < N * N; ++ij) gs_in[((b * H + h) * N) * N + ij] = G[ij];
+        }
+    }
+    free(S);
+    free(G);
+    free(wt);
+    return bad;
+}
+
+int64_t oracle_wkv5_backward(int64_t B, int64_t T, int64_t H, int64_t N, const double *r, const double *k,
+                             const double *v, const double *omega, const double *u, const double *s_in,
+                             const double *gy, const double *gs_out, double *gr, double *gk, double *gv,
+                             double *gomega, double *gu, double *gs_in)
+{
+    return wkv56_backward(B, T, H, N, r, k, v, omega, 0, u, s_in, gy, gs_out, gr, gk, gv, gomega, gu, gs_in);
+}
+
+int64_t oracle_wkv6_backward(int64_t B, int64_t T, int64_t H, int64_t N, const double *r, const double *k,
+                             const double *v, const double *omega, const double *u, const double *s_in,
+                             const double *gy, const double *gs_out, double *gr, double *gk, double *gv,
+                             double *gomega, double *gu, double *gs_in)
+{
+    return wkv56_backward(B, T, H, N, r, k, v, omega, 1, u, s_in, gy, gs_out, gr, gk, gv, gomega, gu, gs_in);
 }
