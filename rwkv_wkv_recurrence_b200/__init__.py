@@ -23,7 +23,6 @@ __all__ = [
     "ALGO_CHUNKED", "CHUNK_LEN", "NOALLOC_MAX_LANES", "rwkv_wkv4_forward", "rwkv_wkv4_backward",
     "rwkv_wkv4_backward_noalloc", "rwkv_wkv4_step", "rwkv_wkv4_forward_gated", "rwkv_wkv4_backward_gated",
     "rwkv_wkv5_forward", "rwkv_wkv5_step", "rwkv_wkv6_forward", "rwkv_wkv6_step", "rwkv_check_device_error",
-    "state_to_ab",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "librwkv_wkv.so")
@@ -170,9 +169,16 @@ def rwkv_wkv4_backward(w, u, k, v, gy, ckpt=None, state_in=None, *, stream=None,
 
     _need_cuda(w, u, k, v, gy, ckpt, state_in)
     B, T, C = k.shape
-    if gy.shape != k.shape or gy.dtype != k.dtype:
-        raise ValueError("gy must match k in shape and dtype")
+    for name, t in (("v", v), ("gy", gy)):
+        if t.shape != k.shape or t.dtype != k.dtype:
+            raise ValueError(f"{name} must match k in shape and dtype")
+    _f32("w", w, C)
+    _f32("u", u, C)
     h = lib()
+    if ckpt is not None:
+        _f32("ckpt", ckpt, int(h.rwkv_wkv4_num_checkpoints(T, CHUNK_LEN)) * 3 * B * C)
+    if state_in is not None:
+        _f32("state_in", state_in, 3 * B * C)
     if out is None:
         gk, gv = torch.empty_like(k), torch.empty_like(v)
         gw = torch.empty(C, dtype=torch.float32, device=k.device)
@@ -233,7 +239,13 @@ def rwkv_wkv4_backward_gated(w, u, k, v, r, go, ckpt=None, state_in=None, *, str
     for name, t in (("v", v), ("r", r), ("go", go)):
         if t.shape != k.shape or t.dtype != k.dtype:
             raise ValueError(f"{name} must match k in shape and dtype")
+    _f32("w", w, C)
+    _f32("u", u, C)
     h = lib()
+    if ckpt is not None:
+        _f32("ckpt", ckpt, int(h.rwkv_wkv4_num_checkpoints(T, CHUNK_LEN)) * 3 * B * C)
+    if state_in is not None:
+        _f32("state_in", state_in, 3 * B * C)
     if out is None:
         gk, gv, gr = torch.empty_like(k), torch.empty_like(v), torch.empty_like(r)
         gw = torch.empty(C, dtype=torch.float32, device=k.device)
@@ -259,6 +271,12 @@ def rwkv_wkv4_backward_noalloc(w, u, k, v, gy, ckpt, *, stream=None, out=None):
 
     _need_cuda(w, u, k, v, gy, ckpt)
     B, T, C = k.shape
+    for name, t in (("v", v), ("gy", gy)):
+        if t.shape != k.shape or t.dtype != k.dtype:
+            raise ValueError(f"{name} must match k in shape and dtype")
+    _f32("w", w, C)
+    _f32("u", u, C)
+    _f32("ckpt", ckpt, int(lib().rwkv_wkv4_num_checkpoints(T, CHUNK_LEN)) * 3 * B * C)
     if out is None:
         gk, gv = torch.empty_like(k), torch.empty_like(v)
         gw = torch.empty(C, dtype=torch.float32, device=k.device)
@@ -381,11 +399,3 @@ def rwkv_check_device_error(stream=None):
     """Synchronise the stream and raise if a kernel's bounded wait timed out."""
     _check("rwkv_check_device_error", lib().rwkv_check_device_error(_stream(stream)))
 
-
-def state_to_ab(state):
-    """(a, b, p) planes -> float64 (A, B) = (a 2^p, b 2^p), for comparisons."""
-    import torch
-
-    s = state.double()
-    scale = torch.pow(2.0, s[2])
-    return torch.stack([s[0] * scale, s[1] * scale])

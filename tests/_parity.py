@@ -2,9 +2,10 @@
 
 Tolerances (stated once, used everywhere):
 * fp32 WKV-4 outputs:      |got - ref| <= 1e-5 * max(1, |ref|)
-* fp32 WKV-4 gradients gk, gv:   |got - ref| <= 1e-4 * max(1, |ref|) elementwise
-* fp32 WKV-4 gradients gw, gu (each entry a sum over B*T terms that cancel):
-                           max |got - ref| <= 1e-4 * max(1, max |ref|)  (norm-wise)
+* fp32 WKV-4 gradients gk, gv, gw, gu (and gr of the gated operator):
+                           |got - ref| <= 1e-4 * max(1, |ref|) elementwise;
+  for gw, gu (each entry a sum over B*T terms) the norm-wise ratio
+  max |got - ref| / max(1, max |ref|) is reported beside it
 * bf16 I/O (fp32 inside):  |got - ref| <= 8e-3 * max(|ref|, rms(ref))
   (rms over the compared tensor; a bf16 output alone is rounded by <= 2^-9 relative)
 * WKV-4 states compare through a/b (1e-5 * max(1, |A/B|)) and log2 b + p
@@ -52,13 +53,23 @@ def assert_close_normwise(got, ref, tol, what=""):
     return err / bound
 
 
-def assert_grads_close(got, ref, what=""):
-    """(gk, gv, gw, gu) against the oracle: elementwise for gk, gv, norm-wise for gw, gu."""
-    for g, r, name in zip(got, ref, ("gk", "gv", "gw", "gu")):
-        if name in ("gk", "gv"):
-            assert_close_abs1(g, r, TOL_GRAD, f"{what}{name}")
-        else:
-            assert_close_normwise(g, r, TOL_GRAD, f"{what}{name}")
+def normwise_ratio(got, ref):
+    """max |got - ref| / max(1, max |ref|): the error of a vector of reductions against its
+    largest entry (reported beside the elementwise check, not a looser bound)."""
+    g, r = _np(got), _np(ref)
+    return float(np.max(np.abs(g - r))) / max(1.0, float(np.max(np.abs(r))))
+
+
+def assert_grads_close(got, ref, what="", names=("gk", "gv", "gw", "gu")):
+    """Gradients against the oracle, every one elementwise: |got - ref| <= 1e-4 max(1, |ref|).
+    Returns the worst elementwise error/bound ratio and, for gw and gu, the norm-wise ratio."""
+    report = {}
+    for g, r, name in zip(got, ref, names):
+        report[name] = assert_close_abs1(g, r, TOL_GRAD, f"{what}{name}")
+        if name in ("gw", "gu"):
+            report[name + "_normwise"] = normwise_ratio(g, r)
+    print(f"{what}gradient error / bound: " + ", ".join(f"{k} {v:.3g}" for k, v in report.items()))
+    return report
 
 
 def assert_close_rms(got, ref, tol, what=""):
@@ -91,3 +102,10 @@ def sample_lanes(B, C, n, seed=0):
     rng = np.random.default_rng(seed)
     flat = rng.choice(B * C, size=min(n, B * C), replace=False)
     return torch.from_numpy(flat // C), torch.from_numpy(flat % C)
+
+
+def state_to_ab(state):
+    """(a, b, p) planes -> float64 (A, B) = (a 2^p, b 2^p), for comparisons."""
+    s = state.double()
+    scale = torch.pow(2.0, s[2])
+    return torch.stack([s[0] * scale, s[1] * scale])

@@ -9,7 +9,7 @@ import torch
 import oracle
 import rwkv_wkv_recurrence_b200 as rw
 import wkv_inputs as wi
-from _parity import TOL_BF16, TOL_GRAD, TOL_Y, assert_close_abs1, assert_close_rms
+from _parity import TOL_BF16, TOL_GRAD, TOL_Y, assert_close_abs1, assert_close_rms, state_to_ab
 
 pytestmark = pytest.mark.gpu
 
@@ -112,7 +112,7 @@ def test_wkv4_past_2pow31_elements(cuda_device):
     # the state before the window, from the forward over batch 1's prefix
     _, st = rw.rwkv_wkv4_forward(p["w"], p["u"], p["k"][1:2, :T - W].contiguous(),
                                  p["v"][1:2, :T - W].contiguous(), return_state=True)
-    ab = rw.state_to_ab(st)[:, :, chans.to(cuda_device)].cpu().numpy()
+    ab = state_to_ab(st)[:, :, chans.to(cuda_device)].cpu().numpy()
     w, u = p["w"][chans.to(cuda_device)].cpu(), p["u"][chans.to(cuda_device)].cpu()
     ref_y = oracle.wkv4_forward(w, u, win["k"], win["v"], state_in=ab)
     assert_close_abs1(y_win, ref_y, TOL_Y, "y at 64-bit offsets")

@@ -170,25 +170,26 @@ def test_backward_deterministic(cuda_device):
 
 def test_training_workload_full_size(cuda_device):
     # 8 x 4096 x 2048, keys with 1 % outliers, gy ~ N(0, 1): forward + backward
-    # in the launch configuration the benchmark times; every output of 48
-    # sampled channels (all 8 batch rows, so gw and gu are complete) checked.
+    # in the launch configuration the benchmark times; every output element
+    # (y, gk, gv over all 2048 channels and 8 batch rows, gw and gu per channel)
+    # checked against the fp64 oracle over the whole problem.
     B, T, C = 8, 4096, 2048
     p = wi.wkv4_problem(B, T, C, SEED + 2, outliers=True, with_gy=True)
     g = _cuda(p, cuda_device)
     y, ck = rw.rwkv_wkv4_forward(g["w"], g["u"], g["k"], g["v"], checkpoints=True)
     gk, gv, gw, gu = rw.rwkv_wkv4_backward(g["w"], g["u"], g["k"], g["v"], g["gy"], ckpt=ck)
-    chans = torch.from_numpy(np.random.default_rng(2).choice(C, 48, replace=False))
-    sub = {k: (v[:, :, chans] if v.dim() == 3 else v[chans]) for k, v in p.items()}
-    ref_y = oracle.wkv4_forward(sub["w"], sub["u"], sub["k"], sub["v"])
-    assert_close_abs1(y[:, :, chans.to(cuda_device)], ref_y, TOL_Y, "y")
-    r = oracle.wkv4_backward(sub["w"], sub["u"], sub["k"], sub["v"], sub["gy"])
-    cg = chans.to(cuda_device)
-    assert_grads_close((gk[:, :, cg], gv[:, :, cg], gw[cg], gu[cg]), r)
+    rw.rwkv_check_device_error()
+    del ck, g
+    ref_y = oracle.wkv4_forward(p["w"], p["u"], p["k"], p["v"])
+    assert_close_abs1(y, ref_y, TOL_Y, "y")
+    del ref_y, y
+    r = oracle.wkv4_backward(p["w"], p["u"], p["k"], p["v"], p["gy"])
+    assert_grads_close((gk, gv, gw, gu), r)
     # properties that hold for every lane: sum_t gk = 0 and sum_t gv = sum_t gy
     # (fp32 sums of 4096 terms: compared against the sum of magnitudes)
     sk = gk.double().sum(1)
     assert torch.all(sk.abs() <= 1e-4 * gk.double().abs().sum(1) + 1e-4)
-    sv = gv.double().sum(1) - g["gy"].double().sum(1)
+    sv = gv.double().sum(1) - p["gy"].to(gv.device).double().sum(1)
     assert torch.all(sv.abs() <= 1e-4 * gv.double().abs().sum(1) + 1e-4)
 
 

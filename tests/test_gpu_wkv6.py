@@ -3,7 +3,6 @@ decode step against the fp64 oracle, through the C-ABI.  bf16 inputs are
 widened exactly for the oracle; omega is fp32 on both sides.
 Tolerance for the bf16 output y and the fp32 final state alike:
 |got - ref| <= 8e-3 * max(|ref|, rms(ref))."""
-import numpy as np
 import pytest
 import torch
 
@@ -105,19 +104,18 @@ def test_state_in_place(cuda_device):
 
 
 def test_finch_workload_full_size(cuda_device):
-    # B4 T4096 H40 N64 with per-token omega = U(-6, 0) base + 0.5 N(0, 1): the whole output on the
-    # GPU, 8 sampled (b, h) heads checked element by element (output and final state).
+    # B4 T4096 H40 N64 with per-token omega = U(-6, 0) base + 0.5 N(0, 1): the whole
+    # output and final state of all 160 (b, h) heads checked element by element.
     B, T, H, N = 4, 4096, 40, 64
     p = wi.wkv6_problem(B, T, H, N, seed=SEED + 6)
     y, s = rw.rwkv_wkv6_forward(**_cuda(p, cuda_device), return_state=True)
     rw.rwkv_check_device_error()
-    rng = np.random.default_rng(6)
-    for b, h in zip(rng.integers(0, B, 8), rng.integers(0, H, 8)):
-        sub = lambda x: x[b:b + 1, :, h:h + 1]
-        ref, ref_s = oracle.wkv6_forward(sub(p["r"]), sub(p["k"]), sub(p["v"]), sub(p["omega"]),
-                                         p["u"][h:h + 1], return_state=True)
-        assert_close_rms(y[b:b + 1, :, h:h + 1], ref, TOL_BF16, f"y head ({b},{h})")
-        assert_close_rms(s[b:b + 1, h:h + 1], ref_s, TOL_BF16, f"s head ({b},{h})")
+    ref, ref_s = oracle.wkv6_forward(p["r"], p["k"], p["v"], p["omega"], p["u"], return_state=True)
+    yc, sc = y.cpu(), s.cpu()
+    for b in range(B):
+        for h in range(H):  # the rms of each rule is taken per head
+            assert_close_rms(yc[b, :, h], ref[b, :, h], TOL_BF16, f"y head ({b},{h})")
+            assert_close_rms(sc[b, h], ref_s[b, h], TOL_BF16, f"s head ({b},{h})")
 
 
 # ------------------------------------------------------------------ decode step
