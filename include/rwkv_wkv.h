@@ -272,8 +272,10 @@ RWKV_API rwkv_status rwkv_wkv6_step(int64_t B, int64_t H, int64_t N, const void 
  *   - B * C > RWKV_NOALLOC_MAX_LANES returns RWKV_ERR_WORKSPACE (too big for
  *     the fixed scratch); ckpt == NULL returns RWKV_ERR_INVALID_ARG.
  *   - The first call on each device looks up the array's device address
- *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before any stream capture.
+ *     (cudaGetSymbolAddress) with that device current and caches it for the
+ *     device's current context; the first call after that context is
+ *     replaced (cudaDeviceReset) looks it up again.  Make the first call on
+ *     a device before any stream capture.
  *   - All calls share the array: calls whose GPU work overlaps (other
  *     streams, other threads) race and must be ordered by the caller.
  *   - Calls no cudaMalloc, cudaFree or allocating library routine.
@@ -288,6 +290,11 @@ RWKV_API rwkv_status rwkv_wkv4_backward_noalloc(int64_t B, int64_t T, int64_t C,
  * Synchronises `stream`, then reports and clears the device error word that
  * kernels set when a bounded wait gives up (RWKV_ERR_DEVICE_TIMEOUT), or
  * RWKV_ERR_CUDA if the stream itself failed.
+ * The error word is one per device and process, shared by every call on that
+ * device whatever its stream or host thread: a timeout in work on one stream
+ * is reported to (and cleared by) the first caller that checks, on any
+ * stream.  Callers that run the library from several streams and need to
+ * know which call timed out must check after each call, in stream order.
  */
 RWKV_API rwkv_status rwkv_check_device_error(rwkv_stream_t stream);
 

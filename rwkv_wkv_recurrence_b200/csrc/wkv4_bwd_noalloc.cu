@@ -15,12 +15,15 @@
 // kNoAllocMaxLanes lanes x 2 doubles (4 MiB).  Every GPU that loads the
 // library holds it until the process exits.  In host code its name is only a
 // host-side stand-in, so its device address is looked up with
-// cudaGetSymbolAddress once per device (with that device current) on the
-// first call made on that device, and cached.  All calls share the array and
-// it keeps the last call's contents; the backward writes every partial it
-// later reads within the same call, so nothing needs clearing between calls.
-// Two calls whose work overlaps on the GPU (different streams, or different
-// host threads without ordering) race on the array.
+// cudaGetSymbolAddress, with the device current, on the first call made in
+// that device's context, and cached together with the context's unique id.
+// A context created later for the same device (after cudaDeviceReset, say)
+// has another id, so the next call looks the address up again instead of
+// handing the kernel a stale one.  All calls share the array and it keeps the
+// last call's contents; the backward writes every partial it later reads
+// within the same call, so nothing needs clearing between calls.  Two calls
+// whose work overlaps on the GPU (different streams, or different host
+// threads without ordering) race on the array.
 #include <mutex>
 
 #include "../../include/rwkv_wkv.h"
@@ -35,23 +38,59 @@ constexpr int kMaxDevices = 64;
 // Per-lane gw, gu partial sums of the backward: [2][kNoAllocMaxLanes] fp64.
 static __device__ __align__(256) double g_bwd_scratch[2 * kNoAllocMaxLanes];
 
-std::mutex g_setup_mutex;
-double* g_scratch_ptr[kMaxDevices] = {};
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
 
-// Device address of g_bwd_scratch on the current device, looked up once per device.
+// Unique id of the context current on this thread (driver entry points looked
+// up once); 0 if there is none or the driver cannot say.
+unsigned long long current_context_id() {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+  });
+  if (get_current == nullptr || get_id == nullptr) return 0;
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
+  if (get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
+struct ScratchAddr {
+  unsigned long long ctx_id;  // context the address belongs to (0: none yet)
+  double* ptr;
+};
+
+std::mutex g_setup_mutex;
+ScratchAddr g_scratch[kMaxDevices] = {};
+
+// Device address of g_bwd_scratch in the current device's context, looked up
+// once per context.
 cudaError_t scratch_for_current_device(double** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lock(g_setup_mutex);
-  if (g_scratch_ptr[dev] == nullptr) {
+  ScratchAddr& slot = g_scratch[dev];
+  const unsigned long long id = current_context_id();
+  if (slot.ptr == nullptr || id == 0 || id != slot.ctx_id) {
     void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_bwd_scratch);
+    e = cudaGetSymbolAddress(&p, g_bwd_scratch);  // makes the device's primary context current if needed
     if (e != cudaSuccess) return e;
-    g_scratch_ptr[dev] = static_cast<double*>(p);
+    slot.ptr = static_cast<double*>(p);
+    slot.ctx_id = current_context_id();
   }
-  *out = g_scratch_ptr[dev];
+  *out = slot.ptr;
   return cudaSuccess;
 }
 

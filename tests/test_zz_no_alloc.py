@@ -18,7 +18,7 @@ import torch
 
 import rwkv_wkv_recurrence_b200 as rw
 import wkv_inputs as wi
-from _parity import assert_grads_close
+from _parity import TOL_BF16, assert_close_rms, assert_grads_close
 
 pytestmark = pytest.mark.gpu
 
@@ -44,6 +44,23 @@ def test_noalloc_backward_matches_workspace_backward_twice(cuda_device):
     assert_grads_close(out1, tuple(x.double().cpu() for x in ref1), "first call ")
     out2, ref2 = _run_both(cuda_device, 3, 333, 100, 42)
     assert_grads_close(out2, tuple(x.double().cpu() for x in ref2), "second call ")
+    rw.rwkv_check_device_error()
+
+
+def test_noalloc_bf16_matches_workspace_backward(cuda_device):
+    # bf16 k, v, gy, gk, gv: the 8e-3 rule of the bf16 parity tests, twice in a row
+    for call, (B, T, C, seed) in enumerate(((2, 200, 64, 43), (4, 77, 48, 44))):
+        out, ref = _run_both(cuda_device, B, T, C, seed, dtype=torch.bfloat16)
+        for got, want, name in zip(out, ref, ("gk", "gv", "gw", "gu")):
+            assert_close_rms(got, want, TOL_BF16, f"call {call} {name} bf16")
+    rw.rwkv_check_device_error()
+
+
+def test_noalloc_at_full_capacity(cuda_device):
+    # B * C equal to the fixed scratch's capacity: the last lane of the array is used
+    B, T, C = 1, 16, rw.NOALLOC_MAX_LANES
+    out, ref = _run_both(cuda_device, B, T, C, 45)
+    assert_grads_close(out, tuple(x.double().cpu() for x in ref), "at capacity ")
     rw.rwkv_check_device_error()
 
 
