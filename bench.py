@@ -163,7 +163,7 @@ def _kernel_source_hash(kernel="wkv4_bwd_kernel"):
     csrc = os.path.join(ROOT, "rwkv_wkv_recurrence_b200", "csrc")
     prefix = _TRAFFIC_SOURCES[kernel]
     for f in sorted(os.listdir(csrc)):
-        if f.startswith(prefix) or f.endswith(".cuh") or f == "launch.h":
+        if f == prefix + ".cu" or f.endswith(".cuh") or f == "launch.h":
             with open(os.path.join(csrc, f), "rb") as fh:
                 h.update(fh.read())
     return h.hexdigest()[:16]
@@ -187,63 +187,14 @@ def _dist():
     return world, rank, local
 
 
-def run_reference(args):
-    """The fp64 CPU oracle, as it stands, on a bounded sample of the workload."""
-    world, rank, _ = _dist()
-    if rank != 0:
-        return
+def _oracle_sample(n_ch):
+    """The bounded sample the oracle is timed on: all batch rows and steps of n_ch of the
+    C channels (every C/n_ch-th), as fp64 [B, T, n_ch] arrays."""
     import numpy as np
     import torch
 
-    import oracle
     import wkv_inputs as wi
 
-    n_ch = args.ref_channels
-    chans = torch.arange(0, C, C // n_ch)[:n_ch]
-    w, u = wi.wkv4_params(SEED, C)
-    b_sel = torch.arange(B).repeat_interleave(n_ch)
-    c_sel = chans.repeat(B)
-    k = wi.btc_field("k", SEED, B, T, C, b_sel=b_sel, c_sel=c_sel, outliers=True).T.reshape(B, n_ch, T)
-    v = wi.btc_field("v", SEED, B, T, C, b_sel=b_sel, c_sel=c_sel).T.reshape(B, n_ch, T)
-    gy = wi.btc_field("gy", SEED, B, T, C, b_sel=b_sel, c_sel=c_sel).T.reshape(B, n_ch, T)
-    k, v, gy = (np.ascontiguousarray(x.permute(0, 2, 1).double().numpy()) for x in (k, v, gy))
-    ws, us = w[chans].double().numpy(), u[chans].double().numpy()
-    elems = B * T * n_ch
-
-    def step():
-        oracle.wkv4_forward(ws, us, k, v)
-        oracle.wkv4_backward(ws, us, k, v, gy)
-
-    for _ in range(args.warmup):
-        step()
-    t0 = time.perf_counter()
-    for _ in range(args.steps):
-        step()
-    dt = (time.perf_counter() - t0) / args.steps
-    val = elems / dt
-    sample = f"all {B} batch rows x {T} steps x {n_ch} of {C} channels (every {C // n_ch}th), fp64"
-    line = {
-        "impl": "reference", "metric": METRIC, "value": val, "unit": "elements/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "B": B, "T": T, "C": C, "sample_channels": n_ch},
-        "cpu_baseline": {"value": val, "unit": "elements/s", "cores": oracle.num_threads(), "kind": "oracle",
-                         "sample": sample},
-        "e2e": {"value": val, "unit": "elements/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
-    }
-    print(json.dumps(line), flush=True)
-
-
-def cpu_baseline(seconds_target=10.0):
-    """Times the oracle (fp64, OpenMP) on a bounded sample: all batch rows and
-    steps of a few channels, sized to a few seconds of CPU work."""
-    import numpy as np
-    import torch
-
-    import oracle
-    import wkv_inputs as wi
-
-    n_ch = 32
     chans = torch.arange(0, C, C // n_ch)[:n_ch]
     w, u = wi.wkv4_params(SEED, C)
     b_sel = torch.arange(B).repeat_interleave(n_ch)
@@ -253,18 +204,96 @@ def cpu_baseline(seconds_target=10.0):
         x = wi.btc_field(kind, SEED, B, T, C, b_sel=b_sel, c_sel=c_sel, outliers=out)  # [T, B*n]
         return np.ascontiguousarray(x.T.reshape(B, n_ch, T).permute(0, 2, 1).double().numpy())
 
-    k, v, gy = field("k", True), field("v"), field("gy")
-    ws, us = w[chans].double().numpy(), u[chans].double().numpy()
-    reps, t0 = 0, time.perf_counter()
-    while True:
-        oracle.wkv4_forward(ws, us, k, v)
-        oracle.wkv4_backward(ws, us, k, v, gy)
-        reps += 1
-        if time.perf_counter() - t0 >= seconds_target or reps >= 1000:
-            break
-    dt = (time.perf_counter() - t0) / reps
-    return {"value": B * T * n_ch / dt, "unit": "elements/s", "cores": oracle.num_threads(), "kind": "oracle",
-            "sample": f"{reps} x forward+backward over all {B} batch rows x {T} steps x {n_ch} of {C} channels, fp64"}
+    return (w[chans].double().numpy(), u[chans].double().numpy(), field("k", True), field("v"), field("gy"),
+            f"all {B} batch rows x {T} steps x {n_ch} of {C} channels (every {C // n_ch}th), fp64")
+
+
+def _oracle_step(oracle, ws, us, k, v, gy):
+    oracle.wkv4_forward(ws, us, k, v)
+    oracle.wkv4_backward(ws, us, k, v, gy)
+
+
+def run_reference(args):
+    """The fp64 CPU oracle, as it stands, on a bounded sample of the workload."""
+    world, rank, _ = _dist()
+    if rank != 0:
+        return
+    import oracle
+
+    ws, us, k, v, gy, sample = _oracle_sample(args.ref_channels)
+    elems = B * T * args.ref_channels
+    for _ in range(args.warmup):
+        _oracle_step(oracle, ws, us, k, v, gy)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        _oracle_step(oracle, ws, us, k, v, gy)
+    dt = (time.perf_counter() - t0) / args.steps
+    val = elems / dt
+    line = {
+        "impl": "reference", "metric": METRIC, "value": val, "unit": "elements/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "B": B, "T": T, "C": C, "sample_channels": args.ref_channels},
+        "cpu_baseline": {"value": val, "unit": "elements/s", "cores": oracle.num_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": val, "unit": "elements/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def cpu_baseline(seconds_target=10.0, n_ch=256):
+    """Times the oracle (fp64, OpenMP) on the reference arm's sample (all batch rows and
+    steps of n_ch channels), on all host cores and on one thread, about seconds_target
+    in total."""
+    import oracle
+
+    ws, us, k, v, gy, sample = _oracle_sample(n_ch)
+    all_cores = oracle.num_threads()
+
+    def timed(budget):
+        reps, t0 = 0, time.perf_counter()
+        while True:
+            _oracle_step(oracle, ws, us, k, v, gy)
+            reps += 1
+            if time.perf_counter() - t0 >= budget or reps >= 1000:
+                return reps, (time.perf_counter() - t0) / reps
+
+    _oracle_step(oracle, ws, us, k, v, gy)  # warm
+    reps, dt = timed(0.5 * seconds_target)
+    oracle.set_num_threads(1)
+    try:
+        reps1, dt1 = timed(0.5 * seconds_target)
+    finally:
+        oracle.set_num_threads(all_cores)
+    elems = B * T * n_ch
+    return {"value": elems / dt, "unit": "elements/s", "cores": all_cores, "kind": "oracle",
+            "one_thread": {"value": elems / dt1, "unit": "elements/s", "cores": 1, "reps": reps1},
+            "sample": f"{reps} x forward+backward over {sample}"}
+
+
+class _Nvtx:
+    """NVTX range around a library call (names the call in an nsys or ncu timeline)."""
+
+    def __init__(self, name):
+        self.name = name
+
+    def __enter__(self):
+        import torch
+
+        torch.cuda.nvtx.range_push(self.name)
+
+    def __exit__(self, *a):
+        import torch
+
+        torch.cuda.nvtx.range_pop()
+
+
+def _stats(ms_list):
+    """Mean, median and min of per-step device times (ms)."""
+    xs = sorted(ms_list)
+    n = len(xs)
+    med = xs[n // 2] if n % 2 else 0.5 * (xs[n // 2 - 1] + xs[n // 2])
+    return {"mean": sum(xs) / n, "median": med, "min": xs[0], "n": n}
 
 
 def run_ours(args):
@@ -305,14 +334,16 @@ def run_ours(args):
     P = rw._ptr
 
     def fwd():
-        s = h.rwkv_wkv4_forward(B, T, C, rw.F32, P(w), P(u), P(k), P(v), P(y), None, None, P(ck), rw.CHUNK_LEN,
-                                rw.ALGO_AUTO, P(fw), fws, sp)
+        with _Nvtx("rwkv_wkv4_forward"):
+            s = h.rwkv_wkv4_forward(B, T, C, rw.F32, P(w), P(u), P(k), P(v), P(y), None, None, P(ck),
+                                    rw.CHUNK_LEN, rw.ALGO_AUTO, P(fw), fws, sp)
         if s:
             raise rw.RwkvError("rwkv_wkv4_forward", s)
 
     def bwd():
-        s = h.rwkv_wkv4_backward(B, T, C, rw.F32, P(w), P(u), P(k), P(v), P(gy), None, P(ck), rw.CHUNK_LEN,
-                                 P(gk), P(gv), P(gw), P(gu), P(bw), bws, sp)
+        with _Nvtx("rwkv_wkv4_backward"):
+            s = h.rwkv_wkv4_backward(B, T, C, rw.F32, P(w), P(u), P(k), P(v), P(gy), None, P(ck), rw.CHUNK_LEN,
+                                     P(gk), P(gv), P(gw), P(gu), P(bw), bws, sp)
         if s:
             raise rw.RwkvError("rwkv_wkv4_backward", s)
 
@@ -346,22 +377,25 @@ def run_ours(args):
     total_ms = start.elapsed_time(end)
     fwd_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
     bwd_ms = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
+    step_stats = _stats([e[0].elapsed_time(e[2]) for e in evs])
     ms_step = max_over_ranks(total_ms, dev) / args.steps
     value = weak_scaling_throughput(ELEM, world, ms_step)
 
     # end to end through the public API with host buffers (pinned), copies timed
     hk, hv, hgy = (x.cpu().pin_memory() for x in (k, v, gy))
     hw, hu = w.cpu().pin_memory(), u.cpu().pin_memory()
-    hgk, hgv = torch.empty_like(hk).pin_memory(), torch.empty_like(hv).pin_memory()
+    hy, hgk, hgv = (torch.empty_like(hk).pin_memory() for _ in range(3))
     hgw, hgu = torch.empty(C).pin_memory(), torch.empty(C).pin_memory()
 
     def e2e_step():
-        for dst, src in ((k, hk), (v, hv), (gy, hgy), (w, hw), (u, hu)):
-            dst.copy_(src, non_blocking=True)
+        with _Nvtx("e2e h2d"):
+            for dst, src in ((k, hk), (v, hv), (gy, hgy), (w, hw), (u, hu)):
+                dst.copy_(src, non_blocking=True)
         fwd()
         bwd()
-        for dst, src in ((hgk, gk), (hgv, gv), (hgw, gw), (hgu, gu)):
-            dst.copy_(src, non_blocking=True)
+        with _Nvtx("e2e d2h"):
+            for dst, src in ((hy, y), (hgk, gk), (hgv, gv), (hgw, gw), (hgu, gu)):
+                dst.copy_(src, non_blocking=True)
 
     e2e_steps = max(1, min(args.steps, 5))
     e2e_step()
@@ -386,13 +420,14 @@ def run_ours(args):
                        "l2": "no flush: every input (k, v, gy: 268 MB each) is larger than the 126 MB L2",
                        "parallelism": f"{world} independent problems, no collective"},
             "hbm_gbs_step": step_gbs, "hbm_frac_step": step_gbs / peak,
+            "step_ms": step_stats,
             "kernels_ms": {"wkv4_forward": fwd_ms, "wkv4_backward": bwd_ms},
             "roofline": {"bound": "hbm", "kernel": "wkv4_bwd_kernel (+ its gw/gu batch reduction)",
                          "achieved": bwd_gbs, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                          "frac": bwd_gbs / peak,
                          "traffic": args.traffic if args.traffic is not None else _recorded_traffic()},
             "e2e": {"value": e2e_val, "unit": "elements/s",
-                    "h2d_bytes_per_step": 3 * 4 * ELEM + 2 * 4 * C, "d2h_bytes_per_step": 2 * 4 * ELEM + 2 * 4 * C},
+                    "h2d_bytes_per_step": 3 * 4 * ELEM + 2 * 4 * C, "d2h_bytes_per_step": 3 * 4 * ELEM + 2 * 4 * C},
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clk.summary(),
         }
@@ -406,23 +441,25 @@ def run_ours(args):
 
 def _timed(fn, steps, warmup, stream, local):
     """W untimed calls, then K calls bracketed by synchronisation, CUDA events
-    on the launching stream; returns (ms per call, clock summary)."""
+    on the launching stream; returns (mean ms per call, clock summary, per-call
+    mean/median/min)."""
     import torch
 
     for _ in range(warmup):
         fn(0)
     torch.cuda.synchronize()
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
     with ClockSampler(local) as clk:
         torch.cuda.synchronize()
         wall0 = time.perf_counter()
-        start.record(stream)
+        evs[0].record(stream)
         for i in range(steps):
             fn(i)
-        end.record(stream)
+            evs[i + 1].record(stream)
         torch.cuda.synchronize()
         clk.mark(wall0, time.perf_counter())
-    return start.elapsed_time(end) / steps, clk.summary()
+    stats = _stats([evs[i].elapsed_time(evs[i + 1]) for i in range(steps)])
+    return evs[0].elapsed_time(evs[-1]) / steps, clk.summary(), stats
 
 
 def run_decode(args):
@@ -459,7 +496,7 @@ def run_decode(args):
         if s:
             raise rw.RwkvError("rwkv_wkv4_step", s)
 
-    ms, clk = _timed(step, args.steps, args.warmup, stream, local)
+    ms, clk, stats = _timed(step, args.steps, args.warmup, stream, local)
     rw.rwkv_check_device_error()
     graph = _graph_decode_timing(rw, h, st, w, u, ks, vs, y, Bd, Cd, Td, dev)
     lanes = Bd * Cd
@@ -475,7 +512,7 @@ def run_decode(args):
         "roofline": {"bound": "hbm", "kernel": "wkv4_step_kernel", "achieved": gbs, "peak": peak,
                      "peak_kind": kind, "unit": "GB/s", "frac": gbs / peak,
                      "traffic": _recorded_traffic("wkv4_step_kernel")},
-        "gpu_launches": args.steps, "clocks": clk, "cuda_graph": graph}), flush=True)
+        "gpu_launches": args.steps, "clocks": clk, "call_ms": stats, "cuda_graph": graph}), flush=True)
 
 
 def _graph_decode_timing(rw, h, st, w, u, ks, vs, y, Bd, Cd, Td, dev):
@@ -567,9 +604,9 @@ def run_train_gated(args):
         fwd()
         bwd()
 
-    ms, clk = _timed(step, args.steps, args.warmup, stream, local)
-    fwd_ms, _ = _timed(fwd, args.steps, args.warmup, stream, local)
-    bwd_ms, _ = _timed(bwd, args.steps, args.warmup, stream, local)
+    ms, clk, stats = _timed(step, args.steps, args.warmup, stream, local)
+    fwd_ms, _, _ = _timed(fwd, args.steps, args.warmup, stream, local)
+    bwd_ms, _, _ = _timed(bwd, args.steps, args.warmup, stream, local)
     rw.rwkv_check_device_error()
     fwd_bytes = 4 * 4 * ELEM                      # k, v, r read; o written
     bwd_bytes = 7 * 4 * ELEM + 2 * 4 * C          # k, v, r, go read; gk, gv, gr written; gw, gu
@@ -588,7 +625,86 @@ def run_train_gated(args):
         "roofline": {"bound": "hbm", "kernel": "wkv4_bwd_kernel<float, gated> (+ its gw/gu batch reduction)",
                      "achieved": bwd_gbs, "peak": peak, "peak_kind": kind, "unit": "GB/s",
                      "frac": bwd_gbs / peak, "traffic": _recorded_traffic("wkv4_bwd_kernel/gated")},
-        "gpu_launches": 3 * args.steps, "clocks": clk}), flush=True)
+        "gpu_launches": 3 * args.steps, "clocks": clk, "call_ms": stats}), flush=True)
+
+
+def run_chunked(args):
+    """The few-channel forward: B=8 T=1024 C=768 fp32 with 1 % +-U(20,40) key outliers
+    (6,144 channel lanes, too few to fill the GPU one thread per lane).  Its 75.5 MB
+    fit in the 126 MB L2, so every timed call follows a write of a 256 MB buffer that
+    evicts them (cold); back-to-back calls without the flush are reported beside
+    (warm).  AUTO (which picks the chunked schedule here), SEQUENTIAL and CHUNKED are
+    timed side by side."""
+    import torch
+
+    import rwkv_wkv_recurrence_b200 as rw
+    import wkv_inputs as wi
+
+    _, _, local = _dist()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    Bc, Tc, Cc = 8, 1024, 768
+    p = wi.wkv4_problem(Bc, Tc, Cc, wi.CONFIG_SEED_BASE + 1, outliers=True, device=dev)
+    w, u, k, v = p["w"], p["u"], p["k"], p["v"]
+    y = torch.empty_like(k)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    h = rw.lib()
+    stream = torch.cuda.current_stream()
+    sp, P = rw._stream(stream), rw._ptr
+    elems = Bc * Tc * Cc
+    nbytes = 3 * 4 * elems + 2 * 4 * Cc  # k, v read, y written; w, u
+    peak, kind = _peaks()
+    names = {rw.ALGO_AUTO: "auto", rw.ALGO_SEQUENTIAL: "sequential", rw.ALGO_CHUNKED: "chunked"}
+    res = {}
+    clk_all = None
+    for algo in (rw.ALGO_AUTO, rw.ALGO_SEQUENTIAL, rw.ALGO_CHUNKED):
+        wsb = int(h.rwkv_wkv4_forward_workspace_bytes(Bc, Tc, Cc, algo))
+        ws = torch.empty(max(wsb, 1), dtype=torch.uint8, device=dev)
+
+        def call(i=0):
+            with _Nvtx("rwkv_wkv4_forward"):
+                s = h.rwkv_wkv4_forward(Bc, Tc, Cc, rw.F32, P(w), P(u), P(k), P(v), P(y), None, None, None,
+                                        rw.CHUNK_LEN, algo, P(ws), wsb, sp)
+            if s:
+                raise rw.RwkvError("rwkv_wkv4_forward", s)
+
+        for _ in range(args.warmup):
+            call()
+        reps = max(20, min(args.steps, 200))
+        cold = []
+        with ClockSampler(local) as clk:
+            torch.cuda.synchronize()
+            wall0 = time.perf_counter()
+            for _ in range(reps):
+                flush.zero_()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                call()
+                e1.record(stream)
+                e1.synchronize()
+                cold.append(e0.elapsed_time(e1))
+            clk.mark(wall0, time.perf_counter())
+        warm_ms, _, warm = _timed(call, reps, 1, stream, local)
+        rw.rwkv_check_device_error()
+        st = _stats(cold)
+        res[names[algo]] = {"cold_ms": st, "warm_ms": warm, "workspace_bytes": wsb,
+                            "cold_gbs_median": nbytes / (st["median"] * 1e-3) / 1e9,
+                            "warm_gbs_median": nbytes / (warm["median"] * 1e-3) / 1e9}
+        if algo == rw.ALGO_AUTO:
+            clk_all = clk.summary()
+    auto = res["auto"]["cold_ms"]["median"]
+    gbs = nbytes / (auto * 1e-3) / 1e9
+    print(json.dumps({
+        "metric": "WKV-4 forward elements/s and HBM GB/s, few channels (B8 T1024 C768)",
+        "value": elems / (auto * 1e-3), "unit": "elements/s", "n_gpus": 1, "steps": len(res["auto"]["cold_ms"]),
+        "warmup": args.warmup, "ms_per_step": auto, "higher_is_better": True, "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": "RWKV-4 WKV forward, fp32, B=8 T=1024 C=768, 1% +-U(20,40) key outliers",
+                   "l2": "flushed: a 256 MB buffer is written before every timed call (inputs fit in L2)"},
+        "roofline": {"bound": "hbm", "kernel": "wkv4_fwd_kernel x2 + wkv4_carry_kernel (AUTO picks chunked)",
+                     "achieved": gbs, "peak": peak, "peak_kind": kind, "unit": "GB/s", "frac": gbs / peak,
+                     "traffic": None},
+        "schedules": res, "gpu_launches": 3, "clocks": clk_all}), flush=True)
 
 
 def run_eagle(args, finch=False):
@@ -623,7 +739,7 @@ def run_eagle(args, finch=False):
         if s:
             raise rw.RwkvError(name, s)
 
-    ms, clk = _timed(call, args.steps, args.warmup, stream, local)
+    ms, clk, stats = _timed(call, args.steps, args.warmup, stream, local)
     rw.rwkv_check_device_error()
     elems = Be * Te * He * Ne
     # r, k, v, y bf16; s_out; u (and omega: per token fp32 for Finch, [H,N] fp32 for Eagle)
@@ -648,7 +764,7 @@ def run_eagle(args, finch=False):
         "config": {"workload": workload, "l2": l2},
         "roofline": {"bound": "hbm", "kernel": kernel, "achieved": gbs, "peak": peak, "peak_kind": kind,
                      "unit": "GB/s", "frac": gbs / peak, "traffic": _recorded_traffic(kernel)},
-        "gpu_launches": args.steps, "clocks": clk}), flush=True)
+        "gpu_launches": args.steps, "clocks": clk, "call_ms": stats}), flush=True)
 
 
 def run_eagle_decode(args, finch=False):
@@ -685,7 +801,7 @@ def run_eagle_decode(args, finch=False):
         if s:
             raise rw.RwkvError("rwkv_wkv6_step" if finch else "rwkv_wkv5_step", s)
 
-    ms, clk = _timed(step, args.steps, args.warmup, stream, local)
+    ms, clk, stats = _timed(step, args.steps, args.warmup, stream, local)
     heads = Bs * Hs
     # state in + out; r, k, v, y bf16; u (and omega: per stream for Finch, per head for Eagle)
     bytes_step = heads * (2 * Ns * Ns * 4 + 4 * Ns * 2) + Hs * Ns * 4 + (heads * Ns * 4 if finch else Hs * Ns * 4)
@@ -703,7 +819,7 @@ def run_eagle_decode(args, finch=False):
         "roofline": {"bound": "hbm", "kernel": "wkv5_step_kernel", "achieved": gbs, "peak": peak,
                      "peak_kind": kind, "unit": "GB/s", "frac": gbs / peak,
                      "traffic": _recorded_traffic("wkv5_step_kernel/finch" if finch else "wkv5_step_kernel")},
-        "gpu_launches": args.steps, "clocks": clk}), flush=True)
+        "gpu_launches": args.steps, "clocks": clk, "call_ms": stats}), flush=True)
 
 
 def main():
@@ -712,11 +828,11 @@ def main():
     ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["train", "train_gated", "decode", "eagle", "eagle_decode", "finch",
-                                           "finch_decode"],
+    ap.add_argument("--workload", choices=["train", "train_gated", "decode", "chunked", "eagle", "eagle_decode",
+                                           "finch", "finch_decode"],
                     default="train",
-                    help="train: the headline forward+backward step; train_gated, decode, eagle, eagle_decode, "
-                         "finch, finch_decode: the other hot-path rows")
+                    help="train: the headline forward+backward step; train_gated, decode, chunked, eagle, "
+                         "eagle_decode, finch, finch_decode: the other hot-path rows")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--ref-channels", type=int, default=256)
@@ -729,6 +845,8 @@ def main():
         run_reference(args)
     elif args.workload == "decode":
         run_decode(args)
+    elif args.workload == "chunked":
+        run_chunked(args)
     elif args.workload == "train_gated":
         run_train_gated(args)
     elif args.workload == "eagle":

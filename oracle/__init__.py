@@ -61,6 +61,8 @@ def _load():
             f.argtypes = args
             f.restype = ctypes.c_int64
         lib.oracle_num_threads.restype = ctypes.c_int
+        lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
+        lib.oracle_set_num_threads.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -68,6 +70,11 @@ def _load():
 def num_threads() -> int:
     """OpenMP threads the oracle runs on (OMP_NUM_THREADS, else all cores)."""
     return int(_load().oracle_num_threads())
+
+
+def set_num_threads(n: int) -> int:
+    """Runs later oracle calls on n OpenMP threads; returns the count in force."""
+    return int(_load().oracle_set_num_threads(int(n)))
 
 
 def _f64(x):

@@ -77,6 +77,18 @@ int oracle_num_threads(void)
 #endif
 }
 
+/* Sets the OpenMP thread count of later calls (n >= 1); returns the count in force. */
+int oracle_set_num_threads(int n)
+{
+#ifdef _OPENMP
+    if (n >= 1) omp_set_num_threads(n);
+    return omp_get_max_threads();
+#else
+    (void)n;
+    return 1;
+#endif
+}
+
 #define IDX3(b, t, c) ((((int64_t)(b)) * T + (t)) * C + (c))
 
 /*
