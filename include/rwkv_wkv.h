@@ -44,10 +44,15 @@
  *     before anything is enqueued.  A launch failure gives RWKV_ERR_CUDA.
  *     Zero-sized problems are a successful no-op (T = 0 copies the state).
  *   - Values are data: no range validation; NaN and Inf propagate.
- *   - Alignment: the WKV-4 [B,T,C] tensors k, v, y, gy, gk, gv, r, o, go, gr (and the WKV-5
- *     tensors r, k, v, y, and Finch's omega) must be 16-byte aligned with
- *     C·sizeof(element) a multiple of 16 (TMA row pitch), else
- *     RWKV_ERR_UNSUPPORTED.
+ *   - Alignment.  WKV-4 [B,T,C] tensors (k, v, y, gy, gk, gv, r, o, go, gr)
+ *     whose bases are all 16-byte aligned, with C·sizeof(element) a multiple
+ *     of 16, move through TMA; any other element-aligned bases or C take the
+ *     plain-access instances of the same kernels (same results, fewer bytes
+ *     in flight).  A pointer not aligned to its element size (4 bytes fp32,
+ *     2 bytes bf16) gives RWKV_ERR_UNSUPPORTED.  The WKV-5/6 tensors r, k, v,
+ *     y (and Finch's omega) must be 16-byte aligned (their rows are whole
+ *     heads of 64), else RWKV_ERR_UNSUPPORTED; rwkv_wkv4_backward_noalloc
+ *     keeps to the TMA conditions.
  */
 #ifndef RWKV_WKV_H
 #define RWKV_WKV_H
@@ -266,7 +271,9 @@ RWKV_API rwkv_status rwkv_wkv6_step(int64_t B, int64_t H, int64_t N, const void 
  * memory owned in full by another allocator, latency-critical loops that
  * must not pay cudaMalloc's implicit synchronisation, systems that allocate
  * only at start-up).  Same arguments and results as rwkv_wkv4_backward with
- * ckpt required (the forward's checkpoints) and no workspace; the per-lane
+ * ckpt required (the forward's checkpoints), no workspace, and the TMA
+ * alignment (16-byte bases, C·sizeof(element) a multiple of 16; else
+ * RWKV_ERR_UNSUPPORTED); the per-lane
  * scratch lives in a fixed array inside the library (RWKV_NOALLOC_MAX_LANES
  * lanes, 4 MiB, held on every GPU that loads the library until exit).
  *   - B * C > RWKV_NOALLOC_MAX_LANES returns RWKV_ERR_WORKSPACE (too big for
@@ -297,6 +304,25 @@ RWKV_API rwkv_status rwkv_wkv4_backward_noalloc(int64_t B, int64_t T, int64_t C,
  * know which call timed out must check after each call, in stream order.
  */
 RWKV_API rwkv_status rwkv_check_device_error(rwkv_stream_t stream);
+
+/*
+ * Test hooks for the failure path of the bounded waits (the pages have no
+ * counterpart; they exist so that a test can watch a wait give up without
+ * faulting or hanging the GPU).  Both act on the current device, synchronise
+ * it first, and hold until changed; they are not meant for production use.
+ *
+ * rwkv_debug_set_wait_limit_ns: how long every bounded wait of the library's
+ *   kernels polls before giving up (it then sets RWKV_ERR_DEVICE_TIMEOUT in
+ *   the device error word and the CTA leaves at its next barrier, after
+ *   waiting, bounded again, for the copies and MMAs it had issued).  ns = 0
+ *   restores the default of one second.
+ * rwkv_debug_withhold_loads: on != 0 makes the thread that issues a kernel's
+ *   TMA loads arm its barrier and issue none, so the first wait of every CTA
+ *   runs out with nothing in flight; on = 0 restores normal operation.
+ *   Calls return RWKV_OK meanwhile and their outputs are undefined.
+ */
+RWKV_API rwkv_status rwkv_debug_set_wait_limit_ns(uint64_t ns);
+RWKV_API rwkv_status rwkv_debug_withhold_loads(int on);
 
 #ifdef __cplusplus
 }

@@ -72,6 +72,8 @@ def lib():
         "rwkv_wkv6_forward": ([I64, I64, I64, I64, P, P, P, P, P, P, P, P, P, S, P], I),
         "rwkv_wkv6_step": ([I64, I64, I64, P, P, P, P, P, P, P, P, P], I),
         "rwkv_check_device_error": ([P], I),
+        "rwkv_debug_set_wait_limit_ns": ([ctypes.c_uint64], I),
+        "rwkv_debug_withhold_loads": ([I], I),
     }
     for name, (args, res) in sig.items():
         f = getattr(h, name)

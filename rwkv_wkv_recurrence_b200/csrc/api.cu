@@ -1,16 +1,20 @@
 // C-ABI layer: argument validation, workspace planning, TMA descriptors and
 // kernel dispatch for the calls declared in include/rwkv_wkv.h.
 #include <climits>
+#include <cstddef>
 #include <cstring>
+#include <initializer_list>
 #include <mutex>
 
 #include "../../include/rwkv_wkv.h"
 #include "launch.h"
+#include "wkv_common.cuh"
 
 namespace rwkv {
 
-// The library's device error word (one per device that loads the library).
-__device__ unsigned int g_device_error = 0;
+// The library's device control block (one per device that loads the library):
+// error word, load-withholding test hook, bounded-wait limit.
+__device__ DevCtl g_ctl = {0u, 0u, kDefaultWaitLimitNs};
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -73,9 +77,9 @@ bool make_f32_box32_map(CUtensorMap* m, const void* base, int B, int T, int W) {
   return r == CUDA_SUCCESS;
 }
 
-unsigned int* device_error_word() {
-  unsigned int* p = nullptr;
-  if (cudaGetSymbolAddress(reinterpret_cast<void**>(&p), g_device_error) != cudaSuccess) return nullptr;
+DevCtl* device_ctl() {
+  DevCtl* p = nullptr;
+  if (cudaGetSymbolAddress(reinterpret_cast<void**>(&p), g_ctl) != cudaSuccess) return nullptr;
   return p;
 }
 
@@ -85,6 +89,25 @@ constexpr int kDesignSMs = 148;  // B200 SM count the schedules are planned for
 constexpr int kCkLen = 16;       // checkpoint interval the backward reads
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Element alignment (4 bytes for fp32, 2 for bf16): the least the kernels' plain accesses need.
+bool elem_aligned(const void* p, bool bf16) { return (reinterpret_cast<uintptr_t>(p) & (bf16 ? 1u : 3u)) == 0; }
+
+// The WKV-4 [B,T,C] tensors go through TMA when every base is 16-byte aligned and the row pitch
+// C * sizeof(element) is a multiple of 16 bytes; otherwise the same kernels use plain element
+// loads and stores (null entries are skipped).
+bool tma_ok(int64_t C, bool bf16, std::initializer_list<const void*> ptrs) {
+  if ((C * (bf16 ? 2 : 4)) % 16 != 0) return false;
+  for (const void* q : ptrs)
+    if (q != nullptr && !aligned16(q)) return false;
+  return true;
+}
+
+bool all_elem_aligned(bool bf16, std::initializer_list<const void*> ptrs) {
+  for (const void* q : ptrs)
+    if (q != nullptr && !elem_aligned(q, bf16)) return false;
+  return true;
+}
 
 bool fits_int(int64_t x) { return x >= 0 && x <= INT_MAX; }
 
@@ -125,35 +148,44 @@ FwdPlan plan_forward(int64_t B, int64_t T, int64_t C, int algo) {
 rwkv_status run_forward(int B, int T, int C, bool bf16, const float* w, const float* u, const void* k,
                         const void* v, void* y, const float* state_in, float* state_out, float* ckpt, int ckpt_len,
                         const FwdPlan& pl, void* ws, cudaStream_t st, const void* r = nullptr) {
-  unsigned int* err = device_error_word();
-  if (err == nullptr) return RWKV_ERR_CUDA;
+  DevCtl* ctl = device_ctl();
+  if (ctl == nullptr) return RWKV_ERR_CUDA;
   const int tt = fwd_tile_steps();
   const bool gate = r != nullptr && y != nullptr;
+  const bool tma = tma_ok(C, bf16, {k, v, y, gate ? r : nullptr});
   CUtensorMap mk, mv, my, mr;
-  if (!make_btc_map(&mk, k, bf16, B, T, C, tt) || !make_btc_map(&mv, v, bf16, B, T, C, tt)) return RWKV_ERR_CUDA;
-  if (gate && !make_btc_map(&mr, r, bf16, B, T, C, tt)) return RWKV_ERR_CUDA;
+  std::memset(&mk, 0, sizeof(mk));  // the plain-access path reads no map
+  mv = my = mr = mk;
+  if (tma) {
+    if (!make_btc_map(&mk, k, bf16, B, T, C, tt) || !make_btc_map(&mv, v, bf16, B, T, C, tt)) return RWKV_ERR_CUDA;
+    if (gate && !make_btc_map(&mr, r, bf16, B, T, C, tt)) return RWKV_ERR_CUDA;
+    if (y != nullptr) {
+      if (!make_btc_map(&my, y, bf16, B, T, C, fwd_store_steps())) return RWKV_ERR_CUDA;
+    } else {
+      my = mk;  // not read without y
+    }
+  }
   auto launch_out = [&](const Fwd4Params& q) {  // the pass that writes the outputs
     return gate ? launch_wkv4_fwd_gated(bf16, mk, mv, my, mr, q, st) : launch_wkv4_fwd(bf16, mk, mv, my, q, st);
   };
-  if (y != nullptr) {
-    if (!make_btc_map(&my, y, bf16, B, T, C, fwd_store_steps())) return RWKV_ERR_CUDA;
-  } else {
-    my = mk;  // not read without y
-  }
   Fwd4Params p{};
+  p.tma = tma ? 1 : 0;
+  p.k = k;
+  p.v = v;
+  p.r = gate ? r : nullptr;
   p.B = B;
   p.T = T;
   p.C = C;
   p.ctiles = (C + 31) / 32;
   p.w = w;
   p.u = u;
-  p.err = err;
+  p.ctl = ctl;
   p.ckpt_len = ckpt_len;
   const long long seg_stride = 3LL * B * C;
   if (pl.algo == RWKV_ALGO_SEQUENTIAL) {
     p.seg_len = pl.seg_len;
     p.nseg = 1;
-    p.stages = fwd_stages(bf16, pl.seg_len, gate);
+    p.stages = fwd_stages(bf16, pl.seg_len, gate, tma);
     p.y = y;
     p.start = state_in;
     p.end = state_out;
@@ -165,7 +197,7 @@ rwkv_status run_forward(int B, int T, int C, bool bf16, const float* w, const fl
   // 1) segment summaries from a zero state
   p.seg_len = pl.seg_len;
   p.nseg = pl.nseg;
-  p.stages = fwd_stages(bf16, pl.seg_len);
+  p.stages = fwd_stages(bf16, pl.seg_len, false, tma);
   p.y = nullptr;
   p.start = nullptr;
   p.end = wsf;
@@ -181,7 +213,7 @@ rwkv_status run_forward(int B, int T, int C, bool bf16, const float* w, const fl
   p.start_seg_stride = seg_stride;
   p.end = nullptr;
   p.ckpt = ckpt;
-  p.stages = fwd_stages(bf16, pl.seg_len, gate);
+  p.stages = fwd_stages(bf16, pl.seg_len, gate, tma);
   if (launch_out(p) != cudaSuccess) return RWKV_ERR_CUDA;
   return RWKV_OK;
 }
@@ -237,8 +269,7 @@ rwkv_status rwkv_wkv4_forward(int64_t B, int64_t T, int64_t C, rwkv_dtype dtype,
   if (k == nullptr || v == nullptr) return RWKV_ERR_INVALID_ARG;
   if (y == nullptr && state_out == nullptr && ckpt == nullptr) return RWKV_ERR_INVALID_ARG;
   const bool bf16 = dtype == RWKV_BF16;
-  if (!aligned16(k) || !aligned16(v) || (y != nullptr && !aligned16(y)) || (C * (bf16 ? 2 : 4)) % 16 != 0)
-    return RWKV_ERR_UNSUPPORTED;
+  if (!all_elem_aligned(bf16, {k, v, y})) return RWKV_ERR_UNSUPPORTED;
   const FwdPlan pl = plan_forward(B, T, C, algo);
   if (pl.ws_bytes > 0 && (workspace == nullptr || workspace_bytes < pl.ws_bytes)) return RWKV_ERR_WORKSPACE;
   return run_forward((int)B, (int)T, (int)C, bf16, w, u, k, v, y, state_in, state_out, ckpt, (int)chunk_len, pl,
@@ -264,8 +295,7 @@ rwkv_status rwkv_wkv4_forward_gated(int64_t B, int64_t T, int64_t C, rwkv_dtype 
   }
   if (k == nullptr || v == nullptr || r == nullptr || o == nullptr) return RWKV_ERR_INVALID_ARG;
   const bool bf16 = dtype == RWKV_BF16;
-  if (!aligned16(k) || !aligned16(v) || !aligned16(r) || !aligned16(o) || (C * (bf16 ? 2 : 4)) % 16 != 0)
-    return RWKV_ERR_UNSUPPORTED;
+  if (!all_elem_aligned(bf16, {k, v, r, o})) return RWKV_ERR_UNSUPPORTED;
   const FwdPlan pl = plan_forward(B, T, C, algo);
   if (pl.ws_bytes > 0 && (workspace == nullptr || workspace_bytes < pl.ws_bytes)) return RWKV_ERR_WORKSPACE;
   return run_forward((int)B, (int)T, (int)C, bf16, w, u, k, v, o, state_in, state_out, ckpt, (int)chunk_len, pl,
@@ -305,10 +335,9 @@ rwkv_status backward_impl(bool gate, int64_t B, int64_t T, int64_t C, rwkv_dtype
   if (k == nullptr || v == nullptr || gk == nullptr || gv == nullptr) return RWKV_ERR_INVALID_ARG;
   if (gate ? (r == nullptr || go == nullptr || gr == nullptr) : gy == nullptr) return RWKV_ERR_INVALID_ARG;
   const bool bf16 = dtype == RWKV_BF16;
-  const bool in_ok = gate ? aligned16(r) && aligned16(go) && aligned16(gr) : aligned16(gy);
-  if (!aligned16(k) || !aligned16(v) || !in_ok || !aligned16(gk) || !aligned16(gv) ||
-      (C * (bf16 ? 2 : 4)) % 16 != 0)
-    return RWKV_ERR_UNSUPPORTED;
+  if (!all_elem_aligned(bf16, {k, v, gy, r, go, gr, gk, gv})) return RWKV_ERR_UNSUPPORTED;
+  // r and gr are read and written with plain accesses on either path
+  const bool tma = tma_ok(C, bf16, {k, v, gate ? go : gy, gk, gv});
   const size_t need = rwkv_wkv4_backward_workspace_bytes(B, T, C, chunk_len, ckpt != nullptr);
   if (workspace == nullptr || workspace_bytes < need) return RWKV_ERR_WORKSPACE;
   const int iB = (int)B, iT = (int)T, iC = (int)C;
@@ -322,28 +351,34 @@ rwkv_status backward_impl(bool gate, int64_t B, int64_t T, int64_t C, rwkv_dtype
     if (s != RWKV_OK) return s;
     ck = ckw;
   }
-  unsigned int* err = device_error_word();
-  if (err == nullptr) return RWKV_ERR_CUDA;
+  DevCtl* ctl = device_ctl();
+  if (ctl == nullptr) return RWKV_ERR_CUDA;
   const int box_t = bwd_tile_steps();
   CUtensorMap mk, mv, mg, mgk, mgv;
-  if (!make_btc_map(&mk, k, bf16, iB, iT, iC, box_t) || !make_btc_map(&mv, v, bf16, iB, iT, iC, box_t) ||
-      !make_btc_map(&mg, gate ? go : gy, bf16, iB, iT, iC, box_t) ||
-      !make_btc_map(&mgk, gk, bf16, iB, iT, iC, bwd_store_steps()) ||
-      !make_btc_map(&mgv, gv, bf16, iB, iT, iC, bwd_store_steps()))
+  std::memset(&mk, 0, sizeof(mk));  // the plain-access path reads no map
+  mv = mg = mgk = mgv = mk;
+  if (tma && (!make_btc_map(&mk, k, bf16, iB, iT, iC, box_t) || !make_btc_map(&mv, v, bf16, iB, iT, iC, box_t) ||
+              !make_btc_map(&mg, gate ? go : gy, bf16, iB, iT, iC, box_t) ||
+              !make_btc_map(&mgk, gk, bf16, iB, iT, iC, bwd_store_steps()) ||
+              !make_btc_map(&mgv, gv, bf16, iB, iT, iC, bwd_store_steps())))
     return RWKV_ERR_CUDA;
   Bwd4Params p{};
   p.B = iB;
   p.T = iT;
   p.C = iC;
   p.ctiles = (iC + 31) / 32;
-  p.stages = bwd_stages(bf16, iT, gate);
+  p.stages = bwd_stages(bf16, iT, gate, tma);
+  p.tma = tma ? 1 : 0;
+  p.k = k;
+  p.v = v;
+  p.g = gate ? go : gy;
   p.w = w;
   p.u = u;
   p.ckpt = ck;
   p.gk = gk;
   p.gv = gv;
   p.part = part;
-  p.err = err;
+  p.ctl = ctl;
   p.r = r;
   p.gr = gr;
   const cudaError_t e = gate ? launch_wkv4_bwd_gated(bf16, mk, mv, mg, mgk, mgv, p, st)
@@ -421,8 +456,8 @@ rwkv_status rwkv_wkv5_forward(int64_t B, int64_t T, int64_t H, int64_t N, const 
   if (r == nullptr || k == nullptr || v == nullptr || y == nullptr) return RWKV_ERR_INVALID_ARG;
   if (!aligned16(r) || !aligned16(k) || !aligned16(v) || !aligned16(y)) return RWKV_ERR_UNSUPPORTED;
   if ((int64_t)H * 64 > INT_MAX || (int64_t)B * H > INT_MAX) return RWKV_ERR_UNSUPPORTED;
-  unsigned int* err = device_error_word();
-  if (err == nullptr) return RWKV_ERR_CUDA;
+  DevCtl* ctl = device_ctl();
+  if (ctl == nullptr) return RWKV_ERR_CUDA;
   const int iB = (int)B, iT = (int)T, iH = (int)H;
   CUtensorMap mr, mk, mv;
   if (!make_bf16_box64_map(&mr, r, iB, iT, iH * 64) || !make_bf16_box64_map(&mk, k, iB, iT, iH * 64) ||
@@ -440,7 +475,7 @@ rwkv_status rwkv_wkv5_forward(int64_t B, int64_t T, int64_t H, int64_t N, const 
   p.y = static_cast<__nv_bfloat16*>(y);
   p.s_in = s_in;
   p.s_out = s_out;
-  p.err = err;
+  p.ctl = ctl;
   if (launch_wkv5_fwd(mr, mk, mv, p, st) != cudaSuccess) return RWKV_ERR_CUDA;
   return RWKV_OK;
 }
@@ -503,8 +538,8 @@ rwkv_status rwkv_wkv6_forward(int64_t B, int64_t T, int64_t H, int64_t N, const 
   if (!aligned16(r) || !aligned16(k) || !aligned16(v) || !aligned16(y) || !aligned16(omega))
     return RWKV_ERR_UNSUPPORTED;
   if ((int64_t)H * 64 > INT_MAX || (int64_t)B * H > INT_MAX) return RWKV_ERR_UNSUPPORTED;
-  unsigned int* err = device_error_word();
-  if (err == nullptr) return RWKV_ERR_CUDA;
+  DevCtl* ctl = device_ctl();
+  if (ctl == nullptr) return RWKV_ERR_CUDA;
   const int iB = (int)B, iT = (int)T, iH = (int)H;
   CUtensorMap mr, mk, mv, mw;
   if (!make_bf16_box64_map(&mr, r, iB, iT, iH * 64) || !make_bf16_box64_map(&mk, k, iB, iT, iH * 64) ||
@@ -522,7 +557,7 @@ rwkv_status rwkv_wkv6_forward(int64_t B, int64_t T, int64_t H, int64_t N, const 
   p.y = static_cast<__nv_bfloat16*>(y);
   p.s_in = s_in;
   p.s_out = s_out;
-  p.err = err;
+  p.ctl = ctl;
   if (launch_wkv6_fwd(mr, mk, mv, mw, p, st) != cudaSuccess) return RWKV_ERR_CUDA;
   return RWKV_OK;
 }
@@ -557,12 +592,26 @@ rwkv_status rwkv_wkv6_step(int64_t B, int64_t H, int64_t N, const void* r, const
 rwkv_status rwkv_check_device_error(rwkv_stream_t stream) {
   if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return RWKV_ERR_CUDA;
   unsigned int v = 0;
-  if (cudaMemcpyFromSymbol(&v, g_device_error, sizeof(v)) != cudaSuccess) return RWKV_ERR_CUDA;
+  if (cudaMemcpyFromSymbol(&v, g_ctl, sizeof(v), offsetof(DevCtl, err)) != cudaSuccess) return RWKV_ERR_CUDA;
   if (v != 0) {
     const unsigned int zero = 0;
-    if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero)) != cudaSuccess) return RWKV_ERR_CUDA;
+    if (cudaMemcpyToSymbol(g_ctl, &zero, sizeof(zero), offsetof(DevCtl, err)) != cudaSuccess) return RWKV_ERR_CUDA;
     return RWKV_ERR_DEVICE_TIMEOUT;
   }
+  return RWKV_OK;
+}
+
+rwkv_status rwkv_debug_set_wait_limit_ns(uint64_t ns) {
+  const unsigned long long v = ns == 0 ? kDefaultWaitLimitNs : (unsigned long long)ns;
+  if (cudaDeviceSynchronize() != cudaSuccess) return RWKV_ERR_CUDA;
+  if (cudaMemcpyToSymbol(g_ctl, &v, sizeof(v), offsetof(DevCtl, wait_limit_ns)) != cudaSuccess) return RWKV_ERR_CUDA;
+  return RWKV_OK;
+}
+
+rwkv_status rwkv_debug_withhold_loads(int on) {
+  const unsigned int v = on ? 1u : 0u;
+  if (cudaDeviceSynchronize() != cudaSuccess) return RWKV_ERR_CUDA;
+  if (cudaMemcpyToSymbol(g_ctl, &v, sizeof(v), offsetof(DevCtl, withhold)) != cudaSuccess) return RWKV_ERR_CUDA;
   return RWKV_OK;
 }
 

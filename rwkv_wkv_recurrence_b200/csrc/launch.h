@@ -8,6 +8,8 @@
 
 namespace rwkv {
 
+struct DevCtl;  // the device control block (wkv_common.cuh)
+
 // Parameters of the WKV-4 forward kernel.  A CTA owns 32 channels of one
 // batch row over one time segment [seg*seg_len, min(T, (seg+1)*seg_len)).
 struct Fwd4Params {
@@ -25,7 +27,12 @@ struct Fwd4Params {
   long long end_seg_stride;
   float* ckpt;                    // [nck,3,B,C] states before tokens 0, L, 2L, ... or null
   int ckpt_len;                   // L (multiple of 16) when ckpt != null
-  unsigned int* err;              // device error word
+  int tma;                        // 1: k, v (, r) arrive by TMA and y leaves by TMA stores; 0: plain
+                                  // element loads and stores (any element-aligned base, any C)
+  const void* k;                  // [B,T,C] (read directly when tma == 0)
+  const void* v;
+  const void* r;                  // [B,T,C] receptance of the gated forward (tma == 0), else null
+  DevCtl* ctl;                    // device control block (error word, wait limit)
 };
 
 struct Bwd4Params {
@@ -38,9 +45,13 @@ struct Bwd4Params {
   void* gk;
   void* gv;
   double* part;       // [2,B,C] per-lane gw, gu partial sums
-  unsigned int* err;  // device error word
+  DevCtl* ctl;        // device control block
   const void* r;      // [B,T,C] receptance (gated backward only)
   void* gr;           // [B,T,C] its gradient (gated backward only)
+  int tma;            // 1: k, v, gy (go) by TMA, gk, gv by TMA stores; 0: plain element accesses
+  const void* k;      // [B,T,C] (read directly when tma == 0)
+  const void* v;
+  const void* g;      // gy, or go with the gate (tma == 0)
 };
 
 struct Wkv5StepParams {
@@ -66,7 +77,7 @@ struct Wkv5Params {
   __nv_bfloat16* y;
   const float* s_in;    // [B,H,64,64] or null
   float* s_out;         // [B,H,64,64] or null
-  unsigned int* err;
+  DevCtl* ctl;
 };
 
 struct Wkv6Params {
@@ -79,17 +90,18 @@ struct Wkv6Params {
   __nv_bfloat16* y;
   const float* s_in;    // [B,H,64,64] or null
   float* s_out;         // [B,H,64,64] or null
-  unsigned int* err;
+  DevCtl* ctl;
 };
 
 int fwd_tile_steps();
 int fwd_store_steps();
-int fwd_stages(bool bf16, int seg_len, bool gate = false);
+// Stage count of the forward's input pipeline (1 on the plain-access path, which has no pipeline).
+int fwd_stages(bool bf16, int seg_len, bool gate = false, bool tma = true);
 int bwd_tile_steps();
 int bwd_store_steps();
-int bwd_stages(bool bf16, int T, bool gate = false);
+int bwd_stages(bool bf16, int T, bool gate = false, bool tma = true);
 // mk, mv: [fwd_tile_steps() x 32] boxes over k, v; my: [fwd_store_steps() x 32] boxes over y
-// (TMA stores; any valid map when p.y is null).
+// (TMA stores; any valid map when p.y is null).  With p.tma == 0 the maps are not read (any value).
 cudaError_t launch_wkv4_fwd(bool bf16, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& my,
                             const Fwd4Params& p, cudaStream_t st);
 // The receptance-gated forward: also reads r ([fwd_tile_steps() x 32] boxes) and writes σ(r) ⊙ WKV.
@@ -123,8 +135,8 @@ cudaError_t launch_wkv6_fwd(const CUtensorMap& mr, const CUtensorMap& mk, const 
                             const CUtensorMap& mw, const Wkv6Params& p, cudaStream_t st);
 // Tensor map over an fp32 [B, T, W] tensor with [1, 64, 32] boxes and the 128-byte swizzle.
 bool make_f32_box32_map(CUtensorMap* m, const void* base, int B, int T, int W);
-// Device address of the library's error word on the current device (null on failure).
-unsigned int* device_error_word();
+// Device address of the library's control block on the current device (null on failure).
+DevCtl* device_ctl();
 
 // Sets the dynamic shared-memory limit of `func` once per device.
 cudaError_t ensure_smem_attr(const void* func, int bytes, unsigned* device_mask);

@@ -163,7 +163,7 @@ struct RCarry {  // reverse carry at a chunk boundary, per lane (see phase C)
 };
 
 // mg: gy boxes, or with GATE go boxes.
-template <typename T, bool GATE>
+template <typename T, bool GATE, bool TMA>
 __global__ void __launch_bounds__(kW * 32, 4) wkv4_bwd_kernel(const __grid_constant__ CUtensorMap mk,
                                                               const __grid_constant__ CUtensorMap mv,
                                                               const __grid_constant__ CUtensorMap mg,
@@ -188,17 +188,21 @@ __global__ void __launch_bounds__(kW * 32, 4) wkv4_bwd_kernel(const __grid_const
   const bool valid = c < p.C;
   const int ntile = (p.T + kTile - 1) / kTile;
 
-  if (threadIdx.x == 0) {
+  // thread 0 issues every load; with the test hook set it arms the barriers and issues none
+  if (!TMA && threadIdx.x == 0) *abort_flag = 0;
+  if (TMA && threadIdx.x == 0) {
+    const bool withheld = loads_withheld(p.ctl);
+    const int pre = min(p.stages, ntile);
     *abort_flag = 0;
     prefetch_tensormap(&mk);
     prefetch_tensormap(&mv);
     prefetch_tensormap(&mg);
     for (int s = 0; s < p.stages; ++s) mbar_init(&bars[s], 1);
     fence_mbar_init();
-    const int pre = min(p.stages, ntile);
     for (int s = 0; s < pre; ++s) {
       const int tc = (ntile - 1 - s) * kTile;
       mbar_arrive_expect_tx(&bars[s], kNB * kBoxBytes);
+      if (withheld) continue;
       tma_load_3d(tiles + (size_t)(kNB * s) * kBoxElems, &mk, &bars[s], ct * 32, tc, bb);
       tma_load_3d(tiles + (size_t)(kNB * s + 1) * kBoxElems, &mv, &bars[s], ct * 32, tc, bb);
       tma_load_3d(tiles + (size_t)(kNB * s + 2) * kBoxElems, &mg, &bars[s], ct * 32, tc, bb);
@@ -228,7 +232,8 @@ __global__ void __launch_bounds__(kW * 32, 4) wkv4_bwd_kernel(const __grid_const
     }
   }
 
-  for (int i = 0; i < ntile; ++i) {
+  int i = 0;
+  for (; i < ntile; ++i) {
     const int tile = ntile - 1 - i;
     const int s = i % p.stages;
     const uint32_t ph = (uint32_t)(i / p.stages) & 1u;
@@ -259,12 +264,21 @@ __global__ void __launch_bounds__(kW * 32, 4) wkv4_bwd_kernel(const __grid_const
         asm volatile("prefetch.global.L2 [%0];" ::"l"(ck2 + 2 * plane) : "memory");
       }
     }
-    if (!mbar_wait_bounded(&bars[s], ph, p.err)) *abort_flag = 1;
+    if constexpr (TMA) {
+      if (!mbar_wait_bounded(&bars[s], ph, p.ctl)) *abort_flag = 1;
+    }
     T* const kw = tiles + (size_t)(kNB * s) * kBoxElems + warp * kL * 32;  // this warp's [16][32] rows
     T* const vw = kw + kBoxElems;
     T* const ks = kw + lane;
     T* const vs = vw + lane;
     const T* gs = vs + kBoxElems;  // gy rows (go with GATE)
+    if constexpr (!TMA) {  // this warp's own rows, by plain loads (nothing else reads them)
+      warp_rows_in<T, kL>(kw, static_cast<const T*>(p.k), bb, p.T, p.C, ts, cnt, c, valid, lane, -kTile);
+      warp_rows_in<T, kL>(vw, static_cast<const T*>(p.v), bb, p.T, p.C, ts, cnt, c, valid, lane, -kTile);
+      warp_rows_in<T, kL>(vw + kBoxElems, static_cast<const T*>(p.g), bb, p.T, p.C, ts, cnt, c, valid, lane,
+                          -kTile);
+      __syncwarp();
+    }
     // GATE: this lane's r and gr of the chunk, token stride C
     const size_t tok0 = ((size_t)bb * p.T + (size_t)max(ts, 0)) * p.C + (size_t)c;
     const T* rg = (GATE && valid) ? static_cast<const T*>(p.r) + tok0 : nullptr;  // lanes past C: no access
@@ -294,7 +308,8 @@ __global__ void __launch_bounds__(kW * 32, 4) wkv4_bwd_kernel(const __grid_const
     if (lane == 0) bulk_wait_read();
     __syncthreads();
     if (*abort_flag) break;
-    if (threadIdx.x == 0 && i >= 1 && i - 1 + p.stages < ntile) {
+    // (never reached with the loads withheld: the first wait gives up)
+    if (TMA && threadIdx.x == 0 && i >= 1 && i - 1 + p.stages < ntile) {
       const int sp = (i - 1) % p.stages;
       const int tc = (ntile - 1 - (i - 1 + p.stages)) * kTile;
       fence_proxy_async();
@@ -349,17 +364,27 @@ __global__ void __launch_bounds__(kW * 32, 4) wkv4_bwd_kernel(const __grid_const
         chunk_walk<T, false>(ks, vs, cnt, E, G, Y, BP, U, lh, ll, (float)ae, (float)ge, gws, gus);
       gw_acc += (double)gws;
       gu_acc += (double)gus;
-      // gk, gv of the chunk: one [16 x 32] box each (rows past T and channels past C are clipped)
-      fence_proxy_async();
-      __syncwarp();
-      if (lane == 0) {
-        tma_store_3d(&mgk, kw, ct * 32, ts, bb);
-        tma_store_3d(&mgv, vw, ct * 32, ts, bb);
-
-        bulk_commit();
+      if constexpr (TMA) {
+        // gk, gv of the chunk: one [16 x 32] box each (rows past T and channels past C are clipped)
+        fence_proxy_async();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_3d(&mgk, kw, ct * 32, ts, bb);
+          tma_store_3d(&mgv, vw, ct * 32, ts, bb);
+          bulk_commit();
+        }
+      } else if (valid) {  // each lane stores its own channel's gradients
+        const size_t o = ((size_t)bb * p.T + ts) * p.C + c;
+        T* gkg = static_cast<T*>(p.gk) + o;
+        T* gvg = static_cast<T*>(p.gv) + o;
+        for (int j = 0; j < cnt; ++j) {
+          gkg[(size_t)j * p.C] = ks[j * 32];
+          gvg[(size_t)j * p.C] = vs[j * 32];
+        }
       }
     }
   }
+  if (TMA && threadIdx.x == 0 && *abort_flag) drain_loads(bars, p.stages, i, ntile, p.ctl);  // a wait gave up
   if (lane == 0) bulk_wait_all();
 
   // reduce the four warps' gw, gu partials of each lane
@@ -400,17 +425,24 @@ size_t bwd_smem_bytes(int stages) {
          (size_t)stages * 8 + 16;
 }
 
-template <typename T, bool GATE>
-cudaError_t launch_bwd_t(const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mg, const CUtensorMap& mgk,
-                         const CUtensorMap& mgv, const Bwd4Params& p, cudaStream_t st) {
+template <typename T, bool GATE, bool TMA>
+cudaError_t launch_bwd_tt(const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mg, const CUtensorMap& mgk,
+                          const CUtensorMap& mgv, const Bwd4Params& p, cudaStream_t st) {
   const size_t smem = bwd_smem_bytes<T>(p.stages);
   static unsigned device_mask = 0;
   cudaError_t e =
-      ensure_smem_attr(reinterpret_cast<const void*>(wkv4_bwd_kernel<T, GATE>), (int)smem, &device_mask);
+      ensure_smem_attr(reinterpret_cast<const void*>(wkv4_bwd_kernel<T, GATE, TMA>), (int)smem, &device_mask);
   if (e != cudaSuccess) return e;
   const long long nblk = (long long)p.ctiles * p.B;
-  wkv4_bwd_kernel<T, GATE><<<(unsigned)nblk, kW * 32, smem, st>>>(mk, mv, mg, mgk, mgv, p);
+  wkv4_bwd_kernel<T, GATE, TMA><<<(unsigned)nblk, kW * 32, smem, st>>>(mk, mv, mg, mgk, mgv, p);
   return cudaGetLastError();
+}
+
+template <typename T, bool GATE>
+cudaError_t launch_bwd_t(const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mg, const CUtensorMap& mgk,
+                         const CUtensorMap& mgv, const Bwd4Params& p, cudaStream_t st) {
+  return p.tma ? launch_bwd_tt<T, GATE, true>(mk, mv, mg, mgk, mgv, p, st)
+               : launch_bwd_tt<T, GATE, false>(mk, mv, mg, mgk, mgv, p, st);
 }
 
 }  // namespace
@@ -419,8 +451,9 @@ int bwd_tile_steps() { return kTile; }
 
 int bwd_store_steps() { return kL; }
 
-int bwd_stages(bool bf16, int T, bool gate) {
+int bwd_stages(bool bf16, int T, bool gate, bool tma) {
   (void)gate;  // the gated kernel streams the same three boxes (k, v, go)
+  if (!tma) return 1;  // the plain path reads each warp's rows into one buffer, no pipeline
   const int want = bf16 ? 4 : 2;  // 48 KB of boxes keeps four CTAs per SM
   const int ntile = (T + kTile - 1) / kTile;
   return max(2, min(want, ntile));

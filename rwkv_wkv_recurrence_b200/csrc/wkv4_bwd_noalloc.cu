@@ -123,11 +123,11 @@ extern "C" rwkv_status rwkv_wkv4_backward_noalloc(int64_t B, int64_t T, int64_t 
   const bool bf16 = dtype == RWKV_BF16;
   if (!aligned16(k) || !aligned16(v) || !aligned16(gy) || !aligned16(gk) || !aligned16(gv) ||
       (C * (bf16 ? 2 : 4)) % 16 != 0)
-    return RWKV_ERR_UNSUPPORTED;
+    return RWKV_ERR_UNSUPPORTED;  // this entry point keeps to the TMA path
   double* scratch = nullptr;
   if (scratch_for_current_device(&scratch) != cudaSuccess) return RWKV_ERR_CUDA;
-  unsigned int* err = device_error_word();
-  if (err == nullptr) return RWKV_ERR_CUDA;
+  DevCtl* ctl = device_ctl();
+  if (ctl == nullptr) return RWKV_ERR_CUDA;
   const int iB = (int)B, iT = (int)T, iC = (int)C;
   const int box_t = bwd_tile_steps();
   CUtensorMap mk, mv, mg, mgk, mgv;
@@ -142,13 +142,14 @@ extern "C" rwkv_status rwkv_wkv4_backward_noalloc(int64_t B, int64_t T, int64_t 
   p.C = iC;
   p.ctiles = (iC + 31) / 32;
   p.stages = bwd_stages(bf16, iT);
+  p.tma = 1;
   p.w = w;
   p.u = u;
   p.ckpt = ckpt;
   p.gk = gk;
   p.gv = gv;
   p.part = scratch;  // [2][B*C] within the fixed array
-  p.err = err;
+  p.ctl = ctl;
   if (launch_wkv4_bwd(bf16, mk, mv, mg, mgk, mgv, p, st) != cudaSuccess) return RWKV_ERR_CUDA;
   if (launch_wkv4_reduce_wu(iB, iC, scratch, gw, gu, st) != cudaSuccess) return RWKV_ERR_CUDA;
   return RWKV_OK;

@@ -103,7 +103,7 @@ struct CarrySlot {  // CTA running state at a tile boundary, per lane
   int p, pad;
 };
 
-template <typename T, bool GATE>
+template <typename T, bool GATE, bool TMA>
 __global__ void __launch_bounds__(kW * 32, 4) wkv4_fwd_kernel(const __grid_constant__ CUtensorMap mk,
                                                               const __grid_constant__ CUtensorMap mv,
                                                               const __grid_constant__ CUtensorMap my,
@@ -132,16 +132,20 @@ __global__ void __launch_bounds__(kW * 32, 4) wkv4_fwd_kernel(const __grid_const
   const int t1 = min(p.T, t0 + p.seg_len);
   const int ntile = (t1 - t0 + kTile - 1) / kTile;
 
-  if (threadIdx.x == 0) {
+  // thread 0 issues every load; with the test hook set it arms the barriers and issues none
+  if (!TMA && threadIdx.x == 0) *abort_flag = 0;
+  if (TMA && threadIdx.x == 0) {
+    const bool withheld = loads_withheld(p.ctl);
+    const int pre = min(p.stages, ntile);
     *abort_flag = 0;
     prefetch_tensormap(&mk);
     prefetch_tensormap(&mv);
     if constexpr (GATE) prefetch_tensormap(&mr);
     for (int s = 0; s < p.stages; ++s) mbar_init(&bars[s], 1);
     fence_mbar_init();
-    const int pre = min(p.stages, ntile);
     for (int s = 0; s < pre; ++s) {
       mbar_arrive_expect_tx(&bars[s], kNB * kBoxBytes);
+      if (withheld) continue;
       tma_load_3d(tiles + (size_t)(kNB * s) * kBoxElems, &mk, &bars[s], ct * 32, t0 + s * kTile, bb);
       tma_load_3d(tiles + (size_t)(kNB * s + 1) * kBoxElems, &mv, &bars[s], ct * 32, t0 + s * kTile, bb);
       if constexpr (GATE)
@@ -172,16 +176,28 @@ __global__ void __launch_bounds__(kW * 32, 4) wkv4_fwd_kernel(const __grid_const
   const bool rescan = (p.y != nullptr) || (p.ckpt != nullptr);
   State total{0.0, 0.0, 0};
 
-  for (int i = 0; i < ntile; ++i) {
+  int i = 0;
+  for (; i < ntile; ++i) {
     const int s = i % p.stages;
     const uint32_t ph = (uint32_t)(i / p.stages) & 1u;
-    if (!mbar_wait_bounded(&bars[s], ph, p.err)) *abort_flag = 1;
+    if constexpr (TMA) {
+      if (!mbar_wait_bounded(&bars[s], ph, p.ctl)) *abort_flag = 1;
+    }
     const int tb = t0 + i * kTile;
     const int ts = tb + warp * kL;
     const int cnt = max(0, min(kL, t1 - ts));
     const T* ks = tiles + (size_t)(kNB * s) * kBoxElems + warp * kL * 32 + lane;
     const T* vs = ks + kBoxElems;
     const T* rs = vs + kBoxElems;  // the r rows (GATE only)
+    if constexpr (!TMA) {  // this warp's own rows, by plain loads (nothing else reads them)
+      T* kw = const_cast<T*>(ks) - lane;
+      warp_rows_in<T, kL>(kw, static_cast<const T*>(p.k), bb, p.T, p.C, ts, cnt, c, valid, lane, kTile);
+      warp_rows_in<T, kL>(kw + kBoxElems, static_cast<const T*>(p.v), bb, p.T, p.C, ts, cnt, c, valid, lane, kTile);
+      if constexpr (GATE)
+        warp_rows_in<T, kL>(kw + 2 * kBoxElems, static_cast<const T*>(p.r), bb, p.T, p.C, ts, cnt, c, valid, lane,
+                        kTile);
+      __syncwarp();
+    }
 
     // 1. this warp's segment from a zero state
     float E[kL], kmax = -INFINITY, la = 0.f, lb = 0.f;
@@ -197,11 +213,12 @@ __global__ void __launch_bounds__(kW * 32, 4) wkv4_fwd_kernel(const __grid_const
     __syncthreads();
     if (*abort_flag) break;
     // every warp is done with tile i-1: refill its stage
-    if (threadIdx.x == 0 && i >= 1 && i - 1 + p.stages < ntile) {
+    if (TMA && threadIdx.x == 0 && i >= 1 && i - 1 + p.stages < ntile) {
       const int sp = (i - 1) % p.stages;
       const int tn = t0 + (i - 1 + p.stages) * kTile;
       fence_proxy_async();
       mbar_arrive_expect_tx(&bars[sp], kNB * kBoxBytes);
+      // (never reached with the loads withheld: the first wait gives up)
       tma_load_3d(tiles + (size_t)(kNB * sp) * kBoxElems, &mk, &bars[sp], ct * 32, tn, bb);
       tma_load_3d(tiles + (size_t)(kNB * sp + 1) * kBoxElems, &mv, &bars[sp], ct * 32, tn, bb);
       if constexpr (GATE) tma_load_3d(tiles + (size_t)(kNB * sp + 2) * kBoxElems, &mr, &bars[sp], ct * 32, tn, bb);
@@ -244,16 +261,22 @@ __global__ void __launch_bounds__(kW * 32, 4) wkv4_fwd_kernel(const __grid_const
           seg_output<T, true, GATE>(vs, rs, cnt, E, f, U, (float)sc.a, (float)sc.b, lh, ll, yw + lane);
         else
           seg_output<T, false, GATE>(vs, rs, cnt, E, f, U, (float)sc.a, (float)sc.b, lh, ll, yw + lane);
-        // y of the segment as one [16 x 32] box (rows past T and channels past C are clipped)
-        fence_proxy_async();
-        __syncwarp();
-        if (lane == 0) {
-          tma_store_3d(&my, yw, ct * 32, ts, bb);
-          bulk_commit();
+        if constexpr (TMA) {
+          // y of the segment as one [16 x 32] box (rows past T and channels past C are clipped)
+          fence_proxy_async();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_3d(&my, yw, ct * 32, ts, bb);
+            bulk_commit();
+          }
+        } else if (valid) {  // each lane stores its own channel's outputs
+          T* yg = static_cast<T*>(p.y) + ((size_t)bb * p.T + ts) * p.C + c;
+          for (int j = 0; j < cnt; ++j) yg[(size_t)j * p.C] = yw[j * 32 + lane];
         }
       }
     }
   }
+  if (TMA && threadIdx.x == 0 && *abort_flag) drain_loads(bars, p.stages, i, ntile, p.ctl);  // a wait gave up
   if (lane == 0) bulk_wait_all();
 
   if (p.end != nullptr && valid && warp == kW - 1) {
@@ -292,22 +315,29 @@ __global__ void wkv4_carry_kernel(int B, int C, int T, int nseg, int seg_len, co
 }
 
 template <typename T, bool GATE>
-size_t fwd_smem_bytes(int stages) {
+size_t fwd_smem_bytes(int stages) {  // also the plain path's (one stage)
   return (size_t)stages * (GATE ? 3 : 2) * kTile * 32 * sizeof(T) + 2 * kW * 32 * sizeof(Summ) +
          2 * 32 * sizeof(CarrySlot) + (size_t)stages * 8 + 16;
+}
+
+template <typename T, bool GATE, bool TMA>
+cudaError_t launch_fwd_tt(const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& my, const CUtensorMap& mr,
+                          const Fwd4Params& p, cudaStream_t st) {
+  const size_t smem = fwd_smem_bytes<T, GATE>(p.stages);
+  static unsigned device_mask = 0;
+  cudaError_t e =
+      ensure_smem_attr(reinterpret_cast<const void*>(wkv4_fwd_kernel<T, GATE, TMA>), (int)smem, &device_mask);
+  if (e != cudaSuccess) return e;
+  const long long nblk = (long long)p.ctiles * p.B * p.nseg;
+  wkv4_fwd_kernel<T, GATE, TMA><<<(unsigned)nblk, kW * 32, smem, st>>>(mk, mv, my, mr, p);
+  return cudaGetLastError();
 }
 
 template <typename T, bool GATE>
 cudaError_t launch_fwd_t(const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& my, const CUtensorMap& mr,
                          const Fwd4Params& p, cudaStream_t st) {
-  const size_t smem = fwd_smem_bytes<T, GATE>(p.stages);
-  static unsigned device_mask = 0;
-  cudaError_t e =
-      ensure_smem_attr(reinterpret_cast<const void*>(wkv4_fwd_kernel<T, GATE>), (int)smem, &device_mask);
-  if (e != cudaSuccess) return e;
-  const long long nblk = (long long)p.ctiles * p.B * p.nseg;
-  wkv4_fwd_kernel<T, GATE><<<(unsigned)nblk, kW * 32, smem, st>>>(mk, mv, my, mr, p);
-  return cudaGetLastError();
+  return p.tma ? launch_fwd_tt<T, GATE, true>(mk, mv, my, mr, p, st)
+               : launch_fwd_tt<T, GATE, false>(mk, mv, my, mr, p, st);
 }
 
 }  // namespace
@@ -316,7 +346,8 @@ int fwd_tile_steps() { return kTile; }
 
 int fwd_store_steps() { return kL; }
 
-int fwd_stages(bool bf16, int seg_len, bool gate) {
+int fwd_stages(bool bf16, int seg_len, bool gate, bool tma) {
+  if (!tma) return 1;  // the plain path reads each warp's rows into one buffer, no pipeline
   // three stages of fp32 k, v boxes (48 KB) keep four CTAs per SM; bf16 boxes are half as big; with the
   // gate's r box, two stages (fp32) or four (bf16) stay within the same 48 KB
   const int want = gate ? (bf16 ? 4 : 2) : (bf16 ? 6 : 3);

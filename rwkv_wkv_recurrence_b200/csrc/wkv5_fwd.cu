@@ -155,6 +155,8 @@ __global__ void __launch_bounds__(kThreads, 2) wkv5_fwd_tc_kernel(const __grid_c
   }
 
   if (warp == 0) tmem_alloc(&sm.tmem_base, kTmemCols);
+  // thread 0 issues every load; with the test hook set it arms the barrier and issues none
+  const bool withheld = tid == 0 && loads_withheld(p.ctl);
   if (tid == 0) {
     prefetch_tensormap(&mr);
     prefetch_tensormap(&mk);
@@ -165,9 +167,11 @@ __global__ void __launch_bounds__(kThreads, 2) wkv5_fwd_tc_kernel(const __grid_c
     mbar_init(&sm.bar_ds, 1);
     fence_mbar_init();
     mbar_arrive_expect_tx(&sm.bar_tma, 3 * kRawBytes);
-    tma_load_3d(sm.raw[0], &mr, &sm.bar_tma, h * kN, 0, b);
-    tma_load_3d(sm.raw[1], &mk, &sm.bar_tma, h * kN, 0, b);
-    tma_load_3d(sm.raw[2], &mv, &sm.bar_tma, h * kN, 0, b);
+    if (!withheld) {
+      tma_load_3d(sm.raw[0], &mr, &sm.bar_tma, h * kN, 0, b);
+      tma_load_3d(sm.raw[1], &mk, &sm.bar_tma, h * kN, 0, b);
+      tma_load_3d(sm.raw[2], &mv, &sm.bar_tma, h * kN, 0, b);
+    }
   }
 
   // ---- r̃, k̃: warp w owns channels 8w..8w+7; lane holds token row 8 ib + rr, channels dR, dR + 1.
@@ -232,11 +236,13 @@ __global__ void __launch_bounds__(kThreads, 2) wkv5_fwd_tc_kernel(const __grid_c
   const uint32_t rawR = smem_u32(sm.raw[0]), rawK = smem_u32(sm.raw[1]), rawV = smem_u32(sm.raw[2]);
   const bool issuer = tid == 0;
 
-  for (int c = 0; c < nchunk; ++c) {
+  int c = 0;
+  bool aborted = false;
+  for (; c < nchunk; ++c) {
     const int t0 = c * kL;
     const int cnt = min(kL, p.T - t0);
     const uint32_t ph = (uint32_t)c & 1u;
-    if (!mbar_wait_bounded(&sm.bar_tma, ph, p.err)) sm.abort_flag = 1;
+    if (!mbar_wait_bounded(&sm.bar_tma, ph, p.ctl)) sm.abort_flag = 1;
 
     // T1a: r̃, k̃ and the bonus parts (rows past the sequence end hold zeros from the TMA fill)
     {
@@ -262,7 +268,10 @@ __global__ void __launch_bounds__(kThreads, 2) wkv5_fwd_tc_kernel(const __grid_c
     fence_proxy_async();
     tc_fence_before();
     __syncthreads();
-    if (sm.abort_flag) break;
+    if (sm.abort_flag) {
+      aborted = true;
+      break;
+    }
     // [scores | Y] = r̃ [k̃ ; e^{32λ} Sᵀ]ᵀ: causal scores [τ][ι] and the state read [τ][j].  The
     // issuing thread hands the eight K steps out in pairs between its warp's T1b steps, so that
     // the warp never waits on a full MMA queue.
@@ -333,7 +342,7 @@ __global__ void __launch_bounds__(kThreads, 2) wkv5_fwd_tc_kernel(const __grid_c
 
     // T2a: causal mask of the scores (ι < τ kept, ι = τ the bonus Σ_d r u k, ι > τ zero) -> opA.
     // .16x128b fragment: rows τ = 16 q4 + t4 + 8 r, columns ι = 32 hc + 4 q + tq  ->  register 2 q + r
-    if (!mbar_wait_bounded(&sm.bar_sc, ph, p.err)) sm.abort_flag = 1;
+    if (!mbar_wait_bounded(&sm.bar_sc, ph, p.ctl)) sm.abort_flag = 1;
     tc_fence_after();
     {
       const int tau0 = 16 * q4 + t4;
@@ -376,7 +385,7 @@ __global__ void __launch_bounds__(kThreads, 2) wkv5_fwd_tc_kernel(const __grid_c
     }
 
     // T3: Y rows -> bf16 -> global (TMEM lanes 0..15 of each quarter hold the rows)
-    if (!mbar_wait_bounded(&sm.bar_av, ph, p.err)) sm.abort_flag = 1;
+    if (!mbar_wait_bounded(&sm.bar_av, ph, p.ctl)) sm.abort_flag = 1;
     tc_fence_after();
     {
       float yv[32];
@@ -396,7 +405,7 @@ __global__ void __launch_bounds__(kThreads, 2) wkv5_fwd_tc_kernel(const __grid_c
     }
 
     // T2b: S <- e^{cnt λ} S + e^{(cnt-32) λ} ΔS; e^{32λ} Sᵀ into opS for the next chunk
-    if (!mbar_wait_bounded(&sm.bar_ds, ph, p.err)) sm.abort_flag = 1;
+    if (!mbar_wait_bounded(&sm.bar_ds, ph, p.ctl)) sm.abort_flag = 1;
     tc_fence_after();
     {
       float ds[16];
@@ -423,6 +432,13 @@ __global__ void __launch_bounds__(kThreads, 2) wkv5_fwd_tc_kernel(const __grid_c
     }
   }
 
+  if (aborted && tid == 0) {
+    // a wait gave up at chunk c: the previous chunk's MMA chains (committed last on bar_ds) and
+    // this chunk's loads must finish before the tensor memory and shared memory are released,
+    // each wait bounded again
+    if (c >= 1) mbar_wait_bounded(&sm.bar_ds, (uint32_t)(c - 1) & 1u, p.ctl);
+    if (!withheld) mbar_wait_bounded(&sm.bar_tma, (uint32_t)c & 1u, p.ctl);
+  }
   if (p.s_out != nullptr) {
 #pragma unroll
     for (int q = 0; q < 8; ++q)

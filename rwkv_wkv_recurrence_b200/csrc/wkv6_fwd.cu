@@ -190,6 +190,8 @@ __global__ void __launch_bounds__(kThreads, 2) wkv6_fwd_tc_kernel(const __grid_c
 
   if (tid == 0) sm.abort_flag = 0;
   if (warp == 0) tmem_alloc(&sm.tmem_base, kTmemCols);
+  // thread 0 issues every load; with the test hook set it arms the barrier and issues none
+  const bool withheld = tid == 0 && loads_withheld(p.ctl);
   if (tid == 0) {
     prefetch_tensormap(&mr);
     prefetch_tensormap(&mk);
@@ -201,11 +203,13 @@ __global__ void __launch_bounds__(kThreads, 2) wkv6_fwd_tc_kernel(const __grid_c
     mbar_init(&sm.bar_ds, 1);
     fence_mbar_init();
     mbar_arrive_expect_tx(&sm.bar_tma, 3 * kRawBytes + 2 * kOmBytes);
-    tma_load_3d(sm.raw[0], &mr, &sm.bar_tma, h * kN, 0, b);
-    tma_load_3d(sm.raw[1], &mk, &sm.bar_tma, h * kN, 0, b);
-    tma_load_3d(sm.raw[2], &mv, &sm.bar_tma, h * kN, 0, b);
-    tma_load_3d(sm.om[0], &mw, &sm.bar_tma, h * kN, 0, b);
-    tma_load_3d(sm.om[1], &mw, &sm.bar_tma, h * kN + 32, 0, b);
+    if (!withheld) {
+      tma_load_3d(sm.raw[0], &mr, &sm.bar_tma, h * kN, 0, b);
+      tma_load_3d(sm.raw[1], &mk, &sm.bar_tma, h * kN, 0, b);
+      tma_load_3d(sm.raw[2], &mv, &sm.bar_tma, h * kN, 0, b);
+      tma_load_3d(sm.om[0], &mw, &sm.bar_tma, h * kN, 0, b);
+      tma_load_3d(sm.om[1], &mw, &sm.bar_tma, h * kN + 32, 0, b);
+    }
   }
 
   // ---- decay prologue and r̃, k̃: warp w owns channels 8w..8w+7; lane holds token rows 8 ib + rr
@@ -246,11 +250,13 @@ __global__ void __launch_bounds__(kThreads, 2) wkv6_fwd_tc_kernel(const __grid_c
   uint32_t nfast = 0;  // chunks done on the tensor cores (phase of the MMA barriers)
   float Rnext[2] = {0.f, 0.f};  // reference of the next chunk: half the log-decay of this one
 
-  for (int c = 0; c < nchunk; ++c) {
+  int c = 0;
+  bool aborted = false;
+  for (; c < nchunk; ++c) {
     const int t0 = c * kL;
     const int cnt = min(kL, p.T - t0);
     const int par = c & 1;
-    if (!mbar_wait_bounded(&sm.bar_tma, (uint32_t)c & 1u, p.err)) sm.abort_flag = 1;
+    if (!mbar_wait_bounded(&sm.bar_tma, (uint32_t)c & 1u, p.ctl)) sm.abort_flag = 1;
 
     // T1a: λ, the cumulative log-decay, the reference R and the chunk decay; then r̃, k̃ and the
     // bonus parts.  Rows past the sequence end (zeros from the TMA fill) get λ = 0.
@@ -335,7 +341,10 @@ __global__ void __launch_bounds__(kThreads, 2) wkv6_fwd_tc_kernel(const __grid_c
     fence_proxy_async();
     tc_fence_before();
     const int slow = __syncthreads_or(bad);
-    if (sm.abort_flag) break;
+    if (sm.abort_flag) {
+      aborted = true;
+      break;
+    }
 
     if (slow) {  // some channel decays too fast for the factorization: per-token recurrence
       S = chunk_recurrent(S, sm, p, b, h, t0, cnt);
@@ -436,7 +445,7 @@ __global__ void __launch_bounds__(kThreads, 2) wkv6_fwd_tc_kernel(const __grid_c
     }
 
     // T2a: causal mask of the scores (ι < τ kept, ι = τ the bonus, ι > τ zero) -> opRA
-    if (!mbar_wait_bounded(&sm.bar_sc, phm, p.err)) sm.abort_flag = 1;
+    if (!mbar_wait_bounded(&sm.bar_sc, phm, p.ctl)) sm.abort_flag = 1;
     tc_fence_after();
     {
       const int tau0 = 16 * q4 + t4;
@@ -477,7 +486,7 @@ __global__ void __launch_bounds__(kThreads, 2) wkv6_fwd_tc_kernel(const __grid_c
     }
 
     // T3: output rows -> bf16 -> global
-    if (!mbar_wait_bounded(&sm.bar_av, phm, p.err)) sm.abort_flag = 1;
+    if (!mbar_wait_bounded(&sm.bar_av, phm, p.ctl)) sm.abort_flag = 1;
     tc_fence_after();
     {
       float yv[32];
@@ -497,7 +506,7 @@ __global__ void __launch_bounds__(kThreads, 2) wkv6_fwd_tc_kernel(const __grid_c
     }
 
     // T2b: S <- e^{Λ_last} S + e^{Λ_last - R} ΔS
-    if (!mbar_wait_bounded(&sm.bar_ds, phm, p.err)) sm.abort_flag = 1;
+    if (!mbar_wait_bounded(&sm.bar_ds, phm, p.ctl)) sm.abort_flag = 1;
     tc_fence_after();
     {
       float ds[16];
@@ -516,6 +525,13 @@ __global__ void __launch_bounds__(kThreads, 2) wkv6_fwd_tc_kernel(const __grid_c
     ++nfast;
   }
 
+  if (aborted && tid == 0) {
+    // a wait gave up at chunk c: the last committed MMA chains (bar_ds, one phase per chunk on
+    // the tensor cores) and this chunk's loads must finish before the tensor memory and shared
+    // memory are released, each wait bounded again
+    if (nfast >= 1) mbar_wait_bounded(&sm.bar_ds, (nfast - 1) & 1u, p.ctl);
+    if (!withheld) mbar_wait_bounded(&sm.bar_tma, (uint32_t)c & 1u, p.ctl);
+  }
   if (p.s_out != nullptr) {
 #pragma unroll
     for (int q = 0; q < 8; ++q)

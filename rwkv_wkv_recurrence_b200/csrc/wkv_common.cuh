@@ -20,10 +20,26 @@
 namespace rwkv {
 
 
-// Bit set in the library's device error word (whose address every kernel
-// with a wait receives) when a bounded wait gives up.  Read and cleared by
-// rwkv_check_device_error().
+// Bit set in the library's device error word when a bounded wait gives up.
+// Read and cleared by rwkv_check_device_error().
 constexpr unsigned int kErrTmaTimeout = 1u;
+
+// Default limit of a bounded wait.  A TMA load or an MMA chain completes in
+// microseconds; a wait that lasts this long means its arrival will not come.
+constexpr unsigned long long kDefaultWaitLimitNs = 1000000000ull;  // 1 s
+
+// The library's device control block (one per device), whose address every
+// kernel with a wait receives:
+//   err            error bits (kErrTmaTimeout), set by a wait that gives up;
+//   withhold       test hook: when nonzero the TMA-issuing thread arms its
+//                  barriers but issues no load, so the first wait runs out with
+//                  nothing in flight (set by rwkv_debug_withhold_loads);
+//   wait_limit_ns  how long a bounded wait polls before giving up.
+struct DevCtl {
+  unsigned int err;
+  unsigned int withhold;
+  unsigned long long wait_limit_ns;
+};
 
 // ---------------------------------------------------------------- PTX helpers
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -59,16 +75,44 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t phase) {
   return ok != 0;
 }
 
-// Wait for phase `phase` of an mbarrier, giving up after a bounded number of
-// polls (each poll may suspend the thread for a hardware-chosen interval).
-// Returns false, and records kErrTmaTimeout, if the phase never completed.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t phase, unsigned int* err) {
-  constexpr uint32_t kMaxPolls = 1u << 24;
-  for (uint32_t i = 0; i < kMaxPolls; ++i) {
-    if (mbar_try_wait(bar, phase)) return true;
+// Nanoseconds of the GPU's global timer.
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Wait for phase `phase` of an mbarrier, giving up once ctl->wait_limit_ns
+// have passed (each poll may suspend the thread for a hardware-chosen
+// interval).  Returns false, and records kErrTmaTimeout, if the phase never
+// completed.  The first poll needs no clock read.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t phase, DevCtl* ctl) {
+  if (mbar_try_wait(bar, phase)) return true;
+  const unsigned long long t0 = global_ns();
+  const unsigned long long limit = *reinterpret_cast<volatile unsigned long long*>(&ctl->wait_limit_ns);
+  while (!mbar_try_wait(bar, phase)) {
+    if (global_ns() - t0 > limit) {
+      atomicOr(&ctl->err, kErrTmaTimeout);
+      return false;
+    }
   }
-  atomicOr(err, kErrTmaTimeout);
-  return false;
+  return true;
+}
+
+// True when the test hook asks the issuing thread to withhold its loads.
+__device__ __forceinline__ bool loads_withheld(const DevCtl* ctl) {
+  return *reinterpret_cast<const volatile unsigned int*>(&ctl->withhold) != 0u;
+}
+
+// Abort path of a `stages`-deep load pipeline whose wait for iteration i gave up: the loads
+// issued for iterations i .. (refills run stages - 1 iterations ahead, never past ntile) may
+// still be in flight, so the issuing thread waits for each, bounded again, before its CTA
+// leaves.  Nothing was issued when the loads were withheld.  Not inlined: it runs only on the
+// abort path and keeps its registers out of the kernel's main loop.
+static __device__ __noinline__ void drain_loads(uint64_t* bars, int stages, int i, int ntile, DevCtl* ctl) {
+  if (loads_withheld(ctl)) return;
+  const int issued = min(ntile, max(stages, i - 1 + stages));
+  for (int j = i; j < issued; ++j) mbar_wait_bounded(&bars[j % stages], (uint32_t)(j / stages) & 1u, ctl);
 }
 
 // 3-D tiled TMA load (no multicast) into shared memory, completing on `bar`.
@@ -139,6 +183,23 @@ struct IO<__nv_bfloat16> {
   __device__ __forceinline__ static float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
   __device__ __forceinline__ static __nv_bfloat16 from_f(float x) { return __float2bfloat16_rn(x); }
 };
+
+// Plain-access path of the WKV-4 kernels (any element-aligned base, any C):
+// warp-local copy of rows [ts, ts + cnt) of one [B,T,C] tensor into ROWS
+// shared-memory rows of 32 channels (lane = channel; rows past cnt and lanes
+// past C get zeros, as the TMA fill would), plus an L2 prefetch of the rows
+// `ahead` steps later for the warp's next visit.
+template <typename T, int ROWS>
+__device__ __forceinline__ void warp_rows_in(T* rows, const T* __restrict__ g, int bb, int T_, int C, int ts,
+                                             int cnt, int c, bool valid, int lane, int ahead) {
+  const size_t base = ((size_t)bb * T_ + (size_t)max(ts, 0)) * C + (size_t)c;
+#pragma unroll
+  for (int j = 0; j < ROWS; ++j)
+    rows[j * 32 + lane] = (valid && j < cnt) ? g[base + (size_t)j * C] : IO<T>::from_f(0.f);
+  const int tn = ts + ahead + lane;
+  if (lane < ROWS && tn >= 0 && tn < T_ && valid)
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(g + ((size_t)bb * T_ + tn) * C + c) : "memory");
+}
 
 // ---------------------------------------------------------------- WKV-4 state
 // log2(e) split into an fp32 head and tail: x = k*kL2eHi + k*kL2eLo carries

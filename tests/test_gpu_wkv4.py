@@ -285,8 +285,16 @@ def test_workspace_and_alignment_errors(cuda_device):
     ws = torch.empty(need, dtype=torch.uint8, device=cuda_device)
     assert h.rwkv_wkv4_forward(*args, rw._ptr(ws), need - 4, rw._stream(None)) == 3
     assert h.rwkv_wkv4_forward(*args, rw._ptr(ws), need, rw._stream(None)) == 0
-    kk = torch.empty(8 * 1024 * 768 + 1, device=cuda_device)[1:]
+    # k off 16-byte alignment: the plain-access instance serves it, with the TMA path's arithmetic
+    kk = torch.empty(8 * 1024 * 768 + 1, device=cuda_device)[1:].view(8, 1024, 768)
+    kk.copy_(p["k"])
+    y_plain = torch.empty_like(y)
     assert h.rwkv_wkv4_forward(8, 1024, 768, rw.F32, rw._ptr(p["w"]), rw._ptr(p["u"]), rw._ptr(kk),
-                               rw._ptr(p["v"]), rw._ptr(y), None, None, None, 16, 1, None, 0,
-                               rw._stream(None)) == 2
+                               rw._ptr(p["v"]), rw._ptr(y_plain), None, None, None, 16, 1, None, 0,
+                               rw._stream(None)) == 0
+    y_tma = torch.empty_like(y)
+    assert h.rwkv_wkv4_forward(8, 1024, 768, rw.F32, rw._ptr(p["w"]), rw._ptr(p["u"]), rw._ptr(p["k"]),
+                               rw._ptr(p["v"]), rw._ptr(y_tma), None, None, None, 16, 1, None, 0,
+                               rw._stream(None)) == 0
     rw.rwkv_check_device_error()
+    assert torch.equal(y_plain, y_tma)
