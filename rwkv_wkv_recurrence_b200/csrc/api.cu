@@ -1,5 +1,6 @@
 // C-ABI layer: argument validation, workspace planning, TMA descriptors and
 // kernel dispatch for the calls declared in include/rwkv_wkv.h.
+#include <algorithm>
 #include <climits>
 #include <cstddef>
 #include <cstring>
@@ -86,6 +87,7 @@ DevCtl* device_ctl() {
 namespace {
 
 constexpr int kDesignSMs = 148;  // B200 SM count the schedules are planned for
+constexpr int kCtasPerSM = 4;    // resident WKV-4 forward CTAs per SM (registers and 48 KB of boxes)
 constexpr int kCkLen = 16;       // checkpoint interval the backward reads
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -125,7 +127,9 @@ FwdPlan plan_forward(int64_t B, int64_t T, int64_t C, int algo) {
   int a = algo;
   if (a == RWKV_ALGO_AUTO) a = (lane_tiles >= 3 * kDesignSMs || T <= 128) ? RWKV_ALGO_SEQUENTIAL : RWKV_ALGO_CHUNKED;
   if (a == RWKV_ALGO_CHUNKED && T > 0 && lane_tiles > 0) {
-    const int64_t want = (8 * kDesignSMs + lane_tiles - 1) / lane_tiles;
+    // as many time segments as keep every CTA of a pass resident at once (four per SM): a
+    // second wave would cost a whole segment's latency again
+    const int64_t want = std::max<int64_t>(1, (int64_t)(kCtasPerSM * kDesignSMs) / lane_tiles);
     int64_t seg = (T + want - 1) / want;
     seg = ((seg + tt - 1) / tt) * tt;
     if (seg < 64) seg = 64;

@@ -12,7 +12,7 @@ import oracle
 import rwkv_wkv_recurrence_b200 as rw
 import wkv_inputs as wi
 from _parity import (TOL_BF16, TOL_GRAD, TOL_Y, assert_close_abs1, assert_close_rms, assert_grads_close,
-                     assert_state_close)
+                     assert_state_close, wkv4_input_sensitivity)
 
 pytestmark = pytest.mark.gpu
 SEED = wi.CONFIG_SEED_BASE
@@ -184,7 +184,11 @@ def test_training_workload_full_size(cuda_device):
     assert_close_abs1(y, ref_y, TOL_Y, "y")
     del ref_y, y
     r = oracle.wkv4_backward(p["w"], p["u"], p["k"], p["v"], p["gy"])
-    assert_grads_close((gk, gv, gw, gu), r)
+    # gw and gu entries are sums over 32,768 terms; where one is small beside its terms, half-ulp
+    # perturbations of the fp32 inputs move the exact result by more than 1e-4 (the oracle shows it)
+    floor = wkv4_input_sensitivity(oracle, p["w"], p["u"], p["k"], p["v"], p["gy"])
+    rep = assert_grads_close((gk, gv, gw, gu), r, floor=floor)
+    assert rep["gw_on_floor"] <= C // 8 and rep["gu_on_floor"] <= C // 8, rep
     # properties that hold for every lane: sum_t gk = 0 and sum_t gv = sum_t gy
     # (fp32 sums of 4096 terms: compared against the sum of magnitudes)
     sk = gk.double().sum(1)

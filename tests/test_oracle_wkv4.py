@@ -173,3 +173,31 @@ def test_backward_recurrent_equals_time_parallel(outliers):
     b = oracle.wkv4_backward_bruteforce(p["w"], p["u"], p["k"], p["v"], p["gy"])
     for x, y in zip(a, b):
         np.testing.assert_allclose(x, y, rtol=1e-10, atol=1e-10)
+
+
+def test_gw_entry_is_conditioned_beyond_the_elementwise_bound():
+    # Channel 1593 of the 8 x 4096 x 2048 training workload: gw is a sum of 32,768 terms whose
+    # magnitudes add up to ~1e4 while the sum is ~-0.1.  Perturbing the fp32 inputs by up to half
+    # an ulp moves the exact (fp64) result by more than 1e-4 * max(1, |gw|): no computation that
+    # rounds its intermediates to fp32 can hold that entry to the plain elementwise bound, which
+    # is why the full-size GPU test gives each gw, gu entry a floor of twice this movement.
+    import torch
+
+    B, T, C, c = 8, 4096, 2048, 1593
+    seed = wi.CONFIG_SEED_BASE + 2
+    w, u = wi.wkv4_params(seed, C)
+    b_sel, c_sel = torch.arange(B), torch.full((B,), c)
+
+    def field(kind, out=False):
+        x = wi.btc_field(kind, seed, B, T, C, b_sel=b_sel, c_sel=c_sel, outliers=out)
+        return x.T.reshape(B, T, 1).double().numpy()
+
+    k, v, gy = field("k", True), field("v"), field("gy")
+    W, U = w[c:c + 1].double().numpy(), u[c:c + 1].double().numpy()
+    gw0 = oracle.wkv4_backward(W, U, k, v, gy)[2][0]
+    rng = np.random.default_rng(0)
+    pert = lambda x: x * (1.0 + rng.uniform(-2.0 ** -24, 2.0 ** -24, x.shape))
+    moved = max(abs(oracle.wkv4_backward(pert(W), pert(U), pert(k), pert(v), pert(gy))[2][0] - gw0)
+                for _ in range(2))
+    assert abs(gw0) < 1.0
+    assert moved > 1e-4 * max(1.0, abs(gw0)), moved
