@@ -207,6 +207,38 @@ RWKV_API rwkv_status rwkv_wkv5_forward(int64_t B, int64_t T, int64_t H, int64_t 
                               const float *s_in, float *s_out,
                               void *workspace, size_t workspace_bytes, rwkv_stream_t stream);
 
+/* Workspace bytes rwkv_wkv5_backward needs (0 for an empty problem or N != 64). */
+RWKV_API size_t rwkv_wkv5_backward_workspace_bytes(int64_t B, int64_t T, int64_t H, int64_t N);
+
+/*
+ * Eagle / RWKV-5 backward: gradients of L = Σ gy·y + Σ gs_out ∘ s_out for the
+ * forward above ("RWKV-5 Eagle과 RWKV-6 Finch", section Eagle; the pages print
+ * no backward, this is the chain rule through its recurrence).  With
+ * G_T = gs_out and G_t = diag(w) G_{t+1} + r_tᵀ gy_t (the gradient of the
+ * state after token t-1):
+ *   gr_t = s_t gy_tᵀ + u ⊙ k_t (v_t·gy_t),   gk_t = G_{t+1} v_tᵀ + u ⊙ r_t (v_t·gy_t),
+ *   gv_t = G_{t+1}ᵀ k_t + (Σ r_t u k_t) gy_t,  gs_in = G_0,
+ *   gomega_d = Σ_{b,t} (Σ_j G_{t+1}[d][j] s_t[d][j]) · dw_d/dω_d,  gu_d = Σ_{b,t} r_t[d] k_t[d] (v_t·gy_t).
+ *   r, k, v, gy   [B,T,H,N] bf16, read.      gr, gk, gv [B,T,H,N] bf16, written.
+ *   omega, u      [H,N] fp32, read.          gomega, gu [H,N] fp32, OVERWRITTEN with the sums over
+ *                                            batch and time.
+ *   s_in          [B,H,N,N] fp32, the forward's initial state, or NULL (zero).
+ *   gs_out        [B,H,N,N] fp32, the gradient of the final state, or NULL (zero).
+ *   gs_in         [B,H,N,N] fp32, written with the gradient of s_in, or NULL (not wanted).
+ *   workspace     device scratch of rwkv_wkv5_backward_workspace_bytes() bytes (time-reversed
+ *                 copies of the inputs, the forward states at every 64th token, per-row sums).
+ *   N must be 64; the [B,T,H,N] tensors 16-byte aligned (RWKV_ERR_UNSUPPORTED otherwise).
+ *   A channel decaying faster than exp(omega) = 2.5 (w < 0.082) is outside the
+ *   range this backward computes: the call returns RWKV_OK, the outputs of
+ *   that channel's heads are undefined, and rwkv_check_device_error reports
+ *   RWKV_ERR_UNSUPPORTED.  Deterministic.
+ */
+RWKV_API rwkv_status rwkv_wkv5_backward(int64_t B, int64_t T, int64_t H, int64_t N, const void *r, const void *k,
+                               const void *v, const float *omega, const float *u, const float *s_in,
+                               const void *gy, const float *gs_out, void *gr, void *gk, void *gv,
+                               float *gomega, float *gu, float *gs_in, void *workspace, size_t workspace_bytes,
+                               rwkv_stream_t stream);
+
 /*
  * Eagle / RWKV-5 recurrent decode: one token for each of B independent
  * streams ("RWKV-5 Eagle과 RWKV-6 Finch", section Eagle): per head,
@@ -295,7 +327,8 @@ RWKV_API rwkv_status rwkv_wkv4_backward_noalloc(int64_t B, int64_t T, int64_t C,
 
 /*
  * Synchronises `stream`, then reports and clears the device error word that
- * kernels set when a bounded wait gives up (RWKV_ERR_DEVICE_TIMEOUT), or
+ * kernels set when a bounded wait gives up (RWKV_ERR_DEVICE_TIMEOUT) or when
+ * a backward met a decay outside its range (RWKV_ERR_UNSUPPORTED), or
  * RWKV_ERR_CUDA if the stream itself failed.
  * The error word is one per device and process, shared by every call on that
  * device whatever its stream or host thread: a timeout in work on one stream

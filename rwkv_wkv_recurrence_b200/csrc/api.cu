@@ -593,6 +593,172 @@ rwkv_status rwkv_wkv6_step(int64_t B, int64_t H, int64_t N, const void* r, const
   return RWKV_OK;
 }
 
+}  // extern "C"
+
+namespace rwkv {
+namespace {
+
+// Byte layout of the Eagle backward's workspace (every region 256-byte aligned).
+struct Wkv5BwdWs {
+  size_t rev[4];  // time-reversed k, r, gy, v (bf16 [B,T,H,64])
+  size_t gv_rev, gk_rev;
+  size_t ckpt;    // fp32 [B,H,nchunk,64,64]
+  size_t part_f, part_r;  // fp64 [B,H,64]
+  size_t total;
+};
+
+Wkv5BwdWs wkv5_bwd_ws(int64_t B, int64_t T, int64_t H) {
+  auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  Wkv5BwdWs w{};
+  const size_t seq = up((size_t)B * T * H * 64 * 2);
+  size_t o = 0;
+  for (int i = 0; i < 4; ++i) {
+    w.rev[i] = o;
+    o += seq;
+  }
+  w.gv_rev = o;
+  o += seq;
+  w.gk_rev = o;
+  o += seq;
+  w.ckpt = o;
+  o += up((size_t)B * H * ((T + 63) / 64) * 64 * 64 * 4);
+  w.part_f = o;
+  o += up((size_t)B * H * 64 * 8);
+  w.part_r = o;
+  o += up((size_t)B * H * 64 * 8);
+  w.total = o;
+  return w;
+}
+
+}  // namespace
+}  // namespace rwkv
+
+extern "C" {
+
+size_t rwkv_wkv5_backward_workspace_bytes(int64_t B, int64_t T, int64_t H, int64_t N) {
+  if (B <= 0 || T <= 0 || H <= 0 || N != 64) return 0;
+  return wkv5_bwd_ws(B, T, H).total;
+}
+
+rwkv_status rwkv_wkv5_backward(int64_t B, int64_t T, int64_t H, int64_t N, const void* r, const void* k,
+                               const void* v, const float* omega, const float* u, const float* s_in, const void* gy,
+                               const float* gs_out, void* gr, void* gk, void* gv, float* gomega, float* gu,
+                               float* gs_in, void* workspace, size_t workspace_bytes, rwkv_stream_t stream) {
+  if (!fits_int(B) || !fits_int(T) || !fits_int(H) || !fits_int(N)) return RWKV_ERR_INVALID_ARG;
+  if (N != 64) return RWKV_ERR_UNSUPPORTED;
+  if (B == 0 || H == 0) return RWKV_OK;
+  if (omega == nullptr || u == nullptr || gomega == nullptr || gu == nullptr) return RWKV_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (T == 0) {  // no tokens: the sums are empty and the state gradient passes through
+    if (cudaMemsetAsync(gomega, 0, H * 64 * sizeof(float), st) != cudaSuccess) return RWKV_ERR_CUDA;
+    if (cudaMemsetAsync(gu, 0, H * 64 * sizeof(float), st) != cudaSuccess) return RWKV_ERR_CUDA;
+    if (gs_in != nullptr) {
+      const size_t n = (size_t)B * H * 64 * 64 * sizeof(float);
+      cudaError_t e = gs_out ? cudaMemcpyAsync(gs_in, gs_out, n, cudaMemcpyDeviceToDevice, st)
+                             : cudaMemsetAsync(gs_in, 0, n, st);
+      if (e != cudaSuccess) return RWKV_ERR_CUDA;
+    }
+    return RWKV_OK;
+  }
+  if (r == nullptr || k == nullptr || v == nullptr || gy == nullptr || gr == nullptr || gk == nullptr ||
+      gv == nullptr)
+    return RWKV_ERR_INVALID_ARG;
+  if (!aligned16(r) || !aligned16(k) || !aligned16(v) || !aligned16(gy) || !aligned16(gr) || !aligned16(gk) ||
+      !aligned16(gv))
+    return RWKV_ERR_UNSUPPORTED;
+  if ((int64_t)H * 64 > INT_MAX || (int64_t)B * H > INT_MAX || (int64_t)T + 64 > INT_MAX) return RWKV_ERR_UNSUPPORTED;
+  const Wkv5BwdWs L = wkv5_bwd_ws(B, T, H);
+  if (workspace == nullptr || workspace_bytes < L.total) return RWKV_ERR_WORKSPACE;
+  DevCtl* ctl = device_ctl();
+  if (ctl == nullptr) return RWKV_ERR_CUDA;
+  const int iB = (int)B, iT = (int)T, iH = (int)H, W = iH * 64;
+  char* ws = static_cast<char*>(workspace);
+  const void* src[4] = {k, r, gy, v};
+  __nv_bfloat16* rv[4];
+  for (int i = 0; i < 4; ++i) {
+    rv[i] = reinterpret_cast<__nv_bfloat16*>(ws + L.rev[i]);
+    if (launch_flip_time(src[i], rv[i], iB, iT, W, st) != cudaSuccess) return RWKV_ERR_CUDA;
+  }
+  __nv_bfloat16 *k_rev = rv[0], *r_rev = rv[1], *gy_rev = rv[2], *v_rev = rv[3];
+  auto* gv_rev = reinterpret_cast<__nv_bfloat16*>(ws + L.gv_rev);
+  auto* gk_rev = reinterpret_cast<__nv_bfloat16*>(ws + L.gk_rev);
+  float* ckpt = reinterpret_cast<float*>(ws + L.ckpt);
+  double* part_f = reinterpret_cast<double*>(ws + L.part_f);
+  double* part_r = reinterpret_cast<double*>(ws + L.part_r);
+
+  // gv and the initial-state gradient: the forward operator over reversed time with r and k
+  // swapped and gy as the value, started from gs_out
+  {
+    CUtensorMap mr, mk, mv;
+    if (!make_bf16_box64_map(&mr, k_rev, iB, iT, W) || !make_bf16_box64_map(&mk, r_rev, iB, iT, W) ||
+        !make_bf16_box64_map(&mv, gy_rev, iB, iT, W))
+      return RWKV_ERR_CUDA;
+    Wkv5Params p{};
+    p.B = iB;
+    p.T = iT;
+    p.H = iH;
+    p.r = k_rev;
+    p.k = r_rev;
+    p.v = gy_rev;
+    p.omega = omega;
+    p.u = u;
+    p.y = gv_rev;
+    p.s_in = gs_out;
+    p.s_out = gs_in;
+    p.ctl = ctl;
+    if (launch_wkv5_fwd(mr, mk, mv, p, st) != cudaSuccess) return RWKV_ERR_CUDA;
+    if (launch_flip_time(gv_rev, gv, iB, iT, W, st) != cudaSuccess) return RWKV_ERR_CUDA;
+  }
+  const int nchunk = (iT + 63) / 64;
+  // gr, the forward states at chunk starts, the gu sums
+  {
+    CUtensorMap mq, mp, mc;
+    if (!make_bf16_box64_map(&mq, gy, iB, iT, W) || !make_bf16_box64_map(&mp, v, iB, iT, W) ||
+        !make_bf16_box64_map(&mc, k, iB, iT, W))
+      return RWKV_ERR_CUDA;
+    Wkv5BwdParams p{};
+    p.B = iB;
+    p.T = iT;
+    p.H = iH;
+    p.lead = 0;
+    p.m = static_cast<const __nv_bfloat16*>(r);
+    p.c = static_cast<const __nv_bfloat16*>(k);
+    p.omega = omega;
+    p.u = u;
+    p.x0 = s_in;
+    p.out = static_cast<__nv_bfloat16*>(gr);
+    p.ckpt = ckpt;
+    p.part = part_f;
+    p.ctl = ctl;
+    if (launch_wkv5_bwd_pass(false, mq, mp, mc, p, st) != cudaSuccess) return RWKV_ERR_CUDA;
+  }
+  // gk and the decay-gradient sums: reversed time, chunks aligned with the forward pass's
+  {
+    CUtensorMap mq, mp, mc;
+    if (!make_bf16_box64_map(&mq, v_rev, iB, iT, W) || !make_bf16_box64_map(&mp, gy_rev, iB, iT, W) ||
+        !make_bf16_box64_map(&mc, r_rev, iB, iT, W))
+      return RWKV_ERR_CUDA;
+    Wkv5BwdParams p{};
+    p.B = iB;
+    p.T = iT;
+    p.H = iH;
+    p.lead = 64 * nchunk - iT;
+    p.m = k_rev;
+    p.c = r_rev;
+    p.omega = omega;
+    p.u = u;
+    p.x0 = gs_out;
+    p.out = gk_rev;
+    p.ckpt = ckpt;
+    p.part = part_r;
+    p.ctl = ctl;
+    if (launch_wkv5_bwd_pass(true, mq, mp, mc, p, st) != cudaSuccess) return RWKV_ERR_CUDA;
+    if (launch_flip_time(gk_rev, gk, iB, iT, W, st) != cudaSuccess) return RWKV_ERR_CUDA;
+  }
+  if (launch_wkv5_bwd_reduce(iB, iH, part_f, part_r, omega, gomega, gu, st) != cudaSuccess) return RWKV_ERR_CUDA;
+  return RWKV_OK;
+}
+
 rwkv_status rwkv_check_device_error(rwkv_stream_t stream) {
   if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return RWKV_ERR_CUDA;
   unsigned int v = 0;
@@ -600,7 +766,7 @@ rwkv_status rwkv_check_device_error(rwkv_stream_t stream) {
   if (v != 0) {
     const unsigned int zero = 0;
     if (cudaMemcpyToSymbol(g_ctl, &zero, sizeof(zero), offsetof(DevCtl, err)) != cudaSuccess) return RWKV_ERR_CUDA;
-    return RWKV_ERR_DEVICE_TIMEOUT;
+    return (v & kErrTmaTimeout) ? RWKV_ERR_DEVICE_TIMEOUT : RWKV_ERR_UNSUPPORTED;
   }
   return RWKV_OK;
 }

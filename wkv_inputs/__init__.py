@@ -66,6 +66,8 @@ TID = {
     "omega": 7,
     "k_outlier": 8,
     "omega_t": 9,
+    "s_in": 10,
+    "gs_out": 11,
 }
 
 
@@ -237,4 +239,22 @@ def wkv6_problem(B: int, T: int, H: int, N: int, seed: int, device="cpu",
         om[s:s + blk] = (base.reshape(-1)[ix % (H * N)].double() +
                          omega_jitter * normal(seed, TID["omega_t"], ix)).to(torch.float32)
     out["omega"] = om.view(B, T, H, N)
+    return out
+
+
+def wkv5_grads(B: int, T: int, H: int, N: int, seed: int, device="cpu", states: bool = False) -> dict:
+    """Upstream gradients for the Eagle / Finch backward: gy [B, T, H, N] bf16 ~ N(0, 1) (rounded
+    to nearest even); with ``states``, an initial state s_in and a final-state gradient gs_out,
+    [B, H, N, N] fp32 ~ N(0, 1)/N (the scale of a state built from N(0,1)/sqrt(N) keys and values)."""
+    n = B * T * H * N
+    idx = torch.arange(n, dtype=torch.int64, device=device)
+    gy = torch.empty(n, dtype=torch.bfloat16, device=device)
+    blk = 1 << 23
+    for s in range(0, n, blk):
+        gy[s:s + blk] = normal(seed, TID["gy"], idx[s:s + blk]).to(torch.bfloat16)
+    out = {"gy": gy.view(B, T, H, N)}
+    if states:
+        m = torch.arange(B * H * N * N, dtype=torch.int64, device=device)
+        for name in ("s_in", "gs_out"):
+            out[name] = (normal(seed, TID[name], m) / N).to(torch.float32).view(B, H, N, N)
     return out
