@@ -643,7 +643,7 @@ def run_chunked(args):
     _, _, local = _dist()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    Bc, Tc, Cc = 8, 1024, 768
+    Bc, Tc, Cc = (1, 4096, 768) if args.chunked_shape == "1x4096x768" else (8, 1024, 768)
     p = wi.wkv4_problem(Bc, Tc, Cc, wi.CONFIG_SEED_BASE + 1, outliers=True, device=dev)
     w, u, k, v = p["w"], p["u"], p["k"], p["v"]
     y = torch.empty_like(k)
@@ -694,17 +694,19 @@ def run_chunked(args):
             clk_all = clk.summary()
     auto = res["auto"]["cold_ms"]["median"]
     gbs = nbytes / (auto * 1e-3) / 1e9
+    picked = "chunked" if int(h.rwkv_wkv4_forward_workspace_bytes(Bc, Tc, Cc, rw.ALGO_AUTO)) > 0 else "sequential"
     print(json.dumps({
-        "metric": "WKV-4 forward elements/s and HBM GB/s, few channels (B8 T1024 C768)",
+        "metric": f"WKV-4 forward elements/s and HBM GB/s, few channels (B{Bc} T{Tc} C{Cc})",
         "value": elems / (auto * 1e-3), "unit": "elements/s", "n_gpus": 1, "steps": len(res["auto"]["cold_ms"]),
         "warmup": args.warmup, "ms_per_step": auto, "higher_is_better": True, "dtype": "f32",
         "data": "synthetic",
-        "config": {"workload": "RWKV-4 WKV forward, fp32, B=8 T=1024 C=768, 1% +-U(20,40) key outliers",
+        "config": {"workload": f"RWKV-4 WKV forward, fp32, B={Bc} T={Tc} C={Cc}, 1% +-U(20,40) key outliers",
+                   "auto_picks": picked,
                    "l2": "flushed: a 256 MB buffer is written before every timed call (inputs fit in L2)"},
-        "roofline": {"bound": "hbm", "kernel": "wkv4_fwd_kernel x2 + wkv4_carry_kernel (AUTO picks chunked)",
+        "roofline": {"bound": "hbm", "kernel": f"wkv4_fwd_kernel (AUTO: {picked} schedule)",
                      "achieved": gbs, "peak": peak, "peak_kind": kind, "unit": "GB/s", "frac": gbs / peak,
                      "traffic": None},
-        "schedules": res, "gpu_launches": 3, "clocks": clk_all}), flush=True)
+        "schedules": res, "gpu_launches": 3 if picked == "chunked" else 1, "clocks": clk_all}), flush=True)
 
 
 def run_eagle(args, finch=False):
@@ -765,6 +767,54 @@ def run_eagle(args, finch=False):
         "roofline": {"bound": "hbm", "kernel": kernel, "achieved": gbs, "peak": peak, "peak_kind": kind,
                      "unit": "GB/s", "frac": gbs / peak, "traffic": _recorded_traffic(kernel)},
         "gpu_launches": args.steps, "clocks": clk, "call_ms": stats}), flush=True)
+
+
+def run_eagle_backward(args):
+    """Eagle / RWKV-5 backward on the forward workload's shape, B4 T4096 H40 N64 bf16, gy ~ N(0,1),
+    zero initial state and no final-state gradient: gr, gk, gv, gomega, gu."""
+    import torch
+
+    import rwkv_wkv_recurrence_b200 as rw
+    import wkv_inputs as wi
+
+    _, _, local = _dist()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    Be, Te, He, Ne = 4, 4096, 40, 64
+    q = wi.wkv5_problem(Be, Te, He, Ne, seed=SEED + 2, device=dev)
+    g = wi.wkv5_grads(Be, Te, He, Ne, seed=SEED + 6, device=dev)
+    gr, gk, gv = (torch.empty_like(q["r"]) for _ in range(3))
+    gom, gu = torch.empty(He, Ne, device=dev), torch.empty(He, Ne, device=dev)
+    h = rw.lib()
+    wsb = int(h.rwkv_wkv5_backward_workspace_bytes(Be, Te, He, Ne))
+    ws = torch.empty(max(wsb, 1), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    sp, P = rw._stream(stream), rw._ptr
+
+    def call(i):
+        with _Nvtx("rwkv_wkv5_backward"):
+            s = h.rwkv_wkv5_backward(Be, Te, He, Ne, P(q["r"]), P(q["k"]), P(q["v"]), P(q["omega"]), P(q["u"]), None,
+                                     P(g["gy"]), None, P(gr), P(gk), P(gv), P(gom), P(gu), None, P(ws), wsb, sp)
+        if s:
+            raise rw.RwkvError("rwkv_wkv5_backward", s)
+
+    ms, clk, stats = _timed(call, args.steps, args.warmup, stream, local)
+    rw.rwkv_check_device_error()
+    elems = Be * Te * He * Ne
+    nbytes = 7 * 2 * elems + 4 * He * Ne * 4  # r, k, v, gy read, gr, gk, gv written (bf16); omega, u, gomega, gu
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    peak, kind = _peaks()
+    print(json.dumps({
+        "metric": "Eagle WKV backward elements/s and HBM GB/s (B4 T4096 H40 N64)", "value": elems / (ms * 1e-3),
+        "unit": "elements/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "dtype": "bf16 I/O, fp32 state", "data": "synthetic",
+        "config": {"workload": "Eagle / RWKV-5 WKV backward, B=4 T=4096 H=40 N=64, bf16 r,k,v,gy,gr,gk,gv, "
+                               "gy ~ N(0,1), zero initial state, no final-state gradient",
+                   "l2": "no flush: 587 MB moved per call, above the 126 MB L2"},
+        "roofline": {"bound": "hbm", "kernel": "rwkv_wkv5_backward (reversed forward + two backward passes + "
+                                               "reduction)", "achieved": gbs, "peak": peak, "peak_kind": kind,
+                     "unit": "GB/s", "frac": gbs / peak, "traffic": None},
+        "gpu_launches": 4 * args.steps, "clocks": clk, "call_ms": stats}), flush=True)
 
 
 def run_eagle_decode(args, finch=False):
@@ -828,11 +878,13 @@ def main():
     ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["train", "train_gated", "decode", "chunked", "eagle", "eagle_decode",
-                                           "finch", "finch_decode"],
+    ap.add_argument("--workload", choices=["train", "train_gated", "decode", "chunked", "eagle", "eagle_bwd",
+                                           "eagle_decode", "finch", "finch_decode"],
                     default="train",
                     help="train: the headline forward+backward step; train_gated, decode, chunked, eagle, "
-                         "eagle_decode, finch, finch_decode: the other hot-path rows")
+                         "eagle_bwd, eagle_decode, finch, finch_decode: the other hot-path rows")
+    ap.add_argument("--chunked-shape", choices=["8x1024x768", "1x4096x768"], default="8x1024x768",
+                    help="the few-channel forward's shape (chunked workload)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--ref-channels", type=int, default=256)
@@ -851,6 +903,8 @@ def main():
         run_train_gated(args)
     elif args.workload == "eagle":
         run_eagle(args)
+    elif args.workload == "eagle_bwd":
+        run_eagle_backward(args)
     elif args.workload == "eagle_decode":
         run_eagle_decode(args)
     elif args.workload == "finch":

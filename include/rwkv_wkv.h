@@ -225,8 +225,8 @@ RWKV_API size_t rwkv_wkv5_backward_workspace_bytes(int64_t B, int64_t T, int64_t
  *   s_in          [B,H,N,N] fp32, the forward's initial state, or NULL (zero).
  *   gs_out        [B,H,N,N] fp32, the gradient of the final state, or NULL (zero).
  *   gs_in         [B,H,N,N] fp32, written with the gradient of s_in, or NULL (not wanted).
- *   workspace     device scratch of rwkv_wkv5_backward_workspace_bytes() bytes (time-reversed
- *                 copies of the inputs, the forward states at every 64th token, per-row sums).
+ *   workspace     device scratch of rwkv_wkv5_backward_workspace_bytes() bytes (the forward
+ *                 states at every 64th token, per-row sums).
  *   N must be 64; the [B,T,H,N] tensors 16-byte aligned (RWKV_ERR_UNSUPPORTED otherwise).
  *   A channel decaying faster than exp(omega) = 2.5 (w < 0.082) is outside the
  *   range this backward computes: the call returns RWKV_OK, the outputs of

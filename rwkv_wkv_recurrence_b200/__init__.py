@@ -69,7 +69,7 @@ def lib():
         "rwkv_wkv4_backward_noalloc": ([I64, I64, I64, I, P, P, P, P, P, P, I64, P, P, P, P, P], I),
         "rwkv_wkv5_step": ([I64, I64, I64, P, P, P, P, P, P, P, P, P], I),
         "rwkv_wkv5_backward_workspace_bytes": ([I64, I64, I64, I64], S),
-        "rwkv_wkv5_backward": ([I64, I64, I64, I64] + [P] * 14 + [S, P], I),
+        "rwkv_wkv5_backward": ([I64, I64, I64, I64] + [P] * 15 + [S, P], I),
         "rwkv_wkv6_forward_workspace_bytes": ([I64, I64, I64, I64], S),
         "rwkv_wkv6_forward": ([I64, I64, I64, I64, P, P, P, P, P, P, P, P, P, S, P], I),
         "rwkv_wkv6_step": ([I64, I64, I64, P, P, P, P, P, P, P, P, P], I),

@@ -125,7 +125,10 @@ FwdPlan plan_forward(int64_t B, int64_t T, int64_t C, int algo) {
   const int tt = fwd_tile_steps();
   const int64_t lane_tiles = B * ((C + 31) / 32);
   int a = algo;
-  if (a == RWKV_ALGO_AUTO) a = (lane_tiles >= 3 * kDesignSMs || T <= 128) ? RWKV_ALGO_SEQUENTIAL : RWKV_ALGO_CHUNKED;
+  // AUTO cuts time into segments only when one 32-channel tile per SM or fewer would run alone: at
+  // 8 x 1024 x 768 (192 tiles) the chunked schedule measured 42 us against 33 us sequential (its
+  // two passes share the SMs four CTAs at a time), at 1 x 4096 x 768 (24 tiles) it wins
+  if (a == RWKV_ALGO_AUTO) a = (lane_tiles < kDesignSMs && T >= 512) ? RWKV_ALGO_CHUNKED : RWKV_ALGO_SEQUENTIAL;
   if (a == RWKV_ALGO_CHUNKED && T > 0 && lane_tiles > 0) {
     // as many time segments as keep every CTA of a pass resident at once (four per SM): a
     // second wave would cost a whole segment's latency again
@@ -600,26 +603,15 @@ namespace {
 
 // Byte layout of the Eagle backward's workspace (every region 256-byte aligned).
 struct Wkv5BwdWs {
-  size_t rev[4];  // time-reversed k, r, gy, v (bf16 [B,T,H,64])
-  size_t gv_rev, gk_rev;
-  size_t ckpt;    // fp32 [B,H,nchunk,64,64]
-  size_t part_f, part_r;  // fp64 [B,H,64]
+  size_t ckpt;            // fp32 [B,H,nchunk,64,64]: forward states at chunk starts
+  size_t part_f, part_r;  // fp64 [B,H,64]: per-row sums of the two passes
   size_t total;
 };
 
 Wkv5BwdWs wkv5_bwd_ws(int64_t B, int64_t T, int64_t H) {
   auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
   Wkv5BwdWs w{};
-  const size_t seq = up((size_t)B * T * H * 64 * 2);
   size_t o = 0;
-  for (int i = 0; i < 4; ++i) {
-    w.rev[i] = o;
-    o += seq;
-  }
-  w.gv_rev = o;
-  o += seq;
-  w.gk_rev = o;
-  o += seq;
   w.ckpt = o;
   o += up((size_t)B * H * ((T + 63) / 64) * 64 * 64 * 4);
   w.part_f = o;
@@ -673,49 +665,35 @@ rwkv_status rwkv_wkv5_backward(int64_t B, int64_t T, int64_t H, int64_t N, const
   if (ctl == nullptr) return RWKV_ERR_CUDA;
   const int iB = (int)B, iT = (int)T, iH = (int)H, W = iH * 64;
   char* ws = static_cast<char*>(workspace);
-  const void* src[4] = {k, r, gy, v};
-  __nv_bfloat16* rv[4];
-  for (int i = 0; i < 4; ++i) {
-    rv[i] = reinterpret_cast<__nv_bfloat16*>(ws + L.rev[i]);
-    if (launch_flip_time(src[i], rv[i], iB, iT, W, st) != cudaSuccess) return RWKV_ERR_CUDA;
-  }
-  __nv_bfloat16 *k_rev = rv[0], *r_rev = rv[1], *gy_rev = rv[2], *v_rev = rv[3];
-  auto* gv_rev = reinterpret_cast<__nv_bfloat16*>(ws + L.gv_rev);
-  auto* gk_rev = reinterpret_cast<__nv_bfloat16*>(ws + L.gk_rev);
   float* ckpt = reinterpret_cast<float*>(ws + L.ckpt);
   double* part_f = reinterpret_cast<double*>(ws + L.part_f);
   double* part_r = reinterpret_cast<double*>(ws + L.part_r);
+  CUtensorMap mr, mk, mv, mg;
+  if (!make_bf16_box64_map(&mr, r, iB, iT, W) || !make_bf16_box64_map(&mk, k, iB, iT, W) ||
+      !make_bf16_box64_map(&mv, v, iB, iT, W) || !make_bf16_box64_map(&mg, gy, iB, iT, W))
+    return RWKV_ERR_CUDA;
 
   // gv and the initial-state gradient: the forward operator over reversed time with r and k
-  // swapped and gy as the value, started from gs_out
+  // swapped and gy as the value, started from gs_out (time reversed inside the kernel)
   {
-    CUtensorMap mr, mk, mv;
-    if (!make_bf16_box64_map(&mr, k_rev, iB, iT, W) || !make_bf16_box64_map(&mk, r_rev, iB, iT, W) ||
-        !make_bf16_box64_map(&mv, gy_rev, iB, iT, W))
-      return RWKV_ERR_CUDA;
     Wkv5Params p{};
     p.B = iB;
     p.T = iT;
     p.H = iH;
-    p.r = k_rev;
-    p.k = r_rev;
-    p.v = gy_rev;
+    p.r = static_cast<const __nv_bfloat16*>(k);
+    p.k = static_cast<const __nv_bfloat16*>(r);
+    p.v = static_cast<const __nv_bfloat16*>(gy);
     p.omega = omega;
     p.u = u;
-    p.y = gv_rev;
+    p.y = static_cast<__nv_bfloat16*>(gv);
     p.s_in = gs_out;
     p.s_out = gs_in;
     p.ctl = ctl;
-    if (launch_wkv5_fwd(mr, mk, mv, p, st) != cudaSuccess) return RWKV_ERR_CUDA;
-    if (launch_flip_time(gv_rev, gv, iB, iT, W, st) != cudaSuccess) return RWKV_ERR_CUDA;
+    if (launch_wkv5_fwd(mk, mr, mg, p, st, true) != cudaSuccess) return RWKV_ERR_CUDA;
   }
   const int nchunk = (iT + 63) / 64;
-  // gr, the forward states at chunk starts, the gu sums
+  // gr, the forward states at chunk starts, the gu sums: (q, p, c, m) = (gy, v, k, r)
   {
-    CUtensorMap mq, mp, mc;
-    if (!make_bf16_box64_map(&mq, gy, iB, iT, W) || !make_bf16_box64_map(&mp, v, iB, iT, W) ||
-        !make_bf16_box64_map(&mc, k, iB, iT, W))
-      return RWKV_ERR_CUDA;
     Wkv5BwdParams p{};
     p.B = iB;
     p.T = iT;
@@ -730,30 +708,26 @@ rwkv_status rwkv_wkv5_backward(int64_t B, int64_t T, int64_t H, int64_t N, const
     p.ckpt = ckpt;
     p.part = part_f;
     p.ctl = ctl;
-    if (launch_wkv5_bwd_pass(false, mq, mp, mc, p, st) != cudaSuccess) return RWKV_ERR_CUDA;
+    if (launch_wkv5_bwd_pass(false, mg, mv, mk, p, st) != cudaSuccess) return RWKV_ERR_CUDA;
   }
-  // gk and the decay-gradient sums: reversed time, chunks aligned with the forward pass's
+  // gk and the decay-gradient sums: (q, p, c, m) = (v, gy, r, k) over reversed time, chunks aligned
+  // with the forward pass's
   {
-    CUtensorMap mq, mp, mc;
-    if (!make_bf16_box64_map(&mq, v_rev, iB, iT, W) || !make_bf16_box64_map(&mp, gy_rev, iB, iT, W) ||
-        !make_bf16_box64_map(&mc, r_rev, iB, iT, W))
-      return RWKV_ERR_CUDA;
     Wkv5BwdParams p{};
     p.B = iB;
     p.T = iT;
     p.H = iH;
     p.lead = 64 * nchunk - iT;
-    p.m = k_rev;
-    p.c = r_rev;
+    p.m = static_cast<const __nv_bfloat16*>(k);
+    p.c = static_cast<const __nv_bfloat16*>(r);
     p.omega = omega;
     p.u = u;
     p.x0 = gs_out;
-    p.out = gk_rev;
+    p.out = static_cast<__nv_bfloat16*>(gk);
     p.ckpt = ckpt;
     p.part = part_r;
     p.ctl = ctl;
-    if (launch_wkv5_bwd_pass(true, mq, mp, mc, p, st) != cudaSuccess) return RWKV_ERR_CUDA;
-    if (launch_flip_time(gk_rev, gk, iB, iT, W, st) != cudaSuccess) return RWKV_ERR_CUDA;
+    if (launch_wkv5_bwd_pass(true, mv, mg, mr, p, st) != cudaSuccess) return RWKV_ERR_CUDA;
   }
   if (launch_wkv5_bwd_reduce(iB, iH, part_f, part_r, omega, gomega, gu, st) != cudaSuccess) return RWKV_ERR_CUDA;
   return RWKV_OK;

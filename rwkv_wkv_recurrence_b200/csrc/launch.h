@@ -95,8 +95,9 @@ struct Wkv6Params {
 
 // One pass of the Eagle backward (wkv5_bwd.cu): for queries q, keys p (both through TMA maps),
 // coefficients c and multipliers m (read directly), the state read with the decay on the output
-// channel.  Forward pass: gr, the state checkpoints and the gu sums; reversed pass (time-reversed
-// inputs, chunks aligned to the forward ones by `lead`): gk and the decay-gradient sums.
+// channel.  Forward pass: gr, the state checkpoints and the gu sums; reversed pass (time reversed
+// inside the kernel, the tensors read and written in their own order, chunks those of the forward
+// pass, the first `lead` positions empty): gk and the decay-gradient sums.
 struct Wkv5BwdParams {
   int B, T, H;
   int lead;                  // positions the first chunk starts before the sequence (reversed pass)
@@ -105,7 +106,7 @@ struct Wkv5BwdParams {
   const float* omega;        // [H,64]
   const float* u;            // [H,64]
   const float* x0;           // [B,H,64,64] carried state at the start, or null (zero)
-  __nv_bfloat16* out;        // [B,T,H,64]: gr, or gk in reversed time
+  __nv_bfloat16* out;        // [B,T,H,64]: gr (forward pass) or gk (reversed)
   float* ckpt;               // [B,H,nchunk,64,64] forward states at chunk starts (written / read)
   double* part;              // [B,H,64] per-row sums (gu parts / decay-gradient parts)
   DevCtl* ctl;
@@ -146,17 +147,17 @@ bool make_btc_map(CUtensorMap* m, const void* base, bool bf16, int B, int T, int
 // Tensor map over a bf16 [B, T, W] tensor with [1, 64, 64] boxes and the 128-byte swizzle.
 bool make_bf16_box64_map(CUtensorMap* m, const void* base, int B, int T, int W);
 cudaError_t launch_wkv5_step(const Wkv5StepParams& p, cudaStream_t st);
+// reversed: the operator over reversed time on tensors kept in their own order (token t of the
+// reversed problem is token T-1-t of r, k, v and y).
 cudaError_t launch_wkv5_fwd(const CUtensorMap& mr, const CUtensorMap& mk, const CUtensorMap& mv, const Wkv5Params& p,
-                            cudaStream_t st);
+                            cudaStream_t st, bool reversed = false);
 // mw: [1, 64, 32] fp32 boxes (128-byte swizzle) over omega [B, T, H*64].
 cudaError_t launch_wkv6_fwd(const CUtensorMap& mr, const CUtensorMap& mk, const CUtensorMap& mv,
                             const CUtensorMap& mw, const Wkv6Params& p, cudaStream_t st);
-// Eagle backward passes (maps over q, p, c: [1, 64, 64] bf16 boxes, 128-byte swizzle), the time
-// reversal of a bf16 [B, T, W] tensor (W a multiple of 8), and the batch reduction of the passes'
-// per-row sums into gomega and gu.
+// Eagle backward passes (maps over q, p, c: [1, 64, 64] bf16 boxes, 128-byte swizzle) and the batch
+// reduction of the passes' per-row sums into gomega and gu.
 cudaError_t launch_wkv5_bwd_pass(bool rev, const CUtensorMap& mq, const CUtensorMap& mp, const CUtensorMap& mc,
                                  const Wkv5BwdParams& p, cudaStream_t st);
-cudaError_t launch_flip_time(const void* in, void* out, int B, int T, int W, cudaStream_t st);
 cudaError_t launch_wkv5_bwd_reduce(int B, int H, const double* part_fwd, const double* part_rev, const float* omega,
                                    float* gomega, float* gu, cudaStream_t st);
 // Tensor map over an fp32 [B, T, W] tensor with [1, 64, 32] boxes and the 128-byte swizzle.

@@ -75,26 +75,34 @@ struct RSumm {  // a chunk's own reverse sums from a zero carry, at scale 2^q
 // scale 2^q, keeping e_t, G_t = gy_t / d_t, y_t and b_{t-1}.  gs holds the gy
 // rows, or with GATE the go rows: then gy_t = σ(r_t) go_t with r_t read from
 // rg[t * C], and gr_t is stored to grg[t * C].
+// The state recurrence, d_t and the numerator run in fp64 (lam = e^{-w}), and
+// y_t gets one correction step: gw sums 32,768 products of y-differences per
+// channel, and the fp32 recurrence's ~1e-6 error in y_t alone moved gw by up to
+// 5e-4 relative, against the 1e-4 bound.
 template <typename T, bool FULL, bool GATE>
 __device__ __forceinline__ void chunk_recompute(const T* ks, const T* vs, const T* gs, const T* rg, T* grg,
-                                                int C, int cnt, float qf, float U, float lh, float ll, float a,
-                                                float b, float (&E)[kL], float (&G)[kL], float (&Y)[kL],
-                                                float (&BP)[kL]) {
+                                                int C, int cnt, float qf, float U, double lam, double a, double b,
+                                                float (&E)[kL], float (&G)[kL], float (&Y)[kL], float (&BP)[kL]) {
   float rv[GATE ? kL : 1];
   if constexpr (GATE) {
 #pragma unroll
     for (int j = 0; j < kL; ++j) rv[j] = (rg != nullptr && (FULL || j < cnt)) ? IO<T>::load(rg + (size_t)j * C) : 0.f;
   }
+  const double Ud = (double)U;
 #pragma unroll
   for (int j = 0; j < kL; ++j) {
     if (FULL || j < cnt) {
       const float e = tok_weight(IO<T>::to_f(ks[j * 32]), qf);
-      const float eu = e * U;
       const float vj = IO<T>::to_f(vs[j * 32]);
-      const float d = b + eu;
+      const double ed = (double)e;
+      const double eud = ed * Ud;
+      const double dd = b + eud;
+      const double nd = fma(eud, (double)vj, a);
+      const float d = (float)dd;
       const float rd = rcp_approx(d);
       const bool ok = !(d < kMinDen);  // else no history and e^{u+k} underflowed: WKV = v locally (NaN: ok)
-      Y[j] = ok ? fmaf(eu, vj, a) * rd : vj;
+      const float y0 = (float)nd * rd;
+      Y[j] = ok ? fmaf((float)fma(-(double)y0, dd, nd), rd, y0) : vj;  // y0 + (n - y0 d) / d
       float gy;
       if constexpr (GATE) {
         const float sg = sigmoid(rv[j]);
@@ -106,9 +114,9 @@ __device__ __forceinline__ void chunk_recompute(const T* ks, const T* vs, const 
       }
       G[j] = ok ? gy * rd : 0.f;
       E[j] = e;
-      BP[j] = b;
-      a = decay_add(a, e * vj, lh, ll);
-      b = decay_add(b, e, lh, ll);
+      BP[j] = (float)b;  // b_{t-1}
+      a = fma(ed, (double)vj, lam * a);
+      b = fma(lam, b, ed);
     }
   }
 }
@@ -290,11 +298,9 @@ __global__ void __launch_bounds__(kW * 32, 4) wkv4_bwd_kernel(const __grid_const
     float E[kL], G[kL], Y[kL], BP[kL];
     const int q = st.p;
     if (cnt == kL)
-      chunk_recompute<T, true, GATE>(ks, vs, gs, rg, grg, p.C, cnt, (float)q, U, lh, ll, (float)st.a, (float)st.b,
-                                     E, G, Y, BP);
+      chunk_recompute<T, true, GATE>(ks, vs, gs, rg, grg, p.C, cnt, (float)q, U, lam, st.a, st.b, E, G, Y, BP);
     else if (cnt > 0)
-      chunk_recompute<T, false, GATE>(ks, vs, gs, rg, grg, p.C, cnt, (float)q, U, lh, ll, (float)st.a,
-                                      (float)st.b, E, G, Y, BP);
+      chunk_recompute<T, false, GATE>(ks, vs, gs, rg, grg, p.C, cnt, (float)q, U, lam, st.a, st.b, E, G, Y, BP);
 
     // B. the chunk's own reverse sums
     float la = 0.f, lg = 0.f, ye = 0.f;

@@ -15,7 +15,9 @@
 //              + u_d c_t[d] (q_t·p_t),      X ← diag(w) X + c_tᵀ p_t,
 // which is gr for (q, p, c, X_0) = (gy, v, k, s_in) in forward time, and gk for
 // (q, p, c, X_0) = (v, gy, r, gs_out) with time reversed.  One kernel runs
-// either pass (REV = the reversed one).
+// either pass (REV = the reversed one).  The reversed pass reads and writes
+// the tensors in their own order: its chunk c is forward chunk nchunk-1-c,
+// loaded as usual, with its rows taken bottom up.
 //
 // Chunked form (chunk of 64 positions, λ_d = -exp(ω_d), c̃_ι = c_ι e^{λ(31-ι)}):
 //   A[τ][ι]  = q_τ·p_ι                                 (no decay: a plain product)
@@ -41,9 +43,9 @@
 // (checkpoints): the first term is elementwise, the second is its own state
 // read weighted by position, the third one more chain (X_c · gyᵀ), the last
 // one more chain with the masked scores weighted by the lag.  The reversed
-// pass aligns its chunks with the forward ones: its first chunk starts `lead`
-// positions early (TMA rows at negative coordinates read as zero) and its
-// carried state enters at position `lead`.
+// pass's chunks are the forward ones: its first (the partial last forward
+// chunk, whose rows past the sequence read as zero) has `lead` empty positions
+// before the carried state enters.
 //
 // CTA: one (batch, head), 8 warps.  Forward pass: ~105 KB of shared memory,
 // 256 TMEM columns, two CTAs per SM.  Reversed pass: ~140 KB, 512 columns, one
@@ -128,6 +130,7 @@ __global__ void __launch_bounds__(kThreads, REV ? 1 : 2) wkv5_bwd_tc_kernel(cons
   if (warp == 0) tmem_alloc(&sm.tmem_base, REV ? 512u : 256u);
   const bool withheld = tid == 0 && loads_withheld(p.ctl);
   // chunk c covers positions [c*64 - lead, c*64 - lead + 64) of the pass's own time
+  // the box of chunk c starts at token 64 c (forward pass) or 64 (nchunk-1-c) (reversed pass)
   if (tid == 0) {
     prefetch_tensormap(&mq);
     prefetch_tensormap(&mp);
@@ -139,23 +142,27 @@ __global__ void __launch_bounds__(kThreads, REV ? 1 : 2) wkv5_bwd_tc_kernel(cons
     fence_mbar_init();
     mbar_arrive_expect_tx(&sm.bar_tma, 3 * kRawBytes);
     if (!withheld) {
-      tma_load_3d(sm.raw[0], &mq, &sm.bar_tma, h * kN, -p.lead, b);
-      tma_load_3d(sm.raw[1], &mp, &sm.bar_tma, h * kN, -p.lead, b);
-      tma_load_3d(sm.raw[2], &mc, &sm.bar_tma, h * kN, -p.lead, b);
+      const int row0 = REV ? kL * (nchunk - 1) : 0;
+      tma_load_3d(sm.raw[0], &mq, &sm.bar_tma, h * kN, row0, b);
+      tma_load_3d(sm.raw[1], &mp, &sm.bar_tma, h * kN, row0, b);
+      tma_load_3d(sm.raw[2], &mc, &sm.bar_tma, h * kN, row0, b);
     }
   }
 
-  // ---- q, p (shared memory, unscaled): warp w owns channels 8w..8w+7, lane holds rows 8 ib + rr,
-  // channels dR, dR + 1; a half-warp writes one whole core matrix
+  // ---- q, p (shared memory, unscaled): warp w owns channels 8w..8w+7, lane holds positions
+  // 8 ib + rr, channels dR, dR + 1; a half-warp writes one whole core matrix.  Position τ is box
+  // row τ, or 63 - τ in the reversed pass.
   const int rr = lane & 7, rp = lane >> 3;
   const int dR = 8 * warp + 2 * rp;
-  const uint32_t offRK = (uint32_t)rr * 128u + (uint32_t)((warp ^ rr) << 4) + (uint32_t)rp * 4u;
+  const int rb = REV ? 7 - rr : rr;
+  const uint32_t offRK = (uint32_t)rb * 128u + (uint32_t)((warp ^ rb) << 4) + (uint32_t)rp * 4u;
   const int lrow = lane & 7, lmat = lane >> 3;
   // ---- pᵀ (shared memory): ldmatrix.trans of block column w; lanes whose bit 1 and bit 4 differ
   // trade their pair with lane ^ 18 so that each half-warp covers one core matrix
   const int sw = ((lane >> 1) ^ (lane >> 4)) & 1;
   const int srow = t4 ^ (sw << 2), stq = tq ^ (sw << 1);
-  const uint32_t offT = (uint32_t)(lmat * 8 + lrow) * 128u + (uint32_t)((warp ^ lrow) << 4);
+  const uint32_t offT = REV ? (uint32_t)(63 - lmat * 8 - lrow) * 128u + (uint32_t)((warp ^ (7 - lrow)) << 4)
+                            : (uint32_t)(lmat * 8 + lrow) * 128u + (uint32_t)((warp ^ lrow) << 4);
   // ---- c̃ᵀ (tensor memory, A of the intra term and of the state increment), .16x256b fragment:
   // rows d = 16 q4 + t4 + 8 r, columns ι = 32 hc + 8 i + 2 tq + e  ->  register 4 i + 2 r + e
   float fc0[2][2], fcs[2];
@@ -166,8 +173,9 @@ __global__ void __launch_bounds__(kThreads, REV ? 1 : 2) wkv5_bwd_tc_kernel(cons
     for (int e = 0; e < 2; ++e) fc0[r][e] = expf(-rate * (float)(31 - 32 * hc - 2 * tq - e));
     fcs[r] = expf(8.f * rate);
   }
-  const uint32_t offKt = (uint32_t)((4 * hc + (lmat >> 1)) * 8 + lrow) * 128u +
-                         (uint32_t)(((2 * q4 + (lmat & 1)) ^ lrow) << 4);
+  const uint32_t offKt =
+      REV ? (uint32_t)(63 - (4 * hc + (lmat >> 1)) * 8 - lrow) * 128u + (uint32_t)(((2 * q4 + (lmat & 1)) ^ (7 - lrow)) << 4)
+          : (uint32_t)((4 * hc + (lmat >> 1)) * 8 + lrow) * 128u + (uint32_t)(((2 * q4 + (lmat & 1)) ^ lrow) << 4);
 
   // ---- carried state X[d][j] (fp32) in the .16x128b fragment: d = 16 q4 + t4 + 8 r,
   // j = 32 hc + 4 q + tq  ->  X[2 q + r]
@@ -213,9 +221,9 @@ __global__ void __launch_bounds__(kThreads, REV ? 1 : 2) wkv5_bwd_tc_kernel(cons
   int c = 0;
   bool aborted = false;
   for (; c < nchunk; ++c) {
-    const int t0 = c * kL - p.lead;            // pass position of row 0 of this chunk
-    const int lo = max(0, -t0);                // rows before the sequence start (first reversed chunk)
-    const int cnt = min(kL, p.T - t0);         // rows up to the sequence end (last forward chunk)
+    const int t0 = c * kL - p.lead;            // pass position of position 0 of this chunk
+    const int lo = max(0, -t0);                // positions before the sequence start (first reversed chunk)
+    const int cnt = min(kL, p.T - t0);         // positions up to the sequence end (last forward chunk)
     const uint32_t ph = (uint32_t)c & 1u;
     const int cf = nchunk - 1 - c;             // reversed pass: the forward chunk this one mirrors
 
@@ -249,8 +257,9 @@ __global__ void __launch_bounds__(kThreads, REV ? 1 : 2) wkv5_bwd_tc_kernel(cons
 #pragma unroll
     for (int ib = 0; ib < 8; ++ib) {
       const int row = 8 * ib + rr;
-      *reinterpret_cast<float2*>(&sm.opQ[op_off(row, dR)]) = bf2_to_f2(lds_u32(rawQ + offRK + ib * 1024u));
-      *reinterpret_cast<float2*>(&sm.opP[op_off(row, dR)]) = bf2_to_f2(lds_u32(rawP + offRK + ib * 1024u));
+      const uint32_t ibo = (uint32_t)(REV ? 7 - ib : ib) * 1024u;
+      *reinterpret_cast<float2*>(&sm.opQ[op_off(row, dR)]) = bf2_to_f2(lds_u32(rawQ + offRK + ibo));
+      *reinterpret_cast<float2*>(&sm.opP[op_off(row, dR)]) = bf2_to_f2(lds_u32(rawP + offRK + ibo));
     }
     fence_proxy_async();
     tc_fence_before();
@@ -283,7 +292,7 @@ __global__ void __launch_bounds__(kThreads, REV ? 1 : 2) wkv5_bwd_tc_kernel(cons
 #pragma unroll
       for (int pp = 0; pp < 2; ++pp) {
         uint32_t qk[4];
-        ldsm_x4_t(rawC + offKt + pp * 2048u, qk);
+        ldsm_x4_t(REV ? rawC + offKt - pp * 2048u : rawC + offKt + pp * 2048u, qk);
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
           const int i = 2 * pp + (m >> 1), r = m & 1;
@@ -298,7 +307,7 @@ __global__ void __launch_bounds__(kThreads, REV ? 1 : 2) wkv5_bwd_tc_kernel(cons
 #pragma unroll
       for (int pp = 0; pp < 2; ++pp) {
         uint32_t qv[4];
-        ldsm_x4_t(rawP + offT + pp * 4096u, qv);
+        ldsm_x4_t(REV ? rawP + offT - pp * 4096u : rawP + offT + pp * 4096u, qv);
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
           const int ib = 4 * pp + m;
@@ -318,9 +327,10 @@ __global__ void __launch_bounds__(kThreads, REV ? 1 : 2) wkv5_bwd_tc_kernel(cons
       if (c + 1 < nchunk) {
         fence_proxy_async();
         mbar_arrive_expect_tx(&sm.bar_tma, 3 * kRawBytes);
-        tma_load_3d(sm.raw[0], &mq, &sm.bar_tma, h * kN, t0 + kL, b);
-        tma_load_3d(sm.raw[1], &mp, &sm.bar_tma, h * kN, t0 + kL, b);
-        tma_load_3d(sm.raw[2], &mc, &sm.bar_tma, h * kN, t0 + kL, b);
+        const int rown = REV ? kL * (cf - 1) : t0 + kL;
+        tma_load_3d(sm.raw[0], &mq, &sm.bar_tma, h * kN, rown, b);
+        tma_load_3d(sm.raw[1], &mp, &sm.bar_tma, h * kN, rown, b);
+        tma_load_3d(sm.raw[2], &mc, &sm.bar_tma, h * kN, rown, b);
       }
     }
 
@@ -396,8 +406,8 @@ __global__ void __launch_bounds__(kThreads, REV ? 1 : 2) wkv5_bwd_tc_kernel(cons
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const int pos = (int)col + i;
-          const int t = t0 + pos;
           if (pos < lo || pos >= cnt) continue;
+          const int t = REV ? kL * cf + (kL - 1 - pos) : t0 + pos;  // token of this position
           const size_t off = ((row0 + (size_t)t * p.H) * kN) + de;
           const float cval = bf(p.c + off), mval = bf(p.m + off);
           const float dg = sm.diag[pos];
@@ -479,16 +489,6 @@ __global__ void __launch_bounds__(kThreads, REV ? 1 : 2) wkv5_bwd_tc_kernel(cons
   }
 }
 
-// Reverses the time axis of a bf16 [B, T, W] tensor (W a multiple of 8): out[b][T-1-t] = in[b][t].
-__global__ void flip_time_kernel(const uint4* __restrict__ in, uint4* __restrict__ out, int B, int T, int wv) {
-  const size_t n = (size_t)B * T * wv;
-  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
-    const size_t v = i % wv, bt = i / wv;
-    const size_t t = bt % T, bb = bt / T;
-    out[(bb * T + (T - 1 - t)) * wv + v] = in[i];
-  }
-}
-
 // gomega[h][d] = Σ_b part_rev[b][h][d] · dw/dω (dw/dω = -e^ω w), gu[h][d] = Σ_b part_fwd[b][h][d], in
 // batch order (deterministic).
 __global__ void wkv5_reduce_kernel(int B, int H, const double* __restrict__ part_fwd,
@@ -522,14 +522,6 @@ cudaError_t launch_wkv5_bwd_pass(bool rev, const CUtensorMap& mq, const CUtensor
     wkv5_bwd_tc_kernel<true><<<(unsigned)(p.B * p.H), kThreads, smem, st>>>(mq, mp, mc, p);
   else
     wkv5_bwd_tc_kernel<false><<<(unsigned)(p.B * p.H), kThreads, smem, st>>>(mq, mp, mc, p);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_flip_time(const void* in, void* out, int B, int T, int W, cudaStream_t st) {
-  const int wv = W / 8;
-  const size_t n = (size_t)B * T * wv;
-  const unsigned grid = (unsigned)std::min<size_t>((n + 255) / 256, 148 * 16);
-  flip_time_kernel<<<grid, 256, 0, st>>>(static_cast<const uint4*>(in), static_cast<uint4*>(out), B, T, wv);
   return cudaGetLastError();
 }
 

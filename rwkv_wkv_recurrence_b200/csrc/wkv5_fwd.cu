@@ -63,10 +63,11 @@ constexpr uint32_t kTmemCols = 256;  // [scores | output rows], state increment,
 
 // The recurrence for one head (used when a channel decays too fast for the
 // chunked factorization): thread j < 64 owns value column j of the state.
+// With rev, step t reads and writes token T-1-t (the operator over reversed time).
 __device__ __noinline__ void head_recurrent(int b, int h, int T, int H, const __nv_bfloat16* __restrict__ r,
                                const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
                                const float* wdec, const float* ud, __nv_bfloat16* __restrict__ y,
-                               const float* s_in, float* s_out, float* sm_r, float* sm_k) {
+                               const float* s_in, float* s_out, float* sm_r, float* sm_k, bool rev) {
   const int j = threadIdx.x;
   const size_t sbase = ((size_t)b * H + h) * kN * kN;
   float s[kN];
@@ -75,7 +76,7 @@ __device__ __noinline__ void head_recurrent(int b, int h, int T, int H, const __
     for (int i = 0; i < kN; ++i) s[i] = s_in ? s_in[sbase + (size_t)i * kN + j] : 0.f;
   }
   for (int t = 0; t < T; ++t) {
-    const size_t off = (((size_t)b * T + t) * H + h) * kN;
+    const size_t off = (((size_t)b * T + (rev ? T - 1 - t : t)) * H + h) * kN;
     __syncthreads();
     if (j < kN) {
       sm_r[j] = __bfloat162float(r[off + j]);
@@ -122,6 +123,10 @@ struct Wkv5Smem {
 static_assert(offsetof(Wkv5Smem, opS) == offsetof(Wkv5Smem, opK) + 64 * 64 * sizeof(float),
               "the first product reads k̃ and e^{32λ} Sᵀ as one 128-row operand");
 
+// REV: the operator over reversed time (position τ of chunk c is token T-1-(64c+τ)), reading and
+// writing the tensors in their own order: chunk c's box starts at token T-64(c+1) (rows before
+// token 0 read as zeros), its rows are taken bottom up, and y row τ goes to token T-1-(64c+τ).
+template <bool REV>
 __global__ void __launch_bounds__(kThreads, 2) wkv5_fwd_tc_kernel(const __grid_constant__ CUtensorMap mr,
                                                                   const __grid_constant__ CUtensorMap mk,
                                                                   const __grid_constant__ CUtensorMap mv,
@@ -150,7 +155,7 @@ __global__ void __launch_bounds__(kThreads, 2) wkv5_fwd_tc_kernel(const __grid_c
       sm.opS[64 + tid] = p.u[h * kN + tid];
     }
     __syncthreads();
-    head_recurrent(b, h, p.T, p.H, p.r, p.k, p.v, &sm.opS[0], &sm.opS[64], p.y, p.s_in, p.s_out, sm.opR, sm.opK);
+    head_recurrent(b, h, p.T, p.H, p.r, p.k, p.v, &sm.opS[0], &sm.opS[64], p.y, p.s_in, p.s_out, sm.opR, sm.opK, REV);
     return;
   }
 
@@ -168,9 +173,10 @@ __global__ void __launch_bounds__(kThreads, 2) wkv5_fwd_tc_kernel(const __grid_c
     fence_mbar_init();
     mbar_arrive_expect_tx(&sm.bar_tma, 3 * kRawBytes);
     if (!withheld) {
-      tma_load_3d(sm.raw[0], &mr, &sm.bar_tma, h * kN, 0, b);
-      tma_load_3d(sm.raw[1], &mk, &sm.bar_tma, h * kN, 0, b);
-      tma_load_3d(sm.raw[2], &mv, &sm.bar_tma, h * kN, 0, b);
+      const int row0 = REV ? p.T - kL : 0;
+      tma_load_3d(sm.raw[0], &mr, &sm.bar_tma, h * kN, row0, b);
+      tma_load_3d(sm.raw[1], &mk, &sm.bar_tma, h * kN, row0, b);
+      tma_load_3d(sm.raw[2], &mv, &sm.bar_tma, h * kN, row0, b);
     }
   }
 
@@ -188,13 +194,17 @@ __global__ void __launch_bounds__(kThreads, 2) wkv5_fwd_tc_kernel(const __grid_c
     fks[e] = expf(8.f * rate);
     uA[e] = p.u[h * kN + dR + e];
   }
-  const uint32_t offRK = (uint32_t)rr * 128u + (uint32_t)((warp ^ rr) << 4) + (uint32_t)rp * 4u;
+  // box row of position 8 ib + rr: 8 ib + rr, or 63 - (8 ib + rr) = 8 (7 - ib) + (7 - rr) reversed
+  const int rb = REV ? 7 - rr : rr;
+  const uint32_t offRK = (uint32_t)rb * 128u + (uint32_t)((warp ^ rb) << 4) + (uint32_t)rp * 4u;
   const int lrow = lane & 7, lmat = lane >> 3;
   // ---- vᵀ (shared memory): ldmatrix.trans of block column w; lanes whose bit 1 and bit 4 differ
   // trade their pair with lane ^ 18 so that each half-warp again covers one core matrix.
   const int sw = ((lane >> 1) ^ (lane >> 4)) & 1;
   const int srow = t4 ^ (sw << 2), stq = tq ^ (sw << 1);
-  const uint32_t offT = (uint32_t)(lmat * 8 + lrow) * 128u + (uint32_t)((warp ^ lrow) << 4);
+  // lane's row address for ldmatrix: position 8 lmat + lrow (+ 32 per pp), its box row bottom up when REV
+  const uint32_t offT = REV ? (uint32_t)(63 - lmat * 8 - lrow) * 128u + (uint32_t)((warp ^ (7 - lrow)) << 4)
+                            : (uint32_t)(lmat * 8 + lrow) * 128u + (uint32_t)((warp ^ lrow) << 4);
   // ---- k̃ᵀ (tensor memory, A of the state increment), .16x256b fragment of warp w:
   // rows d = 16 q4 + t4 + 8 r, columns ι = 32 hc + 8 i + 2 tq + e  ->  register 4 i + 2 r + e
   float fc0[2][2], fcs[2];
@@ -205,8 +215,10 @@ __global__ void __launch_bounds__(kThreads, 2) wkv5_fwd_tc_kernel(const __grid_c
     for (int e = 0; e < 2; ++e) fc0[r][e] = expf(-rate * (float)(31 - 32 * hc - 2 * tq - e));
     fcs[r] = expf(8.f * rate);
   }
-  const uint32_t offKt = (uint32_t)((4 * hc + (lmat >> 1)) * 8 + lrow) * 128u +
-                         (uint32_t)(((2 * q4 + (lmat & 1)) ^ lrow) << 4);
+  // position 32 hc + 8 (lmat >> 1) + lrow (+ 16 per pp); its box row bottom up when REV
+  const uint32_t offKt =
+      REV ? (uint32_t)(63 - (4 * hc + (lmat >> 1)) * 8 - lrow) * 128u + (uint32_t)(((2 * q4 + (lmat & 1)) ^ (7 - lrow)) << 4)
+          : (uint32_t)((4 * hc + (lmat >> 1)) * 8 + lrow) * 128u + (uint32_t)(((2 * q4 + (lmat & 1)) ^ lrow) << 4);
 
   // ---- state S[d][j] (fp32 master copy) in the .16x128b fragment of warp w:
   // d = 16 q4 + t4 + 8 r, j = 32 hc + 4 q + tq  ->  S[2 q + r]
@@ -249,8 +261,9 @@ __global__ void __launch_bounds__(kThreads, 2) wkv5_fwd_tc_kernel(const __grid_c
       float fr[2] = {fr0[0], fr0[1]}, fk[2] = {fk0[0], fk0[1]};
 #pragma unroll
       for (int ib = 0; ib < 8; ++ib) {
-        const float2 rv = bf2_to_f2(lds_u32(rawR + offRK + ib * 1024u));
-        const float2 kv = bf2_to_f2(lds_u32(rawK + offRK + ib * 1024u));
+        const uint32_t ibo = (uint32_t)(REV ? 7 - ib : ib) * 1024u;
+        const float2 rv = bf2_to_f2(lds_u32(rawR + offRK + ibo));
+        const float2 kv = bf2_to_f2(lds_u32(rawK + offRK + ibo));
         const int row = 8 * ib + rr;
         *reinterpret_cast<float2*>(&sm.opR[op_off(row, dR)]) = make_float2(rv.x * fr[0], rv.y * fr[1]);
         *reinterpret_cast<float2*>(&sm.opK[op_off(row, dR)]) = make_float2(kv.x * fk[0], kv.y * fk[1]);
@@ -299,7 +312,7 @@ __global__ void __launch_bounds__(kThreads, 2) wkv5_fwd_tc_kernel(const __grid_c
 #pragma unroll
       for (int pp = 0; pp < 2; ++pp) {
         uint32_t qk[4];
-        ldsm_x4_t(rawK + offKt + pp * 2048u, qk);
+        ldsm_x4_t(REV ? rawK + offKt - pp * 2048u : rawK + offKt + pp * 2048u, qk);
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
           const int i = 2 * pp + (m >> 1), r = m & 1;
@@ -314,7 +327,7 @@ __global__ void __launch_bounds__(kThreads, 2) wkv5_fwd_tc_kernel(const __grid_c
 #pragma unroll
       for (int pp = 0; pp < 2; ++pp) {
         uint32_t qv[4];
-        ldsm_x4_t(rawV + offT + pp * 4096u, qv);
+        ldsm_x4_t(REV ? rawV + offT - pp * 4096u : rawV + offT + pp * 4096u, qv);
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
           const int ib = 4 * pp + m;
@@ -334,9 +347,10 @@ __global__ void __launch_bounds__(kThreads, 2) wkv5_fwd_tc_kernel(const __grid_c
       if (c + 1 < nchunk) {
         fence_proxy_async();
         mbar_arrive_expect_tx(&sm.bar_tma, 3 * kRawBytes);
-        tma_load_3d(sm.raw[0], &mr, &sm.bar_tma, h * kN, (c + 1) * kL, b);
-        tma_load_3d(sm.raw[1], &mk, &sm.bar_tma, h * kN, (c + 1) * kL, b);
-        tma_load_3d(sm.raw[2], &mv, &sm.bar_tma, h * kN, (c + 1) * kL, b);
+        const int rown = REV ? p.T - (c + 2) * kL : (c + 1) * kL;
+        tma_load_3d(sm.raw[0], &mr, &sm.bar_tma, h * kN, rown, b);
+        tma_load_3d(sm.raw[1], &mk, &sm.bar_tma, h * kN, rown, b);
+        tma_load_3d(sm.raw[2], &mv, &sm.bar_tma, h * kN, rown, b);
       }
     }
 
@@ -392,7 +406,8 @@ __global__ void __launch_bounds__(kThreads, 2) wkv5_fwd_tc_kernel(const __grid_c
       tmem_ld32(tY + tquar + (uint32_t)(32 * hc), yv);
       const int tau = 16 * q4 + lane;
       if (lane < 16 && tau < cnt) {
-        __nv_bfloat16* yp = p.y + (((size_t)b * p.T + t0 + tau) * p.H + h) * kN + 32 * hc;
+        const int ty = REV ? p.T - 1 - (t0 + tau) : t0 + tau;
+        __nv_bfloat16* yp = p.y + (((size_t)b * p.T + ty) * p.H + h) * kN + 32 * hc;
 #pragma unroll
         for (int j = 0; j < 32; j += 8) {
           uint4 pk;
@@ -458,12 +473,17 @@ __global__ void __launch_bounds__(kThreads, 2) wkv5_fwd_tc_kernel(const __grid_c
 size_t wkv5_smem_bytes() { return sizeof(Wkv5Smem) + 1024; }  // + alignment slack
 
 cudaError_t launch_wkv5_fwd(const CUtensorMap& mr, const CUtensorMap& mk, const CUtensorMap& mv, const Wkv5Params& p,
-                            cudaStream_t st) {
+                            cudaStream_t st, bool reversed) {
   const size_t smem = wkv5_smem_bytes();
-  static unsigned device_mask = 0;
-  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(wkv5_fwd_tc_kernel), (int)smem, &device_mask);
+  static unsigned mask_f = 0, mask_r = 0;
+  const void* fn = reversed ? reinterpret_cast<const void*>(wkv5_fwd_tc_kernel<true>)
+                            : reinterpret_cast<const void*>(wkv5_fwd_tc_kernel<false>);
+  cudaError_t e = ensure_smem_attr(fn, (int)smem, reversed ? &mask_r : &mask_f);
   if (e != cudaSuccess) return e;
-  wkv5_fwd_tc_kernel<<<(unsigned)(p.B * p.H), kThreads, smem, st>>>(mr, mk, mv, p);
+  if (reversed)
+    wkv5_fwd_tc_kernel<true><<<(unsigned)(p.B * p.H), kThreads, smem, st>>>(mr, mk, mv, p);
+  else
+    wkv5_fwd_tc_kernel<false><<<(unsigned)(p.B * p.H), kThreads, smem, st>>>(mr, mk, mv, p);
   return cudaGetLastError();
 }
 

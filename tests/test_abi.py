@@ -52,9 +52,12 @@ def test_checkpoint_and_workspace_queries():
     # many channels: the sequential schedule needs no workspace
     assert h.rwkv_wkv4_forward_workspace_bytes(B, T, C, rw.ALGO_AUTO) == 0
     assert h.rwkv_wkv4_forward_workspace_bytes(B, T, C, rw.ALGO_SEQUENTIAL) == 0
-    # few channels: the chunked schedule keeps one state per segment
-    ws = h.rwkv_wkv4_forward_workspace_bytes(8, 1024, 768, rw.ALGO_AUTO)
-    assert ws > 0 and ws % (3 * 8 * 768 * 4) == 0
+    # 192 channel tiles (8 x 768): AUTO keeps the sequential schedule, which measured faster there;
+    # 24 tiles (1 x 768) over 4096 steps: AUTO cuts time into segments, one state per segment
+    assert h.rwkv_wkv4_forward_workspace_bytes(8, 1024, 768, rw.ALGO_AUTO) == 0
+    ws = h.rwkv_wkv4_forward_workspace_bytes(1, 4096, 768, rw.ALGO_AUTO)
+    assert ws > 0 and ws % (3 * 1 * 768 * 4) == 0
+    assert h.rwkv_wkv4_forward_workspace_bytes(8, 1024, 768, rw.ALGO_CHUNKED) > 0
     assert h.rwkv_wkv4_forward_workspace_bytes(0, 10, 10, 0) == 0
 
 

@@ -196,7 +196,10 @@ def test_wkv4_step_guarded(cuda_device, C, dt):
 def test_matrix_state_guarded(cuda_device, finch):
     B, T, H = 2, 150, 3
     dev = cuda_device
-    p = (wi.wkv6_problem if finch else wi.wkv5_problem)(B, T, H, 64, seed=74)
+    # one problem of T + 1 tokens: the forward runs over the first T, the decode step takes the last
+    q = (wi.wkv6_problem if finch else wi.wkv5_problem)(B, T + 1, H, 64, seed=74)
+    names = ("r", "k", "v", "omega") if finch else ("r", "k", "v")
+    p = {n: (q[n][:, :T].contiguous() if n in names else q[n]) for n in q}
     g = {k: v.to(dev) for k, v in p.items()}
     h = rw.lib()
     P, S = rw._ptr, rw._stream(None)
@@ -213,8 +216,6 @@ def test_matrix_state_guarded(cuda_device, finch):
     assert_close_rms(y.t, ref, TOL_BF16, "y")
     assert_close_rms(so.t, ref_s, TOL_BF16, "s_out")
     # one decode step from that state, into guarded outputs
-    q = (wi.wkv6_problem if finch else wi.wkv5_problem)(B, T + 1, H, 64, seed=74)
-    names = ("r", "k", "v", "omega") if finch else ("r", "k", "v")
     tok = {n: q[n][:, T].contiguous().to(dev) for n in names}
     ys = Guarded((B, H, 64), torch.bfloat16, dev)
     s1 = Guarded((B, H, 64, 64), torch.float32, dev)
