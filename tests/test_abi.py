@@ -94,8 +94,10 @@ def test_validation_before_any_cuda_work():
     assert h.rwkv_wkv4_forward(1, 4, 4, 1, fake, fake, fake, P(0x1001), fake, None, None, None, 16, 0, None,
                                0, None) == 2
     # chunked schedule without its workspace
-    assert h.rwkv_wkv4_forward(8, 1024, 768, 0, fake, fake, fake, fake, fake, None, None, None, 16, 0, None, 0,
-                               None) == 3
+    assert h.rwkv_wkv4_forward(8, 1024, 768, 0, fake, fake, fake, fake, fake, None, None, None, 16,
+                               rw.ALGO_CHUNKED, None, 0, None) == 3
+    assert h.rwkv_wkv4_forward(1, 4096, 768, 0, fake, fake, fake, fake, fake, None, None, None, 16, rw.ALGO_AUTO,
+                               None, 0, None) == 3
     # backward: bad interval, missing workspace, null gradient
     assert h.rwkv_wkv4_backward(1, 4, 4, 0, fake, fake, fake, fake, fake, None, fake, 8, fake, fake, fake,
                                 fake, fake, 1 << 20, None) == 1

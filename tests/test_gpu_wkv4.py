@@ -53,6 +53,16 @@ def test_forward_outlier_workload_full(cuda_device, algo):
     assert_state_close(st, ref_st)
 
 
+def test_forward_few_channels_long_sequence(cuda_device):
+    # 1 x 4096 x 768 (24 channel tiles): AUTO cuts time into segments; every element checked
+    p = wi.wkv4_problem(1, 4096, 768, SEED + 1, outliers=True)
+    assert rw.lib().rwkv_wkv4_forward_workspace_bytes(1, 4096, 768, rw.ALGO_AUTO) > 0
+    y, st = rw.rwkv_wkv4_forward(**_cuda(p, cuda_device), algo=rw.ALGO_AUTO, return_state=True)
+    ref, ref_st = oracle.wkv4_forward(p["w"], p["u"], p["k"], p["v"], return_state=True)
+    assert_close_abs1(y, ref, TOL_Y, "y")
+    assert_state_close(st, ref_st)
+
+
 def test_forward_single_large_outlier_slow_decay(cuda_device):
     # One +40 key at t = 1 and w = 0.01: the outlier dominates the state for
     # hundreds of steps, the case where per-step rounding of a running-max
