@@ -75,37 +75,40 @@ struct RSumm {  // a chunk's own reverse sums from a zero carry, at scale 2^q
 // scale 2^q, keeping e_t, G_t = gy_t / d_t, y_t and b_{t-1}.  gs holds the gy
 // rows, or with GATE the go rows: then gy_t = σ(r_t) go_t with r_t read from
 // rg[t * C], and gr_t is stored to grg[t * C].
-// The state recurrence, d_t and the numerator run in fp64 (lam = e^{-w}), and
-// y_t gets one correction step: gw sums 32,768 products of y-differences per
-// channel, and the fp32 recurrence's ~1e-6 error in y_t alone moved gw by up to
-// 5e-4 relative, against the 1e-4 bound.
+// The state recurrence runs in fp64 (lam = e^{-w}); d_t and the numerator are
+// formed in fp32 from it.  A large term that persists in the state (an outlier
+// key) would otherwise be re-rounded at every fp32 step: over 16 steps that
+// drift in y_t and b_t moved gw by up to 5e-4 relative, against the 1e-4 bound.
+// With GATE the chunk's r values are loaded eight steps at a time (their rows
+// were prefetched into L2 a tile ahead), which keeps the kernel in 128
+// registers without spills.
 template <typename T, bool FULL, bool GATE>
 __device__ __forceinline__ void chunk_recompute(const T* ks, const T* vs, const T* gs, const T* rg, T* grg,
                                                 int C, int cnt, float qf, float U, double lam, double a, double b,
                                                 float (&E)[kL], float (&G)[kL], float (&Y)[kL], float (&BP)[kL]) {
-  float rv[GATE ? kL : 1];
-  if constexpr (GATE) {
-#pragma unroll
-    for (int j = 0; j < kL; ++j) rv[j] = (rg != nullptr && (FULL || j < cnt)) ? IO<T>::load(rg + (size_t)j * C) : 0.f;
-  }
-  const double Ud = (double)U;
+  constexpr int kHalf = kL / 2;
+  float rv[GATE ? kHalf : 1];
 #pragma unroll
   for (int j = 0; j < kL; ++j) {
+    if constexpr (GATE) {
+      if (j % kHalf == 0) {
+#pragma unroll
+        for (int i = 0; i < kHalf; ++i)
+          rv[i] = (rg != nullptr && (FULL || j + i < cnt)) ? IO<T>::load(rg + (size_t)(j + i) * C) : 0.f;
+      }
+    }
     if (FULL || j < cnt) {
       const float e = tok_weight(IO<T>::to_f(ks[j * 32]), qf);
+      const float eu = e * U;
       const float vj = IO<T>::to_f(vs[j * 32]);
-      const double ed = (double)e;
-      const double eud = ed * Ud;
-      const double dd = b + eud;
-      const double nd = fma(eud, (double)vj, a);
-      const float d = (float)dd;
+      const float bf = (float)b;
+      const float d = bf + eu;
       const float rd = rcp_approx(d);
       const bool ok = !(d < kMinDen);  // else no history and e^{u+k} underflowed: WKV = v locally (NaN: ok)
-      const float y0 = (float)nd * rd;
-      Y[j] = ok ? fmaf((float)fma(-(double)y0, dd, nd), rd, y0) : vj;  // y0 + (n - y0 d) / d
+      Y[j] = ok ? fmaf(eu, vj, (float)a) * rd : vj;
       float gy;
       if constexpr (GATE) {
-        const float sg = sigmoid(rv[j]);
+        const float sg = sigmoid(rv[j % kHalf]);
         const float go = IO<T>::to_f(gs[j * 32]);
         gy = sg * go;
         if (grg != nullptr) grg[(size_t)j * C] = IO<T>::from_f(go * Y[j] * (sg - sg * sg));
@@ -114,9 +117,9 @@ __device__ __forceinline__ void chunk_recompute(const T* ks, const T* vs, const 
       }
       G[j] = ok ? gy * rd : 0.f;
       E[j] = e;
-      BP[j] = (float)b;  // b_{t-1}
-      a = fma(ed, (double)vj, lam * a);
-      b = fma(lam, b, ed);
+      BP[j] = bf;
+      a = fma(lam, a, (double)(e * vj));
+      b = fma(lam, b, (double)e);
     }
   }
 }
