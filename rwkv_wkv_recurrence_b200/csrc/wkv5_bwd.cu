@@ -47,6 +47,12 @@
 // chunk, whose rows past the sequence read as zero) has `lead` empty positions
 // before the carried state enters.
 //
+// Memory: q, p, c arrive as TMA boxes; the epilogue's c and m rows are fetched with 16-byte loads at
+// the top of the chunk, parked in shared memory once the first chains have released their operand
+// buffer, and the outputs leave through the same rows as 16-byte stores.  The forward pass stores
+// each checkpoint in the tf32 operand layout, so the reversed pass brings it in with one bulk copy a
+// chunk ahead.
+//
 // CTA: one (batch, head), 8 warps.  Forward pass: ~105 KB of shared memory,
 // 256 TMEM columns, two CTAs per SM.  Reversed pass: ~140 KB, 512 columns, one
 // CTA per SM.  A head with some channel decaying faster than the chunked
@@ -68,6 +74,7 @@ constexpr int kL = 64;
 constexpr int kThreads = 256;
 constexpr uint32_t kRawBytes = kL * kN * 2;
 constexpr float kMaxRate = 2.5f;
+constexpr uint32_t kCkBytes = kN * kN * 4;  // one forward-state checkpoint (fp32, operand layout)
 
 struct Wkv5BwdSmem {
   alignas(1024) __nv_bfloat16 raw[3][kL * kN];  // q, p, c boxes [position][channel] (128-byte swizzle)
@@ -81,11 +88,12 @@ struct Wkv5BwdSmem {
   alignas(8) uint64_t bar_sc;        // scores and state read (and the X_c read) done
   alignas(8) uint64_t bar_av;        // intra term (and the lag-weighted term) done
   alignas(8) uint64_t bar_ds;        // state increment done
+  alignas(8) uint64_t bar_ck;        // reversed pass: the forward state X_c has arrived in opXc
   uint32_t tmem_base;
   int slow;
   int abort_flag;
   // reversed pass only (not part of the forward pass's shared memory)
-  alignas(128) float opXc[64 * 64];  // forward state X_c [d][j]: A of the X_c read
+  alignas(128) float opXc[64 * 64];  // forward state X_c [d][j]: A of the X_c read (bulk-copied)
   alignas(128) float opAl[64 * 64];  // lag-weighted scores (τ-1-ι) A [τ][ι]: B of the lag term
   double red[kN];                    // per key row: the decay-gradient sum of this CTA
 };
@@ -94,7 +102,11 @@ size_t bwd_smem_bytes(bool rev) {
   return (rev ? sizeof(Wkv5BwdSmem) : offsetof(Wkv5BwdSmem, opXc)) + 1024;  // + alignment slack
 }
 
-__device__ __forceinline__ float bf(const __nv_bfloat16* p) { return __bfloat162float(*p); }
+// Checkpoint of forward chunk `cf` of (b, h): X_c stored in the tf32 operand layout (op_off), so
+// that the reversed pass copies it into shared memory as one contiguous block.
+__device__ __forceinline__ float* ckpt_at(const Wkv5BwdParams& p, int b, int h, int nchunk, int cf) {
+  return p.ckpt + (((size_t)b * p.H + h) * nchunk + cf) * (kN * kN);
+}
 
 template <bool REV>
 __global__ void __launch_bounds__(kThreads, REV ? 1 : 2) wkv5_bwd_tc_kernel(const __grid_constant__ CUtensorMap mq,
@@ -139,6 +151,7 @@ __global__ void __launch_bounds__(kThreads, REV ? 1 : 2) wkv5_bwd_tc_kernel(cons
     mbar_init(&sm.bar_sc, 1);
     mbar_init(&sm.bar_av, 1);
     mbar_init(&sm.bar_ds, 1);
+    mbar_init(&sm.bar_ck, 1);
     fence_mbar_init();
     mbar_arrive_expect_tx(&sm.bar_tma, 3 * kRawBytes);
     if (!withheld) {
@@ -146,6 +159,10 @@ __global__ void __launch_bounds__(kThreads, REV ? 1 : 2) wkv5_bwd_tc_kernel(cons
       tma_load_3d(sm.raw[0], &mq, &sm.bar_tma, h * kN, row0, b);
       tma_load_3d(sm.raw[1], &mp, &sm.bar_tma, h * kN, row0, b);
       tma_load_3d(sm.raw[2], &mc, &sm.bar_tma, h * kN, row0, b);
+    }
+    if constexpr (REV) {
+      mbar_arrive_expect_tx(&sm.bar_ck, kCkBytes);
+      if (!withheld) bulk_load(sm.opXc, ckpt_at(p, b, h, nchunk, nchunk - 1), kCkBytes, &sm.bar_ck);
     }
   }
 
@@ -216,6 +233,10 @@ __global__ void __launch_bounds__(kThreads, REV ? 1 : 2) wkv5_bwd_tc_kernel(cons
   const uint32_t tA = tbase, tZ = tbase + 64, tDS = tbase + 128, tCt = tbase + 192;
   const uint32_t tI = tbase + 256, tX3 = tbase + 320, tX4 = tbase + 384;  // reversed pass only
   const uint32_t rawQ = smem_u32(sm.raw[0]), rawP = smem_u32(sm.raw[1]), rawC = smem_u32(sm.raw[2]);
+  // staging rows [token][channel] bf16 of c (then out) and m, in opQ between the first chains and
+  // the next chunk's conversion
+  __nv_bfloat16* stC = reinterpret_cast<__nv_bfloat16*>(sm.opQ);
+  __nv_bfloat16* stM = stC + kL * kN;
   const bool issuer = tid == 0;
 
   int c = 0;
@@ -227,26 +248,37 @@ __global__ void __launch_bounds__(kThreads, REV ? 1 : 2) wkv5_bwd_tc_kernel(cons
     const uint32_t ph = (uint32_t)c & 1u;
     const int cf = nchunk - 1 - c;             // reversed pass: the forward chunk this one mirrors
 
+    // this chunk's box of c and m (tokens tb .. tb + 63, rows past the sequence end zero): two
+    // 16-byte loads per tensor and thread, staged in shared memory for the epilogue after the first
+    // chains have released opQ
+    const int tb = REV ? kL * cf : t0;
+    const int nrow = min(kL, p.T - tb);
+    uint4 pre[2][2];
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      const int row = 32 * hh + (tid >> 3);
+      const size_t off = (((size_t)b * p.T + tb + row) * p.H + h) * kN + 8 * (tid & 7);
+      const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+      pre[0][hh] = row < nrow ? __ldg(reinterpret_cast<const uint4*>(p.c + off)) : z;
+      pre[1][hh] = row < nrow ? __ldg(reinterpret_cast<const uint4*>(p.m + off)) : z;
+    }
+
     // forward pass: the state at this chunk's start is the checkpoint the reversed pass reads
     if constexpr (!REV) {
-      float* ck = p.ckpt + ((((size_t)b * p.H + h) * nchunk + c) * kN) * kN;
+      float* ck = ckpt_at(p, b, h, nchunk, c);
 #pragma unroll
       for (int q = 0; q < 8; ++q)
 #pragma unroll
-        for (int r = 0; r < 2; ++r) ck[(size_t)(drow + 8 * r) * kN + jcol + 4 * q] = X[2 * q + r];
+        for (int r = 0; r < 2; ++r) ck[op_off(drow + 8 * r, jcol + 4 * q)] = X[2 * q + r];
     } else {
-      // X_c (the forward state at the mirrored chunk's start) into opXc, and the elementwise term
-      // n w^{n-1} Σ_j G∘X_c with n = 64 - lo positions in the chunk
-      const float* ck = p.ckpt + ((((size_t)b * p.H + h) * nchunk + cf) * kN) * kN;
+      // X_c (the forward state at the mirrored chunk's start, copied into opXc) and the elementwise
+      // term n w^{n-1} Σ_j G∘X_c with n = 64 - lo positions in the chunk
+      if (!mbar_wait_bounded(&sm.bar_ck, ph, p.ctl)) sm.abort_flag = 1;
       float part[2] = {0.f, 0.f};
 #pragma unroll
       for (int q = 0; q < 8; ++q)
 #pragma unroll
-        for (int r = 0; r < 2; ++r) {
-          const float xc = ck[(size_t)(drow + 8 * r) * kN + jcol + 4 * q];
-          sm.opXc[op_off(drow + 8 * r, jcol + 4 * q)] = xc;
-          part[r] = fmaf(X[2 * q + r], xc, part[r]);
-        }
+        for (int r = 0; r < 2; ++r) part[r] = fmaf(X[2 * q + r], sm.opXc[op_off(drow + 8 * r, jcol + 4 * q)], part[r]);
       const float n = (float)(kL - lo);
 #pragma unroll
       for (int r = 0; r < 2; ++r) acc_t1[r] += (double)(n * expf((n - 1.f) * lamr[r]) * part[r]);
@@ -338,6 +370,21 @@ __global__ void __launch_bounds__(kThreads, REV ? 1 : 2) wkv5_bwd_tc_kernel(cons
     // q_τ·p_τ -> diag.  .16x128b fragment: rows τ = 16 q4 + t4 + 8 r, columns ι = 32 hc + 4 q + tq
     if (!mbar_wait_bounded(&sm.bar_sc, ph, p.ctl)) sm.abort_flag = 1;
     tc_fence_after();
+    // the first chains have read opQ, opP and opXc: c and m into the staging rows (opQ), and
+    // (reversed) the next chunk's checkpoint into opXc
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      const int row = 32 * hh + (tid >> 3);
+      *reinterpret_cast<uint4*>(&stC[row * kN + 8 * (tid & 7)]) = pre[0][hh];
+      *reinterpret_cast<uint4*>(&stM[row * kN + 8 * (tid & 7)]) = pre[1][hh];
+    }
+    if constexpr (REV) {
+      if (issuer && c + 1 < nchunk) {
+        fence_proxy_async();
+        mbar_arrive_expect_tx(&sm.bar_ck, kCkBytes);
+        bulk_load(sm.opXc, ckpt_at(p, b, h, nchunk, cf - 1), kCkBytes, &sm.bar_ck);
+      }
+    }
     {
       const int tau0 = 16 * q4 + t4;
       if (hc > (q4 >> 1)) {  // strictly above the diagonal
@@ -401,22 +448,21 @@ __global__ void __launch_bounds__(kThreads, REV ? 1 : 2) wkv5_bwd_tc_kernel(cons
         tmem_ld32x16(tX4 + tquar + col, x4);
       }
       if (lane < 16) {
-        const size_t row0 = ((size_t)b * p.T) * p.H + h;  // (row0 + position * H) * 64 + channel
         float acc = 0.f;
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const int pos = (int)col + i;
           if (pos < lo || pos >= cnt) continue;
-          const int t = REV ? kL * cf + (kL - 1 - pos) : t0 + pos;  // token of this position
-          const size_t off = ((row0 + (size_t)t * p.H) * kN) + de;
-          const float cval = bf(p.c + off), mval = bf(p.m + off);
+          // staging row of this position (the box holds the tokens in forward order); out replaces c
+          const int so = (REV ? kL - 1 - pos : pos) * kN + de;
+          const float cval = __bfloat162float(stC[so]), mval = __bfloat162float(stM[so]);
           const float dg = sm.diag[pos];
           const float f = __expf(lam_e * (float)(pos - 32));
           float o;
           if constexpr (REV) o = f * (zv[i] + iv[i]);
           else o = f * zv[i];
           o = fmaf(u_e * cval, dg, o);
-          p.out[off] = __float2bfloat16_rn(o);
+          stC[so] = __float2bfloat16_rn(o);
           if constexpr (REV) {
             // position-weighted state read, lag-weighted intra term, and the X_c read
             const float f1 = __expf(lam_e * (float)(pos - 33));
@@ -429,6 +475,15 @@ __global__ void __launch_bounds__(kThreads, REV ? 1 : 2) wkv5_bwd_tc_kernel(cons
         }
         acc_e += (double)acc;
       }
+    }
+    // the chunk's out rows, 16 bytes a thread
+    __syncthreads();
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      const int row = 32 * hh + (tid >> 3);
+      if (row < nrow)
+        *reinterpret_cast<uint4*>(p.out + (((size_t)b * p.T + tb + row) * p.H + h) * kN + 8 * (tid & 7)) =
+            *reinterpret_cast<const uint4*>(&stC[row * kN + 8 * (tid & 7)]);
     }
 
     // T2b: X <- e^{nλ} X + e^{32λ} (c̃ᵀ p) with n the positions since the state entered
@@ -458,13 +513,17 @@ __global__ void __launch_bounds__(kThreads, REV ? 1 : 2) wkv5_bwd_tc_kernel(cons
         }
       }
     }
+    __syncthreads();  // the staging rows (opQ) are read out before the next chunk converts q into it
   }
 
   if (aborted && tid == 0) {
     // a wait gave up at chunk c: the last MMA chains and this chunk's loads must finish before the
     // tensor memory and shared memory are released, each wait bounded again
     if (c >= 1) mbar_wait_bounded(&sm.bar_ds, (uint32_t)(c - 1) & 1u, p.ctl);
-    if (!withheld) mbar_wait_bounded(&sm.bar_tma, (uint32_t)c & 1u, p.ctl);
+    if (!withheld) {
+      mbar_wait_bounded(&sm.bar_tma, (uint32_t)c & 1u, p.ctl);
+      if constexpr (REV) mbar_wait_bounded(&sm.bar_ck, (uint32_t)c & 1u, p.ctl);  // checkpoint copy c
+    }
   }
   // per-row sums of the CTA: forward gu parts, reversed decay-gradient parts
   double* part = p.part + ((size_t)b * p.H + h) * kN;
