@@ -632,6 +632,43 @@ size_t rwkv_wkv5_backward_workspace_bytes(int64_t B, int64_t T, int64_t H, int64
   return wkv5_bwd_ws(B, T, H).total;
 }
 
+}  // extern "C"
+
+namespace rwkv {
+namespace {
+// One non-blocking stream per (device, context), made on first use: the Eagle backward runs its
+// reversed forward pass there, next to the reversed gradient pass (whose last CTAs leave most SMs
+// idle).  Each call orders it against the caller's stream with its own pair of events.  Returns
+// nullptr (run everything on the caller's stream) when no stream can be had: no context id, the
+// caller's stream is being captured before the side stream exists, or a CUDA error.
+cudaStream_t side_stream(cudaStream_t caller) {
+  constexpr int kMaxDev = 64;
+  struct Slot {
+    cudaStream_t s;
+    unsigned long long ctx;
+  };
+  static std::mutex mu;
+  static Slot slots[kMaxDev] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return nullptr;
+  const unsigned long long id = current_context_id();
+  if (id == 0) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  Slot& sl = slots[dev];
+  if (sl.s != nullptr && sl.ctx == id) return sl.s;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(caller, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone) return nullptr;
+  cudaStream_t s = nullptr;
+  if (cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking) != cudaSuccess) return nullptr;
+  sl.s = s;
+  sl.ctx = id;
+  return s;
+}
+}  // namespace
+}  // namespace rwkv
+
+extern "C" {
+
 rwkv_status rwkv_wkv5_backward(int64_t B, int64_t T, int64_t H, int64_t N, const void* r, const void* k,
                                const void* v, const float* omega, const float* u, const float* s_in, const void* gy,
                                const float* gs_out, void* gr, void* gk, void* gv, float* gomega, float* gu,
@@ -673,24 +710,6 @@ rwkv_status rwkv_wkv5_backward(int64_t B, int64_t T, int64_t H, int64_t N, const
       !make_bf16_box64_map(&mv, v, iB, iT, W) || !make_bf16_box64_map(&mg, gy, iB, iT, W))
     return RWKV_ERR_CUDA;
 
-  // gv and the initial-state gradient: the forward operator over reversed time with r and k
-  // swapped and gy as the value, started from gs_out (time reversed inside the kernel)
-  {
-    Wkv5Params p{};
-    p.B = iB;
-    p.T = iT;
-    p.H = iH;
-    p.r = static_cast<const __nv_bfloat16*>(k);
-    p.k = static_cast<const __nv_bfloat16*>(r);
-    p.v = static_cast<const __nv_bfloat16*>(gy);
-    p.omega = omega;
-    p.u = u;
-    p.y = static_cast<__nv_bfloat16*>(gv);
-    p.s_in = gs_out;
-    p.s_out = gs_in;
-    p.ctl = ctl;
-    if (launch_wkv5_fwd(mk, mr, mg, p, st, true) != cudaSuccess) return RWKV_ERR_CUDA;
-  }
   const int nchunk = (iT + 63) / 64;
   // gr, the forward states at chunk starts, the gu sums: (q, p, c, m) = (gy, v, k, r)
   {
@@ -710,6 +729,23 @@ rwkv_status rwkv_wkv5_backward(int64_t B, int64_t T, int64_t H, int64_t N, const
     p.ctl = ctl;
     if (launch_wkv5_bwd_pass(false, mg, mv, mk, p, st) != cudaSuccess) return RWKV_ERR_CUDA;
   }
+  // the reversed forward pass below needs nothing from the two gradient passes: it runs on a side
+  // stream, ordered after the forward-time pass so that the reversed pass is dispatched first
+  cudaStream_t side = side_stream(st);
+  cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
+  if (side != nullptr) {
+    if (cudaEventCreateWithFlags(&ev_fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&ev_join, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventRecord(ev_fork, st) != cudaSuccess || cudaStreamWaitEvent(side, ev_fork, 0) != cudaSuccess) {
+      if (ev_fork) cudaEventDestroy(ev_fork);
+      if (ev_join) cudaEventDestroy(ev_join);
+      return RWKV_ERR_CUDA;
+    }
+  }
+  auto release = [&]() {
+    if (ev_fork) cudaEventDestroy(ev_fork);
+    if (ev_join) cudaEventDestroy(ev_join);
+  };
   // gk and the decay-gradient sums: (q, p, c, m) = (v, gy, r, k) over reversed time, chunks aligned
   // with the forward pass's
   {
@@ -727,8 +763,39 @@ rwkv_status rwkv_wkv5_backward(int64_t B, int64_t T, int64_t H, int64_t N, const
     p.ckpt = ckpt;
     p.part = part_r;
     p.ctl = ctl;
-    if (launch_wkv5_bwd_pass(true, mv, mg, mr, p, st) != cudaSuccess) return RWKV_ERR_CUDA;
+    if (launch_wkv5_bwd_pass(true, mv, mg, mr, p, st) != cudaSuccess) {
+      release();
+      return RWKV_ERR_CUDA;
+    }
   }
+  // gv and the initial-state gradient: the forward operator over reversed time with r and k
+  // swapped and gy as the value, started from gs_out (time reversed inside the kernel)
+  {
+    Wkv5Params p{};
+    p.B = iB;
+    p.T = iT;
+    p.H = iH;
+    p.r = static_cast<const __nv_bfloat16*>(k);
+    p.k = static_cast<const __nv_bfloat16*>(r);
+    p.v = static_cast<const __nv_bfloat16*>(gy);
+    p.omega = omega;
+    p.u = u;
+    p.y = static_cast<__nv_bfloat16*>(gv);
+    p.s_in = gs_out;
+    p.s_out = gs_in;
+    p.ctl = ctl;
+    if (launch_wkv5_fwd(mk, mr, mg, p, side != nullptr ? side : st, true) != cudaSuccess) {
+      release();
+      return RWKV_ERR_CUDA;
+    }
+  }
+  if (side != nullptr) {
+    if (cudaEventRecord(ev_join, side) != cudaSuccess || cudaStreamWaitEvent(st, ev_join, 0) != cudaSuccess) {
+      release();
+      return RWKV_ERR_CUDA;
+    }
+  }
+  release();
   if (launch_wkv5_bwd_reduce(iB, iH, part_f, part_r, omega, gomega, gu, st) != cudaSuccess) return RWKV_ERR_CUDA;
   return RWKV_OK;
 }

@@ -168,4 +168,7 @@ DevCtl* device_ctl();
 // Sets the dynamic shared-memory limit of `func` once per device.
 cudaError_t ensure_smem_attr(const void* func, int bytes, unsigned* device_mask);
 
+// Unique id of the context current on this thread; 0 if there is none or the driver cannot say.
+unsigned long long current_context_id();
+
 }  // namespace rwkv

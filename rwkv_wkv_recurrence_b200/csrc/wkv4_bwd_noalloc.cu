@@ -30,14 +30,6 @@
 #include "launch.h"
 
 namespace rwkv {
-namespace {
-
-constexpr int64_t kNoAllocMaxLanes = RWKV_NOALLOC_MAX_LANES;
-constexpr int kMaxDevices = 64;
-
-// Per-lane gw, gu partial sums of the backward: [2][kNoAllocMaxLanes] fp64.
-static __device__ __align__(256) double g_bwd_scratch[2 * kNoAllocMaxLanes];
-
 using CtxGetCurrentFn = CUresult (*)(CUcontext*);
 using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
 
@@ -64,6 +56,14 @@ unsigned long long current_context_id() {
   if (get_id(ctx, &id) != CUDA_SUCCESS) return 0;
   return id;
 }
+
+namespace {
+
+constexpr int64_t kNoAllocMaxLanes = RWKV_NOALLOC_MAX_LANES;
+constexpr int kMaxDevices = 64;
+
+// Per-lane gw, gu partial sums of the backward: [2][kNoAllocMaxLanes] fp64.
+static __device__ __align__(256) double g_bwd_scratch[2 * kNoAllocMaxLanes];
 
 struct ScratchAddr {
   unsigned long long ctx_id;  // context the address belongs to (0: none yet)

@@ -355,6 +355,10 @@ __global__ void __launch_bounds__(kThreads, REV ? 1 : 2) wkv5_bwd_tc_kernel(cons
     __syncthreads();
     if (issuer) {
       tc_fence_after();
+      // state increment c̃ᵀ p [d][j]: needs only this chunk's operands, runs while the scores are masked
+#pragma unroll
+      for (int s = 0; s < 8; ++s) umma_tf32_ts(tDS, tCt + 8 * s, smem_desc(&sm.opPt[s * 64], kLbo, kSbo), kIdesc, s);
+      umma_commit(&sm.bar_ds);
       // the raw boxes are consumed: load the next chunk while this one computes
       if (c + 1 < nchunk) {
         fence_proxy_async();
@@ -427,12 +431,35 @@ __global__ void __launch_bounds__(kThreads, REV ? 1 : 2) wkv5_bwd_tc_kernel(cons
         }
       }
       umma_commit(&sm.bar_av);
-      // state increment c̃ᵀ p [d][j]
-#pragma unroll
-      for (int s = 0; s < 8; ++s) umma_tf32_ts(tDS, tCt + 8 * s, smem_desc(&sm.opPt[s * 64], kLbo, kSbo), kIdesc, s);
-      umma_commit(&sm.bar_ds);
     }
 
+    // T2b: X <- e^{nλ} X + e^{32λ} (c̃ᵀ p) with n the positions since the state entered
+    // (64 - lead in the first reversed chunk), or the partial last chunk's own form
+    if (!mbar_wait_bounded(&sm.bar_ds, ph, p.ctl)) sm.abort_flag = 1;
+    tc_fence_after();
+    {
+      float ds[16];
+      tmem_ld16x128(tDS + tquar + (uint32_t)(32 * hc), ds);
+      if (cnt == kL) {
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          const float gx = lo == 0 ? e32[r] * e32[r] : expf((float)(kL - lo) * lamr[r]);
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const int x = 2 * q + r;
+            X[x] = fmaf(gx, X[x], e32[r] * ds[x]);
+            sm.opX[op_off(drow + 8 * r, jcol + 4 * q)] = e32[r] * X[x];
+          }
+        }
+      } else {  // partial last chunk (forward pass): no later chunk reads opX
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          const float dl = expf(lamr[r] * (float)cnt), gs = expf(lamr[r] * (float)(cnt - 32));
+#pragma unroll
+          for (int q = 0; q < 8; ++q) X[2 * q + r] = fmaf(dl, X[2 * q + r], gs * ds[2 * q + r]);
+        }
+      }
+    }
     // T3: out[τ][de] = e^{λ(τ-32)} (state read + intra)[de][τ] + u c_τ A[τ][τ], and the sums; 16
     // positions at a time (lanes 0..15 of each quarter hold the rows of the M = 64 accumulators)
     if (!mbar_wait_bounded(&sm.bar_av, ph, p.ctl)) sm.abort_flag = 1;
@@ -486,40 +513,13 @@ __global__ void __launch_bounds__(kThreads, REV ? 1 : 2) wkv5_bwd_tc_kernel(cons
             *reinterpret_cast<const uint4*>(&stC[row * kN + 8 * (tid & 7)]);
     }
 
-    // T2b: X <- e^{nλ} X + e^{32λ} (c̃ᵀ p) with n the positions since the state entered
-    // (64 - lead in the first reversed chunk), or the partial last chunk's own form
-    if (!mbar_wait_bounded(&sm.bar_ds, ph, p.ctl)) sm.abort_flag = 1;
-    tc_fence_after();
-    {
-      float ds[16];
-      tmem_ld16x128(tDS + tquar + (uint32_t)(32 * hc), ds);
-      if (cnt == kL) {
-#pragma unroll
-        for (int r = 0; r < 2; ++r) {
-          const float gx = lo == 0 ? e32[r] * e32[r] : expf((float)(kL - lo) * lamr[r]);
-#pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            const int x = 2 * q + r;
-            X[x] = fmaf(gx, X[x], e32[r] * ds[x]);
-            sm.opX[op_off(drow + 8 * r, jcol + 4 * q)] = e32[r] * X[x];
-          }
-        }
-      } else {  // partial last chunk (forward pass): no later chunk reads opX
-#pragma unroll
-        for (int r = 0; r < 2; ++r) {
-          const float dl = expf(lamr[r] * (float)cnt), gs = expf(lamr[r] * (float)(cnt - 32));
-#pragma unroll
-          for (int q = 0; q < 8; ++q) X[2 * q + r] = fmaf(dl, X[2 * q + r], gs * ds[2 * q + r]);
-        }
-      }
-    }
     __syncthreads();  // the staging rows (opQ) are read out before the next chunk converts q into it
   }
 
   if (aborted && tid == 0) {
     // a wait gave up at chunk c: the last MMA chains and this chunk's loads must finish before the
     // tensor memory and shared memory are released, each wait bounded again
-    if (c >= 1) mbar_wait_bounded(&sm.bar_ds, (uint32_t)(c - 1) & 1u, p.ctl);
+    if (c >= 1) mbar_wait_bounded(&sm.bar_av, (uint32_t)(c - 1) & 1u, p.ctl);  // the last chains of c-1
     if (!withheld) {
       mbar_wait_bounded(&sm.bar_tma, (uint32_t)c & 1u, p.ctl);
       if constexpr (REV) mbar_wait_bounded(&sm.bar_ck, (uint32_t)c & 1u, p.ctl);  // checkpoint copy c

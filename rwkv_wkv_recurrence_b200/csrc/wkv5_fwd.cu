@@ -19,8 +19,11 @@
 // memory) run three chains of eight K = 8 steps:
 //   [A | Y] = r̃ [k̃ ; e^{32λ} Sᵀ]ᵀ          M = 64, N = 128: scores [τ][ι] and the
 //                                           inter-chunk read [τ][j] share operand r̃
-//   Y      += A_masked vᵀᵀ                 M = 64, N = 64 (intra-chunk term)
 //   ΔS      = k̃ᵀ vᵀᵀ                       M = 64, N = 64, k̃ᵀ read from tensor memory
+//   Y      += A_masked vᵀᵀ                 M = 64, N = 64 (intra-chunk term), the masked scores
+//                                           read in place from tensor memory
+// ΔS needs only the chunk's own operands, so it is issued as soon as they exist
+// and runs while the scores are masked; the state fold then overlaps A v.
 // with r̃ = r e^{λ(τ-32)}, k̃ = k e^{λ(31-ι)}, so that r̃·k̃ = r e^{λ(τ-1-ι)} k and
 // e^{32λ} (r̃ S) = r e^{λτ} S; the state increment is scaled by e^{λ(cnt-32)} per
 // key channel when it is folded into the fp32 master state, which lives in
@@ -38,7 +41,7 @@
 // the data allows (N = 128 for the first chain) and the issuing thread hands
 // the first chain out in pairs between the other work of its warp.
 //
-// CTA: one (batch, head), 8 warps, about 106 KB of shared memory and 256 TMEM
+// CTA: one (batch, head), 8 warps, about 90 KB of shared memory and 256 TMEM
 // columns, two CTAs per SM.  Thread 0 issues the TMA loads of the raw r, k, v
 // tiles (one [64 tokens x 64] bf16 box each, 128-byte swizzle, no multicast)
 // and the MMAs; all warps build operands, mask the scores, fold the state and
@@ -109,7 +112,6 @@ struct Wkv5Smem {
   alignas(128) float opK[64 * 64];   // k̃ = k e^{λ(31-ι)}   [ι][d]: B rows 0..63 of the first product
   alignas(128) float opS[64 * 64];   // e^{32λ} ⊙ Sᵀ         [j][d]: B rows 64..127 of the first product
   alignas(128) float opVt[64 * 64];  // vᵀ                   [j][ι]: B of A v and of the state increment
-  alignas(128) float opA[64 * 64];   // masked scores       [τ][ι]: A of A v
   float diag_part[8][kL];            // per-warp parts of Σ_d r u k (the bonus term)
   float diag[kL];                    // Σ_d r u k per token
   alignas(8) uint64_t bar_tma;
@@ -343,6 +345,10 @@ __global__ void __launch_bounds__(kThreads, 2) wkv5_fwd_tc_kernel(const __grid_c
     __syncthreads();
     if (issuer) {
       tc_fence_after();
+      // ΔS = k̃ᵀ v [d][j] needs only this chunk's operands: it runs while the scores are masked
+#pragma unroll
+      for (int s = 0; s < 8; ++s) umma_tf32_ts(tDS, tKt + 8 * s, smem_desc(&sm.opVt[s * 64], kLbo, kSbo), kIdesc, s);
+      umma_commit(&sm.bar_ds);
       // the raw boxes are consumed: load the next chunk while this one computes
       if (c + 1 < nchunk) {
         fence_proxy_async();
@@ -354,17 +360,18 @@ __global__ void __launch_bounds__(kThreads, 2) wkv5_fwd_tc_kernel(const __grid_c
       }
     }
 
-    // T2a: causal mask of the scores (ι < τ kept, ι = τ the bonus Σ_d r u k, ι > τ zero) -> opA.
+    // T2a: causal mask of the scores in tensor memory, in place (ι < τ kept, ι = τ the bonus
+    // Σ_d r u k, ι > τ zero): the A operand of A v.
     // .16x128b fragment: rows τ = 16 q4 + t4 + 8 r, columns ι = 32 hc + 4 q + tq  ->  register 2 q + r
     if (!mbar_wait_bounded(&sm.bar_sc, ph, p.ctl)) sm.abort_flag = 1;
     tc_fence_after();
     {
       const int tau0 = 16 * q4 + t4;
       if (hc > (q4 >> 1)) {  // strictly above the diagonal
+        float a[16];
 #pragma unroll
-        for (int q = 0; q < 8; ++q)
-#pragma unroll
-          for (int r = 0; r < 2; ++r) sm.opA[op_off(tau0 + 8 * r, 32 * hc + 4 * q + tq)] = 0.f;
+        for (int i = 0; i < 16; ++i) a[i] = 0.f;
+        tmem_st16x128(tSc + tquar + (uint32_t)(32 * hc), a);
       } else {
         float a[16];
         tmem_ld16x128(tSc + tquar + (uint32_t)(32 * hc), a);
@@ -378,48 +385,23 @@ __global__ void __launch_bounds__(kThreads, 2) wkv5_fwd_tc_kernel(const __grid_c
 #pragma unroll
           for (int r = 0; r < 2; ++r) {
             const int io = 32 * hc + 4 * q + tq, tau = tau0 + 8 * r;
-            sm.opA[op_off(tau, io)] = io < tau ? a[2 * q + r] : (io == tau ? dg[r] : 0.f);
+            a[2 * q + r] = io < tau ? a[2 * q + r] : (io == tau ? dg[r] : 0.f);
           }
+        tmem_st16x128(tSc + tquar + (uint32_t)(32 * hc), a);
       }
     }
-    fence_proxy_async();
     tc_fence_before();
     __syncthreads();
     if (issuer) {
       tc_fence_after();
-      // Y += (masked scores) v
+      // Y += (masked scores) v, the scores read from tensor memory
 #pragma unroll
-      for (int s = 0; s < 8; ++s)
-        umma_tf32(tY, smem_desc(&sm.opA[s * 64], kLbo, kSbo), smem_desc(&sm.opVt[s * 64], kLbo, kSbo), kIdesc, 1);
+      for (int s = 0; s < 8; ++s) umma_tf32_ts(tY, tSc + 8 * s, smem_desc(&sm.opVt[s * 64], kLbo, kSbo), kIdesc, 1);
       umma_commit(&sm.bar_av);
-      // ΔS = k̃ᵀ v [d][j], k̃ᵀ read from tensor memory
-#pragma unroll
-      for (int s = 0; s < 8; ++s) umma_tf32_ts(tDS, tKt + 8 * s, smem_desc(&sm.opVt[s * 64], kLbo, kSbo), kIdesc, s);
-      umma_commit(&sm.bar_ds);
     }
 
-    // T3: Y rows -> bf16 -> global (TMEM lanes 0..15 of each quarter hold the rows)
-    if (!mbar_wait_bounded(&sm.bar_av, ph, p.ctl)) sm.abort_flag = 1;
-    tc_fence_after();
-    {
-      float yv[32];
-      tmem_ld32(tY + tquar + (uint32_t)(32 * hc), yv);
-      const int tau = 16 * q4 + lane;
-      if (lane < 16 && tau < cnt) {
-        const int ty = REV ? p.T - 1 - (t0 + tau) : t0 + tau;
-        __nv_bfloat16* yp = p.y + (((size_t)b * p.T + ty) * p.H + h) * kN + 32 * hc;
-#pragma unroll
-        for (int j = 0; j < 32; j += 8) {
-          uint4 pk;
-          __nv_bfloat162* q2 = reinterpret_cast<__nv_bfloat162*>(&pk);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) q2[e] = __floats2bfloat162_rn(yv[j + 2 * e], yv[j + 2 * e + 1]);
-          *reinterpret_cast<uint4*>(yp + j) = pk;
-        }
-      }
-    }
-
-    // T2b: S <- e^{cnt λ} S + e^{(cnt-32) λ} ΔS; e^{32λ} Sᵀ into opS for the next chunk
+    // T2b: S <- e^{cnt λ} S + e^{(cnt-32) λ} ΔS; e^{32λ} Sᵀ into opS for the next chunk (while A v
+    // still runs)
     if (!mbar_wait_bounded(&sm.bar_ds, ph, p.ctl)) sm.abort_flag = 1;
     tc_fence_after();
     {
@@ -445,13 +427,34 @@ __global__ void __launch_bounds__(kThreads, 2) wkv5_fwd_tc_kernel(const __grid_c
         }
       }
     }
+
+    // T3: Y rows -> bf16 -> global (TMEM lanes 0..15 of each quarter hold the rows)
+    if (!mbar_wait_bounded(&sm.bar_av, ph, p.ctl)) sm.abort_flag = 1;
+    tc_fence_after();
+    {
+      float yv[32];
+      tmem_ld32(tY + tquar + (uint32_t)(32 * hc), yv);
+      const int tau = 16 * q4 + lane;
+      if (lane < 16 && tau < cnt) {
+        const int ty = REV ? p.T - 1 - (t0 + tau) : t0 + tau;
+        __nv_bfloat16* yp = p.y + (((size_t)b * p.T + ty) * p.H + h) * kN + 32 * hc;
+#pragma unroll
+        for (int j = 0; j < 32; j += 8) {
+          uint4 pk;
+          __nv_bfloat162* q2 = reinterpret_cast<__nv_bfloat162*>(&pk);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) q2[e] = __floats2bfloat162_rn(yv[j + 2 * e], yv[j + 2 * e + 1]);
+          *reinterpret_cast<uint4*>(yp + j) = pk;
+        }
+      }
+    }
   }
 
   if (aborted && tid == 0) {
-    // a wait gave up at chunk c: the previous chunk's MMA chains (committed last on bar_ds) and
+    // a wait gave up at chunk c: the previous chunk's MMA chains (committed last on bar_av) and
     // this chunk's loads must finish before the tensor memory and shared memory are released,
     // each wait bounded again
-    if (c >= 1) mbar_wait_bounded(&sm.bar_ds, (uint32_t)(c - 1) & 1u, p.ctl);
+    if (c >= 1) mbar_wait_bounded(&sm.bar_av, (uint32_t)(c - 1) & 1u, p.ctl);
     if (!withheld) mbar_wait_bounded(&sm.bar_tma, (uint32_t)c & 1u, p.ctl);
   }
   if (p.s_out != nullptr) {
