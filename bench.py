@@ -709,6 +709,13 @@ def run_chunked(args):
         "schedules": res, "gpu_launches": 3 if picked == "chunked" else 1, "clocks": clk_all}), flush=True)
 
 
+def _omega_range(args):
+    lo, hi = (float(x) for x in args.omega_range.split(","))
+    if not lo < hi:
+        raise SystemExit("--omega-range wants LO,HI with LO < HI")
+    return lo, hi
+
+
 def run_eagle(args, finch=False):
     """Eagle / RWKV-5 forward, B4 T4096 H40 N64 bf16, zero initial state; with
     finch, the Finch / RWKV-6 forward on the same shape with a per-token fp32
@@ -723,7 +730,8 @@ def run_eagle(args, finch=False):
     dev = torch.device("cuda", local)
     Be, Te, He, Ne = 4, 4096, 40, 64
     gen = wi.wkv6_problem if finch else wi.wkv5_problem
-    q = gen(Be, Te, He, Ne, seed=SEED + (4 if finch else 2), device=dev)
+    om_lo, om_hi = _omega_range(args)
+    q = gen(Be, Te, He, Ne, seed=SEED + (4 if finch else 2), device=dev, omega_range=(om_lo, om_hi))
     y = torch.empty_like(q["r"])
     s_out = torch.empty(Be, He, Ne, Ne, device=dev)
     h = rw.lib()
@@ -751,12 +759,13 @@ def run_eagle(args, finch=False):
     if finch:
         metric = "Finch WKV forward elements/s and HBM GB/s (B4 T4096 H40 N64, per-token decay)"
         workload = ("Finch / RWKV-6 WKV forward, B=4 T=4096 H=40 N=64, bf16 r,k,v,y, fp32 per-token omega "
-                    "(U(-6,0) per channel + 0.5 N(0,1) per token), fp32 state")
+                    f"(U({om_lo:g},{om_hi:g}) per channel + 0.5 N(0,1) per token), fp32 state")
         l2 = "no flush: 506 MB moved per call, above the 126 MB L2"
         kernel = "wkv6_fwd_tc_kernel"
     else:
         metric = "Eagle WKV forward elements/s and HBM GB/s (B4 T4096 H40 N64)"
-        workload = "Eagle / RWKV-5 WKV forward, B=4 T=4096 H=40 N=64, bf16 r,k,v,y, fp32 state"
+        workload = ("Eagle / RWKV-5 WKV forward, B=4 T=4096 H=40 N=64, bf16 r,k,v,y, fp32 state"
+                    + ("" if (om_lo, om_hi) == (-6.0, 0.0) else f", omega U({om_lo:g},{om_hi:g})"))
         l2 = "no flush: 338 MB moved per call, above the 126 MB L2"
         kernel = "wkv5_fwd_tc_kernel"
     print(json.dumps({
@@ -886,6 +895,8 @@ def main():
     ap.add_argument("--chunked-shape", choices=["8x1024x768", "1x4096x768"], default="8x1024x768",
                     help="the few-channel forward's shape (chunked workload)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--omega-range", default="-6,0",
+                    help="eagle / finch workloads: the per-channel omega range U(LO,HI) (w = exp(-exp(omega)))")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--ref-channels", type=int, default=256)
     ap.add_argument("--traffic", type=float, default=None,

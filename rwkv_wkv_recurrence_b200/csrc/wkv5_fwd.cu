@@ -30,8 +30,8 @@
 // registers (S' = e^{cnt λ} S + e^{(cnt-32) λ} ΔS), so the state is never
 // rounded below fp32.  Splitting e^{λ(τ-1-ι)} around the chunk middle keeps
 // every factor within e^{±32|λ|}; a head with -λ > 2.5 in any channel
-// (w < 0.082) would leave the fp32 range there and is computed by the
-// recurrence instead.
+// (w < 0.082) would leave the fp32 range there: its chunks run token by token
+// on the CUDA cores instead (chunk_recur), with the same TMA boxes and state.
 //
 // The tensor core takes tf32 operands K-major only, so the operand tiles are
 // fp32 [rows][64] in the K-major core-matrix layout without swizzle (8 rows x
@@ -51,6 +51,7 @@
 #include "launch.h"
 #include "tc_common.cuh"
 #include "wkv_common.cuh"
+#include "wkv_recur.cuh"
 
 namespace rwkv {
 namespace {
@@ -64,48 +65,6 @@ constexpr uint32_t kRawBytes = kL * kN * 2;    // one bf16 [64 x 64] box
 constexpr float kMaxRate = 2.5f;       // largest -λ the chunked factorization accepts
 constexpr uint32_t kTmemCols = 256;  // [scores | output rows], state increment, k̃ᵀ (64 columns each)
 
-// The recurrence for one head (used when a channel decays too fast for the
-// chunked factorization): thread j < 64 owns value column j of the state.
-// With rev, step t reads and writes token T-1-t (the operator over reversed time).
-__device__ __noinline__ void head_recurrent(int b, int h, int T, int H, const __nv_bfloat16* __restrict__ r,
-                               const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
-                               const float* wdec, const float* ud, __nv_bfloat16* __restrict__ y,
-                               const float* s_in, float* s_out, float* sm_r, float* sm_k, bool rev) {
-  const int j = threadIdx.x;
-  const size_t sbase = ((size_t)b * H + h) * kN * kN;
-  float s[kN];
-  if (j < kN) {
-#pragma unroll
-    for (int i = 0; i < kN; ++i) s[i] = s_in ? s_in[sbase + (size_t)i * kN + j] : 0.f;
-  }
-  for (int t = 0; t < T; ++t) {
-    const size_t off = (((size_t)b * T + (rev ? T - 1 - t : t)) * H + h) * kN;
-    __syncthreads();
-    if (j < kN) {
-      sm_r[j] = __bfloat162float(r[off + j]);
-      sm_k[j] = __bfloat162float(k[off + j]);
-    }
-    __syncthreads();
-    if (j < kN) {
-      const float vj = __bfloat162float(v[off + j]);
-      float bonus = 0.f, acc = 0.f;
-#pragma unroll
-      for (int i = 0; i < kN; ++i) {
-        bonus = fmaf(sm_r[i] * ud[i], sm_k[i], bonus);
-        acc = fmaf(sm_r[i], s[i], acc);
-      }
-      acc = fmaf(bonus, vj, acc);
-#pragma unroll
-      for (int i = 0; i < kN; ++i) s[i] = fmaf(wdec[i], s[i], sm_k[i] * vj);
-      y[off + j] = __float2bfloat16_rn(acc);
-    }
-  }
-  if (s_out != nullptr && j < kN) {
-#pragma unroll
-    for (int i = 0; i < kN; ++i) s_out[sbase + (size_t)i * kN + j] = s[i];
-  }
-}
-
 struct Wkv5Smem {
   alignas(1024) __nv_bfloat16 raw[3][kL * kN];  // r, k, v boxes [token][channel] (128-byte swizzle)
   alignas(128) float opR[64 * 64];   // r̃ = r e^{λ(τ-32)}   [τ][d]: A of the scores and of the state read
@@ -114,6 +73,7 @@ struct Wkv5Smem {
   alignas(128) float opVt[64 * 64];  // vᵀ                   [j][ι]: B of A v and of the state increment
   float diag_part[8][kL];            // per-warp parts of Σ_d r u k (the bonus term)
   float diag[kL];                    // Σ_d r u k per token
+  float wdec[kN];                    // w per key channel (heads on the recurrent path)
   alignas(8) uint64_t bar_tma;
   alignas(8) uint64_t bar_sc;        // scores and state read done
   alignas(8) uint64_t bar_av;        // A v done
@@ -122,6 +82,9 @@ struct Wkv5Smem {
   int slow;
   int abort_flag;
 };
+static_assert(offsetof(Wkv5Smem, opK) == offsetof(Wkv5Smem, opR) + 64 * 64 * sizeof(float) &&
+                  recur::kScratchFloats <= 2 * 64 * 64 && recur::kRedFloats <= 64 * 64,
+              "the recurrent path's state copy spans opR and opK, its output parts fit opVt");
 static_assert(offsetof(Wkv5Smem, opS) == offsetof(Wkv5Smem, opK) + 64 * 64 * sizeof(float),
               "the first product reads k̃ and e^{32λ} Sᵀ as one 128-row operand");
 
@@ -150,16 +113,10 @@ __global__ void __launch_bounds__(kThreads, 2) wkv5_fwd_tc_kernel(const __grid_c
   }
   __syncthreads();
   if (tid < kN && !(expf(om[tid]) <= kMaxRate)) atomicOr(&sm.slow, 1);
+  if (tid < kN) sm.wdec[tid] = expf(-expf(om[tid]));
   __syncthreads();
-  if (sm.slow) {
-    if (tid < kN) {  // opR/opK double as scratch for the recurrence
-      sm.opS[tid] = expf(-expf(om[tid]));
-      sm.opS[64 + tid] = p.u[h * kN + tid];
-    }
-    __syncthreads();
-    head_recurrent(b, h, p.T, p.H, p.r, p.k, p.v, &sm.opS[0], &sm.opS[64], p.y, p.s_in, p.s_out, sm.opR, sm.opK, REV);
-    return;
-  }
+  // a head with some channel outside the factorization's range runs every chunk by the recurrence
+  const bool fast = sm.slow != 0;
 
   if (warp == 0) tmem_alloc(&sm.tmem_base, kTmemCols);
   // thread 0 issues every load; with the test hook set it arms the barrier and issues none
@@ -257,6 +214,44 @@ __global__ void __launch_bounds__(kThreads, 2) wkv5_fwd_tc_kernel(const __grid_c
     const int cnt = min(kL, p.T - t0);
     const uint32_t ph = (uint32_t)c & 1u;
     if (!mbar_wait_bounded(&sm.bar_tma, ph, p.ctl)) sm.abort_flag = 1;
+
+    if (fast) {  // the chunk's tokens one by one on the CUDA cores (opR, opK, opVt, diag as scratch)
+      __syncthreads();
+      if (sm.abort_flag) {
+        aborted = true;
+        break;
+      }
+      recur::ChunkArgs ca;
+      ca.rawR = reinterpret_cast<const unsigned char*>(sm.raw[0]);
+      ca.rawK = reinterpret_cast<const unsigned char*>(sm.raw[1]);
+      ca.rawV = reinterpret_cast<const unsigned char*>(sm.raw[2]);
+      ca.wconst = sm.wdec;
+      ca.wtok = nullptr;
+      ca.u = p.u + h * kN;
+      ca.scratch = sm.opR;
+      ca.red = sm.opVt;
+      ca.bonus = sm.diag;
+      ca.ystride = (size_t)p.H * kN;
+      ca.y = p.y + (((size_t)b * p.T + (REV ? p.T - 1 - t0 : t0)) * p.H + h) * kN;
+      ca.cnt = cnt;
+      ca.drow = drow;
+      ca.jcol = jcol;
+      recur::Frag16 f;
+#pragma unroll
+      for (int x = 0; x < 16; ++x) f.v[x] = S[x];
+      f = recur::chunk_recur<REV>(f, ca);
+#pragma unroll
+      for (int x = 0; x < 16; ++x) S[x] = f.v[x];
+      if (issuer && c + 1 < nchunk) {  // the boxes are consumed (the routine ends on a barrier)
+        fence_proxy_async();
+        mbar_arrive_expect_tx(&sm.bar_tma, 3 * kRawBytes);
+        const int rown = REV ? p.T - (c + 2) * kL : (c + 1) * kL;
+        tma_load_3d(sm.raw[0], &mr, &sm.bar_tma, h * kN, rown, b);
+        tma_load_3d(sm.raw[1], &mk, &sm.bar_tma, h * kN, rown, b);
+        tma_load_3d(sm.raw[2], &mv, &sm.bar_tma, h * kN, rown, b);
+      }
+      continue;
+    }
 
     // T1a: r̃, k̃ and the bonus parts (rows past the sequence end hold zeros from the TMA fill)
     {
@@ -454,7 +449,7 @@ __global__ void __launch_bounds__(kThreads, 2) wkv5_fwd_tc_kernel(const __grid_c
     // a wait gave up at chunk c: the previous chunk's MMA chains (committed last on bar_av) and
     // this chunk's loads must finish before the tensor memory and shared memory are released,
     // each wait bounded again
-    if (c >= 1) mbar_wait_bounded(&sm.bar_av, (uint32_t)(c - 1) & 1u, p.ctl);
+    if (c >= 1 && !fast) mbar_wait_bounded(&sm.bar_av, (uint32_t)(c - 1) & 1u, p.ctl);
     if (!withheld) mbar_wait_bounded(&sm.bar_tma, (uint32_t)c & 1u, p.ctl);
   }
   if (p.s_out != nullptr) {

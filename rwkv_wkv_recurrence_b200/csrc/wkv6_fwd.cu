@@ -25,7 +25,8 @@
 // the previous chunk folds its state, so that fold also writes e^{R} ⊙ Sᵀ for
 // the next chunk's state read as in the Eagle kernel.  A chunk whose decay
 // leaves that range in some channel (a fast decay, or one that jumps) is
-// computed by the per-token recurrence instead, on the same state registers.
+// computed by the per-token recurrence on the CUDA cores instead (chunk_recur,
+// all 256 threads), on the same state registers.
 //
 // Decay prologue per chunk: each thread forms λ for 8 tokens x 2 channels
 // (ω arrives by TMA as two fp32 [64 tokens x 32 channels] boxes); the
@@ -43,6 +44,7 @@
 #include "launch.h"
 #include "tc_common.cuh"
 #include "wkv_common.cuh"
+#include "wkv_recur.cuh"
 
 namespace rwkv {
 namespace {
@@ -75,6 +77,9 @@ struct Wkv6Smem {
   uint32_t tmem_base;
   int abort_flag;
 };
+static_assert(offsetof(Wkv6Smem, opK) == offsetof(Wkv6Smem, opRA) + 64 * 64 * sizeof(float) &&
+                  recur::kScratchFloats <= 2 * 64 * 64 && recur::kRedFloats <= 64 * 64,
+              "the recurrent path's state copy spans opRA and opK, its output parts fit opVt");
 static_assert(offsetof(Wkv6Smem, opS) == offsetof(Wkv6Smem, opK) + 64 * 64 * sizeof(float),
               "the first product reads k̃ and e^{R} Sᵀ as one 128-row operand");
 
@@ -90,17 +95,6 @@ __device__ __forceinline__ float lds_f32(uint32_t addr) {
   return v;
 }
 
-__device__ __forceinline__ float lds_bf16(uint32_t addr) {
-  unsigned short x;
-  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(x) : "r"(addr) : "memory");
-  return __uint_as_float((uint32_t)x << 16);
-}
-
-// Byte offset of (token τ, channel d) in a [64 x 64] bf16 box with the 128-byte swizzle.
-__device__ __forceinline__ uint32_t raw_off(int tau, int d) {
-  return (uint32_t)tau * 128u + ((uint32_t)((d >> 3) ^ (tau & 7)) << 4) + (uint32_t)(d & 7) * 2u;
-}
-
 // Byte offset of (token τ, channel d) in the two fp32 ω boxes with the 128-byte swizzle.
 __device__ __forceinline__ uint32_t om_off(int tau, int d) {
   return (uint32_t)(d >> 5) * kOmBytes + (uint32_t)tau * 128u + ((uint32_t)(((d & 31) >> 2) ^ (tau & 7)) << 4) +
@@ -111,68 +105,7 @@ __device__ __forceinline__ uint32_t om_off(int tau, int d) {
 // (the middle of the chunk if the decay rate stays put), no lower than -79.
 __device__ __forceinline__ float next_ref(float lend) { return fmaxf(0.5f * lend, -79.f); }
 
-struct Frag16 {
-  float v[16];
-};
-
-// One chunk by the per-token recurrence, for a chunk whose decay is too fast
-// for the factorization.  S is the state fragment of this thread (rows
-// drow, drow + 8; columns jcol + 4 q); the raw r, k, v and ω boxes of the
-// chunk are in shared memory and the bonus parts of every token in diag_part.
-__device__ __noinline__ Frag16 chunk_recurrent(Frag16 S, Wkv6Smem& sm, const Wkv6Params& p, int b, int h, int t0,
-                                               int cnt) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int t4 = lane >> 2, tq = lane & 3, q4 = warp & 3, hc = warp >> 2;
-  const int drow = 16 * q4 + t4, jcol = 32 * hc + tq;
-  if (tid < kL) {
-    float sum = 0.f;
-#pragma unroll
-    for (int w = 0; w < 8; ++w) sum += sm.diag_part[w][tid];
-    sm.diag[tid] = sum;
-  }
-  __syncthreads();
-  const uint32_t rawR = smem_u32(sm.raw[0]), rawK = smem_u32(sm.raw[1]), rawV = smem_u32(sm.raw[2]);
-  const uint32_t omS = smem_u32(sm.om[0]);
-  float* red = sm.opVt;  // [2][4][64]: per-quarter partial outputs, double-buffered by token parity
-  for (int tau = 0; tau < cnt; ++tau) {
-    float rd[2], kd[2], wd[2], vq[8], part[8];
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      const int d = drow + 8 * r;
-      rd[r] = lds_bf16(rawR + raw_off(tau, d));
-      kd[r] = lds_bf16(rawK + raw_off(tau, d));
-      wd[r] = __expf(-__expf(lds_f32(omS + om_off(tau, d))));
-    }
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      vq[q] = lds_bf16(rawV + raw_off(tau, jcol + 4 * q));
-      part[q] = fmaf(rd[0], S.v[2 * q], rd[1] * S.v[2 * q + 1]);
-    }
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      part[q] += __shfl_xor_sync(0xffffffffu, part[q], 4);
-      part[q] += __shfl_xor_sync(0xffffffffu, part[q], 8);
-      part[q] += __shfl_xor_sync(0xffffffffu, part[q], 16);
-    }
-    if (t4 == 0) {
-#pragma unroll
-      for (int q = 0; q < 8; ++q) red[(tau & 1) * 256 + q4 * 64 + jcol + 4 * q] = part[q];
-    }
-#pragma unroll
-    for (int q = 0; q < 8; ++q)
-#pragma unroll
-      for (int r = 0; r < 2; ++r) S.v[2 * q + r] = fmaf(wd[r], S.v[2 * q + r], kd[r] * vq[q]);
-    __syncthreads();
-    if (tid < kN) {
-      const float* rb = red + (tau & 1) * 256;
-      float y = (rb[tid] + rb[64 + tid]) + (rb[128 + tid] + rb[192 + tid]);
-      y = fmaf(sm.diag[tau], lds_bf16(rawV + raw_off(tau, tid)), y);
-      p.y[(((size_t)b * p.T + t0 + tau) * p.H + h) * kN + tid] = __float2bfloat16_rn(y);
-    }
-  }
-  __syncthreads();
-  return S;
-}
+using recur::Frag16;
 
 __global__ void __launch_bounds__(kThreads, 2) wkv6_fwd_tc_kernel(const __grid_constant__ CUtensorMap mr,
                                                                   const __grid_constant__ CUtensorMap mk,
@@ -347,7 +280,28 @@ __global__ void __launch_bounds__(kThreads, 2) wkv6_fwd_tc_kernel(const __grid_c
     }
 
     if (slow) {  // some channel decays too fast for the factorization: per-token recurrence
-      S = chunk_recurrent(S, sm, p, b, h, t0, cnt);
+      // the decay of every (token, key) into opS (rewritten below from the new state)
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int tau = tid >> 2, d = 16 * (tid & 3) + i;
+        sm.opS[tau * kN + d] = __expf(-__expf(lds_f32(omS + om_off(tau, d))));
+      }
+      recur::ChunkArgs ca;
+      ca.rawR = reinterpret_cast<const unsigned char*>(sm.raw[0]);
+      ca.rawK = reinterpret_cast<const unsigned char*>(sm.raw[1]);
+      ca.rawV = reinterpret_cast<const unsigned char*>(sm.raw[2]);
+      ca.wconst = nullptr;
+      ca.wtok = sm.opS;
+      ca.u = p.u + h * kN;
+      ca.scratch = sm.opRA;
+      ca.red = sm.opVt;
+      ca.bonus = sm.diag;
+      ca.ystride = (size_t)p.H * kN;
+      ca.y = p.y + (((size_t)b * p.T + t0) * p.H + h) * kN;
+      ca.cnt = cnt;
+      ca.drow = drow;
+      ca.jcol = jcol;
+      S = recur::chunk_recur<false>(S, ca);
       if (c + 1 < nchunk) {
 #pragma unroll
         for (int r = 0; r < 2; ++r) {

@@ -118,6 +118,22 @@ def test_finch_workload_full_size(cuda_device):
             assert_close_rms(sc[b, h], ref_s[b, h], TOL_BF16, f"s head ({b},{h})")
 
 
+def test_finch_fast_decay_full_size(cuda_device):
+    # B4 T4096 H40 N64 with per-token omega = U(-1, 2) base + 0.5 N(0, 1): nearly
+    # every chunk decays too fast for the factorization and runs by the recurrence;
+    # all 160 heads checked element by element
+    B, T, H, N = 4, 4096, 40, 64
+    p = wi.wkv6_problem(B, T, H, N, seed=SEED + 7, omega_range=(-1.0, 2.0))
+    y, s = rw.rwkv_wkv6_forward(**_cuda(p, cuda_device), return_state=True)
+    rw.rwkv_check_device_error()
+    ref, ref_s = oracle.wkv6_forward(p["r"], p["k"], p["v"], p["omega"], p["u"], return_state=True)
+    yc, sc = y.cpu(), s.cpu()
+    for b in range(B):
+        for h in range(H):
+            assert_close_rms(yc[b, :, h], ref[b, :, h], TOL_BF16, f"y head ({b},{h})")
+            assert_close_rms(sc[b, h], ref_s[b, h], TOL_BF16, f"s head ({b},{h})")
+
+
 # ------------------------------------------------------------------ decode step
 def _token(p, t):
     return {n: p[n][:, t].contiguous() for n in ("r", "k", "v", "omega")}
