@@ -228,7 +228,7 @@ RWKV_API size_t rwkv_wkv5_backward_workspace_bytes(int64_t B, int64_t T, int64_t
  *   workspace     device scratch of rwkv_wkv5_backward_workspace_bytes() bytes (the forward
  *                 states at every 64th token, per-row sums).
  *   N must be 64; the [B,T,H,N] tensors 16-byte aligned (RWKV_ERR_UNSUPPORTED otherwise).
- *   A channel decaying faster than exp(omega) = 2.5 (w < 0.082) is outside the
+ *   A channel decaying faster than exp(omega) = 2 (w < 0.135) is outside the
  *   range this backward computes: the call returns RWKV_OK, the outputs of
  *   that channel's heads are undefined, and rwkv_check_device_error reports
  *   RWKV_ERR_UNSUPPORTED.  Deterministic.

@@ -120,6 +120,12 @@ __device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
   return v;
 }
 
+__device__ __forceinline__ unsigned short lds_u16(uint32_t addr) {
+  unsigned short v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr) : "memory");
+  return v;
+}
+
 // D[tmem] (+)= A[tmem] * B[smem]ᵀ, kind::tf32 (A rows in the accumulator layout).
 __device__ __forceinline__ void umma_tf32_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
                                              uint32_t accumulate) {
@@ -138,6 +144,15 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&q)[4]) {
                : "=r"(q[0]), "=r"(q[1]), "=r"(q[2]), "=r"(q[3])
                : "r"(addr)
                : "memory");
+}
+
+// fp32 to tf32 rounded to nearest (ties away from zero), the 13 low mantissa bits cleared.  The
+// tensor core reads only the top 19 bits of a tf32 operand, so without this it would truncate:
+// a relative error up to 2^-10 with a bias toward zero, which adds up across a product's terms.
+__device__ __forceinline__ float to_tf32(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return __uint_as_float(r);
 }
 
 // Two packed bf16 (low half first) to fp32.

@@ -56,7 +56,8 @@
 // CTA: one (batch, head), 8 warps.  Forward pass: ~105 KB of shared memory,
 // 256 TMEM columns, two CTAs per SM.  Reversed pass: ~140 KB, 512 columns, one
 // CTA per SM.  A head with some channel decaying faster than the chunked
-// factorization allows (exp(ω) > 2.5) is not handled: the kernel sets
+// factorization takes (exp(ω) > 2: factors beyond e^{±64} would push small
+// operands into the subnormal range) is not handled: the kernel sets
 // kErrFastDecay in the device error word and leaves that head's outputs unset.
 #include <cstddef>
 
@@ -73,7 +74,7 @@ constexpr int kN = 64;
 constexpr int kL = 64;
 constexpr int kThreads = 256;
 constexpr uint32_t kRawBytes = kL * kN * 2;
-constexpr float kMaxRate = 2.5f;
+constexpr float kMaxRate = 2.f;
 constexpr uint32_t kCkBytes = kN * kN * 4;  // one forward-state checkpoint (fp32, operand layout)
 
 struct Wkv5BwdSmem {
@@ -216,7 +217,7 @@ __global__ void __launch_bounds__(kThreads, REV ? 1 : 2) wkv5_bwd_tc_kernel(cons
   for (int r = 0; r < 2; ++r) {
     const float f0 = expf((32.f - (float)p.lead) * lamr[r]);
 #pragma unroll
-    for (int q = 0; q < 8; ++q) sm.opX[op_off(drow + 8 * r, jcol + 4 * q)] = f0 * X[2 * q + r];
+    for (int q = 0; q < 8; ++q) sm.opX[op_off(drow + 8 * r, jcol + 4 * q)] = to_tf32(f0 * X[2 * q + r]);
   }
 
   // ---- epilogue rows: lane < 16 of quarter q4 holds key row de = 16 q4 + lane, positions 32 hc + i
@@ -278,7 +279,11 @@ __global__ void __launch_bounds__(kThreads, REV ? 1 : 2) wkv5_bwd_tc_kernel(cons
 #pragma unroll
       for (int q = 0; q < 8; ++q)
 #pragma unroll
-        for (int r = 0; r < 2; ++r) part[r] = fmaf(X[2 * q + r], sm.opXc[op_off(drow + 8 * r, jcol + 4 * q)], part[r]);
+        for (int r = 0; r < 2; ++r) {
+          float& xc = sm.opXc[op_off(drow + 8 * r, jcol + 4 * q)];
+          part[r] = fmaf(X[2 * q + r], xc, part[r]);
+          xc = to_tf32(xc);  // the X_c read below takes it rounded to nearest
+        }
       const float n = (float)(kL - lo);
 #pragma unroll
       for (int r = 0; r < 2; ++r) acc_t1[r] += (double)(n * expf((n - 1.f) * lamr[r]) * part[r]);
@@ -330,8 +335,8 @@ __global__ void __launch_bounds__(kThreads, REV ? 1 : 2) wkv5_bwd_tc_kernel(cons
           const int i = 2 * pp + (m >> 1), r = m & 1;
           const float2 f = bf2_to_f2(qk[m]);
           const float g = i == 0 ? 1.f : (i == 1 ? fcs[r] : (i == 2 ? fcs[r] * fcs[r] : fcs[r] * fcs[r] * fcs[r]));
-          kt[4 * i + 2 * r] = __float_as_uint(f.x * fc0[r][0] * g);
-          kt[4 * i + 2 * r + 1] = __float_as_uint(f.y * fc0[r][1] * g);
+          kt[4 * i + 2 * r] = __float_as_uint(to_tf32(f.x * fc0[r][0] * g));
+          kt[4 * i + 2 * r + 1] = __float_as_uint(to_tf32(f.y * fc0[r][1] * g));
         }
         issue_first(2 + 2 * pp);
       }
@@ -408,8 +413,8 @@ __global__ void __launch_bounds__(kThreads, REV ? 1 : 2) wkv5_bwd_tc_kernel(cons
           for (int r = 0; r < 2; ++r) {
             const int io = 32 * hc + 4 * q + tq, tau = tau0 + 8 * r;
             const float am = io < tau ? a[2 * q + r] : 0.f;
-            sm.opAm[op_off(tau, io)] = am;
-            if constexpr (REV) sm.opAl[op_off(tau, io)] = (float)(tau - 1 - io) * am;
+            sm.opAm[op_off(tau, io)] = to_tf32(am);
+            if constexpr (REV) sm.opAl[op_off(tau, io)] = to_tf32((float)(tau - 1 - io) * am);
             if (io == tau) sm.diag[tau] = a[2 * q + r];
           }
       }
@@ -448,7 +453,7 @@ __global__ void __launch_bounds__(kThreads, REV ? 1 : 2) wkv5_bwd_tc_kernel(cons
           for (int q = 0; q < 8; ++q) {
             const int x = 2 * q + r;
             X[x] = fmaf(gx, X[x], e32[r] * ds[x]);
-            sm.opX[op_off(drow + 8 * r, jcol + 4 * q)] = e32[r] * X[x];
+            sm.opX[op_off(drow + 8 * r, jcol + 4 * q)] = to_tf32(e32[r] * X[x]);
           }
         }
       } else {  // partial last chunk (forward pass): no later chunk reads opX

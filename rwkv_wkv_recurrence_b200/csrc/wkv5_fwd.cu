@@ -29,9 +29,17 @@
 // key channel when it is folded into the fp32 master state, which lives in
 // registers (S' = e^{cnt λ} S + e^{(cnt-32) λ} ΔS), so the state is never
 // rounded below fp32.  Splitting e^{λ(τ-1-ι)} around the chunk middle keeps
-// every factor within e^{±32|λ|}; a head with -λ > 2.5 in any channel
-// (w < 0.082) would leave the fp32 range there: its chunks run token by token
-// on the CUDA cores instead (chunk_recur), with the same TMA boxes and state.
+// every factor within e^{±32|λ|}: for -λ ≤ 2 (w ≥ 0.135) within e^{±64}, which
+// leaves the small operands (a factor e^{-64} times a value down to 1e-10)
+// clear of the subnormal range, where a tf32 operand keeps few bits.  A
+// faster channel enters the products only where its factor is at most 1: its r̃
+// column is r e^{λτ} with e^{λ·0} Sᵀ unscaled in opS (the state read), its k̃
+// column is zero (no part in the scores), and its k̃ᵀ row is k e^{λ(cnt-1-ι)}
+// (the state increment, folded without a further factor).  Its intra-chunk
+// scores Σ_c r_τ[c] k_ι[c] e^{λ_c (τ-1-ι)} are added on the CUDA cores while the
+// scores are masked, at lags τ-1-ι ≤ 15: beyond that e^{λn} < 2^-46 of the lag-0
+// weight, far below the fp32 rounding of the output rows those terms would join.  Any w in [0, 1] is
+// therefore handled on the same path, down to w = 0.
 //
 // The tensor core takes tf32 operands K-major only, so the operand tiles are
 // fp32 [rows][64] in the K-major core-matrix layout without swizzle (8 rows x
@@ -51,7 +59,6 @@
 #include "launch.h"
 #include "tc_common.cuh"
 #include "wkv_common.cuh"
-#include "wkv_recur.cuh"
 
 namespace rwkv {
 namespace {
@@ -62,7 +69,9 @@ constexpr int kN = 64;                 // head size
 constexpr int kL = 64;                 // tokens per chunk
 constexpr int kThreads = 256;
 constexpr uint32_t kRawBytes = kL * kN * 2;    // one bf16 [64 x 64] box
-constexpr float kMaxRate = 2.5f;       // largest -λ the chunked factorization accepts
+constexpr float kMaxRate = 2.f;        // largest -λ the chunked factorization takes
+constexpr int kBand = 15;              // lags a fast channel keeps in the scores: e^{-2 (kBand+1)} < 2^-46
+static_assert(kBand == 15, "the band pass gives each thread 4 of the 16 lags of one position");
 constexpr uint32_t kTmemCols = 256;  // [scores | output rows], state increment, k̃ᵀ (64 columns each)
 
 struct Wkv5Smem {
@@ -71,20 +80,31 @@ struct Wkv5Smem {
   alignas(128) float opK[64 * 64];   // k̃ = k e^{λ(31-ι)}   [ι][d]: B rows 0..63 of the first product
   alignas(128) float opS[64 * 64];   // e^{32λ} ⊙ Sᵀ         [j][d]: B rows 64..127 of the first product
   alignas(128) float opVt[64 * 64];  // vᵀ                   [j][ι]: B of A v and of the state increment
-  float diag_part[8][kL];            // per-warp parts of Σ_d r u k (the bonus term)
+  union {
+    float diag_part[8][kL];          // per-warp parts of Σ_d r u k (the bonus term), T1a -> T1b
+    float AF[kL][kBand + 1];         // the fast channels' scores [τ][n = τ-1-ι], T1b (after the
+  } u;                               // bonus sums) -> T2a
   float diag[kL];                    // Σ_d r u k per token
-  float wdec[kN];                    // w per key channel (heads on the recurrent path)
+  // fast channels: r and k as bf16 pairs of fast indices, word w of row x at column w ^ (x & 31)
+  // (lanes on different rows meet different banks)
+  uint32_t RFw[kL][kN / 2];
+  uint32_t KFw[kL][kN / 2];
+  alignas(16) float E4[kN][4];           // e^{λ n} for n = 0, 4, 8, 12 [fast index][n / 4]
+  float E1[kN];                          // e^{λ} [fast index]
+  int fidx[kN];                          // fast index of each key channel, -1 for a slow one
+  int flist[kN];                         // key channel of each fast index
+  unsigned fmask[2];
   alignas(8) uint64_t bar_tma;
   alignas(8) uint64_t bar_sc;        // scores and state read done
   alignas(8) uint64_t bar_av;        // A v done
   alignas(8) uint64_t bar_ds;        // state increment done
   uint32_t tmem_base;
-  int slow;
+  int nfast;
   int abort_flag;
 };
-static_assert(offsetof(Wkv5Smem, opK) == offsetof(Wkv5Smem, opR) + 64 * 64 * sizeof(float) &&
-                  recur::kScratchFloats <= 2 * 64 * 64 && recur::kRedFloats <= 64 * 64,
-              "the recurrent path's state copy spans opR and opK, its output parts fit opVt");
+// dynamic shared memory = the struct + 1024 bytes of alignment slack; an SM has 228 KB, of which
+// each resident CTA also takes 1 KB: two CTAs per SM
+static_assert(2 * (sizeof(Wkv5Smem) + 1024 + 1024) <= 228 * 1024, "two CTAs per SM");
 static_assert(offsetof(Wkv5Smem, opS) == offsetof(Wkv5Smem, opK) + 64 * 64 * sizeof(float),
               "the first product reads k̃ and e^{32λ} Sᵀ as one 128-row operand");
 
@@ -107,16 +127,36 @@ __global__ void __launch_bounds__(kThreads, 2) wkv5_fwd_tc_kernel(const __grid_c
   const int nchunk = (p.T + kL - 1) / kL;
   const float* om = p.omega + h * kN;
 
-  if (tid == 0) {
-    sm.slow = 0;
-    sm.abort_flag = 0;
+  // ---- fast channels (-λ > 2): outside the factorization's range.  They enter the tensor-core
+  // products only where the factor stays at most 1 (state read e^{λτ}, state increment
+  // e^{λ(cnt-1-ι)}); their intra-chunk scores are summed on the CUDA cores over lags 0..kBand.
+  if (tid == 0) sm.abort_flag = 0;
+  for (int i = tid; i < kL * kN / 2; i += kThreads) {
+    (&sm.RFw[0][0])[i] = 0u;
+    (&sm.KFw[0][0])[i] = 0u;
+  }
+  if (tid < kN) {
+    const bool f = !(expf(om[tid]) <= kMaxRate);
+    const unsigned m = __ballot_sync(0xffffffffu, f);
+    if (lane == 0) sm.fmask[warp] = m;
   }
   __syncthreads();
-  if (tid < kN && !(expf(om[tid]) <= kMaxRate)) atomicOr(&sm.slow, 1);
-  if (tid < kN) sm.wdec[tid] = expf(-expf(om[tid]));
+  if (tid < kN) {
+    const unsigned m0 = sm.fmask[0], m1 = sm.fmask[1];
+    const bool f = ((tid < 32 ? m0 : m1) >> (tid & 31)) & 1u;
+    const int below = tid < 32 ? __popc(m0 & ((1u << tid) - 1u)) : __popc(m0) + __popc(m1 & ((1u << (tid & 31)) - 1u));
+    sm.fidx[tid] = f ? below : -1;
+    if (f) {
+      sm.flist[below] = tid;
+      const float lam = -expf(om[tid]);
+#pragma unroll
+      for (int g = 0; g < 4; ++g) sm.E4[below][g] = g == 0 ? 1.f : expf(lam * (float)(4 * g));
+      sm.E1[below] = expf(lam);
+    }
+    if (tid == 0) sm.nfast = __popc(m0) + __popc(m1);
+  }
   __syncthreads();
-  // a head with some channel outside the factorization's range runs every chunk by the recurrence
-  const bool fast = sm.slow != 0;
+  const int nfast = sm.nfast;
 
   if (warp == 0) tmem_alloc(&sm.tmem_base, kTmemCols);
   // thread 0 issues every load; with the test hook set it arms the barrier and issues none
@@ -143,14 +183,17 @@ __global__ void __launch_bounds__(kThreads, 2) wkv5_fwd_tc_kernel(const __grid_c
   // A half-warp then writes one whole core matrix (eight 16-byte rows): no bank conflicts.
   const int rr = lane & 7, rp = lane >> 3;
   const int dR = 8 * warp + 2 * rp;
+  // a fast channel: r e^{λτ} (read only; its k̃ is zero, so it adds nothing to the scores)
   float fr0[2], frs[2], fk0[2], fks[2], uA[2];
+  int fiA[2];
 #pragma unroll
   for (int e = 0; e < 2; ++e) {
     const float rate = expf(om[dR + e]);  // -λ
-    fr0[e] = expf(-rate * (float)(rr - 32));
+    fiA[e] = sm.fidx[dR + e];
+    fr0[e] = fiA[e] >= 0 ? (rr == 0 ? 1.f : expf(-rate * (float)rr)) : expf(-rate * (float)(rr - 32));
     frs[e] = expf(-8.f * rate);
-    fk0[e] = expf(-rate * (float)(31 - rr));
-    fks[e] = expf(8.f * rate);
+    fk0[e] = fiA[e] >= 0 ? 0.f : expf(-rate * (float)(31 - rr));
+    fks[e] = fiA[e] >= 0 ? 0.f : expf(8.f * rate);
     uA[e] = p.u[h * kN + dR + e];
   }
   // box row of position 8 ib + rr: 8 ib + rr, or 63 - (8 ib + rr) = 8 (7 - ib) + (7 - rr) reversed
@@ -166,13 +209,17 @@ __global__ void __launch_bounds__(kThreads, 2) wkv5_fwd_tc_kernel(const __grid_c
                             : (uint32_t)(lmat * 8 + lrow) * 128u + (uint32_t)((warp ^ lrow) << 4);
   // ---- k̃ᵀ (tensor memory, A of the state increment), .16x256b fragment of warp w:
   // rows d = 16 q4 + t4 + 8 r, columns ι = 32 hc + 8 i + 2 tq + e  ->  register 4 i + 2 r + e
-  float fc0[2][2], fcs[2];
+  // (a fast row's factor is e^{λ(cnt-1-ι)}, formed per chunk)
+  float fc0[2][2], fcs[2], lamT[2];
+  bool fastT[2];
 #pragma unroll
   for (int r = 0; r < 2; ++r) {
     const float rate = expf(om[16 * q4 + 8 * r + t4]);
+    lamT[r] = -rate;
+    fastT[r] = sm.fidx[16 * q4 + 8 * r + t4] >= 0;
 #pragma unroll
-    for (int e = 0; e < 2; ++e) fc0[r][e] = expf(-rate * (float)(31 - 32 * hc - 2 * tq - e));
-    fcs[r] = expf(8.f * rate);
+    for (int e = 0; e < 2; ++e) fc0[r][e] = fastT[r] ? 0.f : expf(-rate * (float)(31 - 32 * hc - 2 * tq - e));
+    fcs[r] = fastT[r] ? 0.f : expf(8.f * rate);
   }
   // position 32 hc + 8 (lmat >> 1) + lrow (+ 16 per pp); its box row bottom up when REV
   const uint32_t offKt =
@@ -197,7 +244,8 @@ __global__ void __launch_bounds__(kThreads, 2) wkv5_fwd_tc_kernel(const __grid_c
 #pragma unroll
   for (int q = 0; q < 8; ++q)
 #pragma unroll
-    for (int r = 0; r < 2; ++r) sm.opS[op_off(jcol + 4 * q, drow + 8 * r)] = e32[r] * S[2 * q + r];
+    for (int r = 0; r < 2; ++r)
+      sm.opS[op_off(jcol + 4 * q, drow + 8 * r)] = (fastT[r] ? 1.f : e32[r]) * S[2 * q + r];
 
   tc_fence_before();
   __syncthreads();
@@ -215,45 +263,9 @@ __global__ void __launch_bounds__(kThreads, 2) wkv5_fwd_tc_kernel(const __grid_c
     const uint32_t ph = (uint32_t)c & 1u;
     if (!mbar_wait_bounded(&sm.bar_tma, ph, p.ctl)) sm.abort_flag = 1;
 
-    if (fast) {  // the chunk's tokens one by one on the CUDA cores (opR, opK, opVt, diag as scratch)
-      __syncthreads();
-      if (sm.abort_flag) {
-        aborted = true;
-        break;
-      }
-      recur::ChunkArgs ca;
-      ca.rawR = reinterpret_cast<const unsigned char*>(sm.raw[0]);
-      ca.rawK = reinterpret_cast<const unsigned char*>(sm.raw[1]);
-      ca.rawV = reinterpret_cast<const unsigned char*>(sm.raw[2]);
-      ca.wconst = sm.wdec;
-      ca.wtok = nullptr;
-      ca.u = p.u + h * kN;
-      ca.scratch = sm.opR;
-      ca.red = sm.opVt;
-      ca.bonus = sm.diag;
-      ca.ystride = (size_t)p.H * kN;
-      ca.y = p.y + (((size_t)b * p.T + (REV ? p.T - 1 - t0 : t0)) * p.H + h) * kN;
-      ca.cnt = cnt;
-      ca.drow = drow;
-      ca.jcol = jcol;
-      recur::Frag16 f;
-#pragma unroll
-      for (int x = 0; x < 16; ++x) f.v[x] = S[x];
-      f = recur::chunk_recur<REV>(f, ca);
-#pragma unroll
-      for (int x = 0; x < 16; ++x) S[x] = f.v[x];
-      if (issuer && c + 1 < nchunk) {  // the boxes are consumed (the routine ends on a barrier)
-        fence_proxy_async();
-        mbar_arrive_expect_tx(&sm.bar_tma, 3 * kRawBytes);
-        const int rown = REV ? p.T - (c + 2) * kL : (c + 1) * kL;
-        tma_load_3d(sm.raw[0], &mr, &sm.bar_tma, h * kN, rown, b);
-        tma_load_3d(sm.raw[1], &mk, &sm.bar_tma, h * kN, rown, b);
-        tma_load_3d(sm.raw[2], &mv, &sm.bar_tma, h * kN, rown, b);
-      }
-      continue;
-    }
-
-    // T1a: r̃, k̃ and the bonus parts (rows past the sequence end hold zeros from the TMA fill)
+    // T1a: r̃, k̃ and the bonus parts (rows past the sequence end hold zeros from the TMA fill).
+    // r̃ and k̃ are rounded to nearest tf32: the tensor core would truncate both, and the two
+    // biases toward zero add in every score.
     {
       float fr[2] = {fr0[0], fr0[1]}, fk[2] = {fk0[0], fk0[1]};
 #pragma unroll
@@ -262,17 +274,34 @@ __global__ void __launch_bounds__(kThreads, 2) wkv5_fwd_tc_kernel(const __grid_c
         const float2 rv = bf2_to_f2(lds_u32(rawR + offRK + ibo));
         const float2 kv = bf2_to_f2(lds_u32(rawK + offRK + ibo));
         const int row = 8 * ib + rr;
-        *reinterpret_cast<float2*>(&sm.opR[op_off(row, dR)]) = make_float2(rv.x * fr[0], rv.y * fr[1]);
-        *reinterpret_cast<float2*>(&sm.opK[op_off(row, dR)]) = make_float2(kv.x * fk[0], kv.y * fk[1]);
+        *reinterpret_cast<float2*>(&sm.opR[op_off(row, dR)]) = make_float2(to_tf32(rv.x * fr[0]), to_tf32(rv.y * fr[1]));
+        *reinterpret_cast<float2*>(&sm.opK[op_off(row, dR)]) = make_float2(to_tf32(kv.x * fk[0]), to_tf32(kv.y * fk[1]));
         float part = fmaf(rv.x * uA[0], kv.x, rv.y * uA[1] * kv.y);
         part += __shfl_xor_sync(0xffffffffu, part, 8);
         part += __shfl_xor_sync(0xffffffffu, part, 16);
-        if (rp == 0) sm.diag_part[warp][row] = part;
+        if (rp == 0) sm.u.diag_part[warp][row] = part;
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
           fr[e] *= frs[e];
           fk[e] *= fks[e];
         }
+      }
+    }
+    if (nfast > 0) {  // the fast channels' r and k into the compact rows (bf16 as loaded)
+#pragma unroll
+      for (int ib = 0; ib < 8; ++ib) {
+        const uint32_t ibo = (uint32_t)(REV ? 7 - ib : ib) * 1024u;
+        const uint32_t rw = lds_u32(rawR + offRK + ibo), kw = lds_u32(rawK + offRK + ibo);
+        const int row = 8 * ib + rr;
+#pragma unroll
+        for (int e = 0; e < 2; ++e)
+          if (fiA[e] >= 0) {
+            const int col = ((fiA[e] >> 1) ^ (row & 31));
+            unsigned short* rh = reinterpret_cast<unsigned short*>(&sm.RFw[row][col]) + (fiA[e] & 1);
+            unsigned short* kh = reinterpret_cast<unsigned short*>(&sm.KFw[row][col]) + (fiA[e] & 1);
+            *rh = (unsigned short)(e ? rw >> 16 : rw & 0xFFFFu);
+            *kh = (unsigned short)(e ? kw >> 16 : kw & 0xFFFFu);
+          }
       }
     }
     fence_proxy_async();
@@ -302,7 +331,7 @@ __global__ void __launch_bounds__(kThreads, 2) wkv5_fwd_tc_kernel(const __grid_c
       if (tid < kL) {
         float sum = 0.f;
 #pragma unroll
-        for (int w = 0; w < 8; ++w) sum += sm.diag_part[w][tid];
+        for (int w = 0; w < 8; ++w) sum += sm.u.diag_part[w][tid];
         sm.diag[tid] = sum;
       }
       uint32_t kt[16];
@@ -319,6 +348,67 @@ __global__ void __launch_bounds__(kThreads, 2) wkv5_fwd_tc_kernel(const __grid_c
           kt[4 * i + 2 * r + 1] = __float_as_uint(f.y * fc0[r][1] * g);
         }
         issue_first(2 + 2 * pp);
+      }
+      if (nfast > 0) {
+        // the fast channels' scores at lags n = 0..kBand, Σ_c r_τ[c] k_{τ-1-n}[c] e^{λ_c n}: thread
+        // (τ, 4 lags), every CTA thread busy; AF overlays the bonus parts, summed above
+        __syncthreads();
+        const int tau = tid >> 2, g4 = tid & 3, n0 = 4 * g4;
+        int rk[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) rk[e] = tau - 1 - (n0 + e);  // ι of lag n0 + e (negative: none)
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        const int npair = (nfast + 1) >> 1;
+#pragma unroll 2
+        for (int w = 0; w < npair; ++w) {
+          const float2 rv = bf2_to_f2(sm.RFw[tau][w ^ (tau & 31)]);
+          float ew[2][4];
+#pragma unroll
+          for (int h2 = 0; h2 < 2; ++h2) {
+            const int cfi = 2 * w + h2;
+            const float e1 = sm.E1[cfi];
+            ew[h2][0] = sm.E4[cfi][g4];
+            ew[h2][1] = ew[h2][0] * e1;
+            ew[h2][2] = ew[h2][1] * e1;
+            ew[h2][3] = ew[h2][2] * e1;
+          }
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            if (rk[e] >= 0) {
+              const float2 kv = bf2_to_f2(sm.KFw[rk[e]][w ^ (rk[e] & 31)]);
+              acc[e] = fmaf(rv.x * kv.x, ew[0][e], acc[e]);
+              acc[e] = fmaf(rv.y * kv.y, ew[1][e], acc[e]);
+            }
+          }
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) sm.u.AF[tau][n0 + e] = acc[e];
+      }
+      if (nfast > 0) {  // a fast row: k e^{λ(cnt-1-ι)}, zero past the chunk's tokens
+#pragma unroll
+        for (int pp = 0; pp < 2; ++pp) {
+          uint32_t qk[4];
+          ldsm_x4_t(REV ? rawK + offKt - pp * 2048u : rawK + offKt + pp * 2048u, qk);
+#pragma unroll
+          for (int m = 0; m < 4; ++m) {
+            const int i = 2 * pp + (m >> 1), r = m & 1;
+            if (fastT[r]) {
+              const float2 f = bf2_to_f2(qk[m]);
+              const int io = 32 * hc + 8 * i + 2 * tq;
+              // e^{λ n}, n = cnt-1-ι: the tabled powers up to n = 15, zero beyond (below 2^-46)
+              const int cf = sm.fidx[16 * q4 + 8 * r + t4];
+              auto pw = [&](int n) {
+                if (n < 0 || n > kBand) return 0.f;
+                float x = sm.E4[cf][n >> 2];
+                for (int t = 0; t < (n & 3); ++t) x *= sm.E1[cf];
+                return x;
+              };
+              const float c0 = pw(cnt - 1 - io), c1 = pw(cnt - 2 - io);
+              kt[4 * i + 2 * r] = __float_as_uint(f.x * c0);
+              kt[4 * i + 2 * r + 1] = __float_as_uint(f.y * c1);
+            }
+          }
+        }
       }
       tmem_st16(tKt + tquar + (uint32_t)(32 * hc), kt);
 #pragma unroll
@@ -370,6 +460,15 @@ __global__ void __launch_bounds__(kThreads, 2) wkv5_fwd_tc_kernel(const __grid_c
       } else {
         float a[16];
         tmem_ld16x128(tSc + tquar + (uint32_t)(32 * hc), a);
+        if (nfast > 0) {  // the fast channels' scores at lags 0..kBand (formed in T1b)
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+              const int io = 32 * hc + 4 * q + tq, tau = tau0 + 8 * r, n = tau - 1 - io;
+              if (n >= 0 && n <= kBand) a[2 * q + r] += sm.u.AF[tau][n];
+            }
+        }
         float dg[2] = {0.f, 0.f};
         if ((q4 >> 1) == hc) {  // the fragment holds the diagonal
           dg[0] = sm.diag[tau0];
@@ -396,7 +495,7 @@ __global__ void __launch_bounds__(kThreads, 2) wkv5_fwd_tc_kernel(const __grid_c
     }
 
     // T2b: S <- e^{cnt λ} S + e^{(cnt-32) λ} ΔS; e^{32λ} Sᵀ into opS for the next chunk (while A v
-    // still runs)
+    // still runs).  A fast row's ΔS already carries e^{λ(cnt-1-ι)}, and its opS row is S itself.
     if (!mbar_wait_bounded(&sm.bar_ds, ph, p.ctl)) sm.abort_flag = 1;
     tc_fence_after();
     {
@@ -409,14 +508,19 @@ __global__ void __launch_bounds__(kThreads, 2) wkv5_fwd_tc_kernel(const __grid_c
           for (int r = 0; r < 2; ++r) {
             const int x = 2 * q + r;
             const float g = e32[r];
-            S[x] = g * fmaf(g, S[x], ds[x]);
-            sm.opS[op_off(jcol + 4 * q, drow + 8 * r)] = g * S[x];
+            if (fastT[r]) {
+              S[x] = fmaf(g * g, S[x], ds[x]);
+              sm.opS[op_off(jcol + 4 * q, drow + 8 * r)] = S[x];
+            } else {
+              S[x] = g * fmaf(g, S[x], ds[x]);
+              sm.opS[op_off(jcol + 4 * q, drow + 8 * r)] = g * S[x];
+            }
           }
       } else {  // last, partial chunk: no later chunk reads opS
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
           const float rate = expf(om[drow + 8 * r]);
-          const float dl = expf(-rate * (float)cnt), gs = expf(-rate * (float)(cnt - 32));
+          const float dl = expf(-rate * (float)cnt), gs = fastT[r] ? 1.f : expf(-rate * (float)(cnt - 32));
 #pragma unroll
           for (int q = 0; q < 8; ++q) S[2 * q + r] = fmaf(dl, S[2 * q + r], gs * ds[2 * q + r]);
         }
@@ -449,7 +553,7 @@ __global__ void __launch_bounds__(kThreads, 2) wkv5_fwd_tc_kernel(const __grid_c
     // a wait gave up at chunk c: the previous chunk's MMA chains (committed last on bar_av) and
     // this chunk's loads must finish before the tensor memory and shared memory are released,
     // each wait bounded again
-    if (c >= 1 && !fast) mbar_wait_bounded(&sm.bar_av, (uint32_t)(c - 1) & 1u, p.ctl);
+    if (c >= 1) mbar_wait_bounded(&sm.bar_av, (uint32_t)(c - 1) & 1u, p.ctl);
     if (!withheld) mbar_wait_bounded(&sm.bar_tma, (uint32_t)c & 1u, p.ctl);
   }
   if (p.s_out != nullptr) {

@@ -18,8 +18,9 @@
 // kernel's three tensor-core chains
 //   [A | Y] = r̃ [k̃ ; e^{R} Sᵀ]ᵀ,   Y += A_masked v,   ΔS = k̃ᵀ v
 // (the Eagle kernel is the case Λ_τ = λ (τ + 1), R = Λ_31).  Any R gives the
-// same products; every factor stays in fp32 range while -R and R - Λ_last
-// are at most 80 in every channel.  The first chunk takes R = Λ_31, the middle
+// same products; every factor stays within e^{±64} while -R and R - Λ_last
+// are at most 64 in every channel (wider factors would push small operands
+// into the subnormal range, where a tf32 operand keeps few bits).  The first chunk takes R = Λ_31, the middle
 // of its own decay; every later chunk takes half the log-decay of the chunk
 // before it (the middle again while the decay rate holds), which is known when
 // the previous chunk folds its state, so that fold also writes e^{R} ⊙ Sᵀ for
@@ -56,7 +57,7 @@ constexpr int kL = 64;                      // tokens per chunk
 constexpr int kThreads = 256;
 constexpr uint32_t kRawBytes = kL * kN * 2;  // one bf16 [64 x 64] box
 constexpr uint32_t kOmBytes = kL * 32 * 4;   // one fp32 [64 tokens x 32 channels] box
-constexpr float kMaxHalfDecay = 80.f;       // largest log-decay of half a chunk the factorization accepts
+constexpr float kMaxHalfDecay = 64.f;       // largest log-decay of half a chunk the factorization takes
 constexpr uint32_t kTmemCols = 256;         // [scores | output rows], state increment, k̃ᵀ
 
 struct Wkv6Smem {
@@ -258,8 +259,9 @@ __global__ void __launch_bounds__(kThreads, 2) wkv6_fwd_tc_kernel(const __grid_c
         const int row = 8 * ib + rr;
         const float fr0 = __expf(lin[ib][0] - lam[ib][0] - R[0]), fr1 = __expf(lin[ib][1] - lam[ib][1] - R[1]);
         const float fk0 = __expf(R[0] - lin[ib][0]), fk1 = __expf(R[1] - lin[ib][1]);
-        *reinterpret_cast<float2*>(&sm.opRA[op_off(row, dR)]) = make_float2(rv.x * fr0, rv.y * fr1);
-        *reinterpret_cast<float2*>(&sm.opK[op_off(row, dR)]) = make_float2(kv.x * fk0, kv.y * fk1);
+        // rounded to nearest tf32: truncation by the tensor core would bias both factors of every score
+        *reinterpret_cast<float2*>(&sm.opRA[op_off(row, dR)]) = make_float2(to_tf32(rv.x * fr0), to_tf32(rv.y * fr1));
+        *reinterpret_cast<float2*>(&sm.opK[op_off(row, dR)]) = make_float2(to_tf32(kv.x * fk0), to_tf32(kv.y * fk1));
         part[ib] = fmaf(rv.x * uA[0], kv.x, rv.y * uA[1] * kv.y);
       }
 #pragma unroll

@@ -49,9 +49,9 @@ def test_backward_small(cuda_device, shape, states):
     _check(out, ref)
 
 
-@pytest.mark.parametrize("omega_range", [(-8.0, -4.0), (-3.0, 0.9), (0.5, 0.9)])
+@pytest.mark.parametrize("omega_range", [(-8.0, -4.0), (-3.0, 0.69), (0.3, 0.69)])
 def test_backward_decay_ranges(cuda_device, omega_range):
-    # slow, mixed and fast decays (exp(omega) up to 2.46, inside the chunked factorization's range)
+    # slow, mixed and fast decays (exp(omega) up to 1.99, inside the chunked factorization's range)
     p = wi.wkv5_problem(2, 150, 3, 64, seed=82, omega_range=omega_range)
     g = wi.wkv5_grads(2, 150, 3, 64, seed=83, states=True)
     out, ref = _run(p, g, cuda_device, True)
@@ -59,7 +59,7 @@ def test_backward_decay_ranges(cuda_device, omega_range):
 
 
 def test_backward_fast_decay_is_reported(cuda_device):
-    # exp(omega) above 2.5 in some channel: outside the backward's range, reported, not computed
+    # exp(omega) above 2 in some channel: outside the backward's range, reported, not computed
     p = wi.wkv5_problem(1, 70, 2, 64, seed=84, omega_range=(-1.0, 2.0))
     g = wi.wkv5_grads(1, 70, 2, 64, seed=85)
     c = {k: v.to(cuda_device) for k, v in p.items()}
