@@ -153,7 +153,8 @@ class ClockSampler:
 # kernel name in profiles/traffic.json -> prefix of the source files it is built from
 _TRAFFIC_SOURCES = {"wkv4_bwd_kernel": "wkv4_bwd", "wkv5_fwd_tc_kernel": "wkv5_fwd", "wkv4_step_kernel": "wkv4_step",
                     "wkv5_step_kernel": "wkv5_step", "wkv6_fwd_tc_kernel": "wkv6_fwd",
-                    "wkv5_step_kernel/finch": "wkv5_step", "wkv4_bwd_kernel/gated": "wkv4_bwd"}
+                    "wkv5_step_kernel/finch": "wkv5_step", "wkv4_bwd_kernel/gated": "wkv4_bwd",
+                    "rwkv_wkv5_backward": ("wkv5_fwd", "wkv5_bwd")}
 
 
 def _kernel_source_hash(kernel="wkv4_bwd_kernel"):
@@ -161,9 +162,10 @@ def _kernel_source_hash(kernel="wkv4_bwd_kernel"):
 
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "rwkv_wkv_recurrence_b200", "csrc")
-    prefix = _TRAFFIC_SOURCES[kernel]
+    prefixes = _TRAFFIC_SOURCES[kernel]
+    units = {p + ".cu" for p in ((prefixes,) if isinstance(prefixes, str) else prefixes)}
     for f in sorted(os.listdir(csrc)):
-        if f == prefix + ".cu" or f.endswith(".cuh") or f == "launch.h":
+        if f in units or f.endswith(".cuh") or f == "launch.h":
             with open(os.path.join(csrc, f), "rb") as fh:
                 h.update(fh.read())
     return h.hexdigest()[:16]
@@ -774,7 +776,9 @@ def run_eagle(args, finch=False):
         "higher_is_better": True, "dtype": "bf16 I/O, fp32 state", "data": "synthetic",
         "config": {"workload": workload, "l2": l2},
         "roofline": {"bound": "hbm", "kernel": kernel, "achieved": gbs, "peak": peak, "peak_kind": kind,
-                     "unit": "GB/s", "frac": gbs / peak, "traffic": _recorded_traffic(kernel)},
+                     "unit": "GB/s", "frac": gbs / peak,
+                     # the capture was taken on the default decay range
+                     "traffic": _recorded_traffic(kernel) if (om_lo, om_hi) == (-6.0, 0.0) else None},
         "gpu_launches": args.steps, "clocks": clk, "call_ms": stats}), flush=True)
 
 
@@ -822,7 +826,7 @@ def run_eagle_backward(args):
                    "l2": "no flush: 587 MB moved per call, above the 126 MB L2"},
         "roofline": {"bound": "hbm", "kernel": "rwkv_wkv5_backward (reversed forward + two backward passes + "
                                                "reduction)", "achieved": gbs, "peak": peak, "peak_kind": kind,
-                     "unit": "GB/s", "frac": gbs / peak, "traffic": None},
+                     "unit": "GB/s", "frac": gbs / peak, "traffic": _recorded_traffic("rwkv_wkv5_backward")},
         "gpu_launches": 4 * args.steps, "clocks": clk, "call_ms": stats}), flush=True)
 
 
