@@ -85,10 +85,11 @@ struct Wkv5Smem {
     float AF[kL][kBand + 1];         // the fast channels' scores [τ][n = τ-1-ι], T1b (after the
   } u;                               // bonus sums) -> T2a
   float diag[kL];                    // Σ_d r u k per token
-  // fast channels: r and k as bf16 pairs of fast indices, word w of row x at column w ^ (x & 31)
-  // (lanes on different rows meet different banks)
-  uint32_t RFw[kL][kN / 2];
-  uint32_t KFw[kL][kN / 2];
+  // fast channels: r and k as bf16 pairs of fast indices [position][pair], rows padded to 33 words
+  // (lanes on different rows meet different banks); KFw's extra row is zero: the k row of a lag
+  // that reaches before the chunk
+  uint32_t RFw[kL][kN / 2 + 1];
+  uint32_t KFw[kL + 1][kN / 2 + 1];
   alignas(16) float E4[kN][4];           // e^{λ n} for n = 0, 4, 8, 12 [fast index][n / 4]
   float E1[kN];                          // e^{λ} [fast index]
   int fidx[kN];                          // fast index of each key channel, -1 for a slow one
@@ -131,8 +132,8 @@ __global__ void __launch_bounds__(kThreads, 2) wkv5_fwd_tc_kernel(const __grid_c
   // products only where the factor stays at most 1 (state read e^{λτ}, state increment
   // e^{λ(cnt-1-ι)}); their intra-chunk scores are summed on the CUDA cores over lags 0..kBand.
   if (tid == 0) sm.abort_flag = 0;
-  for (int i = tid; i < kL * kN / 2; i += kThreads) {
-    (&sm.RFw[0][0])[i] = 0u;
+  for (int i = tid; i < (kL + 1) * (kN / 2 + 1); i += kThreads) {
+    if (i < kL * (kN / 2 + 1)) (&sm.RFw[0][0])[i] = 0u;
     (&sm.KFw[0][0])[i] = 0u;
   }
   if (tid < kN) {
@@ -296,7 +297,7 @@ __global__ void __launch_bounds__(kThreads, 2) wkv5_fwd_tc_kernel(const __grid_c
 #pragma unroll
         for (int e = 0; e < 2; ++e)
           if (fiA[e] >= 0) {
-            const int col = ((fiA[e] >> 1) ^ (row & 31));
+            const int col = fiA[e] >> 1;
             unsigned short* rh = reinterpret_cast<unsigned short*>(&sm.RFw[row][col]) + (fiA[e] & 1);
             unsigned short* kh = reinterpret_cast<unsigned short*>(&sm.KFw[row][col]) + (fiA[e] & 1);
             *rh = (unsigned short)(e ? rw >> 16 : rw & 0xFFFFu);
@@ -354,14 +355,19 @@ __global__ void __launch_bounds__(kThreads, 2) wkv5_fwd_tc_kernel(const __grid_c
         // (τ, 4 lags), every CTA thread busy; AF overlays the bonus parts, summed above
         __syncthreads();
         const int tau = tid >> 2, g4 = tid & 3, n0 = 4 * g4;
-        int rk[4];
+        // k rows of the four lags (a lag reaching before the chunk reads the zero row)
+        const uint32_t* kp[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) rk[e] = tau - 1 - (n0 + e);  // ι of lag n0 + e (negative: none)
+        for (int e = 0; e < 4; ++e) {
+          const int io = tau - 1 - (n0 + e);
+          kp[e] = &sm.KFw[io < 0 ? kL : io][0];
+        }
+        const uint32_t* rp = &sm.RFw[tau][0];
         float acc[4] = {0.f, 0.f, 0.f, 0.f};
         const int npair = (nfast + 1) >> 1;
 #pragma unroll 2
         for (int w = 0; w < npair; ++w) {
-          const float2 rv = bf2_to_f2(sm.RFw[tau][w ^ (tau & 31)]);
+          const float2 rv = bf2_to_f2(rp[w]);
           float ew[2][4];
 #pragma unroll
           for (int h2 = 0; h2 < 2; ++h2) {
@@ -374,11 +380,9 @@ __global__ void __launch_bounds__(kThreads, 2) wkv5_fwd_tc_kernel(const __grid_c
           }
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            if (rk[e] >= 0) {
-              const float2 kv = bf2_to_f2(sm.KFw[rk[e]][w ^ (rk[e] & 31)]);
-              acc[e] = fmaf(rv.x * kv.x, ew[0][e], acc[e]);
-              acc[e] = fmaf(rv.y * kv.y, ew[1][e], acc[e]);
-            }
+            const float2 kv = bf2_to_f2(kp[e][w]);
+            acc[e] = fmaf(rv.x * kv.x, ew[0][e], acc[e]);
+            acc[e] = fmaf(rv.y * kv.y, ew[1][e], acc[e]);
           }
         }
 #pragma unroll
