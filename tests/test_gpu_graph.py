@@ -70,3 +70,35 @@ def test_matrix_state_step_graph(cuda_device, finch):
 
     run.init = lambda: s0.clone()
     _replay_equals_eager(cuda_device, run)
+
+
+@pytest.mark.parametrize("with_state", [False, True])
+def test_eagle_forward_and_backward_graph(cuda_device, with_state):
+    # the Eagle forward and backward (whose reversed forward pass runs on a side stream, forked
+    # and joined with events) captured in one graph, replayed: bit for bit the eager results
+    B, T, H = 2, 150, 3
+    p = {k: v.to(cuda_device) for k, v in wi.wkv5_problem(B, T, H, 64, seed=63).items()}
+    g = {k: v.to(cuda_device) for k, v in wi.wkv5_grads(B, T, H, 64, seed=64, states=with_state).items()}
+
+    def run():
+        y = rw.rwkv_wkv5_forward(p["r"], p["k"], p["v"], p["omega"], p["u"], g.get("s_in"),
+                                 stream=torch.cuda.current_stream())
+        grads = rw.rwkv_wkv5_backward(p["r"], p["k"], p["v"], p["omega"], p["u"], g["gy"], g.get("s_in"),
+                                      g.get("gs_out"), want_gs_in=True, stream=torch.cuda.current_stream())
+        return (y,) + tuple(grads)
+
+    eager = run()
+    torch.cuda.synchronize()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        run()  # warm-up on a side stream, as capture requires
+    torch.cuda.current_stream().wait_stream(side)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        captured = run()
+    graph.replay()
+    torch.cuda.synchronize()
+    rw.rwkv_check_device_error()
+    for a, b in zip(eager, captured):
+        assert torch.equal(a, b)
