@@ -794,7 +794,8 @@ def run_eagle_backward(args):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     Be, Te, He, Ne = 4, 4096, 40, 64
-    q = wi.wkv5_problem(Be, Te, He, Ne, seed=SEED + 2, device=dev)
+    om_lo, om_hi = _omega_range(args)
+    q = wi.wkv5_problem(Be, Te, He, Ne, seed=SEED + 2, device=dev, omega_range=(om_lo, om_hi))
     g = wi.wkv5_grads(Be, Te, He, Ne, seed=SEED + 6, device=dev)
     gr, gk, gv = (torch.empty_like(q["r"]) for _ in range(3))
     gom, gu = torch.empty(He, Ne, device=dev), torch.empty(He, Ne, device=dev)
@@ -822,11 +823,13 @@ def run_eagle_backward(args):
         "unit": "elements/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "dtype": "bf16 I/O, fp32 state", "data": "synthetic",
         "config": {"workload": "Eagle / RWKV-5 WKV backward, B=4 T=4096 H=40 N=64, bf16 r,k,v,gy,gr,gk,gv, "
-                               "gy ~ N(0,1), zero initial state, no final-state gradient",
+                               "gy ~ N(0,1), zero initial state, no final-state gradient"
+                               + ("" if (om_lo, om_hi) == (-6.0, 0.0) else f", omega U({om_lo:g},{om_hi:g})"),
                    "l2": "no flush: 587 MB moved per call, above the 126 MB L2"},
         "roofline": {"bound": "hbm", "kernel": "rwkv_wkv5_backward (reversed forward + two backward passes + "
                                                "reduction)", "achieved": gbs, "peak": peak, "peak_kind": kind,
-                     "unit": "GB/s", "frac": gbs / peak, "traffic": _recorded_traffic("rwkv_wkv5_backward")},
+                     "unit": "GB/s", "frac": gbs / peak,
+                     "traffic": _recorded_traffic("rwkv_wkv5_backward") if (om_lo, om_hi) == (-6.0, 0.0) else None},
         "gpu_launches": 4 * args.steps, "clocks": clk, "call_ms": stats}), flush=True)
 
 

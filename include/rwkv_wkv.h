@@ -228,10 +228,12 @@ RWKV_API size_t rwkv_wkv5_backward_workspace_bytes(int64_t B, int64_t T, int64_t
  *   workspace     device scratch of rwkv_wkv5_backward_workspace_bytes() bytes (the forward
  *                 states at every 64th token, per-row sums).
  *   N must be 64; the [B,T,H,N] tensors 16-byte aligned (RWKV_ERR_UNSUPPORTED otherwise).
- *   A channel decaying faster than exp(omega) = 2 (w < 0.135) is outside the
- *   range this backward computes: the call returns RWKV_OK, the outputs of
- *   that channel's heads are undefined, and rwkv_check_device_error reports
- *   RWKV_ERR_UNSUPPORTED.  Deterministic.
+ *   Any decay w in [0, 1]: channels decaying faster than exp(omega) = 2
+ *   (w < 0.135) are summed over lags up to 15 where the rest stays on the
+ *   chunked tensor-core form.  The reversed forward pass (gv, gs_in) runs on an
+ *   internal non-blocking stream per device, ordered after and before the
+ *   caller's stream with events (capture-safe once a first call has made it).
+ *   Deterministic.
  */
 RWKV_API rwkv_status rwkv_wkv5_backward(int64_t B, int64_t T, int64_t H, int64_t N, const void *r, const void *k,
                                const void *v, const float *omega, const float *u, const float *s_in,
@@ -327,8 +329,7 @@ RWKV_API rwkv_status rwkv_wkv4_backward_noalloc(int64_t B, int64_t T, int64_t C,
 
 /*
  * Synchronises `stream`, then reports and clears the device error word that
- * kernels set when a bounded wait gives up (RWKV_ERR_DEVICE_TIMEOUT) or when
- * a backward met a decay outside its range (RWKV_ERR_UNSUPPORTED), or
+ * kernels set when a bounded wait gives up (RWKV_ERR_DEVICE_TIMEOUT), or
  * RWKV_ERR_CUDA if the stream itself failed.
  * The error word is one per device and process, shared by every call on that
  * device whatever its stream or host thread: a timeout in work on one stream

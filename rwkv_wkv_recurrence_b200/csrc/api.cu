@@ -807,7 +807,7 @@ rwkv_status rwkv_check_device_error(rwkv_stream_t stream) {
   if (v != 0) {
     const unsigned int zero = 0;
     if (cudaMemcpyToSymbol(g_ctl, &zero, sizeof(zero), offsetof(DevCtl, err)) != cudaSuccess) return RWKV_ERR_CUDA;
-    return (v & kErrTmaTimeout) ? RWKV_ERR_DEVICE_TIMEOUT : RWKV_ERR_UNSUPPORTED;
+    return RWKV_ERR_DEVICE_TIMEOUT;  // the one condition a kernel reports there
   }
   return RWKV_OK;
 }

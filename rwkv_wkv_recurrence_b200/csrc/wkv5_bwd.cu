@@ -53,12 +53,18 @@
 // each checkpoint in the tf32 operand layout, so the reversed pass brings it in with one bulk copy a
 // chunk ahead.
 //
-// CTA: one (batch, head), 8 warps.  Forward pass: ~105 KB of shared memory,
-// 256 TMEM columns, two CTAs per SM.  Reversed pass: ~140 KB, 512 columns, one
-// CTA per SM.  A head with some channel decaying faster than the chunked
-// factorization takes (exp(ω) > 2: factors beyond e^{±64} would push small
-// operands into the subnormal range) is not handled: the kernel sets
-// kErrFastDecay in the device error word and leaves that head's outputs unset.
+// Fast rows.  A key row decaying faster than the factorization takes (exp(ω) > 2:
+// factors beyond e^{±64} would push small operands into the subnormal range)
+// stays out of the factorized products: its c̃ᵀ row is zero, its state row is
+// read unscaled and its output takes e^{λ(τ-lo)}.  Its intra-chunk terms (the
+// plain one and, reversed, the lag-weighted one) are summed on the CUDA cores in
+// the epilogue over lags 0..15, from the masked scores and the staged c rows,
+// and its state increment in the fold over the chunk's last 16 positions:
+// beyond that e^{λn} < 2^-46 of the lag-0 weight.  Any w in [0, 1] is handled.
+//
+// CTA: one (batch, head), 8 warps.  Forward pass: ~110 KB of shared memory,
+// 256 TMEM columns, two CTAs per SM.  Reversed pass: ~145 KB, 512 columns, one
+// CTA per SM.
 #include <cstddef>
 
 #include "launch.h"
@@ -74,7 +80,8 @@ constexpr int kN = 64;
 constexpr int kL = 64;
 constexpr int kThreads = 256;
 constexpr uint32_t kRawBytes = kL * kN * 2;
-constexpr float kMaxRate = 2.f;
+constexpr float kMaxRate = 2.f;  // largest rate the chunked factorization takes
+constexpr int kBand = 15;         // lags a fast row keeps: e^{-2 (kBand+1)} < 2^-46
 constexpr uint32_t kCkBytes = kN * kN * 4;  // one forward-state checkpoint (fp32, operand layout)
 
 struct Wkv5BwdSmem {
@@ -85,19 +92,23 @@ struct Wkv5BwdSmem {
   alignas(128) float opPt[64 * 64];  // pᵀ [j][ι]: B of the state increment
   alignas(128) float opAm[64 * 64];  // strictly causal scores [τ][ι]: B of the intra term
   float diag[kL];                    // A[τ][τ] = q_τ·p_τ
+  float EB[kBand + 1][kN];           // e^{λ_d n} [n][key row d], n = 0..kBand (fast rows)
   alignas(8) uint64_t bar_tma;
   alignas(8) uint64_t bar_sc;        // scores and state read (and the X_c read) done
   alignas(8) uint64_t bar_av;        // intra term (and the lag-weighted term) done
   alignas(8) uint64_t bar_ds;        // state increment done
   alignas(8) uint64_t bar_ck;        // reversed pass: the forward state X_c has arrived in opXc
   uint32_t tmem_base;
-  int slow;
   int abort_flag;
   // reversed pass only (not part of the forward pass's shared memory)
   alignas(128) float opXc[64 * 64];  // forward state X_c [d][j]: A of the X_c read (bulk-copied)
   alignas(128) float opAl[64 * 64];  // lag-weighted scores (τ-1-ι) A [τ][ι]: B of the lag term
   double red[kN];                    // per key row: the decay-gradient sum of this CTA
 };
+
+// dynamic shared memory = the struct (or its forward-pass prefix) + 1024 bytes of alignment slack;
+// an SM has 228 KB, of which each resident CTA also takes 1 KB: two forward-pass CTAs per SM
+static_assert(2 * (offsetof(Wkv5BwdSmem, opXc) + 1024 + 1024) <= 228 * 1024, "two CTAs per SM");
 
 size_t bwd_smem_bytes(bool rev) {
   return (rev ? sizeof(Wkv5BwdSmem) : offsetof(Wkv5BwdSmem, opXc)) + 1024;  // + alignment slack
@@ -125,20 +136,20 @@ __global__ void __launch_bounds__(kThreads, REV ? 1 : 2) wkv5_bwd_tc_kernel(cons
   const float* om = p.omega + h * kN;
   const size_t sbase = ((size_t)b * p.H + h) * kN * kN;
 
-  if (tid == 0) {
-    sm.slow = 0;
-    sm.abort_flag = 0;
-  }
+  if (tid == 0) sm.abort_flag = 0;
   if constexpr (REV) {
     if (tid < kN) sm.red[tid] = 0.0;
   }
-  __syncthreads();
-  if (tid < kN && !(expf(om[tid]) <= kMaxRate)) atomicOr(&sm.slow, 1);
-  __syncthreads();
-  if (sm.slow) {  // outside the chunked factorization's range: reported, not computed
-    if (tid == 0) atomicOr(&p.ctl->err, kErrFastDecay);
-    return;
+  // fast rows (rate > 2) stay out of the factorized products (their c̃ᵀ row is zero); their
+  // intra-chunk terms and state increment are summed on the CUDA cores over lags 0..kBand
+  bool fast_any = false;
+  if (tid < kN) {
+    const float lam = -expf(om[tid]);
+    fast_any = !(-lam <= kMaxRate);
+#pragma unroll 1
+    for (int n = 0; n <= kBand; ++n) sm.EB[n][tid] = n == 0 ? 1.f : expf(lam * (float)n);
   }
+  const bool nfast = __syncthreads_or(fast_any) != 0;
 
   if (warp == 0) tmem_alloc(&sm.tmem_base, REV ? 512u : 256u);
   const bool withheld = tid == 0 && loads_withheld(p.ctl);
@@ -187,9 +198,10 @@ __global__ void __launch_bounds__(kThreads, REV ? 1 : 2) wkv5_bwd_tc_kernel(cons
 #pragma unroll
   for (int r = 0; r < 2; ++r) {
     const float rate = expf(om[16 * q4 + 8 * r + t4]);
+    const bool fr = !(rate <= kMaxRate);  // a fast row: zero, its terms are formed elsewhere
 #pragma unroll
-    for (int e = 0; e < 2; ++e) fc0[r][e] = expf(-rate * (float)(31 - 32 * hc - 2 * tq - e));
-    fcs[r] = expf(8.f * rate);
+    for (int e = 0; e < 2; ++e) fc0[r][e] = fr ? 0.f : expf(-rate * (float)(31 - 32 * hc - 2 * tq - e));
+    fcs[r] = fr ? 0.f : expf(8.f * rate);
   }
   const uint32_t offKt =
       REV ? (uint32_t)(63 - (4 * hc + (lmat >> 1)) * 8 - lrow) * 128u + (uint32_t)(((2 * q4 + (lmat & 1)) ^ (7 - lrow)) << 4)
@@ -201,10 +213,12 @@ __global__ void __launch_bounds__(kThreads, REV ? 1 : 2) wkv5_bwd_tc_kernel(cons
   const int jcol = 32 * hc + tq;
   const uint32_t tquar = (uint32_t)(32 * q4) << 16;
   float lamr[2], e32[2];
+  bool fastR[2];
 #pragma unroll
   for (int r = 0; r < 2; ++r) {
     lamr[r] = -expf(om[drow + 8 * r]);
     e32[r] = expf(32.f * lamr[r]);
+    fastR[r] = !(-lamr[r] <= kMaxRate);
   }
   float X[16];
 #pragma unroll
@@ -215,7 +229,8 @@ __global__ void __launch_bounds__(kThreads, REV ? 1 : 2) wkv5_bwd_tc_kernel(cons
   // the carried state enters at position `lead` of the first chunk: its read factor is e^{(32-lead)λ}
 #pragma unroll
   for (int r = 0; r < 2; ++r) {
-    const float f0 = expf((32.f - (float)p.lead) * lamr[r]);
+    // (a fast row is read unscaled: its factor e^{λ(τ-lo)} is applied to the output)
+    const float f0 = fastR[r] ? 1.f : expf((32.f - (float)p.lead) * lamr[r]);
 #pragma unroll
     for (int q = 0; q < 8; ++q) sm.opX[op_off(drow + 8 * r, jcol + 4 * q)] = to_tf32(f0 * X[2 * q + r]);
   }
@@ -223,6 +238,7 @@ __global__ void __launch_bounds__(kThreads, REV ? 1 : 2) wkv5_bwd_tc_kernel(cons
   // ---- epilogue rows: lane < 16 of quarter q4 holds key row de = 16 q4 + lane, positions 32 hc + i
   const int de = 16 * q4 + (lane & 15);
   const float lam_e = -expf(om[de]);
+  const bool fast_e = !(-lam_e <= kMaxRate);
   const float u_e = p.u[h * kN + de];
   double acc_e = 0.0;              // forward pass: the gu sum of row de; reversed: its decay-gradient terms
   double acc_t1[2] = {0.0, 0.0};   // reversed pass: the elementwise term of rows drow, drow + 8
@@ -238,6 +254,9 @@ __global__ void __launch_bounds__(kThreads, REV ? 1 : 2) wkv5_bwd_tc_kernel(cons
   // the next chunk's conversion
   __nv_bfloat16* stC = reinterpret_cast<__nv_bfloat16*>(sm.opQ);
   __nv_bfloat16* stM = stC + kL * kN;
+  // the output rows, in opP (free from the first chains' end to the next chunk's conversion), so
+  // that c stays readable for the fast rows' terms
+  __nv_bfloat16* stO = reinterpret_cast<__nv_bfloat16*>(sm.opP);
   const bool issuer = tid == 0;
 
   int c = 0;
@@ -286,7 +305,7 @@ __global__ void __launch_bounds__(kThreads, REV ? 1 : 2) wkv5_bwd_tc_kernel(cons
         }
       const float n = (float)(kL - lo);
 #pragma unroll
-      for (int r = 0; r < 2; ++r) acc_t1[r] += (double)(n * expf((n - 1.f) * lamr[r]) * part[r]);
+      for (int r = 0; r < 2; ++r) acc_t1[r] += (double)(n * (n == 1.f ? 1.f : expf((n - 1.f) * lamr[r])) * part[r]);
     }
 
     if (!mbar_wait_bounded(&sm.bar_tma, ph, p.ctl)) sm.abort_flag = 1;
@@ -456,6 +475,31 @@ __global__ void __launch_bounds__(kThreads, REV ? 1 : 2) wkv5_bwd_tc_kernel(cons
             sm.opX[op_off(drow + 8 * r, jcol + 4 * q)] = to_tf32(e32[r] * X[x]);
           }
         }
+        if (nfast) {
+#pragma unroll
+          for (int r = 0; r < 2; ++r) {  // unrolled: X stays in registers
+            if (!fastR[r]) continue;
+            // a fast row (its tensor-core increment is zero): Σ_ι c_ι[d] e^{λ(63-ι)} p_ι[j] over the
+            // chunk's last kBand + 1 positions, and the row read unscaled
+            const int d = drow + 8 * r;
+            float dsf[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int n = 0; n <= kBand; ++n) {
+              const int io = kL - 1 - n;
+              if (io >= lo) {
+                const float cw = __bfloat162float(stC[(REV ? kL - 1 - io : io) * kN + d]) * sm.EB[n][d];
+#pragma unroll
+                for (int q = 0; q < 8; ++q) dsf[q] = fmaf(cw, sm.opPt[op_off(jcol + 4 * q, io)], dsf[q]);
+              }
+            }
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              const int x = 2 * q + r;
+              X[x] += dsf[q];
+              sm.opX[op_off(d, jcol + 4 * q)] = to_tf32(X[x]);
+            }
+          }
+        }
       } else {  // partial last chunk (forward pass): no later chunk reads opX
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
@@ -485,7 +529,7 @@ __global__ void __launch_bounds__(kThreads, REV ? 1 : 2) wkv5_bwd_tc_kernel(cons
         for (int i = 0; i < 16; ++i) {
           const int pos = (int)col + i;
           if (pos < lo || pos >= cnt) continue;
-          // staging row of this position (the box holds the tokens in forward order); out replaces c
+          // staging row of this position (the box holds the tokens in forward order)
           const int so = (REV ? kL - 1 - pos : pos) * kN + de;
           const float cval = __bfloat162float(stC[so]), mval = __bfloat162float(stM[so]);
           const float dg = sm.diag[pos];
@@ -494,9 +538,9 @@ __global__ void __launch_bounds__(kThreads, REV ? 1 : 2) wkv5_bwd_tc_kernel(cons
           if constexpr (REV) o = f * (zv[i] + iv[i]);
           else o = f * zv[i];
           o = fmaf(u_e * cval, dg, o);
-          stC[so] = __float2bfloat16_rn(o);
           if constexpr (REV) {
-            // position-weighted state read, lag-weighted intra term, and the X_c read
+            // position-weighted state read, lag-weighted intra term, and the X_c read (for a fast row
+            // these are not its sums, which are formed below; its acc is dropped after the loop)
             const float f1 = __expf(lam_e * (float)(pos - 33));
             const float f3 = pos < kL - 1 ? (float)(kL - 1 - pos) * __expf(lam_e * (float)(kL - 2 - pos)) : 0.f;
             acc = fmaf(mval * f1, fmaf((float)(pos - lo), zv[i], x4[i]), acc);
@@ -504,8 +548,53 @@ __global__ void __launch_bounds__(kThreads, REV ? 1 : 2) wkv5_bwd_tc_kernel(cons
           } else {
             acc = fmaf(mval * cval, dg, acc);  // gu: r k (v·gy)
           }
+          stO[so] = __float2bfloat16_rn(o);
         }
-        acc_e += (double)acc;
+        if (nfast && fast_e) {
+          // a fast row: the state read (unscaled) times e^{λ(pos-lo)}, and the intra-chunk terms over
+          // lags n = 0..kBand, Σ_n A[pos][pos-1-n] c_{pos-1-n} e^{λn} (and, reversed, the lag-weighted
+          // Σ_n n A c e^{λ(n-1)}), from the masked scores and the staged c rows
+          float accf = 0.f;
+#pragma unroll 1
+          for (int i = 0; i < 16; ++i) {
+            const int pos = (int)col + i;
+            if (pos < lo || pos >= cnt) continue;
+            float zi = 0.f, x3i = 0.f;  // zv[i], x3[i] by selects: the arrays stay in registers
+#pragma unroll
+            for (int t = 0; t < 16; ++t) {
+              if (t == i) {
+                zi = zv[t];
+                if constexpr (REV) x3i = x3[t];
+              }
+            }
+            const int so = (REV ? kL - 1 - pos : pos) * kN + de;
+            const float cval = __bfloat162float(stC[so]), mval = __bfloat162float(stM[so]);
+            float b0 = 0.f, b1 = 0.f;
+#pragma unroll
+            for (int n = 0; n <= kBand; ++n) {
+              const int io = pos - 1 - n;
+              if (io >= lo) {
+                const float ac =
+                    sm.opAm[op_off(pos, io)] * __bfloat162float(stC[(REV ? kL - 1 - io : io) * kN + de]);
+                b0 = fmaf(ac, sm.EB[n][de], b0);
+                if constexpr (REV) {
+                  if (n >= 1) b1 = fmaf((float)n * ac, sm.EB[n - 1][de], b1);
+                }
+              }
+            }
+            const float fr = pos == lo ? 1.f : __expf(lam_e * (float)(pos - lo));
+            stO[so] = __float2bfloat16_rn(fmaf(u_e * cval, sm.diag[pos], fmaf(fr, zi, b0)));
+            if constexpr (REV) {
+              const float fz = pos > lo ? (float)(pos - lo) * __expf(lam_e * (float)(pos - 1 - lo)) : 0.f;
+              const float f3 = pos < kL - 1 ? (float)(kL - 1 - pos) * __expf(lam_e * (float)(kL - 2 - pos)) : 0.f;
+              accf = fmaf(mval, fmaf(fz, zi, b1), accf);
+              accf = fmaf(f3 * cval, x3i, accf);
+            }
+          }
+          acc_e += (double)accf;
+        }
+        if constexpr (REV) acc_e += fast_e ? 0.0 : (double)acc;  // (the gu sum has no decay factor)
+        else acc_e += (double)acc;
       }
     }
     // the chunk's out rows, 16 bytes a thread
@@ -515,7 +604,7 @@ __global__ void __launch_bounds__(kThreads, REV ? 1 : 2) wkv5_bwd_tc_kernel(cons
       const int row = 32 * hh + (tid >> 3);
       if (row < nrow)
         *reinterpret_cast<uint4*>(p.out + (((size_t)b * p.T + tb + row) * p.H + h) * kN + 8 * (tid & 7)) =
-            *reinterpret_cast<const uint4*>(&stC[row * kN + 8 * (tid & 7)]);
+            *reinterpret_cast<const uint4*>(&stO[row * kN + 8 * (tid & 7)]);
     }
 
     __syncthreads();  // the staging rows (opQ) are read out before the next chunk converts q into it

@@ -136,6 +136,11 @@ __global__ void __launch_bounds__(kThreads, 2) wkv5_fwd_tc_kernel(const __grid_c
     if (i < kL * (kN / 2 + 1)) (&sm.RFw[0][0])[i] = 0u;
     (&sm.KFw[0][0])[i] = 0u;
   }
+  if (tid < kN) {  // the weights of an odd count's padding channel must read as zero too
+#pragma unroll
+    for (int g = 0; g < 4; ++g) sm.E4[tid][g] = 0.f;
+    sm.E1[tid] = 0.f;
+  }
   if (tid < kN) {
     const bool f = !(expf(om[tid]) <= kMaxRate);
     const unsigned m = __ballot_sync(0xffffffffu, f);

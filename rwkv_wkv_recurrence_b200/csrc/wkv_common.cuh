@@ -19,13 +19,9 @@
 
 namespace rwkv {
 
-
 // Bit set in the library's device error word when a bounded wait gives up.
 // Read and cleared by rwkv_check_device_error().
 constexpr unsigned int kErrTmaTimeout = 1u;
-// Bit set when a kernel met a decay outside the range it computes (reported
-// by rwkv_check_device_error as RWKV_ERR_UNSUPPORTED).
-constexpr unsigned int kErrFastDecay = 2u;
 
 // Default limit of a bounded wait.  A TMA load or an MMA chain completes in
 // microseconds; a wait that lasts this long means its arrival will not come.

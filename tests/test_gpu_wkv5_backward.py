@@ -49,23 +49,24 @@ def test_backward_small(cuda_device, shape, states):
     _check(out, ref)
 
 
-@pytest.mark.parametrize("omega_range", [(-8.0, -4.0), (-3.0, 0.69), (0.3, 0.69)])
+@pytest.mark.parametrize("omega_range", [(-8.0, -4.0), (-3.0, 0.69), (0.3, 0.69), (-1.0, 2.0), (0.7, 2.0), (2.0, 3.0)])
 def test_backward_decay_ranges(cuda_device, omega_range):
-    # slow, mixed and fast decays (exp(omega) up to 1.99, inside the chunked factorization's range)
+    # slow, mixed and fast decays: exp(omega) up to 1.99 inside the chunked factorization's range;
+    # (-1, 2) mixes in rows above it, (0.7, 2) and (2, 3) (w down to e^-20) have every row above it
     p = wi.wkv5_problem(2, 150, 3, 64, seed=82, omega_range=omega_range)
     g = wi.wkv5_grads(2, 150, 3, 64, seed=83, states=True)
     out, ref = _run(p, g, cuda_device, True)
     _check(out, ref, f"omega {omega_range}: ")
 
 
-def test_backward_fast_decay_is_reported(cuda_device):
-    # exp(omega) above 2 in some channel: outside the backward's range, reported, not computed
-    p = wi.wkv5_problem(1, 70, 2, 64, seed=84, omega_range=(-1.0, 2.0))
-    g = wi.wkv5_grads(1, 70, 2, 64, seed=85)
-    c = {k: v.to(cuda_device) for k, v in p.items()}
-    rw.rwkv_wkv5_backward(c["r"], c["k"], c["v"], c["omega"], c["u"], g["gy"].to(cuda_device))
-    assert rw.lib().rwkv_check_device_error(rw._stream(None)) == 2
-    assert rw.lib().rwkv_check_device_error(rw._stream(None)) == 0
+@pytest.mark.parametrize("shape", [(1, 64, 2), (1, 65, 2), (2, 127, 2), (1, 1, 1)])
+def test_backward_fast_decay_ragged(cuda_device, shape):
+    # fast rows at ragged lengths: the reversed pass's first chunk has `lead` empty positions
+    B, T, H = shape
+    p = wi.wkv5_problem(B, T, H, 64, seed=84, omega_range=(-1.0, 2.0))
+    g = wi.wkv5_grads(B, T, H, 64, seed=85, states=True)
+    out, ref = _run(p, g, cuda_device, True)
+    _check(out, ref, f"shape {shape}: ")
 
 
 def test_backward_deterministic(cuda_device):
@@ -83,5 +84,14 @@ def test_backward_workload_full_size(cuda_device):
     B, T, H, N = 4, 4096, 40, 64
     p = wi.wkv5_problem(B, T, H, N, seed=SEED + 4)
     g = wi.wkv5_grads(B, T, H, N, seed=SEED + 8)
+    out, ref = _run(p, g, cuda_device, False)
+    _check(out, ref)
+
+
+def test_backward_fast_decay_full_size(cuda_device):
+    # the same workload with omega ~ U(-1, 2): every head has rows above the factorization's range
+    B, T, H, N = 4, 4096, 40, 64
+    p = wi.wkv5_problem(B, T, H, N, seed=SEED + 5, omega_range=(-1.0, 2.0))
+    g = wi.wkv5_grads(B, T, H, N, seed=SEED + 9)
     out, ref = _run(p, g, cuda_device, False)
     _check(out, ref)
