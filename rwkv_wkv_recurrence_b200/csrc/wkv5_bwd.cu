@@ -66,6 +66,7 @@
 // 256 TMEM columns, two CTAs per SM.  Reversed pass: ~145 KB, 512 columns, one
 // CTA per SM.
 #include <cstddef>
+#include <type_traits>
 
 #include "launch.h"
 #include "tc_common.cuh"
@@ -93,6 +94,8 @@ struct Wkv5BwdSmem {
   alignas(128) float opAm[64 * 64];  // strictly causal scores [τ][ι]: B of the intra term
   float diag[kL];                    // A[τ][τ] = q_τ·p_τ
   float EB[kBand + 1][kN];           // e^{λ_d n} [n][key row d], n = 0..kBand (fast rows)
+  int flist[kN];                     // the fast rows, in order
+  int nfl;                           // their count
   alignas(8) uint64_t bar_tma;
   alignas(8) uint64_t bar_sc;        // scores and state read (and the X_c read) done
   alignas(8) uint64_t bar_av;        // intra term (and the lag-weighted term) done
@@ -118,6 +121,85 @@ size_t bwd_smem_bytes(bool rev) {
 // that the reversed pass copies it into shared memory as one contiguous block.
 __device__ __forceinline__ float* ckpt_at(const Wkv5BwdParams& p, int b, int h, int nchunk, int cf) {
   return p.ckpt + (((size_t)b * p.H + h) * nchunk + cf) * (kN * kN);
+}
+
+// Fast rows' intra-chunk terms over lags 0..kBand, by all threads (thread = position x one quarter
+// of the fast rows): BF0[pos][d] = Σ_n A[pos][pos-1-n] c_{pos-1-n}[d] e^{λ_d n} and, reversed,
+// BF1[pos][d] = Σ_{n≥1} n A[pos][pos-1-n] c_{pos-1-n}[d] e^{λ_d (n-1)}.  Out of line: it runs only
+// for heads with fast rows and keeps the main loop's code as it is for the others.
+template <bool REV>
+__device__ __noinline__ void fast_band(Wkv5BwdSmem& sm, const __nv_bfloat16* stC, float* BF0, float* BF1, int lo) {
+  const int tid = threadIdx.x;
+  const int pos = tid >> 2, g = tid & 3;
+  float an[kBand + 1];
+#pragma unroll
+  for (int n = 0; n <= kBand; ++n) {
+    const int io = pos - 1 - n;
+    an[n] = io >= lo ? sm.opAm[op_off(pos, io)] : 0.f;
+  }
+  const int nf = sm.nfl;
+#pragma unroll 1
+  for (int cf = g; cf < nf; cf += 4) {
+    const int d = sm.flist[cf];
+    float b0 = 0.f, b1 = 0.f;
+#pragma unroll
+    for (int n = 0; n <= kBand; ++n) {
+      const int io = pos - 1 - n;
+      const float ac = io >= 0 ? an[n] * __bfloat162float(stC[(REV ? kL - 1 - io : io) * kN + d]) : 0.f;
+      b0 = fmaf(ac, sm.EB[n][d], b0);
+      if constexpr (REV) {
+        if (n >= 1) b1 = fmaf((float)n * ac, sm.EB[n - 1][d], b1);
+      }
+    }
+    BF0[pos * kN + d] = b0;
+    if constexpr (REV) BF1[pos * kN + d] = b1;
+  }
+}
+
+// A fast row's state increment over the chunk's last kBand + 1 positions, Σ_ι c_ι[d] e^{λ(63-ι)}
+// p_ι[j] for the thread's eight columns j = jcol + 4 q (its tensor-core increment is zero).
+template <bool REV>
+__device__ __noinline__ void fast_increment(const Wkv5BwdSmem& sm, const __nv_bfloat16* stC, int d, int jcol, int lo,
+                                            float (&dsf)[8]) {
+#pragma unroll
+  for (int q = 0; q < 8; ++q) dsf[q] = 0.f;
+#pragma unroll
+  for (int n = 0; n <= kBand; ++n) {
+    const int io = kL - 1 - n;
+    if (io >= lo) {
+      const float cw = __bfloat162float(stC[(REV ? kL - 1 - io : io) * kN + d]) * sm.EB[n][d];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) dsf[q] = fmaf(cw, sm.opPt[op_off(jcol + 4 * q, io)], dsf[q]);
+    }
+  }
+}
+
+// A fast row's epilogue for 16 positions col.. (z: its state read, unscaled; x3: the X_c read):
+// out = e^{λ(pos-lo)} z + BF0 + u c A[pos][pos] into the output rows, and (reversed) the returned
+// sum of its decay-gradient terms, m ((pos-lo) e^{λ(pos-1-lo)} z + BF1) + f3 c x3.  Out of line, so
+// that heads without fast rows run the main epilogue untouched.
+template <bool REV>
+__device__ __noinline__ float fast_epilogue(const Wkv5BwdSmem& sm, const __nv_bfloat16* stC,
+                                            const __nv_bfloat16* stM, __nv_bfloat16* stO, const float* BF0,
+                                            const float* BF1, const float (&z)[16], const float (&x3)[16], int col,
+                                            int lo, int cnt, int de, float lam_e, float u_e) {
+  float accf = 0.f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const int pos = col + i;
+    if (pos < lo || pos >= cnt) continue;
+    const int so = (REV ? kL - 1 - pos : pos) * kN + de;
+    const float cval = __bfloat162float(stC[so]), mval = __bfloat162float(stM[so]);
+    const float fr = pos == lo ? 1.f : __expf(lam_e * (float)(pos - lo));
+    stO[so] = __float2bfloat16_rn(fmaf(u_e * cval, sm.diag[pos], fmaf(fr, z[i], BF0[pos * kN + de])));
+    if constexpr (REV) {
+      const float fz = pos > lo ? (float)(pos - lo) * __expf(lam_e * (float)(pos - 1 - lo)) : 0.f;
+      const float f3 = pos < kL - 1 ? (float)(kL - 1 - pos) * __expf(lam_e * (float)(kL - 2 - pos)) : 0.f;
+      accf = fmaf(mval, fmaf(fz, z[i], BF1[pos * kN + de]), accf);
+      accf = fmaf(f3 * cval, x3[i], accf);
+    }
+  }
+  return accf;
 }
 
 template <bool REV>
@@ -148,6 +230,12 @@ __global__ void __launch_bounds__(kThreads, REV ? 1 : 2) wkv5_bwd_tc_kernel(cons
     fast_any = !(-lam <= kMaxRate);
 #pragma unroll 1
     for (int n = 0; n <= kBand; ++n) sm.EB[n][tid] = n == 0 ? 1.f : expf(lam * (float)n);
+  }
+  if (tid == 0) {  // the fast rows in order (once per CTA)
+    int nf = 0;
+    for (int d = 0; d < kN; ++d)
+      if (!(expf(om[d]) <= kMaxRate)) sm.flist[nf++] = d;
+    sm.nfl = nf;
   }
   const bool nfast = __syncthreads_or(fast_any) != 0;
 
@@ -261,354 +349,334 @@ __global__ void __launch_bounds__(kThreads, REV ? 1 : 2) wkv5_bwd_tc_kernel(cons
 
   int c = 0;
   bool aborted = false;
-  for (; c < nchunk; ++c) {
-    const int t0 = c * kL - p.lead;            // pass position of position 0 of this chunk
-    const int lo = max(0, -t0);                // positions before the sequence start (first reversed chunk)
-    const int cnt = min(kL, p.T - t0);         // positions up to the sequence end (last forward chunk)
-    const uint32_t ph = (uint32_t)c & 1u;
-    const int cf = nchunk - 1 - c;             // reversed pass: the forward chunk this one mirrors
+  // the chunk loop, in two instances: heads with fast rows take the one with their extra terms,
+  // the others one without a trace of them
+  auto chunks = [&](auto fast_tag) {
+    constexpr bool FAST = decltype(fast_tag)::value;
+    for (; c < nchunk; ++c) {
+      const int t0 = c * kL - p.lead;            // pass position of position 0 of this chunk
+      const int lo = max(0, -t0);                // positions before the sequence start (first reversed chunk)
+      const int cnt = min(kL, p.T - t0);         // positions up to the sequence end (last forward chunk)
+      const uint32_t ph = (uint32_t)c & 1u;
+      const int cf = nchunk - 1 - c;             // reversed pass: the forward chunk this one mirrors
 
-    // this chunk's box of c and m (tokens tb .. tb + 63, rows past the sequence end zero): two
-    // 16-byte loads per tensor and thread, staged in shared memory for the epilogue after the first
-    // chains have released opQ
-    const int tb = REV ? kL * cf : t0;
-    const int nrow = min(kL, p.T - tb);
-    uint4 pre[2][2];
-#pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-      const int row = 32 * hh + (tid >> 3);
-      const size_t off = (((size_t)b * p.T + tb + row) * p.H + h) * kN + 8 * (tid & 7);
-      const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-      pre[0][hh] = row < nrow ? __ldg(reinterpret_cast<const uint4*>(p.c + off)) : z;
-      pre[1][hh] = row < nrow ? __ldg(reinterpret_cast<const uint4*>(p.m + off)) : z;
-    }
+      // this chunk's box of c and m (tokens tb .. tb + 63, rows past the sequence end zero): two
+      // 16-byte loads per tensor and thread, staged in shared memory for the epilogue after the first
+      // chains have released opQ
+      const int tb = REV ? kL * cf : t0;
+      const int nrow = min(kL, p.T - tb);
+      uint4 pre[2][2];
+  #pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int row = 32 * hh + (tid >> 3);
+        const size_t off = (((size_t)b * p.T + tb + row) * p.H + h) * kN + 8 * (tid & 7);
+        const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+        pre[0][hh] = row < nrow ? __ldg(reinterpret_cast<const uint4*>(p.c + off)) : z;
+        pre[1][hh] = row < nrow ? __ldg(reinterpret_cast<const uint4*>(p.m + off)) : z;
+      }
 
-    // forward pass: the state at this chunk's start is the checkpoint the reversed pass reads
-    if constexpr (!REV) {
-      float* ck = ckpt_at(p, b, h, nchunk, c);
-#pragma unroll
-      for (int q = 0; q < 8; ++q)
-#pragma unroll
-        for (int r = 0; r < 2; ++r) ck[op_off(drow + 8 * r, jcol + 4 * q)] = X[2 * q + r];
-    } else {
-      // X_c (the forward state at the mirrored chunk's start, copied into opXc) and the elementwise
-      // term n w^{n-1} Σ_j G∘X_c with n = 64 - lo positions in the chunk
-      if (!mbar_wait_bounded(&sm.bar_ck, ph, p.ctl)) sm.abort_flag = 1;
-      float part[2] = {0.f, 0.f};
-#pragma unroll
-      for (int q = 0; q < 8; ++q)
-#pragma unroll
-        for (int r = 0; r < 2; ++r) {
-          float& xc = sm.opXc[op_off(drow + 8 * r, jcol + 4 * q)];
-          part[r] = fmaf(X[2 * q + r], xc, part[r]);
-          xc = to_tf32(xc);  // the X_c read below takes it rounded to nearest
-        }
-      const float n = (float)(kL - lo);
-#pragma unroll
-      for (int r = 0; r < 2; ++r) acc_t1[r] += (double)(n * (n == 1.f ? 1.f : expf((n - 1.f) * lamr[r])) * part[r]);
-    }
-
-    if (!mbar_wait_bounded(&sm.bar_tma, ph, p.ctl)) sm.abort_flag = 1;
-    // T1a: q, p as fp32 operands (rows outside the sequence hold zeros from the TMA fill)
-#pragma unroll
-    for (int ib = 0; ib < 8; ++ib) {
-      const int row = 8 * ib + rr;
-      const uint32_t ibo = (uint32_t)(REV ? 7 - ib : ib) * 1024u;
-      *reinterpret_cast<float2*>(&sm.opQ[op_off(row, dR)]) = bf2_to_f2(lds_u32(rawQ + offRK + ibo));
-      *reinterpret_cast<float2*>(&sm.opP[op_off(row, dR)]) = bf2_to_f2(lds_u32(rawP + offRK + ibo));
-    }
-    fence_proxy_async();
-    tc_fence_before();
-    __syncthreads();
-    if (sm.abort_flag) {
-      aborted = true;
-      break;
-    }
-    // scores A = q pᵀ [τ][ι], state read (e^{32λ} X) qᵀ [d][τ], and (reversed) X_c pᵀ [d][ι]; the
-    // issuing thread hands the K steps out in groups between its warp's T1b steps
-    auto issue_first = [&](int s0) {
-      if (issuer) {
-        if (s0 == 0) tc_fence_after();
-#pragma unroll
-        for (int s = s0; s < s0 + 2; ++s) {
-          umma_tf32(tA, smem_desc(&sm.opQ[s * 64], kLbo, kSbo), smem_desc(&sm.opP[s * 64], kLbo, kSbo), kIdesc, s);
-          umma_tf32(tZ, smem_desc(&sm.opX[s * 64], kLbo, kSbo), smem_desc(&sm.opQ[s * 64], kLbo, kSbo), kIdesc, s);
-          if constexpr (REV)
-            umma_tf32(tX3, smem_desc(&sm.opXc[s * 64], kLbo, kSbo), smem_desc(&sm.opP[s * 64], kLbo, kSbo), kIdesc,
-                      s);
-        }
-        if (s0 == 6) umma_commit(&sm.bar_sc);
-      }
-    };
-    issue_first(0);
-
-    // T1b: c̃ᵀ into tensor memory, pᵀ into shared memory
-    {
-      uint32_t kt[16];
-#pragma unroll
-      for (int pp = 0; pp < 2; ++pp) {
-        uint32_t qk[4];
-        ldsm_x4_t(REV ? rawC + offKt - pp * 2048u : rawC + offKt + pp * 2048u, qk);
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {
-          const int i = 2 * pp + (m >> 1), r = m & 1;
-          const float2 f = bf2_to_f2(qk[m]);
-          const float g = i == 0 ? 1.f : (i == 1 ? fcs[r] : (i == 2 ? fcs[r] * fcs[r] : fcs[r] * fcs[r] * fcs[r]));
-          kt[4 * i + 2 * r] = __float_as_uint(to_tf32(f.x * fc0[r][0] * g));
-          kt[4 * i + 2 * r + 1] = __float_as_uint(to_tf32(f.y * fc0[r][1] * g));
-        }
-        issue_first(2 + 2 * pp);
-      }
-      tmem_st16(tCt + tquar + (uint32_t)(32 * hc), kt);
-#pragma unroll
-      for (int pp = 0; pp < 2; ++pp) {
-        uint32_t qv[4];
-        ldsm_x4_t(REV ? rawP + offT - pp * 4096u : rawP + offT + pp * 4096u, qv);
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {
-          const int ib = 4 * pp + m;
-          const uint32_t xv = __shfl_xor_sync(0xffffffffu, qv[m], 18);
-          *reinterpret_cast<float2*>(&sm.opPt[op_off(8 * warp + srow, 8 * ib + 2 * stq)]) =
-              bf2_to_f2(sw ? xv : qv[m]);
-        }
-        if (pp == 0) issue_first(6);
-      }
-    }
-    fence_proxy_async();
-    tc_fence_before();
-    __syncthreads();
-    if (issuer) {
-      tc_fence_after();
-      // state increment c̃ᵀ p [d][j]: needs only this chunk's operands, runs while the scores are masked
-#pragma unroll
-      for (int s = 0; s < 8; ++s) umma_tf32_ts(tDS, tCt + 8 * s, smem_desc(&sm.opPt[s * 64], kLbo, kSbo), kIdesc, s);
-      umma_commit(&sm.bar_ds);
-      // the raw boxes are consumed: load the next chunk while this one computes
-      if (c + 1 < nchunk) {
-        fence_proxy_async();
-        mbar_arrive_expect_tx(&sm.bar_tma, 3 * kRawBytes);
-        const int rown = REV ? kL * (cf - 1) : t0 + kL;
-        tma_load_3d(sm.raw[0], &mq, &sm.bar_tma, h * kN, rown, b);
-        tma_load_3d(sm.raw[1], &mp, &sm.bar_tma, h * kN, rown, b);
-        tma_load_3d(sm.raw[2], &mc, &sm.bar_tma, h * kN, rown, b);
-      }
-    }
-
-    // T2a: strictly causal scores -> opAm (and, reversed, weighted by the lag -> opAl); the diagonal
-    // q_τ·p_τ -> diag.  .16x128b fragment: rows τ = 16 q4 + t4 + 8 r, columns ι = 32 hc + 4 q + tq
-    if (!mbar_wait_bounded(&sm.bar_sc, ph, p.ctl)) sm.abort_flag = 1;
-    tc_fence_after();
-    // the first chains have read opQ, opP and opXc: c and m into the staging rows (opQ), and
-    // (reversed) the next chunk's checkpoint into opXc
-#pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-      const int row = 32 * hh + (tid >> 3);
-      *reinterpret_cast<uint4*>(&stC[row * kN + 8 * (tid & 7)]) = pre[0][hh];
-      *reinterpret_cast<uint4*>(&stM[row * kN + 8 * (tid & 7)]) = pre[1][hh];
-    }
-    if constexpr (REV) {
-      if (issuer && c + 1 < nchunk) {
-        fence_proxy_async();
-        mbar_arrive_expect_tx(&sm.bar_ck, kCkBytes);
-        bulk_load(sm.opXc, ckpt_at(p, b, h, nchunk, cf - 1), kCkBytes, &sm.bar_ck);
-      }
-    }
-    {
-      const int tau0 = 16 * q4 + t4;
-      if (hc > (q4 >> 1)) {  // strictly above the diagonal
-#pragma unroll
+      // forward pass: the state at this chunk's start is the checkpoint the reversed pass reads
+      if constexpr (!REV) {
+        float* ck = ckpt_at(p, b, h, nchunk, c);
+  #pragma unroll
         for (int q = 0; q < 8; ++q)
-#pragma unroll
-          for (int r = 0; r < 2; ++r) {
-            sm.opAm[op_off(tau0 + 8 * r, 32 * hc + 4 * q + tq)] = 0.f;
-            if constexpr (REV) sm.opAl[op_off(tau0 + 8 * r, 32 * hc + 4 * q + tq)] = 0.f;
-          }
+  #pragma unroll
+          for (int r = 0; r < 2; ++r) ck[op_off(drow + 8 * r, jcol + 4 * q)] = X[2 * q + r];
       } else {
-        float a[16];
-        tmem_ld16x128(tA + tquar + (uint32_t)(32 * hc), a);
-#pragma unroll
+        // X_c (the forward state at the mirrored chunk's start, copied into opXc) and the elementwise
+        // term n w^{n-1} Σ_j G∘X_c with n = 64 - lo positions in the chunk
+        if (!mbar_wait_bounded(&sm.bar_ck, ph, p.ctl)) sm.abort_flag = 1;
+        float part[2] = {0.f, 0.f};
+  #pragma unroll
         for (int q = 0; q < 8; ++q)
-#pragma unroll
+  #pragma unroll
           for (int r = 0; r < 2; ++r) {
-            const int io = 32 * hc + 4 * q + tq, tau = tau0 + 8 * r;
-            const float am = io < tau ? a[2 * q + r] : 0.f;
-            sm.opAm[op_off(tau, io)] = to_tf32(am);
-            if constexpr (REV) sm.opAl[op_off(tau, io)] = to_tf32((float)(tau - 1 - io) * am);
-            if (io == tau) sm.diag[tau] = a[2 * q + r];
+            float& xc = sm.opXc[op_off(drow + 8 * r, jcol + 4 * q)];
+            part[r] = fmaf(X[2 * q + r], xc, part[r]);
+            xc = to_tf32(xc);  // the X_c read below takes it rounded to nearest
           }
+        const float n = (float)(kL - lo);
+  #pragma unroll
+        for (int r = 0; r < 2; ++r) acc_t1[r] += (double)(n * (n == 1.f ? 1.f : expf((n - 1.f) * lamr[r])) * part[r]);
       }
-    }
-    fence_proxy_async();
-    tc_fence_before();
-    __syncthreads();
-    if (issuer) {
-      tc_fence_after();
-      // intra term: forward pass into the state-read accumulator, reversed pass into its own (the
-      // decay gradient weights the state read alone); reversed also the lag-weighted term
-#pragma unroll
-      for (int s = 0; s < 8; ++s) {
-        if constexpr (REV) {
-          umma_tf32_ts(tI, tCt + 8 * s, smem_desc(&sm.opAm[s * 64], kLbo, kSbo), kIdesc, s);
-          umma_tf32_ts(tX4, tCt + 8 * s, smem_desc(&sm.opAl[s * 64], kLbo, kSbo), kIdesc, s);
-        } else {
-          umma_tf32_ts(tZ, tCt + 8 * s, smem_desc(&sm.opAm[s * 64], kLbo, kSbo), kIdesc, 1);
-        }
-      }
-      umma_commit(&sm.bar_av);
-    }
 
-    // T2b: X <- e^{nλ} X + e^{32λ} (c̃ᵀ p) with n the positions since the state entered
-    // (64 - lead in the first reversed chunk), or the partial last chunk's own form
-    if (!mbar_wait_bounded(&sm.bar_ds, ph, p.ctl)) sm.abort_flag = 1;
-    tc_fence_after();
-    {
-      float ds[16];
-      tmem_ld16x128(tDS + tquar + (uint32_t)(32 * hc), ds);
-      if (cnt == kL) {
-#pragma unroll
-        for (int r = 0; r < 2; ++r) {
-          const float gx = lo == 0 ? e32[r] * e32[r] : expf((float)(kL - lo) * lamr[r]);
-#pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            const int x = 2 * q + r;
-            X[x] = fmaf(gx, X[x], e32[r] * ds[x]);
-            sm.opX[op_off(drow + 8 * r, jcol + 4 * q)] = to_tf32(e32[r] * X[x]);
+      if (!mbar_wait_bounded(&sm.bar_tma, ph, p.ctl)) sm.abort_flag = 1;
+      // T1a: q, p as fp32 operands (rows outside the sequence hold zeros from the TMA fill)
+  #pragma unroll
+      for (int ib = 0; ib < 8; ++ib) {
+        const int row = 8 * ib + rr;
+        const uint32_t ibo = (uint32_t)(REV ? 7 - ib : ib) * 1024u;
+        *reinterpret_cast<float2*>(&sm.opQ[op_off(row, dR)]) = bf2_to_f2(lds_u32(rawQ + offRK + ibo));
+        *reinterpret_cast<float2*>(&sm.opP[op_off(row, dR)]) = bf2_to_f2(lds_u32(rawP + offRK + ibo));
+      }
+      fence_proxy_async();
+      tc_fence_before();
+      __syncthreads();
+      if (sm.abort_flag) {
+        aborted = true;
+        break;
+      }
+      // scores A = q pᵀ [τ][ι], state read (e^{32λ} X) qᵀ [d][τ], and (reversed) X_c pᵀ [d][ι]; the
+      // issuing thread hands the K steps out in groups between its warp's T1b steps
+      auto issue_first = [&](int s0) {
+        if (issuer) {
+          if (s0 == 0) tc_fence_after();
+  #pragma unroll
+          for (int s = s0; s < s0 + 2; ++s) {
+            umma_tf32(tA, smem_desc(&sm.opQ[s * 64], kLbo, kSbo), smem_desc(&sm.opP[s * 64], kLbo, kSbo), kIdesc, s);
+            umma_tf32(tZ, smem_desc(&sm.opX[s * 64], kLbo, kSbo), smem_desc(&sm.opQ[s * 64], kLbo, kSbo), kIdesc, s);
+            if constexpr (REV)
+              umma_tf32(tX3, smem_desc(&sm.opXc[s * 64], kLbo, kSbo), smem_desc(&sm.opP[s * 64], kLbo, kSbo), kIdesc,
+                        s);
+          }
+          if (s0 == 6) umma_commit(&sm.bar_sc);
+        }
+      };
+      issue_first(0);
+
+      // T1b: c̃ᵀ into tensor memory, pᵀ into shared memory
+      {
+        uint32_t kt[16];
+  #pragma unroll
+        for (int pp = 0; pp < 2; ++pp) {
+          uint32_t qk[4];
+          ldsm_x4_t(REV ? rawC + offKt - pp * 2048u : rawC + offKt + pp * 2048u, qk);
+  #pragma unroll
+          for (int m = 0; m < 4; ++m) {
+            const int i = 2 * pp + (m >> 1), r = m & 1;
+            const float2 f = bf2_to_f2(qk[m]);
+            const float g = i == 0 ? 1.f : (i == 1 ? fcs[r] : (i == 2 ? fcs[r] * fcs[r] : fcs[r] * fcs[r] * fcs[r]));
+            kt[4 * i + 2 * r] = __float_as_uint(to_tf32(f.x * fc0[r][0] * g));
+            kt[4 * i + 2 * r + 1] = __float_as_uint(to_tf32(f.y * fc0[r][1] * g));
+          }
+          issue_first(2 + 2 * pp);
+        }
+        tmem_st16(tCt + tquar + (uint32_t)(32 * hc), kt);
+  #pragma unroll
+        for (int pp = 0; pp < 2; ++pp) {
+          uint32_t qv[4];
+          ldsm_x4_t(REV ? rawP + offT - pp * 4096u : rawP + offT + pp * 4096u, qv);
+  #pragma unroll
+          for (int m = 0; m < 4; ++m) {
+            const int ib = 4 * pp + m;
+            const uint32_t xv = __shfl_xor_sync(0xffffffffu, qv[m], 18);
+            *reinterpret_cast<float2*>(&sm.opPt[op_off(8 * warp + srow, 8 * ib + 2 * stq)]) =
+                bf2_to_f2(sw ? xv : qv[m]);
+          }
+          if (pp == 0) issue_first(6);
+        }
+      }
+      fence_proxy_async();
+      tc_fence_before();
+      __syncthreads();
+      if (issuer) {
+        tc_fence_after();
+        // state increment c̃ᵀ p [d][j]: needs only this chunk's operands, runs while the scores are masked
+  #pragma unroll
+        for (int s = 0; s < 8; ++s) umma_tf32_ts(tDS, tCt + 8 * s, smem_desc(&sm.opPt[s * 64], kLbo, kSbo), kIdesc, s);
+        umma_commit(&sm.bar_ds);
+        // the raw boxes are consumed: load the next chunk while this one computes
+        if (c + 1 < nchunk) {
+          fence_proxy_async();
+          mbar_arrive_expect_tx(&sm.bar_tma, 3 * kRawBytes);
+          const int rown = REV ? kL * (cf - 1) : t0 + kL;
+          tma_load_3d(sm.raw[0], &mq, &sm.bar_tma, h * kN, rown, b);
+          tma_load_3d(sm.raw[1], &mp, &sm.bar_tma, h * kN, rown, b);
+          tma_load_3d(sm.raw[2], &mc, &sm.bar_tma, h * kN, rown, b);
+        }
+      }
+
+      // T2a: strictly causal scores -> opAm (and, reversed, weighted by the lag -> opAl); the diagonal
+      // q_τ·p_τ -> diag.  .16x128b fragment: rows τ = 16 q4 + t4 + 8 r, columns ι = 32 hc + 4 q + tq
+      if (!mbar_wait_bounded(&sm.bar_sc, ph, p.ctl)) sm.abort_flag = 1;
+      tc_fence_after();
+      // the first chains have read opQ, opP and opXc: c and m into the staging rows (opQ), and
+      // (reversed) the next chunk's checkpoint into opXc
+  #pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int row = 32 * hh + (tid >> 3);
+        *reinterpret_cast<uint4*>(&stC[row * kN + 8 * (tid & 7)]) = pre[0][hh];
+        *reinterpret_cast<uint4*>(&stM[row * kN + 8 * (tid & 7)]) = pre[1][hh];
+      }
+      if constexpr (REV) {
+        if (issuer && c + 1 < nchunk) {
+          fence_proxy_async();
+          mbar_arrive_expect_tx(&sm.bar_ck, kCkBytes);
+          bulk_load(sm.opXc, ckpt_at(p, b, h, nchunk, cf - 1), kCkBytes, &sm.bar_ck);
+        }
+      }
+      {
+        const int tau0 = 16 * q4 + t4;
+        if (hc > (q4 >> 1)) {  // strictly above the diagonal
+  #pragma unroll
+          for (int q = 0; q < 8; ++q)
+  #pragma unroll
+            for (int r = 0; r < 2; ++r) {
+              sm.opAm[op_off(tau0 + 8 * r, 32 * hc + 4 * q + tq)] = 0.f;
+              if constexpr (REV) sm.opAl[op_off(tau0 + 8 * r, 32 * hc + 4 * q + tq)] = 0.f;
+            }
+        } else {
+          float a[16];
+          tmem_ld16x128(tA + tquar + (uint32_t)(32 * hc), a);
+  #pragma unroll
+          for (int q = 0; q < 8; ++q)
+  #pragma unroll
+            for (int r = 0; r < 2; ++r) {
+              const int io = 32 * hc + 4 * q + tq, tau = tau0 + 8 * r;
+              const float am = io < tau ? a[2 * q + r] : 0.f;
+              sm.opAm[op_off(tau, io)] = to_tf32(am);
+              if constexpr (REV) sm.opAl[op_off(tau, io)] = to_tf32((float)(tau - 1 - io) * am);
+              if (io == tau) sm.diag[tau] = a[2 * q + r];
+            }
+        }
+      }
+      fence_proxy_async();
+      tc_fence_before();
+      __syncthreads();
+      if (issuer) {
+        tc_fence_after();
+        // intra term: forward pass into the state-read accumulator, reversed pass into its own (the
+        // decay gradient weights the state read alone); reversed also the lag-weighted term
+  #pragma unroll
+        for (int s = 0; s < 8; ++s) {
+          if constexpr (REV) {
+            umma_tf32_ts(tI, tCt + 8 * s, smem_desc(&sm.opAm[s * 64], kLbo, kSbo), kIdesc, s);
+            umma_tf32_ts(tX4, tCt + 8 * s, smem_desc(&sm.opAl[s * 64], kLbo, kSbo), kIdesc, s);
+          } else {
+            umma_tf32_ts(tZ, tCt + 8 * s, smem_desc(&sm.opAm[s * 64], kLbo, kSbo), kIdesc, 1);
           }
         }
-        if (nfast) {
-#pragma unroll
-          for (int r = 0; r < 2; ++r) {  // unrolled: X stays in registers
-            if (!fastR[r]) continue;
-            // a fast row (its tensor-core increment is zero): Σ_ι c_ι[d] e^{λ(63-ι)} p_ι[j] over the
-            // chunk's last kBand + 1 positions, and the row read unscaled
-            const int d = drow + 8 * r;
-            float dsf[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int n = 0; n <= kBand; ++n) {
-              const int io = kL - 1 - n;
-              if (io >= lo) {
-                const float cw = __bfloat162float(stC[(REV ? kL - 1 - io : io) * kN + d]) * sm.EB[n][d];
-#pragma unroll
-                for (int q = 0; q < 8; ++q) dsf[q] = fmaf(cw, sm.opPt[op_off(jcol + 4 * q, io)], dsf[q]);
-              }
-            }
-#pragma unroll
+        umma_commit(&sm.bar_av);
+      }
+
+      // T2b: X <- e^{nλ} X + e^{32λ} (c̃ᵀ p) with n the positions since the state entered
+      // (64 - lead in the first reversed chunk), or the partial last chunk's own form
+      if (!mbar_wait_bounded(&sm.bar_ds, ph, p.ctl)) sm.abort_flag = 1;
+      tc_fence_after();
+      {
+        float ds[16];
+        tmem_ld16x128(tDS + tquar + (uint32_t)(32 * hc), ds);
+        if (cnt == kL) {
+  #pragma unroll
+          for (int r = 0; r < 2; ++r) {
+            const float gx = lo == 0 ? e32[r] * e32[r] : expf((float)(kL - lo) * lamr[r]);
+  #pragma unroll
             for (int q = 0; q < 8; ++q) {
               const int x = 2 * q + r;
-              X[x] += dsf[q];
-              sm.opX[op_off(d, jcol + 4 * q)] = to_tf32(X[x]);
+              X[x] = fmaf(gx, X[x], e32[r] * ds[x]);
+              sm.opX[op_off(drow + 8 * r, jcol + 4 * q)] = to_tf32(e32[r] * X[x]);
             }
           }
-        }
-      } else {  // partial last chunk (forward pass): no later chunk reads opX
-#pragma unroll
-        for (int r = 0; r < 2; ++r) {
-          const float dl = expf(lamr[r] * (float)cnt), gs = expf(lamr[r] * (float)(cnt - 32));
-#pragma unroll
-          for (int q = 0; q < 8; ++q) X[2 * q + r] = fmaf(dl, X[2 * q + r], gs * ds[2 * q + r]);
-        }
-      }
-    }
-    // T3: out[τ][de] = e^{λ(τ-32)} (state read + intra)[de][τ] + u c_τ A[τ][τ], and the sums; 16
-    // positions at a time (lanes 0..15 of each quarter hold the rows of the M = 64 accumulators)
-    if (!mbar_wait_bounded(&sm.bar_av, ph, p.ctl)) sm.abort_flag = 1;
-    tc_fence_after();
-#pragma unroll 1
-    for (int half = 0; half < 2; ++half) {
-      const uint32_t col = (uint32_t)(32 * hc + 16 * half);
-      float zv[16], iv[REV ? 16 : 1], x3[REV ? 16 : 1], x4[REV ? 16 : 1];
-      tmem_ld32x16(tZ + tquar + col, zv);
-      if constexpr (REV) {
-        tmem_ld32x16(tI + tquar + col, iv);
-        tmem_ld32x16(tX3 + tquar + col, x3);
-        tmem_ld32x16(tX4 + tquar + col, x4);
-      }
-      if (lane < 16) {
-        float acc = 0.f;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int pos = (int)col + i;
-          if (pos < lo || pos >= cnt) continue;
-          // staging row of this position (the box holds the tokens in forward order)
-          const int so = (REV ? kL - 1 - pos : pos) * kN + de;
-          const float cval = __bfloat162float(stC[so]), mval = __bfloat162float(stM[so]);
-          const float dg = sm.diag[pos];
-          const float f = __expf(lam_e * (float)(pos - 32));
-          float o;
-          if constexpr (REV) o = f * (zv[i] + iv[i]);
-          else o = f * zv[i];
-          o = fmaf(u_e * cval, dg, o);
-          if constexpr (REV) {
-            // position-weighted state read, lag-weighted intra term, and the X_c read (for a fast row
-            // these are not its sums, which are formed below; its acc is dropped after the loop)
-            const float f1 = __expf(lam_e * (float)(pos - 33));
-            const float f3 = pos < kL - 1 ? (float)(kL - 1 - pos) * __expf(lam_e * (float)(kL - 2 - pos)) : 0.f;
-            acc = fmaf(mval * f1, fmaf((float)(pos - lo), zv[i], x4[i]), acc);
-            acc = fmaf(f3 * cval, x3[i], acc);
-          } else {
-            acc = fmaf(mval * cval, dg, acc);  // gu: r k (v·gy)
+          if (FAST) {
+  #pragma unroll
+            for (int r = 0; r < 2; ++r) {  // unrolled: X stays in registers
+              if (!fastR[r]) continue;
+              // a fast row (its tensor-core increment is zero): Σ_ι c_ι[d] e^{λ(63-ι)} p_ι[j] over the
+              // chunk's last kBand + 1 positions, and the row read unscaled
+              const int d = drow + 8 * r;
+              float dsf[8];
+              fast_increment<REV>(sm, stC, d, jcol, lo, dsf);
+  #pragma unroll
+              for (int q = 0; q < 8; ++q) {
+                const int x = 2 * q + r;
+                X[x] += dsf[q];
+                sm.opX[op_off(d, jcol + 4 * q)] = to_tf32(X[x]);
+              }
+            }
           }
-          stO[so] = __float2bfloat16_rn(o);
+        } else {  // partial last chunk (forward pass): no later chunk reads opX
+  #pragma unroll
+          for (int r = 0; r < 2; ++r) {
+            const float dl = expf(lamr[r] * (float)cnt), gs = expf(lamr[r] * (float)(cnt - 32));
+  #pragma unroll
+            for (int q = 0; q < 8; ++q) X[2 * q + r] = fmaf(dl, X[2 * q + r], gs * ds[2 * q + r]);
+          }
         }
-        if (nfast && fast_e) {
-          // a fast row: the state read (unscaled) times e^{λ(pos-lo)}, and the intra-chunk terms over
-          // lags n = 0..kBand, Σ_n A[pos][pos-1-n] c_{pos-1-n} e^{λn} (and, reversed, the lag-weighted
-          // Σ_n n A c e^{λ(n-1)}), from the masked scores and the staged c rows
-          float accf = 0.f;
-#pragma unroll 1
+      }
+      // T3: out[τ][de] = e^{λ(τ-32)} (state read + intra)[de][τ] + u c_τ A[τ][τ], and the sums; 16
+      // positions at a time (lanes 0..15 of each quarter hold the rows of the M = 64 accumulators)
+      if (!mbar_wait_bounded(&sm.bar_av, ph, p.ctl)) sm.abort_flag = 1;
+      tc_fence_after();
+      // fast rows: their intra-chunk terms over lags 0..kBand, by all threads (thread = position x one
+      // quarter of the fast rows) into opPt (free after the fold) and, reversed, the lag-weighted ones
+      // into opAl (free after the intra chains): BF0[pos][d] = Σ_n A[pos][pos-1-n] c_{pos-1-n}[d]
+      // e^{λ_d n}, BF1[pos][d] = Σ_{n≥1} n A[pos][pos-1-n] c_{pos-1-n}[d] e^{λ_d (n-1)}
+      float* BF0 = sm.opPt;
+      float* BF1 = REV ? sm.opAl : nullptr;
+      if (FAST) {
+        __syncthreads();  // every fold has read opPt
+        fast_band<REV>(sm, stC, BF0, BF1, lo);
+        __syncthreads();
+      }
+  #pragma unroll 1
+      for (int half = 0; half < 2; ++half) {
+        const uint32_t col = (uint32_t)(32 * hc + 16 * half);
+        float zv[16];
+        [[maybe_unused]] float iv[REV ? 16 : 1], x3[REV ? 16 : 1], x4[REV ? 16 : 1];
+        tmem_ld32x16(tZ + tquar + col, zv);
+        if constexpr (REV) {
+          tmem_ld32x16(tI + tquar + col, iv);
+          tmem_ld32x16(tX3 + tquar + col, x3);
+          tmem_ld32x16(tX4 + tquar + col, x4);
+        }
+        if (lane < 16) {
+          float acc = 0.f;
+  #pragma unroll
           for (int i = 0; i < 16; ++i) {
             const int pos = (int)col + i;
             if (pos < lo || pos >= cnt) continue;
-            float zi = 0.f, x3i = 0.f;  // zv[i], x3[i] by selects: the arrays stay in registers
-#pragma unroll
-            for (int t = 0; t < 16; ++t) {
-              if (t == i) {
-                zi = zv[t];
-                if constexpr (REV) x3i = x3[t];
-              }
-            }
+            // staging row of this position (the box holds the tokens in forward order)
             const int so = (REV ? kL - 1 - pos : pos) * kN + de;
             const float cval = __bfloat162float(stC[so]), mval = __bfloat162float(stM[so]);
-            float b0 = 0.f, b1 = 0.f;
-#pragma unroll
-            for (int n = 0; n <= kBand; ++n) {
-              const int io = pos - 1 - n;
-              if (io >= lo) {
-                const float ac =
-                    sm.opAm[op_off(pos, io)] * __bfloat162float(stC[(REV ? kL - 1 - io : io) * kN + de]);
-                b0 = fmaf(ac, sm.EB[n][de], b0);
-                if constexpr (REV) {
-                  if (n >= 1) b1 = fmaf((float)n * ac, sm.EB[n - 1][de], b1);
-                }
-              }
-            }
-            const float fr = pos == lo ? 1.f : __expf(lam_e * (float)(pos - lo));
-            stO[so] = __float2bfloat16_rn(fmaf(u_e * cval, sm.diag[pos], fmaf(fr, zi, b0)));
+            const float dg = sm.diag[pos];
+            const float f = __expf(lam_e * (float)(pos - 32));
+            float o;
+            if constexpr (REV) o = f * (zv[i] + iv[i]);
+            else o = f * zv[i];
+            o = fmaf(u_e * cval, dg, o);
             if constexpr (REV) {
-              const float fz = pos > lo ? (float)(pos - lo) * __expf(lam_e * (float)(pos - 1 - lo)) : 0.f;
+              // position-weighted state read, lag-weighted intra term, and the X_c read (for a fast row
+              // these are not its sums, which are formed below; its acc is dropped after the loop)
+              const float f1 = __expf(lam_e * (float)(pos - 33));
               const float f3 = pos < kL - 1 ? (float)(kL - 1 - pos) * __expf(lam_e * (float)(kL - 2 - pos)) : 0.f;
-              accf = fmaf(mval, fmaf(fz, zi, b1), accf);
-              accf = fmaf(f3 * cval, x3i, accf);
+              acc = fmaf(mval * f1, fmaf((float)(pos - lo), zv[i], x4[i]), acc);
+              acc = fmaf(f3 * cval, x3[i], acc);
+            } else {
+              acc = fmaf(mval * cval, dg, acc);  // gu: r k (v·gy)
             }
+            stO[so] = __float2bfloat16_rn(o);
           }
-          acc_e += (double)accf;
+          if (FAST && fast_e) {
+            // a fast row: its output and (reversed) its sums, out of line
+            float zl[16], xl[16];
+  #pragma unroll
+            for (int t = 0; t < 16; ++t) {
+              zl[t] = zv[t];
+              xl[t] = REV ? x3[REV ? t : 0] : 0.f;
+            }
+            acc_e += (double)fast_epilogue<REV>(sm, stC, stM, stO, BF0, BF1, zl, xl, (int)col, lo, cnt, de, lam_e, u_e);
+          }
+          if constexpr (REV && FAST) acc_e += fast_e ? 0.0 : (double)acc;  // (the gu sum has no decay factor)
+          else acc_e += (double)acc;
         }
-        if constexpr (REV) acc_e += fast_e ? 0.0 : (double)acc;  // (the gu sum has no decay factor)
-        else acc_e += (double)acc;
       }
-    }
-    // the chunk's out rows, 16 bytes a thread
-    __syncthreads();
-#pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-      const int row = 32 * hh + (tid >> 3);
-      if (row < nrow)
-        *reinterpret_cast<uint4*>(p.out + (((size_t)b * p.T + tb + row) * p.H + h) * kN + 8 * (tid & 7)) =
-            *reinterpret_cast<const uint4*>(&stO[row * kN + 8 * (tid & 7)]);
-    }
+      // the chunk's out rows, 16 bytes a thread
+      __syncthreads();
+  #pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int row = 32 * hh + (tid >> 3);
+        if (row < nrow)
+          *reinterpret_cast<uint4*>(p.out + (((size_t)b * p.T + tb + row) * p.H + h) * kN + 8 * (tid & 7)) =
+              *reinterpret_cast<const uint4*>(&stO[row * kN + 8 * (tid & 7)]);
+      }
 
-    __syncthreads();  // the staging rows (opQ) are read out before the next chunk converts q into it
-  }
+      __syncthreads();  // the staging rows (opQ) are read out before the next chunk converts q into it
+    }
+  };
+  if (nfast)
+    chunks(std::true_type{});
+  else
+    chunks(std::false_type{});
 
   if (aborted && tid == 0) {
     // a wait gave up at chunk c: the last MMA chains and this chunk's loads must finish before the
