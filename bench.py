@@ -782,9 +782,10 @@ def run_eagle(args, finch=False):
         "gpu_launches": args.steps, "clocks": clk, "call_ms": stats}), flush=True)
 
 
-def run_eagle_backward(args):
+def run_eagle_backward(args, finch=False):
     """Eagle / RWKV-5 backward on the forward workload's shape, B4 T4096 H40 N64 bf16, gy ~ N(0,1),
-    zero initial state and no final-state gradient: gr, gk, gv, gomega, gu."""
+    zero initial state and no final-state gradient: gr, gk, gv, gomega, gu.  With finch, the
+    Finch / RWKV-6 backward on the same shape with a per-token fp32 omega (and a per-token gomega)."""
     import torch
 
     import rwkv_wkv_recurrence_b200 as rw
@@ -795,42 +796,68 @@ def run_eagle_backward(args):
     dev = torch.device("cuda", local)
     Be, Te, He, Ne = 4, 4096, 40, 64
     om_lo, om_hi = _omega_range(args)
-    q = wi.wkv5_problem(Be, Te, He, Ne, seed=SEED + 2, device=dev, omega_range=(om_lo, om_hi))
+    gen = wi.wkv6_problem if finch else wi.wkv5_problem
+    q = gen(Be, Te, He, Ne, seed=SEED + (4 if finch else 2), device=dev, omega_range=(om_lo, om_hi))
     g = wi.wkv5_grads(Be, Te, He, Ne, seed=SEED + 6, device=dev)
     gr, gk, gv = (torch.empty_like(q["r"]) for _ in range(3))
-    gom, gu = torch.empty(He, Ne, device=dev), torch.empty(He, Ne, device=dev)
+    gom = torch.empty(Be, Te, He, Ne, device=dev) if finch else torch.empty(He, Ne, device=dev)
+    gu = torch.empty(He, Ne, device=dev)
     h = rw.lib()
-    wsb = int(h.rwkv_wkv5_backward_workspace_bytes(Be, Te, He, Ne))
+    name = "rwkv_wkv6_backward" if finch else "rwkv_wkv5_backward"
+    fn = getattr(h, name)
+    wsb = int(getattr(h, name + "_workspace_bytes")(Be, Te, He, Ne))
     ws = torch.empty(max(wsb, 1), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
     sp, P = rw._stream(stream), rw._ptr
 
     def call(i):
-        with _Nvtx("rwkv_wkv5_backward"):
-            s = h.rwkv_wkv5_backward(Be, Te, He, Ne, P(q["r"]), P(q["k"]), P(q["v"]), P(q["omega"]), P(q["u"]), None,
-                                     P(g["gy"]), None, P(gr), P(gk), P(gv), P(gom), P(gu), None, P(ws), wsb, sp)
+        with _Nvtx(name):
+            s = fn(Be, Te, He, Ne, P(q["r"]), P(q["k"]), P(q["v"]), P(q["omega"]), P(q["u"]), None, P(g["gy"]), None,
+                   P(gr), P(gk), P(gv), P(gom), P(gu), None, P(ws), wsb, sp)
         if s:
-            raise rw.RwkvError("rwkv_wkv5_backward", s)
+            raise rw.RwkvError(name, s)
 
     ms, clk, stats = _timed(call, args.steps, args.warmup, stream, local)
     rw.rwkv_check_device_error()
     elems = Be * Te * He * Ne
-    nbytes = 7 * 2 * elems + 4 * He * Ne * 4  # r, k, v, gy read, gr, gk, gv written (bf16); omega, u, gomega, gu
-    gbs = nbytes / (ms * 1e-3) / 1e9
-    peak, kind = _peaks()
+    om_note = "" if (om_lo, om_hi) == (-6.0, 0.0) else f", omega U({om_lo:g},{om_hi:g})"
+    if finch:
+        # r, k, v, gy read and gr, gk, gv written (bf16); omega read and gomega written (fp32, per token)
+        nbytes = 7 * 2 * elems + 2 * 4 * elems + 2 * He * Ne * 4
+        # algorithmic flops: six N x N multiply-adds per token and head (gr, the state step, gk, gv, the
+        # gomega row sums, the gradient-state step), 12 N flops per element; the kernel is bound by the
+        # CUDA cores' fp32 issue, so its fraction is taken against the fp32 FMA peak
+        flops = 12.0 * Ne * elems
+        tf = flops / (ms * 1e-3) / 1e12
+        peak_tf = 148 * 128 * 2 * 1.965e9 / 1e12
+        metric = "Finch WKV backward elements/s (B4 T4096 H40 N64, per-token decay)"
+        workload = ("Finch / RWKV-6 WKV backward, B=4 T=4096 H=40 N=64, bf16 r,k,v,gy,gr,gk,gv, fp32 per-token "
+                    "omega and gomega, gy ~ N(0,1), zero initial state, no final-state gradient" + om_note)
+        roof = {"bound": "alu", "kernel": "wkv6_bwd_kernel (+ its gu batch reduction)", "achieved": tf,
+                "peak": peak_tf, "peak_kind": "derived: 148 SMs x 128 fp32 FMA/clk x 2 flops x 1.965 GHz",
+                "unit": "TFLOP/s", "frac": tf / peak_tf, "hbm_gbs": nbytes / (ms * 1e-3) / 1e9,
+                "traffic": None}
+        l2 = f"no flush: {nbytes / 1e6:.0f} MB moved per call, above the 126 MB L2"
+        launches = 2
+    else:
+        nbytes = 7 * 2 * elems + 4 * He * Ne * 4  # r, k, v, gy read, gr, gk, gv written (bf16); omega, u, gomega, gu
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        peak, kind = _peaks()
+        metric = "Eagle WKV backward elements/s and HBM GB/s (B4 T4096 H40 N64)"
+        workload = ("Eagle / RWKV-5 WKV backward, B=4 T=4096 H=40 N=64, bf16 r,k,v,gy,gr,gk,gv, "
+                    "gy ~ N(0,1), zero initial state, no final-state gradient" + om_note)
+        roof = {"bound": "hbm", "kernel": "rwkv_wkv5_backward (reversed forward + two backward passes + "
+                                          "reduction)", "achieved": gbs, "peak": peak, "peak_kind": kind,
+                "unit": "GB/s", "frac": gbs / peak,
+                "traffic": _recorded_traffic("rwkv_wkv5_backward") if (om_lo, om_hi) == (-6.0, 0.0) else None}
+        l2 = "no flush: 587 MB moved per call, above the 126 MB L2"
+        launches = 4
     print(json.dumps({
-        "metric": "Eagle WKV backward elements/s and HBM GB/s (B4 T4096 H40 N64)", "value": elems / (ms * 1e-3),
+        "metric": metric, "value": elems / (ms * 1e-3),
         "unit": "elements/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "dtype": "bf16 I/O, fp32 state", "data": "synthetic",
-        "config": {"workload": "Eagle / RWKV-5 WKV backward, B=4 T=4096 H=40 N=64, bf16 r,k,v,gy,gr,gk,gv, "
-                               "gy ~ N(0,1), zero initial state, no final-state gradient"
-                               + ("" if (om_lo, om_hi) == (-6.0, 0.0) else f", omega U({om_lo:g},{om_hi:g})"),
-                   "l2": "no flush: 587 MB moved per call, above the 126 MB L2"},
-        "roofline": {"bound": "hbm", "kernel": "rwkv_wkv5_backward (reversed forward + two backward passes + "
-                                               "reduction)", "achieved": gbs, "peak": peak, "peak_kind": kind,
-                     "unit": "GB/s", "frac": gbs / peak,
-                     "traffic": _recorded_traffic("rwkv_wkv5_backward") if (om_lo, om_hi) == (-6.0, 0.0) else None},
-        "gpu_launches": 4 * args.steps, "clocks": clk, "call_ms": stats}), flush=True)
+        "config": {"workload": workload, "l2": l2}, "roofline": roof,
+        "gpu_launches": launches * args.steps, "clocks": clk, "call_ms": stats}), flush=True)
 
 
 def run_eagle_decode(args, finch=False):
@@ -895,10 +922,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=["train", "train_gated", "decode", "chunked", "eagle", "eagle_bwd",
-                                           "eagle_decode", "finch", "finch_decode"],
+                                           "eagle_decode", "finch", "finch_bwd", "finch_decode"],
                     default="train",
                     help="train: the headline forward+backward step; train_gated, decode, chunked, eagle, "
-                         "eagle_bwd, eagle_decode, finch, finch_decode: the other hot-path rows")
+                         "eagle_bwd, eagle_decode, finch, finch_bwd, finch_decode: the other hot-path rows")
     ap.add_argument("--chunked-shape", choices=["8x1024x768", "1x4096x768"], default="8x1024x768",
                     help="the few-channel forward's shape (chunked workload)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -927,6 +954,8 @@ def main():
         run_eagle_decode(args)
     elif args.workload == "finch":
         run_eagle(args, finch=True)
+    elif args.workload == "finch_bwd":
+        run_eagle_backward(args, finch=True)
     elif args.workload == "finch_decode":
         run_eagle_decode(args, finch=True)
     else:

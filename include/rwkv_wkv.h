@@ -295,6 +295,40 @@ RWKV_API rwkv_status rwkv_wkv6_step(int64_t B, int64_t H, int64_t N, const void 
                            const void *v, const float *omega, const float *u, void *y,
                            const float *s_in, float *s_out, rwkv_stream_t stream);
 
+/* Workspace bytes rwkv_wkv6_backward needs (0 for an empty problem or N != 64). */
+RWKV_API size_t rwkv_wkv6_backward_workspace_bytes(int64_t B, int64_t T, int64_t H, int64_t N);
+
+/*
+ * Finch / RWKV-6 backward: gradients of L = Σ gy·y + Σ gs_out ∘ s_out for
+ * rwkv_wkv6_forward ("RWKV-5 Eagle과 RWKV-6 Finch", section Finch; the pages
+ * print no backward, this is the chain rule through its recurrence).  With s_t
+ * the state before token t, G_T = gs_out and G_t = diag(w_t) G_{t+1} + r_tᵀ gy_t:
+ *   gr_t = s_t gy_tᵀ + u ⊙ k_t (v_t·gy_t),   gk_t = G_{t+1} v_tᵀ + u ⊙ r_t (v_t·gy_t),
+ *   gv_t = G_{t+1}ᵀ k_t + (Σ r_t u k_t) gy_t,  gs_in = G_0,
+ *   gomega_t[d] = (Σ_j G_{t+1}[d][j] s_t[d][j]) · dw_t[d]/dω_t[d]   (dw/dω = -e^ω w),
+ *   gu_d = Σ_{b,t} r_t[d] k_t[d] (v_t·gy_t).
+ *   r, k, v, gy   [B,T,H,N] bf16, read.      gr, gk, gv [B,T,H,N] bf16, written.
+ *   omega         [B,T,H,N] fp32, read.      gomega [B,T,H,N] fp32, written (one value per
+ *                                            token and channel, as omega).
+ *   u             [H,N] fp32, read.          gu [H,N] fp32, OVERWRITTEN with the sum over
+ *                                            batch and time.
+ *   s_in          [B,H,N,N] fp32, the forward's initial state, or NULL (zero).
+ *   gs_out        [B,H,N,N] fp32, the gradient of the final state, or NULL (zero).
+ *   gs_in         [B,H,N,N] fp32, written with the gradient of s_in, or NULL (not wanted).
+ *   workspace     device scratch of rwkv_wkv6_backward_workspace_bytes() bytes (the forward
+ *                 states at every 64th token, per-CTA scratch, the gu parts);
+ *                 RWKV_ERR_WORKSPACE if smaller.
+ *   N must be 64 and every tensor 16-byte aligned (RWKV_ERR_UNSUPPORTED otherwise).
+ *   Any decay w in [0, 1]: the recurrence runs token by token on the CUDA cores,
+ *   so no factorization range applies.  Deterministic (gu is reduced in a fixed
+ *   order).  Runs on `stream` only; allocates nothing.
+ */
+RWKV_API rwkv_status rwkv_wkv6_backward(int64_t B, int64_t T, int64_t H, int64_t N, const void *r, const void *k,
+                               const void *v, const float *omega, const float *u, const float *s_in,
+                               const void *gy, const float *gs_out, void *gr, void *gk, void *gv,
+                               float *gomega, float *gu, float *gs_in, void *workspace, size_t workspace_bytes,
+                               rwkv_stream_t stream);
+
 /* Largest B * C that rwkv_wkv4_backward_noalloc accepts. */
 #define RWKV_NOALLOC_MAX_LANES 262144
 

@@ -22,7 +22,8 @@ __all__ = [
     "LIB_PATH", "lib", "RwkvError", "RWKV_OK", "F32", "BF16", "ALGO_AUTO", "ALGO_SEQUENTIAL",
     "ALGO_CHUNKED", "CHUNK_LEN", "NOALLOC_MAX_LANES", "rwkv_wkv4_forward", "rwkv_wkv4_backward",
     "rwkv_wkv4_backward_noalloc", "rwkv_wkv4_step", "rwkv_wkv4_forward_gated", "rwkv_wkv4_backward_gated",
-    "rwkv_wkv5_forward", "rwkv_wkv5_backward", "rwkv_wkv5_step", "rwkv_wkv6_forward", "rwkv_wkv6_step", "rwkv_check_device_error",
+    "rwkv_wkv5_forward", "rwkv_wkv5_backward", "rwkv_wkv5_step", "rwkv_wkv6_forward", "rwkv_wkv6_backward",
+    "rwkv_wkv6_step", "rwkv_check_device_error",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "librwkv_wkv.so")
@@ -72,6 +73,8 @@ def lib():
         "rwkv_wkv5_backward": ([I64, I64, I64, I64] + [P] * 15 + [S, P], I),
         "rwkv_wkv6_forward_workspace_bytes": ([I64, I64, I64, I64], S),
         "rwkv_wkv6_forward": ([I64, I64, I64, I64, P, P, P, P, P, P, P, P, P, S, P], I),
+        "rwkv_wkv6_backward_workspace_bytes": ([I64, I64, I64, I64], S),
+        "rwkv_wkv6_backward": ([I64, I64, I64, I64] + [P] * 15 + [S, P], I),
         "rwkv_wkv6_step": ([I64, I64, I64, P, P, P, P, P, P, P, P, P], I),
         "rwkv_check_device_error": ([P], I),
         "rwkv_debug_set_wait_limit_ns": ([ctypes.c_uint64], I),
@@ -357,6 +360,38 @@ def rwkv_wkv5_backward(r, k, v, omega, u, gy, s_in=None, gs_out=None, *, want_gs
     ws = torch.empty(max(wsb, 1), dtype=torch.uint8, device=r.device)
     _check("rwkv_wkv5_backward",
            h.rwkv_wkv5_backward(B, T, H, N, _ptr(r), _ptr(k), _ptr(v), _ptr(omega), _ptr(u), _ptr(s_in), _ptr(gy),
+                                _ptr(gs_out), _ptr(gr), _ptr(gk), _ptr(gv), _ptr(gomega), _ptr(gu), _ptr(gsi),
+                                _ptr(ws), wsb, _stream(stream)))
+    res = (gr, gk, gv, gomega, gu)
+    return res + (gsi,) if want_gs_in else res
+
+
+def rwkv_wkv6_backward(r, k, v, omega, u, gy, s_in=None, gs_out=None, *, want_gs_in=False, stream=None):
+    """Finch / RWKV-6 backward: gradients of sum(gy * y) + sum(gs_out * s_out).  r, k, v, gy
+    [B,T,H,N] bf16; omega [B,T,H,N] fp32 (per token); u [H,N] fp32; s_in, gs_out [B,H,N,N] fp32 or
+    None.  Returns (gr, gk, gv, gomega [B,T,H,N], gu [H,N]) and, with ``want_gs_in``, the gradient
+    of s_in as well."""
+    import torch
+
+    _need_cuda(r, k, v, omega, u, gy, s_in, gs_out)
+    B, T, H, N = r.shape
+    for t in (r, k, v, gy):
+        if t.dtype != torch.bfloat16 or t.shape != r.shape:
+            raise ValueError("r, k, v, gy must be bf16 of the same shape")
+    _f32("omega", omega, B * T * H * N)
+    _f32("u", u, H * N)
+    for name, t in (("s_in", s_in), ("gs_out", gs_out)):
+        if t is not None:
+            _f32(name, t, B * H * N * N)
+    h = lib()
+    gr, gk, gv = torch.empty_like(r), torch.empty_like(k), torch.empty_like(v)
+    gomega = torch.empty((B, T, H, N), dtype=torch.float32, device=r.device)
+    gu = torch.empty((H, N), dtype=torch.float32, device=r.device)
+    gsi = torch.empty((B, H, N, N), dtype=torch.float32, device=r.device) if want_gs_in else None
+    wsb = int(h.rwkv_wkv6_backward_workspace_bytes(B, T, H, N))
+    ws = torch.empty(max(wsb, 1), dtype=torch.uint8, device=r.device)
+    _check("rwkv_wkv6_backward",
+           h.rwkv_wkv6_backward(B, T, H, N, _ptr(r), _ptr(k), _ptr(v), _ptr(omega), _ptr(u), _ptr(s_in), _ptr(gy),
                                 _ptr(gs_out), _ptr(gr), _ptr(gk), _ptr(gv), _ptr(gomega), _ptr(gu), _ptr(gsi),
                                 _ptr(ws), wsb, _stream(stream)))
     res = (gr, gk, gv, gomega, gu)

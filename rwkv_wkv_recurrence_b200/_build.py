@@ -18,7 +18,7 @@ LIB = os.path.join(PKG, "librwkv_wkv.so")
 HEADER = os.path.join(ROOT, "include", "rwkv_wkv.h")
 
 SOURCES = ["api.cu", "wkv4_fwd.cu", "wkv4_bwd.cu", "wkv4_bwd_noalloc.cu", "wkv4_step.cu", "wkv5_fwd.cu", "wkv6_fwd.cu",
-           "wkv5_step.cu", "wkv5_bwd.cu"]
+           "wkv5_step.cu", "wkv5_bwd.cu", "wkv6_bwd.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

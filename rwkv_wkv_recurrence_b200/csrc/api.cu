@@ -800,6 +800,72 @@ rwkv_status rwkv_wkv5_backward(int64_t B, int64_t T, int64_t H, int64_t N, const
   return RWKV_OK;
 }
 
+size_t rwkv_wkv6_backward_workspace_bytes(int64_t B, int64_t T, int64_t H, int64_t N) {
+  if (B <= 0 || T <= 0 || H <= 0 || N != 64) return 0;
+  if (!fits_int(B) || !fits_int(T) || !fits_int(H)) return 0;
+  auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  return up(wkv6_bwd_ckpt_floats((int)B, (int)T, (int)H) * 4) + up(wkv6_bwd_sub_floats((int)B, (int)H) * 4) +
+         up((size_t)B * H * 64 * 8);
+}
+
+rwkv_status rwkv_wkv6_backward(int64_t B, int64_t T, int64_t H, int64_t N, const void* r, const void* k,
+                               const void* v, const float* omega, const float* u, const float* s_in, const void* gy,
+                               const float* gs_out, void* gr, void* gk, void* gv, float* gomega, float* gu,
+                               float* gs_in, void* workspace, size_t workspace_bytes, rwkv_stream_t stream) {
+  if (!fits_int(B) || !fits_int(T) || !fits_int(H) || !fits_int(N)) return RWKV_ERR_INVALID_ARG;
+  if (N != 64) return RWKV_ERR_UNSUPPORTED;
+  if (B == 0 || H == 0) return RWKV_OK;
+  if (u == nullptr || gu == nullptr) return RWKV_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (T == 0) {  // no tokens: gu is an empty sum and the state gradient passes through
+    if (cudaMemsetAsync(gu, 0, H * 64 * sizeof(float), st) != cudaSuccess) return RWKV_ERR_CUDA;
+    if (gs_in != nullptr) {
+      const size_t n = (size_t)B * H * 64 * 64 * sizeof(float);
+      cudaError_t e = gs_out ? cudaMemcpyAsync(gs_in, gs_out, n, cudaMemcpyDeviceToDevice, st)
+                             : cudaMemsetAsync(gs_in, 0, n, st);
+      if (e != cudaSuccess) return RWKV_ERR_CUDA;
+    }
+    return RWKV_OK;
+  }
+  if (r == nullptr || k == nullptr || v == nullptr || gy == nullptr || omega == nullptr || gr == nullptr ||
+      gk == nullptr || gv == nullptr || gomega == nullptr)
+    return RWKV_ERR_INVALID_ARG;
+  if (!aligned16(r) || !aligned16(k) || !aligned16(v) || !aligned16(gy) || !aligned16(omega) || !aligned16(gr) ||
+      !aligned16(gk) || !aligned16(gv) || !aligned16(gomega) || (s_in && !aligned16(s_in)) ||
+      (gs_out && !aligned16(gs_out)) || (gs_in && !aligned16(gs_in)))
+    return RWKV_ERR_UNSUPPORTED;
+  if ((int64_t)H * 64 > INT_MAX || (int64_t)B * H > INT_MAX || (int64_t)T + 64 > INT_MAX) return RWKV_ERR_UNSUPPORTED;
+  const size_t need = rwkv_wkv6_backward_workspace_bytes(B, T, H, N);
+  if (workspace == nullptr || workspace_bytes < need) return RWKV_ERR_WORKSPACE;
+  auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  char* ws = static_cast<char*>(workspace);
+  Wkv6BwdParams p{};
+  p.B = (int)B;
+  p.T = (int)T;
+  p.H = (int)H;
+  p.r = static_cast<const __nv_bfloat16*>(r);
+  p.k = static_cast<const __nv_bfloat16*>(k);
+  p.v = static_cast<const __nv_bfloat16*>(v);
+  p.gy = static_cast<const __nv_bfloat16*>(gy);
+  p.omega = omega;
+  p.u = u;
+  p.s_in = s_in;
+  p.gs_out = gs_out;
+  p.gr = static_cast<__nv_bfloat16*>(gr);
+  p.gk = static_cast<__nv_bfloat16*>(gk);
+  p.gv = static_cast<__nv_bfloat16*>(gv);
+  p.gomega = gomega;
+  p.gu = gu;
+  p.gs_in = gs_in;
+  const size_t ck_bytes = up(wkv6_bwd_ckpt_floats(p.B, p.T, p.H) * 4);
+  const size_t sub_bytes = up(wkv6_bwd_sub_floats(p.B, p.H) * 4);
+  p.ckpt = reinterpret_cast<float*>(ws);
+  p.sub = reinterpret_cast<float*>(ws + ck_bytes);
+  p.part = reinterpret_cast<double*>(ws + ck_bytes + sub_bytes);
+  if (launch_wkv6_bwd(p, st) != cudaSuccess) return RWKV_ERR_CUDA;
+  return RWKV_OK;
+}
+
 rwkv_status rwkv_check_device_error(rwkv_stream_t stream) {
   if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return RWKV_ERR_CUDA;
   unsigned int v = 0;

@@ -112,6 +112,33 @@ struct Wkv5BwdParams {
   DevCtl* ctl;
 };
 
+// Finch backward (wkv6_bwd.cu): one CTA per (batch row, head) runs the recurrence forward (gr, the
+// state at every 64th token into ckpt) and then backward (gk, gv, the per-token gomega, gs_in and the
+// gu parts); a second kernel sums the gu parts over the batch.
+struct Wkv6BwdParams {
+  int B, T, H;
+  const __nv_bfloat16* r;
+  const __nv_bfloat16* k;
+  const __nv_bfloat16* v;
+  const __nv_bfloat16* gy;
+  const float* omega;    // [B,T,H,64]
+  const float* u;        // [H,64]
+  const float* s_in;     // [B,H,64,64] or null (zero)
+  const float* gs_out;   // [B,H,64,64] or null (zero)
+  __nv_bfloat16* gr;
+  __nv_bfloat16* gk;
+  __nv_bfloat16* gv;
+  float* gomega;         // [B,T,H,64]
+  float* gu;             // [H,64]
+  float* gs_in;          // [B,H,64,64] or null (not wanted)
+  float* ckpt;           // wkv6_bwd_ckpt_floats() floats of workspace
+  float* sub;            // wkv6_bwd_sub_floats() floats of workspace
+  double* part;          // [B,H,64] gu parts
+};
+size_t wkv6_bwd_ckpt_floats(int B, int T, int H);
+size_t wkv6_bwd_sub_floats(int B, int H);
+cudaError_t launch_wkv6_bwd(const Wkv6BwdParams& p, cudaStream_t st);
+
 int fwd_tile_steps();
 int fwd_store_steps();
 // Stage count of the forward's input pipeline (1 on the plain-access path, which has no pipeline).
