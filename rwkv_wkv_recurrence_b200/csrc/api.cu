@@ -804,8 +804,8 @@ size_t rwkv_wkv6_backward_workspace_bytes(int64_t B, int64_t T, int64_t H, int64
   if (B <= 0 || T <= 0 || H <= 0 || N != 64) return 0;
   if (!fits_int(B) || !fits_int(T) || !fits_int(H)) return 0;
   auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
-  return up(wkv6_bwd_ckpt_floats((int)B, (int)T, (int)H) * 4) + up(wkv6_bwd_sub_floats((int)B, (int)H) * 4) +
-         up((size_t)B * H * 64 * 8);
+  return 2 * up(wkv6_bwd_block_floats((int)B, (int)T, (int)H) * 4) +
+         2 * up(wkv6_bwd_row_floats((int)B, (int)T, (int)H) * 4);
 }
 
 rwkv_status rwkv_wkv6_backward(int64_t B, int64_t T, int64_t H, int64_t N, const void* r, const void* k,
@@ -857,11 +857,12 @@ rwkv_status rwkv_wkv6_backward(int64_t B, int64_t T, int64_t H, int64_t N, const
   p.gomega = gomega;
   p.gu = gu;
   p.gs_in = gs_in;
-  const size_t ck_bytes = up(wkv6_bwd_ckpt_floats(p.B, p.T, p.H) * 4);
-  const size_t sub_bytes = up(wkv6_bwd_sub_floats(p.B, p.H) * 4);
-  p.ckpt = reinterpret_cast<float*>(ws);
-  p.sub = reinterpret_cast<float*>(ws + ck_bytes);
-  p.part = reinterpret_cast<double*>(ws + ck_bytes + sub_bytes);
+  const size_t blk_bytes = up(wkv6_bwd_block_floats(p.B, p.T, p.H) * 4);
+  const size_t row_bytes = up(wkv6_bwd_row_floats(p.B, p.T, p.H) * 4);
+  p.xs = reinterpret_cast<float*>(ws);
+  p.xg = reinterpret_cast<float*>(ws + blk_bytes);
+  p.dec = reinterpret_cast<float*>(ws + 2 * blk_bytes);
+  p.part = reinterpret_cast<float*>(ws + 2 * blk_bytes + row_bytes);
   if (launch_wkv6_bwd(p, st) != cudaSuccess) return RWKV_ERR_CUDA;
   return RWKV_OK;
 }

@@ -112,9 +112,10 @@ struct Wkv5BwdParams {
   DevCtl* ctl;
 };
 
-// Finch backward (wkv6_bwd.cu): one CTA per (batch row, head) runs the recurrence forward (gr, the
-// state at every 64th token into ckpt) and then backward (gk, gv, the per-token gomega, gs_in and the
-// gu parts); a second kernel sums the gu parts over the batch.
+// Finch backward (wkv6_bwd.cu), chunk-parallel: per 64-token chunk the state and gradient increments
+// and the decay product (xs, xg, dec); per (batch row, head) the state entering and the gradient
+// leaving every chunk (in place over xs, xg) and gs_in; per chunk gr, gk, gv, gomega and the gu
+// parts; the gu parts summed over batch rows and chunks.
 struct Wkv6BwdParams {
   int B, T, H;
   const __nv_bfloat16* r;
@@ -131,12 +132,13 @@ struct Wkv6BwdParams {
   float* gomega;         // [B,T,H,64]
   float* gu;             // [H,64]
   float* gs_in;          // [B,H,64,64] or null (not wanted)
-  float* ckpt;           // wkv6_bwd_ckpt_floats() floats of workspace
-  float* sub;            // wkv6_bwd_sub_floats() floats of workspace
-  double* part;          // [B,H,64] gu parts
+  float* xs;             // wkv6_bwd_block_floats() floats of workspace
+  float* xg;             // wkv6_bwd_block_floats() floats
+  float* dec;            // wkv6_bwd_row_floats() floats
+  float* part;           // wkv6_bwd_row_floats() floats (gu parts)
 };
-size_t wkv6_bwd_ckpt_floats(int B, int T, int H);
-size_t wkv6_bwd_sub_floats(int B, int H);
+size_t wkv6_bwd_block_floats(int B, int T, int H);
+size_t wkv6_bwd_row_floats(int B, int T, int H);
 cudaError_t launch_wkv6_bwd(const Wkv6BwdParams& p, cudaStream_t st);
 
 int fwd_tile_steps();
