@@ -359,24 +359,29 @@ __global__ void __launch_bounds__(kThreads, 1) wkv6_bwd_chunk_kernel(const Wkv6B
   {
     float s[kBlock];
     load_own(p.xs + slot, s);
-    for (int t = 0; t < cnt; ++t) {
-      if (t % kS == 0) {
+    const float ud = sm.uu[dr];
+    for (int tb = 0; tb < cnt; tb += kS) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-          sm.sub[t / kS][i][tid] = make_float4(s[4 * i], s[4 * i + 1], s[4 * i + 2], s[4 * i + 3]);
+      for (int i = 0; i < 4; ++i)
+        sm.sub[tb / kS][i][tid] = make_float4(s[4 * i], s[4 * i + 1], s[4 * i + 2], s[4 * i + 3]);
+#pragma unroll
+      for (int m = 0; m < kS; ++m) {
+        const int t = tb + m;
+        if (t < cnt) {
+          float gf[4], part[4];
+          bf16x4(&S.g[t][j0], gf);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            part[i] = s[4 * i] * gf[0];
+#pragma unroll
+            for (int cc = 1; cc < 4; ++cc) part[i] = fmaf(s[4 * i + cc], gf[cc], part[i]);
+          }
+          const float x = butterfly4(part, lane);
+          if ((lane & 3) == 0)
+            p.gr[tok_off(p, bb, h, t0 + t) + dr] = __float2bfloat16_rn(fmaf(ud * bf(S.k[t][dr]), sm.vg[t], x));
+          state_step(s, S, sm.w, t, d0, j0);
+        }
       }
-      float gf[4], part[4];
-      bf16x4(&S.g[t][j0], gf);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        part[i] = s[4 * i] * gf[0];
-#pragma unroll
-        for (int cc = 1; cc < 4; ++cc) part[i] = fmaf(s[4 * i + cc], gf[cc], part[i]);
-      }
-      const float x = butterfly4(part, lane);
-      if ((lane & 3) == 0)
-        p.gr[tok_off(p, bb, h, t0 + t) + dr] = __float2bfloat16_rn(fmaf(sm.uu[dr] * bf(S.k[t][dr]), sm.vg[t], x));
-      state_step(s, S, sm.w, t, d0, j0);
     }
   }
 

@@ -1,6 +1,6 @@
-// Per-chunk WKV recurrence on the CUDA cores (sm_100a), shared by the Eagle and
-// Finch tensor-core kernels for chunks whose decay is too fast for their
-// chunked factorization (some channel's decay leaves the fp32 range there).
+// Per-chunk WKV recurrence on the CUDA cores (sm_100a), used by the Finch
+// tensor-core kernel for chunks whose decay is too fast for its chunked
+// factorization (some channel's decay leaves the fp32 range there).
 //
 // "RWKV-5 Eagle과 RWKV-6 Finch", sections Eagle and Finch: per token t of the
 // chunk, with the state s[d][j] (key d, value j) entering the chunk,
