@@ -249,7 +249,7 @@ __global__ void __launch_bounds__(kThreads, REV ? 1 : 2) wkv5_bwd_tc_kernel(cons
     prefetch_tensormap(&mc);
     mbar_init(&sm.bar_tma, 1);
     mbar_init(&sm.bar_sc, 1);
-    mbar_init(&sm.bar_av, 1);
+    mbar_init(&sm.bar_av, REV ? 2 : 1);  // reversed: the intra and lag-weighted chains commit apart
     mbar_init(&sm.bar_ds, 1);
     mbar_init(&sm.bar_ck, 1);
     fence_mbar_init();
@@ -346,6 +346,7 @@ __global__ void __launch_bounds__(kThreads, REV ? 1 : 2) wkv5_bwd_tc_kernel(cons
   // that c stays readable for the fast rows' terms
   __nv_bfloat16* stO = reinterpret_cast<__nv_bfloat16*>(sm.opP);
   const bool issuer = tid == 0;
+  const bool ds_issuer = tid == 128;  // warp 4 (q4 = 0, hc = 1): its scores quarter lies above the diagonal
 
   int c = 0;
   bool aborted = false;
@@ -469,12 +470,15 @@ __global__ void __launch_bounds__(kThreads, REV ? 1 : 2) wkv5_bwd_tc_kernel(cons
       fence_proxy_async();
       tc_fence_before();
       __syncthreads();
-      if (issuer) {
+      if (ds_issuer) {
         tc_fence_after();
-        // state increment c̃ᵀ p [d][j]: needs only this chunk's operands, runs while the scores are masked
+        // state increment c̃ᵀ p [d][j]: needs only this chunk's operands, runs while the scores are
+        // masked; issued from warp 4, whose share of the masking is a zero fill
   #pragma unroll
         for (int s = 0; s < 8; ++s) umma_tf32_ts(tDS, tCt + 8 * s, smem_desc(&sm.opPt[s * 64], kLbo, kSbo), kIdesc, s);
         umma_commit(&sm.bar_ds);
+      }
+      if (issuer) {
         // the raw boxes are consumed: load the next chunk while this one computes
         if (c + 1 < nchunk) {
           fence_proxy_async();
@@ -533,20 +537,27 @@ __global__ void __launch_bounds__(kThreads, REV ? 1 : 2) wkv5_bwd_tc_kernel(cons
       fence_proxy_async();
       tc_fence_before();
       __syncthreads();
+      // intra term: forward pass into the state-read accumulator, reversed pass into its own (the
+      // decay gradient weights the state read alone); reversed also the lag-weighted term, from a
+      // second thread (bar_av then takes two commits)
       if (issuer) {
         tc_fence_after();
-        // intra term: forward pass into the state-read accumulator, reversed pass into its own (the
-        // decay gradient weights the state read alone); reversed also the lag-weighted term
   #pragma unroll
         for (int s = 0; s < 8; ++s) {
-          if constexpr (REV) {
+          if constexpr (REV)
             umma_tf32_ts(tI, tCt + 8 * s, smem_desc(&sm.opAm[s * 64], kLbo, kSbo), kIdesc, s);
-            umma_tf32_ts(tX4, tCt + 8 * s, smem_desc(&sm.opAl[s * 64], kLbo, kSbo), kIdesc, s);
-          } else {
+          else
             umma_tf32_ts(tZ, tCt + 8 * s, smem_desc(&sm.opAm[s * 64], kLbo, kSbo), kIdesc, 1);
-          }
         }
         umma_commit(&sm.bar_av);
+      }
+      if constexpr (REV) {
+        if (ds_issuer) {
+          tc_fence_after();
+  #pragma unroll
+          for (int s = 0; s < 8; ++s) umma_tf32_ts(tX4, tCt + 8 * s, smem_desc(&sm.opAl[s * 64], kLbo, kSbo), kIdesc, s);
+          umma_commit(&sm.bar_av);
+        }
       }
 
       // T2b: X <- e^{nλ} X + e^{32λ} (c̃ᵀ p) with n the positions since the state entered
@@ -681,7 +692,10 @@ __global__ void __launch_bounds__(kThreads, REV ? 1 : 2) wkv5_bwd_tc_kernel(cons
   if (aborted && tid == 0) {
     // a wait gave up at chunk c: the last MMA chains and this chunk's loads must finish before the
     // tensor memory and shared memory are released, each wait bounded again
-    if (c >= 1) mbar_wait_bounded(&sm.bar_av, (uint32_t)(c - 1) & 1u, p.ctl);  // the last chains of c-1
+    if (c >= 1) {  // the last chains of c-1 (bar_av, and bar_ds from the second issuer)
+      mbar_wait_bounded(&sm.bar_av, (uint32_t)(c - 1) & 1u, p.ctl);
+      mbar_wait_bounded(&sm.bar_ds, (uint32_t)(c - 1) & 1u, p.ctl);
+    }
     if (!withheld) {
       mbar_wait_bounded(&sm.bar_tma, (uint32_t)c & 1u, p.ctl);
       if constexpr (REV) mbar_wait_bounded(&sm.bar_ck, (uint32_t)c & 1u, p.ctl);  // checkpoint copy c

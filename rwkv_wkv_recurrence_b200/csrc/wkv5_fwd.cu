@@ -260,6 +260,8 @@ __global__ void __launch_bounds__(kThreads, 2) wkv5_fwd_tc_kernel(const __grid_c
   const uint32_t tSc = tbase, tY = tbase + 64, tDS = tbase + 128, tKt = tbase + 192;
   const uint32_t rawR = smem_u32(sm.raw[0]), rawK = smem_u32(sm.raw[1]), rawV = smem_u32(sm.raw[2]);
   const bool issuer = tid == 0;
+  const bool ds_issuer = tid == 128;  // warp 4 (q4 = 0, hc = 1): its scores quarter lies above the diagonal
+  static_assert(kThreads > 128, "the state-increment chain's issuing thread");
 
   int c = 0;
   bool aborted = false;
@@ -437,12 +439,16 @@ __global__ void __launch_bounds__(kThreads, 2) wkv5_fwd_tc_kernel(const __grid_c
     fence_proxy_async();
     tc_fence_before();
     __syncthreads();
-    if (issuer) {
+    if (ds_issuer) {
       tc_fence_after();
-      // ΔS = k̃ᵀ v [d][j] needs only this chunk's operands: it runs while the scores are masked
+      // ΔS = k̃ᵀ v [d][j] needs only this chunk's operands: it runs while the scores are masked.
+      // Issued from warp 4, whose share of the masking is a zero fill, so that the ≈ 0.9k cycles
+      // the chain holds its issuing thread do not delay the masking barrier.
 #pragma unroll
       for (int s = 0; s < 8; ++s) umma_tf32_ts(tDS, tKt + 8 * s, smem_desc(&sm.opVt[s * 64], kLbo, kSbo), kIdesc, s);
       umma_commit(&sm.bar_ds);
+    }
+    if (issuer) {
       // the raw boxes are consumed: load the next chunk while this one computes
       if (c + 1 < nchunk) {
         fence_proxy_async();
@@ -559,10 +565,13 @@ __global__ void __launch_bounds__(kThreads, 2) wkv5_fwd_tc_kernel(const __grid_c
   }
 
   if (aborted && tid == 0) {
-    // a wait gave up at chunk c: the previous chunk's MMA chains (committed last on bar_av) and
-    // this chunk's loads must finish before the tensor memory and shared memory are released,
-    // each wait bounded again
-    if (c >= 1) mbar_wait_bounded(&sm.bar_av, (uint32_t)(c - 1) & 1u, p.ctl);
+    // a wait gave up at chunk c: the previous chunk's MMA chains (A v committed last by this
+    // thread on bar_av, ΔS by warp 4's on bar_ds) and this chunk's loads must finish before the
+    // tensor memory and shared memory are released, each wait bounded again
+    if (c >= 1) {
+      mbar_wait_bounded(&sm.bar_av, (uint32_t)(c - 1) & 1u, p.ctl);
+      mbar_wait_bounded(&sm.bar_ds, (uint32_t)(c - 1) & 1u, p.ctl);
+    }
     if (!withheld) mbar_wait_bounded(&sm.bar_tma, (uint32_t)c & 1u, p.ctl);
   }
   if (p.s_out != nullptr) {
