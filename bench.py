@@ -154,7 +154,7 @@ class ClockSampler:
 _TRAFFIC_SOURCES = {"wkv4_bwd_kernel": "wkv4_bwd", "wkv5_fwd_tc_kernel": "wkv5_fwd", "wkv4_step_kernel": "wkv4_step",
                     "wkv5_step_kernel": "wkv5_step", "wkv6_fwd_tc_kernel": "wkv6_fwd",
                     "wkv5_step_kernel/finch": "wkv5_step", "wkv4_bwd_kernel/gated": "wkv4_bwd",
-                    "rwkv_wkv5_backward": ("wkv5_fwd", "wkv5_bwd")}
+                    "rwkv_wkv5_backward": ("wkv5_fwd", "wkv5_bwd"), "rwkv_wkv6_backward": "wkv6_bwd"}
 
 
 def _kernel_source_hash(kernel="wkv4_bwd_kernel"):
@@ -836,7 +836,8 @@ def run_eagle_backward(args, finch=False):
         roof = {"bound": "alu", "kernel": "wkv6_bwd_kernel (+ its gu batch reduction)", "achieved": tf,
                 "peak": peak_tf, "peak_kind": "derived: 148 SMs x 128 fp32 FMA/clk x 2 flops x 1.965 GHz",
                 "unit": "TFLOP/s", "frac": tf / peak_tf, "hbm_gbs": nbytes / (ms * 1e-3) / 1e9,
-                "traffic": None}
+                # DRAM bytes of one call (its four launches), from the capture on the default decays
+                "traffic": _recorded_traffic("rwkv_wkv6_backward") if (om_lo, om_hi) == (-6.0, 0.0) else None}
         l2 = f"no flush: {nbytes / 1e6:.0f} MB moved per call, above the 126 MB L2"
         launches = 2
     else:
