@@ -93,6 +93,38 @@ def test_wkv6_nan_decay_enters_the_state(cuda_device):
     assert torch.equal(y1[mask], y0[mask])
 
 
+@pytest.mark.parametrize("finch", [False, True])
+def test_matrix_state_backward_nan_stays_in_its_head(cuda_device, finch):
+    # a NaN in gy at (b=1, t=120, h=2, j=5): every gradient of that (batch row, head) may turn NaN,
+    # and gomega / gu of head 2 (sums over the batch); every other (batch row, head) and the other
+    # heads' sums are bit for bit those of the clean run
+    B, T, H = 2, 200, 3
+    p = _cuda((wi.wkv6_problem if finch else wi.wkv5_problem)(B, T, H, 64, seed=54), cuda_device)
+    g = _cuda(wi.wkv5_grads(B, T, H, 64, seed=55, states=True), cuda_device)
+    bwd = rw.rwkv_wkv6_backward if finch else rw.rwkv_wkv5_backward
+    clean = bwd(p["r"], p["k"], p["v"], p["omega"], p["u"], g["gy"], g["s_in"], g["gs_out"], want_gs_in=True)
+    gy = g["gy"].clone()
+    gy[1, 120, 2, 5] = float("nan")
+    dirty = bwd(p["r"], p["k"], p["v"], p["omega"], p["u"], gy, g["s_in"], g["gs_out"], want_gs_in=True)
+    rw.rwkv_check_device_error()
+    assert torch.isnan(dirty[0][1, 120, 2].float()).any()  # gr of the token itself
+    for i, name in enumerate(("gr", "gk", "gv")):
+        m = torch.ones_like(dirty[i], dtype=torch.bool)
+        m[1, :, 2] = False
+        assert torch.equal(dirty[i][m], clean[i][m]), name
+    om_clean, om_dirty = clean[3], dirty[3]
+    if finch:  # per token: the other (batch row, head) pairs
+        m = torch.ones_like(om_dirty, dtype=torch.bool)
+        m[1, :, 2] = False
+        assert torch.equal(om_dirty[m], om_clean[m]), "gomega"
+    else:  # per head, summed over the batch
+        assert torch.equal(om_dirty[:2], om_clean[:2]), "gomega"
+    assert torch.equal(dirty[4][:2], clean[4][:2]), "gu"
+    m = torch.ones_like(dirty[5], dtype=torch.bool)
+    m[1, 2] = False
+    assert torch.equal(dirty[5][m], clean[5][m]), "gs_in"
+
+
 def test_wkv4_past_2pow31_elements(cuda_device):
     # B=2, T=2^19+2^12, C=2048 fp32: 2.16e9 elements per tensor.  The last 2048 steps of batch 1 (the
     # highest offsets) against the oracle from the GPU's own state before them, for 8 channels;

@@ -72,19 +72,23 @@ def test_matrix_state_step_graph(cuda_device, finch):
     _replay_equals_eager(cuda_device, run)
 
 
+@pytest.mark.parametrize("finch", [False, True])
 @pytest.mark.parametrize("with_state", [False, True])
-def test_eagle_forward_and_backward_graph(cuda_device, with_state):
+def test_matrix_state_forward_and_backward_graph(cuda_device, with_state, finch):
     # the Eagle forward and backward (whose reversed forward pass runs on a side stream, forked
-    # and joined with events) captured in one graph, replayed: bit for bit the eager results
+    # and joined with events), or the Finch forward and backward (four launches), captured in one
+    # graph, replayed: bit for bit the eager results
     B, T, H = 2, 150, 3
-    p = {k: v.to(cuda_device) for k, v in wi.wkv5_problem(B, T, H, 64, seed=63).items()}
+    gen = wi.wkv6_problem if finch else wi.wkv5_problem
+    p = {k: v.to(cuda_device) for k, v in gen(B, T, H, 64, seed=63).items()}
     g = {k: v.to(cuda_device) for k, v in wi.wkv5_grads(B, T, H, 64, seed=64, states=with_state).items()}
+    fwd = rw.rwkv_wkv6_forward if finch else rw.rwkv_wkv5_forward
+    bwd = rw.rwkv_wkv6_backward if finch else rw.rwkv_wkv5_backward
 
     def run():
-        y = rw.rwkv_wkv5_forward(p["r"], p["k"], p["v"], p["omega"], p["u"], g.get("s_in"),
-                                 stream=torch.cuda.current_stream())
-        grads = rw.rwkv_wkv5_backward(p["r"], p["k"], p["v"], p["omega"], p["u"], g["gy"], g.get("s_in"),
-                                      g.get("gs_out"), want_gs_in=True, stream=torch.cuda.current_stream())
+        y = fwd(p["r"], p["k"], p["v"], p["omega"], p["u"], g.get("s_in"), stream=torch.cuda.current_stream())
+        grads = bwd(p["r"], p["k"], p["v"], p["omega"], p["u"], g["gy"], g.get("s_in"), g.get("gs_out"),
+                    want_gs_in=True, stream=torch.cuda.current_stream())
         return (y,) + tuple(grads)
 
     eager = run()

@@ -3,7 +3,8 @@ WKV-4 kernels.
 
 Each output is carved out of a larger buffer whose head and tail hold a
 sentinel; after the call the sentinel must be intact (no write outside the
-output) and the output must match the fp64 oracle.  compute-sanitizer is not
+output) and the output must match the fp64 oracle (the Eagle and Finch backward
+too, every one of their six outputs).  compute-sanitizer is not
 available, so this is the out-of-bounds check of every entry point.
 
 The WKV-4 calls are exercised on both of their paths: tensors whose bases are
@@ -228,6 +229,35 @@ def test_matrix_state_guarded(cuda_device, finch):
     s1.check("step s_out")
     ref1 = (oracle.wkv6_forward if finch else oracle.wkv5_forward)(q["r"], q["k"], q["v"], q["omega"], q["u"])
     assert_close_rms(ys.t, ref1[:, T], TOL_BF16, "step y")
+
+
+@pytest.mark.parametrize("finch", [False, True])
+def test_matrix_state_backward_guarded(cuda_device, finch):
+    # the Eagle and Finch backward: every output (gr, gk, gv, gomega, gu, gs_in) carved out of a
+    # sentinel-guarded buffer, checked against the oracle
+    B, T, H = 2, 130, 3
+    dev = cuda_device
+    p = (wi.wkv6_problem if finch else wi.wkv5_problem)(B, T, H, 64, seed=75)
+    g = wi.wkv5_grads(B, T, H, 64, seed=76, states=True)
+    c = {k: v.to(dev) for k, v in list(p.items()) + list(g.items())}
+    h = rw.lib()
+    P, S = rw._ptr, rw._stream(None)
+    outs = {name: Guarded((B, T, H, 64), torch.bfloat16, dev) for name in ("gr", "gk", "gv")}
+    outs["gomega"] = Guarded((B, T, H, 64) if finch else (H, 64), torch.float32, dev)
+    outs["gu"] = Guarded((H, 64), torch.float32, dev)
+    outs["gs_in"] = Guarded((B, H, 64, 64), torch.float32, dev)
+    name = "rwkv_wkv6_backward" if finch else "rwkv_wkv5_backward"
+    wsb = int(getattr(h, name + "_workspace_bytes")(B, T, H, 64))
+    ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
+    assert getattr(h, name)(B, T, H, 64, P(c["r"]), P(c["k"]), P(c["v"]), P(c["omega"]), P(c["u"]), P(c["s_in"]),
+                            P(c["gy"]), P(c["gs_out"]), outs["gr"].ptr(), outs["gk"].ptr(), outs["gv"].ptr(),
+                            outs["gomega"].ptr(), outs["gu"].ptr(), outs["gs_in"].ptr(), P(ws), wsb, S) == 0
+    rw.rwkv_check_device_error()
+    ref = (oracle.wkv6_backward if finch else oracle.wkv5_backward)(p["r"], p["k"], p["v"], p["omega"], p["u"],
+                                                                   g["gy"], s_in=g["s_in"], gs_out=g["gs_out"])
+    for key, want in zip(("gr", "gk", "gv", "gomega", "gu", "gs_in"), ref):
+        outs[key].check(key)
+        assert_close_rms(outs[key].t, want, TOL_BF16, key)
 
 
 def test_element_misaligned_pointer_is_refused(cuda_device):
