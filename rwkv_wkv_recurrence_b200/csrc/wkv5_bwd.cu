@@ -57,14 +57,19 @@
 // factors beyond e^{±64} would push small operands into the subnormal range)
 // stays out of the factorized products: its c̃ᵀ row is zero, its state row is
 // read unscaled and its output takes e^{λ(τ-lo)}.  Its intra-chunk terms (the
-// plain one and, reversed, the lag-weighted one) are summed on the CUDA cores in
-// the epilogue over lags 0..15, from the masked scores and the staged c rows,
-// and its state increment in the fold over the chunk's last 16 positions:
-// beyond that e^{λn} < 2^-46 of the lag-0 weight.  Any w in [0, 1] is handled.
+// plain one and, reversed, the lag-weighted one) are summed on the CUDA cores
+// over lags 0..15 by all threads, from the masked scores and the staged c rows,
+// into operand tiles that are free at that point, and read by that row's
+// epilogue; its state increment is summed in the fold over the chunk's last 16
+// positions: beyond that e^{λn} < 2^-46 of the lag-0 weight.  Any w in [0, 1]
+// is handled.  Heads without fast rows run a second instance of the chunk loop
+// that has none of this code.
 //
-// CTA: one (batch, head), 8 warps.  Forward pass: ~110 KB of shared memory,
-// 256 TMEM columns, two CTAs per SM.  Reversed pass: ~145 KB, 512 columns, one
-// CTA per SM.
+// CTA: one (batch, head), 8 warps.  Forward pass: ~112 KB of shared memory,
+// 256 TMEM columns, two CTAs per SM.  Reversed pass: ~146 KB, 512 columns, one
+// CTA per SM.  Thread 0 issues the TMA loads and the scores, state-read and
+// intra chains; a thread of warp 4 (whose share of the masking is a zero fill)
+// issues the state-increment chain and, reversed, the lag-weighted chain.
 #include <cstddef>
 #include <type_traits>
 

@@ -49,11 +49,14 @@
 // the data allows (N = 128 for the first chain) and the issuing thread hands
 // the first chain out in pairs between the other work of its warp.
 //
-// CTA: one (batch, head), 8 warps, about 90 KB of shared memory and 256 TMEM
+// CTA: one (batch, head), 8 warps, about 113 KB of shared memory and 256 TMEM
 // columns, two CTAs per SM.  Thread 0 issues the TMA loads of the raw r, k, v
-// tiles (one [64 tokens x 64] bf16 box each, 128-byte swizzle, no multicast)
-// and the MMAs; all warps build operands, mask the scores, fold the state and
-// write the output rows.
+// tiles (one [64 tokens x 64] bf16 box each, 128-byte swizzle, no multicast),
+// the scores chain and the A v chain; a thread of warp 4 (whose share of the
+// masking is a zero fill) issues the state-increment chain, so that the time
+// that chain holds its issuing thread does not delay the masking barrier.  All
+// warps build operands, mask the scores, fold the state and write the output
+// rows.
 #include <cstddef>
 
 #include "launch.h"
