@@ -165,6 +165,36 @@ def test_validation_before_any_cuda_work():
     assert h.rwkv_wkv6_step(2, 3, 64, fake, fake, fake, fake, fake, fake, None, None, None) == 1
     assert h.rwkv_wkv6_step(2, 3, 64, fake, fake, fake, fake, fake, fake, None, P(0x1004), None) == 2
     assert h.rwkv_wkv6_step(0, 3, 64, fake, fake, fake, fake, fake, fake, None, fake, None) == 0
+    # WKV-5 / WKV-6 backward: only N = 64; the tensors and gradients required and 16-byte aligned; the
+    # workspace at least the query's size; B = 0 a no-op
+    for name in ("rwkv_wkv5_backward", "rwkv_wkv6_backward"):
+        f = getattr(h, name)
+        ok = [fake] * 15  # r, k, v, omega, u, s_in, gy, gs_out, gr, gk, gv, gomega, gu, gs_in, workspace
+
+        def call(B=1, T=4, H=2, N=64, ptrs=None, wsb=1 << 30):
+            a = list(ok if ptrs is None else ptrs)
+            return f(B, T, H, N, *a[:14], a[14], wsb, None)
+
+        def with_ptr(i, val):
+            a = list(ok)
+            a[i] = val
+            return a
+
+        assert call(N=32) == 2, name
+        assert call(B=-1) == 1, name
+        assert call(B=0) == 0, name
+        assert call(ptrs=with_ptr(0, None)) == 1, name    # r
+        assert call(ptrs=with_ptr(6, None)) == 1, name    # gy
+        assert call(ptrs=with_ptr(12, None)) == 1, name   # gu
+        assert call(ptrs=with_ptr(10, None)) == 1, name   # gv
+        assert call(ptrs=with_ptr(1, P(0x1008))) == 2, name
+        assert call(ptrs=with_ptr(8, P(0x1004))) == 2, name
+        assert call(ptrs=with_ptr(14, None)) == 3, name   # no workspace
+        need = int(getattr(h, name + "_workspace_bytes")(1, 4, 2, 64))
+        assert need > 0 and call(wsb=need - 1) == 3, name
+    # the Finch backward runs one CTA per 64-token chunk: more than 2^31 - 1 chunks is refused
+    big = h.rwkv_wkv6_backward(1 << 16, 1 << 17, 1 << 10, 64, *([fake] * 15), 1 << 62, None)
+    assert big == 2
 
 
 def test_binding_fails_loudly_without_library(monkeypatch):
