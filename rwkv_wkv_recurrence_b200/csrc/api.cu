@@ -835,7 +835,8 @@ rwkv_status rwkv_wkv6_backward(int64_t B, int64_t T, int64_t H, int64_t N, const
       (gs_out && !aligned16(gs_out)) || (gs_in && !aligned16(gs_in)))
     return RWKV_ERR_UNSUPPORTED;
   if ((int64_t)H * 64 > INT_MAX || (int64_t)B * H > INT_MAX || (int64_t)T + 64 > INT_MAX) return RWKV_ERR_UNSUPPORTED;
-  if ((int64_t)B * H * ((T + 63) / 64) > INT_MAX) return RWKV_ERR_UNSUPPORTED;  // one CTA per 64-token chunk
+  // one CTA per 64-token chunk, and two per (batch row, head) for the boundary scans
+  if ((int64_t)B * H * ((T + 63) / 64) > INT_MAX || 2 * (int64_t)B * H > INT_MAX) return RWKV_ERR_UNSUPPORTED;
   const size_t need = rwkv_wkv6_backward_workspace_bytes(B, T, H, N);
   if (workspace == nullptr || workspace_bytes < need) return RWKV_ERR_WORKSPACE;
   auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };

@@ -20,9 +20,9 @@
 //   1. per chunk, in parallel: the chunk's own state increment ΔS (its tokens from a zero state),
 //      its own gradient increment ΔG = Σ_τ diag(Π_{a<=m<τ} w_m) r_τᵀ gy_τ (a = the chunk's first
 //      token) and its decay product D = Π_m w_m;
-//   2. per (batch row, head), sequentially over the chunks: the state entering every chunk,
-//      S_{c+1} = D_c ⊙ S_c + ΔS_c, and the gradient leaving it, G_{c-1} = ΔG_c + D_c ⊙ G_c
-//      (in place over the increments), and gs_in;
+//   2. per (batch row, head), sequentially over the chunks, one CTA per scan: the state entering
+//      every chunk, S_{c+1} = D_c ⊙ S_c + ΔS_c, and the gradient leaving it,
+//      G_{c-1} = ΔG_c + D_c ⊙ G_c (in place over the increments), and gs_in;
 //   3. per chunk, in parallel: the chunk's tokens forward from its entering state (gr_t, and the
 //      state every 8 tokens into shared memory), then backwards from its leaving gradient, 8
 //      tokens at a time: the 8 states are recomputed into registers and walked with G, forming gk,
@@ -247,55 +247,41 @@ __global__ void __launch_bounds__(kThreads) wkv6_bwd_sums_kernel(const Wkv6BwdPa
     *reinterpret_cast<float4*>(p.dec + ((size_t)bh * nch + c) * kN + d0) = make_float4(P[0], P[1], P[2], P[3]);
 }
 
-// 2. Per (batch row, head): the state entering every chunk and the gradient leaving it, in place
-//    over the increments, and gs_in.
+// 2. Per (batch row, head), two CTAs: the state entering every chunk (even CTA) and the gradient
+//    leaving it with gs_in (odd CTA), each in place over its increments.  The two scans are
+//    independent.
 __global__ void __launch_bounds__(kThreads) wkv6_bwd_carry_kernel(const Wkv6BwdParams p) {
   const int tid = threadIdx.x;
   const int d0 = 4 * (tid >> 4), j0 = 4 * (tid & 15);
   const int nch = (p.T + kL - 1) / kL;
-  const int bh = blockIdx.x;
+  const int bh = blockIdx.x >> 1;
+  const bool grad = blockIdx.x & 1;
   const size_t state_off = (size_t)bh * kN * kN;
-  float* xs = p.xs + (size_t)bh * nch * kN * kN;
-  float* xg = p.xg + (size_t)bh * nch * kN * kN;
+  float* xs = (grad ? p.xg : p.xs) + (size_t)bh * nch * kN * kN;
   const float* dec = p.dec + (size_t)bh * nch * kN;
+  const float* init = grad ? p.gs_out : p.s_in;
   float a[kBlock], x[kBlock], xn[kBlock];
-  if (p.s_in != nullptr)
-    load_block(p.s_in + state_off, d0, j0, a);
+  if (init != nullptr)
+    load_block(init + state_off, d0, j0, a);
   else
 #pragma unroll
     for (int e = 0; e < kBlock; ++e) a[e] = 0.f;
-  load_own(xs, x);
-  for (int c = 0; c < nch; ++c) {
-    if (c + 1 < nch) load_own(xs + (size_t)(c + 1) * kN * kN, xn);  // the next increment, ahead of the chain
+  // the state runs forward over the chunks, the gradient backward
+  const int c0 = grad ? nch - 1 : 0, dc = grad ? -1 : 1;
+  load_own(xs + (size_t)c0 * kN * kN, x);
+  for (int i = 0, c = c0; i < nch; ++i, c += dc) {
+    if (i + 1 < nch) load_own(xs + (size_t)(c + dc) * kN * kN, xn);  // the next increment, ahead of the chain
     const float4 D = *reinterpret_cast<const float4*>(dec + (size_t)c * kN + d0);
     const float df[4] = {D.x, D.y, D.z, D.w};
     save_own(xs + (size_t)c * kN * kN, a);
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+    for (int ii = 0; ii < 4; ++ii)
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) a[4 * i + cc] = fmaf(df[i], a[4 * i + cc], x[4 * i + cc]);
-#pragma unroll
-    for (int e = 0; e < kBlock; ++e) x[e] = xn[e];
-  }
-  if (p.gs_out != nullptr)
-    load_block(p.gs_out + state_off, d0, j0, a);
-  else
-#pragma unroll
-    for (int e = 0; e < kBlock; ++e) a[e] = 0.f;
-  load_own(xg + (size_t)(nch - 1) * kN * kN, x);
-  for (int c = nch - 1; c >= 0; --c) {
-    if (c >= 1) load_own(xg + (size_t)(c - 1) * kN * kN, xn);
-    const float4 D = *reinterpret_cast<const float4*>(dec + (size_t)c * kN + d0);
-    const float df[4] = {D.x, D.y, D.z, D.w};
-    save_own(xg + (size_t)c * kN * kN, a);
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int cc = 0; cc < 4; ++cc) a[4 * i + cc] = fmaf(df[i], a[4 * i + cc], x[4 * i + cc]);
+      for (int cc = 0; cc < 4; ++cc) a[4 * ii + cc] = fmaf(df[ii], a[4 * ii + cc], x[4 * ii + cc]);
 #pragma unroll
     for (int e = 0; e < kBlock; ++e) x[e] = xn[e];
   }
-  if (p.gs_in != nullptr) store_block(p.gs_in + state_off, d0, j0, a);
+  if (grad && p.gs_in != nullptr) store_block(p.gs_in + state_off, d0, j0, a);
 }
 
 // 3. Per chunk: gr forward in time from the entering state; gk, gv, gω backward from the leaving
@@ -490,7 +476,7 @@ cudaError_t launch_wkv6_bwd(const Wkv6BwdParams& p, cudaStream_t st) {
   e = ensure_smem_attr(reinterpret_cast<const void*>(wkv6_bwd_chunk_kernel), (int)sizeof(ChunkSmem), &mask_c);
   if (e != cudaSuccess) return e;
   wkv6_bwd_sums_kernel<<<nblk, kThreads, sizeof(SumsSmem), st>>>(p);
-  wkv6_bwd_carry_kernel<<<(unsigned)(p.B * p.H), kThreads, 0, st>>>(p);
+  wkv6_bwd_carry_kernel<<<(unsigned)(2LL * p.B * p.H), kThreads, 0, st>>>(p);
   wkv6_bwd_chunk_kernel<<<nblk, kThreads, sizeof(ChunkSmem), st>>>(p);
   wkv6_bwd_reduce_kernel<<<(p.H * kN + 127) / 128, 128, 0, st>>>(p.B, p.H, nch, p.part, p.gu);
   return cudaGetLastError();
