@@ -319,7 +319,8 @@ RWKV_API size_t rwkv_wkv6_backward_workspace_bytes(int64_t B, int64_t T, int64_t
  *                 states at every 64th token, per-CTA scratch, the gu parts);
  *                 RWKV_ERR_WORKSPACE if smaller.
  *   N must be 64 and every tensor 16-byte aligned, and B·H·ceil(T/64) (one CTA per
- *   64-token chunk) at most 2^31 - 1 (RWKV_ERR_UNSUPPORTED otherwise).
+ *   64-token chunk) and 2·B·H (two per head for the boundary scans) at most 2^31 - 1
+ *   (RWKV_ERR_UNSUPPORTED otherwise).
  *   Any decay w in [0, 1]: the recurrence runs token by token on the CUDA cores,
  *   so no factorization range applies.  Deterministic (gu is reduced in a fixed
  *   order).  Runs on `stream` only; allocates nothing.
