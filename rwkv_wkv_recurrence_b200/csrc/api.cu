@@ -120,6 +120,21 @@ struct FwdPlan {
   size_t ws_bytes;
 };
 
+// Workspace of the one-launch chunked forward: [nseg][B*C][3] doubles, then the flags.
+struct LookbackWs {
+  size_t agg, flag, flag_bytes, total;
+};
+LookbackWs lookback_ws(int64_t nseg, int64_t B, int64_t C) {
+  auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  LookbackWs w{};
+  const size_t states = (size_t)nseg * B * C * 3 * sizeof(double);
+  w.agg = 0;
+  w.flag = up(states);
+  w.flag_bytes = (size_t)nseg * ((C + 31) / 32) * B * sizeof(unsigned int);
+  w.total = w.flag + up(w.flag_bytes);
+  return w;
+}
+
 FwdPlan plan_forward(int64_t B, int64_t T, int64_t C, int algo) {
   FwdPlan pl{RWKV_ALGO_SEQUENTIAL, 0, 1, 0};
   const int tt = fwd_tile_steps();
@@ -141,7 +156,9 @@ FwdPlan plan_forward(int64_t B, int64_t T, int64_t C, int algo) {
       pl.algo = RWKV_ALGO_CHUNKED;
       pl.seg_len = (int)seg;
       pl.nseg = (int)nseg;
-      pl.ws_bytes = (size_t)nseg * 3 * B * C * sizeof(float);
+      // the one-launch form's per-segment summaries ((a, b, p) doubles) and flags; the three-launch
+      // form's fp32 states ([nseg][3][B*C]) fit in the same bytes
+      pl.ws_bytes = lookback_ws(nseg, B, C).total;
       return pl;
     }
   }
@@ -198,6 +215,27 @@ rwkv_status run_forward(int B, int T, int C, bool bf16, const float* w, const fl
     p.end = state_out;
     p.ckpt = ckpt;
     if (launch_out(p) != cudaSuccess) return RWKV_ERR_CUDA;
+    return RWKV_OK;
+  }
+  // one launch when every tile of a segment stays resident in the pipeline: summaries, look-back
+  // across segments, outputs
+  const int lb_stages = fwd_stages(bf16, pl.seg_len, false, tma);
+  if (tma && !gate && (pl.seg_len + tt - 1) / tt <= lb_stages) {
+    const LookbackWs L = lookback_ws(pl.nseg, B, C);
+    char* wsc = static_cast<char*>(ws);
+    if (cudaMemsetAsync(wsc + L.flag, 0, L.flag_bytes, st) != cudaSuccess) return RWKV_ERR_CUDA;
+    p.seg_len = pl.seg_len;
+    p.nseg = pl.nseg;
+    p.stages = lb_stages;
+    p.y = y;
+    p.start = nullptr;  // the first pass runs from a zero state
+    p.end = state_out;  // written by the last segment
+    p.end_seg_stride = 0;
+    p.ckpt = ckpt;
+    p.lb_agg = reinterpret_cast<double*>(wsc + L.agg);
+    p.lb_flag = reinterpret_cast<unsigned int*>(wsc + L.flag);
+    p.lb_in = state_in;
+    if (launch_wkv4_fwd_lookback(bf16, mk, mv, my, p, st) != cudaSuccess) return RWKV_ERR_CUDA;
     return RWKV_OK;
   }
   float* wsf = static_cast<float*>(ws);

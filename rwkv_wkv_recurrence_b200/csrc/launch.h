@@ -33,6 +33,12 @@ struct Fwd4Params {
   const void* v;
   const void* r;                  // [B,T,C] receptance of the gated forward (tma == 0), else null
   DevCtl* ctl;                    // device control block (error word, wait limit)
+  // the one-launch chunked schedule (launch_wkv4_fwd_lookback): per segment and lane the summary as
+  // (a, b, p) doubles, one flag per (segment, CTA) zeroed before the launch, and the sequence's
+  // start state (or null = zero)
+  double* lb_agg;                 // [nseg][B*C][3]
+  unsigned int* lb_flag;          // [nseg][ctiles*B]
+  const float* lb_in;             // [3,B,C] or null
 };
 
 struct Bwd4Params {
@@ -152,6 +158,10 @@ int bwd_stages(bool bf16, int T, bool gate = false, bool tma = true);
 // (TMA stores; any valid map when p.y is null).  With p.tma == 0 the maps are not read (any value).
 cudaError_t launch_wkv4_fwd(bool bf16, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& my,
                             const Fwd4Params& p, cudaStream_t st);
+// The chunked schedule in one launch (TMA only, every tile of a segment resident in the stages,
+// p.start null, p.end the final state written by the last segment, p.lb_* set).
+cudaError_t launch_wkv4_fwd_lookback(bool bf16, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& my,
+                                     const Fwd4Params& p, cudaStream_t st);
 // The receptance-gated forward: also reads r ([fwd_tile_steps() x 32] boxes) and writes σ(r) ⊙ WKV.
 cudaError_t launch_wkv4_fwd_gated(bool bf16, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& my,
                                   const CUtensorMap& mr, const Fwd4Params& p, cudaStream_t st);

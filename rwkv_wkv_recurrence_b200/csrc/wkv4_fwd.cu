@@ -103,7 +103,49 @@ struct CarrySlot {  // CTA running state at a tile boundary, per lane
   int p, pad;
 };
 
-template <typename T, bool GATE, bool TMA>
+// Look-back flags of the one-launch chunked schedule (release / acquire at GPU scope).
+__device__ __forceinline__ void flag_release(unsigned int* f, unsigned int v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(f), "r"(v) : "memory");
+}
+__device__ __forceinline__ unsigned int flag_acquire(const unsigned int* f) {
+  unsigned int v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(f) : "memory");
+  return v;
+}
+// Polls a flag until it is non-zero or the control block's time limit passes; 0 then (and the
+// timeout bit is set in the error word).
+__device__ __forceinline__ unsigned int flag_wait_bounded(const unsigned int* f, DevCtl* ctl) {
+  unsigned int v = flag_acquire(f);
+  if (v != 0u) return v;
+  const unsigned long long t0 = global_ns();
+  const unsigned long long limit = *reinterpret_cast<volatile unsigned long long*>(&ctl->wait_limit_ns);
+  while ((v = flag_acquire(f)) == 0u) {
+    if (global_ns() - t0 > limit) {
+      atomicOr(&ctl->err, kErrTmaTimeout);
+      return 0u;
+    }
+    __nanosleep(64);
+  }
+  return v;
+}
+
+// e^{-w len} in fp64: 16-step powers and the remainder, as the carry pass forms them.
+__device__ __forceinline__ double lam_len(double lam, double lam16, int len) {
+  double r = lam_pow(lam, len & 15);
+  for (int q = 0; q < (len >> 4); ++q) r *= lam16;
+  return r;
+}
+
+constexpr unsigned int kFlagAggregate = 1u;  // the segment's own summary is published
+
+// LB: the chunked schedule in one launch (p.lb_* set; TMA, every tile of the segment resident in
+// the pipeline's stages).  The CTA scans its resident tiles once from a zero state for its
+// segment's summary and publishes it; it then waits (bounded) until every earlier segment of its
+// lanes has published its own, folds them in order from the sequence's start state into its own
+// start state (the flags polled, and the summaries loaded, by all lanes at once: no chain of
+// round trips), and scans the same tiles again from that state for the outputs.  Every CTA of a
+// launch is resident at once (the schedule keeps to four CTAs per SM).
+template <typename T, bool GATE, bool TMA, bool LB>
 __global__ void __launch_bounds__(kW * 32, 4) wkv4_fwd_kernel(const __grid_constant__ CUtensorMap mk,
                                                               const __grid_constant__ CUtensorMap mv,
                                                               const __grid_constant__ CUtensorMap my,
@@ -173,11 +215,13 @@ __global__ void __launch_bounds__(kW * 32, 4) wkv4_fwd_kernel(const __grid_const
   __syncthreads();
 
   const bool write_y = p.y != nullptr;
-  const bool rescan = (p.y != nullptr) || (p.ckpt != nullptr);
   State total{0.0, 0.0, 0};
 
   int i = 0;
-  for (; i < ntile; ++i) {
+  for (int pass = 0; pass < (LB ? 2 : 1); ++pass) {
+  // LB: the first pass only sums the segment (from the zero state set above)
+  const bool rescan = (!LB || pass == 1) && ((p.y != nullptr) || (p.ckpt != nullptr));
+  for (i = 0; i < ntile; ++i) {
     const int s = i % p.stages;
     const uint32_t ph = (uint32_t)(i / p.stages) & 1u;
     if constexpr (TMA) {
@@ -276,10 +320,74 @@ __global__ void __launch_bounds__(kW * 32, 4) wkv4_fwd_kernel(const __grid_const
       }
     }
   }
+  if constexpr (LB) {
+    if (pass == 0) {
+      __syncthreads();
+      if (*abort_flag) break;
+      if (warp == kW - 1) {
+        // the segment's summary (total, from the zero state) out; the state before it in
+        const size_t ncta = (size_t)p.ctiles * p.B;
+        const size_t cta = (size_t)ct + (size_t)p.ctiles * bb;
+        const size_t me = ((size_t)seg * plane + lane_off) * 3;
+        if (valid) {
+          p.lb_agg[me] = total.a;
+          p.lb_agg[me + 1] = total.b;
+          p.lb_agg[me + 2] = (double)total.p;
+        }
+        __syncwarp();
+        if (lane == 0) {
+          __threadfence();
+          flag_release(&p.lb_flag[(size_t)seg * ncta + cta], kFlagAggregate);
+        }
+        // wait until every earlier segment has published its summary: the lanes poll up to 32
+        // flags at once (segment seg - 1 - lane, then 32 further back, ...)
+        bool failed = false;
+        for (int j0 = 0; j0 < seg && !failed; j0 += 32) {
+          const int j = seg - 1 - (j0 + lane);
+          unsigned int f = 1u;
+          if (j0 + lane < seg) f = flag_wait_bounded(&p.lb_flag[(size_t)j * ncta + cta], p.ctl);
+          failed = __any_sync(0xffffffffu, f == 0u);
+        }
+        // each lane reads after the acquires and the barrier, bypassing L1
+        __syncwarp();
+        if (failed) {
+          if (lane == 0) *abort_flag = 1;
+        } else {
+          State st{0.0, 0.0, 0};
+          if (valid) {
+            if (p.lb_in != nullptr)
+              st = load_state(p.lb_in[lane_off], p.lb_in[plane + lane_off], p.lb_in[2 * plane + lane_off]);
+            const double lam_seg = lam_len(lam, lam16, p.seg_len);  // every earlier segment is whole
+            // the earlier summaries in order, eight at a time, their loads in flight together
+            constexpr int kBatch = 8;
+            for (int m0 = 0; m0 < seg; m0 += kBatch) {
+              double ag[kBatch][3];
+#pragma unroll
+              for (int e = 0; e < kBatch; ++e) {
+                if (m0 + e < seg) {
+                  const size_t o = ((size_t)(m0 + e) * plane + lane_off) * 3;
+                  ag[e][0] = __ldcg(&p.lb_agg[o]);
+                  ag[e][1] = __ldcg(&p.lb_agg[o + 1]);
+                  ag[e][2] = __ldcg(&p.lb_agg[o + 2]);
+                }
+              }
+#pragma unroll
+              for (int e = 0; e < kBatch; ++e)
+                if (m0 + e < seg) st = fold(st, lam_seg, State{ag[e][0], ag[e][1], (int)ag[e][2]});
+            }
+          }
+          cslot[32 + lane] = CarrySlot{st.a, st.b, st.p, 0};  // the second pass starts from it
+        }
+      }
+      __syncthreads();
+      if (*abort_flag) break;
+    }
+  }
+  }
   if (TMA && threadIdx.x == 0 && *abort_flag) drain_loads(bars, p.stages, i, ntile, p.ctl);  // a wait gave up
   if (lane == 0) bulk_wait_all();
 
-  if (p.end != nullptr && valid && warp == kW - 1) {
+  if (p.end != nullptr && valid && warp == kW - 1 && !*abort_flag && (!LB || seg == p.nseg - 1)) {
     float* e = p.end + (size_t)seg * p.end_seg_stride;
     store_state(total, &e[lane_off], &e[plane + lane_off], &e[2 * plane + lane_off]);
   }
@@ -320,16 +428,16 @@ size_t fwd_smem_bytes(int stages) {  // also the plain path's (one stage)
          2 * 32 * sizeof(CarrySlot) + (size_t)stages * 8 + 16;
 }
 
-template <typename T, bool GATE, bool TMA>
+template <typename T, bool GATE, bool TMA, bool LB = false>
 cudaError_t launch_fwd_tt(const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& my, const CUtensorMap& mr,
                           const Fwd4Params& p, cudaStream_t st) {
   const size_t smem = fwd_smem_bytes<T, GATE>(p.stages);
   static unsigned device_mask = 0;
   cudaError_t e =
-      ensure_smem_attr(reinterpret_cast<const void*>(wkv4_fwd_kernel<T, GATE, TMA>), (int)smem, &device_mask);
+      ensure_smem_attr(reinterpret_cast<const void*>(wkv4_fwd_kernel<T, GATE, TMA, LB>), (int)smem, &device_mask);
   if (e != cudaSuccess) return e;
   const long long nblk = (long long)p.ctiles * p.B * p.nseg;
-  wkv4_fwd_kernel<T, GATE, TMA><<<(unsigned)nblk, kW * 32, smem, st>>>(mk, mv, my, mr, p);
+  wkv4_fwd_kernel<T, GATE, TMA, LB><<<(unsigned)nblk, kW * 32, smem, st>>>(mk, mv, my, mr, p);
   return cudaGetLastError();
 }
 
@@ -359,6 +467,12 @@ cudaError_t launch_wkv4_fwd(bool bf16, const CUtensorMap& mk, const CUtensorMap&
                             const Fwd4Params& p, cudaStream_t st) {
   return bf16 ? launch_fwd_t<__nv_bfloat16, false>(mk, mv, my, mk, p, st)
               : launch_fwd_t<float, false>(mk, mv, my, mk, p, st);
+}
+
+cudaError_t launch_wkv4_fwd_lookback(bool bf16, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& my,
+                                     const Fwd4Params& p, cudaStream_t st) {
+  return bf16 ? launch_fwd_tt<__nv_bfloat16, false, true, true>(mk, mv, my, mk, p, st)
+              : launch_fwd_tt<float, false, true, true>(mk, mv, my, mk, p, st);
 }
 
 cudaError_t launch_wkv4_fwd_gated(bool bf16, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& my,

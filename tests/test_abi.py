@@ -55,8 +55,10 @@ def test_checkpoint_and_workspace_queries():
     # 192 channel tiles (8 x 768): AUTO keeps the sequential schedule, which measured faster there;
     # 24 tiles (1 x 768) over 4096 steps: AUTO cuts time into segments, one state per segment
     assert h.rwkv_wkv4_forward_workspace_bytes(8, 1024, 768, rw.ALGO_AUTO) == 0
+    # (22 segments of 192 steps: per segment and lane a summary as three doubles, and a flag per
+    # segment and CTA, for the one-launch form)
     ws = h.rwkv_wkv4_forward_workspace_bytes(1, 4096, 768, rw.ALGO_AUTO)
-    assert ws > 0 and ws % (3 * 1 * 768 * 4) == 0
+    assert ws >= 22 * 768 * 3 * 8 + 22 * 24 * 4 and ws < 22 * 768 * 3 * 8 + 4096
     assert h.rwkv_wkv4_forward_workspace_bytes(8, 1024, 768, rw.ALGO_CHUNKED) > 0
     assert h.rwkv_wkv4_forward_workspace_bytes(0, 10, 10, 0) == 0
 
