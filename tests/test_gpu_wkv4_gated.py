@@ -9,7 +9,8 @@ import torch
 import oracle
 import rwkv_wkv_recurrence_b200 as rw
 import wkv_inputs as wi
-from _parity import TOL_BF16, TOL_Y, assert_close_abs1, assert_close_rms, assert_grads_close
+from _parity import (TOL_BF16, TOL_Y, assert_close_abs1, assert_close_rms, assert_grads_close, assert_state_close,
+                     state_to_ab)
 
 pytestmark = pytest.mark.gpu
 SEED = wi.CONFIG_SEED_BASE
@@ -32,9 +33,15 @@ def test_gated_forward(cuda_device, algo, shape):
     g = _cuda(p, cuda_device)
     o, st = rw.rwkv_wkv4_forward_gated(g["w"], g["u"], g["k"], g["v"], g["r"], algo=algo, return_state=True)
     assert_close_abs1(o, oracle.wkv4_gated_forward(p["w"], p["u"], p["k"], p["v"], p["r"]), TOL_Y, "o")
-    # the gate does not enter the recurrence: state and checkpoints are the plain forward's, bitwise
+    # the gate does not enter the recurrence: the state is the plain forward's, bitwise on the same
+    # schedule.  The chunked schedule of the plain forward runs in one launch (fp64 segment summaries)
+    # where the gated one, with three input boxes per stage, keeps three launches (fp32 summaries):
+    # there the two agree within the state tolerance.
     _, st0 = rw.rwkv_wkv4_forward(g["w"], g["u"], g["k"], g["v"], algo=algo, return_state=True)
-    assert torch.equal(st, st0)
+    if algo == rw.ALGO_SEQUENTIAL:
+        assert torch.equal(st, st0)
+    else:
+        assert_state_close(st, state_to_ab(st0), "state")
 
 
 @pytest.mark.parametrize("shape", [(1, 64, 128), (3, 333, 100), (2, 7, 4), (5, 250, 36)])
