@@ -134,3 +134,62 @@ def test_backward_fast_decay_full_size(cuda_device):
     g = wi.wkv5_grads(B, T, H, N, seed=SEED + 11, states=True)
     out, ref = _run(p, g, cuda_device)
     _check(out, ref)
+
+
+@pytest.mark.parametrize("finch", [False, True])
+@pytest.mark.parametrize("which", ["s_in", "gs_out"])
+def test_backward_one_state_only(cuda_device, finch, which):
+    # an initial state without a final-state gradient, and the reverse (the Eagle backward too)
+    B, T, H = 2, 90, 2
+    p = (wi.wkv6_problem if finch else wi.wkv5_problem)(B, T, H, 64, seed=102)
+    g = wi.wkv5_grads(B, T, H, 64, seed=103, states=True)
+    g.pop("gs_out" if which == "s_in" else "s_in")
+    c = {k: v.to(cuda_device) for k, v in list(p.items()) + list(g.items())}
+    bwd = rw.rwkv_wkv6_backward if finch else rw.rwkv_wkv5_backward
+    out = bwd(c["r"], c["k"], c["v"], c["omega"], c["u"], c["gy"], c.get("s_in"), c.get("gs_out"), want_gs_in=True)
+    rw.rwkv_check_device_error()
+    ref = (oracle.wkv6_backward if finch else oracle.wkv5_backward)(
+        p["r"], p["k"], p["v"], p["omega"], p["u"], g["gy"], s_in=g.get("s_in"), gs_out=g.get("gs_out"))
+    if finch:
+        _check(out, ref, which + " only: ")
+    else:
+        for got, want, name in zip(out, ref, ("gr", "gk", "gv", "gomega", "gu", "gs_in")):
+            assert_close_rms(got.cpu(), want, TOL_BF16, f"{which} only: {name}")
+
+
+@pytest.mark.parametrize("finch", [False, True])
+def test_backward_resumes_across_a_split(cuda_device, finch):
+    # the backward of a sequence is the backward of its two halves chained through the state: the
+    # first half's final state is the second half's s_in, and the second half's gs_in is the first
+    # half's gs_out.  Per-token gradients then agree with the whole-sequence call, and the batch and
+    # time sums (gu; Eagle's gomega) are the sums of the halves'
+    B, T, H, T1 = 2, 200, 2, 77
+    gen = wi.wkv6_problem if finch else wi.wkv5_problem
+    p = {k: v.to(cuda_device) for k, v in gen(B, T, H, 64, seed=104).items()}
+    g = {k: v.to(cuda_device) for k, v in wi.wkv5_grads(B, T, H, 64, seed=105, states=True).items()}
+    fwd = rw.rwkv_wkv6_forward if finch else rw.rwkv_wkv5_forward
+    bwd = rw.rwkv_wkv6_backward if finch else rw.rwkv_wkv5_backward
+
+    def part(x, a, b):  # tokens [a, b) of a [B,T,H,N] tensor (omega too for Finch)
+        return x[:, a:b].contiguous()
+
+    om = (lambda a, b: part(p["omega"], a, b)) if finch else (lambda a, b: p["omega"])
+    whole = bwd(p["r"], p["k"], p["v"], p["omega"], p["u"], g["gy"], g["s_in"], g["gs_out"], want_gs_in=True)
+    _, s_mid = fwd(part(p["r"], 0, T1), part(p["k"], 0, T1), part(p["v"], 0, T1), om(0, T1), p["u"], g["s_in"],
+                   return_state=True)
+    second = bwd(part(p["r"], T1, T), part(p["k"], T1, T), part(p["v"], T1, T), om(T1, T), p["u"],
+                 part(g["gy"], T1, T), s_mid, g["gs_out"], want_gs_in=True)
+    first = bwd(part(p["r"], 0, T1), part(p["k"], 0, T1), part(p["v"], 0, T1), om(0, T1), p["u"],
+                part(g["gy"], 0, T1), g["s_in"], second[5], want_gs_in=True)
+    rw.rwkv_check_device_error()
+    names = ("gr", "gk", "gv")
+    for i, name in enumerate(names):
+        joined = torch.cat([first[i], second[i]], dim=1)
+        assert_close_rms(joined.cpu(), whole[i].cpu().double().numpy(), 2 * TOL_BF16, name)
+    if finch:
+        joined = torch.cat([first[3], second[3]], dim=1)
+        assert_close_rms(joined.cpu(), whole[3].cpu().double().numpy(), 2 * TOL_BF16, "gomega")
+    else:
+        assert_close_rms((first[3] + second[3]).cpu(), whole[3].cpu().double().numpy(), 2 * TOL_BF16, "gomega")
+    assert_close_rms((first[4] + second[4]).cpu(), whole[4].cpu().double().numpy(), 2 * TOL_BF16, "gu")
+    assert_close_rms(first[5].cpu(), whole[5].cpu().double().numpy(), 2 * TOL_BF16, "gs_in")
