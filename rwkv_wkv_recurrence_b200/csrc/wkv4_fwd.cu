@@ -157,8 +157,9 @@ __global__ void __launch_bounds__(kW * 32, 4) wkv4_fwd_kernel(const __grid_const
   constexpr int kNB = GATE ? 3 : 2;  // boxes per stage: k, v (, r)
   T* tiles = reinterpret_cast<T*>(smem_raw);  // [stages][k|v(|r)][kTile][32]
   Summ* summ = reinterpret_cast<Summ*>(smem_raw + (size_t)p.stages * kNB * kBoxBytes);  // [2][kW][32]
-  CarrySlot* cslot = reinterpret_cast<CarrySlot*>(summ + 2 * kW * 32);                // [2][32]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(cslot + 2 * 32);                         // [stages]
+  // [2][32]; LB: [3][32], the third the sequence's start state
+  CarrySlot* cslot = reinterpret_cast<CarrySlot*>(summ + 2 * kW * 32);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(cslot + (LB ? 3 : 2) * 32);  // [stages]
   int* abort_flag = reinterpret_cast<int*>(bars + p.stages);
 
   const int lane = threadIdx.x & 31;
@@ -211,6 +212,14 @@ __global__ void __launch_bounds__(kW * 32, 4) wkv4_fwd_kernel(const __grid_const
       s0 = load_state(sp[lane_off], sp[plane + lane_off], sp[2 * plane + lane_off]);
     }
     cslot[32 + lane] = CarrySlot{s0.a, s0.b, s0.p, 0};  // slot of "tile -1"
+    if constexpr (LB) {
+      // read before this CTA publishes its summary: state_out may be state_in, and the last
+      // segment overwrites it as soon as every summary is out
+      State si{0.0, 0.0, 0};
+      if (p.lb_in != nullptr && valid)
+        si = load_state(p.lb_in[lane_off], p.lb_in[plane + lane_off], p.lb_in[2 * plane + lane_off]);
+      cslot[64 + lane] = CarrySlot{si.a, si.b, si.p, 0};
+    }
   }
   __syncthreads();
 
@@ -353,10 +362,8 @@ __global__ void __launch_bounds__(kW * 32, 4) wkv4_fwd_kernel(const __grid_const
         if (failed) {
           if (lane == 0) *abort_flag = 1;
         } else {
-          State st{0.0, 0.0, 0};
+          State st{cslot[64 + lane].a, cslot[64 + lane].b, cslot[64 + lane].p};
           if (valid) {
-            if (p.lb_in != nullptr)
-              st = load_state(p.lb_in[lane_off], p.lb_in[plane + lane_off], p.lb_in[2 * plane + lane_off]);
             const double lam_seg = lam_len(lam, lam16, p.seg_len);  // every earlier segment is whole
             // the earlier summaries in order, eight at a time, their loads in flight together
             constexpr int kBatch = 8;
@@ -399,8 +406,8 @@ __global__ void __launch_bounds__(kW * 32, 4) wkv4_fwd_kernel(const __grid_const
 //   S_{<=j} = e^{-w len_j} S_{<=j-1}  (+)  summary_j,
 // and writes the final state.  One thread per lane (b, c), fp64 arithmetic.
 __global__ void wkv4_carry_kernel(int B, int C, int T, int nseg, int seg_len, const float* __restrict__ w,
-                                  const float* __restrict__ state_in, float* __restrict__ ws,
-                                  float* __restrict__ state_out) {
+                                  const float* state_in, float* __restrict__ ws,
+                                  float* state_out) {  // state_out may be state_in
   const size_t plane = (size_t)B * C;
   const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= plane) return;
@@ -422,16 +429,16 @@ __global__ void wkv4_carry_kernel(int B, int C, int T, int nseg, int seg_len, co
   if (state_out != nullptr) store_state(st, &state_out[i], &state_out[plane + i], &state_out[2 * plane + i]);
 }
 
-template <typename T, bool GATE>
+template <typename T, bool GATE, bool LB = false>
 size_t fwd_smem_bytes(int stages) {  // also the plain path's (one stage)
   return (size_t)stages * (GATE ? 3 : 2) * kTile * 32 * sizeof(T) + 2 * kW * 32 * sizeof(Summ) +
-         2 * 32 * sizeof(CarrySlot) + (size_t)stages * 8 + 16;
+         (LB ? 3 : 2) * 32 * sizeof(CarrySlot) + (size_t)stages * 8 + 16;
 }
 
 template <typename T, bool GATE, bool TMA, bool LB = false>
 cudaError_t launch_fwd_tt(const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& my, const CUtensorMap& mr,
                           const Fwd4Params& p, cudaStream_t st) {
-  const size_t smem = fwd_smem_bytes<T, GATE>(p.stages);
+  const size_t smem = fwd_smem_bytes<T, GATE, LB>(p.stages);
   static unsigned device_mask = 0;
   cudaError_t e =
       ensure_smem_attr(reinterpret_cast<const void*>(wkv4_fwd_kernel<T, GATE, TMA, LB>), (int)smem, &device_mask);

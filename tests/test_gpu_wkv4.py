@@ -63,6 +63,54 @@ def test_forward_few_channels_long_sequence(cuda_device):
     assert_state_close(st, ref_st)
 
 
+@pytest.mark.parametrize("shape", [(1, 4096, 32), (1, 20001, 40), (2, 9000, 32)])
+@pytest.mark.parametrize("with_state", [False, True])
+def test_forward_many_segments(cuda_device, shape, with_state):
+    # One or two lane tiles over a long sequence: the chunked schedule cuts it into 64 to 157
+    # segments of one or two 64-step tiles (one launch, every tile resident), so a segment waits
+    # for and folds up to 156 earlier summaries, more than the 32 polled at once; the last
+    # segment is partial in the two ragged cases
+    B, T, C = shape
+    p = wi.wkv4_problem(B, T, C, SEED + 2, outliers=True)
+    s_in = None
+    if with_state:
+        _, s_in = oracle.wkv4_forward(p["w"], p["u"], p["k"][:, :300], p["v"][:, :300], return_state=True)
+    g = _cuda(p, cuda_device)
+    st_dev = None
+    if s_in is not None:
+        st_dev = torch.zeros(3, B, C, dtype=torch.float32)
+        st_dev[0], st_dev[1] = torch.from_numpy(s_in[0]).float(), torch.from_numpy(s_in[1]).float()
+        st_dev = st_dev.to(cuda_device)
+    y, st = rw.rwkv_wkv4_forward(g["w"], g["u"], g["k"], g["v"], st_dev, algo=rw.ALGO_CHUNKED, return_state=True)
+    ref, ref_st = oracle.wkv4_forward(p["w"], p["u"], p["k"], p["v"], state_in=s_in, return_state=True)
+    assert_close_abs1(y, ref, TOL_Y, "y")
+    assert_state_close(st, ref_st)
+
+
+@pytest.mark.parametrize("shape", [(1, 20001, 40), (8, 1024, 768)])
+def test_forward_chunked_state_in_place(cuda_device, shape):
+    # state_out is state_in on the chunked schedule: the final state is written while other
+    # segments fold the start state into theirs, so each must have read it first
+    B, T, C = shape
+    p = wi.wkv4_problem(B, T, C, SEED + 3, outliers=True)
+    _, s_ref = oracle.wkv4_forward(p["w"], p["u"], p["k"][:, :100], p["v"][:, :100], return_state=True)
+    st = torch.zeros(3, B, C, dtype=torch.float32)
+    st[0], st[1] = torch.from_numpy(s_ref[0]).float(), torch.from_numpy(s_ref[1]).float()
+    g = _cuda(p, cuda_device)
+    st = st.to(cuda_device)
+    h = rw.lib()
+    wsb = int(h.rwkv_wkv4_forward_workspace_bytes(B, T, C, rw.ALGO_CHUNKED))
+    assert wsb > 0
+    ws = torch.empty(wsb, dtype=torch.uint8, device=cuda_device)
+    y = torch.empty(B, T, C, device=cuda_device)
+    assert h.rwkv_wkv4_forward(B, T, C, rw.F32, rw._ptr(g["w"]), rw._ptr(g["u"]), rw._ptr(g["k"]), rw._ptr(g["v"]),
+                               rw._ptr(y), rw._ptr(st), rw._ptr(st), None, 16, rw.ALGO_CHUNKED, rw._ptr(ws), wsb,
+                               rw._stream(None)) == 0
+    ref, ref_st = oracle.wkv4_forward(p["w"], p["u"], p["k"], p["v"], state_in=s_ref, return_state=True)
+    assert_close_abs1(y, ref, TOL_Y, "y")
+    assert_state_close(st, ref_st)
+
+
 def test_forward_single_large_outlier_slow_decay(cuda_device):
     # One +40 key at t = 1 and w = 0.01: the outlier dominates the state for
     # hundreds of steps, the case where per-step rounding of a running-max
