@@ -190,7 +190,10 @@ RWKV_API rwkv_status rwkv_wkv4_step(int64_t B, int64_t C, rwkv_dtype dtype, cons
                            const void *k, const void *v, void *y, const float *state_in,
                            float *state_out, rwkv_stream_t stream);
 
-/* Workspace bytes rwkv_wkv5_forward needs (0 if none). */
+/* Workspace bytes rwkv_wkv5_forward needs (0 if none): with two or more 64-token chunks per head,
+ * a 64 x 64 fp32 summary and a flag for each of up to 296 CTAs (the heads' chunks are dealt out
+ * evenly to two CTAs per SM; a CTA whose chunks end inside a head publishes the state they reach
+ * from a zero state, and the CTAs holding the rest of that head fold it into their start). */
 RWKV_API size_t rwkv_wkv5_forward_workspace_bytes(int64_t B, int64_t T, int64_t H, int64_t N);
 
 /*
@@ -199,6 +202,10 @@ RWKV_API size_t rwkv_wkv5_forward_workspace_bytes(int64_t B, int64_t T, int64_t 
  *   omega, u  [H,N] fp32 (w = exp(-exp(omega)) is formed inside).
  *   s_in      [B,H,N,N] fp32 or NULL (zero).  s_out [B,H,N,N] fp32 or NULL;
  *             may equal s_in.
+ *   workspace device scratch of rwkv_wkv5_forward_workspace_bytes() bytes, 16-byte aligned
+ *             (RWKV_ERR_WORKSPACE if NULL or smaller, RWKV_ERR_UNSUPPORTED if misaligned;
+ *             may be NULL if the query gives 0).  Calls that share one workspace must be
+ *             ordered (the same stream): it holds flags the kernel waits on.
  *   N must be 64 (RWKV_ERR_UNSUPPORTED otherwise).
  */
 RWKV_API rwkv_status rwkv_wkv5_forward(int64_t B, int64_t T, int64_t H, int64_t N,

@@ -167,6 +167,34 @@ FwdPlan plan_forward(int64_t B, int64_t T, int64_t C, int algo) {
   return pl;
 }
 
+// Eagle forward: a head's chunks form a chain (each reads the state the one before leaves), and
+// one CTA per head leaves the call as long as one head's chain however many SMs are idle, or
+// twice that when a few heads are over two per SM.  The slot plan deals the heads' chunks, laid
+// end to end, out evenly to two CTAs per SM; a CTA whose chunks end inside a head first scans
+// them for a summary (the state they reach from a zero state) that the CTAs holding the rest of
+// that head fold into their start states.
+constexpr int kEagleSlotsPerSM = 2;  // resident CTAs per SM (shared memory)
+
+struct Wkv5Slots {
+  int nslot = 0;
+  size_t sum = 0, flag = 0, flag_bytes = 0, total = 0;  // workspace offsets and bytes
+};
+
+Wkv5Slots plan_wkv5_slots(int64_t B, int64_t T, int64_t H) {
+  Wkv5Slots pl;
+  const int64_t nchunk = (T + 63) / 64, nflat = B * H * nchunk;
+  // one chunk per head: nothing to split; the flat index times the slot count must fit 64 bits
+  if (nchunk < 2 || nflat >= ((int64_t)1 << 40)) return pl;
+  const int64_t nslot = std::min<int64_t>((int64_t)kEagleSlotsPerSM * kDesignSMs, nflat);
+  auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  pl.nslot = (int)nslot;
+  pl.sum = 0;
+  pl.flag = up((size_t)nslot * 64 * 64 * sizeof(float));
+  pl.flag_bytes = ((size_t)nslot + 1) * sizeof(unsigned int);
+  pl.total = pl.flag + up(pl.flag_bytes);
+  return pl;
+}
+
 // Runs the forward pass (outputs optional) on already-validated arguments.  With r, the
 // output pass writes σ(r) ⊙ WKV (the receptance-gated kernel) instead of WKV.
 rwkv_status run_forward(int B, int T, int C, bool bf16, const float* w, const float* u, const void* k,
@@ -472,18 +500,13 @@ rwkv_status rwkv_wkv4_step(int64_t B, int64_t C, rwkv_dtype dtype, const float* 
 }
 
 size_t rwkv_wkv5_forward_workspace_bytes(int64_t B, int64_t T, int64_t H, int64_t N) {
-  (void)B;
-  (void)T;
-  (void)H;
-  (void)N;
-  return 0;
+  if (N != 64 || B <= 0 || T <= 0 || H <= 0 || !fits_int(B) || !fits_int(H) || !fits_int(B * H)) return 0;
+  return plan_wkv5_slots(B, T, H).total;
 }
 
 rwkv_status rwkv_wkv5_forward(int64_t B, int64_t T, int64_t H, int64_t N, const void* r, const void* k,
                               const void* v, const float* omega, const float* u, void* y, const float* s_in,
                               float* s_out, void* workspace, size_t workspace_bytes, rwkv_stream_t stream) {
-  (void)workspace;
-  (void)workspace_bytes;
   if (!fits_int(B) || !fits_int(T) || !fits_int(H) || !fits_int(N)) return RWKV_ERR_INVALID_ARG;
   if (N != 64) return RWKV_ERR_UNSUPPORTED;
   if (B == 0 || H == 0) return RWKV_OK;
@@ -501,6 +524,9 @@ rwkv_status rwkv_wkv5_forward(int64_t B, int64_t T, int64_t H, int64_t N, const 
   if (r == nullptr || k == nullptr || v == nullptr || y == nullptr) return RWKV_ERR_INVALID_ARG;
   if (!aligned16(r) || !aligned16(k) || !aligned16(v) || !aligned16(y)) return RWKV_ERR_UNSUPPORTED;
   if ((int64_t)H * 64 > INT_MAX || (int64_t)B * H > INT_MAX) return RWKV_ERR_UNSUPPORTED;
+  const Wkv5Slots plan = plan_wkv5_slots(B, T, H);
+  if (plan.nslot > 0 && (workspace == nullptr || workspace_bytes < plan.total)) return RWKV_ERR_WORKSPACE;
+  if (plan.nslot > 0 && !aligned16(workspace)) return RWKV_ERR_UNSUPPORTED;
   DevCtl* ctl = device_ctl();
   if (ctl == nullptr) return RWKV_ERR_CUDA;
   const int iB = (int)B, iT = (int)T, iH = (int)H;
@@ -521,6 +547,13 @@ rwkv_status rwkv_wkv5_forward(int64_t B, int64_t T, int64_t H, int64_t N, const 
   p.s_in = s_in;
   p.s_out = s_out;
   p.ctl = ctl;
+  if (plan.nslot > 0) {
+    char* ws = static_cast<char*>(workspace);
+    if (cudaMemsetAsync(ws + plan.flag, 0, plan.flag_bytes, st) != cudaSuccess) return RWKV_ERR_CUDA;
+    p.nslot = plan.nslot;
+    p.slot_sum = reinterpret_cast<float*>(ws + plan.sum);
+    p.slot_flag = reinterpret_cast<unsigned int*>(ws + plan.flag);
+  }
   if (launch_wkv5_fwd(mr, mk, mv, p, st) != cudaSuccess) return RWKV_ERR_CUDA;
   return RWKV_OK;
 }

@@ -84,6 +84,11 @@ struct Wkv5Params {
   const float* s_in;    // [B,H,64,64] or null
   float* s_out;         // [B,H,64,64] or null
   DevCtl* ctl;
+  // Slot plan (forward only; nslot = 0: one CTA per head).  The heads' 64-token chunks, laid end
+  // to end, are dealt out evenly to nslot CTAs in the order they start.
+  int nslot;
+  float* slot_sum;          // [nslot][64][64]: a slot's last segment from a zero state
+  unsigned int* slot_flag;  // [nslot] flags, then the ticket counter; zeroed before the launch
 };
 
 struct Wkv6Params {

@@ -75,7 +75,9 @@ constexpr uint32_t kRawBytes = kL * kN * 2;    // one bf16 [64 x 64] box
 constexpr float kMaxRate = 2.f;        // largest -λ the chunked factorization takes
 constexpr int kBand = 15;              // lags a fast channel keeps in the scores: e^{-2 (kBand+1)} < 2^-46
 static_assert(kBand == 15, "the band pass gives each thread 4 of the 16 lags of one position");
-constexpr uint32_t kTmemCols = 256;  // [scores | output rows], state increment, k̃ᵀ (64 columns each)
+constexpr uint32_t kTmemCols = 256;
+constexpr unsigned int kSlotReady = 1u;   // a slot's summary is published
+constexpr unsigned int kSlotGaveUp = 2u;  // a slot's wait gave up: it publishes no summary  // [scores | output rows], state increment, k̃ᵀ (64 columns each)
 
 struct Wkv5Smem {
   alignas(1024) __nv_bfloat16 raw[3][kL * kN];  // r, k, v boxes [token][channel] (128-byte swizzle)
@@ -102,15 +104,19 @@ struct Wkv5Smem {
   alignas(8) uint64_t bar_sc;        // scores and state read done
   alignas(8) uint64_t bar_av;        // A v done
   alignas(8) uint64_t bar_ds;        // state increment done
+  alignas(8) uint64_t bar_scan[3];   // a summary scan's k, v boxes, three stages
   uint32_t tmem_base;
   int nfast;
   int abort_flag;
+  int ticket;                        // the CTA's slot (slot plan)
 };
 // dynamic shared memory = the struct + 1024 bytes of alignment slack; an SM has 228 KB, of which
 // each resident CTA also takes 1 KB: two CTAs per SM
 static_assert(2 * (sizeof(Wkv5Smem) + 1024 + 1024) <= 228 * 1024, "two CTAs per SM");
 static_assert(offsetof(Wkv5Smem, opS) == offsetof(Wkv5Smem, opK) + 64 * 64 * sizeof(float),
               "the first product reads k̃ and e^{32λ} Sᵀ as one 128-row operand");
+static_assert(offsetof(Wkv5Smem, opR) % 1024 == 0 && offsetof(Wkv5Smem, opK) % 1024 == 0 && kRawBytes % 1024 == 0,
+              "a summary scan loads 128-byte-swizzled boxes into the r̃ and k̃ tiles");
 
 // REV: the operator over reversed time (position τ of chunk c is token T-1-(64c+τ)), reading and
 // writing the tensors in their own order: chunk c's box starts at token T-64(c+1) (rows before
@@ -127,48 +133,41 @@ __global__ void __launch_bounds__(kThreads, 2) wkv5_fwd_tc_kernel(const __grid_c
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int t4 = lane >> 2, tq = lane & 3;
   const int q4 = warp & 3, hc = warp >> 2;  // TMEM lane quarter and column half of this warp
-  const int b = blockIdx.x / p.H, h = blockIdx.x % p.H;
   const int nchunk = (p.T + kL - 1) / kL;
-  const float* om = p.omega + h * kN;
+  // ---- the CTA's work.  Reversed, or without a slot plan: one whole head (blockIdx).  With a
+  // plan, the heads' chunks laid end to end (head-major, N = B H nchunk of them) are dealt out
+  // evenly: slot s takes [F(s), F(s+1)), F(s) = floor(s N / nslot), the tail of one head, whole
+  // heads and the start of another.  s is a ticket drawn in the order the CTAs start, so a CTA
+  // only ever waits for slots that are already running.
+  const bool slots = !REV && p.nslot > 0;
+  const long long nflat = (long long)p.B * p.H * nchunk;
+  auto slot_first = [&](long long s) { return s * nflat / p.nslot; };  // F(s)
+  int slot = 0;
+  long long f0 = (long long)blockIdx.x * nchunk, f1 = f0 + nchunk;
+  if (slots) {
+    if (tid == 0) sm.ticket = (int)atomicAdd(&p.slot_flag[p.nslot], 1u);
+    __syncthreads();
+    slot = sm.ticket;
+    f0 = slot_first(slot);
+    f1 = slot_first(slot + 1);
+  }
+  const int bh_first = (int)(f0 / nchunk);
+  const int nseg = (int)((f1 - 1) / nchunk) - bh_first + 1;
+  // segment k of the CTA: head bh_first + k, its chunks [cb, ce)
+  auto seg_range = [&](int k, int& cb, int& ce) {
+    const long long base = (long long)(bh_first + k) * nchunk;
+    cb = (int)(max(f0, base) - base);
+    ce = (int)(min(f1, base + nchunk) - base);
+  };
+  // when the last segment ends before its head does, the CTA first scans it for the summary that
+  // the slots after it fold into their start states
+  int last_cb, last_ce;
+  seg_range(nseg - 1, last_cb, last_ce);
+  const bool summary = slots && last_ce < nchunk;
 
-  // ---- fast channels (-λ > 2): outside the factorization's range.  They enter the tensor-core
-  // products only where the factor stays at most 1 (state read e^{λτ}, state increment
-  // e^{λ(cnt-1-ι)}); their intra-chunk scores are summed on the CUDA cores over lags 0..kBand.
   if (tid == 0) sm.abort_flag = 0;
-  for (int i = tid; i < (kL + 1) * (kN / 2 + 1); i += kThreads) {
-    if (i < kL * (kN / 2 + 1)) (&sm.RFw[0][0])[i] = 0u;
-    (&sm.KFw[0][0])[i] = 0u;
-  }
-  if (tid < kN) {  // the weights of an odd count's padding channel must read as zero too
-#pragma unroll
-    for (int g = 0; g < 4; ++g) sm.E4[tid][g] = 0.f;
-    sm.E1[tid] = 0.f;
-  }
-  if (tid < kN) {
-    const bool f = !(expf(om[tid]) <= kMaxRate);
-    const unsigned m = __ballot_sync(0xffffffffu, f);
-    if (lane == 0) sm.fmask[warp] = m;
-  }
-  __syncthreads();
-  if (tid < kN) {
-    const unsigned m0 = sm.fmask[0], m1 = sm.fmask[1];
-    const bool f = ((tid < 32 ? m0 : m1) >> (tid & 31)) & 1u;
-    const int below = tid < 32 ? __popc(m0 & ((1u << tid) - 1u)) : __popc(m0) + __popc(m1 & ((1u << (tid & 31)) - 1u));
-    sm.fidx[tid] = f ? below : -1;
-    if (f) {
-      sm.flist[below] = tid;
-      const float lam = -expf(om[tid]);
-#pragma unroll
-      for (int g = 0; g < 4; ++g) sm.E4[below][g] = g == 0 ? 1.f : expf(lam * (float)(4 * g));
-      sm.E1[below] = expf(lam);
-    }
-    if (tid == 0) sm.nfast = __popc(m0) + __popc(m1);
-  }
-  __syncthreads();
-  const int nfast = sm.nfast;
-
   if (warp == 0) tmem_alloc(&sm.tmem_base, kTmemCols);
-  // thread 0 issues every load; with the test hook set it arms the barrier and issues none
+  // thread 0 issues every load; with the test hook set it arms the barriers and issues none
   const bool withheld = tid == 0 && loads_withheld(p.ctl);
   if (tid == 0) {
     prefetch_tensormap(&mr);
@@ -178,33 +177,14 @@ __global__ void __launch_bounds__(kThreads, 2) wkv5_fwd_tc_kernel(const __grid_c
     mbar_init(&sm.bar_sc, 1);
     mbar_init(&sm.bar_av, 1);
     mbar_init(&sm.bar_ds, 1);
+    for (int st = 0; st < 3; ++st) mbar_init(&sm.bar_scan[st], 1);
     fence_mbar_init();
-    mbar_arrive_expect_tx(&sm.bar_tma, 3 * kRawBytes);
-    if (!withheld) {
-      const int row0 = REV ? p.T - kL : 0;
-      tma_load_3d(sm.raw[0], &mr, &sm.bar_tma, h * kN, row0, b);
-      tma_load_3d(sm.raw[1], &mk, &sm.bar_tma, h * kN, row0, b);
-      tma_load_3d(sm.raw[2], &mv, &sm.bar_tma, h * kN, row0, b);
-    }
   }
 
   // ---- r̃, k̃: warp w owns channels 8w..8w+7; lane holds token row 8 ib + rr, channels dR, dR + 1.
   // A half-warp then writes one whole core matrix (eight 16-byte rows): no bank conflicts.
   const int rr = lane & 7, rp = lane >> 3;
   const int dR = 8 * warp + 2 * rp;
-  // a fast channel: r e^{λτ} (read only; its k̃ is zero, so it adds nothing to the scores)
-  float fr0[2], frs[2], fk0[2], fks[2], uA[2];
-  int fiA[2];
-#pragma unroll
-  for (int e = 0; e < 2; ++e) {
-    const float rate = expf(om[dR + e]);  // -λ
-    fiA[e] = sm.fidx[dR + e];
-    fr0[e] = fiA[e] >= 0 ? (rr == 0 ? 1.f : expf(-rate * (float)rr)) : expf(-rate * (float)(rr - 32));
-    frs[e] = expf(-8.f * rate);
-    fk0[e] = fiA[e] >= 0 ? 0.f : expf(-rate * (float)(31 - rr));
-    fks[e] = fiA[e] >= 0 ? 0.f : expf(8.f * rate);
-    uA[e] = p.u[h * kN + dR + e];
-  }
   // box row of position 8 ib + rr: 8 ib + rr, or 63 - (8 ib + rr) = 8 (7 - ib) + (7 - rr) reversed
   const int rb = REV ? 7 - rr : rr;
   const uint32_t offRK = (uint32_t)rb * 128u + (uint32_t)((warp ^ rb) << 4) + (uint32_t)rp * 4u;
@@ -218,43 +198,97 @@ __global__ void __launch_bounds__(kThreads, 2) wkv5_fwd_tc_kernel(const __grid_c
                             : (uint32_t)(lmat * 8 + lrow) * 128u + (uint32_t)((warp ^ lrow) << 4);
   // ---- k̃ᵀ (tensor memory, A of the state increment), .16x256b fragment of warp w:
   // rows d = 16 q4 + t4 + 8 r, columns ι = 32 hc + 8 i + 2 tq + e  ->  register 4 i + 2 r + e
-  // (a fast row's factor is e^{λ(cnt-1-ι)}, formed per chunk)
-  float fc0[2][2], fcs[2], lamT[2];
-  bool fastT[2];
-#pragma unroll
-  for (int r = 0; r < 2; ++r) {
-    const float rate = expf(om[16 * q4 + 8 * r + t4]);
-    lamT[r] = -rate;
-    fastT[r] = sm.fidx[16 * q4 + 8 * r + t4] >= 0;
-#pragma unroll
-    for (int e = 0; e < 2; ++e) fc0[r][e] = fastT[r] ? 0.f : expf(-rate * (float)(31 - 32 * hc - 2 * tq - e));
-    fcs[r] = fastT[r] ? 0.f : expf(8.f * rate);
-  }
   // position 32 hc + 8 (lmat >> 1) + lrow (+ 16 per pp); its box row bottom up when REV
   const uint32_t offKt =
       REV ? (uint32_t)(63 - (4 * hc + (lmat >> 1)) * 8 - lrow) * 128u + (uint32_t)(((2 * q4 + (lmat & 1)) ^ (7 - lrow)) << 4)
           : (uint32_t)((4 * hc + (lmat >> 1)) * 8 + lrow) * 128u + (uint32_t)(((2 * q4 + (lmat & 1)) ^ lrow) << 4);
-
   // ---- state S[d][j] (fp32 master copy) in the .16x128b fragment of warp w:
   // d = 16 q4 + t4 + 8 r, j = 32 hc + 4 q + tq  ->  S[2 q + r]
   const int drow = 16 * q4 + t4;
   const int jcol = 32 * hc + tq;
   const uint32_t tquar = (uint32_t)(32 * q4) << 16;
-  float e32[2];
+
+  // ---- per head: its fast channels and every thread's decay factors
+  int b = 0, h = 0, nfast = 0;
+  const float* om = p.omega;
+  // r̃, k̃ build: a fast channel's r e^{λτ} (read only; its k̃ is zero, so it adds nothing to the scores)
+  float fr0[2], frs[2], fk0[2], fks[2], uA[2];
+  int fiA[2];
+  // k̃ᵀ rows (a fast row's factor is e^{λ(cnt-1-ι)}, formed per chunk)
+  float fc0[2][2], fcs[2], lamT[2];
+  bool fastT[2];
+  float e32[2];  // e^{32λ} of the state rows
+  auto setup_head = [&](int bh) {
+    // the previous segment's reads of the tables, of tensor memory and of opS are done
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    b = bh / p.H;
+    h = bh % p.H;
+    om = p.omega + h * kN;
+    // fast channels (-λ > 2): outside the factorization's range.  They enter the tensor-core
+    // products only where the factor stays at most 1 (state read e^{λτ}, state increment
+    // e^{λ(cnt-1-ι)}); their intra-chunk scores are summed on the CUDA cores over lags 0..kBand.
+    for (int i = tid; i < (kL + 1) * (kN / 2 + 1); i += kThreads) {
+      if (i < kL * (kN / 2 + 1)) (&sm.RFw[0][0])[i] = 0u;
+      (&sm.KFw[0][0])[i] = 0u;
+    }
+    if (tid < kN) {  // the weights of an odd count's padding channel must read as zero too
 #pragma unroll
-  for (int r = 0; r < 2; ++r) e32[r] = expf(-32.f * expf(om[drow + 8 * r]));
-  const size_t sbase = ((size_t)b * p.H + h) * kN * kN;
+      for (int g = 0; g < 4; ++g) sm.E4[tid][g] = 0.f;
+      sm.E1[tid] = 0.f;
+    }
+    if (tid < kN) {
+      const bool f = !(expf(om[tid]) <= kMaxRate);
+      const unsigned m = __ballot_sync(0xffffffffu, f);
+      if (lane == 0) sm.fmask[warp] = m;
+    }
+    __syncthreads();
+    if (tid < kN) {
+      const unsigned m0 = sm.fmask[0], m1 = sm.fmask[1];
+      const bool f = ((tid < 32 ? m0 : m1) >> (tid & 31)) & 1u;
+      const int below = tid < 32 ? __popc(m0 & ((1u << tid) - 1u)) : __popc(m0) + __popc(m1 & ((1u << (tid & 31)) - 1u));
+      sm.fidx[tid] = f ? below : -1;
+      if (f) {
+        sm.flist[below] = tid;
+        const float lam = -expf(om[tid]);
+#pragma unroll
+        for (int g = 0; g < 4; ++g) sm.E4[below][g] = g == 0 ? 1.f : expf(lam * (float)(4 * g));
+        sm.E1[below] = expf(lam);
+      }
+      if (tid == 0) sm.nfast = __popc(m0) + __popc(m1);
+    }
+    __syncthreads();
+    nfast = sm.nfast;
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const float rate = expf(om[dR + e]);  // -λ
+      fiA[e] = sm.fidx[dR + e];
+      fr0[e] = fiA[e] >= 0 ? (rr == 0 ? 1.f : expf(-rate * (float)rr)) : expf(-rate * (float)(rr - 32));
+      frs[e] = expf(-8.f * rate);
+      fk0[e] = fiA[e] >= 0 ? 0.f : expf(-rate * (float)(31 - rr));
+      fks[e] = fiA[e] >= 0 ? 0.f : expf(8.f * rate);
+      uA[e] = p.u[h * kN + dR + e];
+    }
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const float rate = expf(om[16 * q4 + 8 * r + t4]);
+      lamT[r] = -rate;
+      fastT[r] = sm.fidx[16 * q4 + 8 * r + t4] >= 0;
+#pragma unroll
+      for (int e = 0; e < 2; ++e) fc0[r][e] = fastT[r] ? 0.f : expf(-rate * (float)(31 - 32 * hc - 2 * tq - e));
+      fcs[r] = fastT[r] ? 0.f : expf(8.f * rate);
+      e32[r] = expf(-32.f * expf(om[drow + 8 * r]));
+    }
+  };
   float S[16];
+  auto load_s_in = [&]() {
+    const size_t sb = ((size_t)b * p.H + h) * kN * kN;
 #pragma unroll
-  for (int q = 0; q < 8; ++q)
+    for (int q = 0; q < 8; ++q)
 #pragma unroll
-    for (int r = 0; r < 2; ++r)
-      S[2 * q + r] = p.s_in ? p.s_in[sbase + (size_t)(drow + 8 * r) * kN + jcol + 4 * q] : 0.f;
-#pragma unroll
-  for (int q = 0; q < 8; ++q)
-#pragma unroll
-    for (int r = 0; r < 2; ++r)
-      sm.opS[op_off(jcol + 4 * q, drow + 8 * r)] = (fastT[r] ? 1.f : e32[r]) * S[2 * q + r];
+      for (int r = 0; r < 2; ++r) S[2 * q + r] = p.s_in ? p.s_in[sb + (size_t)(drow + 8 * r) * kN + jcol + 4 * q] : 0.f;
+  };
 
   tc_fence_before();
   __syncthreads();
@@ -266,322 +300,510 @@ __global__ void __launch_bounds__(kThreads, 2) wkv5_fwd_tc_kernel(const __grid_c
   const bool ds_issuer = tid == 128;  // warp 4 (q4 = 0, hc = 1): its scores quarter lies above the diagonal
   static_assert(kThreads > 128, "the state-increment chain's issuing thread");
 
-  int c = 0;
-  bool aborted = false;
-  for (; c < nchunk; ++c) {
-    const int t0 = c * kL;
-    const int cnt = min(kL, p.T - t0);
-    const uint32_t ph = (uint32_t)c & 1u;
-    if (!mbar_wait_bounded(&sm.bar_tma, ph, p.ctl)) sm.abort_flag = 1;
-
-    // T1a: r̃, k̃ and the bonus parts (rows past the sequence end hold zeros from the TMA fill).
-    // r̃ and k̃ are rounded to nearest tf32: the tensor core would truncate both, and the two
-    // biases toward zero add in every score.
-    {
-      float fr[2] = {fr0[0], fr0[1]}, fk[2] = {fk0[0], fk0[1]};
+  // k̃ᵀ fragment from the k box at kbox, step pp of two: a slow row's k e^{λ(31-ι)} (a fast row's
+  // factor is zero here)
+  auto kt_slow = [&](int pp, uint32_t(&kt)[16], uint32_t kbox) {
+    uint32_t qk[4];
+    ldsm_x4_t(REV ? kbox + offKt - pp * 2048u : kbox + offKt + pp * 2048u, qk);
 #pragma unroll
-      for (int ib = 0; ib < 8; ++ib) {
-        const uint32_t ibo = (uint32_t)(REV ? 7 - ib : ib) * 1024u;
-        const float2 rv = bf2_to_f2(lds_u32(rawR + offRK + ibo));
-        const float2 kv = bf2_to_f2(lds_u32(rawK + offRK + ibo));
-        const int row = 8 * ib + rr;
-        *reinterpret_cast<float2*>(&sm.opR[op_off(row, dR)]) = make_float2(to_tf32(rv.x * fr[0]), to_tf32(rv.y * fr[1]));
-        *reinterpret_cast<float2*>(&sm.opK[op_off(row, dR)]) = make_float2(to_tf32(kv.x * fk[0]), to_tf32(kv.y * fk[1]));
-        float part = fmaf(rv.x * uA[0], kv.x, rv.y * uA[1] * kv.y);
-        part += __shfl_xor_sync(0xffffffffu, part, 8);
-        part += __shfl_xor_sync(0xffffffffu, part, 16);
-        if (rp == 0) sm.u.diag_part[warp][row] = part;
+    for (int m = 0; m < 4; ++m) {
+      const int i = 2 * pp + (m >> 1), r = m & 1;
+      const float2 f = bf2_to_f2(qk[m]);
+      const float g = i == 0 ? 1.f : (i == 1 ? fcs[r] : (i == 2 ? fcs[r] * fcs[r] : fcs[r] * fcs[r] * fcs[r]));
+      kt[4 * i + 2 * r] = __float_as_uint(f.x * fc0[r][0] * g);
+      kt[4 * i + 2 * r + 1] = __float_as_uint(f.y * fc0[r][1] * g);
+    }
+  };
+  // a fast row of k̃ᵀ: k e^{λ(cnt-1-ι)}, zero past the chunk's tokens
+  auto kt_fast = [&](int cnt, uint32_t(&kt)[16], uint32_t kbox) {
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          fr[e] *= frs[e];
-          fk[e] *= fks[e];
+    for (int pp = 0; pp < 2; ++pp) {
+      uint32_t qk[4];
+      ldsm_x4_t(REV ? kbox + offKt - pp * 2048u : kbox + offKt + pp * 2048u, qk);
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const int i = 2 * pp + (m >> 1), r = m & 1;
+        if (fastT[r]) {
+          const float2 f = bf2_to_f2(qk[m]);
+          const int io = 32 * hc + 8 * i + 2 * tq;
+          // e^{λ n}, n = cnt-1-ι: the tabled powers up to n = 15, zero beyond (below 2^-46)
+          const int cf = sm.fidx[16 * q4 + 8 * r + t4];
+          auto pw = [&](int n) {
+            if (n < 0 || n > kBand) return 0.f;
+            float x = sm.E4[cf][n >> 2];
+            for (int t = 0; t < (n & 3); ++t) x *= sm.E1[cf];
+            return x;
+          };
+          const float c0 = pw(cnt - 1 - io), c1 = pw(cnt - 2 - io);
+          kt[4 * i + 2 * r] = __float_as_uint(f.x * c0);
+          kt[4 * i + 2 * r + 1] = __float_as_uint(f.y * c1);
         }
       }
     }
-    if (nfast > 0) {  // the fast channels' r and k into the compact rows (bf16 as loaded)
+  };
+  // vᵀ from the v box at vbox into opVt, step pp of two
+  auto vt_step = [&](int pp, uint32_t vbox) {
+    uint32_t qv[4];
+    ldsm_x4_t(REV ? vbox + offT - pp * 4096u : vbox + offT + pp * 4096u, qv);
 #pragma unroll
-      for (int ib = 0; ib < 8; ++ib) {
-        const uint32_t ibo = (uint32_t)(REV ? 7 - ib : ib) * 1024u;
-        const uint32_t rw = lds_u32(rawR + offRK + ibo), kw = lds_u32(rawK + offRK + ibo);
-        const int row = 8 * ib + rr;
-#pragma unroll
-        for (int e = 0; e < 2; ++e)
-          if (fiA[e] >= 0) {
-            const int col = fiA[e] >> 1;
-            unsigned short* rh = reinterpret_cast<unsigned short*>(&sm.RFw[row][col]) + (fiA[e] & 1);
-            unsigned short* kh = reinterpret_cast<unsigned short*>(&sm.KFw[row][col]) + (fiA[e] & 1);
-            *rh = (unsigned short)(e ? rw >> 16 : rw & 0xFFFFu);
-            *kh = (unsigned short)(e ? kw >> 16 : kw & 0xFFFFu);
-          }
-      }
+    for (int m = 0; m < 4; ++m) {
+      const int ib = 4 * pp + m;
+      const uint32_t xv = __shfl_xor_sync(0xffffffffu, qv[m], 18);
+      *reinterpret_cast<float2*>(&sm.opVt[op_off(8 * warp + srow, 8 * ib + 2 * stq)]) = bf2_to_f2(sw ? xv : qv[m]);
     }
-    fence_proxy_async();
-    tc_fence_before();
-    __syncthreads();
-    if (sm.abort_flag) {
-      aborted = true;
-      break;
-    }
-    // [scores | Y] = r̃ [k̃ ; e^{32λ} Sᵀ]ᵀ: causal scores [τ][ι] and the state read [τ][j].  The
-    // issuing thread hands the eight K steps out in pairs between its warp's T1b steps, so that
-    // the warp never waits on a full MMA queue.
-    auto issue_first = [&](int s0) {
-      if (issuer) {
-        if (s0 == 0) tc_fence_after();
-#pragma unroll
-        for (int s = s0; s < s0 + 2; ++s)
-          umma_tf32(tSc, smem_desc(&sm.opR[s * 64], kLbo, kSbo), smem_desc(&sm.opK[s * 64], kLbo, kSbo),
-                    kIdesc128, s);
-        if (s0 == 6) umma_commit(&sm.bar_sc);
+  };
+
+  // counts the abort path needs: output-pass chunks begun, chains committed, load batches armed
+  int m_it = 0, n_ds = 0, n_av = 0, tma_armed = 0;
+  int scan_loaded = 0;  // chunks of the summary scan whose loads were issued (chunk i in stage i % 3)
+  bool aborted = false;
+
+  if (summary) {
+    // ---- the summary of the last segment: the state its chunks reach from a zero state,
+    // Σ_t e^{λ(E-1-t)} k_tᵀ v_t up to its end E, accumulated in tensor memory chunk after chunk
+    // (no fold).  Its k, v boxes arrive three chunks ahead in the raw k, v boxes and in the r̃, k̃
+    // operand tiles, which the scan does not use; k̃ᵀ alternates between two tensor-memory tiles.
+    setup_head(bh_first + nseg - 1);
+    load_s_in();  // kept through the scan: s_out may be s_in, so it is read before the summary goes out
+    const int n = last_ce - last_cb;  // whole chunks: the segment ends before its head does
+    // stage st: its k box, its v box 8 KB after it (the raw boxes are adjacent too)
+    auto stage_k = [&](int st) {
+      return st == 0 ? reinterpret_cast<unsigned char*>(sm.raw[1])
+                     : reinterpret_cast<unsigned char*>(st == 1 ? sm.opR : sm.opK);
+    };
+    static_assert(offsetof(Wkv5Smem, raw) + 3 * kRawBytes == offsetof(Wkv5Smem, opR), "raw boxes, then opR");
+    auto scan_load = [&](int i) {  // chunk i of the segment into stage i % 3 (thread 0)
+      const int st = i % 3, row = (last_cb + i) * kL;
+      fence_proxy_async();
+      mbar_arrive_expect_tx(&sm.bar_scan[st], 2 * kRawBytes);
+      if (!withheld) {
+        tma_load_3d(stage_k(st), &mk, &sm.bar_scan[st], h * kN, row, b);
+        tma_load_3d(stage_k(st) + kRawBytes, &mv, &sm.bar_scan[st], h * kN, row, b);
       }
     };
-    issue_first(0);
+    for (; scan_loaded < min(3, n); ++scan_loaded)
+      if (issuer) scan_load(scan_loaded);
+    for (int i = 0; i < n; ++i) {
+      const int st = i % 3;
+      if (!mbar_wait_bounded(&sm.bar_scan[st], (uint32_t)(i / 3) & 1u, p.ctl)) sm.abort_flag = 1;
+      {
+        uint32_t kt[16];
+        const uint32_t kbox = smem_u32(stage_k(st));
+        kt_slow(0, kt, kbox);
+        kt_slow(1, kt, kbox);
+        // a slow row's k e^{λ(31-ι)} times e^{λ(32 + 64 (n-1-i))}: the weight e^{λ(E-1-t)}
+        const float rest = (float)(32 + kL * (n - 1 - i));
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          const float sc = expf(lamT[r] * rest);
+#pragma unroll
+          for (int x = 0; x < 4; ++x)
+#pragma unroll
+            for (int e = 0; e < 2; ++e)
+              kt[4 * x + 2 * r + e] = __float_as_uint(__uint_as_float(kt[4 * x + 2 * r + e]) * sc);
+        }
+        // a fast row keeps the last 16 positions only (beyond, its weight is below 2^-46)
+        if (nfast > 0 && i == n - 1) kt_fast(kL, kt, kbox);
+        tmem_st16(((i & 1) ? tSc : tKt) + tquar + (uint32_t)(32 * hc), kt);
+      }
+      // the previous chunk's products have read vᵀ (and the k̃ᵀ tile this chunk overwrites)
+      if (i > 0 && !mbar_wait_bounded(&sm.bar_ds, (uint32_t)(n_ds - 1) & 1u, p.ctl)) sm.abort_flag = 1;
+      vt_step(0, smem_u32(stage_k(st)) + kRawBytes);
+      vt_step(1, smem_u32(stage_k(st)) + kRawBytes);
+      fence_proxy_async();
+      tc_fence_before();
+      __syncthreads();
+      if (sm.abort_flag) {
+        aborted = true;
+        break;
+      }
+      if (ds_issuer) {
+        tc_fence_after();
+#pragma unroll
+        for (int s = 0; s < 8; ++s)
+          umma_tf32_ts(tDS, ((i & 1) ? tSc : tKt) + 8 * s, smem_desc(&sm.opVt[s * 64], kLbo, kSbo), kIdesc,
+                       (i > 0 || s > 0) ? 1u : 0u);
+        umma_commit(&sm.bar_ds);
+      }
+      ++n_ds;
+      if (scan_loaded < n) {  // stage st is consumed: chunk i + 3 into it
+        if (issuer) scan_load(scan_loaded);
+        ++scan_loaded;
+      }
+    }
+    if (!aborted) {
+      if (!mbar_wait_bounded(&sm.bar_ds, (uint32_t)(n_ds - 1) & 1u, p.ctl)) sm.abort_flag = 1;
+      tc_fence_after();
+      float sum[16];
+      tmem_ld16x128(tDS + tquar + (uint32_t)(32 * hc), sum);
+      tc_fence_before();
+      __syncthreads();
+      aborted = sm.abort_flag != 0;
+      if (!aborted) {
+        float* dst = p.slot_sum + (size_t)slot * kN * kN;
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+#pragma unroll
+          for (int r = 0; r < 2; ++r) dst[(size_t)(drow + 8 * r) * kN + jcol + 4 * q] = sum[2 * q + r];
+      }
+    }
+    // publish it, or that this slot gave up (the slots waiting for it then stop at once)
+    __syncthreads();
+    if (tid == 0) {
+      __threadfence();
+      flag_release(&p.slot_flag[slot], aborted ? kSlotGaveUp : kSlotReady);
+    }
+  }
 
-    // T1b: k̃ᵀ into tensor memory, vᵀ into shared memory, the bonus sums
-    {
-      if (tid < kL) {
-        float sum = 0.f;
-#pragma unroll
-        for (int w = 0; w < 8; ++w) sum += sm.u.diag_part[w][tid];
-        sm.diag[tid] = sum;
-      }
-      uint32_t kt[16];
-#pragma unroll
-      for (int pp = 0; pp < 2; ++pp) {
-        uint32_t qk[4];
-        ldsm_x4_t(REV ? rawK + offKt - pp * 2048u : rawK + offKt + pp * 2048u, qk);
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {
-          const int i = 2 * pp + (m >> 1), r = m & 1;
-          const float2 f = bf2_to_f2(qk[m]);
-          const float g = i == 0 ? 1.f : (i == 1 ? fcs[r] : (i == 2 ? fcs[r] * fcs[r] : fcs[r] * fcs[r] * fcs[r]));
-          kt[4 * i + 2 * r] = __float_as_uint(f.x * fc0[r][0] * g);
-          kt[4 * i + 2 * r + 1] = __float_as_uint(f.y * fc0[r][1] * g);
+  // ---- the outputs, segment by segment: the scanned one first (its s_in is already in S), then
+  // the others in order
+  for (int j = 0; j < nseg && !aborted; ++j) {
+    const int k = summary ? (j == 0 ? nseg - 1 : j - 1) : j;
+    int cb, ce;
+    seg_range(k, cb, ce);
+    const int bh = bh_first + k;
+    if (summary && j == 0) {
+      tc_fence_before();
+      __syncthreads();
+      tc_fence_after();
+    } else {
+      setup_head(bh);
+      load_s_in();
+    }
+    if (cb > 0) {
+      // the start state: s_in carried over the head's earlier chunks, which the slots before this
+      // one have summarized.  Wait (bounded) for their flags, warp 0's lanes polling 32 at once.
+      const long long hb = (long long)bh * nchunk;
+      const int s_lo = (int)(((hb + 1) * p.nslot + nflat - 1) / nflat) - 1;  // the slot of chunk hb
+      if (warp == 0) {
+        bool ok = true;
+        for (int s0 = s_lo; s0 < slot && ok; s0 += 32) {
+          unsigned int fl = kSlotReady;
+          if (s0 + lane < slot) fl = flag_wait_bounded(&p.slot_flag[s0 + lane], p.ctl);
+          ok = __all_sync(0xffffffffu, fl == kSlotReady);
         }
-        issue_first(2 + 2 * pp);
+        if (!ok && lane == 0) sm.abort_flag = 1;
       }
-      if (nfast > 0) {
-        // the fast channels' scores at lags n = 0..kBand, Σ_c r_τ[c] k_{τ-1-n}[c] e^{λ_c n}: thread
-        // (τ, 4 lags), every CTA thread busy; AF overlays the bonus parts, summed above
-        __syncthreads();
-        const int tau = tid >> 2, g4 = tid & 3, n0 = 4 * g4;
-        // k rows of the four lags (a lag reaching before the chunk reads the zero row)
-        const uint32_t* kp[4];
+      __syncthreads();
+      if (sm.abort_flag) {
+        aborted = true;
+        break;
+      }
+      for (int s2 = s_lo; s2 < slot; ++s2) {
+        const long long a0 = max(slot_first(s2), hb), a1 = slot_first(s2 + 1);
+        const float len = (float)((a1 - a0) * kL);
+        const float* src = p.slot_sum + (size_t)s2 * kN * kN;
+        float x[16];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int io = tau - 1 - (n0 + e);
-          kp[e] = &sm.KFw[io < 0 ? kL : io][0];
+        for (int q = 0; q < 8; ++q)
+#pragma unroll
+          for (int r = 0; r < 2; ++r) x[2 * q + r] = __ldcg(&src[(size_t)(drow + 8 * r) * kN + jcol + 4 * q]);
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          const float d = expf(lamT[r] * len);
+#pragma unroll
+          for (int q = 0; q < 8; ++q) S[2 * q + r] = fmaf(d, S[2 * q + r], x[2 * q + r]);
         }
-        const uint32_t* rp = &sm.RFw[tau][0];
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
-        const int npair = (nfast + 1) >> 1;
-#pragma unroll 2
-        for (int w = 0; w < npair; ++w) {
-          const float2 rv = bf2_to_f2(rp[w]);
-          float ew[2][4];
+      }
+    }
+    // e^{32λ} Sᵀ into opS for the first state read (a fast row's unscaled)
 #pragma unroll
-          for (int h2 = 0; h2 < 2; ++h2) {
-            const int cfi = 2 * w + h2;
-            const float e1 = sm.E1[cfi];
-            ew[h2][0] = sm.E4[cfi][g4];
-            ew[h2][1] = ew[h2][0] * e1;
-            ew[h2][2] = ew[h2][1] * e1;
-            ew[h2][3] = ew[h2][2] * e1;
+    for (int q = 0; q < 8; ++q)
+#pragma unroll
+      for (int r = 0; r < 2; ++r) sm.opS[op_off(jcol + 4 * q, drow + 8 * r)] = (fastT[r] ? 1.f : e32[r]) * S[2 * q + r];
+    if (issuer) {
+      mbar_arrive_expect_tx(&sm.bar_tma, 3 * kRawBytes);
+      if (!withheld) {
+        const int row0 = REV ? p.T - kL : cb * kL;
+        tma_load_3d(sm.raw[0], &mr, &sm.bar_tma, h * kN, row0, b);
+        tma_load_3d(sm.raw[1], &mk, &sm.bar_tma, h * kN, row0, b);
+        tma_load_3d(sm.raw[2], &mv, &sm.bar_tma, h * kN, row0, b);
+      }
+    }
+    ++tma_armed;
+
+    for (int c = cb; c < ce; ++c, ++m_it) {
+      const int t0 = c * kL;
+      const int cnt = min(kL, p.T - t0);
+      const uint32_t ph = (uint32_t)m_it & 1u;  // bar_tma, bar_sc, bar_av: the output pass's chunks
+      const uint32_t pg = (uint32_t)n_ds & 1u;  // bar_ds: after the scan's chains
+      if (!mbar_wait_bounded(&sm.bar_tma, ph, p.ctl)) sm.abort_flag = 1;
+
+      // T1a: r̃, k̃ and the bonus parts (rows past the sequence end hold zeros from the TMA fill).
+      // r̃ and k̃ are rounded to nearest tf32: the tensor core would truncate both, and the two
+      // biases toward zero add in every score.
+      {
+        float fr[2] = {fr0[0], fr0[1]}, fk[2] = {fk0[0], fk0[1]};
+#pragma unroll
+        for (int ib = 0; ib < 8; ++ib) {
+          const uint32_t ibo = (uint32_t)(REV ? 7 - ib : ib) * 1024u;
+          const float2 rv = bf2_to_f2(lds_u32(rawR + offRK + ibo));
+          const float2 kv = bf2_to_f2(lds_u32(rawK + offRK + ibo));
+          const int row = 8 * ib + rr;
+          *reinterpret_cast<float2*>(&sm.opR[op_off(row, dR)]) = make_float2(to_tf32(rv.x * fr[0]), to_tf32(rv.y * fr[1]));
+          *reinterpret_cast<float2*>(&sm.opK[op_off(row, dR)]) = make_float2(to_tf32(kv.x * fk[0]), to_tf32(kv.y * fk[1]));
+          float part = fmaf(rv.x * uA[0], kv.x, rv.y * uA[1] * kv.y);
+          part += __shfl_xor_sync(0xffffffffu, part, 8);
+          part += __shfl_xor_sync(0xffffffffu, part, 16);
+          if (rp == 0) sm.u.diag_part[warp][row] = part;
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            fr[e] *= frs[e];
+            fk[e] *= fks[e];
           }
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 kv = bf2_to_f2(kp[e][w]);
-            acc[e] = fmaf(rv.x * kv.x, ew[0][e], acc[e]);
-            acc[e] = fmaf(rv.y * kv.y, ew[1][e], acc[e]);
-          }
         }
-#pragma unroll
-        for (int e = 0; e < 4; ++e) sm.u.AF[tau][n0 + e] = acc[e];
       }
-      if (nfast > 0) {  // a fast row: k e^{λ(cnt-1-ι)}, zero past the chunk's tokens
+      if (nfast > 0) {  // the fast channels' r and k into the compact rows (bf16 as loaded)
+#pragma unroll
+        for (int ib = 0; ib < 8; ++ib) {
+          const uint32_t ibo = (uint32_t)(REV ? 7 - ib : ib) * 1024u;
+          const uint32_t rw = lds_u32(rawR + offRK + ibo), kw = lds_u32(rawK + offRK + ibo);
+          const int row = 8 * ib + rr;
+#pragma unroll
+          for (int e = 0; e < 2; ++e)
+            if (fiA[e] >= 0) {
+              const int col = fiA[e] >> 1;
+              unsigned short* rh = reinterpret_cast<unsigned short*>(&sm.RFw[row][col]) + (fiA[e] & 1);
+              unsigned short* kh = reinterpret_cast<unsigned short*>(&sm.KFw[row][col]) + (fiA[e] & 1);
+              *rh = (unsigned short)(e ? rw >> 16 : rw & 0xFFFFu);
+              *kh = (unsigned short)(e ? kw >> 16 : kw & 0xFFFFu);
+            }
+        }
+      }
+      fence_proxy_async();
+      tc_fence_before();
+      __syncthreads();
+      if (sm.abort_flag) {
+        aborted = true;
+        break;
+      }
+      // [scores | Y] = r̃ [k̃ ; e^{32λ} Sᵀ]ᵀ: causal scores [τ][ι] and the state read [τ][j].  The
+      // issuing thread hands the eight K steps out in pairs between its warp's T1b steps, so that
+      // the warp never waits on a full MMA queue.
+      auto issue_first = [&](int s0) {
+        if (issuer) {
+          if (s0 == 0) tc_fence_after();
+#pragma unroll
+          for (int s = s0; s < s0 + 2; ++s)
+            umma_tf32(tSc, smem_desc(&sm.opR[s * 64], kLbo, kSbo), smem_desc(&sm.opK[s * 64], kLbo, kSbo),
+                      kIdesc128, s);
+          if (s0 == 6) umma_commit(&sm.bar_sc);
+        }
+      };
+      issue_first(0);
+
+      // T1b: k̃ᵀ into tensor memory, vᵀ into shared memory, the bonus sums
+      {
+        if (tid < kL) {
+          float sum = 0.f;
+#pragma unroll
+          for (int w = 0; w < 8; ++w) sum += sm.u.diag_part[w][tid];
+          sm.diag[tid] = sum;
+        }
+        uint32_t kt[16];
 #pragma unroll
         for (int pp = 0; pp < 2; ++pp) {
-          uint32_t qk[4];
-          ldsm_x4_t(REV ? rawK + offKt - pp * 2048u : rawK + offKt + pp * 2048u, qk);
+          kt_slow(pp, kt, rawK);
+          issue_first(2 + 2 * pp);
+        }
+        if (nfast > 0) {
+          // the fast channels' scores at lags n = 0..kBand, Σ_c r_τ[c] k_{τ-1-n}[c] e^{λ_c n}: thread
+          // (τ, 4 lags), every CTA thread busy; AF overlays the bonus parts, summed above
+          __syncthreads();
+          const int tau = tid >> 2, g4 = tid & 3, n0 = 4 * g4;
+          // k rows of the four lags (a lag reaching before the chunk reads the zero row)
+          const uint32_t* kp[4];
 #pragma unroll
-          for (int m = 0; m < 4; ++m) {
-            const int i = 2 * pp + (m >> 1), r = m & 1;
-            if (fastT[r]) {
-              const float2 f = bf2_to_f2(qk[m]);
-              const int io = 32 * hc + 8 * i + 2 * tq;
-              // e^{λ n}, n = cnt-1-ι: the tabled powers up to n = 15, zero beyond (below 2^-46)
-              const int cf = sm.fidx[16 * q4 + 8 * r + t4];
-              auto pw = [&](int n) {
-                if (n < 0 || n > kBand) return 0.f;
-                float x = sm.E4[cf][n >> 2];
-                for (int t = 0; t < (n & 3); ++t) x *= sm.E1[cf];
-                return x;
-              };
-              const float c0 = pw(cnt - 1 - io), c1 = pw(cnt - 2 - io);
-              kt[4 * i + 2 * r] = __float_as_uint(f.x * c0);
-              kt[4 * i + 2 * r + 1] = __float_as_uint(f.y * c1);
+          for (int e = 0; e < 4; ++e) {
+            const int io = tau - 1 - (n0 + e);
+            kp[e] = &sm.KFw[io < 0 ? kL : io][0];
+          }
+          const uint32_t* rp = &sm.RFw[tau][0];
+          float acc[4] = {0.f, 0.f, 0.f, 0.f};
+          const int npair = (nfast + 1) >> 1;
+#pragma unroll 2
+          for (int w = 0; w < npair; ++w) {
+            const float2 rv = bf2_to_f2(rp[w]);
+            float ew[2][4];
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+              const int cfi = 2 * w + h2;
+              const float e1 = sm.E1[cfi];
+              ew[h2][0] = sm.E4[cfi][g4];
+              ew[h2][1] = ew[h2][0] * e1;
+              ew[h2][2] = ew[h2][1] * e1;
+              ew[h2][3] = ew[h2][2] * e1;
+            }
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 kv = bf2_to_f2(kp[e][w]);
+              acc[e] = fmaf(rv.x * kv.x, ew[0][e], acc[e]);
+              acc[e] = fmaf(rv.y * kv.y, ew[1][e], acc[e]);
             }
           }
+#pragma unroll
+          for (int e = 0; e < 4; ++e) sm.u.AF[tau][n0 + e] = acc[e];
+        }
+        if (nfast > 0) kt_fast(cnt, kt, rawK);
+        tmem_st16(tKt + tquar + (uint32_t)(32 * hc), kt);
+#pragma unroll
+        for (int pp = 0; pp < 2; ++pp) {
+          vt_step(pp, rawV);
+          if (pp == 0) issue_first(6);
         }
       }
-      tmem_st16(tKt + tquar + (uint32_t)(32 * hc), kt);
+      fence_proxy_async();
+      tc_fence_before();
+      __syncthreads();
+      if (ds_issuer) {
+        tc_fence_after();
+        // ΔS = k̃ᵀ v [d][j] needs only this chunk's operands: it runs while the scores are masked.
+        // Issued from warp 4, whose share of the masking is a zero fill, so that the ≈ 0.9k cycles
+        // the chain holds its issuing thread do not delay the masking barrier.
 #pragma unroll
-      for (int pp = 0; pp < 2; ++pp) {
-        uint32_t qv[4];
-        ldsm_x4_t(REV ? rawV + offT - pp * 4096u : rawV + offT + pp * 4096u, qv);
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {
-          const int ib = 4 * pp + m;
-          const uint32_t xv = __shfl_xor_sync(0xffffffffu, qv[m], 18);
-          *reinterpret_cast<float2*>(&sm.opVt[op_off(8 * warp + srow, 8 * ib + 2 * stq)]) =
-              bf2_to_f2(sw ? xv : qv[m]);
+        for (int s = 0; s < 8; ++s) umma_tf32_ts(tDS, tKt + 8 * s, smem_desc(&sm.opVt[s * 64], kLbo, kSbo), kIdesc, s);
+        umma_commit(&sm.bar_ds);
+      }
+      ++n_ds;
+      if (issuer) {
+        // the raw boxes are consumed: load the next chunk while this one computes
+        if (c + 1 < ce) {
+          fence_proxy_async();
+          mbar_arrive_expect_tx(&sm.bar_tma, 3 * kRawBytes);
+          const int rown = REV ? p.T - (c + 2) * kL : (c + 1) * kL;
+          tma_load_3d(sm.raw[0], &mr, &sm.bar_tma, h * kN, rown, b);
+          tma_load_3d(sm.raw[1], &mk, &sm.bar_tma, h * kN, rown, b);
+          tma_load_3d(sm.raw[2], &mv, &sm.bar_tma, h * kN, rown, b);
         }
-        if (pp == 0) issue_first(6);
       }
-    }
-    fence_proxy_async();
-    tc_fence_before();
-    __syncthreads();
-    if (ds_issuer) {
-      tc_fence_after();
-      // ΔS = k̃ᵀ v [d][j] needs only this chunk's operands: it runs while the scores are masked.
-      // Issued from warp 4, whose share of the masking is a zero fill, so that the ≈ 0.9k cycles
-      // the chain holds its issuing thread do not delay the masking barrier.
-#pragma unroll
-      for (int s = 0; s < 8; ++s) umma_tf32_ts(tDS, tKt + 8 * s, smem_desc(&sm.opVt[s * 64], kLbo, kSbo), kIdesc, s);
-      umma_commit(&sm.bar_ds);
-    }
-    if (issuer) {
-      // the raw boxes are consumed: load the next chunk while this one computes
-      if (c + 1 < nchunk) {
-        fence_proxy_async();
-        mbar_arrive_expect_tx(&sm.bar_tma, 3 * kRawBytes);
-        const int rown = REV ? p.T - (c + 2) * kL : (c + 1) * kL;
-        tma_load_3d(sm.raw[0], &mr, &sm.bar_tma, h * kN, rown, b);
-        tma_load_3d(sm.raw[1], &mk, &sm.bar_tma, h * kN, rown, b);
-        tma_load_3d(sm.raw[2], &mv, &sm.bar_tma, h * kN, rown, b);
-      }
-    }
+      if (c + 1 < ce) ++tma_armed;
 
-    // T2a: causal mask of the scores in tensor memory, in place (ι < τ kept, ι = τ the bonus
-    // Σ_d r u k, ι > τ zero): the A operand of A v.
-    // .16x128b fragment: rows τ = 16 q4 + t4 + 8 r, columns ι = 32 hc + 4 q + tq  ->  register 2 q + r
-    if (!mbar_wait_bounded(&sm.bar_sc, ph, p.ctl)) sm.abort_flag = 1;
-    tc_fence_after();
-    {
-      const int tau0 = 16 * q4 + t4;
-      if (hc > (q4 >> 1)) {  // strictly above the diagonal
-        float a[16];
+      // T2a: causal mask of the scores in tensor memory, in place (ι < τ kept, ι = τ the bonus
+      // Σ_d r u k, ι > τ zero): the A operand of A v.
+      // .16x128b fragment: rows τ = 16 q4 + t4 + 8 r, columns ι = 32 hc + 4 q + tq  ->  register 2 q + r
+      if (!mbar_wait_bounded(&sm.bar_sc, ph, p.ctl)) sm.abort_flag = 1;
+      tc_fence_after();
+      {
+        const int tau0 = 16 * q4 + t4;
+        if (hc > (q4 >> 1)) {  // strictly above the diagonal
+          float a[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) a[i] = 0.f;
-        tmem_st16x128(tSc + tquar + (uint32_t)(32 * hc), a);
-      } else {
-        float a[16];
-        tmem_ld16x128(tSc + tquar + (uint32_t)(32 * hc), a);
-        if (nfast > 0) {  // the fast channels' scores at lags 0..kBand (formed in T1b)
+          for (int i = 0; i < 16; ++i) a[i] = 0.f;
+          tmem_st16x128(tSc + tquar + (uint32_t)(32 * hc), a);
+        } else {
+          float a[16];
+          tmem_ld16x128(tSc + tquar + (uint32_t)(32 * hc), a);
+          if (nfast > 0) {  // the fast channels' scores at lags 0..kBand (formed in T1b)
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+#pragma unroll
+              for (int r = 0; r < 2; ++r) {
+                const int io = 32 * hc + 4 * q + tq, tau = tau0 + 8 * r, n = tau - 1 - io;
+                if (n >= 0 && n <= kBand) a[2 * q + r] += sm.u.AF[tau][n];
+              }
+          }
+          float dg[2] = {0.f, 0.f};
+          if ((q4 >> 1) == hc) {  // the fragment holds the diagonal
+            dg[0] = sm.diag[tau0];
+            dg[1] = sm.diag[tau0 + 8];
+          }
 #pragma unroll
           for (int q = 0; q < 8; ++q)
 #pragma unroll
             for (int r = 0; r < 2; ++r) {
-              const int io = 32 * hc + 4 * q + tq, tau = tau0 + 8 * r, n = tau - 1 - io;
-              if (n >= 0 && n <= kBand) a[2 * q + r] += sm.u.AF[tau][n];
+              const int io = 32 * hc + 4 * q + tq, tau = tau0 + 8 * r;
+              a[2 * q + r] = io < tau ? a[2 * q + r] : (io == tau ? dg[r] : 0.f);
             }
+          tmem_st16x128(tSc + tquar + (uint32_t)(32 * hc), a);
         }
-        float dg[2] = {0.f, 0.f};
-        if ((q4 >> 1) == hc) {  // the fragment holds the diagonal
-          dg[0] = sm.diag[tau0];
-          dg[1] = sm.diag[tau0 + 8];
-        }
-#pragma unroll
-        for (int q = 0; q < 8; ++q)
-#pragma unroll
-          for (int r = 0; r < 2; ++r) {
-            const int io = 32 * hc + 4 * q + tq, tau = tau0 + 8 * r;
-            a[2 * q + r] = io < tau ? a[2 * q + r] : (io == tau ? dg[r] : 0.f);
-          }
-        tmem_st16x128(tSc + tquar + (uint32_t)(32 * hc), a);
       }
-    }
-    tc_fence_before();
-    __syncthreads();
-    if (issuer) {
+      tc_fence_before();
+      __syncthreads();
+      if (issuer) {
+        tc_fence_after();
+        // Y += (masked scores) v, the scores read from tensor memory
+#pragma unroll
+        for (int s = 0; s < 8; ++s) umma_tf32_ts(tY, tSc + 8 * s, smem_desc(&sm.opVt[s * 64], kLbo, kSbo), kIdesc, 1);
+        umma_commit(&sm.bar_av);
+      }
+      ++n_av;
+
+      // T2b: S <- e^{cnt λ} S + e^{(cnt-32) λ} ΔS; e^{32λ} Sᵀ into opS for the next chunk (while A v
+      // still runs).  A fast row's ΔS already carries e^{λ(cnt-1-ι)}, and its opS row is S itself.
+      if (!mbar_wait_bounded(&sm.bar_ds, pg, p.ctl)) sm.abort_flag = 1;
       tc_fence_after();
-      // Y += (masked scores) v, the scores read from tensor memory
+      {
+        float ds[16];
+        tmem_ld16x128(tDS + tquar + (uint32_t)(32 * hc), ds);
+        if (cnt == kL) {
 #pragma unroll
-      for (int s = 0; s < 8; ++s) umma_tf32_ts(tY, tSc + 8 * s, smem_desc(&sm.opVt[s * 64], kLbo, kSbo), kIdesc, 1);
-      umma_commit(&sm.bar_av);
-    }
-
-    // T2b: S <- e^{cnt λ} S + e^{(cnt-32) λ} ΔS; e^{32λ} Sᵀ into opS for the next chunk (while A v
-    // still runs).  A fast row's ΔS already carries e^{λ(cnt-1-ι)}, and its opS row is S itself.
-    if (!mbar_wait_bounded(&sm.bar_ds, ph, p.ctl)) sm.abort_flag = 1;
-    tc_fence_after();
-    {
-      float ds[16];
-      tmem_ld16x128(tDS + tquar + (uint32_t)(32 * hc), ds);
-      if (cnt == kL) {
+          for (int q = 0; q < 8; ++q)
 #pragma unroll
-        for (int q = 0; q < 8; ++q)
+            for (int r = 0; r < 2; ++r) {
+              const int x = 2 * q + r;
+              const float g = e32[r];
+              if (fastT[r]) {
+                S[x] = fmaf(g * g, S[x], ds[x]);
+                sm.opS[op_off(jcol + 4 * q, drow + 8 * r)] = S[x];
+              } else {
+                S[x] = g * fmaf(g, S[x], ds[x]);
+                sm.opS[op_off(jcol + 4 * q, drow + 8 * r)] = g * S[x];
+              }
+            }
+        } else {  // last, partial chunk: no later chunk reads opS
 #pragma unroll
           for (int r = 0; r < 2; ++r) {
-            const int x = 2 * q + r;
-            const float g = e32[r];
-            if (fastT[r]) {
-              S[x] = fmaf(g * g, S[x], ds[x]);
-              sm.opS[op_off(jcol + 4 * q, drow + 8 * r)] = S[x];
-            } else {
-              S[x] = g * fmaf(g, S[x], ds[x]);
-              sm.opS[op_off(jcol + 4 * q, drow + 8 * r)] = g * S[x];
-            }
+            const float rate = expf(om[drow + 8 * r]);
+            const float dl = expf(-rate * (float)cnt), gs = fastT[r] ? 1.f : expf(-rate * (float)(cnt - 32));
+#pragma unroll
+            for (int q = 0; q < 8; ++q) S[2 * q + r] = fmaf(dl, S[2 * q + r], gs * ds[2 * q + r]);
           }
-      } else {  // last, partial chunk: no later chunk reads opS
+        }
+      }
+
+      // T3: Y rows -> bf16 -> global (TMEM lanes 0..15 of each quarter hold the rows)
+      if (!mbar_wait_bounded(&sm.bar_av, ph, p.ctl)) sm.abort_flag = 1;
+      tc_fence_after();
+      {
+        float yv[32];
+        tmem_ld32(tY + tquar + (uint32_t)(32 * hc), yv);
+        const int tau = 16 * q4 + lane;
+        if (lane < 16 && tau < cnt) {
+          const int ty = REV ? p.T - 1 - (t0 + tau) : t0 + tau;
+          __nv_bfloat16* yp = p.y + (((size_t)b * p.T + ty) * p.H + h) * kN + 32 * hc;
 #pragma unroll
-        for (int r = 0; r < 2; ++r) {
-          const float rate = expf(om[drow + 8 * r]);
-          const float dl = expf(-rate * (float)cnt), gs = fastT[r] ? 1.f : expf(-rate * (float)(cnt - 32));
+          for (int j = 0; j < 32; j += 8) {
+            uint4 pk;
+            __nv_bfloat162* q2 = reinterpret_cast<__nv_bfloat162*>(&pk);
 #pragma unroll
-          for (int q = 0; q < 8; ++q) S[2 * q + r] = fmaf(dl, S[2 * q + r], gs * ds[2 * q + r]);
+            for (int e = 0; e < 4; ++e) q2[e] = __floats2bfloat162_rn(yv[j + 2 * e], yv[j + 2 * e + 1]);
+            *reinterpret_cast<uint4*>(yp + j) = pk;
+          }
         }
       }
     }
-
-    // T3: Y rows -> bf16 -> global (TMEM lanes 0..15 of each quarter hold the rows)
-    if (!mbar_wait_bounded(&sm.bar_av, ph, p.ctl)) sm.abort_flag = 1;
-    tc_fence_after();
-    {
-      float yv[32];
-      tmem_ld32(tY + tquar + (uint32_t)(32 * hc), yv);
-      const int tau = 16 * q4 + lane;
-      if (lane < 16 && tau < cnt) {
-        const int ty = REV ? p.T - 1 - (t0 + tau) : t0 + tau;
-        __nv_bfloat16* yp = p.y + (((size_t)b * p.T + ty) * p.H + h) * kN + 32 * hc;
+    if (aborted) break;
+    if (ce == nchunk && p.s_out != nullptr) {  // the head's last chunk: its final state
+      const size_t sb = ((size_t)b * p.H + h) * kN * kN;
 #pragma unroll
-        for (int j = 0; j < 32; j += 8) {
-          uint4 pk;
-          __nv_bfloat162* q2 = reinterpret_cast<__nv_bfloat162*>(&pk);
+      for (int q = 0; q < 8; ++q)
 #pragma unroll
-          for (int e = 0; e < 4; ++e) q2[e] = __floats2bfloat162_rn(yv[j + 2 * e], yv[j + 2 * e + 1]);
-          *reinterpret_cast<uint4*>(yp + j) = pk;
-        }
-      }
+        for (int r = 0; r < 2; ++r) p.s_out[sb + (size_t)(drow + 8 * r) * kN + jcol + 4 * q] = S[2 * q + r];
     }
   }
 
   if (aborted && tid == 0) {
-    // a wait gave up at chunk c: the previous chunk's MMA chains (A v committed last by this
-    // thread on bar_av, ΔS by warp 4's on bar_ds) and this chunk's loads must finish before the
-    // tensor memory and shared memory are released, each wait bounded again
-    if (c >= 1) {
-      mbar_wait_bounded(&sm.bar_av, (uint32_t)(c - 1) & 1u, p.ctl);
-      mbar_wait_bounded(&sm.bar_ds, (uint32_t)(c - 1) & 1u, p.ctl);
+    // a wait gave up: what was issued before it must finish before the tensor memory and shared
+    // memory are released, each wait bounded again: the last A v and state-increment chains (a
+    // commit covers every earlier chain of its issuing thread), the last batch of output-pass
+    // loads and each scan stage's last loads
+    if (n_av > 0) mbar_wait_bounded(&sm.bar_av, (uint32_t)(n_av - 1) & 1u, p.ctl);
+    if (n_ds > 0) mbar_wait_bounded(&sm.bar_ds, (uint32_t)(n_ds - 1) & 1u, p.ctl);
+    if (!withheld) {
+      if (tma_armed > 0) mbar_wait_bounded(&sm.bar_tma, (uint32_t)(tma_armed - 1) & 1u, p.ctl);
+      for (int st = 0; st < min(3, scan_loaded); ++st)  // stage st's last load: its ((scan_loaded - 1 - st) / 3)-th
+        mbar_wait_bounded(&sm.bar_scan[st], (uint32_t)((scan_loaded - 1 - st) / 3) & 1u, p.ctl);
     }
-    if (!withheld) mbar_wait_bounded(&sm.bar_tma, (uint32_t)c & 1u, p.ctl);
-  }
-  if (p.s_out != nullptr) {
-#pragma unroll
-    for (int q = 0; q < 8; ++q)
-#pragma unroll
-      for (int r = 0; r < 2; ++r) p.s_out[sbase + (size_t)(drow + 8 * r) * kN + jcol + 4 * q] = S[2 * q + r];
   }
   tc_fence_before();
   __syncthreads();
@@ -603,10 +825,12 @@ cudaError_t launch_wkv5_fwd(const CUtensorMap& mr, const CUtensorMap& mk, const 
                             : reinterpret_cast<const void*>(wkv5_fwd_tc_kernel<false>);
   cudaError_t e = ensure_smem_attr(fn, (int)smem, reversed ? &mask_r : &mask_f);
   if (e != cudaSuccess) return e;
+  // one CTA per slot, or per head
+  const long long nblk = p.nslot > 0 && !reversed ? (long long)p.nslot : (long long)p.B * p.H;
   if (reversed)
-    wkv5_fwd_tc_kernel<true><<<(unsigned)(p.B * p.H), kThreads, smem, st>>>(mr, mk, mv, p);
+    wkv5_fwd_tc_kernel<true><<<(unsigned)nblk, kThreads, smem, st>>>(mr, mk, mv, p);
   else
-    wkv5_fwd_tc_kernel<false><<<(unsigned)(p.B * p.H), kThreads, smem, st>>>(mr, mk, mv, p);
+    wkv5_fwd_tc_kernel<false><<<(unsigned)nblk, kThreads, smem, st>>>(mr, mk, mv, p);
   return cudaGetLastError();
 }
 

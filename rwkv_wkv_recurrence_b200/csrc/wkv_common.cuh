@@ -98,6 +98,32 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t phase,
   return true;
 }
 
+// Flags one CTA publishes for others of the same launch (release / acquire at GPU scope).
+__device__ __forceinline__ void flag_release(unsigned int* f, unsigned int v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(f), "r"(v) : "memory");
+}
+__device__ __forceinline__ unsigned int flag_acquire(const unsigned int* f) {
+  unsigned int v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(f) : "memory");
+  return v;
+}
+// Polls a flag until it is non-zero or the control block's time limit passes; 0 then (and the
+// timeout bit is set in the error word).
+__device__ __forceinline__ unsigned int flag_wait_bounded(const unsigned int* f, DevCtl* ctl) {
+  unsigned int v = flag_acquire(f);
+  if (v != 0u) return v;
+  const unsigned long long t0 = global_ns();
+  const unsigned long long limit = *reinterpret_cast<volatile unsigned long long*>(&ctl->wait_limit_ns);
+  while ((v = flag_acquire(f)) == 0u) {
+    if (global_ns() - t0 > limit) {
+      atomicOr(&ctl->err, kErrTmaTimeout);
+      return 0u;
+    }
+    __nanosleep(64);
+  }
+  return v;
+}
+
 // True when the test hook asks the issuing thread to withhold its loads.
 __device__ __forceinline__ bool loads_withheld(const DevCtl* ctl) {
   return *reinterpret_cast<const volatile unsigned int*>(&ctl->withhold) != 0u;

@@ -61,6 +61,15 @@ def test_checkpoint_and_workspace_queries():
     assert ws >= 22 * 768 * 3 * 8 + 22 * 24 * 4 and ws < 22 * 768 * 3 * 8 + 4096
     assert h.rwkv_wkv4_forward_workspace_bytes(8, 1024, 768, rw.ALGO_CHUNKED) > 0
     assert h.rwkv_wkv4_forward_workspace_bytes(0, 10, 10, 0) == 0
+    # Eagle forward: the heads' 64-token chunks are dealt out to 296 CTAs (two per SM); per CTA
+    # a 64 x 64 fp32 summary and a flag, and a ticket counter
+    for shape in [(4, 4096, 40), (1, 4096, 40), (8, 4096, 40)]:
+        ws = h.rwkv_wkv5_forward_workspace_bytes(*shape, 64)
+        assert ws >= 296 * 64 * 64 * 4 + 297 * 4 and ws < 296 * 64 * 64 * 4 + 4096, shape
+    ws = h.rwkv_wkv5_forward_workspace_bytes(1, 128, 1, 64)  # two chunks: two CTAs
+    assert ws >= 2 * 64 * 64 * 4 + 3 * 4 and ws < 2 * 64 * 64 * 4 + 1024
+    assert h.rwkv_wkv5_forward_workspace_bytes(4, 64, 40, 64) == 0  # one chunk per head: one CTA per head
+    assert h.rwkv_wkv5_forward_workspace_bytes(4, 4096, 40, 32) == 0
 
 
 def test_validation_before_any_cuda_work():
@@ -120,6 +129,11 @@ def test_validation_before_any_cuda_work():
                                None) == 2
     assert h.rwkv_wkv5_forward(1, 4, 2, 64, fake, fake, fake, None, fake, fake, None, None, None, 0,
                                None) == 1
+    # the slot plan without the workspace it needs
+    assert h.rwkv_wkv5_forward(4, 4096, 40, 64, fake, fake, fake, fake, fake, fake, None, None, None, 0,
+                               None) == 3
+    assert h.rwkv_wkv5_forward(4, 4096, 40, 64, fake, fake, fake, fake, fake, fake, None, None, fake,
+                               h.rwkv_wkv5_forward_workspace_bytes(4, 4096, 40, 64) - 1, None) == 3
     # WKV-5 decode step: only N = 64, output state required, 16-byte aligned states
     assert h.rwkv_wkv5_step(2, 3, 32, fake, fake, fake, fake, fake, fake, None, fake, None) == 2
     assert h.rwkv_wkv5_step(2, 3, 64, fake, fake, fake, fake, fake, fake, None, None, None) == 1

@@ -207,11 +207,14 @@ def test_matrix_state_guarded(cuda_device, finch):
     y = Guarded((B, T, H, 64), torch.bfloat16, dev)
     so = Guarded((B, H, 64, 64), torch.float32, dev)
     fwd = h.rwkv_wkv6_forward if finch else h.rwkv_wkv5_forward
+    wsb = int((h.rwkv_wkv6_forward_workspace_bytes if finch else h.rwkv_wkv5_forward_workspace_bytes)(B, T, H, 64))
+    ws = Guarded((max(wsb, 4) // 4,), torch.float32, dev)  # the scratch, fenced by sentinels too
     assert fwd(B, T, H, 64, P(g["r"]), P(g["k"]), P(g["v"]), P(g["omega"]), P(g["u"]), y.ptr(), None, so.ptr(),
-               None, 0, S) == 0
+               ws.ptr(), wsb, S) == 0
     rw.rwkv_check_device_error()
     y.check("y")
     so.check("s_out")
+    ws.check("workspace")
     ref, ref_s = (oracle.wkv6_forward if finch else oracle.wkv5_forward)(p["r"], p["k"], p["v"], p["omega"], p["u"],
                                                                          return_state=True)
     assert_close_rms(y.t, ref, TOL_BF16, "y")

@@ -21,6 +21,8 @@ def _calls(dev):
     p = {k: v.to(dev) for k, v in wi.wkv4_problem(2, 130, 64, 61, outliers=True, with_gy=True).items()}
     e = {k: v.to(dev) for k, v in wi.wkv5_problem(1, 70, 2, 64, seed=62).items()}
     f = {k: v.to(dev) for k, v in wi.wkv6_problem(1, 70, 2, 64, seed=63).items()}
+    # 160 heads of 4 chunks over 296 CTAs that wait for one another's summaries
+    c = {k: v.to(dev) for k, v in wi.wkv5_problem(4, 200, 40, 64, seed=64).items()}
     ck = rw.rwkv_wkv4_forward(p["w"], p["u"], p["k"], p["v"], checkpoints=True)[1]
     torch.cuda.synchronize()
     return {
@@ -28,6 +30,7 @@ def _calls(dev):
         "wkv4 chunked forward": lambda: rw.rwkv_wkv4_forward(p["w"], p["u"], p["k"], p["v"], algo=rw.ALGO_CHUNKED),
         "wkv4 backward": lambda: rw.rwkv_wkv4_backward(p["w"], p["u"], p["k"], p["v"], p["gy"], ckpt=ck),
         "eagle forward": lambda: rw.rwkv_wkv5_forward(e["r"], e["k"], e["v"], e["omega"], e["u"]),
+        "eagle forward, split heads": lambda: rw.rwkv_wkv5_forward(c["r"], c["k"], c["v"], c["omega"], c["u"]),
         "finch forward": lambda: rw.rwkv_wkv6_forward(f["r"], f["k"], f["v"], f["omega"], f["u"]),
     }
 

@@ -109,6 +109,68 @@ def test_eagle_fast_decay_full_size(cuda_device):
             assert_close_rms(sc[b, h], ref_s[b, h], TOL_BF16, f"s head ({b},{h})")
 
 
+# ------------------------------------------------------------------ the slot plan
+def _state(p, B, H, seed):
+    """A state the recurrence produces: the oracle's after 64 other tokens with p's decays and
+    bonus, rounded to fp32 (so its size matches the decays, as a state handed over would)."""
+    q = wi.wkv5_problem(B, 64, H, 64, seed=seed)
+    _, s = oracle.wkv5_forward(q["r"], q["k"], q["v"], p["omega"], p["u"], return_state=True)
+    return torch.from_numpy(s).float()
+
+
+def _check_heads(y, s, ref, ref_s):
+    yc, sc = y.cpu(), s.cpu()
+    for b in range(yc.shape[0]):
+        for h in range(yc.shape[2]):
+            assert_close_rms(yc[b, :, h], ref[b, :, h], TOL_BF16, f"y head ({b},{h})")
+            assert_close_rms(sc[b, h], ref_s[b, h], TOL_BF16, f"s head ({b},{h})")
+
+
+@pytest.mark.parametrize("shape,omega_range", [((4, 1000, 40), (-6.0, 0.0)), ((1, 700, 150), (-6.0, 0.0)),
+                                               ((2, 333, 80), (-1.0, 2.0)), ((1, 200, 222), (-6.0, 0.0)),
+                                               ((1, 1500, 3), (-6.0, 0.0)), ((8, 300, 40), (-1.0, 2.0)),
+                                               ((1, 64 * 40 + 17, 1), (-1.0, 2.0))])
+def test_forward_slot_plan(cuda_device, shape, omega_range):
+    # The heads' chunks laid end to end and dealt out to 296 CTAs: a CTA holds the tail of one
+    # head, whole heads and the start of another, and folds the summaries of the CTAs before it
+    # into the start state of a head it does not start (one head over 41 CTAs, 3 heads over 8
+    # to 9 each, 320 heads over two per CTA).  Every head against the oracle, from a nonzero
+    # state, T ragged, slow and fast decays.
+    B, T, H = shape
+    assert rw.lib().rwkv_wkv5_forward_workspace_bytes(B, T, H, 64) > 0
+    p = wi.wkv5_problem(B, T, H, 64, seed=36, omega_range=omega_range)
+    s0 = _state(p, B, H, 37)
+    y, s = rw.rwkv_wkv5_forward(**_cuda(p, cuda_device), s_in=s0.to(cuda_device), return_state=True)
+    rw.rwkv_check_device_error()
+    ref, ref_s = oracle.wkv5_forward(p["r"], p["k"], p["v"], p["omega"], p["u"], s_in=s0.double().numpy(),
+                                     return_state=True)
+    _check_heads(y, s, ref, ref_s)
+    y2, s2 = rw.rwkv_wkv5_forward(**_cuda(p, cuda_device), s_in=s0.to(cuda_device), return_state=True)
+    assert torch.equal(y, y2) and torch.equal(s, s2)  # the summaries fold in a fixed order
+
+
+def test_forward_slot_plan_state_in_place(cuda_device):
+    # s_out is s_in: the CTA holding a head's last chunk writes its final state while the CTAs
+    # holding its earlier chunks may still be running, so each reads s_in before it publishes
+    # its summary
+    B, T, H = 4, 1000, 40
+    q = wi.wkv5_problem(B, T, H, 64, seed=38)
+    p = _cuda(q, cuda_device)
+    s0 = _state(q, B, H, 39)
+    st = s0.to(cuda_device)
+    h = rw.lib()
+    wsb = int(h.rwkv_wkv5_forward_workspace_bytes(B, T, H, 64))
+    ws = torch.empty(wsb, dtype=torch.uint8, device=cuda_device)
+    y = torch.empty_like(p["r"])
+    assert h.rwkv_wkv5_forward(B, T, H, 64, rw._ptr(p["r"]), rw._ptr(p["k"]), rw._ptr(p["v"]), rw._ptr(p["omega"]),
+                               rw._ptr(p["u"]), rw._ptr(y), rw._ptr(st), rw._ptr(st), rw._ptr(ws), wsb,
+                               rw._stream(None)) == 0
+    rw.rwkv_check_device_error()
+    ref, ref_s = oracle.wkv5_forward(q["r"], q["k"], q["v"], q["omega"], q["u"], s_in=s0.double().numpy(),
+                                     return_state=True)
+    _check_heads(y, st, ref, ref_s)
+
+
 # ------------------------------------------------------------------ decode step
 def _token(p, t):
     return {n: p[n][:, t].contiguous() for n in ("r", "k", "v")}
