@@ -105,6 +105,7 @@ struct Wkv5Smem {
   alignas(8) uint64_t bar_av;        // A v done
   alignas(8) uint64_t bar_ds;        // state increment done
   alignas(8) uint64_t bar_scan[3];   // a summary scan's k, v boxes, three stages
+  alignas(8) uint64_t bar_scan_ds[4];  // a summary scan's products: [issuer][chunk parity]
   uint32_t tmem_base;
   int nfast;
   int abort_flag;
@@ -178,6 +179,7 @@ __global__ void __launch_bounds__(kThreads, 2) wkv5_fwd_tc_kernel(const __grid_c
     mbar_init(&sm.bar_av, 1);
     mbar_init(&sm.bar_ds, 1);
     for (int st = 0; st < 3; ++st) mbar_init(&sm.bar_scan[st], 1);
+    for (int x = 0; x < 4; ++x) mbar_init(&sm.bar_scan_ds[x], 1);
     fence_mbar_init();
   }
 
@@ -341,21 +343,22 @@ __global__ void __launch_bounds__(kThreads, 2) wkv5_fwd_tc_kernel(const __grid_c
       }
     }
   };
-  // vᵀ from the v box at vbox into opVt, step pp of two
-  auto vt_step = [&](int pp, uint32_t vbox) {
+  // vᵀ from the v box at vbox into the tile vt (opVt; a summary scan alternates with opS), step pp of two
+  auto vt_step = [&](int pp, uint32_t vbox, float* vt) {
     uint32_t qv[4];
     ldsm_x4_t(REV ? vbox + offT - pp * 4096u : vbox + offT + pp * 4096u, qv);
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
       const int ib = 4 * pp + m;
       const uint32_t xv = __shfl_xor_sync(0xffffffffu, qv[m], 18);
-      *reinterpret_cast<float2*>(&sm.opVt[op_off(8 * warp + srow, 8 * ib + 2 * stq)]) = bf2_to_f2(sw ? xv : qv[m]);
+      *reinterpret_cast<float2*>(&vt[op_off(8 * warp + srow, 8 * ib + 2 * stq)]) = bf2_to_f2(sw ? xv : qv[m]);
     }
   };
 
   // counts the abort path needs: output-pass chunks begun, chains committed, load batches armed
   int m_it = 0, n_ds = 0, n_av = 0, tma_armed = 0;
   int scan_loaded = 0;  // chunks of the summary scan whose loads were issued (chunk i in stage i % 3)
+  int scan_done = 0;    // chunks of the summary scan whose products were issued
   bool aborted = false;
 
   if (summary) {
@@ -383,9 +386,23 @@ __global__ void __launch_bounds__(kThreads, 2) wkv5_fwd_tc_kernel(const __grid_c
     };
     for (; scan_loaded < min(3, n); ++scan_loaded)
       if (issuer) scan_load(scan_loaded);
+    // Chunk i's k̃ᵀ and vᵀ go to tile pair i & 1 ((tKt, opVt) or (tSc, opS)), so that a chunk is
+    // built while the one before it is multiplied.  The eight K steps are split between two
+    // issuing threads with an accumulator each (steps 0..3 by thread 0 into tY, 4..7 by warp 4's
+    // into tDS, added at the end): each MMA holds its issuing thread ~70 cycles, and neither
+    // warp then falls far behind the others' share of the next build.  Each issuer commits to
+    // the barrier of its chunk parity, bar_scan_ds[2 x + (i & 1)], once per two chunks.
+    auto scan_bar = [&](int x, int i) { return &sm.bar_scan_ds[2 * x + (i & 1)]; };
     for (int i = 0; i < n; ++i) {
       const int st = i % 3;
+      const uint32_t tk = (i & 1) ? tSc : tKt;
+      float* const vt = (i & 1) ? sm.opS : sm.opVt;
       if (!mbar_wait_bounded(&sm.bar_scan[st], (uint32_t)(i / 3) & 1u, p.ctl)) sm.abort_flag = 1;
+      if (i >= 2) {  // chunk i - 2's products have read this tile pair
+        const uint32_t par = (uint32_t)((i - 2) >> 1) & 1u;
+        if (!mbar_wait_bounded(scan_bar(0, i), par, p.ctl) || !mbar_wait_bounded(scan_bar(1, i), par, p.ctl))
+          sm.abort_flag = 1;
+      }
       {
         uint32_t kt[16];
         const uint32_t kbox = smem_u32(stage_k(st));
@@ -404,12 +421,10 @@ __global__ void __launch_bounds__(kThreads, 2) wkv5_fwd_tc_kernel(const __grid_c
         }
         // a fast row keeps the last 16 positions only (beyond, its weight is below 2^-46)
         if (nfast > 0 && i == n - 1) kt_fast(kL, kt, kbox);
-        tmem_st16(((i & 1) ? tSc : tKt) + tquar + (uint32_t)(32 * hc), kt);
+        tmem_st16(tk + tquar + (uint32_t)(32 * hc), kt);
       }
-      // the previous chunk's products have read vᵀ (and the k̃ᵀ tile this chunk overwrites)
-      if (i > 0 && !mbar_wait_bounded(&sm.bar_ds, (uint32_t)(n_ds - 1) & 1u, p.ctl)) sm.abort_flag = 1;
-      vt_step(0, smem_u32(stage_k(st)) + kRawBytes);
-      vt_step(1, smem_u32(stage_k(st)) + kRawBytes);
+      vt_step(0, smem_u32(stage_k(st)) + kRawBytes, vt);
+      vt_step(1, smem_u32(stage_k(st)) + kRawBytes, vt);
       fence_proxy_async();
       tc_fence_before();
       __syncthreads();
@@ -417,25 +432,31 @@ __global__ void __launch_bounds__(kThreads, 2) wkv5_fwd_tc_kernel(const __grid_c
         aborted = true;
         break;
       }
-      if (ds_issuer) {
+      if (issuer || ds_issuer) {
         tc_fence_after();
+        const int x = issuer ? 0 : 1;
+        const uint32_t acc = issuer ? tY : tDS;
 #pragma unroll
-        for (int s = 0; s < 8; ++s)
-          umma_tf32_ts(tDS, ((i & 1) ? tSc : tKt) + 8 * s, smem_desc(&sm.opVt[s * 64], kLbo, kSbo), kIdesc,
-                       (i > 0 || s > 0) ? 1u : 0u);
-        umma_commit(&sm.bar_ds);
+        for (int s4 = 0; s4 < 4; ++s4) {
+          const int s = 4 * x + s4;
+          umma_tf32_ts(acc, tk + 8 * s, smem_desc(&vt[s * 64], kLbo, kSbo), kIdesc, (i > 0 || s4 > 0) ? 1u : 0u);
+        }
+        umma_commit(scan_bar(x, i));
       }
-      ++n_ds;
+      ++scan_done;
       if (scan_loaded < n) {  // stage st is consumed: chunk i + 3 into it
         if (issuer) scan_load(scan_loaded);
         ++scan_loaded;
       }
     }
     if (!aborted) {
-      if (!mbar_wait_bounded(&sm.bar_ds, (uint32_t)(n_ds - 1) & 1u, p.ctl)) sm.abort_flag = 1;
+      const uint32_t par = (uint32_t)((n - 1) >> 1) & 1u;  // the last chunk's commits cover every earlier product
+      if (!mbar_wait_bounded(scan_bar(0, n - 1), par, p.ctl) || !mbar_wait_bounded(scan_bar(1, n - 1), par, p.ctl))
+        sm.abort_flag = 1;
       tc_fence_after();
-      float sum[16];
+      float sum[16], sum2[16];
       tmem_ld16x128(tDS + tquar + (uint32_t)(32 * hc), sum);
+      tmem_ld16x128(tY + tquar + (uint32_t)(32 * hc), sum2);
       tc_fence_before();
       __syncthreads();
       aborted = sm.abort_flag != 0;
@@ -444,7 +465,8 @@ __global__ void __launch_bounds__(kThreads, 2) wkv5_fwd_tc_kernel(const __grid_c
 #pragma unroll
         for (int q = 0; q < 8; ++q)
 #pragma unroll
-          for (int r = 0; r < 2; ++r) dst[(size_t)(drow + 8 * r) * kN + jcol + 4 * q] = sum[2 * q + r];
+          for (int r = 0; r < 2; ++r)
+            dst[(size_t)(drow + 8 * r) * kN + jcol + 4 * q] = sum[2 * q + r] + sum2[2 * q + r];
       }
     }
     // publish it, or that this slot gave up (the slots waiting for it then stop at once)
@@ -526,7 +548,7 @@ __global__ void __launch_bounds__(kThreads, 2) wkv5_fwd_tc_kernel(const __grid_c
       const int t0 = c * kL;
       const int cnt = min(kL, p.T - t0);
       const uint32_t ph = (uint32_t)m_it & 1u;  // bar_tma, bar_sc, bar_av: the output pass's chunks
-      const uint32_t pg = (uint32_t)n_ds & 1u;  // bar_ds: after the scan's chains
+      const uint32_t pg = (uint32_t)n_ds & 1u;  // bar_ds: the output pass's state increments
       if (!mbar_wait_bounded(&sm.bar_tma, ph, p.ctl)) sm.abort_flag = 1;
 
       // T1a: r̃, k̃ and the bonus parts (rows past the sequence end hold zeros from the TMA fill).
@@ -648,7 +670,7 @@ __global__ void __launch_bounds__(kThreads, 2) wkv5_fwd_tc_kernel(const __grid_c
         tmem_st16(tKt + tquar + (uint32_t)(32 * hc), kt);
 #pragma unroll
         for (int pp = 0; pp < 2; ++pp) {
-          vt_step(pp, rawV);
+          vt_step(pp, rawV, sm.opVt);
           if (pp == 0) issue_first(6);
         }
       }
@@ -799,6 +821,10 @@ __global__ void __launch_bounds__(kThreads, 2) wkv5_fwd_tc_kernel(const __grid_c
     // loads and each scan stage's last loads
     if (n_av > 0) mbar_wait_bounded(&sm.bar_av, (uint32_t)(n_av - 1) & 1u, p.ctl);
     if (n_ds > 0) mbar_wait_bounded(&sm.bar_ds, (uint32_t)(n_ds - 1) & 1u, p.ctl);
+    for (int x = 0; x < 4; ++x) {  // the scan's products: commits on bar_scan_ds[x], one per chunk of parity x & 1
+      const int uses = (scan_done + 1 - (x & 1)) / 2;
+      if (uses > 0) mbar_wait_bounded(&sm.bar_scan_ds[x], (uint32_t)(uses - 1) & 1u, p.ctl);
+    }
     if (!withheld) {
       if (tma_armed > 0) mbar_wait_bounded(&sm.bar_tma, (uint32_t)(tma_armed - 1) & 1u, p.ctl);
       for (int st = 0; st < min(3, scan_loaded); ++st)  // stage st's last load: its ((scan_loaded - 1 - st) / 3)-th
