@@ -70,6 +70,7 @@ def test_checkpoint_and_workspace_queries():
     assert ws >= 2 * 64 * 64 * 4 + 3 * 4 and ws < 2 * 64 * 64 * 4 + 1024
     assert h.rwkv_wkv5_forward_workspace_bytes(4, 64, 40, 64) == 0  # one chunk per head: one CTA per head
     assert h.rwkv_wkv5_forward_workspace_bytes(4, 4096, 40, 32) == 0
+    assert h.rwkv_wkv6_forward_workspace_bytes(4, 4096, 40, 64) == 0  # Finch: one CTA per head
 
 
 def test_validation_before_any_cuda_work():

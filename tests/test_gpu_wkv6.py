@@ -93,9 +93,11 @@ def test_state_in_place(cuda_device):
     s_io = s0.clone()
     h = rw.lib()
     y2 = torch.empty_like(y1)
+    wsb = int(h.rwkv_wkv6_forward_workspace_bytes(B, T, H, 64))
+    ws = torch.empty(max(wsb, 1), dtype=torch.uint8, device=cuda_device)
     assert h.rwkv_wkv6_forward(B, T, H, 64, g["r"].data_ptr(), g["k"].data_ptr(), g["v"].data_ptr(),
                                g["omega"].data_ptr(), g["u"].data_ptr(), y2.data_ptr(), s_io.data_ptr(),
-                               s_io.data_ptr(), None, 0, None) == 0
+                               s_io.data_ptr(), ws.data_ptr(), wsb, None) == 0
     torch.cuda.synchronize()
     assert torch.equal(y1, y2) and torch.equal(s1, s_io)
     ref, ref_s = _ref(p, s_in=s0.cpu().double().numpy())
