@@ -170,26 +170,33 @@ FwdPlan plan_forward(int64_t B, int64_t T, int64_t C, int algo) {
 // Eagle forward: a head's chunks form a chain (each reads the state the one before leaves), and
 // one CTA per head leaves the call as long as one head's chain however many SMs are idle, or
 // twice that when a few heads are over two per SM.  The slot plan deals the heads' chunks, laid
-// end to end, out evenly to two CTAs per SM; a CTA whose chunks end inside a head first scans
-// them for a summary (the state they reach from a zero state) that the CTAs holding the rest of
-// that head fold into their start states.
+// end to end, out evenly to two CTAs per SM; a CTA whose chunks end inside a head first scans them
+// for a summary (the state they reach from a zero state) that the CTAs holding the rest of that
+// head fold into their start states.  (A deal that balanced a modelled cost, giving fewer chunks
+// to a CTA that also scans, measured no faster.)
 constexpr int kEagleSlotsPerSM = 2;  // resident CTAs per SM (shared memory)
+static_assert(kEagleSlotsPerSM * kDesignSMs == kWkv5MaxSlots, "slot bound of the kernel parameters");
 
-struct Wkv5Slots {
+struct MatrixSlots {
   int nslot = 0;
+  int first[kWkv5MaxSlots + 1] = {};  // chunk boundaries: slot s takes [first[s], first[s + 1])
   size_t sum = 0, flag = 0, flag_bytes = 0, total = 0;  // workspace offsets and bytes
 };
 
-Wkv5Slots plan_wkv5_slots(int64_t B, int64_t T, int64_t H) {
-  Wkv5Slots pl;
+// The Eagle forward's plan: slot s takes chunks [floor(s N / nslot), floor((s + 1) N / nslot)) of
+// the N = B H ceil(T / 64) chunks, with a 64 x 64 fp32 summary and a flag per slot and the ticket
+// counter in the workspace.
+MatrixSlots plan_matrix_slots(int64_t B, int64_t T, int64_t H, int64_t slot_floats) {
+  MatrixSlots pl;
   const int64_t nchunk = (T + 63) / 64, nflat = B * H * nchunk;
-  // one chunk per head: nothing to split; the flat index times the slot count must fit 64 bits
-  if (nchunk < 2 || nflat >= ((int64_t)1 << 40)) return pl;
-  const int64_t nslot = std::min<int64_t>((int64_t)kEagleSlotsPerSM * kDesignSMs, nflat);
+  // one chunk per head: nothing to split; the boundaries are ints
+  if (nchunk < 2 || nflat > INT_MAX) return pl;
+  const int64_t nslot = std::min<int64_t>(kWkv5MaxSlots, nflat);
+  for (int64_t s = 0; s <= nslot; ++s) pl.first[s] = (int)(s * nflat / nslot);
   auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
   pl.nslot = (int)nslot;
   pl.sum = 0;
-  pl.flag = up((size_t)nslot * 64 * 64 * sizeof(float));
+  pl.flag = up((size_t)nslot * slot_floats * sizeof(float));
   pl.flag_bytes = ((size_t)nslot + 1) * sizeof(unsigned int);
   pl.total = pl.flag + up(pl.flag_bytes);
   return pl;
@@ -501,7 +508,7 @@ rwkv_status rwkv_wkv4_step(int64_t B, int64_t C, rwkv_dtype dtype, const float* 
 
 size_t rwkv_wkv5_forward_workspace_bytes(int64_t B, int64_t T, int64_t H, int64_t N) {
   if (N != 64 || B <= 0 || T <= 0 || H <= 0 || !fits_int(B) || !fits_int(H) || !fits_int(B * H)) return 0;
-  return plan_wkv5_slots(B, T, H).total;
+  return plan_matrix_slots(B, T, H, 64 * 64).total;
 }
 
 rwkv_status rwkv_wkv5_forward(int64_t B, int64_t T, int64_t H, int64_t N, const void* r, const void* k,
@@ -524,7 +531,7 @@ rwkv_status rwkv_wkv5_forward(int64_t B, int64_t T, int64_t H, int64_t N, const 
   if (r == nullptr || k == nullptr || v == nullptr || y == nullptr) return RWKV_ERR_INVALID_ARG;
   if (!aligned16(r) || !aligned16(k) || !aligned16(v) || !aligned16(y)) return RWKV_ERR_UNSUPPORTED;
   if ((int64_t)H * 64 > INT_MAX || (int64_t)B * H > INT_MAX) return RWKV_ERR_UNSUPPORTED;
-  const Wkv5Slots plan = plan_wkv5_slots(B, T, H);
+  const MatrixSlots plan = plan_matrix_slots(B, T, H, 64 * 64);
   if (plan.nslot > 0 && (workspace == nullptr || workspace_bytes < plan.total)) return RWKV_ERR_WORKSPACE;
   if (plan.nslot > 0 && !aligned16(workspace)) return RWKV_ERR_UNSUPPORTED;
   DevCtl* ctl = device_ctl();
@@ -551,6 +558,7 @@ rwkv_status rwkv_wkv5_forward(int64_t B, int64_t T, int64_t H, int64_t N, const 
     char* ws = static_cast<char*>(workspace);
     if (cudaMemsetAsync(ws + plan.flag, 0, plan.flag_bytes, st) != cudaSuccess) return RWKV_ERR_CUDA;
     p.nslot = plan.nslot;
+    std::copy(plan.first, plan.first + plan.nslot + 1, p.slot_first);
     p.slot_sum = reinterpret_cast<float*>(ws + plan.sum);
     p.slot_flag = reinterpret_cast<unsigned int*>(ws + plan.flag);
   }

@@ -73,6 +73,8 @@ struct Wkv5StepParams {
   float* s_out;            // [B,H,64,64]; may equal s_in
 };
 
+constexpr int kWkv5MaxSlots = 296;  // Eagle forward CTAs: two per SM of a 148-SM part
+
 struct Wkv5Params {
   int B, T, H;
   const __nv_bfloat16* r;
@@ -85,8 +87,10 @@ struct Wkv5Params {
   float* s_out;         // [B,H,64,64] or null
   DevCtl* ctl;
   // Slot plan (forward only; nslot = 0: one CTA per head).  The heads' 64-token chunks, laid end
-  // to end, are dealt out evenly to nslot CTAs in the order they start.
+  // to end, are dealt out to nslot CTAs in the order they start: slot s takes chunks
+  // [slot_first[s], slot_first[s + 1]).
   int nslot;
+  int slot_first[kWkv5MaxSlots + 1];
   float* slot_sum;          // [nslot][64][64]: a slot's last segment from a zero state
   unsigned int* slot_flag;  // [nslot] flags, then the ticket counter; zeroed before the launch
 };

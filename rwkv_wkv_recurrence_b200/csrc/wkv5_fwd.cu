@@ -136,13 +136,12 @@ __global__ void __launch_bounds__(kThreads, 2) wkv5_fwd_tc_kernel(const __grid_c
   const int q4 = warp & 3, hc = warp >> 2;  // TMEM lane quarter and column half of this warp
   const int nchunk = (p.T + kL - 1) / kL;
   // ---- the CTA's work.  Reversed, or without a slot plan: one whole head (blockIdx).  With a
-  // plan, the heads' chunks laid end to end (head-major, N = B H nchunk of them) are dealt out
-  // evenly: slot s takes [F(s), F(s+1)), F(s) = floor(s N / nslot), the tail of one head, whole
-  // heads and the start of another.  s is a ticket drawn in the order the CTAs start, so a CTA
-  // only ever waits for slots that are already running.
+  // plan, the heads' chunks laid end to end (head-major) are dealt out: slot s takes chunks
+  // [F(s), F(s+1)) (F = p.slot_first), the tail of one head, whole heads and the start of
+  // another.  s is a ticket drawn in the order the CTAs start, so a CTA only ever waits for slots
+  // that are already running.
   const bool slots = !REV && p.nslot > 0;
-  const long long nflat = (long long)p.B * p.H * nchunk;
-  auto slot_first = [&](long long s) { return s * nflat / p.nslot; };  // F(s)
+  auto slot_first = [&](int s) { return (long long)p.slot_first[s]; };  // F(s)
   int slot = 0;
   long long f0 = (long long)blockIdx.x * nchunk, f1 = f0 + nchunk;
   if (slots) {
@@ -496,7 +495,8 @@ __global__ void __launch_bounds__(kThreads, 2) wkv5_fwd_tc_kernel(const __grid_c
       // the start state: s_in carried over the head's earlier chunks, which the slots before this
       // one have summarized.  Wait (bounded) for their flags, warp 0's lanes polling 32 at once.
       const long long hb = (long long)bh * nchunk;
-      const int s_lo = (int)(((hb + 1) * p.nslot + nflat - 1) / nflat) - 1;  // the slot of chunk hb
+      int s_lo = slot;  // the slot that holds the head's first chunk hb
+      while (slot_first(s_lo) > hb) --s_lo;
       if (warp == 0) {
         bool ok = true;
         for (int s0 = s_lo; s0 < slot && ok; s0 += 32) {
