@@ -49,8 +49,20 @@
 // the data allows (N = 128 for the first chain) and the issuing thread hands
 // the first chain out in pairs between the other work of its warp.
 //
-// CTA: one (batch, head), 8 warps, about 113 KB of shared memory and 256 TMEM
-// columns, two CTAs per SM.  Thread 0 issues the TMA loads of the raw r, k, v
+// Work distribution (slot plan): the heads' chunks, laid end to end, are dealt
+// out evenly to two CTAs per SM, so a CTA holds the tail of one head, whole
+// heads and the start of another, in the order of a ticket it draws when it
+// starts.  A CTA whose chunks end inside a head first scans them for a summary,
+// the state they reach from a zero state,
+//   Σ_t e^{λ (E-1-t)} k_tᵀ v_t   up to the end E of its chunks,
+// accumulated in tensor memory chunk after chunk, and publishes it behind a
+// flag; the CTAs holding the rest of that head wait for those flags (bounded)
+// and fold the summaries in order into their start state,
+//   S <- e^{64 n λ} S + summary  (n chunks per summary), from s_in.
+// The reversed instance (the backward's gv pass) runs one whole head per CTA.
+//
+// CTA: 8 warps, about 113 KB of shared memory and 256 TMEM columns, two CTAs
+// per SM.  Thread 0 issues the TMA loads of the raw r, k, v
 // tiles (one [64 tokens x 64] bf16 box each, 128-byte swizzle, no multicast),
 // the scores chain and the A v chain; a thread of warp 4 (whose share of the
 // masking is a zero fill) issues the state-increment chain, so that the time
