@@ -130,6 +130,10 @@ def test_validation_before_any_cuda_work():
                                None) == 2
     assert h.rwkv_wkv5_forward(1, 4, 2, 64, fake, fake, fake, None, fake, fake, None, None, None, 0,
                                None) == 1
+    # the slot plan with a workspace that is not 16-byte aligned
+    need = h.rwkv_wkv5_forward_workspace_bytes(4, 4096, 40, 64)
+    assert h.rwkv_wkv5_forward(4, 4096, 40, 64, fake, fake, fake, fake, fake, fake, None, None, P(0x1004),
+                               need, None) == 2
     # the slot plan without the workspace it needs
     assert h.rwkv_wkv5_forward(4, 4096, 40, 64, fake, fake, fake, fake, fake, fake, None, None, None, 0,
                                None) == 3
