@@ -177,7 +177,7 @@ FwdPlan plan_forward(int64_t B, int64_t T, int64_t C, int algo) {
 constexpr int kEagleSlotsPerSM = 2;  // resident CTAs per SM (shared memory)
 static_assert(kEagleSlotsPerSM * kDesignSMs == kWkv5MaxSlots, "slot bound of the kernel parameters");
 
-struct MatrixSlots {
+struct Wkv5Slots {
   int nslot = 0;
   int first[kWkv5MaxSlots + 1] = {};  // chunk boundaries: slot s takes [first[s], first[s + 1])
   size_t sum = 0, flag = 0, flag_bytes = 0, total = 0;  // workspace offsets and bytes
@@ -186,8 +186,8 @@ struct MatrixSlots {
 // The Eagle forward's plan: slot s takes chunks [floor(s N / nslot), floor((s + 1) N / nslot)) of
 // the N = B H ceil(T / 64) chunks, with a 64 x 64 fp32 summary and a flag per slot and the ticket
 // counter in the workspace.
-MatrixSlots plan_matrix_slots(int64_t B, int64_t T, int64_t H, int64_t slot_floats) {
-  MatrixSlots pl;
+Wkv5Slots plan_wkv5_slots(int64_t B, int64_t T, int64_t H) {
+  Wkv5Slots pl;
   const int64_t nchunk = (T + 63) / 64, nflat = B * H * nchunk;
   // one chunk per head: nothing to split; the boundaries are ints
   if (nchunk < 2 || nflat > INT_MAX) return pl;
@@ -196,7 +196,7 @@ MatrixSlots plan_matrix_slots(int64_t B, int64_t T, int64_t H, int64_t slot_floa
   auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
   pl.nslot = (int)nslot;
   pl.sum = 0;
-  pl.flag = up((size_t)nslot * slot_floats * sizeof(float));
+  pl.flag = up((size_t)nslot * 64 * 64 * sizeof(float));
   pl.flag_bytes = ((size_t)nslot + 1) * sizeof(unsigned int);
   pl.total = pl.flag + up(pl.flag_bytes);
   return pl;
@@ -508,7 +508,7 @@ rwkv_status rwkv_wkv4_step(int64_t B, int64_t C, rwkv_dtype dtype, const float* 
 
 size_t rwkv_wkv5_forward_workspace_bytes(int64_t B, int64_t T, int64_t H, int64_t N) {
   if (N != 64 || B <= 0 || T <= 0 || H <= 0 || !fits_int(B) || !fits_int(H) || !fits_int(B * H)) return 0;
-  return plan_matrix_slots(B, T, H, 64 * 64).total;
+  return plan_wkv5_slots(B, T, H).total;
 }
 
 rwkv_status rwkv_wkv5_forward(int64_t B, int64_t T, int64_t H, int64_t N, const void* r, const void* k,
@@ -531,7 +531,7 @@ rwkv_status rwkv_wkv5_forward(int64_t B, int64_t T, int64_t H, int64_t N, const 
   if (r == nullptr || k == nullptr || v == nullptr || y == nullptr) return RWKV_ERR_INVALID_ARG;
   if (!aligned16(r) || !aligned16(k) || !aligned16(v) || !aligned16(y)) return RWKV_ERR_UNSUPPORTED;
   if ((int64_t)H * 64 > INT_MAX || (int64_t)B * H > INT_MAX) return RWKV_ERR_UNSUPPORTED;
-  const MatrixSlots plan = plan_matrix_slots(B, T, H, 64 * 64);
+  const Wkv5Slots plan = plan_wkv5_slots(B, T, H);
   if (plan.nslot > 0 && (workspace == nullptr || workspace_bytes < plan.total)) return RWKV_ERR_WORKSPACE;
   if (plan.nslot > 0 && !aligned16(workspace)) return RWKV_ERR_UNSUPPORTED;
   DevCtl* ctl = device_ctl();
