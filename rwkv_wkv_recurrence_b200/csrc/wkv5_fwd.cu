@@ -230,6 +230,7 @@ __global__ void __launch_bounds__(kThreads, 2) wkv5_fwd_tc_kernel(const __grid_c
   // k̃ᵀ rows (a fast row's factor is e^{λ(cnt-1-ι)}, formed per chunk)
   float fc0[2][2], fcs[2], lamT[2];
   bool fastT[2];
+  int fidxT[2];  // fast index of the row (-1: slow)
   float e32[2];  // e^{32λ} of the state rows
   auto setup_head = [&](int bh) {
     // the previous segment's reads of the tables, of tensor memory and of opS are done
@@ -287,7 +288,8 @@ __global__ void __launch_bounds__(kThreads, 2) wkv5_fwd_tc_kernel(const __grid_c
     for (int r = 0; r < 2; ++r) {
       const float rate = expf(om[16 * q4 + 8 * r + t4]);
       lamT[r] = -rate;
-      fastT[r] = sm.fidx[16 * q4 + 8 * r + t4] >= 0;
+      fidxT[r] = sm.fidx[16 * q4 + 8 * r + t4];
+      fastT[r] = fidxT[r] >= 0;
 #pragma unroll
       for (int e = 0; e < 2; ++e) fc0[r][e] = fastT[r] ? 0.f : expf(-rate * (float)(31 - 32 * hc - 2 * tq - e));
       fcs[r] = fastT[r] ? 0.f : expf(8.f * rate);
@@ -327,10 +329,14 @@ __global__ void __launch_bounds__(kThreads, 2) wkv5_fwd_tc_kernel(const __grid_c
       kt[4 * i + 2 * r + 1] = __float_as_uint(f.y * fc0[r][1] * g);
     }
   };
-  // a fast row of k̃ᵀ: k e^{λ(cnt-1-ι)}, zero past the chunk's tokens
+  // a fast row of k̃ᵀ: k e^{λ(cnt-1-ι)} at the chunk's last kBand + 1 positions, zero past the
+  // chunk's tokens; before those positions the weight is below 2^-46 and kt_slow has left the
+  // entry at zero, so a warp whose positions (32 hc + 16 pp .. + 15 in step pp) all lie before
+  // them skips the step
   auto kt_fast = [&](int cnt, uint32_t(&kt)[16], uint32_t kbox) {
 #pragma unroll
     for (int pp = 0; pp < 2; ++pp) {
+      if (32 * hc + 16 * pp + 15 < cnt - 1 - kBand) continue;
       uint32_t qk[4];
       ldsm_x4_t(REV ? kbox + offKt - pp * 2048u : kbox + offKt + pp * 2048u, qk);
 #pragma unroll
@@ -340,16 +346,16 @@ __global__ void __launch_bounds__(kThreads, 2) wkv5_fwd_tc_kernel(const __grid_c
           const float2 f = bf2_to_f2(qk[m]);
           const int io = 32 * hc + 8 * i + 2 * tq;
           // e^{λ n}, n = cnt-1-ι: the tabled powers up to n = 15, zero beyond (below 2^-46)
-          const int cf = sm.fidx[16 * q4 + 8 * r + t4];
+          const int cf = fidxT[r];
+          const float e1 = sm.E1[cf];
           auto pw = [&](int n) {
             if (n < 0 || n > kBand) return 0.f;
-            float x = sm.E4[cf][n >> 2];
-            for (int t = 0; t < (n & 3); ++t) x *= sm.E1[cf];
-            return x;
+            const float x = sm.E4[cf][n >> 2];
+            const int q = n & 3;
+            return q == 0 ? x : (q == 1 ? x * e1 : (q == 2 ? x * e1 * e1 : x * e1 * e1 * e1));
           };
-          const float c0 = pw(cnt - 1 - io), c1 = pw(cnt - 2 - io);
-          kt[4 * i + 2 * r] = __float_as_uint(f.x * c0);
-          kt[4 * i + 2 * r + 1] = __float_as_uint(f.y * c1);
+          kt[4 * i + 2 * r] = __float_as_uint(f.x * pw(cnt - 1 - io));
+          kt[4 * i + 2 * r + 1] = __float_as_uint(f.y * pw(cnt - 2 - io));
         }
       }
     }
