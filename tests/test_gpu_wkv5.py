@@ -171,6 +171,26 @@ def test_forward_slot_plan_state_in_place(cuda_device):
     _check_heads(y, st, ref, ref_s)
 
 
+def test_forward_slot_plan_two_streams(cuda_device):
+    # Two calls in flight at once on two streams, each with its own workspace: their CTAs share
+    # the SMs (neither call's 296 CTAs are all resident), and a CTA waits only for CTAs of its own
+    # call that have already started.  Both finish, and each equals its call run alone, bit for bit.
+    B, T, H = 4, 600, 40
+    g1 = _cuda(wi.wkv5_problem(B, T, H, 64, seed=51), cuda_device)
+    g2 = _cuda(wi.wkv5_problem(B, T, H, 64, seed=52, omega_range=(-1.0, 2.0)), cuda_device)
+    ref1, ref2 = rw.rwkv_wkv5_forward(**g1), rw.rwkv_wkv5_forward(**g2)
+    torch.cuda.synchronize()
+    s1, s2 = torch.cuda.Stream(device=cuda_device), torch.cuda.Stream(device=cuda_device)
+    for _ in range(3):
+        with torch.cuda.stream(s1):
+            y1 = rw.rwkv_wkv5_forward(**g1, stream=s1)
+        with torch.cuda.stream(s2):
+            y2 = rw.rwkv_wkv5_forward(**g2, stream=s2)
+        torch.cuda.synchronize()
+        rw.rwkv_check_device_error()
+        assert torch.equal(y1, ref1) and torch.equal(y2, ref2)
+
+
 # ------------------------------------------------------------------ decode step
 def _token(p, t):
     return {n: p[n][:, t].contiguous() for n in ("r", "k", "v")}
