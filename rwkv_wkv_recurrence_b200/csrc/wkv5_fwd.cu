@@ -529,6 +529,8 @@ __global__ void __launch_bounds__(kThreads, 2) wkv5_fwd_tc_kernel(const __grid_c
         aborted = true;
         break;
       }
+      // two summaries' loads in flight at once (a head spread over many CTAs folds many)
+#pragma unroll 2
       for (int s2 = s_lo; s2 < slot; ++s2) {
         const long long a0 = max(slot_first(s2), hb), a1 = slot_first(s2 + 1);
         const float len = (float)((a1 - a0) * kL);
