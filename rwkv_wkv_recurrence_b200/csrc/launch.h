@@ -91,7 +91,7 @@ struct Wkv5Params {
   // [slot_first[s], slot_first[s + 1]).
   int nslot;
   int slot_first[kWkv5MaxSlots + 1];
-  float* slot_sum;          // [nslot][64][64]: a slot's last segment from a zero state
+  float* slot_sum;          // [nslot][256 threads][16]: a slot's last segment from a zero state
   unsigned int* slot_flag;  // [nslot] flags, then the ticket counter; zeroed before the launch
 };
 

@@ -478,12 +478,13 @@ __global__ void __launch_bounds__(kThreads, 2) wkv5_fwd_tc_kernel(const __grid_c
       __syncthreads();
       aborted = sm.abort_flag != 0;
       if (!aborted) {
-        float* dst = p.slot_sum + (size_t)slot * kN * kN;
+        // in the fragment order (thread tid's 16 entries S[0..15] at [tid][16]), which only this
+        // kernel reads: four 16-byte stores here, four 16-byte loads for each fold
+        float4* dst = reinterpret_cast<float4*>(p.slot_sum + (size_t)slot * kN * kN) + 4 * tid;
 #pragma unroll
-        for (int q = 0; q < 8; ++q)
-#pragma unroll
-          for (int r = 0; r < 2; ++r)
-            dst[(size_t)(drow + 8 * r) * kN + jcol + 4 * q] = sum[2 * q + r] + sum2[2 * q + r];
+        for (int x = 0; x < 4; ++x)
+          dst[x] = make_float4(sum[4 * x] + sum2[4 * x], sum[4 * x + 1] + sum2[4 * x + 1],
+                               sum[4 * x + 2] + sum2[4 * x + 2], sum[4 * x + 3] + sum2[4 * x + 3]);
       }
     }
     // publish it, or that this slot gave up (the slots waiting for it then stop at once)
@@ -534,12 +535,16 @@ __global__ void __launch_bounds__(kThreads, 2) wkv5_fwd_tc_kernel(const __grid_c
       for (int s2 = s_lo; s2 < slot; ++s2) {
         const long long a0 = max(slot_first(s2), hb), a1 = slot_first(s2 + 1);
         const float len = (float)((a1 - a0) * kL);
-        const float* src = p.slot_sum + (size_t)s2 * kN * kN;
+        const float4* src = reinterpret_cast<const float4*>(p.slot_sum + (size_t)s2 * kN * kN) + 4 * tid;
         float x[16];
 #pragma unroll
-        for (int q = 0; q < 8; ++q)
-#pragma unroll
-          for (int r = 0; r < 2; ++r) x[2 * q + r] = __ldcg(&src[(size_t)(drow + 8 * r) * kN + jcol + 4 * q]);
+        for (int i = 0; i < 4; ++i) {
+          const float4 v = __ldcg(src + i);
+          x[4 * i] = v.x;
+          x[4 * i + 1] = v.y;
+          x[4 * i + 2] = v.z;
+          x[4 * i + 3] = v.w;
+        }
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
           const float d = expf(lamT[r] * len);
